@@ -1,0 +1,22 @@
+"""CPU oracle for the block-sparse attention path (test infrastructure only).
+
+This package is the slow, plain fp64 statement of what the CUDA path computes.
+Only the test-suite, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import it; the product path never
+does, and it shares no code with the CUDA kernels.
+
+Pages followed (titles and sections):
+  * "SpargeAttention2: 論文の技術的サマリー", §2(1) hybrid Top-k + Top-p masking,
+    §2(3) block-sparse FlashAttention that skips masked tiles.
+  * "SLA2" (ai-papers.net), 提案手法 ① mean pooling of queries and keys before
+    scoring, ② O = alpha * O_s + (1 - alpha) * O_l.
+  * "SALAD", §2.1 a linear-attention branch in parallel with sparse attention.
+
+Every function works on one (batch, head) slice in float64 numpy arrays.
+"""
+from .sparse_attention import (  # noqa: F401
+    as_f64, pool_blocks, block_scores, block_softmax, topk_count, descending_order,
+    topp_count, topk_set, topp_set, hybrid_row, build_mask, kv_lists, mask_from_lists,
+    masked_attention, dense_attention, phi, linear_state, linear_out, blend,
+    row_threshold_info, NEAR_TIE_TOL,
+)

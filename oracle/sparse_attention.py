@@ -1,0 +1,257 @@
+"""fp64 oracle: block pooling, hybrid Top-k ∪ Top-p block mask, masked softmax
+attention, the elu+1 linear branch and the alpha blend.
+
+TEST INFRASTRUCTURE: imported only by tests, the smoke check and the bench's
+CPU-baseline leg. Written from the pages' definitions, in their order; numpy
+matmul, exp and a stable sort are the only library steps.
+
+Parity pins (tests/test_oracle_*.py) tie each function to something other than
+itself: brute force on tiny inputs, closed forms, exhaustive subset search for
+Top-p minimality, and torch's float64 scaled_dot_product_attention for dense
+and masked attention.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+# A block whose score lies within this distance of the selection cut, or a row
+# whose cumulative probability lies within it of p, may legitimately differ
+# between an fp32 GPU evaluation and this fp64 one; such cases are reported.
+NEAR_TIE_TOL = 1e-6
+
+
+def as_f64(x) -> np.ndarray:
+    """Exact conversion of a bf16/fp32 torch tensor or numpy array to float64."""
+    if hasattr(x, "detach"):
+        import torch
+        return x.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------
+# Mask prediction: SLA2 提案手法 ① (mean pooling of Q and K per block) and
+# SpargeAttention2 §2(1) (hybrid Top-k + Top-p per attention row).
+# --------------------------------------------------------------------------
+
+def pool_blocks(x: np.ndarray, b: int) -> tuple[np.ndarray, np.ndarray]:
+    """Mean of the rows of x [N, d] over consecutive blocks of b tokens.
+
+    The last block may be partial; it is averaged over its valid tokens only.
+    Returns (means [ceil(N/b), d], counts [ceil(N/b)]).
+    """
+    N, d = x.shape
+    n = -(-N // b)
+    means = np.empty((n, d), dtype=np.float64)
+    counts = np.empty(n, dtype=np.int64)
+    for i in range(n):
+        rows = x[i * b:min(N, (i + 1) * b)]
+        counts[i] = rows.shape[0]
+        means[i] = rows.sum(axis=0) / rows.shape[0]
+    return means, counts
+
+
+def block_scores(q_pool: np.ndarray, k_pool: np.ndarray, scale: float) -> np.ndarray:
+    """s[qb, kb] = scale * <mean q of block qb, mean k of block kb>."""
+    return scale * (q_pool @ k_pool.T)
+
+
+def block_softmax(s: np.ndarray) -> np.ndarray:
+    """Softmax of each row of block scores over all key blocks of that row."""
+    m = s.max(axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def topk_count(k_frac: float, n_kb: int) -> int:
+    """Number of blocks Top-k keeps in a row: ceil(k * n_kb), at least 1.
+
+    The 1e-9 guard keeps exact products such as 0.1 * 10 from rounding up.
+    """
+    return int(min(n_kb, max(1, math.ceil(k_frac * n_kb - 1e-9))))
+
+
+def descending_order(s_row: np.ndarray) -> np.ndarray:
+    """Key blocks by score, largest first; equal scores keep the lower index first."""
+    return np.argsort(-s_row, kind="stable")
+
+
+def topp_count(p_sorted: np.ndarray, p: float) -> int:
+    """Smallest m >= 1 whose m largest probabilities sum to at least p.
+
+    p >= 1 asks for the whole distribution, i.e. every block. If rounding keeps
+    the running sum below p, every block is taken.
+    """
+    n = p_sorted.shape[0]
+    if p >= 1.0:
+        return n
+    csum = 0.0
+    for m in range(1, n + 1):
+        csum += p_sorted[m - 1]
+        if csum >= p:
+            return m
+    return n
+
+
+def topk_set(s_row: np.ndarray, k_frac: float) -> set:
+    order = descending_order(s_row)
+    return set(order[:topk_count(k_frac, s_row.shape[0])].tolist())
+
+
+def topp_set(s_row: np.ndarray, p: float) -> set:
+    order = descending_order(s_row)
+    P = block_softmax(s_row)
+    return set(order[:topp_count(P[order], p)].tolist())
+
+
+def hybrid_row(s_row: np.ndarray, k_frac: float, p: float):
+    """Hybrid mask of one query-block row: Top-k ∪ Top-p.
+
+    Both sets are prefixes of the same descending order, so their union is the
+    prefix of length L = max(K_sel, m_p). Returns (bool mask [n_kb], L, K_sel, m_p).
+    """
+    n = s_row.shape[0]
+    order = descending_order(s_row)
+    P = block_softmax(s_row)
+    k_sel = topk_count(k_frac, n)
+    m_p = topp_count(P[order], p)
+    L = max(k_sel, m_p)
+    mask = np.zeros(n, dtype=bool)
+    mask[order[:L]] = True
+    union = set(order[:k_sel].tolist()) | set(order[:m_p].tolist())
+    assert union == set(np.nonzero(mask)[0].tolist())
+    return mask, L, k_sel, m_p
+
+
+def build_mask(q: np.ndarray, k: np.ndarray, bq: int, bk: int, k_frac: float, p: float,
+               scale: float | None = None):
+    """Block mask for one head from Q, K [N, d].
+
+    Returns dict(mask [n_qb, n_kb] bool, s scores, P probabilities, L, k_sel, m_p).
+    """
+    d = q.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    qp, _ = pool_blocks(q, bq)
+    kp, _ = pool_blocks(k, bk)
+    s = block_scores(qp, kp, scale)
+    n_qb, n_kb = s.shape
+    mask = np.zeros((n_qb, n_kb), dtype=bool)
+    L = np.zeros(n_qb, dtype=np.int64)
+    ks = np.zeros(n_qb, dtype=np.int64)
+    mp = np.zeros(n_qb, dtype=np.int64)
+    for r in range(n_qb):
+        mask[r], L[r], ks[r], mp[r] = hybrid_row(s[r], k_frac, p)
+    return {"mask": mask, "s": s, "P": block_softmax(s), "L": L, "k_sel": ks, "m_p": mp,
+            "q_pool": qp, "k_pool": kp}
+
+
+def row_threshold_info(s_row: np.ndarray, k_frac: float, p: float, tol: float = NEAR_TIE_TOL):
+    """Describe how close a row's decision is to a tie.
+
+    Returns dict with the order, L, the cumulative sums, the blocks whose score is
+    within tol of the last kept or first dropped score (score ties at the cut), and
+    the ranks r where the cumulative sum up to r lies within tol of p (cumsum ties).
+    """
+    order = descending_order(s_row)
+    P = block_softmax(s_row)[order]
+    n = s_row.shape[0]
+    _, L, k_sel, m_p = hybrid_row(s_row, k_frac, p)
+    csum = np.cumsum(P)
+    cut_scores = [s_row[order[L - 1]]]
+    if L < n:
+        cut_scores.append(s_row[order[L]])
+    near_blocks = set()
+    for c in cut_scores:
+        near_blocks |= set(np.nonzero(np.abs(s_row - c) <= tol)[0].tolist())
+    near_ranks = set(np.nonzero(np.abs(csum - p) <= tol)[0].tolist()) if p < 1.0 else set()
+    return {"order": order, "L": L, "k_sel": k_sel, "m_p": m_p, "csum": csum,
+            "near_blocks": near_blocks, "near_ranks": near_ranks}
+
+
+def kv_lists(mask: np.ndarray):
+    """Compacted form of a block mask: ascending kept key-block indices per row."""
+    n_qb, n_kb = mask.shape
+    kv_idx = np.full((n_qb, n_kb), -1, dtype=np.int64)
+    kv_cnt = np.zeros(n_qb, dtype=np.int64)
+    for r in range(n_qb):
+        idx = np.nonzero(mask[r])[0]
+        kv_cnt[r] = idx.shape[0]
+        kv_idx[r, :idx.shape[0]] = idx
+    return kv_idx, kv_cnt
+
+
+def mask_from_lists(kv_idx: np.ndarray, kv_cnt: np.ndarray, n_kb: int) -> np.ndarray:
+    n_qb = kv_cnt.shape[0]
+    mask = np.zeros((n_qb, n_kb), dtype=bool)
+    for r in range(n_qb):
+        mask[r, kv_idx[r, :kv_cnt[r]]] = True
+    return mask
+
+
+# --------------------------------------------------------------------------
+# Attention: SpargeAttention2 §2(3) — exact softmax attention restricted to the
+# kept (query-block, key-block) tiles; masked tiles contribute nothing.
+# --------------------------------------------------------------------------
+
+def masked_attention(q, k, v, mask, bq, bk, scale=None, rows=None):
+    """O[i] = sum_j softmax_j(scale * q_i . k_j) v_j over keys j in kept blocks.
+
+    rows: iterable of query indices to evaluate (default: all). Returns
+    (O [len(rows), d], LSE [len(rows)]); a row with no kept key gives O = 0 and
+    LSE = -inf.
+    """
+    N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rows = np.arange(N) if rows is None else np.asarray(list(rows), dtype=np.int64)
+    out = np.zeros((rows.shape[0], d), dtype=np.float64)
+    lse = np.full(rows.shape[0], -np.inf, dtype=np.float64)
+    for n, i in enumerate(rows):
+        kept = np.nonzero(mask[i // bq])[0]
+        if kept.shape[0] == 0:
+            continue
+        keys = np.concatenate([np.arange(kb * bk, min(N, (kb + 1) * bk)) for kb in kept])
+        logits = scale * (k[keys] @ q[i])
+        m = logits.max()
+        w = np.exp(logits - m)
+        z = w.sum()
+        out[n] = (w @ v[keys]) / z
+        lse[n] = m + math.log(z)
+    return out, lse
+
+
+def dense_attention(q, k, v, scale=None):
+    N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    logits = scale * (q @ k.T)
+    m = logits.max(axis=1, keepdims=True)
+    w = np.exp(logits - m)
+    z = w.sum(axis=1, keepdims=True)
+    return (w @ v) / z, (m + np.log(z))[:, 0]
+
+
+# --------------------------------------------------------------------------
+# Linear branch (SALAD §2.1, SLA2 提案手法 ②): phi(x) = elu(x) + 1,
+# O_l[i] = phi(q_i)^T S / phi(q_i)^T z with S = sum_j phi(k_j) v_j^T and
+# z = sum_j phi(k_j) over all N keys; then O = alpha * O_s + (1 - alpha) * O_l.
+# --------------------------------------------------------------------------
+
+def phi(x: np.ndarray) -> np.ndarray:
+    return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+
+
+def linear_state(k: np.ndarray, v: np.ndarray):
+    fk = phi(k)
+    return fk.T @ v, fk.sum(axis=0)
+
+
+def linear_out(q: np.ndarray, S: np.ndarray, z: np.ndarray) -> np.ndarray:
+    fq = phi(q)
+    return (fq @ S) / (fq @ z)[:, None]
+
+
+def blend(o_s: np.ndarray, o_l: np.ndarray, alpha_h: np.ndarray) -> np.ndarray:
+    return alpha_h[None, :] * o_s + (1.0 - alpha_h[None, :]) * o_l

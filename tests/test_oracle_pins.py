@@ -1,0 +1,266 @@
+"""Pins of the fp64 oracle against things other than itself.
+
+Each test below ties one oracle function to brute force, a closed form, an
+exhaustive search or a library routine (torch float64 SDPA), so that a dropped
+term, a wrong index or a transposed operand in the oracle fails here.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_softmax_b200.workloads import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.filterwarnings("ignore::UserWarning")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- pooling
+def test_pool_matches_brute_force_loops_with_partial_tail():
+    x = _rng(0).standard_normal((37, 5))
+    means, counts = oracle.pool_blocks(x, 8)
+    assert means.shape == (5, 5) and counts.tolist() == [8, 8, 8, 8, 5]
+    for blk in range(5):
+        for c in range(5):
+            acc, n = 0.0, 0
+            for t in range(37):
+                if t // 8 == blk:
+                    acc += x[t, c]
+                    n += 1
+            assert abs(means[blk, c] - acc / n) < 1e-14
+
+
+def test_pool_constant_blocks_and_token_sum_identity():
+    x = np.repeat(np.arange(6, dtype=np.float64)[:, None] * 0.5, 10, axis=0)[:, :1].repeat(3, 1)
+    x = x[:57]  # last block partial
+    means, counts = oracle.pool_blocks(x, 10)
+    assert np.allclose(means[:, 0], [0, 0.5, 1.0, 1.5, 2.0, 2.5])
+    y = _rng(1).standard_normal((57, 4))
+    m2, c2 = oracle.pool_blocks(y, 10)
+    assert np.allclose((m2 * c2[:, None]).sum(0), y.sum(0), atol=1e-12)
+
+
+# ---------------------------------------------------------------- scores + softmax
+def test_block_scores_brute_force_and_softmax():
+    qp = _rng(2).standard_normal((3, 4))
+    kp = _rng(3).standard_normal((5, 4))
+    s = oracle.block_scores(qp, kp, 0.5)
+    for i in range(3):
+        for j in range(5):
+            assert abs(s[i, j] - 0.5 * sum(qp[i, c] * kp[j, c] for c in range(4))) < 1e-14
+    P = oracle.block_softmax(s)
+    for i in range(3):
+        z = sum(math.exp(s[i, j]) for j in range(5))
+        for j in range(5):
+            assert abs(P[i, j] - math.exp(s[i, j]) / z) < 1e-15
+    assert np.allclose(P.sum(1), 1.0)
+    assert np.allclose(oracle.block_softmax(s + 123.0), P)
+
+
+# ---------------------------------------------------------------- Top-k count
+@pytest.mark.parametrize("k,n,want", [(0.10, 16, 2), (0.05, 512, 26), (0.03, 1182, 36),
+                                      (0.05, 1182, 60), (0.05, 3840, 192), (0.1, 10, 1),
+                                      (1.0, 77, 77), (1e-6, 50, 1), (0.5, 3, 2)])
+def test_topk_count_closed_form(k, n, want):
+    assert oracle.topk_count(k, n) == want
+
+
+# ---------------------------------------------------------------- Top-p minimality
+def _tiny_rows():
+    wl = WORKLOADS["tiny"]
+    x = make_inputs(wl, "cpu")
+    rows = []
+    for h in range(wl.H):
+        out = oracle.build_mask(oracle.as_f64(x["q"][0, h]), oracle.as_f64(x["k"][0, h]),
+                                wl.bq, wl.bk, wl.topk, wl.topp)
+        rows += [(out["s"][r], out["mask"][r], out["m_p"][r], out["L"][r]) for r in range(out["s"].shape[0])]
+    return wl, rows
+
+
+def test_topp_minimal_by_exhaustive_subsets_on_tiny_workload():
+    """Every row of the tiny workload has 16 key blocks: try all 2^16 subsets."""
+    wl, rows = _tiny_rows()
+    n = 16
+    bits = ((np.arange(1 << n)[:, None] >> np.arange(n)[None, :]) & 1).astype(np.float64)
+    sizes = bits.sum(1)
+    for p in (wl.topp, 0.5, 0.99):
+        for s_row, _, _, _ in rows:
+            P = oracle.block_softmax(s_row)
+            sums = bits @ P
+            min_size = int(sizes[sums >= p - 0.0].min())
+            order = oracle.descending_order(s_row)
+            m_p = oracle.topp_count(P[order], p)
+            # rounding of the running sum is allowed to differ only within the tie band
+            if abs(np.cumsum(P[order])[m_p - 1] - p) > 1e-12 and (m_p < 2 or abs(np.cumsum(P[order])[m_p - 2] - p) > 1e-12):
+                assert m_p == min_size
+            assert P[order][:m_p].sum() >= p - 1e-12
+
+
+def test_hybrid_equals_union_of_rank_defined_sets():
+    """Top-k and Top-p built from the rank definition, with deliberate ties."""
+    rng = _rng(5)
+    for trial in range(200):
+        n = int(rng.integers(1, 12))
+        s = np.round(rng.standard_normal(n) * 2, 1)   # rounding creates ties
+        k = float(rng.uniform(0.01, 1.0))
+        p = float(rng.uniform(0.0, 0.999))
+        rank = np.array([sum(1 for j in range(n) if s[j] > s[i] or (s[j] == s[i] and j < i))
+                         for i in range(n)])
+        k_sel = oracle.topk_count(k, n)
+        topk = {i for i in range(n) if rank[i] < k_sel}
+        P = np.exp(s - s.max()); P /= P.sum()
+        by_rank = P[np.argsort(rank)]
+        m_p = next((m for m in range(1, n + 1) if by_rank[:m].sum() >= p), n)
+        topp = {i for i in range(n) if rank[i] < m_p}
+        mask, L, ks, mp = oracle.hybrid_row(s, k, p)
+        assert set(np.nonzero(mask)[0].tolist()) == topk | topp
+        assert ks == k_sel and L == max(k_sel, m_p)
+
+
+def test_hybrid_special_cases():
+    rng = _rng(6)
+    s = rng.standard_normal(40)
+    assert oracle.hybrid_row(s, 1.0, 0.5)[0].all()                       # k = 100%
+    m, L, ks, mp = oracle.hybrid_row(s, 0.1, 0.0)                        # p = 0: Top-k only
+    assert m.sum() == 4 and L == ks == 4
+    assert oracle.hybrid_row(s, 1e-6, 1.0)[0].all()                       # p = 1: every block
+    sink = np.full(40, -20.0); sink[7] = 20.0                             # one-hot sink row
+    m, L, ks, mp = oracle.hybrid_row(sink, 0.05, 0.9)
+    assert mp == 1 and L == ks == 2 and m[7] and m[0]                     # tie order: lowest index
+    flat = np.zeros(16)                                                   # uniform row
+    m, L, ks, mp = oracle.hybrid_row(flat, 0.1, 0.9)
+    assert mp == 15 and L == 15 and m[:15].all() and not m[15]
+
+
+def test_hybrid_worked_example_from_the_failure_modes():
+    """SpargeAttention2 §1: Top-k misses mass on flat rows, Top-p collapses onto sinks."""
+    flat = np.log(np.array([0.2, 0.2, 0.2, 0.2, 0.2]))
+    m, L, ks, mp = oracle.hybrid_row(flat, 0.2, 0.7)
+    assert ks == 1 and mp == 4 and L == 4           # Top-p rescues the flat row
+    skew = np.log(np.array([0.91, 0.03, 0.03, 0.02, 0.01]))
+    m, L, ks, mp = oracle.hybrid_row(skew, 0.4, 0.9)
+    assert mp == 1 and ks == 2 and L == 2           # Top-k rescues the sink row
+    assert m.tolist() == [True, True, False, False, False]
+
+
+def test_kv_lists_round_trip():
+    mask = _rng(7).random((9, 13)) < 0.3
+    idx, cnt = oracle.kv_lists(mask)
+    assert (oracle.mask_from_lists(idx, cnt, 13) == mask).all()
+    for r in range(9):
+        assert (np.diff(idx[r, :cnt[r]]) > 0).all()
+
+
+# ---------------------------------------------------------------- attention
+def _sdpa(q, k, v, mask=None, scale=None):
+    t = lambda a: torch.from_numpy(a)[None, None]
+    am = None if mask is None else torch.from_numpy(mask)[None, None]
+    o = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), attn_mask=am, scale=scale)
+    return o[0, 0].numpy()
+
+
+def test_all_ones_mask_is_dense_attention_sdpa():
+    rng = _rng(8)
+    N, d = 100, 16
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    mask = np.ones((-(-N // 32), -(-N // 16)), dtype=bool)
+    o, lse = oracle.masked_attention(q, k, v, mask, 32, 16)
+    assert np.abs(o - _sdpa(q, k, v)).max() < 1e-12
+    od, lsed = oracle.dense_attention(q, k, v)
+    assert np.abs(o - od).max() < 1e-12
+    ref_lse = torch.logsumexp(torch.from_numpy(q @ k.T / math.sqrt(d)), dim=1).numpy()
+    assert np.abs(lse - ref_lse).max() < 1e-12
+
+
+def test_block_mask_equals_sdpa_with_expanded_token_mask():
+    rng = _rng(9)
+    N, d, bq, bk = 70, 8, 16, 8
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    q *= 2.0
+    mask = rng.random((-(-N // bq), -(-N // bk))) < 0.4
+    mask[:, 0] = True
+    tok = np.zeros((N, N), dtype=bool)
+    for i in range(N):
+        for j in range(N):
+            tok[i, j] = mask[i // bq, j // bk]
+    o, _ = oracle.masked_attention(q, k, v, mask, bq, bk, scale=0.3)
+    assert np.abs(o - _sdpa(q, k, v, tok, scale=0.3)).max() < 1e-12
+
+
+def test_attention_invariants():
+    rng = _rng(10)
+    N, d = 50, 8
+    q, k = rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    v_const = np.tile(rng.standard_normal(d), (N, 1))
+    mask = rng.random((4, 7)) < 0.5
+    mask[:, 3] = True
+    o, _ = oracle.masked_attention(q, k, v_const, mask, 16, 8)
+    assert np.abs(o - v_const).max() < 1e-12
+    v = rng.standard_normal((N, d))
+    o, _ = oracle.masked_attention(q, k, v, mask, 16, 8)
+    assert (np.abs(o) <= np.abs(v).max(0) + 1e-12).all()
+    empty = np.zeros((4, 7), dtype=bool)
+    o, lse = oracle.masked_attention(q, k, v, empty, 16, 8, rows=[0, 49])
+    assert (o == 0).all() and np.isneginf(lse).all()
+
+
+# ---------------------------------------------------------------- linear branch + blend
+def test_phi_is_elu_plus_one():
+    x = np.linspace(-30, 30, 1001)
+    ref = torch.nn.functional.elu(torch.from_numpy(x)).numpy() + 1.0
+    assert np.abs(oracle.phi(x) - ref).max() < 1e-15
+    assert (oracle.phi(x) > 0).all()
+
+
+def test_linear_branch_equals_quadratic_brute_force():
+    rng = _rng(11)
+    N, d = 40, 6
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    S, z = oracle.linear_state(k, v)
+    o = oracle.linear_out(q, S, z)
+    for i in range(N):
+        num = np.zeros(d)
+        den = 0.0
+        for j in range(N):
+            w = float(np.dot(oracle.phi(q[i]), oracle.phi(k[j])))
+            num += w * v[j]
+            den += w
+        assert np.abs(o[i] - num / den).max() < 1e-12
+    vc = np.tile(rng.standard_normal(d), (N, 1))
+    S, z = oracle.linear_state(k, vc)
+    assert np.abs(oracle.linear_out(q, S, z) - vc).max() < 1e-12
+
+
+def test_blend_endpoints_and_midpoint():
+    rng = _rng(12)
+    a, b = rng.standard_normal((5, 4)), rng.standard_normal((5, 4))
+    assert np.array_equal(oracle.blend(a, b, np.ones(4)), a)
+    assert np.array_equal(oracle.blend(a, b, np.zeros(4)), b)
+    assert np.allclose(oracle.blend(a, b, np.full(4, 0.5)), (a + b) / 2)
+
+
+# ---------------------------------------------------------------- golden regression
+def test_tiny_workload_masks_match_golden():
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "tiny_kv_lists.txt")
+    want = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            h, r, cnt, idx = line.split(":")
+            want[(int(h), int(r))] = (int(cnt), [int(t) for t in idx.split()])
+    wl = WORKLOADS["tiny"]
+    x = make_inputs(wl, "cpu")
+    for h in range(wl.H):
+        out = oracle.build_mask(oracle.as_f64(x["q"][0, h]), oracle.as_f64(x["k"][0, h]),
+                                wl.bq, wl.bk, wl.topk, wl.topp)
+        idx, cnt = oracle.kv_lists(out["mask"])
+        for r in range(idx.shape[0]):
+            assert want[(h, r)] == (int(cnt[r]), idx[r, :cnt[r]].tolist())
