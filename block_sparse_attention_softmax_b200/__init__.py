@@ -1,0 +1,13 @@
+"""B200 block-sparse attention with a hybrid Top-k ∪ Top-p block mask.
+
+The compute lives in libsa.so (CUDA kernels for sm_100a behind the C ABI of
+include/sa.h). This package is its thin Python binding: the functions below
+carry the C names, marshal torch tensors into pointers and sizes, allocate
+outputs and workspaces with torch, and raise on any non-zero status. There is
+no CPU fallback: without the built library or a CUDA device every call raises.
+"""
+from ._binding import (  # noqa: F401
+    SAError, load, lib_path, sa_version, sa_status_string, sa_device_status,
+    sa_pool_blocks, sa_build_mask, sa_sparse_attn_fwd, sa_dense_attn_fwd,
+    sa_linear_branch, sa_blend, block_sparse_attention, header_symbols,
+)

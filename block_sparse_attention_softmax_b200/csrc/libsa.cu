@@ -1,0 +1,7 @@
+// libsa.cu — single translation unit of libsa.so, so that the kernels and the
+// C ABI share device symbols (the device status word) without relocatable
+// device code.
+#include "mask_kernels.cu"
+#include "attn_kernel.cu"
+#include "linear_kernels.cu"
+#include "sa_api.cu"

@@ -1,0 +1,301 @@
+// sa_api.cu — the extern "C" boundary of libsa: argument validation, workspace
+// carving, kernel dispatch and error reporting. Declarations and the contract
+// of every entry point are in include/sa.h.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "../../include/sa.h"
+#include "sa_internal.h"
+
+namespace sa {
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(SA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr int kMaxKeyBlocks = 16384;  // selection keeps one row of scores in shared memory
+
+int check_shape(int B, int H, int N, int d, int bq, int bk) {
+  if (B <= 0 || H <= 0 || N <= 0) return fail(SA_ERR_INVALID_ARG, "B, H and N must be positive (got %d, %d, %d)", B, H, N);
+  if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "head dim %d unsupported (64 or 128)", d);
+  if (bq != 64 && bq != 128) return fail(SA_ERR_UNSUPPORTED, "query block %d unsupported (64 or 128)", bq);
+  if (bk != 64) return fail(SA_ERR_UNSUPPORTED, "key block %d unsupported (64)", bk);
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH > 65535) return fail(SA_ERR_UNSUPPORTED, "B*H = %lld exceeds 65535", BH);
+  if (BH * N * d >= (1LL << 40)) return fail(SA_ERR_UNSUPPORTED, "tensor too large");
+  const long long nkb = (N + bk - 1) / bk, nqb = (N + bq - 1) / bq;
+  if (BH * nqb * nkb >= (1LL << 34)) return fail(SA_ERR_UNSUPPORTED, "block mask too large");
+  return SA_OK;
+}
+
+struct MaskWs {
+  size_t q_pool, k_pool, s, total;
+  long long s_ld;
+};
+
+MaskWs mask_ws(int B, int H, int N, int d, int bq, int bk, bool need_q, bool need_k) {
+  const long long BH = static_cast<long long>(B) * H;
+  const long long nqb = (N + bq - 1) / bq, nkb = (N + bk - 1) / bk;
+  MaskWs w{};
+  w.s_ld = (nkb + 3) / 4 * 4;
+  size_t off = 0;
+  w.q_pool = off;
+  if (need_q) off += round_up(static_cast<size_t>(BH * nqb * d) * 4, 256);
+  w.k_pool = off;
+  if (need_k) off += round_up(static_cast<size_t>(BH * nkb * d) * 4, 256);
+  w.s = off;
+  off += round_up(static_cast<size_t>(BH * nqb) * w.s_ld * 4, 256);
+  w.total = off;
+  return w;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+CUresult encode_tensor_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t inner,
+                                   uint64_t rows, uint64_t planes, uint32_t box_inner,
+                                   uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return CUDA_ERROR_NOT_SUPPORTED;
+  const cuuint64_t dims[3] = {inner, rows, planes};
+  const cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  const cuuint32_t box[3] = {box_inner, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+}  // namespace sa
+
+using namespace sa;
+
+extern "C" {
+
+int sa_version(void) { return 100; }
+
+const char* sa_status_string(int status) {
+  switch (status) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID_ARG: return "SA_ERR_INVALID_ARG";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED";
+    case SA_ERR_ALIGN: return "SA_ERR_ALIGN";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA";
+    case SA_ERR_DEVICE_TIMEOUT: return "SA_ERR_DEVICE_TIMEOUT";
+    case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE";
+    default: return "SA_ERR_UNKNOWN";
+  }
+}
+
+const char* sa_last_error(void) { return g_last_error.c_str(); }
+
+int sa_device_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "sa_device_status");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "sa_device_status");
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+    return fail(SA_ERR_DEVICE_TIMEOUT, "a bounded device-side wait ran out (code %d)", v);
+  }
+  return SA_OK;
+}
+
+int sa_pool_blocks(const uint16_t* q, const uint16_t* k, int B, int H, int N, int d, int bq,
+                   int bk, float* q_pool, float* k_pool, void* stream) {
+  int rc = check_shape(B, H, N, d, bq, bk);
+  if (rc) return rc;
+  if (!q || !k || !q_pool || !k_pool) return fail(SA_ERR_INVALID_ARG, "sa_pool_blocks: null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool))
+    return fail(SA_ERR_ALIGN, "sa_pool_blocks: pointers must be 16-byte aligned");
+  cudaError_t e = launch_pool(q, k, B * H, N, d, bq, bk, q_pool, k_pool, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_pool_blocks");
+}
+
+size_t sa_build_mask_workspace_size(int B, int H, int N, int d, int bq, int bk) {
+  if (check_shape(B, H, N, d, bq, bk)) return 0;
+  return mask_ws(B, H, N, d, bq, bk, true, true).total;
+}
+
+int sa_build_mask(const uint16_t* q, const uint16_t* k, int B, int H, int N, int d, int bq, int bk,
+                  double topk_frac, double topp, double scale, int32_t* kv_idx, int32_t* kv_cnt,
+                  uint8_t* mask_opt, float* q_pool_opt, float* k_pool_opt, void* workspace,
+                  size_t ws_bytes, void* stream) {
+  int rc = check_shape(B, H, N, d, bq, bk);
+  if (rc) return rc;
+  if (!q || !k || !kv_idx || !kv_cnt) return fail(SA_ERR_INVALID_ARG, "sa_build_mask: null pointer");
+  if (!(topk_frac > 0.0 && topk_frac <= 1.0)) return fail(SA_ERR_INVALID_ARG, "topk_frac %g outside (0, 1]", topk_frac);
+  if (!(topp >= 0.0 && topp <= 1.0)) return fail(SA_ERR_INVALID_ARG, "topp %g outside [0, 1]", topp);
+  if (!isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "scale must be finite");
+  const int nkb = (N + bk - 1) / bk, nqb = (N + bq - 1) / bq;
+  if (nkb > kMaxKeyBlocks) return fail(SA_ERR_UNSUPPORTED, "n_kb = %d exceeds %d", nkb, kMaxKeyBlocks);
+  const void* ptrs[] = {q, k, kv_idx, kv_cnt, mask_opt, q_pool_opt, k_pool_opt, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "sa_build_mask: pointers must be 16-byte aligned");
+  const MaskWs w = mask_ws(B, H, N, d, bq, bk, q_pool_opt == nullptr, k_pool_opt == nullptr);
+  if (!workspace || ws_bytes < w.total)
+    return fail(SA_ERR_WORKSPACE, "sa_build_mask: workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
+  if (scale <= 0.0) scale = 1.0 / sqrt(static_cast<double>(d));
+  char* ws = static_cast<char*>(workspace);
+  float* qp = q_pool_opt ? q_pool_opt : reinterpret_cast<float*>(ws + w.q_pool);
+  float* kp = k_pool_opt ? k_pool_opt : reinterpret_cast<float*>(ws + w.k_pool);
+  float* s = reinterpret_cast<float*>(ws + w.s);
+  const int BH = B * H;
+  const int k_sel = static_cast<int>(fmin(static_cast<double>(nkb), fmax(1.0, ceil(topk_frac * nkb - 1e-9))));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_pool(q, k, BH, N, d, bq, bk, qp, kp, st);
+  if (e == cudaSuccess) e = launch_scores(qp, kp, BH, nqb, nkb, d, scale, s, w.s_ld, st);
+  if (e == cudaSuccess) e = launch_select(s, w.s_ld, BH * nqb, nkb, k_sel, topp, kv_idx, kv_cnt, mask_opt, st);
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_build_mask");
+}
+
+size_t sa_sparse_attn_workspace_size(int B, int H, int N, int d, int bq, int bk, int ext_mask) {
+  if (check_shape(B, H, N, d, bq, bk) || !ext_mask) return 0;
+  const long long BH = static_cast<long long>(B) * H;
+  const long long nqb = (N + bq - 1) / bq, nkb = (N + bk - 1) / bk;
+  return round_up(static_cast<size_t>(BH * nqb * nkb) * 4, 256) + round_up(static_cast<size_t>(BH * nqb) * 4, 256);
+}
+
+int sa_sparse_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H,
+                       int N, int d, int bq, int bk, const int32_t* kv_idx,
+                       const int32_t* kv_cnt, const uint8_t* ext_mask, double scale, uint16_t* o,
+                       float* lse_opt, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_shape(B, H, N, d, bq, bk);
+  if (rc) return rc;
+  if (!q || !k || !v || !o) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: null tensor pointer");
+  const bool lists = kv_idx && kv_cnt;
+  if (lists == (ext_mask != nullptr) || (!lists && (kv_idx || kv_cnt)))
+    return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: give exactly one of (kv_idx, kv_cnt) or ext_mask");
+  if (!isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "scale must be finite");
+  const void* ptrs[] = {q, k, v, o, kv_idx, kv_cnt, lse_opt, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "sa_sparse_attn_fwd: pointers must be 16-byte aligned");
+  if (scale <= 0.0) scale = 1.0 / sqrt(static_cast<double>(d));
+  const int BH = B * H;
+  const int nqb = (N + bq - 1) / bq, nkb = (N + bk - 1) / bk;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int* idx = kv_idx;
+  const int* cnt = kv_cnt;
+  if (!lists) {
+    const size_t need = sa_sparse_attn_workspace_size(B, H, N, d, bq, bk, 1);
+    if (!workspace || ws_bytes < need)
+      return fail(SA_ERR_WORKSPACE, "sa_sparse_attn_fwd: workspace of %zu bytes needed for ext_mask", need);
+    int* widx = static_cast<int*>(workspace);
+    int* wcnt = reinterpret_cast<int*>(static_cast<char*>(workspace) + round_up(static_cast<size_t>(BH) * nqb * nkb * 4, 256));
+    cudaError_t e = launch_compact_mask(ext_mask, BH * nqb, nkb, widx, wcnt, st);
+    if (e != cudaSuccess) return cuda_fail(e, "sa_sparse_attn_fwd (mask compaction)");
+    idx = widx;
+    cnt = wcnt;
+  }
+  AttnArgs a{q, k, v, o, lse_opt, idx, cnt, BH, N, d, bq, bk, nqb, nkb,
+             static_cast<float>(scale * 1.4426950408889634), 0};
+  cudaError_t e = launch_sparse_attn(a, st);
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_sparse_attn_fwd");
+}
+
+int sa_dense_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H, int N,
+                      int d, int bq, double scale, uint16_t* o, float* lse_opt, void* stream) {
+  int rc = check_shape(B, H, N, d, bq, 64);
+  if (rc) return rc;
+  if (!q || !k || !v || !o) return fail(SA_ERR_INVALID_ARG, "sa_dense_attn_fwd: null tensor pointer");
+  if (!isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "scale must be finite");
+  const void* ptrs[] = {q, k, v, o, lse_opt};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "sa_dense_attn_fwd: pointers must be 16-byte aligned");
+  if (scale <= 0.0) scale = 1.0 / sqrt(static_cast<double>(d));
+  const int BH = B * H;
+  const int nqb = (N + bq - 1) / bq, nkb = (N + 63) / 64;
+  AttnArgs a{q, k, v, o, lse_opt, nullptr, nullptr, BH, N, d, bq, 64, nqb, nkb,
+             static_cast<float>(scale * 1.4426950408889634), 1};
+  cudaError_t e = launch_sparse_attn(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_dense_attn_fwd");
+}
+
+size_t sa_linear_workspace_size(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d, 64, 64)) return 0;
+  return linear_state_ws_bytes(B * H, N, d);
+}
+
+int sa_linear_branch(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H, int N,
+                     int d, float* kv_state, float* ksum, uint16_t* o_l_opt, void* workspace,
+                     size_t ws_bytes, void* stream) {
+  int rc = check_shape(B, H, N, d, 64, 64);
+  if (rc) return rc;
+  if (!k || !v || !kv_state || !ksum) return fail(SA_ERR_INVALID_ARG, "sa_linear_branch: null pointer");
+  if (o_l_opt && !q) return fail(SA_ERR_INVALID_ARG, "sa_linear_branch: O_l needs q");
+  const void* ptrs[] = {q, k, v, kv_state, ksum, o_l_opt, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "sa_linear_branch: pointers must be 16-byte aligned");
+  const size_t need = linear_state_ws_bytes(B * H, N, d);
+  if (!workspace || ws_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "sa_linear_branch: workspace of %zu bytes needed", need);
+  LinearArgs a{q, k, v, nullptr, nullptr, kv_state, ksum, o_l_opt, B, H, N, d, workspace};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_linear_state(a, st);
+  if (e == cudaSuccess && o_l_opt) e = launch_linear_out(a, st);
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_linear_branch");
+}
+
+size_t sa_blend_workspace_size(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d, 64, 64)) return 0;
+  return linear_out_ws_bytes(B * H, d);
+}
+
+int sa_blend(const uint16_t* o_s, const uint16_t* q, const float* kv_state, const float* ksum,
+             const float* alpha, int B, int H, int N, int d, uint16_t* o, void* workspace,
+             size_t ws_bytes, void* stream) {
+  int rc = check_shape(B, H, N, d, 64, 64);
+  if (rc) return rc;
+  if (!o_s || !q || !kv_state || !ksum || !alpha || !o) return fail(SA_ERR_INVALID_ARG, "sa_blend: null pointer");
+  const void* ptrs[] = {o_s, q, kv_state, ksum, alpha, o, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "sa_blend: pointers must be 16-byte aligned");
+  const size_t need = linear_out_ws_bytes(B * H, d);
+  if (need && (!workspace || ws_bytes < need)) return fail(SA_ERR_WORKSPACE, "sa_blend: workspace of %zu bytes needed", need);
+  LinearArgs a{q, nullptr, nullptr, o_s, alpha, const_cast<float*>(kv_state), const_cast<float*>(ksum), o, B, H, N, d, workspace};
+  cudaError_t e = launch_linear_out(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_blend");
+}
+
+}  // extern "C"

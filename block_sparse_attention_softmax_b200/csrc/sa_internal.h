@@ -1,0 +1,65 @@
+// sa_internal.h — declarations shared by the translation units of libsa.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "sa_device.cuh"
+
+namespace sa {
+
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ inline int ceil_div_dev(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ inline long long ceil_div_ll(long long a, long long b) { return (a + b - 1) / b; }
+
+cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, int bq, int bk,
+                        float* q_pool, float* k_pool, cudaStream_t st);
+cudaError_t launch_scores(const float* q_pool, const float* k_pool, int BH, int nqb, int nkb,
+                          int d, double scale, float* s, long long s_ld, cudaStream_t st);
+cudaError_t launch_select(const float* s, long long s_ld, int n_rows, int nkb, int k_sel,
+                          double topp, int* kv_idx, int* kv_cnt, uint8_t* mask,
+                          cudaStream_t st);
+cudaError_t launch_compact_mask(const uint8_t* mask, int n_rows, int nkb, int* kv_idx,
+                                int* kv_cnt, cudaStream_t st);
+
+// Block-sparse attention over compacted lists. dense != 0 ignores the lists
+// and keeps every key block.
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  const int* kv_idx;
+  const int* kv_cnt;
+  int BH, N, d, bq, bk, nqb, nkb;
+  float scale_log2;
+  int dense;
+};
+cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t st);
+
+struct LinearArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o_s;      // blend input (may be null when only O_l is wanted)
+  const float* alpha;   // [H, d] or null (then O = O_l)
+  float* kv_state;
+  float* ksum;
+  void* o;
+  int B, H, N, d;
+  void* ws;
+};
+size_t linear_state_ws_bytes(int BH, int N, int d);
+size_t linear_out_ws_bytes(int BH, int d);
+cudaError_t launch_linear_state(const LinearArgs& a, cudaStream_t st);
+cudaError_t launch_linear_out(const LinearArgs& a, cudaStream_t st);
+
+// Driver entry point for cuTensorMapEncodeTiled, resolved once.
+CUresult encode_tensor_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t inner,
+                                   uint64_t rows, uint64_t planes, uint32_t box_inner,
+                                   uint32_t box_rows);
+
+}  // namespace sa

@@ -1,0 +1,142 @@
+/*
+ * sa.h — C ABI of the B200 block-sparse attention library (libsa.so).
+ *
+ * The operation (pages: "SpargeAttention2: 論文の技術的サマリー" §2(1) and §2(3);
+ * "SLA2" 提案手法 ① and ②; "SALAD" §2.1):
+ *   1. Q and K are mean-pooled per head into query blocks of bq tokens and key
+ *      blocks of bk tokens (SLA2 ①: mean pooling before scoring).
+ *   2. Block scores s[qb,kb] = scale * <Qbar[qb], Kbar[kb]>; a softmax over kb
+ *      turns each query-block row into probabilities P (SpargeAttention2 §2(1)
+ *      needs a cumulative probability, which implies this softmax).
+ *   3. Each row keeps Top-k ∪ Top-p: the ceil(k * n_kb) highest-scoring key
+ *      blocks, united with the smallest set of highest-probability blocks whose
+ *      probabilities sum to at least p (SpargeAttention2 §2(1)).
+ *   4. FlashAttention-style attention over the kept (query-block, key-block)
+ *      tiles only; masked tiles are skipped (SpargeAttention2 §2(3)).
+ *   5. Optional linear branch phi(x) = elu(x) + 1 over all keys (SALAD §2.1)
+ *      blended as O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l (SLA2 ②).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are device pointers, row-major and contiguous:
+ *       Q, K, V, O      [B, H, N, d]  bf16 (passed as uint16_t bit patterns)
+ *       q_pool          [B, H, n_qb, d] fp32,  n_qb = ceil(N / bq)
+ *       k_pool          [B, H, n_kb, d] fp32,  n_kb = ceil(N / bk)
+ *       kv_idx          [B, H, n_qb, n_kb] int32; row r holds kv_cnt[r] kept
+ *                       key-block indices in ascending order; the remaining
+ *                       entries of the row are left unspecified
+ *       kv_cnt          [B, H, n_qb] int32
+ *       mask            [B, H, n_qb, n_kb] uint8 (1 = kept)
+ *       lse             [B, H, N] fp32, natural-log log-sum-exp of each row
+ *       kv_state        [B, H, d, d] fp32, S = sum_j phi(k_j) v_j^T
+ *       ksum            [B, H, d] fp32, z = sum_j phi(k_j)
+ *       alpha           [H, d] fp32
+ *   - Supported shapes: d in {64, 128}; bq in {64, 128}; bk = 64; N >= 1;
+ *     B*H >= 1; every element count below 2^31 per tensor. Other values give
+ *     SA_ERR_UNSUPPORTED.
+ *   - Every device pointer must be 16-byte aligned (SA_ERR_ALIGN otherwise).
+ *   - The caller owns every buffer. The library allocates no device memory; a
+ *     call that needs scratch takes a caller-provided workspace whose size the
+ *     matching *_workspace_size() function returns (0 means none needed).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call is
+ *     asynchronous on it; argument errors are returned before anything is
+ *     launched, launch errors as SA_ERR_CUDA.
+ *   - Device-side waits are bounded. A wait that runs out records
+ *     SA_ERR_DEVICE_TIMEOUT in a device status word, the kernel skips its
+ *     remaining work and returns; sa_device_status() reads and clears it.
+ *   - No exception or abort crosses this boundary. sa_last_error() returns a
+ *     human-readable message for the last failing call on the calling thread.
+ */
+#ifndef SA_H_
+#define SA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SA_OK                   0
+#define SA_ERR_INVALID_ARG     -1
+#define SA_ERR_UNSUPPORTED     -2
+#define SA_ERR_ALIGN           -3
+#define SA_ERR_CUDA            -4
+#define SA_ERR_DEVICE_TIMEOUT  -5
+#define SA_ERR_WORKSPACE       -6
+
+/* Version of this ABI (major * 100 + minor). */
+int sa_version(void);
+
+/* Name of a status code ("SA_OK", "SA_ERR_INVALID_ARG", ...). Never NULL. */
+const char* sa_status_string(int status);
+
+/* Message describing the last failing call made by this thread ("" if none). */
+const char* sa_last_error(void);
+
+/* Synchronises `stream`, then returns and clears the device status word:
+ * SA_OK, or SA_ERR_DEVICE_TIMEOUT if a bounded device-side wait ran out. */
+int sa_device_status(void* stream);
+
+/* Step 1 alone (SLA2 提案手法 ①): block means of Q and K over valid tokens.
+ * The last block of a row may be partial and is averaged over its own tokens. */
+int sa_pool_blocks(const uint16_t* q, const uint16_t* k, int B, int H, int N, int d,
+                   int bq, int bk, float* q_pool, float* k_pool, void* stream);
+
+/* Steps 1-3: hybrid Top-k ∪ Top-p block mask (SpargeAttention2 §2(1)).
+ *   topk_frac  in (0, 1]: Top-k keeps K_sel = min(n_kb, max(1, ceil(k*n_kb - 1e-9)))
+ *   topp       in [0, 1]: Top-p keeps the smallest m >= 1 such that the m most
+ *              probable blocks sum to >= p; p >= 1 keeps every block
+ *   scale      score scale; <= 0 selects 1/sqrt(d)
+ * Order used by both rules: score descending, equal scores by lower block index.
+ * The kept set of a row is therefore the first max(K_sel, m_p) blocks of that
+ * order. Outputs kv_idx/kv_cnt (required) and, when non-NULL, the uint8 mask
+ * and the pooled Q/K. Needs sa_build_mask_workspace_size() bytes of workspace. */
+size_t sa_build_mask_workspace_size(int B, int H, int N, int d, int bq, int bk);
+int sa_build_mask(const uint16_t* q, const uint16_t* k, int B, int H, int N, int d,
+                  int bq, int bk, double topk_frac, double topp, double scale,
+                  int32_t* kv_idx, int32_t* kv_cnt, uint8_t* mask_opt,
+                  float* q_pool_opt, float* k_pool_opt,
+                  void* workspace, size_t ws_bytes, void* stream);
+
+/* Step 4 (SpargeAttention2 §2(3)): O_s[i] = sum over keys j of the kept key
+ * blocks of softmax_j(scale * q_i . k_j) v_j, with fp32 online softmax and
+ * bf16 tensor-core products; tiles not kept are never loaded or computed.
+ * Exactly one of (kv_idx, kv_cnt) or ext_mask must be given. With ext_mask the
+ * uint8 mask is first compacted into the workspace
+ * (sa_sparse_attn_workspace_size(); 0 bytes are needed for the list form).
+ * A row with no kept block outputs zeros and lse = -inf. lse_opt may be NULL.
+ * scale <= 0 selects 1/sqrt(d). */
+size_t sa_sparse_attn_workspace_size(int B, int H, int N, int d, int bq, int bk, int ext_mask);
+int sa_sparse_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                       int B, int H, int N, int d, int bq, int bk,
+                       const int32_t* kv_idx, const int32_t* kv_cnt, const uint8_t* ext_mask,
+                       double scale, uint16_t* o, float* lse_opt,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* Dense attention through the same kernel, every tile kept (the comparison
+ * point for the sparse speed-up). */
+int sa_dense_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                      int B, int H, int N, int d, int bq, double scale,
+                      uint16_t* o, float* lse_opt, void* stream);
+
+/* Step 5a (SALAD §2.1): kv_state = sum_j phi(k_j) v_j^T and ksum = sum_j phi(k_j)
+ * over all N keys, phi(x) = elu(x) + 1 (phi(k) rounded to bf16, fp32 sums).
+ * When o_l_opt is non-NULL also writes O_l[i] = phi(q_i)^T S / phi(q_i)^T z. */
+size_t sa_linear_workspace_size(int B, int H, int N, int d);
+int sa_linear_branch(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                     int B, int H, int N, int d, float* kv_state, float* ksum,
+                     uint16_t* o_l_opt, void* workspace, size_t ws_bytes, void* stream);
+
+/* Step 5b (SLA2 ②): O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l with O_l computed from
+ * q, kv_state and ksum inside the same kernel (the blend is its epilogue).
+ * o may alias o_s. Needs sa_blend_workspace_size() bytes of workspace. */
+size_t sa_blend_workspace_size(int B, int H, int N, int d);
+int sa_blend(const uint16_t* o_s, const uint16_t* q, const float* kv_state, const float* ksum,
+             const float* alpha, int B, int H, int N, int d, uint16_t* o,
+             void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_H_ */

@@ -1,0 +1,247 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Masks must equal the oracle's except at reported near-ties; attention, linear
+branch and blend outputs computed on the oracle's own mask must stay within
+max |err| <= 2e-2 and mean |err| <= 2e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_softmax_b200.workloads import WORKLOADS, make_inputs, random_qkv
+from gpu_helpers import MAX_ABS, MEAN_ABS, assert_close, compare_mask_rows, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _f64(t):
+    return oracle.as_f64(t)
+
+
+def _oracle_head_mask(q, k, b, h, bq, bk, topk, topp):
+    return oracle.build_mask(_f64(q[b, h]), _f64(k[b, h]), bq, bk, topk, topp)
+
+
+def _check_masks(sa, q, k, bq, bk, topk, topp, heads):
+    B, H, N, d = q.shape
+    out = sa.sa_build_mask(q, k, bq, bk, topk, topp, want_mask=True, want_pools=True)
+    torch.cuda.synchronize()
+    idx = out["kv_idx"].cpu().numpy()
+    cnt = out["kv_cnt"].cpu().numpy()
+    msk = out["mask"].cpu().numpy().astype(bool)
+    totals = {"exact": 0, "score_tie": 0, "cumsum_tie": 0}
+    ora_masks = {}
+    for (b, h) in heads:
+        ref = _oracle_head_mask(q, k, b, h, bq, bk, topk, topp)
+        ora_masks[(b, h)] = ref
+        # pooled means: fp32 sums of bf16 values
+        assert_close(out["q_pool"][b, h].cpu().numpy(), ref["q_pool"], "q_pool", 1e-5, 1e-6)
+        assert_close(out["k_pool"][b, h].cpu().numpy(), ref["k_pool"], "k_pool", 1e-5, 1e-6)
+        st = compare_mask_rows(idx[b, h], cnt[b, h], ref["s"], topk, topp)
+        assert not st["bad"], f"head {(b, h)}: rows differ beyond ties: {st['bad'][:3]}"
+        for key in totals:
+            totals[key] += st[key]
+        # kv lists are ascending and agree with the uint8 mask
+        for r in range(idx.shape[2]):
+            row = idx[b, h, r, :cnt[b, h, r]]
+            assert (np.diff(row) > 0).all()
+            assert set(row.tolist()) == set(np.nonzero(msk[b, h, r])[0].tolist())
+    return out, ora_masks, totals
+
+
+def _oracle_attention_rows(q, k, v, mask, b, h, bq, bk, rows):
+    return oracle.masked_attention(_f64(q[b, h]), _f64(k[b, h]), _f64(v[b, h]), mask, bq, bk, rows=rows)
+
+
+# ------------------------------------------------------------------ tiny: everything, every row
+def test_tiny_workload_full(cuda_lib):
+    sa = cuda_lib
+    wl = WORKLOADS["tiny"]
+    x = make_inputs(wl, "cpu")
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    heads = [(0, h) for h in range(wl.H)]
+    out, ora, totals = _check_masks(sa, q, k, wl.bq, wl.bk, wl.topk, wl.topp, heads)
+    print("tiny mask rows:", totals)
+    ext = torch.zeros(1, wl.H, wl.n_qb, wl.n_kb, dtype=torch.uint8)
+    for (b, h), ref in ora.items():
+        ext[b, h] = torch.from_numpy(ref["mask"].astype(np.uint8))
+    o, lse = sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, ext_mask=ext.to(DEV), want_lse=True)
+    o_list = sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=out["kv_idx"], kv_cnt=out["kv_cnt"])
+    torch.cuda.synchronize()
+    for (b, h), ref in ora.items():
+        ro, rl = _oracle_attention_rows(q.cpu(), k.cpu(), v.cpu(), ref["mask"], b, h, wl.bq, wl.bk, None)
+        assert_close(o[b, h].float().cpu().numpy(), ro, f"O head {h}")
+        assert_close(lse[b, h].cpu().numpy(), rl, f"LSE head {h}", 1e-2, 1e-3)
+        same = (out["mask"][b, h].cpu().numpy().astype(bool) == ref["mask"]).all(axis=1)
+        rows_same = np.repeat(same, wl.bq)[:wl.N]
+        assert torch.equal(o_list[b, h][torch.from_numpy(rows_same).to(DEV)],
+                           o[b, h][torch.from_numpy(rows_same).to(DEV)])
+    sa.sa_device_status()
+
+
+def test_tiny_golden_lists(cuda_lib):
+    """The GPU lists reproduce the stored oracle fixture for the tiny workload."""
+    import os
+    sa = cuda_lib
+    wl = WORKLOADS["tiny"]
+    x = make_inputs(wl, "cpu")
+    out = sa.sa_build_mask(x["q"].to(DEV), x["k"].to(DEV), wl.bq, wl.bk, wl.topk, wl.topp)
+    idx, cnt = out["kv_idx"].cpu().numpy(), out["kv_cnt"].cpu().numpy()
+    path = os.path.join(os.path.dirname(__file__), "golden", "tiny_kv_lists.txt")
+    mism = 0
+    for line in open(path):
+        if line.startswith("#"):
+            continue
+        h, r, c, rest = line.split(":")
+        want = [int(t) for t in rest.split()]
+        got = idx[0, int(h), int(r), :cnt[0, int(h), int(r)]].tolist()
+        mism += got != want
+    assert mism == 0
+
+
+# ------------------------------------------------------------------ ragged / edge shapes
+@pytest.mark.parametrize("N,d,bq,H", [(1, 64, 64, 1), (65, 128, 128, 2), (200, 128, 64, 1),
+                                      (333, 64, 128, 3), (1000, 128, 128, 2), (4099, 128, 128, 1)])
+def test_ragged_shapes(cuda_lib, N, d, bq, H):
+    sa = cuda_lib
+    bk = 64
+    q, k, v = random_qkv(1, H, N, d, seed=N * 7 + d, device=DEV)
+    q = (q.float() * 3.0).to(torch.bfloat16)  # sharper block scores
+    heads = [(0, h) for h in range(H)]
+    out, ora, _ = _check_masks(sa, q, k, bq, bk, 0.2, 0.8, heads)
+    ext = torch.zeros(1, H, -(-N // bq), -(-N // bk), dtype=torch.uint8)
+    for (b, h), ref in ora.items():
+        ext[b, h] = torch.from_numpy(ref["mask"].astype(np.uint8))
+    o, lse = sa.sa_sparse_attn_fwd(q, k, v, bq, bk, ext_mask=ext.to(DEV), want_lse=True)
+    torch.cuda.synchronize()
+    for (b, h), ref in ora.items():
+        ro, rl = _oracle_attention_rows(q.cpu(), k.cpu(), v.cpu(), ref["mask"], b, h, bq, bk, None)
+        assert_close(o[b, h].float().cpu().numpy(), ro, f"O N={N}")
+        assert_close(lse[b, h].cpu().numpy(), rl, f"LSE N={N}", 1e-2, 1e-3)
+    sa.sa_device_status()
+
+
+def test_empty_rows_and_all_ones(cuda_lib):
+    sa = cuda_lib
+    N, d, bq, bk, H = 300, 128, 128, 64, 2
+    q, k, v = random_qkv(1, H, N, d, seed=5, device=DEV)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    ext = torch.ones(1, H, nqb, nkb, dtype=torch.uint8)
+    ext[0, 0, 1] = 0                              # a row with no kept block
+    o, lse = sa.sa_sparse_attn_fwd(q, k, v, bq, bk, ext_mask=ext.to(DEV), want_lse=True)
+    torch.cuda.synchronize()
+    assert (o[0, 0, bq:2 * bq] == 0).all()
+    assert torch.isneginf(lse[0, 0, bq:2 * bq]).all()
+    ref, rl = oracle.dense_attention(_f64(q[0, 1]), _f64(k[0, 1]), _f64(v[0, 1]))
+    assert_close(o[0, 1].float().cpu().numpy(), ref, "all-ones = dense")
+    # k = 100% gives the all-ones mask through the builder too
+    m = sa.sa_build_mask(q, k, bq, bk, 1.0, 0.5)
+    assert (m["kv_cnt"] == nkb).all()
+    m = sa.sa_build_mask(q, k, bq, bk, 0.01, 1.0)
+    assert (m["kv_cnt"] == nkb).all()
+    # dense entry point = all-ones mask
+    od, ld = sa.sa_dense_attn_fwd(q, k, v, bq, want_lse=True)
+    ref0, rl0 = oracle.dense_attention(_f64(q[0, 0]), _f64(k[0, 0]), _f64(v[0, 0]))
+    assert_close(od[0, 0].float().cpu().numpy(), ref0, "dense entry point")
+    assert_close(ld[0, 0].cpu().numpy(), rl0, "dense LSE", 1e-2, 1e-3)
+    sa.sa_device_status()
+
+
+def test_uniform_scores_tie_order(cuda_lib):
+    """All-equal block scores: every block ties, lower index first."""
+    sa = cuda_lib
+    N, d, H = 1024, 64, 1
+    q = torch.zeros(1, H, N, d, dtype=torch.bfloat16, device=DEV)
+    _, k, v = random_qkv(1, H, N, d, seed=9, device=DEV)
+    m = sa.sa_build_mask(q, k, 64, 64, 0.1, 0.5)
+    cnt = m["kv_cnt"].cpu().numpy()
+    idx = m["kv_idx"].cpu().numpy()
+    # P = 1/16 each: the smallest m with m/16 >= 0.5 is 8 (exact in binary)
+    assert (cnt == 8).all()
+    assert (idx[0, 0, :, :8] == np.arange(8)).all()
+
+
+# ------------------------------------------------------------------ full-size workloads (sampled)
+FULL = ["wan13b_480p", "wan14b_720p", "sink_skew", "long_245k"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workload(cuda_lib, name):
+    sa = cuda_lib
+    wl = WORKLOADS[name]
+    x = make_inputs(wl, DEV)
+    q, k, v = x["q"], x["k"], x["v"]
+    rng = np.random.default_rng(wl.seed)
+    n_heads = 2 if wl.N > 100000 else 3
+    hs = sorted({0, wl.H - 1} | set(rng.choice(wl.H, size=n_heads, replace=False).tolist()))[:n_heads + 1]
+    if wl.kind == "sink" and x["flat_heads"]:
+        hs = sorted(set(hs) | {x["flat_heads"][0]})
+    heads = [(0, h) for h in hs]
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    out = sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp, want_mask=True)
+    torch.cuda.synchronize()
+    idx, cnt = out["kv_idx"].cpu().numpy(), out["kv_cnt"].cpu().numpy()
+    gmask = out["mask"].clone()
+    totals = {"exact": 0, "score_tie": 0, "cumsum_tie": 0}
+    ora = {}
+    for (b, h) in heads:
+        ref = _oracle_head_mask(qc, kc, b, h, wl.bq, wl.bk, wl.topk, wl.topp)
+        st = compare_mask_rows(idx[b, h], cnt[b, h], ref["s"], wl.topk, wl.topp)
+        assert not st["bad"], f"{name} head {h}: {st['bad'][:3]}"
+        for kk in totals:
+            totals[kk] += st[kk]
+        ora[(b, h)] = ref
+        gmask[b, h] = torch.from_numpy(ref["mask"].astype(np.uint8)).to(DEV)
+    density = float(cnt.sum()) / (wl.H * wl.n_qb * wl.n_kb)
+    print(f"{name}: mask rows {totals}, realised density {density:.4f}")
+    # attention on the oracle's mask for the sampled heads (GPU mask elsewhere)
+    o = sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, ext_mask=gmask)
+    o_list = sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=out["kv_idx"], kv_cnt=out["kv_cnt"])
+    torch.cuda.synchronize()
+    for (b, h), ref in ora.items():
+        rows = sample_rows(wl.n_qb, wl.bq, wl.N, ref["mask"].sum(1), rng)
+        ro, _ = _oracle_attention_rows(qc, kc, vc, ref["mask"], b, h, wl.bq, wl.bk, rows)
+        got = o[b, h][torch.from_numpy(rows).to(DEV)].float().cpu().numpy()
+        assert_close(got, ro, f"{name} O head {h}")
+        same = np.nonzero((out["mask"][b, h].cpu().numpy().astype(bool) == ref["mask"]).all(1))[0]
+        sel = torch.from_numpy(np.concatenate([np.arange(r * wl.bq, min(wl.N, (r + 1) * wl.bq)) for r in same[:8]])).to(DEV)
+        assert torch.equal(o_list[b, h][sel], o[b, h][sel])
+    if wl.linear:
+        alpha = x["alpha"]
+        S, z = sa.sa_linear_branch(q, k, v)
+        ob = sa.sa_blend(o, q, S, z, alpha)
+        torch.cuda.synchronize()
+        for (b, h) in heads[:2]:
+            kS, kz = oracle.linear_state(_f64(kc[b, h]), _f64(vc[b, h]))
+            # phi(k) is rounded to bf16 on the GPU: relative error ~4e-3 per term
+            assert np.abs(S[b, h].cpu().numpy() - kS).max() <= 5e-3 * np.abs(kS).max()
+            assert np.abs(z[b, h].cpu().numpy() - kz).max() <= 5e-3 * np.abs(kz).max()
+            rows = sample_rows(wl.n_qb, wl.bq, wl.N, ora[(b, h)]["mask"].sum(1), rng)
+            ro, _ = _oracle_attention_rows(qc, kc, vc, ora[(b, h)]["mask"], b, h, wl.bq, wl.bk, rows)
+            ol = oracle.linear_out(_f64(qc[b, h])[rows], kS, kz)
+            ref = oracle.blend(ro, ol, alpha[h].double().cpu().numpy())
+            assert_close(ob[b, h][torch.from_numpy(rows).to(DEV)].float().cpu().numpy(), ref, f"{name} blend head {h}")
+    sa.sa_device_status()
+
+
+def test_linear_branch_small(cuda_lib):
+    sa = cuda_lib
+    for (N, d) in [(1000, 128), (257, 64)]:
+        q, k, v = random_qkv(1, 2, N, d, seed=N, device=DEV)
+        S, z, ol = sa.sa_linear_branch(q, k, v, want_ol=True)
+        alpha = torch.rand(2, d, device=DEV)
+        os_ = torch.randn_like(q.float()).to(torch.bfloat16)
+        ob = sa.sa_blend(os_, q, S, z, alpha)
+        torch.cuda.synchronize()
+        for h in range(2):
+            kS, kz = oracle.linear_state(_f64(k[0, h]), _f64(v[0, h]))
+            ref_l = oracle.linear_out(_f64(q[0, h]), kS, kz)
+            assert_close(ol[0, h].float().cpu().numpy(), ref_l, f"O_l N={N}")
+            ref_b = oracle.blend(_f64(os_[0, h]), ref_l, alpha[h].double().cpu().numpy())
+            assert_close(ob[0, h].float().cpu().numpy(), ref_b, f"blend N={N}")
+    sa.sa_device_status()
