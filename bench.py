@@ -217,14 +217,15 @@ def run_ours(args, wl, rank, world, local):
     if not args.no_e2e:
         qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
         ah = alpha.cpu().pin_memory() if alpha is not None else None
-        sa.block_sparse_attention(qh, kh, vh, wl.bq, wl.bk, wl.topk, wl.topp, alpha=ah)
+        oh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        sa.block_sparse_attention(qh, kh, vh, wl.bq, wl.bk, wl.topk, wl.topp, alpha=ah, out=oh)
         torch.cuda.synchronize()
         reps = max(2, min(args.steps, 5))
         tt0 = time.perf_counter()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(reps):
-            sa.block_sparse_attention(qh, kh, vh, wl.bq, wl.bk, wl.topk, wl.topp, alpha=ah)
+            sa.block_sparse_attention(qh, kh, vh, wl.bq, wl.bk, wl.topk, wl.topp, alpha=ah, out=oh)
         e1.record()
         torch.cuda.synchronize()
         e2e_ms = max(e0.elapsed_time(e1), (time.perf_counter() - tt0) * 1e3) / reps

@@ -200,10 +200,11 @@ def sa_blend(o_s, q, kv_state, ksum, alpha, out=None, workspace=None):
 
 
 def block_sparse_attention(q, k, v, bq=128, bk=64, topk=0.05, topp=0.9, alpha=None, scale=0.0,
-                           device=None):
+                           device=None, out=None):
     """Whole path: mask, sparse attention and (when alpha is given) the linear
-    branch blended in. Host tensors are copied to the device and the result
-    copied back; device tensors stay on the device."""
+    branch blended in. Host tensors are copied to the device and the result is
+    copied back into `out` (a pinned host tensor is allocated when out is None);
+    device tensors stay on the device."""
     host = not q.is_cuda
     if host:
         device = device or torch.device("cuda", torch.cuda.current_device())
@@ -216,5 +217,9 @@ def block_sparse_attention(q, k, v, bq=128, bk=64, topk=0.05, topp=0.9, alpha=No
         S, z = sa_linear_branch(q, k, v)
         o = sa_blend(o, q, S, z, alpha, out=o)
     if host:
-        o = o.to("cpu", non_blocking=False)
+        if out is None:
+            out = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        out.copy_(o, non_blocking=True)
+        torch.cuda.current_stream(device).synchronize()
+        return out
     return o

@@ -1,102 +1,250 @@
 // linear_kernels.cu — the parallel linear-attention branch and the alpha blend
-// (pages: "SALAD" §2.1, a linear-attention branch beside sparse attention over
-// the same Q/K/V; "SLA2" 提案手法 ②, O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l).
+// on the sm_100a tensor cores (pages: "SALAD" §2.1, a linear-attention branch
+// beside sparse attention over the same Q/K/V; "SLA2" 提案手法 ②,
+// O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l).
 //
 // phi(x) = elu(x) + 1. For each head:
 //   state:  S = sum_j phi(k_j) v_j^T  [d, d],  z = sum_j phi(k_j)  [d]
 //   output: O_l[i] = phi(q_i)^T S / phi(q_i)^T z
 //   blend:  O[i]   = alpha ⊙ O_s[i] + (1 - alpha) ⊙ O_l[i]
-// The state is summed over token splits into a fp32 workspace, then reduced in
-// a fixed order, so results do not depend on scheduling.
+//
+// linear_state_kernel: one CTA per (token split, head). K and V tiles of 128
+//   tokens arrive by TMA; four warps apply phi to the K tile in shared memory
+//   (rounding phi(k) to bf16) and sum z; one thread issues
+//   tcgen05.mma D[f, e] += phi(K)^T[f, t] V[t, e] with both operands MN-major,
+//   accumulating the split's S in TMEM. Partials are reduced in a fixed order.
+// linear_out_kernel: each CTA stages [S | z] of its head in shared memory as a
+//   bf16 hi + lo pair (two MMAs recover ~16 mantissa bits), then for each
+//   128-token tile: TMA Q, phi in place, D[t, :] = phi(Q)[t, :] [S | z] in TMEM
+//   (double buffered), and an epilogue that divides by the z column and blends
+//   with O_s.
 #include "sa_internal.h"
 
 namespace sa {
 
-namespace {
-constexpr int kLinThreads = 256;
-constexpr int kLinTok = 32;      // tokens staged per step
-constexpr int kSplitTokens = 512;
+namespace lin {
 
-__device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : expf(x); }
+constexpr int kLinTok = 128;       // tokens per tile (K extent of the state MMA)
+constexpr int kLinThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 math
+constexpr int kLinStages = 3;
 
-__device__ __forceinline__ float bf16_bits_to_f(uint16_t b) {
-  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+__device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+
+int splits(int BH, int N) {
+  const int tiles = ceil_div(N, kLinTok);
+  const int want = ceil_div(2 * 148, BH);
+  return max(1, min(tiles, want));
 }
 
-int linear_splits(int BH, int N) {
-  const int by_tokens = ceil_div(N, kSplitTokens);
-  const int want = ceil_div(4 * 148, BH);
-  return max(1, min(by_tokens, want));
+int tiles_per_split(int BH, int N) {
+  return ceil_div(ceil_div(N, kLinTok), splits(BH, N));
 }
-}  // namespace
+
+template <int D>
+struct StateLayout {
+  static constexpr uint32_t CHUNK = kLinTok * 128;               // 128 tokens x 64 features
+  static constexpr uint32_t K_BYTES = 2 * CHUNK;              // A operand spans M = 128 features
+  static constexpr uint32_t V_BYTES = (D / 64) * CHUNK;
+  static constexpr uint32_t STAGE = K_BYTES + V_BYTES;
+  static constexpr uint32_t OFF_BAR = kLinStages * STAGE;
+  static constexpr uint32_t OFF_Z = OFF_BAR + 256;            // [8 or 16 phases][D] fp32
+  static constexpr uint32_t SMEM = OFF_Z + 16 * D * 4 + 1024;
+};
+
+template <int D>
+struct OutLayout {
+  static constexpr int NB = D + 16;                           // MMA N: S columns + z column
+  static constexpr int B_CHUNKS = (NB + 63) / 64;
+  static constexpr uint32_t B_CHUNK = D * 128;                // D rows (K) x 64 columns
+  static constexpr uint32_t B_BYTES = B_CHUNKS * B_CHUNK;     // one of hi / lo
+  static constexpr uint32_t Q_CHUNK = kLinTok * 128;
+  static constexpr uint32_t Q_BYTES = (D / 64) * Q_CHUNK;
+  static constexpr uint32_t OFF_B = 0;
+  static constexpr uint32_t OFF_Q = 2 * B_BYTES;
+  static constexpr uint32_t OFF_ALPHA = OFF_Q + kLinStages * Q_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_ALPHA + D * 4;
+  static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
+  static constexpr uint32_t ACC_STRIDE = NB <= 128 ? 128 : 256;   // TMEM columns per buffer
+  static constexpr uint32_t TM_COLS = 2 * ACC_STRIDE;
+};
+
+__device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+}  // namespace lin
 
 size_t linear_state_ws_bytes(int BH, int N, int d) {
-  return static_cast<size_t>(BH) * linear_splits(BH, N) * (static_cast<size_t>(d) * d + d) * sizeof(float);
+  return static_cast<size_t>(BH) * lin::splits(BH, N) * (static_cast<size_t>(d) * d + d) * sizeof(float);
 }
 
 size_t linear_out_ws_bytes(int, int) { return 0; }
 
-// Partial state of one token split. Thread (ti, tj) of a 16 x 16 grid owns
-// rows [ti*D/16, +D/16) and columns [tj*D/16, +D/16) of S.
+// ---------------------------------------------------------------- state
 template <int D>
-__global__ void __launch_bounds__(kLinThreads) linear_state_kernel(
-    const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, int N, int nsplit,
-    float* __restrict__ part) {
-  constexpr int R = D / 16;
-  __shared__ float fk[kLinTok][D];
-  __shared__ float vv[kLinTok][D];
+__global__ void __launch_bounds__(lin::kLinThreads, 1)
+    linear_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        int N, int nsplit, int tiles_per_split, float* __restrict__ part) {
+  using L = lin::StateLayout<D>;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = lin::align1k(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* full = bars;                 // [lin::kLinStages] TMA landed
+  uint64_t* phi_done = bars + lin::kLinStages;   // [lin::kLinStages] phi applied (4 warps)
+  uint64_t* empty = bars + 2 * lin::kLinStages;  // [lin::kLinStages] MMA consumed
+  uint64_t* done = bars + 3 * lin::kLinStages;   // all MMAs complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* zs = reinterpret_cast<float*>(smem + L::OFF_Z);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, bh = blockIdx.y;
-  const int per = ceil_div_dev(N, nsplit);
-  const int t0 = split * per, t1 = min(N, t0 + per);
-  const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
-  float acc[R][R];
-#pragma unroll
-  for (int i = 0; i < R; ++i)
-#pragma unroll
-    for (int j = 0; j < R; ++j) acc[i][j] = 0.f;
-  float zacc[R];
-#pragma unroll
-  for (int i = 0; i < R; ++i) zacc[i] = 0.f;
-  const uint16_t* kb = k + static_cast<long long>(bh) * N * D;
-  const uint16_t* vb = v + static_cast<long long>(bh) * N * D;
-  for (int t = t0; t < t1; t += kLinTok) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < kLinTok * D; e += blockDim.x) {
-      const int r = e / D, c = e % D;
-      const int tok = t + r;
-      float a = 0.f, b = 0.f;
-      if (tok < t1) {
-        // phi(k) is rounded to bf16, as the tensor-core form of this branch does
-        a = __bfloat162float(__float2bfloat16_rn(phi_f(bf16_bits_to_f(kb[static_cast<long long>(tok) * D + c]))));
-        b = bf16_bits_to_f(vb[static_cast<long long>(tok) * D + c]);
-      }
-      fk[r][c] = a;
-      vv[r][c] = b;
+  const int tile0 = split * tiles_per_split;
+  const int n_tiles = max(0, min(tiles_per_split, ceil_div_dev(N, lin::kLinTok) - tile0));
+  const int t_end = N;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < lin::kLinStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&phi_done[s], 4);
+      mbar_init(&empty[s], 1);
     }
-    __syncthreads();
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (D == 64) {
+    // the A operand always spans 128 features: zero the upper half once
+    for (int s = 0; s < lin::kLinStages; ++s)
+      for (int i = threadIdx.x; i < static_cast<int>(L::CHUNK / 16); i += blockDim.x)
+        reinterpret_cast<uint4*>(smem + s * L::STAGE + L::CHUNK)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % lin::kLinStages;
+        if (!mbar_wait(&empty[s], ((i / lin::kLinStages) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[s], (D / 64) * 2 * L::CHUNK);
+        uint8_t* st = smem + s * L::STAGE;
+        const int row = (tile0 + i) * lin::kLinTok;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(st + c * L::CHUNK, &tmK, &full[s], c * 64, row, bh);
+          tma_load_3d(st + L::K_BYTES + c * L::CHUNK, &tmV, &full[s], c * 64, row, bh);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, D, true, true);
+      for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % lin::kLinStages;
+        if (!mbar_wait(&phi_done[s], (i / lin::kLinStages) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t kb = smem_u32(smem + s * L::STAGE);
+        const uint32_t vb = kb + L::K_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < lin::kLinTok / 16; ++kk) {
+          const uint64_t a = sw128_desc(kb + kk * 2048u, L::CHUNK, 1024);
+          const uint64_t b = sw128_desc(vb + kk * 2048u, L::CHUNK, 1024);
+          umma_ss(tm, a, b, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&empty[s]);
+      }
+      tc_commit(done);
+    }
+  } else {
+    // math warps: phi on the K tile, z sums, then the epilogue
+    constexpr int NG = D / 8;            // 8-feature groups
+    constexpr int NP = 128 / NG;         // token phases
+    const int mt = threadIdx.x - 64;
+    const int gi = mt % NG, phase = mt / NG;
+    const int chunk = gi / 8, lu = gi % 8;
+    const int pu = lu ^ (phase % 8);     // physical 16-B unit (t % 8 == phase % 8 for every visited token)
+    float z[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) z[e] = 0.f;
+    bool ok = true;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int s = i % lin::kLinStages;
+      if (!mbar_wait(&full[s], (i / lin::kLinStages) & 1, abort_flag)) { ok = false; break; }
+      uint8_t* kt = smem + s * L::STAGE + chunk * L::CHUNK + pu * 16;
+      const int tok0 = (tile0 + i) * lin::kLinTok;
 #pragma unroll 4
-    for (int r = 0; r < kLinTok; ++r) {
-      float av[R], bv[R];
+      for (int t = phase; t < lin::kLinTok; t += NP) {
+        uint4* p = reinterpret_cast<uint4*>(kt + t * 128);
+        uint4 w = *p;
+        uint32_t* u = reinterpret_cast<uint32_t*>(&w);
+        if (tok0 + t < t_end) {
 #pragma unroll
-      for (int i = 0; i < R; ++i) av[i] = fk[r][ti * R + i];
+          for (int e = 0; e < 4; ++e) {
+            const float a = lin::phi_f(__uint_as_float(u[e] << 16));
+            const float b = lin::phi_f(__uint_as_float(u[e] & 0xFFFF0000u));
+            const uint32_t pk = pack_bf16x2(a, b);
+            u[e] = pk;
+            z[2 * e] += __uint_as_float(pk << 16);
+            z[2 * e + 1] += __uint_as_float(pk & 0xFFFF0000u);
+          }
+        } else {
+          w = make_uint4(0, 0, 0, 0);
+        }
+        *p = w;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&phi_done[s]);
+    }
+    // z partial: phases of one feature group are summed in a fixed order
 #pragma unroll
-      for (int j = 0; j < R; ++j) bv[j] = vv[r][tj * R + j];
+    for (int e = 0; e < 8; ++e) zs[phase * D + gi * 8 + e] = z[e];
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    float* out = part + (static_cast<long long>(bh) * nsplit + split) * (D * D + D);
+    if (mt < D) {
+      float acc = 0.f;
+      for (int ph = 0; ph < NP; ++ph) acc += zs[ph * D + mt];
+      out[D * D + mt] = acc;
+    }
+    // S rows: TMEM lane = feature row of phi(K)^T
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    if (ok && n_tiles > 0) ok = mbar_wait(done, 0, abort_flag);
+    tc_fence_after();
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t r[32];
+      if (ok && n_tiles > 0) {
+        tmem_ld32_wait(tm + (static_cast<uint32_t>(quad * 32) << 16) + c0, r);
+      } else {
 #pragma unroll
-      for (int i = 0; i < R; ++i) {
+        for (int e = 0; e < 32; ++e) r[e] = 0u;
+      }
+      if (row < D) {
+        float4* dst = reinterpret_cast<float4*>(out + row * D + c0);
 #pragma unroll
-        for (int j = 0; j < R; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-        if (tj == 0) zacc[i] += av[i];
+        for (int e = 0; e < 8; ++e)
+          dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                               __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
       }
     }
   }
-  float* out = part + (static_cast<long long>(bh) * nsplit + split) * (D * D + D);
-#pragma unroll
-  for (int i = 0; i < R; ++i)
-#pragma unroll
-    for (int j = 0; j < R; ++j) out[(ti * R + i) * D + tj * R + j] = acc[i][j];
-  if (tj == 0) {
-#pragma unroll
-    for (int i = 0; i < R; ++i) out[D * D + ti * R + i] = zacc[i];
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tm, 128);
   }
 }
 
@@ -113,108 +261,240 @@ __global__ void linear_reduce_kernel(const float* __restrict__ part, int nsplit,
   else ksum[static_cast<long long>(bh) * D + (e - D * D)] = s;
 }
 
-// O_l (and the blend) for a tile of 64 tokens of one head. Thread (tr, tc) of a
-// 16 x 16 grid computes tokens [tr*4, +4) and columns [tc*D/16, +D/16).
-constexpr int kOutTok = 64;
-
+// ---------------------------------------------------------------- output + blend
 template <int D>
-__global__ void __launch_bounds__(kLinThreads) linear_out_kernel(
-    const uint16_t* __restrict__ q, const float* __restrict__ kv_state,
-    const float* __restrict__ ksum, const uint16_t* __restrict__ o_s,
-    const float* __restrict__ alpha, int H, int N, uint16_t* __restrict__ o) {
-  constexpr int C = D / 16;
-  extern __shared__ float sm_lin[];
-  float* S = sm_lin;                 // [D][D]
-  float* z = S + D * D;              // [D]
-  float* fq = z + D;                 // [kOutTok][D + 1]
-  const int tile = blockIdx.x, bh = blockIdx.y;
+__global__ void __launch_bounds__(lin::kLinThreads, 1)
+    linear_out_kernel(const __grid_constant__ CUtensorMap tmQ, const float* __restrict__ kv_state,
+                      const float* __restrict__ ksum, const uint16_t* __restrict__ o_s,
+                      const float* __restrict__ alpha, int H, int N, int tiles_per_cta,
+                      uint16_t* __restrict__ o) {
+  using L = lin::OutLayout<D>;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = lin::align1k(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* full = bars;                    // [lin::kLinStages]
+  uint64_t* phi_done = bars + lin::kLinStages;      // [lin::kLinStages]
+  uint64_t* empty = bars + 2 * lin::kLinStages;     // [lin::kLinStages]
+  uint64_t* acc_full = bars + 3 * lin::kLinStages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* al = reinterpret_cast<float*>(smem + L::OFF_ALPHA);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
   const int h = bh % H;
-  const int tok0 = tile * kOutTok;
-  const float* Sg = kv_state + static_cast<long long>(bh) * D * D;
-  for (int e = threadIdx.x; e < D * D; e += blockDim.x) S[e] = Sg[e];
-  for (int e = threadIdx.x; e < D; e += blockDim.x) z[e] = ksum[static_cast<long long>(bh) * D + e];
-  const uint16_t* qb = q + static_cast<long long>(bh) * N * D;
-  for (int e = threadIdx.x; e < kOutTok * D; e += blockDim.x) {
-    const int r = e / D, c = e % D;
-    const int tok = tok0 + r;
-    float x = 0.f;
-    if (tok < N) x = __bfloat162float(__float2bfloat16_rn(phi_f(bf16_bits_to_f(qb[static_cast<long long>(tok) * D + c]))));
-    fq[r * (D + 1) + c] = x;
-  }
-  __syncthreads();
-  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
-  float acc[4][C];
-  float den[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    den[i] = 0.f;
-#pragma unroll
-    for (int j = 0; j < C; ++j) acc[i][j] = 0.f;
-  }
-  for (int c = 0; c < D; ++c) {
-    float av[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) av[i] = fq[(tr * 4 + i) * (D + 1) + c];
-    const float zc = z[c];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      den[i] = fmaf(av[i], zc, den[i]);
-#pragma unroll
-      for (int j = 0; j < C; ++j) acc[i][j] = fmaf(av[i], S[c * D + tc * C + j], acc[i][j]);
+  const int tile0 = blockIdx.x * tiles_per_cta;
+  const int n_tiles = max(0, min(tiles_per_cta, ceil_div_dev(N, lin::kLinTok) - tile0));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < lin::kLinStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&phi_done[s], 4);
+      mbar_init(&empty[s], 1);
     }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
   }
+  // B operand [S | z] as bf16 hi and lo, MN-major with 128-B swizzle:
+  // element (row c, column e) sits in chunk e/64, row c, 16-B unit ((e%64)/8) ^ (c%8).
+  {
+    const float* Sg = kv_state + static_cast<long long>(bh) * D * D;
+    const float* zg = ksum + static_cast<long long>(bh) * D;
+    constexpr int UPR = L::B_CHUNKS * 8;    // 16-B units per row (incl. zero padding)
+    for (int i = threadIdx.x; i < D * UPR; i += blockDim.x) {
+      const int c = i / UPR, u = i % UPR;
+      uint32_t hi[4], lo[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int tok = tok0 + tr * 4 + i;
-    if (tok >= N) continue;
-    const long long base = (static_cast<long long>(bh) * N + tok) * D + tc * C;
-    const float inv = 1.f / den[i];
+      for (int e2 = 0; e2 < 4; ++e2) {
+        float v2[2];
 #pragma unroll
-    for (int j = 0; j < C; ++j) {
-      float ol = acc[i][j] * inv;
-      if (alpha) {
-        const float al = alpha[static_cast<long long>(h) * D + tc * C + j];
-        ol = al * bf16_bits_to_f(o_s[base + j]) + (1.f - al) * ol;
+        for (int t = 0; t < 2; ++t) {
+          const int e = u * 8 + e2 * 2 + t;
+          v2[t] = e < D ? Sg[c * D + e] : (e == D ? zg[c] : 0.f);
+        }
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(v2[0], v2[1]);
+        const float2 hf = __bfloat1622float2(hb);
+        hi[e2] = *reinterpret_cast<const uint32_t*>(&hb);
+        lo[e2] = pack_bf16x2(v2[0] - hf.x, v2[1] - hf.y);
       }
-      __nv_bfloat16 r = __float2bfloat16_rn(ol);
-      o[base + j] = *reinterpret_cast<uint16_t*>(&r);
+      const uint32_t off = (u / 8) * L::B_CHUNK + c * 128 + (((u % 8) ^ (c % 8)) * 16);
+      *reinterpret_cast<uint4*>(smem + L::OFF_B + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(smem + L::OFF_B + L::B_BYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
+    for (int e = threadIdx.x; e < D; e += blockDim.x) al[e] = alpha ? alpha[static_cast<long long>(h) * D + e] : 0.f;
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_desc(&tmQ);
+      for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % lin::kLinStages;
+        if (!mbar_wait(&empty[s], ((i / lin::kLinStages) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[s], L::Q_BYTES);
+        uint8_t* st = smem + L::OFF_Q + s * L::Q_BYTES;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) tma_load_3d(st + c * L::Q_CHUNK, &tmQ, &full[s], c * 64, (tile0 + i) * lin::kLinTok, bh);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, L::NB, false, true);
+      const uint32_t bhi = smem_u32(smem + L::OFF_B), blo = bhi + L::B_BYTES;
+      for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % lin::kLinStages, b = i & 1;
+        if (!mbar_wait(&phi_done[s], (i / lin::kLinStages) & 1, abort_flag)) break;
+        if (!mbar_wait(&acc_empty[b], ((i >> 1) & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t qb = smem_u32(smem + L::OFF_Q + s * L::Q_BYTES);
+        const uint32_t d_tm = tm + b * L::ACC_STRIDE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = sw128_desc(qb + (kk >> 2) * L::Q_CHUNK + (kk & 3) * 32u, 16, 1024);
+          umma_ss(d_tm, a, sw128_desc(bhi + kk * 2048u, L::B_CHUNK, 1024), idesc, kk > 0 ? 1u : 0u);
+          umma_ss(d_tm, a, sw128_desc(blo + kk * 2048u, L::B_CHUNK, 1024), idesc, 1u);
+        }
+        tc_commit(&acc_full[b]);
+        tc_commit(&empty[s]);
+      }
+    }
+  } else {
+    const int mt = threadIdx.x - 64;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    bool ok = true;
+    auto epilogue = [&](int i) {
+      const int b = i & 1;
+      if (!mbar_wait(&acc_full[b], (i >> 1) & 1, abort_flag)) { ok = false; return; }
+      tc_fence_after();
+      const int tok = (tile0 + i) * lin::kLinTok + row;
+      uint32_t dz[32];
+      tmem_ld32_wait(tm + lane_addr + b * L::ACC_STRIDE + D, dz);
+      const float inv = 1.f / __uint_as_float(dz[0]);
+      const long long base = (static_cast<long long>(bh) * N + tok) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32_wait(tm + lane_addr + b * L::ACC_STRIDE + c0, r);
+        if (tok < N) {
+          uint32_t pk[16];
+          if (o_s) {
+            const uint4* src = reinterpret_cast<const uint4*>(o_s + base + c0);
+            uint32_t os[16];
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              const uint4 w = src[v4];
+              os[4 * v4] = w.x; os[4 * v4 + 1] = w.y; os[4 * v4 + 2] = w.z; os[4 * v4 + 3] = w.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float a0 = al[c0 + 2 * e], a1 = al[c0 + 2 * e + 1];
+              const float l0 = __uint_as_float(r[2 * e]) * inv, l1 = __uint_as_float(r[2 * e + 1]) * inv;
+              const float s0 = __uint_as_float(os[e] << 16), s1 = __uint_as_float(os[e] & 0xFFFF0000u);
+              pk[e] = pack_bf16x2(fmaf(a0, s0 - l0, l0), fmaf(a1, s1 - l1, l1));
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(o + base + c0);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
+    };
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      const int s = i % lin::kLinStages;
+      if (!mbar_wait(&full[s], (i / lin::kLinStages) & 1, abort_flag)) { ok = false; break; }
+      // phi in place: elementwise, so the swizzled layout does not matter
+      uint4* qt = reinterpret_cast<uint4*>(smem + L::OFF_Q + s * L::Q_BYTES);
+#pragma unroll 4
+      for (int u = mt; u < static_cast<int>(L::Q_BYTES / 16); u += 128) {
+        uint4 w = qt[u];
+        uint32_t* x = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          x[e] = pack_bf16x2(lin::phi_f(__uint_as_float(x[e] << 16)), lin::phi_f(__uint_as_float(x[e] & 0xFFFF0000u)));
+        qt[u] = w;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&phi_done[s]);
+      if (i > 0) epilogue(i - 1);
+    }
+    if (ok && n_tiles > 0) epilogue(n_tiles - 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tm, L::TM_COLS);
   }
 }
 
-cudaError_t launch_linear_state(const LinearArgs& a, cudaStream_t st) {
+// ---------------------------------------------------------------- launchers
+template <int D>
+static cudaError_t state_d(const LinearArgs& a, cudaStream_t st) {
+  using L = lin::StateLayout<D>;
   const int BH = a.B * a.H;
-  const int ns = linear_splits(BH, a.N);
-  float* part = static_cast<float*>(a.ws);
-  dim3 g1(ns, BH);
-  const auto* k = static_cast<const uint16_t*>(a.k);
-  const auto* v = static_cast<const uint16_t*>(a.v);
-  if (a.d == 128) linear_state_kernel<128><<<g1, kLinThreads, 0, st>>>(k, v, a.N, ns, part);
-  else linear_state_kernel<64><<<g1, kLinThreads, 0, st>>>(k, v, a.N, ns, part);
-  cudaError_t e = cudaGetLastError();
+  const int ns = lin::splits(BH, a.N);
+  const int tps = lin::tiles_per_split(BH, a.N);
+  CUtensorMap mk, mv;
+  if (encode_tensor_map_3d_bf16(&mk, a.k, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (encode_tensor_map_3d_bf16(&mv, a.v, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(linear_state_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  const int n = a.d * a.d + a.d;
-  dim3 g2(ceil_div(n, 256), BH);
-  if (a.d == 128) linear_reduce_kernel<128><<<g2, 256, 0, st>>>(part, ns, a.kv_state, a.ksum);
-  else linear_reduce_kernel<64><<<g2, 256, 0, st>>>(part, ns, a.kv_state, a.ksum);
+  float* part = static_cast<float*>(a.ws);
+  linear_state_kernel<D><<<dim3(ns, BH), lin::kLinThreads, L::SMEM, st>>>(mk, mv, a.N, ns, tps, part);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int n = D * D + D;
+  linear_reduce_kernel<D><<<dim3(ceil_div(n, 256), BH), 256, 0, st>>>(part, ns, a.kv_state, a.ksum);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_linear_state(const LinearArgs& a, cudaStream_t st) {
+  return a.d == 128 ? state_d<128>(a, st) : state_d<64>(a, st);
+}
+
+template <int D>
+static cudaError_t out_d(const LinearArgs& a, cudaStream_t st) {
+  using L = lin::OutLayout<D>;
+  const int BH = a.B * a.H;
+  const int tiles = ceil_div(a.N, lin::kLinTok);
+  const int ctas_per_head = max(1, min(tiles, ceil_div(4 * 148, BH)));
+  const int tpc = ceil_div(tiles, ctas_per_head);
+  CUtensorMap mq;
+  if (encode_tensor_map_3d_bf16(&mq, a.q, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(linear_out_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+  if (e != cudaSuccess) return e;
+  linear_out_kernel<D><<<dim3(ceil_div(tiles, tpc), BH), lin::kLinThreads, L::SMEM, st>>>(
+      mq, a.kv_state, a.ksum, static_cast<const uint16_t*>(a.o_s), a.alpha, a.H, a.N, tpc,
+      static_cast<uint16_t*>(a.o));
   return cudaGetLastError();
 }
 
 cudaError_t launch_linear_out(const LinearArgs& a, cudaStream_t st) {
-  const int BH = a.B * a.H;
-  dim3 grid(ceil_div(a.N, kOutTok), BH);
-  const size_t smem = (static_cast<size_t>(a.d) * a.d + a.d + static_cast<size_t>(kOutTok) * (a.d + 1)) * sizeof(float);
-  const auto* q = static_cast<const uint16_t*>(a.q);
-  const auto* os = static_cast<const uint16_t*>(a.o_s);
-  auto* o = static_cast<uint16_t*>(a.o);
-  if (a.d == 128) {
-    cudaFuncSetAttribute(linear_out_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    linear_out_kernel<128><<<grid, kLinThreads, smem, st>>>(q, a.kv_state, a.ksum, os, a.alpha, a.H, a.N, o);
-  } else {
-    cudaFuncSetAttribute(linear_out_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    linear_out_kernel<64><<<grid, kLinThreads, smem, st>>>(q, a.kv_state, a.ksum, os, a.alpha, a.H, a.N, o);
-  }
-  return cudaGetLastError();
+  return a.d == 128 ? out_d<128>(a, st) : out_d<64>(a, st);
 }
 
 }  // namespace sa
