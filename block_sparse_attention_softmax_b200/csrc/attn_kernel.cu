@@ -3,35 +3,56 @@
 // skips the masked QK^T and softmax/PV work; Veda §2.3 describes a
 // producer/consumer split with TMA fetches of non-contiguous K/V tiles).
 //
-// One CTA computes one 128-row query tile of one head against the key blocks
-// its compacted list keeps. Two 64-key blocks form one 128-key tile.
+// Persistent kernel: one CTA per SM walks work items (head, 128-row query
+// tile) round-robin in head-major order, so concurrently running CTAs share
+// the K/V blocks of one head in L2. Inside an item, two 64-key blocks from the
+// item's kept list form one 128-key tile.
 //
-//   warp 0      TMA producer: Q once, then K and V of each kept tile into a
-//               2-stage ring (each 64-key block is its own TMA box, so the two
-//               blocks of a tile need not be adjacent in memory)
-//   warp 1      TMEM allocation and the single MMA-issuing thread:
-//                 S_j = Q K_j^T   (tcgen05.mma, A and B from shared memory,
-//                                  fp32 accumulator in one of 3 TMEM buffers)
-//                 O  += P_j V_j   (tcgen05.mma, A = P_j read from TMEM)
-//   warps 2..5  softmax: thread t owns TMEM lane t = query row t. Loads S_j,
-//               masks keys past N, keeps the running max m (log2 domain) and
-//               sum l, writes P_j = exp2(S_j*scale*log2e - m) as bf16 back into
-//               the S buffer, and rescales O in TMEM when m grows by more than
-//               2^8 (otherwise the stale max is kept: P stays <= 256).
-//               Finally O / l is written as bf16, with the row log-sum-exp.
+// Shared-memory bandwidth is the resource this kernel is shaped around: per
+// tile the TMA writes K and V (64 KB at d = 128) and the tensor core reads K and
+// V once each. Q and P never come from shared memory: Q is copied into TMEM
+// once per item and both products take their A operand from TMEM.
 //
-// TMEM columns: S buffers at 0, 128, 256 (fp32, 128 wide); O at 384 (d wide).
+//   warp 0       TMA producer of Q (one slot) and K (3-stage ring)
+//   warp 10      TMA producer of V (2-stage ring); one TMA box per 64-key
+//                block, so the two blocks of a tile need not be adjacent
+//   warp 1       TMEM allocation and the single MMA-issuing thread:
+//                  S_g = Q K_g^T  (A = Q from TMEM, B = K from shared memory)
+//                  O  += P_g V_g  (A = P_g from TMEM, B = V from shared memory)
+//                QK of tile g+1 is issued before PV of tile g, so the tensor
+//                core has work queued while the softmax of tile g runs. The
+//                QK that overwrites an S buffer is issued after the PV that
+//                reads the P stored there; one thread's tcgen05.mma operations
+//                execute in issue order.
+//   warps 2..9   softmax: TMEM lane quadrant q = warp % 4 holds query rows
+//                32q..32q+31; warp w and w+4 split the 128 columns of those
+//                rows (64 each) and exchange the row max through shared
+//                memory. The running max m is kept in the log2 domain and only
+//                raised when a tile's max exceeds it by more than 8 (P <= 256
+//                otherwise); then O is rescaled in TMEM. P = exp2(S*scale*log2e
+//                - m) is written back over S as packed bf16. The same warps
+//                copy each item's Q tile from shared memory into TMEM (after
+//                the last S of the previous item has landed), then copy O to
+//                registers, release it, and write O / l as bf16 and the row
+//                log-sum-exp.
+//
+// TMEM columns: Q at 0 (d/2 wide, bf16 pairs), S buffers at 128 and 256 (fp32,
+// 128 wide; P aliases their first 64 columns), O at 384 (d wide). Every
+// mbarrier wait is bounded (see sa_device.cuh).
 #include "sa_internal.h"
 
 namespace sa {
 
-namespace {
+namespace attn {
 
-constexpr int kBM = 128;    // query rows per tile
-constexpr int kBN = 128;    // keys per tile (two 64-key blocks)
-constexpr int kStages = 2;  // K/V ring depth
-constexpr int kSBufs = 3;   // S/P buffers in TMEM
-constexpr int kThreads = 192;
+constexpr int kBM = 128;        // query rows per tile
+constexpr int kBN = 128;        // keys per tile (two 64-key blocks)
+constexpr int kSoftWarps = 8;
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr int kSBufs = 2;
+constexpr int kVWarp = 2 + kSoftWarps;               // warp index of the V producer
+constexpr int kThreads = 32 * (kVWarp + 1);
 
 template <int D>
 struct Layout {
@@ -43,70 +64,108 @@ struct Layout {
   static constexpr uint32_t KV_CHUNK = kBN * 128;           // bytes per d-chunk of K/V
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
-  static constexpr uint32_t OFF_V = OFF_K + kStages * TILE_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_V + kStages * TILE_BYTES;
+  static constexpr uint32_t OFF_V = OFF_K + kKStages * TILE_BYTES;
+  static constexpr uint32_t OFF_RED = OFF_V + kVStages * TILE_BYTES;
+  static constexpr uint32_t RED_BYTES = (2 * 2 + 2) * kBM * 4;   // row max [2][2][128], row sum [2][128]
+  static constexpr uint32_t OFF_BAR = OFF_RED + RED_BYTES;
   static constexpr uint32_t USED = OFF_BAR + 256;
-  // Ask for enough shared memory that a second CTA never shares the SM (each
-  // CTA holds all 512 TMEM columns).
+  // at least 120 KB so that a second CTA never shares the SM (all 512 TMEM columns are held)
   static constexpr uint32_t SMEM = (USED + 1024 > 120 * 1024) ? USED + 1024 : 120 * 1024;
 };
 
-__host__ __device__ constexpr uint32_t tm_s(int b) { return static_cast<uint32_t>(b) * 128u; }
+constexpr uint32_t TM_Q = 0;
+__host__ __device__ constexpr uint32_t tm_s(int b) { return 128u + static_cast<uint32_t>(b) * 128u; }
 constexpr uint32_t TM_O = 384;
 constexpr uint32_t TM_COLS = 512;
 
-// barrier slots
 enum {
-  B_Q = 0,
-  B_KFULL = 1,
-  B_KEMPTY = B_KFULL + kStages,
-  B_VFULL = B_KEMPTY + kStages,
-  B_VEMPTY = B_VFULL + kStages,
-  B_SFULL = B_VEMPTY + kStages,
-  B_PFULL = B_SFULL + kSBufs,
-  B_OREADY = B_PFULL + kSBufs,
-  B_COUNT = B_OREADY + kSBufs
+  B_QFULL = 0,                       // Q tile landed in shared memory
+  B_QEMPTY = 1,                      // Q copied out of shared memory (8 warps)
+  B_QTMEM = 2,                       // Q present in TMEM (8 warps)
+  B_KFULL = 3,                       // [kKStages]
+  B_KEMPTY = B_KFULL + kKStages,     // [kKStages]
+  B_VFULL = B_KEMPTY + kKStages,     // [kVStages]
+  B_VEMPTY = B_VFULL + kVStages,     // [kVStages]
+  B_SFULL = B_VEMPTY + kVStages,     // [kSBufs]
+  B_PFULL = B_SFULL + kSBufs,        // [kSBufs]
+  B_PVDONE = B_PFULL + kSBufs,       // [kSBufs] P V of the tile held in that S buffer completed
+  B_OFULL = B_PVDONE + kSBufs,       // last P V of the item completed
+  B_OEMPTY = B_OFULL + 1,            // epilogue has copied O out of TMEM
+  B_COUNT = B_OEMPTY + 1
 };
 
-}  // namespace
+// Per-item facts every role derives the same way.
+struct Item {
+  int bh, qb, cnt, T;
+  bool tail;     // the last kept block is the ragged last key block
+};
+
+__device__ __forceinline__ Item load_item(const AttnArgs& a, int item) {
+  Item it;
+  it.bh = item / a.nqb;
+  it.qb = item % a.nqb;
+  const bool ragged = (a.N % 64) != 0;
+  if (a.dense) {
+    it.cnt = a.nkb;
+    it.tail = ragged;
+  } else {
+    const long long r = static_cast<long long>(it.bh) * a.nqb + it.qb;
+    it.cnt = __ldg(a.kv_cnt + r);
+    it.tail = ragged && it.cnt > 0 && __ldg(a.kv_idx + r * a.nkb + it.cnt - 1) == a.nkb - 1;
+  }
+  it.T = (it.cnt + 1) >> 1;
+  return it;
+}
+
+// First item at or after `item` (stepping by `stride`) with at least one tile.
+__device__ __forceinline__ int next_nonempty(const AttnArgs& a, int item, int stride, int n_items) {
+  for (; item < n_items; item += stride)
+    if (load_item(a, item).T > 0) break;
+  return item;
+}
+
+}  // namespace attn
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(attn::kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, AttnArgs a) {
+  using namespace attn;
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + L::OFF_Q;
   uint8_t* sK = smem + L::OFF_K;
   uint8_t* sV = smem + L::OFF_V;
+  float* red_max = reinterpret_cast<float*>(smem + L::OFF_RED);   // [2 tile parity][2 halves][128 rows]
+  float* red_sum = red_max + 4 * kBM;                              // [2 halves][128 rows]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qb = blockIdx.x;
-  const int bh = blockIdx.y;
-  const int q_row0 = qb * a.bq;
-
-  const int* kv_row = a.dense ? nullptr : a.kv_idx + (static_cast<long long>(bh) * a.nqb + qb) * a.nkb;
-  const int cnt = a.dense ? a.nkb : a.kv_cnt[static_cast<long long>(bh) * a.nqb + qb];
-  const int T = (cnt + 1) >> 1;
+  const int n_items = a.BH * a.nqb;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[B_Q], 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars[B_KFULL + s], 1);
-      mbar_init(&bars[B_KEMPTY + s], 1);
-      mbar_init(&bars[B_VFULL + s], 1);
-      mbar_init(&bars[B_VEMPTY + s], 1);
+    mbar_init(&bars[B_QFULL], 1);
+    mbar_init(&bars[B_QEMPTY], kSoftWarps);
+    mbar_init(&bars[B_QTMEM], kSoftWarps);
+    mbar_init(&bars[B_OFULL], 1);
+    mbar_init(&bars[B_OEMPTY], kSoftWarps);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&bars[B_KFULL + i], 1);
+      mbar_init(&bars[B_KEMPTY + i], 1);
     }
-    for (int b = 0; b < kSBufs; ++b) {
-      mbar_init(&bars[B_SFULL + b], 1);
-      mbar_init(&bars[B_PFULL + b], 4);
-      mbar_init(&bars[B_OREADY + b], 1);
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&bars[B_VFULL + i], 1);
+      mbar_init(&bars[B_VEMPTY + i], 1);
+    }
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(&bars[B_SFULL + i], 1);
+      mbar_init(&bars[B_PFULL + i], kSoftWarps);
+      mbar_init(&bars[B_PVDONE + i], 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -120,207 +179,344 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tm = *tmem_slot;
 
-  auto block_of = [&](int i) -> int { return a.dense ? i : __ldg(kv_row + i); };
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0 && T > 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&bars[B_Q], L::Q_BYTES);
+  if (warp == 0 || warp == kVWarp) {
+    // ------------------------------------------------------------ producers
+    if (lane == 0) {
+      const bool is_k = warp == 0;
+      if (is_k) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+      } else {
+        tma_prefetch_desc(&tmV);
+      }
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      uint8_t* ring = is_k ? sK : sV;
+      const int stages = is_k ? kKStages : kVStages;
+      const int b_full = is_k ? B_KFULL : B_VFULL;
+      const int b_empty = is_k ? B_KEMPTY : B_VEMPTY;
+      int g = 0, qi = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+        const Item it = load_item(a, item);
+        if (it.T == 0) continue;
+        const int* row = a.dense ? nullptr : a.kv_idx + (static_cast<long long>(it.bh) * a.nqb + it.qb) * a.nkb;
+        if (is_k) {
+          if (!(ok = mbar_wait(&bars[B_QEMPTY], (qi & 1) ^ 1, abort_flag))) break;
+          mbar_arrive_expect_tx(&bars[B_QFULL], L::Q_BYTES);
 #pragma unroll
-      for (int c = 0; c < L::NCH; ++c) tma_load_3d(sQ + c * L::Q_CHUNK, &tmQ, &bars[B_Q], c * 64, q_row0, bh);
-      for (int j = 0; j < T; ++j) {
-        const int s = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
-        const int nblk = min(2, cnt - 2 * j);
-        const int kb0 = block_of(2 * j);
-        const int kb1 = nblk > 1 ? block_of(2 * j + 1) : 0;
-        if (!mbar_wait(&bars[B_KEMPTY + s], ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&bars[B_KFULL + s], nblk * L::BLK_BYTES);
-        uint8_t* kdst = sK + s * L::TILE_BYTES;
-#pragma unroll
-        for (int c = 0; c < L::NCH; ++c) {
-          tma_load_3d(kdst + c * L::KV_CHUNK, &tmK, &bars[B_KFULL + s], c * 64, kb0 * 64, bh);
-          if (nblk > 1)
-            tma_load_3d(kdst + c * L::KV_CHUNK + 64 * 128, &tmK, &bars[B_KFULL + s], c * 64, kb1 * 64, bh);
+          for (int c = 0; c < L::NCH; ++c)
+            tma_load_3d(sQ + c * L::Q_CHUNK, &tmQ, &bars[B_QFULL], c * 64, it.qb * a.bq, it.bh);
         }
-        if (!mbar_wait(&bars[B_VEMPTY + s], ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&bars[B_VFULL + s], nblk * L::BLK_BYTES);
-        uint8_t* vdst = sV + s * L::TILE_BYTES;
+        for (int t = 0; t < it.T; ++t, ++g) {
+          const int s = g % stages;
+          const int nblk = min(2, it.cnt - 2 * t);
+          const int kb0 = a.dense ? 2 * t : __ldg(row + 2 * t);
+          const int kb1 = nblk > 1 ? (a.dense ? 2 * t + 1 : __ldg(row + 2 * t + 1)) : 0;
+          if (!(ok = mbar_wait(&bars[b_empty + s], ((g / stages) & 1) ^ 1, abort_flag))) break;
+          mbar_arrive_expect_tx(&bars[b_full + s], nblk * L::BLK_BYTES);
+          uint8_t* dst = ring + s * L::TILE_BYTES;
 #pragma unroll
-        for (int c = 0; c < L::NCH; ++c) {
-          tma_load_3d(vdst + c * L::KV_CHUNK, &tmV, &bars[B_VFULL + s], c * 64, kb0 * 64, bh);
-          if (nblk > 1)
-            tma_load_3d(vdst + c * L::KV_CHUNK + 64 * 128, &tmV, &bars[B_VFULL + s], c * 64, kb1 * 64, bh);
+          for (int c = 0; c < L::NCH; ++c) {
+            tma_load_3d(dst + c * L::KV_CHUNK, map, &bars[b_full + s], c * 64, kb0 * 64, it.bh);
+            if (nblk > 1)
+              tma_load_3d(dst + c * L::KV_CHUNK + 64 * 128, map, &bars[b_full + s], c * 64, kb1 * 64, it.bh);
+          }
         }
+        ++qi;
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && T > 0) {
-      const uint32_t q_base = smem_u32(sQ);
-      const uint32_t k_base = smem_u32(sK);
-      const uint32_t v_base = smem_u32(sV);
+    if (lane == 0) {
+      // The tensor pipe queues little, so this thread keeps the work between
+      // MMA groups minimal: ring slots and phases advance incrementally,
+      // descriptors are precomputed bases plus constant offsets, and the next
+      // item's facts are fetched one item ahead.
+      const uint64_t kdesc0 = sw128_desc(smem_u32(sK), 16, 1024);
+      const uint64_t vdesc0 = sw128_desc(smem_u32(sV), L::KV_CHUNK, 1024);
       const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
-      bool ok = mbar_wait(&bars[B_Q], 0, abort_flag);
-      auto issue_qk = [&](int j) -> bool {
-        const int s = j % kStages;
-        const int b = j % kSBufs;
-        const int nblk = min(2, cnt - 2 * j);
-        if (!mbar_wait(&bars[B_KFULL + s], (j / kStages) & 1, abort_flag)) return false;
-        if (j >= kSBufs && !mbar_wait(&bars[B_OREADY + b], ((j - kSBufs) / kSBufs) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t idesc = idesc_bf16_f32(kBM, nblk * 64, false, false);
-        const uint32_t kt = k_base + s * L::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32u;  // 16 bf16 = 32 B along K inside a 128-B row
-          const uint64_t adesc = sw128_desc(q_base + (kk >> 2) * L::Q_CHUNK + off, 16, 1024);
-          const uint64_t bdesc = sw128_desc(kt + (kk >> 2) * L::KV_CHUNK + off, 16, 1024);
-          umma_ss(tm + tm_s(b), adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+      const uint32_t idesc_qk2 = idesc_bf16_f32(kBM, 128, false, false);
+      const uint32_t idesc_qk1 = idesc_bf16_f32(kBM, 64, false, false);
+      const uint32_t q_tm = tm + TM_Q;
+      const uint32_t o_tm = tm + TM_O;
+      struct Ring {
+        int slot, n;
+        uint32_t phase;
+        __device__ void next() {
+          if (++slot == n) { slot = 0; phase ^= 1u; }
         }
-        tc_commit(&bars[B_SFULL + b]);
-        tc_commit(&bars[B_KEMPTY + s]);
+      };
+      // QK side
+      int qk_item = next_nonempty(a, blockIdx.x, gridDim.x, n_items);
+      Item qk_it = qk_item < n_items ? load_item(a, qk_item) : Item{};
+      int qk_t = 0;
+      uint32_t qk_qphase = 0;
+      Ring qk_k{0, kKStages, 0}, qk_s{0, kSBufs, 0};
+      // PV side
+      int pv_item = qk_item;
+      Item pv_it = qk_it;
+      int pv_t = 0;
+      uint32_t pv_ophase = 0;
+      Ring pv_v{0, kVStages, 0}, pv_s{0, kSBufs, 0};
+      // prefetched facts of the item after the QK cursor's current one
+      int nx_item = qk_item < n_items ? next_nonempty(a, qk_item + gridDim.x, gridDim.x, n_items) : n_items;
+      Item nx_it = nx_item < n_items ? load_item(a, nx_item) : Item{};
+      bool ok = true;
+
+      auto issue_qk = [&]() -> bool {
+        if (qk_t == 0) {
+          if (!mbar_wait(&bars[B_QTMEM], qk_qphase, abort_flag)) return false;
+          qk_qphase ^= 1u;
+        }
+        if (!mbar_wait(&bars[B_KFULL + qk_k.slot], qk_k.phase, abort_flag)) return false;
+        tc_fence_after();
+        const bool two = qk_it.cnt - 2 * qk_t >= 2;
+        const uint32_t idesc = two ? idesc_qk2 : idesc_qk1;
+        const uint64_t kd = kdesc0 + ((qk_k.slot * L::TILE_BYTES) >> 4);
+        const uint32_t s_tm = tm + tm_s(qk_s.slot);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ts(s_tm, q_tm + kk * 8, kd + ((((kk >> 2) * L::KV_CHUNK) + (kk & 3) * 32u) >> 4), idesc,
+                  kk > 0 ? 1u : 0u);
+        tc_commit(&bars[B_SFULL + qk_s.slot]);
+        tc_commit(&bars[B_KEMPTY + qk_k.slot]);
+        qk_k.next();
+        qk_s.next();
+        if (++qk_t == qk_it.T) {
+          qk_t = 0;
+          qk_item = nx_item;
+          qk_it = nx_it;
+          if (qk_item < n_items) {
+            nx_item = next_nonempty(a, qk_item + gridDim.x, gridDim.x, n_items);
+            if (nx_item < n_items) nx_it = load_item(a, nx_item);
+          }
+        }
         return true;
       };
-      if (ok) ok = issue_qk(0);
-      for (int j = 0; ok && j < T; ++j) {
-        if (j + 1 < T && !issue_qk(j + 1)) break;
-        const int s = j % kStages;
-        const int b = j % kSBufs;
-        const int nblk = min(2, cnt - 2 * j);
-        if (!mbar_wait(&bars[B_PFULL + b], (j / kSBufs) & 1, abort_flag)) break;
-        if (!mbar_wait(&bars[B_VFULL + s], (j / kStages) & 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t vt = v_base + s * L::TILE_BYTES;
-        for (int kk = 0; kk < nblk * 4; ++kk) {
-          const uint64_t bdesc = sw128_desc(vt + kk * 2048u, L::KV_CHUNK, 1024);
-          umma_ts(tm + TM_O, tm + tm_s(b) + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+      auto issue_pv = [&]() -> bool {
+        if (!mbar_wait(&bars[B_PFULL + pv_s.slot], pv_s.phase, abort_flag)) return false;
+        if (!mbar_wait(&bars[B_VFULL + pv_v.slot], pv_v.phase, abort_flag)) return false;
+        if (pv_t == 0) {
+          if (!mbar_wait(&bars[B_OEMPTY], pv_ophase ^ 1u, abort_flag)) return false;
+          pv_ophase ^= 1u;
         }
-        tc_commit(&bars[B_OREADY + b]);
-        tc_commit(&bars[B_VEMPTY + s]);
+        tc_fence_after();
+        const int nk = (pv_it.cnt - 2 * pv_t >= 2) ? 8 : 4;
+        const uint64_t vd = vdesc0 + ((pv_v.slot * L::TILE_BYTES) >> 4);
+        const uint32_t p_tm = tm + tm_s(pv_s.slot);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          if (kk < nk) umma_ts(o_tm, p_tm + kk * 8, vd + ((kk * 2048u) >> 4), idesc_pv, (pv_t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&bars[B_PVDONE + pv_s.slot]);
+        tc_commit(&bars[B_VEMPTY + pv_v.slot]);
+        pv_v.next();
+        pv_s.next();
+        if (++pv_t == pv_it.T) {
+          tc_commit(&bars[B_OFULL]);
+          pv_t = 0;
+          pv_item = next_nonempty(a, pv_item + gridDim.x, gridDim.x, n_items);
+          if (pv_item < n_items) pv_it = load_item(a, pv_item);
+        }
+        return true;
+      };
+      if (qk_item < n_items) ok = issue_qk();
+      while (ok && pv_item < n_items) {
+        if (qk_item < n_items && !(ok = issue_qk())) break;
+        if (!(ok = issue_pv())) break;
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax
-    const int quad = warp & 3;                       // TMEM lane quadrant of this warp
-    const int row = quad * 32 + lane;                // query row within the tile
+    // ------------------------------------------------------------ softmax + epilogue
+    const int sw = warp - 2;                  // 0..7
+    const int quad = warp & 3;                // TMEM lane quadrant
+    const int half = sw >> 2;                 // which 64 columns of the tile
+    const int row = quad * 32 + lane;         // query row within the tile
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    const int pair_bar = 1 + quad;            // named barrier of the two warps of this quadrant
     const float sl2 = a.scale_log2;
-    float m = -INFINITY;                             // running max, log2 domain
-    float l = 0.f;
+    const int tail_valid = a.N - (a.nkb - 1) * 64;
+    int g = 0, qi = 0;
     bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      const int b = j % kSBufs;
-      const int nblk = min(2, cnt - 2 * j);
-      const int kb0 = block_of(2 * j);
-      const int kb1 = nblk > 1 ? block_of(2 * j + 1) : 0;
-      const int valid0 = min(64, a.N - kb0 * 64);
-      const int valid1 = nblk > 1 ? min(64, a.N - kb1 * 64) : 0;
-      if (!mbar_wait(&bars[B_SFULL + b], (j / kSBufs) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t r0[32], r1[32], r2[32], r3[32];
-      const uint32_t sa = tm + lane_addr + tm_s(b);
-      tmem_ld32(sa + 0, r0);
-      tmem_ld32(sa + 32, r1);
-      tmem_ld32(sa + 64, r2);
-      tmem_ld32(sa + 96, r3);
-      tmem_wait_ld();
-      reg_fence(r0);
-      reg_fence(r1);
-      reg_fence(r2);
-      reg_fence(r3);
-      float x[128];
+
+    // Q tile of the qi-th non-empty item: shared memory -> TMEM (bf16 pairs,
+    // row = lane), this half's d range.
+    auto copy_q = [&](int q_index) -> bool {
+      if (!mbar_wait(&bars[B_QFULL], q_index & 1, abort_flag)) return false;
+      constexpr int U = D / 16;               // 16-B units per half row
+      uint32_t w[U * 4];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        x[c] = __uint_as_float(r0[c]);
-        x[32 + c] = __uint_as_float(r1[c]);
-        x[64 + c] = __uint_as_float(r2[c]);
-        x[96 + c] = __uint_as_float(r3[c]);
+      for (int j = 0; j < U; ++j) {
+        const int uu = half * U + j;          // unit index along d
+        const uint4 v = *reinterpret_cast<const uint4*>(
+            sQ + (uu >> 3) * L::Q_CHUNK + row * 128 + (((uu & 7) ^ (row & 7)) << 4));
+        w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
       }
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        if (c >= valid0) x[c] = -INFINITY;
-        if (c >= valid1) x[64 + c] = -INFINITY;
-      }
-      float mx = x[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
-      const float m_tile = mx * sl2;
-      float corr = 1.f;
-      if (m_tile > m + 8.f) {
-        corr = fast_exp2(m - m_tile);   // 0 on the first tile (m = -inf)
-        m = m_tile;
-        l *= corr;
-      }
-      float sum = 0.f;
-      uint32_t p0[32], p1[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float e0 = fast_exp2(fmaf(x[2 * c], sl2, -m));
-        const float e1 = fast_exp2(fmaf(x[2 * c + 1], sl2, -m));
-        const float e2 = fast_exp2(fmaf(x[64 + 2 * c], sl2, -m));
-        const float e3 = fast_exp2(fmaf(x[64 + 2 * c + 1], sl2, -m));
-        sum += (e0 + e1) + (e2 + e3);
-        p0[c] = pack_bf16x2(e0, e1);
-        p1[c] = pack_bf16x2(e2, e3);
-      }
-      l += sum;
-      tmem_st32(sa + 0, p0);
-      tmem_st32(sa + 32, p1);
-      if (j > 0) {
-        // O may only be touched once the previous P V product has landed.
-        const int pb = (j - 1) % kSBufs;
-        if (!mbar_wait(&bars[B_OREADY + pb], ((j - 1) / kSBufs) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xFFFFFFFFu, corr != 1.f)) {
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32_wait(tm + lane_addr + TM_O + c0, o);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
-            tmem_st32(tm + lane_addr + TM_O + c0, o);
-          }
-        }
-      }
+      tmem_st_cols<U * 4>(tm + lane_addr + TM_Q + half * (U * 4), w);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_PFULL + b]);
+      if (lane == 0) {
+        mbar_arrive(&bars[B_QEMPTY]);
+        mbar_arrive(&bars[B_QTMEM]);
+      }
+      return true;
+    };
+
+    int item = next_nonempty(a, blockIdx.x, gridDim.x, n_items);
+    if (item < n_items) ok = copy_q(0);
+    // items with no kept block before the first non-empty one
+    for (int z = blockIdx.x; z < item; z += gridDim.x) {
+      const Item it = load_item(a, z);
+      const int grow = it.qb * a.bq + row;
+      if (row < a.bq && grow < a.N) {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(it.bh) * a.N + grow) * D + half * (D / 2));
+        for (int c = 0; c < D / 16; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+        if (a.lse && half == 0) a.lse[static_cast<long long>(it.bh) * a.N + grow] = -INFINITY;
+      }
     }
-    // ------------------------------------------------------------ epilogue
-    const int grow = q_row0 + row;
-    const bool store = row < a.bq && grow < a.N;
-    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(bh) * a.N + grow) * D;
-    if (T > 0 && ok) {
-      const int lb = (T - 1) % kSBufs;
-      ok = mbar_wait(&bars[B_OREADY + lb], ((T - 1) / kSBufs) & 1, abort_flag);
-      tc_fence_after();
-    }
-    if (T > 0 && ok) {
-      const float inv_l = 1.f / l;
+    while (ok && item < n_items) {
+      const Item it = load_item(a, item);
+      const int grow = it.qb * a.bq + row;
+      const bool store = row < a.bq && grow < a.N;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(it.bh) * a.N + grow) * D + half * (D / 2);
+      float m = -INFINITY;     // running max (log2 domain), identical in both halves
+      float l = 0.f;           // this half's share of the row sum
+      for (int t = 0; t < it.T; ++t, ++g) {
+        const int b = g % kSBufs;
+        if (!(ok = mbar_wait(&bars[B_SFULL + b], (g / kSBufs) & 1, abort_flag))) break;
+        tc_fence_after();
+        uint32_t r0[32], r1[32];
+        const uint32_t sa = tm + lane_addr + tm_s(b) + half * 64;
+        tmem_ld32(sa, r0);
+        tmem_ld32(sa + 32, r1);
+        tmem_wait_ld();
+        reg_fence(r0);
+        reg_fence(r1);
+        float x[64];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          x[c] = __uint_as_float(r0[c]);
+          x[32 + c] = __uint_as_float(r1[c]);
+        }
+        if (t == it.T - 1) {
+          // last tile: possibly a single block, possibly the ragged last key block
+          const int nblk = it.cnt - 2 * t;
+          int valid = (half < nblk) ? 64 : 0;
+          if (it.tail && half == nblk - 1) valid = tail_valid;
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c >= valid) x[c] = -INFINITY;
+        }
+        float mx8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mx8[j] = x[j];
+#pragma unroll
+        for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
+        float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        float* rm = red_max + (g & 1) * 2 * kBM;
+        rm[half * kBM + row] = mx;
+        asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+        mx = fmaxf(mx, rm[(half ^ 1) * kBM + row]);
+        const float m_tile = mx * sl2;
+        float corr = 1.f;
+        if (m_tile > m + 8.f) {
+          corr = fast_exp2(m - m_tile);   // 0 on the first tile (m = -inf)
+          m = m_tile;
+          l *= corr;
+        }
+        // A quarter of the exponentials run on the FMA pipe so the MUFU unit
+        // is not the only path; partial sums in 4 chains.
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t p[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float a0 = fmaf(x[2 * c], sl2, -m);
+          const float a1 = fmaf(x[2 * c + 1], sl2, -m);
+          float e0, e1;
+          if ((c & 3) == 3) {
+            e0 = exp2_poly(a0);
+            e1 = exp2_poly(a1);
+          } else {
+            e0 = fast_exp2(a0);
+            e1 = fast_exp2(a1);
+          }
+          sum4[c & 3] += e0 + e1;
+          p[c] = pack_bf16x2(e0, e1);
+        }
+        l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        tmem_st32(tm + lane_addr + tm_s(b) + half * 32, p);
+        if (t > 0 && __any_sync(0xFFFFFFFFu, corr != 1.f)) {
+          // O is complete up to the previous tile once its P V has landed
+          const int pb = (g - 1) % kSBufs;
+          if (!(ok = mbar_wait(&bars[B_PVDONE + pb], ((g - 1) / kSBufs) & 1, abort_flag))) break;
+          tc_fence_after();
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        tmem_ld32_wait(tm + lane_addr + TM_O + c0, o);
-        if (store) {
-          uint32_t pk[16];
+          for (int c0 = 0; c0 < D / 2; c0 += 32) {
+            uint32_t o[32];
+            const uint32_t oa = tm + lane_addr + TM_O + half * (D / 2) + c0;
+            tmem_ld32_wait(oa, o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
+            tmem_st32(oa, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_PFULL + b]);
+      }
+      if (!ok) break;
+      // Every S of this item has landed, so no QK reads Q any more: bring in
+      // the next item's Q before finishing this one.
+      const int next = next_nonempty(a, item + gridDim.x, gridDim.x, n_items);
+      if (next < n_items && !(ok = copy_q(qi + 1))) break;
+      // ---------------------------------------------------------- epilogue
+      if (!(ok = mbar_wait(&bars[B_OFULL], qi & 1, abort_flag))) break;
+      tc_fence_after();
+      uint32_t o0[32], o1[32];
+      tmem_ld32(tm + lane_addr + TM_O + half * (D / 2), o0);
+      if (D == 128) tmem_ld32(tm + lane_addr + TM_O + half * (D / 2) + 32, o1);
+      tmem_wait_ld();
+      reg_fence(o0);
+      if (D == 128) reg_fence(o1);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_OEMPTY]);   // the next item may overwrite O now
+      red_sum[half * kBM + row] = l;
+      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+      const float lt = l + red_sum[(half ^ 1) * kBM + row];
+      const float inv_l = 1.f / lt;
+      if (store) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pk[c] = pack_bf16x2(__uint_as_float(o0[2 * c]) * inv_l, __uint_as_float(o0[2 * c + 1]) * inv_l);
+        uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        if (D == 128) {
 #pragma unroll
           for (int c = 0; c < 16; ++c)
-            pk[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+            pk[c] = pack_bf16x2(__uint_as_float(o1[2 * c]) * inv_l, __uint_as_float(o1[2 * c + 1]) * inv_l);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int c = 0; c < 4; ++c) dst[4 + c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         }
       }
-      if (store && a.lse) a.lse[static_cast<long long>(bh) * a.N + grow] = (m + log2f(l)) * 0.69314718055994531f;
-    } else if (store) {
-      uint4* dst = reinterpret_cast<uint4*>(orow);
-      for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-      if (a.lse) a.lse[static_cast<long long>(bh) * a.N + grow] = -INFINITY;
+      if (store && a.lse && half == 0)
+        a.lse[static_cast<long long>(it.bh) * a.N + grow] = (m + log2f(lt)) * 0.69314718055994531f;
+      // items with no kept block up to the next non-empty one
+      for (int z = item + gridDim.x; z < next; z += gridDim.x) {
+        const Item iz = load_item(a, z);
+        const int gz = iz.qb * a.bq + row;
+        if (row < a.bq && gz < a.N) {
+          uint4* dz = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(iz.bh) * a.N + gz) * D + half * (D / 2));
+          for (int c = 0; c < D / 16; ++c) dz[c] = make_uint4(0, 0, 0, 0);
+          if (a.lse && half == 0) a.lse[static_cast<long long>(iz.bh) * a.N + gz] = -INFINITY;
+        }
+      }
+      item = next;
+      ++qi;
     }
   }
 
@@ -334,20 +530,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D>
 static cudaError_t launch_d(const AttnArgs& a, cudaStream_t st) {
-  using L = Layout<D>;
+  using L = attn::Layout<D>;
   CUtensorMap mq, mk, mv;
-  if (encode_tensor_map_3d_bf16(&mq, a.q, D, a.N, a.BH, 64, kBM) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (encode_tensor_map_3d_bf16(&mq, a.q, D, a.N, a.BH, 64, attn::kBM) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   if (encode_tensor_map_3d_bf16(&mk, a.k, D, a.N, a.BH, 64, 64) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   if (encode_tensor_map_3d_bf16(&mv, a.v, D, a.N, a.BH, 64, 64) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.nqb, a.BH);
-  sparse_attn_kernel<D><<<grid, kThreads, L::SMEM, st>>>(mq, mk, mv, a);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long items = static_cast<long long>(a.BH) * a.nqb;
+  const int grid = static_cast<int>(items < sms ? items : sms);
+  sparse_attn_kernel<D><<<grid, attn::kThreads, L::SMEM, st>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t st) {
-  if (a.nqb > 0x7FFFFFFF || a.BH > 65535) return cudaErrorInvalidValue;
+  if (static_cast<long long>(a.BH) * a.nqb > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   return a.d == 128 ? launch_d<128>(a, st) : launch_d<64>(a, st);
 }
 

@@ -163,6 +163,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+        "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 // Makes later uses of r depend on a point after tcgen05.wait::ld, so the
 // compiler cannot move arithmetic on the loaded registers above the wait.
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
@@ -195,6 +205,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
         "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
+}
+
+// Store N (16 or 32) consecutive columns of this warp's 32 lanes.
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[N]) {
+  static_assert(N == 16 || N == 32, "16 or 32 columns");
+  if constexpr (N == 32) tmem_st32(taddr, r);
+  else tmem_st16(taddr, r);
 }
 
 // ---------------------------------------------------------------- descriptors
@@ -231,6 +249,19 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// 2^x on the FMA pipe, for x <= 127: x = i + f with i = floor(x), f in [0, 1);
+// 2^f by a cubic fitted on [0, 1) for minimum maximum relative error (Lawson's
+// iteratively reweighted least squares; max relative error 7.7e-5), and 2^i
+// added to the exponent field. Inputs below -126 return a value below 2^-125
+// (or 0), which is negligible wherever it is used.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float xi = floorf(x);
+  const float f = x - xi;
+  const float p = fmaf(fmaf(fmaf(0.07809657f, f, 0.22596510f), f, 0.69586831f), f, 0.99992359f);
+  return __int_as_float(__float_as_int(p) + (static_cast<int>(xi) << 23));
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
