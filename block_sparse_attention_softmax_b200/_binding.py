@@ -25,6 +25,9 @@ _SIGNATURES = {
     "sa_build_mask": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                               c_double, c_double, c_double, c_void_p, c_void_p, c_void_p,
                               c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "sa_build_mask_noalloc": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                      c_double, c_double, c_double, c_void_p, c_void_p, c_void_p,
+                                      c_void_p]),
     "sa_sparse_attn_workspace_size": (c_size_t, [c_int] * 7),
     "sa_sparse_attn_fwd": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
                                    c_int, c_int, c_void_p, c_void_p, c_void_p, c_double,

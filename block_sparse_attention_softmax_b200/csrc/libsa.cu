@@ -5,3 +5,4 @@
 #include "attn_kernel.cu"
 #include "linear_kernels.cu"
 #include "sa_api.cu"
+#include "noalloc.cu"

@@ -1,0 +1,91 @@
+// noalloc.cu — sa_build_mask_noalloc: the hybrid Top-k ∪ Top-p mask builder
+// with its scratch (pooled means and block scores) in a fixed device array
+// that is part of the library image, for callers that may not allocate device
+// memory at call time.
+//
+// The array is created when the library's device code is loaded on a GPU and
+// stays allocated on every GPU that loads the library until the process exits.
+// Host code cannot use the array's name as a device address, so the first call
+// on each device looks the address up with cudaGetSymbolAddress (with that
+// device current) and caches it; later calls on that device reuse it.
+//
+// Included from libsa.cu after sa_api.cu (same translation unit), so it reuses
+// that file's argument checks and error reporting.
+#include <mutex>
+
+namespace sa {
+
+// Fixed scratch size. Enough for, e.g., B*H = 12 heads at N = 32760 tokens,
+// d = 128 (about 11 MB of pooled means and scores).
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device (looked up once).
+int static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "sa_build_mask_noalloc (cudaGetDevice)");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SA_ERR_UNSUPPORTED, "device ordinal %d exceeds %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "sa_build_mask_noalloc (cudaGetSymbolAddress)");
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return SA_OK;
+}
+
+}  // namespace
+}  // namespace sa
+
+extern "C" {
+
+int sa_build_mask_noalloc(const uint16_t* q, const uint16_t* k, int B, int H, int N, int d, int bq,
+                          int bk, double topk_frac, double topp, double scale, int32_t* kv_idx,
+                          int32_t* kv_cnt, uint8_t* mask_opt, void* stream) {
+  using namespace sa;
+  int rc = check_shape(B, H, N, d, bq, bk);
+  if (rc) return rc;
+  if (!q || !k || !kv_idx || !kv_cnt) return fail(SA_ERR_INVALID_ARG, "sa_build_mask_noalloc: null pointer");
+  if (!(topk_frac > 0.0 && topk_frac <= 1.0)) return fail(SA_ERR_INVALID_ARG, "topk_frac %g outside (0, 1]", topk_frac);
+  if (!(topp >= 0.0 && topp <= 1.0)) return fail(SA_ERR_INVALID_ARG, "topp %g outside [0, 1]", topp);
+  if (!isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "scale must be finite");
+  const int nkb = (N + bk - 1) / bk, nqb = (N + bq - 1) / bq;
+  if (nkb > kMaxKeyBlocks) return fail(SA_ERR_UNSUPPORTED, "n_kb = %d exceeds %d", nkb, kMaxKeyBlocks);
+  const void* ptrs[] = {q, k, kv_idx, kv_cnt, mask_opt};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "sa_build_mask_noalloc: pointers must be 16-byte aligned");
+  // Same scratch layout as sa_build_mask with internal pooled means.
+  const MaskWs w = mask_ws(B, H, N, d, bq, bk, true, true);
+  if (w.total > kStaticScratchBytes)
+    return fail(SA_ERR_UNSUPPORTED,
+                "sa_build_mask_noalloc: this problem needs %zu bytes of scratch; the fixed scratch holds %zu "
+                "(use sa_build_mask with a caller workspace)", w.total, kStaticScratchBytes);
+  void* scratch = nullptr;
+  rc = static_scratch(&scratch);
+  if (rc) return rc;
+  if (scale <= 0.0) scale = 1.0 / sqrt(static_cast<double>(d));
+  // Nothing here must start at zero: every scratch byte that is read was
+  // written earlier in this call.
+  char* ws = static_cast<char*>(scratch);
+  float* qp = reinterpret_cast<float*>(ws + w.q_pool);
+  float* kp = reinterpret_cast<float*>(ws + w.k_pool);
+  float* s = reinterpret_cast<float*>(ws + w.s);
+  const int BH = B * H;
+  const int k_sel = static_cast<int>(fmin(static_cast<double>(nkb), fmax(1.0, ceil(topk_frac * nkb - 1e-9))));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_pool(q, k, BH, N, d, bq, bk, qp, kp, st);
+  if (e == cudaSuccess) e = launch_scores(qp, kp, BH, nqb, nkb, d, scale, s, w.s_ld, st);
+  if (e == cudaSuccess) e = launch_select(s, w.s_ld, BH * nqb, nkb, k_sel, topp, kv_idx, kv_cnt, mask_opt, st);
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_build_mask_noalloc");
+}
+
+}  // extern "C"

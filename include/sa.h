@@ -135,6 +135,31 @@ int sa_blend(const uint16_t* o_s, const uint16_t* q, const float* kv_state, cons
              const float* alpha, int B, int H, int N, int d, uint16_t* o,
              void* workspace, size_t ws_bytes, void* stream);
 
+/* Mask builder that allocates nothing (no counterpart in the pages: it exists
+ * for callers, not for the method). Some callers may not allocate device memory
+ * when they call in: an inference engine's per-request callback that must not
+ * allocate, or a service that plans its whole device memory budget at start-up
+ * and cannot let a call grow it or synchronise the device to allocate. This
+ * entry point computes exactly what sa_build_mask computes (same kernels, same
+ * results) but keeps its scratch (pooled means and block scores) in a fixed
+ * 16 MiB device array that is part of the library: every GPU that loads the
+ * library holds those 16 MiB until the process exits. The caller still passes
+ * the inputs and the outputs.
+ *   - Problems whose scratch, as counted by sa_build_mask_workspace_size(), is
+ *     above 16 MiB (16777216 bytes) are rejected with SA_ERR_UNSUPPORTED before
+ *     anything is launched; about 12 heads of 32760 tokens at d = 128 fit.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Calls whose work overlaps on the GPU (for example on two streams without
+ *     ordering between them) race on it; order them on one stream or with
+ *     events. Nothing in the array needs to start at zero.
+ *   - It calls no cudaMalloc, cudaFree or allocating library routine. */
+int sa_build_mask_noalloc(const uint16_t* q, const uint16_t* k, int B, int H, int N, int d,
+                          int bq, int bk, double topk_frac, double topp, double scale,
+                          int32_t* kv_idx, int32_t* kv_cnt, uint8_t* mask_opt, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
