@@ -5,11 +5,11 @@
 // Three kernels, all bound by memory or by a small amount of ALU work:
 //   pool_kernel    Q, K [BH, N, d] bf16  ->  block means [BH, nb, d] fp32
 //   score_kernel   means -> s[bh, qb, kb] = scale * <Qbar, Kbar> (fp32 partial
-//                  sums of 16 products, combined in fp64, rounded once)
-//   select_kernel  one query-block row per CTA: radix select of the K_sel-th
-//                  largest score (Top-k), a probability-weighted radix select
-//                  for the Top-p cut when Top-k alone does not reach p, and
-//                  the ascending compacted index list.
+//                  sums of 32 products, combined in fp64, rounded once)
+//   select_kernel  one query-block row per warp: radix select of the K_sel-th
+//                  largest score (Top-k), a probability-mass search for the
+//                  Top-p cut when Top-k alone does not reach p, and the
+//                  ascending compacted index list.
 #include "sa_internal.h"
 
 namespace sa {
@@ -87,8 +87,8 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 
 // ---------------------------------------------------------------- scores
 // 64 x 64 tile of one head per CTA; thread (ty, tx) owns a 4 x 4 sub-tile.
-// Products are summed in fp32 over 16 consecutive channels, the 16-channel
-// partial sums in fp64, so the rounding error stays near 1e-8 of the score
+// Products are summed in fp32 over 32 consecutive channels, the 32-channel
+// partial sums in fp64, so the rounding error stays near 1e-7 of the score
 // scale rather than the ~1e-6 of a 128-term fp32 sum.
 constexpr int kScoreTile = 64;
 constexpr int kScorePad = kScoreTile + 4;
@@ -128,14 +128,14 @@ __global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ q_
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc64[i][j] = 0.0;
-  for (int c0 = 0; c0 < D; c0 += 16) {
+  for (int c0 = 0; c0 < D; c0 += 32) {
     float acc[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 #pragma unroll
-    for (int c = c0; c < c0 + 16; ++c) {
+    for (int c = c0; c < c0 + 32; ++c) {
       const float4 a = *reinterpret_cast<const float4*>(qs + c * kScorePad + ty * 4);
       const float4 b = *reinterpret_cast<const float4*>(ks + c * kScorePad + tx * 4);
       const float av[4] = {a.x, a.y, a.z, a.w};
@@ -164,348 +164,245 @@ __global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ q_
 }
 
 // ---------------------------------------------------------------- selection
-constexpr int kSelThreads = 256;
-constexpr int kSelWarps = kSelThreads / 32;
+// One warp per query-block row; rows of the grid are strided over the warps.
+// Each warp keeps its row's keys and exponentials in its own slice of shared
+// memory, so no block-wide barrier is ever needed.
+//
+//   keys    monotone uint32 image of the fp32 scores (larger score -> larger key)
+//   e       exp(s - max) in fp32; Z and every probability mass in fp64
+//   Top-k   4-pass radix select (8-bit digits, warp histogram with aggregated
+//           atomics) of the K_sel-th largest key; ties at the cut are kept in
+//           ascending block order (ballot prefix counts)
+//   Top-p   only when the Top-k set holds less than p of the mass: bitwise
+//           search for the largest key v with mass(key >= v) >= p * Z, then the
+//           ties at v in block order until the mass is reached
+//   output  the union is the longer of the two prefixes of the common order;
+//           kept indices are written in ascending order (ballot compaction)
+constexpr int kSelWarpsMax = 8;
 
-// Monotone map of an fp32 score to uint32: larger score -> larger key.
 __device__ __forceinline__ uint32_t score_key(float s) {
   const uint32_t u = __float_as_uint(s);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-struct SelShared {
-  uint32_t hist_c[256];
-  double hist_w[256];
-  double red_d[kSelWarps];
-  float red_f[kSelWarps];
-  int red_i[kSelWarps];
-  int scan[kSelThreads];
-  // results broadcast from warp 0
-  uint32_t digit;
-  uint32_t cnt_above;
-  double w_above;
-  int exhausted;
-};
-
-__device__ __forceinline__ float block_max_f(float v, SelShared& sh) {
+__device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  if ((threadIdx.x & 31) == 0) sh.red_f[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float r = sh.red_f[0];
-#pragma unroll
-  for (int i = 1; i < kSelWarps; ++i) r = fmaxf(r, sh.red_f[i]);
-  __syncthreads();
-  return r;
+  return v;
 }
-
-__device__ __forceinline__ double block_sum_d(double v, SelShared& sh) {
+__device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-  if ((threadIdx.x & 31) == 0) sh.red_d[threadIdx.x >> 5] = v;
-  __syncthreads();
-  double r = 0.0;
-#pragma unroll
-  for (int i = 0; i < kSelWarps; ++i) r += sh.red_d[i];
-  __syncthreads();
-  return r;
+  return v;
 }
-
-// Exclusive prefix sum of one int per thread, in thread order; returns the
-// block total through *total.
-__device__ __forceinline__ int block_exclusive_scan(int v, SelShared& sh, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
+__device__ __forceinline__ int warp_sum_i(int v) {
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) sh.red_i[warp] = x;
-  __syncthreads();
-  int before = 0, all = 0;
-#pragma unroll
-  for (int i = 0; i < kSelWarps; ++i) {
-    if (i < warp) before += sh.red_i[i];
-    all += sh.red_i[i];
-  }
-  __syncthreads();
-  *total = all;
-  return before + x - v;
-}
-
-// One radix step over the elements whose key matches (prefix, pmask): builds
-// the 256-bin histogram of the next digit (counts, and weights if weighted)
-// and picks the digit holding the target. Unweighted: the bin holding the
-// `need`-th largest element. Weighted: the first bin, from the top, at which
-// w_above + (weight of bins >= it) reaches `target`.
-template <bool WEIGHTED>
-__device__ void radix_step(const uint32_t* keys, const float* e, int n, uint32_t prefix,
-                           uint32_t pmask, int shift, uint32_t need, double w_above,
-                           double target, SelShared& sh) {
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) {
-    sh.hist_c[i] = 0;
-    if (WEIGHTED) sh.hist_w[i] = 0.0;
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const uint32_t key = keys[i];
-    if ((key & pmask) == prefix) {
-      const uint32_t dg = (key >> shift) & 255u;
-      atomicAdd(&sh.hist_c[dg], 1u);
-      if (WEIGHTED) atomicAdd(&sh.hist_w[dg], static_cast<double>(e[i]));
-    }
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    // lane owns bins [8*lane, 8*lane + 8); suffix sums run from bin 255 down.
-    uint32_t c[8];
-    double w[8];
-    uint32_t lc = 0;
-    double lw = 0.0;
-#pragma unroll
-    for (int j = 7; j >= 0; --j) {
-      lc += sh.hist_c[8 * lane + j];
-      c[j] = lc;
-      if (WEIGHTED) {
-        lw += sh.hist_w[8 * lane + j];
-        w[j] = lw;
-      }
-    }
-    // inclusive suffix over lanes: add totals of higher lanes
-    uint32_t hc = lc;
-    double hw = lw;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t yc = __shfl_down_sync(0xFFFFFFFFu, hc, o);
-      double yw = 0.0;
-      if (WEIGHTED) yw = __shfl_down_sync(0xFFFFFFFFu, hw, o);
-      if (lane + o < 32) {
-        hc += yc;
-        if (WEIGHTED) hw += yw;
-      }
-    }
-    const uint32_t above_c = hc - lc;   // bins of higher lanes
-    const double above_w = WEIGHTED ? hw - lw : 0.0;
-    // largest bin j (in this lane) whose suffix reaches the target
-    int hit = -1;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      bool ok;
-      if (WEIGHTED) ok = (w_above + above_w + w[j] >= target) && (c[j] + above_c > 0);
-      else ok = (c[j] + above_c >= need);
-      if (ok) hit = j;
-    }
-    const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, hit >= 0);
-    if (ballot) {
-      const int src = 31 - __clz(ballot);
-      if (lane == src) {
-        const int dg = 8 * lane + hit;
-        // totals strictly above the chosen bin
-        const uint32_t cnt_above = above_c + (hit < 7 ? c[hit + 1] : 0u);
-        const double wt_above = WEIGHTED ? above_w + (hit < 7 ? w[hit + 1] : 0.0) : 0.0;
-        sh.digit = static_cast<uint32_t>(dg);
-        sh.cnt_above = cnt_above;
-        sh.w_above = wt_above;
-        sh.exhausted = 0;
-      }
-    } else {
-      // Weighted only: rounding kept the bucket below the target; every element
-      // of the bucket is needed, so continue into its lowest non-empty bin.
-      const uint32_t nz = __ballot_sync(0xFFFFFFFFu, lc > 0);
-      const int src = __ffs(nz) - 1;
-      if (lane == src) {
-        int j0 = 0;
-        while (j0 < 7 && sh.hist_c[8 * lane + j0] == 0) ++j0;
-        sh.digit = static_cast<uint32_t>(8 * lane + j0);
-        sh.cnt_above = above_c + (j0 < 7 ? c[j0 + 1] : 0u);
-        sh.w_above = above_w + (j0 < 7 ? w[j0 + 1] : 0.0);
-        sh.exhausted = 1;
-      }
-    }
-  }
-  __syncthreads();
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
 }
 
 struct Cut {
   uint32_t key;    // threshold key value
-  uint32_t above;  // elements strictly above the threshold
-  uint32_t ties;   // elements equal to the threshold to keep, lowest index first
+  int above;       // elements strictly above the threshold
+  int ties;        // elements equal to the threshold that are kept, lowest index first
 };
 
-// The `rank`-th largest key (1-based) and the number of its ties to keep.
-__device__ Cut select_rank(const uint32_t* keys, int n, uint32_t rank, SelShared& sh) {
-  uint32_t prefix = 0, pmask = 0, need = rank, above = 0;
+// The `rank`-th largest key (1-based) of keys[0..n) and how many of its ties to keep.
+__device__ Cut warp_select_rank(const uint32_t* keys, int n, int rank, uint32_t* hist) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0, pmask = 0;
+  int need = rank, above = 0;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    radix_step<false>(keys, nullptr, n, prefix, pmask, shift, need, 0.0, 0.0, sh);
-    const uint32_t dg = sh.digit, ca = sh.cnt_above;
-    need -= ca;
-    above += ca;
-    prefix |= dg << shift;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
+    __syncwarp();
+    for (int base = 0; base < n; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = i < n ? keys[i] : 0u;
+      const bool in = i < n && (key & pmask) == prefix;
+      const uint32_t act = __ballot_sync(0xFFFFFFFFu, in);
+      if (in) {
+        const uint32_t dg = (key >> shift) & 255u;
+        const uint32_t same = __match_any_sync(act, dg);
+        if (lane == __ffs(same) - 1) atomicAdd(&hist[dg], static_cast<uint32_t>(__popc(same)));
+      }
+    }
+    __syncwarp();
+    // lane owns bins [8 lane, 8 lane + 8); suffix counts run from bin 255 down
+    uint32_t c[8];
+    uint32_t run = 0;
+#pragma unroll
+    for (int j = 7; j >= 0; --j) {
+      run += hist[lane * 8 + j];
+      c[j] = run;
+    }
+    uint32_t incl = run;  // inclusive suffix over lanes >= lane
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, incl, o);
+      if (lane + o < 32) incl += y;
+    }
+    const uint32_t higher = incl - run;   // elements in bins of higher lanes
+    int hit = -1;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (static_cast<int>(higher + c[j]) >= need) hit = j;
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, hit >= 0);
+    const int src = 31 - __clz(bal);
+    const int hit_s = __shfl_sync(0xFFFFFFFFu, hit, src);
+    uint32_t above_bin = 0;
+    if (lane == src) above_bin = higher + (hit < 7 ? c[hit + 1] : 0u);
+    above_bin = __shfl_sync(0xFFFFFFFFu, above_bin, src);
+    need -= static_cast<int>(above_bin);
+    above += static_cast<int>(above_bin);
+    prefix |= static_cast<uint32_t>(src * 8 + hit_s) << shift;
     pmask |= 255u << shift;
-    __syncthreads();
+    __syncwarp();
   }
   return Cut{prefix, above, need};
 }
 
+// Mass (fp64) of the elements whose key is >= v.
+__device__ __forceinline__ double warp_mass_ge(const uint32_t* keys, const float* e, int n, uint32_t v) {
+  const int lane = threadIdx.x & 31;
+  double w = 0.0;
+  for (int i = lane; i < n; i += 32)
+    if (keys[i] >= v) w += static_cast<double>(e[i]);
+  return warp_sum_d(w);
+}
+
 // Smallest m such that the m largest-key weights sum to >= target.
-__device__ Cut select_mass(const uint32_t* keys, const float* e, int n, double target,
-                           SelShared& sh) {
-  uint32_t prefix = 0, pmask = 0, above = 0;
-  double w_above = 0.0;
-  int exhausted = 0;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    radix_step<true>(keys, e, n, prefix, pmask, shift, 0, w_above, target, sh);
-    const uint32_t dg = sh.digit;
-    above += sh.cnt_above;
-    w_above += sh.w_above;
-    exhausted |= sh.exhausted;
-    prefix |= dg << shift;
-    pmask |= 255u << shift;
-    __syncthreads();
+__device__ Cut warp_select_mass(const uint32_t* keys, const float* e, int n, double target) {
+  const int lane = threadIdx.x & 31;
+  uint32_t v = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = v | (1u << bit);
+    if (warp_mass_ge(keys, e, n, cand) >= target) v = cand;
   }
-  // Ties at the threshold: identical keys carry identical weights; take them in
-  // index order until the running sum reaches the target.
-  int n_ties = 0;
+  // strictly above v, and the ties at v
+  int above = 0, nties = 0;
+  double w_above = 0.0;
   float e_tie = 0.f;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    if (keys[i] == prefix) {
-      ++n_ties;
+  for (int i = lane; i < n; i += 32) {
+    const uint32_t key = keys[i];
+    if (key > v) {
+      ++above;
+      w_above += static_cast<double>(e[i]);
+    } else if (key == v) {
+      ++nties;
       e_tie = e[i];
     }
   }
-  int total;
-  block_exclusive_scan(n_ties, sh, &total);
-  const float ev = block_max_f(e_tie, sh);  // all ties share one weight
-  uint32_t t = 0;
-  if (exhausted) {
-    t = static_cast<uint32_t>(total);
-  } else {
-    double acc = w_above;
-    while (acc < target && t < static_cast<uint32_t>(total)) {
-      acc += static_cast<double>(ev);
-      ++t;
-    }
-    if (t == 0) t = 1;
+  above = warp_sum_i(above);
+  nties = warp_sum_i(nties);
+  w_above = warp_sum_d(w_above);
+  e_tie = warp_max(e_tie);            // every tie has the same weight
+  int t = 0;
+  double acc = w_above;
+  while (acc < target && t < nties) {
+    acc += static_cast<double>(e_tie);
+    ++t;
   }
-  __syncthreads();
-  return Cut{prefix, above, t};
+  if (acc < target) t = nties;        // rounding kept the total below the target
+  if (above + t == 0) t = 1;
+  return Cut{v, above, t};
 }
 
-// Per-thread contiguous chunk [lo, hi) of the row, used where index order matters.
-__device__ __forceinline__ void chunk_range(int n, int* lo, int* hi) {
-  const int per = (n + blockDim.x - 1) / blockDim.x;
-  *lo = min(n, static_cast<int>(threadIdx.x) * per);
-  *hi = min(n, *lo + per);
-}
-
-// Marks kept elements (key > cut, or equal and among the first `ties` equal
-// ones by index) in `flag`, and returns this thread's fp64 weight of them.
-__device__ double mark_kept(const uint32_t* keys, const float* e, int n, Cut cut, uint8_t* flag,
-                            SelShared& sh) {
-  int lo, hi;
-  chunk_range(n, &lo, &hi);
-  int my_ties = 0;
-  for (int i = lo; i < hi; ++i) my_ties += (keys[i] == cut.key);
-  int total;
-  int rank = block_exclusive_scan(my_ties, sh, &total);
-  double w = 0.0;
-  for (int i = lo; i < hi; ++i) {
-    const uint32_t key = keys[i];
-    bool keep = key > cut.key;
-    if (key == cut.key) {
-      keep = static_cast<uint32_t>(rank) < cut.ties;
-      ++rank;
-    }
-    flag[i] = keep;
-    if (keep && e) w += static_cast<double>(e[i]);
-  }
-  return w;
-}
-
-// One CTA per (bh, qb) row.
-__global__ void __launch_bounds__(kSelThreads) select_kernel(
+__global__ void __launch_bounds__(kSelWarpsMax * 32) select_kernel(
     const float* __restrict__ s, long long s_ld, int n_rows, int nkb, int k_sel, double topp,
     int* __restrict__ kv_idx, int* __restrict__ kv_cnt, uint8_t* __restrict__ mask) {
   extern __shared__ __align__(16) uint8_t sm_sel[];
-  __shared__ SelShared sh;
-  const int row = blockIdx.x;
-  if (row >= n_rows) return;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(sm_sel);
-  float* e = reinterpret_cast<float*>(sm_sel + static_cast<size_t>(nkb) * 4);
-  uint8_t* flag = sm_sel + static_cast<size_t>(nkb) * 8;
-  const float* srow = s + static_cast<long long>(row) * s_ld;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wpc = blockDim.x >> 5;
+  const size_t slice = static_cast<size_t>(nkb) * 8 + 256 * 4;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sm_sel + warp * slice);
+  float* e = reinterpret_cast<float*>(keys + nkb);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(e + nkb);
+  const uint32_t lt = (1u << lane) - 1u;
 
-  float mx = -INFINITY;
-  for (int i = threadIdx.x; i < nkb; i += blockDim.x) {
-    const float v = srow[i];
-    keys[i] = score_key(v);
-    e[i] = v;
-    mx = fmaxf(mx, v);
-  }
-  mx = block_max_f(mx, sh);  // contains __syncthreads
-  double z = 0.0;
-  for (int i = threadIdx.x; i < nkb; i += blockDim.x) {
-    const float v = expf(e[i] - mx);
-    e[i] = v;
-    z += static_cast<double>(v);
-  }
-  z = block_sum_d(z, sh);
+  for (int row = blockIdx.x * wpc + warp; row < n_rows; row += gridDim.x * wpc) {
+    const float* srow = s + static_cast<long long>(row) * s_ld;
+    float mx = -INFINITY;
+    for (int i = lane; i < nkb; i += 32) {
+      const float v = __ldg(srow + i);
+      keys[i] = score_key(v);
+      e[i] = v;
+      mx = fmaxf(mx, v);
+    }
+    mx = warp_max(mx);
+    double z = 0.0;
+    for (int i = lane; i < nkb; i += 32) {
+      const float v = expf(e[i] - mx);
+      e[i] = v;
+      z += static_cast<double>(v);
+    }
+    z = warp_sum_d(z);
+    __syncwarp();
 
-  if (topp >= 1.0 || k_sel >= nkb) {
-    for (int i = threadIdx.x; i < nkb; i += blockDim.x) flag[i] = 1;
-    __syncthreads();
-  } else {
-    const double target = topp * z;
-    const Cut ck = select_rank(keys, nkb, static_cast<uint32_t>(k_sel), sh);
-    double wk = mark_kept(keys, e, nkb, ck, flag, sh);
-    wk = block_sum_d(wk, sh);
-    if (wk < target) {
-      const Cut cp = select_mass(keys, e, nkb, target, sh);
-      const int m_p = static_cast<int>(cp.above + cp.ties);
-      if (m_p > k_sel) {
-        mark_kept(keys, nullptr, nkb, cp, flag, sh);
+    Cut cut{0u, 0, nkb};              // keep everything
+    if (!(topp >= 1.0 || k_sel >= nkb)) {
+      cut = warp_select_rank(keys, nkb, k_sel, hist);
+      const double target = topp * z;
+      // mass of the Top-k set (ties at the cut taken in block order)
+      double wk = 0.0;
+      int tie_before = 0;
+      for (int base = 0; base < nkb; base += 32) {
+        const int i = base + lane;
+        const uint32_t key = i < nkb ? keys[i] : 0u;
+        const bool tie = i < nkb && key == cut.key;
+        const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
+        const bool keep = i < nkb && (key > cut.key || (tie && tie_before + __popc(tb & lt) < cut.ties));
+        if (keep) wk += static_cast<double>(e[i]);
+        tie_before += __popc(tb);
+      }
+      wk = warp_sum_d(wk);
+      if (wk < target) {
+        const Cut cp = warp_select_mass(keys, e, nkb, target);
+        if (cp.above + cp.ties > k_sel) cut = cp;
       }
     }
-    __syncthreads();
-  }
 
-  // Ascending compaction of the kept indices.
-  int lo, hi;
-  chunk_range(nkb, &lo, &hi);
-  int mine = 0;
-  for (int i = lo; i < hi; ++i) mine += flag[i];
-  int total;
-  int pos = block_exclusive_scan(mine, sh, &total);
-  int* out = kv_idx + static_cast<long long>(row) * nkb;
-  for (int i = lo; i < hi; ++i)
-    if (flag[i]) out[pos++] = i;
-  if (mask) {
-    uint8_t* mrow = mask + static_cast<long long>(row) * nkb;
-    for (int i = threadIdx.x; i < nkb; i += blockDim.x) mrow[i] = flag[i];
+    // ascending compaction of the kept indices
+    int* out = kv_idx + static_cast<long long>(row) * nkb;
+    uint8_t* mrow = mask ? mask + static_cast<long long>(row) * nkb : nullptr;
+    int written = 0, tie_before = 0;
+    for (int base = 0; base < nkb; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = i < nkb ? keys[i] : 0u;
+      const bool tie = i < nkb && key == cut.key;
+      const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
+      const bool keep = i < nkb && (key > cut.key || (tie && tie_before + __popc(tb & lt) < cut.ties));
+      const uint32_t kb = __ballot_sync(0xFFFFFFFFu, keep);
+      if (keep) out[written + __popc(kb & lt)] = i;
+      if (mrow && i < nkb) mrow[i] = keep ? 1 : 0;
+      written += __popc(kb);
+      tie_before += __popc(tb);
+    }
+    if (lane == 0) kv_cnt[row] = written;
+    __syncwarp();
   }
-  if (threadIdx.x == 0) kv_cnt[row] = total;
 }
 
 // ---------------------------------------------------------------- uint8 mask -> lists
-__global__ void __launch_bounds__(kSelThreads) compact_mask_kernel(
+__global__ void __launch_bounds__(kSelWarpsMax * 32) compact_mask_kernel(
     const uint8_t* __restrict__ mask, int n_rows, int nkb, int* __restrict__ kv_idx,
     int* __restrict__ kv_cnt) {
-  __shared__ SelShared sh;
-  const int row = blockIdx.x;
-  if (row >= n_rows) return;
-  const uint8_t* mrow = mask + static_cast<long long>(row) * nkb;
-  int lo, hi;
-  chunk_range(nkb, &lo, &hi);
-  int mine = 0;
-  for (int i = lo; i < hi; ++i) mine += (mrow[i] != 0);
-  int total;
-  int pos = block_exclusive_scan(mine, sh, &total);
-  int* out = kv_idx + static_cast<long long>(row) * nkb;
-  for (int i = lo; i < hi; ++i)
-    if (mrow[i]) out[pos++] = i;
-  if (threadIdx.x == 0) kv_cnt[row] = total;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wpc = blockDim.x >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int row = blockIdx.x * wpc + warp; row < n_rows; row += gridDim.x * wpc) {
+    const uint8_t* mrow = mask + static_cast<long long>(row) * nkb;
+    int* out = kv_idx + static_cast<long long>(row) * nkb;
+    int written = 0;
+    for (int base = 0; base < nkb; base += 32) {
+      const int i = base + lane;
+      const bool keep = i < nkb && mrow[i] != 0;
+      const uint32_t kb = __ballot_sync(0xFFFFFFFFu, keep);
+      if (keep) out[written + __popc(kb & lt)] = i;
+      written += __popc(kb);
+    }
+    if (lane == 0) kv_cnt[row] = written;
+  }
 }
 
 // ---------------------------------------------------------------- launchers
@@ -542,15 +439,27 @@ cudaError_t launch_scores(const float* q_pool, const float* k_pool, int BH, int 
 cudaError_t launch_select(const float* s, long long s_ld, int n_rows, int nkb, int k_sel,
                           double topp, int* kv_idx, int* kv_cnt, uint8_t* mask,
                           cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(nkb) * 9 + 16;
-  cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  select_kernel<<<n_rows, kSelThreads, smem, st>>>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask);
+  const size_t slice = static_cast<size_t>(nkb) * 8 + 256 * 4;
+  int wpc = static_cast<int>((200u * 1024u) / slice);
+  wpc = wpc < 1 ? 1 : (wpc > kSelWarpsMax ? kSelWarpsMax : wpc);
+  const size_t smem = slice * wpc;
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int want = (n_rows + wpc - 1) / wpc;
+  const int per_sm = static_cast<int>((228u * 1024u) / (smem + 1024));
+  const int cap = sms * (per_sm < 1 ? 1 : per_sm) * 2;
+  const int grid = want < cap ? want : cap;
+  select_kernel<<<grid, wpc * 32, smem, st>>>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask);
   return cudaGetLastError();
 }
 
 cudaError_t launch_compact_mask(const uint8_t* mask, int n_rows, int nkb, int* kv_idx,
                                 int* kv_cnt, cudaStream_t st) {
-  compact_mask_kernel<<<n_rows, kSelThreads, 0, st>>>(mask, n_rows, nkb, kv_idx, kv_cnt);
+  const int grid = (n_rows + kSelWarpsMax - 1) / kSelWarpsMax;
+  compact_mask_kernel<<<grid < 65535 * 16 ? grid : 65535 * 16, kSelWarpsMax * 32, 0, st>>>(mask, n_rows, nkb, kv_idx, kv_cnt);
   return cudaGetLastError();
 }
 
