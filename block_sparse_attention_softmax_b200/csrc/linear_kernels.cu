@@ -8,11 +8,12 @@
 //   output: O_l[i] = phi(q_i)^T S / phi(q_i)^T z
 //   blend:  O[i]   = alpha ⊙ O_s[i] + (1 - alpha) ⊙ O_l[i]
 //
-// linear_state_kernel: one CTA per (token split, head). K and V tiles of 128
-//   tokens arrive by TMA; four warps apply phi to the K tile in shared memory
-//   (rounding phi(k) to bf16) and sum z; one thread issues
+// linear_state_kernel: persistent, one contiguous range of 128-token tiles per
+//   CTA. K and V tiles arrive by TMA; eight warps apply phi to the K tile in
+//   shared memory (rounding phi(k) to bf16) and sum z; one thread issues
 //   tcgen05.mma D[f, e] += phi(K)^T[f, t] V[t, e] with both operands MN-major,
-//   accumulating the split's S in TMEM. Partials are reduced in a fixed order.
+//   accumulating each head's share in TMEM. Per-(CTA, head) partials are
+//   reduced in a fixed order.
 // linear_out_kernel: each CTA stages [S | z] of its head in shared memory as a
 //   bf16 hi + lo pair (two MMAs recover ~16 mantissa bits), then for each
 //   128-token tile: TMA Q, phi in place, D[t, :] = phi(Q)[t, :] [S | z] in TMEM
@@ -30,14 +31,33 @@ constexpr int kLinStages = 3;
 
 __device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 
-int splits(int BH, int N) {
-  const int tiles = ceil_div(N, kLinTok);
-  const int want = ceil_div(2 * 148, BH);
-  return max(1, min(tiles, want));
+// Persistent geometry of the state kernel: the B*H*ceil(N/128) tiles, head
+// after head, are cut into one contiguous range per CTA. A range spans at most
+// `heads_per_cta` heads, each of which leaves one partial [S | z] slot.
+struct StateGeom {
+  int tph;            // tiles per head
+  int total;          // tiles over all heads
+  int grid;           // CTAs
+  int tpc;            // tiles per CTA
+  int hpc;            // partial slots per CTA
+};
+
+StateGeom state_geom(int BH, int N, int sms) {
+  StateGeom g;
+  g.tph = ceil_div(N, kLinTok);
+  g.total = BH * g.tph;
+  int grid = g.total < sms ? g.total : sms;
+  g.tpc = ceil_div(g.total, grid);
+  g.grid = ceil_div(g.total, g.tpc);
+  g.hpc = ceil_div(g.tpc, g.tph) + 1;
+  return g;
 }
 
-int tiles_per_split(int BH, int N) {
-  return ceil_div(ceil_div(N, kLinTok), splits(BH, N));
+int sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
 }
 
 template <int D>
@@ -47,8 +67,8 @@ struct StateLayout {
   static constexpr uint32_t V_BYTES = (D / 64) * CHUNK;
   static constexpr uint32_t STAGE = K_BYTES + V_BYTES;
   static constexpr uint32_t OFF_BAR = kLinStages * STAGE;
-  static constexpr uint32_t OFF_Z = OFF_BAR + 256;            // [8 or 16 phases][D] fp32
-  static constexpr uint32_t SMEM = OFF_Z + 16 * D * 4 + 1024;
+  static constexpr uint32_t OFF_Z = OFF_BAR + 256;            // [phases][D] fp32 (2048 floats)
+  static constexpr uint32_t SMEM = OFF_Z + 2048 * 4 + 1024;
 };
 
 template <int D>
@@ -75,54 +95,71 @@ __device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
 }  // namespace lin
 
 size_t linear_state_ws_bytes(int BH, int N, int d) {
-  return static_cast<size_t>(BH) * lin::splits(BH, N) * (static_cast<size_t>(d) * d + d) * sizeof(float);
+  const lin::StateGeom g = lin::state_geom(BH, N, lin::sm_count());
+  return static_cast<size_t>(g.grid) * g.hpc * (static_cast<size_t>(d) * d + d) * sizeof(float);
 }
 
 size_t linear_out_ws_bytes(int, int) { return 0; }
 
 // ---------------------------------------------------------------- state
-template <int D>
-__global__ void __launch_bounds__(lin::kLinThreads, 1)
-    linear_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                        int N, int nsplit, int tiles_per_split, float* __restrict__ part) {
-  using L = lin::StateLayout<D>;
+// Persistent: CTA c owns tiles [c*tpc, min(total, (c+1)*tpc)) of the head-major
+// tile list. Warp 0 loads K and V tiles (TMA, 3 stages), warps 2..9 apply phi
+// to K in shared memory and sum z, warp 1 issues the MMAs into one of two TMEM
+// accumulators per head segment; when a segment (the CTA's share of one head)
+// ends, the math warps copy its S and z into a partial slot while the next
+// segment accumulates into the other buffer.
+constexpr int kStateMathWarps = 8;
+constexpr int kStateThreads = 64 + 32 * kStateMathWarps;
 
+template <int D>
+__global__ void __launch_bounds__(kStateThreads, 1)
+    linear_state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        int N, lin::StateGeom geo, float* __restrict__ part) {
+  using L = lin::StateLayout<D>;
+  constexpr int NS = lin::kLinStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = lin::align1k(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint64_t* full = bars;                 // [lin::kLinStages] TMA landed
-  uint64_t* phi_done = bars + lin::kLinStages;   // [lin::kLinStages] phi applied (4 warps)
-  uint64_t* empty = bars + 2 * lin::kLinStages;  // [lin::kLinStages] MMA consumed
-  uint64_t* done = bars + 3 * lin::kLinStages;   // all MMAs complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* full = bars;                 // [NS] TMA landed
+  uint64_t* phi_done = bars + NS;        // [NS] phi applied (math warps)
+  uint64_t* empty = bars + 2 * NS;       // [NS] MMA consumed
+  uint64_t* acc_full = bars + 3 * NS;    // [2] segment accumulated
+  uint64_t* acc_empty = acc_full + 2;    // [2] segment copied out
+  uint64_t* zs_full = acc_empty + 2;     // z partials of a segment written (math warps)
+  uint64_t* zs_free = zs_full + 1;       // z partials of a segment read (math warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(zs_free + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* zs = reinterpret_cast<float*>(smem + L::OFF_Z);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x, bh = blockIdx.y;
-  const int tile0 = split * tiles_per_split;
-  const int n_tiles = max(0, min(tiles_per_split, ceil_div_dev(N, lin::kLinTok) - tile0));
-  const int t_end = N;
+  const int t0 = blockIdx.x * geo.tpc;
+  const int t1 = min(geo.total, t0 + geo.tpc);
+  const int n_tiles = max(0, t1 - t0);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < lin::kLinStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&phi_done[s], 4);
+      mbar_init(&phi_done[s], kStateMathWarps);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kStateMathWarps);
+    }
+    mbar_init(zs_full, kStateMathWarps);
+    mbar_init(zs_free, kStateMathWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (D == 64) {
     // the A operand always spans 128 features: zero the upper half once
-    for (int s = 0; s < lin::kLinStages; ++s)
+    for (int s = 0; s < NS; ++s)
       for (int i = threadIdx.x; i < static_cast<int>(L::CHUNK / 16); i += blockDim.x)
         reinterpret_cast<uint4*>(smem + s * L::STAGE + L::CHUNK)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 128);
+    tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -135,11 +172,13 @@ __global__ void __launch_bounds__(lin::kLinThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       for (int i = 0; i < n_tiles; ++i) {
-        const int s = i % lin::kLinStages;
-        if (!mbar_wait(&empty[s], ((i / lin::kLinStages) & 1) ^ 1, abort_flag)) break;
+        const int s = i % NS;
+        if (!mbar_wait(&empty[s], ((i / NS) & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&full[s], (D / 64) * 2 * L::CHUNK);
         uint8_t* st = smem + s * L::STAGE;
-        const int row = (tile0 + i) * lin::kLinTok;
+        const int t = t0 + i;
+        const int row = (t % geo.tph) * lin::kLinTok;
+        const int bh = t / geo.tph;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           tma_load_3d(st + c * L::CHUNK, &tmK, &full[s], c * 64, row, bh);
@@ -150,9 +189,14 @@ __global__ void __launch_bounds__(lin::kLinThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && n_tiles > 0) {
       const uint32_t idesc = idesc_bf16_f32(128, D, true, true);
+      int seg = 0;
+      bool first = true;
       for (int i = 0; i < n_tiles; ++i) {
-        const int s = i % lin::kLinStages;
-        if (!mbar_wait(&phi_done[s], (i / lin::kLinStages) & 1, abort_flag)) break;
+        const int s = i % NS;
+        const int t = t0 + i;
+        const int ab = seg & 1;
+        if (first && seg >= 2 && !mbar_wait(&acc_empty[ab], ((seg >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(&phi_done[s], (i / NS) & 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t kb = smem_u32(smem + s * L::STAGE);
         const uint32_t vb = kb + L::K_BYTES;
@@ -160,35 +204,44 @@ __global__ void __launch_bounds__(lin::kLinThreads, 1)
         for (int kk = 0; kk < lin::kLinTok / 16; ++kk) {
           const uint64_t a = sw128_desc(kb + kk * 2048u, L::CHUNK, 1024);
           const uint64_t b = sw128_desc(vb + kk * 2048u, L::CHUNK, 1024);
-          umma_ss(tm, a, b, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          umma_ss(tm + ab * 128, a, b, idesc, (!first || kk > 0) ? 1u : 0u);
         }
         tc_commit(&empty[s]);
+        first = false;
+        if (t + 1 == t1 || (t + 1) % geo.tph == 0) {
+          tc_commit(&acc_full[ab]);
+          ++seg;
+          first = true;
+        }
       }
-      tc_commit(done);
     }
   } else {
-    // math warps: phi on the K tile, z sums, then the epilogue
-    constexpr int NG = D / 8;            // 8-feature groups
-    constexpr int NP = 128 / NG;         // token phases
+    // math warps: phi on the K tile, z sums; segment ends copy S and z out
+    constexpr int NG = D / 8;                          // 8-feature groups
+    constexpr int NP = 32 * kStateMathWarps / NG;      // token phases
     const int mt = threadIdx.x - 64;
     const int gi = mt % NG, phase = mt / NG;
     const int chunk = gi / 8, lu = gi % 8;
     const int pu = lu ^ (phase % 8);     // physical 16-B unit (t % 8 == phase % 8 for every visited token)
+    const int quad = warp & 3, half = (warp - 2) >> 2;
+    const int frow = quad * 32 + lane;   // TMEM lane = feature row of phi(K)^T
     float z[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) z[e] = 0.f;
     bool ok = true;
+    int seg = 0;
     for (int i = 0; i < n_tiles; ++i) {
-      const int s = i % lin::kLinStages;
-      if (!mbar_wait(&full[s], (i / lin::kLinStages) & 1, abort_flag)) { ok = false; break; }
+      const int s = i % NS;
+      const int t = t0 + i;
+      if (!mbar_wait(&full[s], (i / NS) & 1, abort_flag)) { ok = false; break; }
       uint8_t* kt = smem + s * L::STAGE + chunk * L::CHUNK + pu * 16;
-      const int tok0 = (tile0 + i) * lin::kLinTok;
+      const int tok0 = (t % geo.tph) * lin::kLinTok;
 #pragma unroll 4
-      for (int t = phase; t < lin::kLinTok; t += NP) {
-        uint4* p = reinterpret_cast<uint4*>(kt + t * 128);
+      for (int tt = phase; tt < lin::kLinTok; tt += NP) {
+        uint4* p = reinterpret_cast<uint4*>(kt + tt * 128);
         uint4 w = *p;
         uint32_t* u = reinterpret_cast<uint32_t*>(&w);
-        if (tok0 + t < t_end) {
+        if (tok0 + tt < N) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float a = lin::phi_f(__uint_as_float(u[e] << 16));
@@ -206,59 +259,74 @@ __global__ void __launch_bounds__(lin::kLinThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&phi_done[s]);
-    }
-    // z partial: phases of one feature group are summed in a fixed order
+      if (t + 1 == t1 || (t + 1) % geo.tph == 0) {
+        // ---- segment end: partial slot (blockIdx.x, seg)
+        float* out = part + (static_cast<long long>(blockIdx.x) * geo.hpc + seg) * (D * D + D);
+        // z: every warp writes its phases, all read once every warp has written
+        if (seg >= 1 && !mbar_wait(zs_free, (seg - 1) & 1, abort_flag)) { ok = false; break; }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) zs[phase * D + gi * 8 + e] = z[e];
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    float* out = part + (static_cast<long long>(bh) * nsplit + split) * (D * D + D);
-    if (mt < D) {
-      float acc = 0.f;
-      for (int ph = 0; ph < NP; ++ph) acc += zs[ph * D + mt];
-      out[D * D + mt] = acc;
-    }
-    // S rows: TMEM lane = feature row of phi(K)^T
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    if (ok && n_tiles > 0) ok = mbar_wait(done, 0, abort_flag);
-    tc_fence_after();
-#pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t r[32];
-      if (ok && n_tiles > 0) {
-        tmem_ld32_wait(tm + (static_cast<uint32_t>(quad * 32) << 16) + c0, r);
-      } else {
+        for (int e = 0; e < 8; ++e) {
+          zs[phase * D + gi * 8 + e] = z[e];
+          z[e] = 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(zs_full);
+        if (!mbar_wait(zs_full, seg & 1, abort_flag)) { ok = false; break; }
+        if (mt < D) {
+          float acc = 0.f;
+          for (int ph = 0; ph < NP; ++ph) acc += zs[ph * D + mt];
+          out[D * D + mt] = acc;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(zs_free);
+        const int ab = seg & 1;
+        if (!mbar_wait(&acc_full[ab], (seg >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        constexpr int HC = D / 2;        // columns per half
 #pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = 0u;
+        for (int c0 = 0; c0 < HC; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32_wait(tm + ab * 128 + (static_cast<uint32_t>(quad * 32) << 16) + half * HC + c0, r);
+          if (frow < D) {
+            float4* dst = reinterpret_cast<float4*>(out + frow * D + half * HC + c0);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                   __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        ++seg;
       }
-      if (row < D) {
-        float4* dst = reinterpret_cast<float4*>(out + row * D + c0);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
-                               __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
-      }
     }
+    (void)ok;
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tm, 128);
+    tmem_dealloc(tm, 256);
   }
 }
 
+// Head h's partial slots, summed in CTA order.
 template <int D>
-__global__ void linear_reduce_kernel(const float* __restrict__ part, int nsplit,
+__global__ void linear_reduce_kernel(const float* __restrict__ part, lin::StateGeom geo,
                                      float* __restrict__ kv_state, float* __restrict__ ksum) {
-  const int bh = blockIdx.y;
+  const int h = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= D * D + D) return;
-  const float* p = part + static_cast<long long>(bh) * nsplit * (D * D + D) + e;
-  float s = 0.f;
-  for (int i = 0; i < nsplit; ++i) s += p[static_cast<long long>(i) * (D * D + D)];
-  if (e < D * D) kv_state[static_cast<long long>(bh) * D * D + e] = s;
-  else ksum[static_cast<long long>(bh) * D + (e - D * D)] = s;
+  const int c_first = (h * geo.tph) / geo.tpc;
+  const int c_last = ((h + 1) * geo.tph - 1) / geo.tpc;
+  float acc = 0.f;
+  for (int c = c_first; c <= c_last; ++c) {
+    const int seg = h - (c * geo.tpc) / geo.tph;
+    acc += part[(static_cast<long long>(c) * geo.hpc + seg) * (D * D + D) + e];
+  }
+  if (e < D * D) kv_state[static_cast<long long>(h) * D * D + e] = acc;
+  else ksum[static_cast<long long>(h) * D + (e - D * D)] = acc;
 }
 
 // ---------------------------------------------------------------- output + blend
@@ -456,19 +524,18 @@ template <int D>
 static cudaError_t state_d(const LinearArgs& a, cudaStream_t st) {
   using L = lin::StateLayout<D>;
   const int BH = a.B * a.H;
-  const int ns = lin::splits(BH, a.N);
-  const int tps = lin::tiles_per_split(BH, a.N);
+  const lin::StateGeom geo = lin::state_geom(BH, a.N, lin::sm_count());
   CUtensorMap mk, mv;
   if (encode_tensor_map_3d_bf16(&mk, a.k, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   if (encode_tensor_map_3d_bf16(&mv, a.v, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(linear_state_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   float* part = static_cast<float*>(a.ws);
-  linear_state_kernel<D><<<dim3(ns, BH), lin::kLinThreads, L::SMEM, st>>>(mk, mv, a.N, ns, tps, part);
+  linear_state_kernel<D><<<geo.grid, kStateThreads, L::SMEM, st>>>(mk, mv, a.N, geo, part);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int n = D * D + D;
-  linear_reduce_kernel<D><<<dim3(ceil_div(n, 256), BH), 256, 0, st>>>(part, ns, a.kv_state, a.ksum);
+  linear_reduce_kernel<D><<<dim3(ceil_div(n, 256), BH), 256, 0, st>>>(part, geo, a.kv_state, a.ksum);
   return cudaGetLastError();
 }
 
