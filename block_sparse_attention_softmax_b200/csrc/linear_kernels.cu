@@ -14,11 +14,11 @@
 //   tcgen05.mma D[f, e] += phi(K)^T[f, t] V[t, e] with both operands MN-major,
 //   accumulating each head's share in TMEM. Per-(CTA, head) partials are
 //   reduced in a fixed order.
-// linear_out_kernel: each CTA stages [S | z] of its head in shared memory as a
-//   bf16 hi + lo pair (two MMAs recover ~16 mantissa bits), then for each
-//   128-token tile: TMA Q, phi in place, D[t, :] = phi(Q)[t, :] [S | z] in TMEM
-//   (double buffered), and an epilogue that divides by the z column and blends
-//   with O_s.
+// linear_out_kernel: persistent over the same tile list; stages S of the
+//   current head in shared memory as a bf16 hi + lo pair (two MMAs recover ~16
+//   mantissa bits); per 128-token tile: TMA Q and O_s, phi(Q) in place,
+//   D[t, :] = phi(Q)[t, :] S in TMEM (double buffered), and an epilogue that
+//   divides by phi(q_t) . z and blends with O_s.
 #include "sa_internal.h"
 
 namespace sa {
@@ -73,19 +73,19 @@ struct StateLayout {
 
 template <int D>
 struct OutLayout {
-  static constexpr int NB = D + 16;                           // MMA N: S columns + z column
-  static constexpr int B_CHUNKS = (NB + 63) / 64;
-  static constexpr uint32_t B_CHUNK = D * 128;                // D rows (K) x 64 columns
-  static constexpr uint32_t B_BYTES = B_CHUNKS * B_CHUNK;     // one of hi / lo
-  static constexpr uint32_t Q_CHUNK = kLinTok * 128;
-  static constexpr uint32_t Q_BYTES = (D / 64) * Q_CHUNK;
+  static constexpr uint32_t B_CHUNK = D * 128;               // D rows (K) x 64 columns of S
+  static constexpr uint32_t B_BYTES = (D / 64) * B_CHUNK;    // one of hi / lo
+  static constexpr uint32_t T_CHUNK = kLinTok * 128;         // 128 tokens x 64 features
+  static constexpr uint32_t T_BYTES = (D / 64) * T_CHUNK;    // one Q or O_s tile
+  static constexpr int NSTG = 2;
   static constexpr uint32_t OFF_B = 0;
   static constexpr uint32_t OFF_Q = 2 * B_BYTES;
-  static constexpr uint32_t OFF_ALPHA = OFF_Q + kLinStages * Q_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_ALPHA + D * 4;
+  static constexpr uint32_t OFF_OS = OFF_Q + NSTG * T_BYTES;
+  static constexpr uint32_t OFF_Z = OFF_OS + NSTG * T_BYTES;  // z of the current head, fp32
+  static constexpr uint32_t OFF_ALPHA = OFF_Z + D * 4;         // alpha of the current head
+  static constexpr uint32_t OFF_RED = OFF_ALPHA + D * 4;       // [2 parity][2 halves][128 rows]
+  static constexpr uint32_t OFF_BAR = OFF_RED + 4 * 128 * 4;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
-  static constexpr uint32_t ACC_STRIDE = NB <= 128 ? 128 : 256;   // TMEM columns per buffer
-  static constexpr uint32_t TM_COLS = 2 * ACC_STRIDE;
 };
 
 __device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
@@ -330,76 +330,100 @@ __global__ void linear_reduce_kernel(const float* __restrict__ part, lin::StateG
 }
 
 // ---------------------------------------------------------------- output + blend
-template <int D>
-__global__ void __launch_bounds__(lin::kLinThreads, 1)
-    linear_out_kernel(const __grid_constant__ CUtensorMap tmQ, const float* __restrict__ kv_state,
-                      const float* __restrict__ ksum, const uint16_t* __restrict__ o_s,
-                      const float* __restrict__ alpha, int H, int N, int tiles_per_cta,
-                      uint16_t* __restrict__ o) {
-  using L = lin::OutLayout<D>;
+// Persistent over the same head-major tile list as the state kernel. Per tile
+// of 128 tokens: TMA brings Q (and O_s when blending) into a 2-stage ring; the
+// math warps apply phi to Q in place; one thread issues
+// D[t, :] = phi(Q)[t, :] S_hi + phi(Q)[t, :] S_lo (tcgen05, TMEM accumulator,
+// double buffered); the math warps then divide by phi(q_t) . z (CUDA cores,
+// from the phi(Q) tile still in shared memory), blend with O_s and store O.
+// Warp w and w+4 share TMEM lane quadrant w % 4 and split the d columns.
+constexpr int kOutMathWarps = 8;
+constexpr int kOutThreads = 64 + 32 * kOutMathWarps;
 
+template <int D>
+__device__ __forceinline__ void build_head_operand(uint8_t* smem, const float* __restrict__ kv_state,
+                                                   const float* __restrict__ ksum, const float* __restrict__ alpha,
+                                                   int bh, int h, int tid, int nthreads) {
+  using L = lin::OutLayout<D>;
+  // S as bf16 hi + lo, MN-major with 128-B swizzle: element (row c, column e)
+  // sits in chunk e/64, row c, 16-B unit ((e % 64) / 8) ^ (c % 8).
+  const float* Sg = kv_state + static_cast<long long>(bh) * D * D;
+  constexpr int UPR = D / 8;
+  for (int i = tid; i < D * UPR; i += nthreads) {
+    const int c = i / UPR, u = i % UPR;
+    const float4 a = *reinterpret_cast<const float4*>(Sg + c * D + u * 8);
+    const float4 b = *reinterpret_cast<const float4*>(Sg + c * D + u * 8 + 4);
+    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e2 = 0; e2 < 4; ++e2) {
+      const __nv_bfloat162 hb = __floats2bfloat162_rn(v[2 * e2], v[2 * e2 + 1]);
+      const float2 hf = __bfloat1622float2(hb);
+      hi[e2] = *reinterpret_cast<const uint32_t*>(&hb);
+      lo[e2] = pack_bf16x2(v[2 * e2] - hf.x, v[2 * e2 + 1] - hf.y);
+    }
+    const uint32_t off = (u / 8) * L::B_CHUNK + c * 128 + (((u % 8) ^ (c % 8)) * 16);
+    *reinterpret_cast<uint4*>(smem + L::OFF_B + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(smem + L::OFF_B + L::B_BYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+  float* zsm = reinterpret_cast<float*>(smem + L::OFF_Z);
+  float* al = reinterpret_cast<float*>(smem + L::OFF_ALPHA);
+  for (int e = tid; e < D; e += nthreads) {
+    zsm[e] = ksum[static_cast<long long>(bh) * D + e];
+    al[e] = alpha ? alpha[static_cast<long long>(h) * D + e] : 0.f;
+  }
+  fence_proxy_async_smem();
+}
+
+template <int D>
+__global__ void __launch_bounds__(kOutThreads, 1)
+    linear_out_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmOs,
+                      const float* __restrict__ kv_state, const float* __restrict__ ksum,
+                      const float* __restrict__ alpha, int H, int N, lin::StateGeom geo,
+                      int blend, uint16_t* __restrict__ o) {
+  using L = lin::OutLayout<D>;
+  constexpr int NS = L::NSTG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = lin::align1k(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint64_t* full = bars;                    // [lin::kLinStages]
-  uint64_t* phi_done = bars + lin::kLinStages;      // [lin::kLinStages]
-  uint64_t* empty = bars + 2 * lin::kLinStages;     // [lin::kLinStages]
-  uint64_t* acc_full = bars + 3 * lin::kLinStages;  // [2]
-  uint64_t* acc_empty = acc_full + 2;       // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* st_full = bars;                 // [NS] Q (+ O_s) landed
+  uint64_t* phi_done = bars + NS;           // [NS] phi applied (math warps)
+  uint64_t* st_empty = bars + 2 * NS;       // [NS] tile finished (math warps)
+  uint64_t* acc_full = bars + 3 * NS;       // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2] (math warps)
+  uint64_t* b_ready = acc_empty + 2;        // operand of a new head built (math warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(b_ready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* al = reinterpret_cast<float*>(smem + L::OFF_ALPHA);
+  const float* zsm = reinterpret_cast<const float*>(smem + L::OFF_Z);
+  const float* al = reinterpret_cast<const float*>(smem + L::OFF_ALPHA);
+  float* red = reinterpret_cast<float*>(smem + L::OFF_RED);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int h = bh % H;
-  const int tile0 = blockIdx.x * tiles_per_cta;
-  const int n_tiles = max(0, min(tiles_per_cta, ceil_div_dev(N, lin::kLinTok) - tile0));
+  const int t0 = blockIdx.x * geo.tpc;
+  const int t1 = min(geo.total, t0 + geo.tpc);
+  const int n_tiles = max(0, t1 - t0);
+  if (n_tiles == 0) return;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < lin::kLinStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&phi_done[s], 4);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&st_full[s], 1);
+      mbar_init(&phi_done[s], kOutMathWarps);
+      mbar_init(&st_empty[s], kOutMathWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], kOutMathWarps);
     }
+    mbar_init(b_ready, kOutMathWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // B operand [S | z] as bf16 hi and lo, MN-major with 128-B swizzle:
-  // element (row c, column e) sits in chunk e/64, row c, 16-B unit ((e%64)/8) ^ (c%8).
   {
-    const float* Sg = kv_state + static_cast<long long>(bh) * D * D;
-    const float* zg = ksum + static_cast<long long>(bh) * D;
-    constexpr int UPR = L::B_CHUNKS * 8;    // 16-B units per row (incl. zero padding)
-    for (int i = threadIdx.x; i < D * UPR; i += blockDim.x) {
-      const int c = i / UPR, u = i % UPR;
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int e2 = 0; e2 < 4; ++e2) {
-        float v2[2];
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const int e = u * 8 + e2 * 2 + t;
-          v2[t] = e < D ? Sg[c * D + e] : (e == D ? zg[c] : 0.f);
-        }
-        const __nv_bfloat162 hb = __floats2bfloat162_rn(v2[0], v2[1]);
-        const float2 hf = __bfloat1622float2(hb);
-        hi[e2] = *reinterpret_cast<const uint32_t*>(&hb);
-        lo[e2] = pack_bf16x2(v2[0] - hf.x, v2[1] - hf.y);
-      }
-      const uint32_t off = (u / 8) * L::B_CHUNK + c * 128 + (((u % 8) ^ (c % 8)) * 16);
-      *reinterpret_cast<uint4*>(smem + L::OFF_B + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(smem + L::OFF_B + L::B_BYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    }
-    for (int e = threadIdx.x; e < D; e += blockDim.x) al[e] = alpha ? alpha[static_cast<long long>(h) * D + e] : 0.f;
-    fence_proxy_async_smem();
+    const int bh0 = t0 / geo.tph;
+    build_head_operand<D>(smem, kv_state, ksum, alpha, bh0, bh0 % H, threadIdx.x, blockDim.x);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, L::TM_COLS);
+    tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -408,95 +432,135 @@ __global__ void __launch_bounds__(lin::kLinThreads, 1)
   const uint32_t tm = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0) {
       tma_prefetch_desc(&tmQ);
+      if (blend) tma_prefetch_desc(&tmOs);
       for (int i = 0; i < n_tiles; ++i) {
-        const int s = i % lin::kLinStages;
-        if (!mbar_wait(&empty[s], ((i / lin::kLinStages) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&full[s], L::Q_BYTES);
-        uint8_t* st = smem + L::OFF_Q + s * L::Q_BYTES;
+        const int s = i % NS;
+        if (!mbar_wait(&st_empty[s], ((i / NS) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&st_full[s], (blend ? 2u : 1u) * L::T_BYTES);
+        const int t = t0 + i;
+        const int row = (t % geo.tph) * lin::kLinTok, bh = t / geo.tph;
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) tma_load_3d(st + c * L::Q_CHUNK, &tmQ, &full[s], c * 64, (tile0 + i) * lin::kLinTok, bh);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(smem + L::OFF_Q + s * L::T_BYTES + c * L::T_CHUNK, &tmQ, &st_full[s], c * 64, row, bh);
+          if (blend)
+            tma_load_3d(smem + L::OFF_OS + s * L::T_BYTES + c * L::T_CHUNK, &tmOs, &st_full[s], c * 64, row, bh);
+        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && n_tiles > 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, L::NB, false, true);
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, D, false, true);
       const uint32_t bhi = smem_u32(smem + L::OFF_B), blo = bhi + L::B_BYTES;
+      int changes = 0;
       for (int i = 0; i < n_tiles; ++i) {
-        const int s = i % lin::kLinStages, b = i & 1;
-        if (!mbar_wait(&phi_done[s], (i / lin::kLinStages) & 1, abort_flag)) break;
-        if (!mbar_wait(&acc_empty[b], ((i >> 1) & 1) ^ 1, abort_flag)) break;
+        const int s = i % NS, ab = i & 1;
+        const int t = t0 + i;
+        if (i > 0 && t / geo.tph != (t - 1) / geo.tph) {
+          if (!mbar_wait(b_ready, changes & 1, abort_flag)) break;
+          ++changes;
+        }
+        if (!mbar_wait(&phi_done[s], (i / NS) & 1, abort_flag)) break;
+        if (!mbar_wait(&acc_empty[ab], ((i >> 1) & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t qb = smem_u32(smem + L::OFF_Q + s * L::Q_BYTES);
-        const uint32_t d_tm = tm + b * L::ACC_STRIDE;
+        const uint32_t qb = smem_u32(smem + L::OFF_Q + s * L::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = sw128_desc(qb + (kk >> 2) * L::Q_CHUNK + (kk & 3) * 32u, 16, 1024);
-          umma_ss(d_tm, a, sw128_desc(bhi + kk * 2048u, L::B_CHUNK, 1024), idesc, kk > 0 ? 1u : 0u);
-          umma_ss(d_tm, a, sw128_desc(blo + kk * 2048u, L::B_CHUNK, 1024), idesc, 1u);
+          const uint64_t a = sw128_desc(qb + (kk >> 2) * L::T_CHUNK + (kk & 3) * 32u, 16, 1024);
+          umma_ss(tm + ab * 128, a, sw128_desc(bhi + kk * 2048u, L::B_CHUNK, 1024), idesc, kk > 0 ? 1u : 0u);
+          umma_ss(tm + ab * 128, a, sw128_desc(blo + kk * 2048u, L::B_CHUNK, 1024), idesc, 1u);
         }
-        tc_commit(&acc_full[b]);
-        tc_commit(&empty[s]);
+        tc_commit(&acc_full[ab]);
       }
     }
   } else {
     const int mt = threadIdx.x - 64;
-    const int quad = warp & 3;
+    const int quad = warp & 3, half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    const int pair_bar = 1 + quad;
+    constexpr int HC = D / 2;                 // columns per half
+    constexpr int HU = HC / 8;                // 16-B units per half row
     bool ok = true;
-    auto epilogue = [&](int i) {
-      const int b = i & 1;
-      if (!mbar_wait(&acc_full[b], (i >> 1) & 1, abort_flag)) { ok = false; return; }
+    int changes = 0;
+    auto epilogue = [&](int j) -> bool {
+      const int ab = j & 1, s = j % NS;
+      const int t = t0 + j;
+      const int bh = t / geo.tph;
+      const int tok = (t % geo.tph) * lin::kLinTok + row;
+      if (!mbar_wait(&acc_full[ab], (j >> 1) & 1, abort_flag)) return false;
       tc_fence_after();
-      const int tok = (tile0 + i) * lin::kLinTok + row;
-      uint32_t dz[32];
-      tmem_ld32_wait(tm + lane_addr + b * L::ACC_STRIDE + D, dz);
-      const float inv = 1.f / __uint_as_float(dz[0]);
-      const long long base = (static_cast<long long>(bh) * N + tok) * D;
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32_wait(tm + lane_addr + b * L::ACC_STRIDE + c0, r);
-        if (tok < N) {
-          uint32_t pk[16];
-          if (o_s) {
-            const uint4* src = reinterpret_cast<const uint4*>(o_s + base + c0);
-            uint32_t os[16];
+      uint32_t x0[32], x1[32];
+      tmem_ld32(tm + ab * 128 + lane_addr + half * HC, x0);
+      if (HC == 64) tmem_ld32(tm + ab * 128 + lane_addr + half * HC + 32, x1);
+      tmem_wait_ld();
+      reg_fence(x0);
+      if (HC == 64) reg_fence(x1);
+      // phi(q) . z over this half's features, from the phi(Q) tile in shared memory
+      const uint8_t* qrow = smem + L::OFF_Q + s * L::T_BYTES;
+      float dz = 0.f;
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
-              const uint4 w = src[v4];
-              os[4 * v4] = w.x; os[4 * v4 + 1] = w.y; os[4 * v4 + 2] = w.z; os[4 * v4 + 3] = w.w;
-            }
+      for (int j2 = 0; j2 < HU; ++j2) {
+        const int uu = half * HU + j2;        // unit along d
+        const uint4 w = *reinterpret_cast<const uint4*>(qrow + (uu >> 3) * L::T_CHUNK + row * 128 + (((uu & 7) ^ (row & 7)) << 4));
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float a0 = al[c0 + 2 * e], a1 = al[c0 + 2 * e + 1];
-              const float l0 = __uint_as_float(r[2 * e]) * inv, l1 = __uint_as_float(r[2 * e + 1]) * inv;
-              const float s0 = __uint_as_float(os[e] << 16), s1 = __uint_as_float(os[e] & 0xFFFF0000u);
-              pk[e] = pack_bf16x2(fmaf(a0, s0 - l0, l0), fmaf(a1, s1 - l1, l1));
+        for (int e = 0; e < 4; ++e) {
+          dz = fmaf(__uint_as_float(wv[e] << 16), zsm[uu * 8 + 2 * e], dz);
+          dz = fmaf(__uint_as_float(wv[e] & 0xFFFF0000u), zsm[uu * 8 + 2 * e + 1], dz);
+        }
+      }
+      float* rj = red + (j & 1) * 2 * 128;
+      rj[half * 128 + row] = dz;
+      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+      const float inv = 1.f / (dz + rj[(half ^ 1) * 128 + row]);
+      if (tok < N) {
+        const uint8_t* osrow = smem + L::OFF_OS + s * L::T_BYTES;
+        uint16_t* orow = o + (static_cast<long long>(bh) * N + tok) * D + half * HC;
+#pragma unroll
+        for (int j2 = 0; j2 < HU; ++j2) {
+          const int uu = half * HU + j2;
+          const int c = j2 * 8;               // column within this half
+          float l[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t bits = (c + e) < 32 ? x0[c + e] : x1[c + e - 32];
+            l[e] = __uint_as_float(bits) * inv;
+          }
+          uint32_t pk[4];
+          if (blend) {
+            const uint4 w = *reinterpret_cast<const uint4*>(osrow + (uu >> 3) * L::T_CHUNK + row * 128 + (((uu & 7) ^ (row & 7)) << 4));
+            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float a0 = al[uu * 8 + 2 * e], a1 = al[uu * 8 + 2 * e + 1];
+              const float s0 = __uint_as_float(wv[e] << 16), s1 = __uint_as_float(wv[e] & 0xFFFF0000u);
+              pk[e] = pack_bf16x2(fmaf(a0, s0 - l[2 * e], l[2 * e]), fmaf(a1, s1 - l[2 * e + 1], l[2 * e + 1]));
             }
           } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
+            for (int e = 0; e < 4; ++e) pk[e] = pack_bf16x2(l[2 * e], l[2 * e + 1]);
           }
-          uint4* dst = reinterpret_cast<uint4*>(o + base + c0);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          reinterpret_cast<uint4*>(orow)[j2] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[b]);
+      if (lane == 0) {
+        mbar_arrive(&acc_empty[ab]);
+        mbar_arrive(&st_empty[s]);
+      }
+      return true;
     };
-    for (int i = 0; i < n_tiles && ok; ++i) {
-      const int s = i % lin::kLinStages;
-      if (!mbar_wait(&full[s], (i / lin::kLinStages) & 1, abort_flag)) { ok = false; break; }
+    for (int i = 0; ok && i < n_tiles; ++i) {
+      const int s = i % NS;
+      const int t = t0 + i;
+      if (!(ok = mbar_wait(&st_full[s], (i / NS) & 1, abort_flag))) break;
       // phi in place: elementwise, so the swizzled layout does not matter
-      uint4* qt = reinterpret_cast<uint4*>(smem + L::OFF_Q + s * L::Q_BYTES);
+      uint4* qt = reinterpret_cast<uint4*>(smem + L::OFF_Q + s * L::T_BYTES);
 #pragma unroll 4
-      for (int u = mt; u < static_cast<int>(L::Q_BYTES / 16); u += 128) {
+      for (int u = mt; u < static_cast<int>(L::T_BYTES / 16); u += 32 * kOutMathWarps) {
         uint4 w = qt[u];
         uint32_t* x = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
@@ -507,15 +571,27 @@ __global__ void __launch_bounds__(lin::kLinThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&phi_done[s]);
-      if (i > 0) epilogue(i - 1);
+      if (i > 0) {
+        if (!(ok = epilogue(i - 1))) break;
+        if (t / geo.tph != (t - 1) / geo.tph) {
+          // every MMA of the previous head has completed (its last accumulator
+          // was just read): rebuild the operand, z and alpha for this head
+          const int bh = t / geo.tph;
+          build_head_operand<D>(smem, kv_state, ksum, alpha, bh, bh % H, mt, 32 * kOutMathWarps);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_ready);
+          if (!(ok = mbar_wait(b_ready, changes & 1, abort_flag))) break;
+          ++changes;
+        }
+      }
     }
-    if (ok && n_tiles > 0) epilogue(n_tiles - 1);
+    if (ok) epilogue(n_tiles - 1);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tm, L::TM_COLS);
+    tmem_dealloc(tm, 256);
   }
 }
 
@@ -547,16 +623,16 @@ template <int D>
 static cudaError_t out_d(const LinearArgs& a, cudaStream_t st) {
   using L = lin::OutLayout<D>;
   const int BH = a.B * a.H;
-  const int tiles = ceil_div(a.N, lin::kLinTok);
-  const int ctas_per_head = max(1, min(tiles, ceil_div(4 * 148, BH)));
-  const int tpc = ceil_div(tiles, ctas_per_head);
-  CUtensorMap mq;
+  const lin::StateGeom geo = lin::state_geom(BH, a.N, lin::sm_count());
+  CUtensorMap mq, mos;
   if (encode_tensor_map_3d_bf16(&mq, a.q, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  const int blend = a.o_s != nullptr;
+  if (encode_tensor_map_3d_bf16(&mos, blend ? a.o_s : a.q, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(linear_out_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  linear_out_kernel<D><<<dim3(ceil_div(tiles, tpc), BH), lin::kLinThreads, L::SMEM, st>>>(
-      mq, a.kv_state, a.ksum, static_cast<const uint16_t*>(a.o_s), a.alpha, a.H, a.N, tpc,
-      static_cast<uint16_t*>(a.o));
+  linear_out_kernel<D><<<geo.grid, kOutThreads, L::SMEM, st>>>(
+      mq, mos, a.kv_state, a.ksum, blend ? a.alpha : nullptr, a.H, a.N, geo, blend, static_cast<uint16_t*>(a.o));
   return cudaGetLastError();
 }
 
