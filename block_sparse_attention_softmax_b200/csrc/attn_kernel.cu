@@ -8,37 +8,33 @@
 // the K/V blocks of one head in L2. Inside an item, two 64-key blocks from the
 // item's kept list form one 128-key tile.
 //
-// Shared-memory bandwidth is the resource this kernel is shaped around: per
-// tile the TMA writes K and V (64 KB at d = 128) and the tensor core reads K and
-// V once each. Q and P never come from shared memory: Q is copied into TMEM
-// once per item and both products take their A operand from TMEM.
+// The per-tile chain QK(g) -> softmax(g) -> PV(g) is what limits this kernel,
+// so the tensor core is kept fed from three S buffers: QK runs two tiles ahead
+// of PV, and the QK that overwrites an S buffer only has to follow the PV of
+// the tile three back (one thread's tcgen05.mma operations execute in issue
+// order, so no wait is needed for that).
 //
-//   warp 0       TMA producer of Q (one slot) and K (3-stage ring)
+//   warp 0       TMA producer of Q (one slot) and K (3-stage ring; a slot is
+//                free once the QK that read it has completed, which is the
+//                same event that fills the S buffer of that tile)
 //   warp 10      TMA producer of V (2-stage ring); one TMA box per 64-key
 //                block, so the two blocks of a tile need not be adjacent
 //   warp 1       TMEM allocation and the single MMA-issuing thread:
-//                  S_g = Q K_g^T  (A = Q from TMEM, B = K from shared memory)
+//                  S_g = Q K_g^T  (A = Q, B = K, both from shared memory)
 //                  O  += P_g V_g  (A = P_g from TMEM, B = V from shared memory)
-//                QK of tile g+1 is issued before PV of tile g, so the tensor
-//                core has work queued while the softmax of tile g runs. The
-//                QK that overwrites an S buffer is issued after the PV that
-//                reads the P stored there; one thread's tcgen05.mma operations
-//                execute in issue order.
 //   warps 2..9   softmax: TMEM lane quadrant q = warp % 4 holds query rows
 //                32q..32q+31; warp w and w+4 split the 128 columns of those
 //                rows (64 each) and exchange the row max through shared
 //                memory. The running max m is kept in the log2 domain and only
 //                raised when a tile's max exceeds it by more than 8 (P <= 256
 //                otherwise); then O is rescaled in TMEM. P = exp2(S*scale*log2e
-//                - m) is written back over S as packed bf16. The same warps
-//                copy each item's Q tile from shared memory into TMEM (after
-//                the last S of the previous item has landed), then copy O to
-//                registers, release it, and write O / l as bf16 and the row
-//                log-sum-exp.
+//                - m) is written back over S as packed bf16. At the end of an
+//                item the warps copy O to registers, release it, and write
+//                O / l as bf16 and the row log-sum-exp.
 //
-// TMEM columns: Q at 0 (d/2 wide, bf16 pairs), S buffers at 128 and 256 (fp32,
-// 128 wide; P aliases their first 64 columns), O at 384 (d wide). Every
-// mbarrier wait is bounded (see sa_device.cuh).
+// TMEM columns: S buffers at 0, 128 and 256 (fp32, 128 wide; P aliases their
+// first 64 columns), O at 384 (d wide). Every mbarrier wait is bounded (see
+// sa_device.cuh).
 #include "sa_internal.h"
 
 namespace sa {
@@ -50,7 +46,7 @@ constexpr int kBN = 128;        // keys per tile (two 64-key blocks)
 constexpr int kSoftWarps = 8;
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
-constexpr int kSBufs = 2;
+constexpr int kSBufs = 3;
 constexpr int kVWarp = 2 + kSoftWarps;               // warp index of the V producer
 constexpr int kThreads = 32 * (kVWarp + 1);
 
@@ -73,18 +69,17 @@ struct Layout {
   static constexpr uint32_t SMEM = (USED + 1024 > 120 * 1024) ? USED + 1024 : 120 * 1024;
 };
 
-constexpr uint32_t TM_Q = 0;
-__host__ __device__ constexpr uint32_t tm_s(int b) { return 128u + static_cast<uint32_t>(b) * 128u; }
+__host__ __device__ constexpr uint32_t tm_s(int b) { return static_cast<uint32_t>(b) * 128u; }
 constexpr uint32_t TM_O = 384;
 constexpr uint32_t TM_COLS = 512;
 
+static_assert(kKStages == kSBufs, "a K slot is freed by the S_FULL commit of its tile");
+
 enum {
   B_QFULL = 0,                       // Q tile landed in shared memory
-  B_QEMPTY = 1,                      // Q copied out of shared memory (8 warps)
-  B_QTMEM = 2,                       // Q present in TMEM (8 warps)
-  B_KFULL = 3,                       // [kKStages]
-  B_KEMPTY = B_KFULL + kKStages,     // [kKStages]
-  B_VFULL = B_KEMPTY + kKStages,     // [kVStages]
+  B_QEMPTY = 1,                      // last QK of the item completed
+  B_KFULL = 2,                       // [kKStages]
+  B_VFULL = B_KFULL + kKStages,      // [kVStages]
   B_VEMPTY = B_VFULL + kVStages,     // [kVStages]
   B_SFULL = B_VEMPTY + kVStages,     // [kSBufs]
   B_PFULL = B_SFULL + kSBufs,        // [kSBufs]
@@ -150,14 +145,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[B_QFULL], 1);
-    mbar_init(&bars[B_QEMPTY], kSoftWarps);
-    mbar_init(&bars[B_QTMEM], kSoftWarps);
+    mbar_init(&bars[B_QEMPTY], 1);
     mbar_init(&bars[B_OFULL], 1);
     mbar_init(&bars[B_OEMPTY], kSoftWarps);
-    for (int i = 0; i < kKStages; ++i) {
-      mbar_init(&bars[B_KFULL + i], 1);
-      mbar_init(&bars[B_KEMPTY + i], 1);
-    }
+    for (int i = 0; i < kKStages; ++i) mbar_init(&bars[B_KFULL + i], 1);
     for (int i = 0; i < kVStages; ++i) {
       mbar_init(&bars[B_VFULL + i], 1);
       mbar_init(&bars[B_VEMPTY + i], 1);
@@ -193,7 +184,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       uint8_t* ring = is_k ? sK : sV;
       const int stages = is_k ? kKStages : kVStages;
       const int b_full = is_k ? B_KFULL : B_VFULL;
-      const int b_empty = is_k ? B_KEMPTY : B_VEMPTY;
+      const int b_empty = is_k ? B_SFULL : B_VEMPTY;
       int g = 0, qi = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
@@ -232,12 +223,12 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       // MMA groups minimal: ring slots and phases advance incrementally,
       // descriptors are precomputed bases plus constant offsets, and the next
       // item's facts are fetched one item ahead.
+      const uint64_t qdesc0 = sw128_desc(smem_u32(sQ), 16, 1024);
       const uint64_t kdesc0 = sw128_desc(smem_u32(sK), 16, 1024);
       const uint64_t vdesc0 = sw128_desc(smem_u32(sV), L::KV_CHUNK, 1024);
       const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
       const uint32_t idesc_qk2 = idesc_bf16_f32(kBM, 128, false, false);
       const uint32_t idesc_qk1 = idesc_bf16_f32(kBM, 64, false, false);
-      const uint32_t q_tm = tm + TM_Q;
       const uint32_t o_tm = tm + TM_O;
       struct Ring {
         int slot, n;
@@ -265,7 +256,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 
       auto issue_qk = [&]() -> bool {
         if (qk_t == 0) {
-          if (!mbar_wait(&bars[B_QTMEM], qk_qphase, abort_flag)) return false;
+          if (!mbar_wait(&bars[B_QFULL], qk_qphase, abort_flag)) return false;
           qk_qphase ^= 1u;
         }
         if (!mbar_wait(&bars[B_KFULL + qk_k.slot], qk_k.phase, abort_flag)) return false;
@@ -276,10 +267,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         const uint32_t s_tm = tm + tm_s(qk_s.slot);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          umma_ts(s_tm, q_tm + kk * 8, kd + ((((kk >> 2) * L::KV_CHUNK) + (kk & 3) * 32u) >> 4), idesc,
-                  kk > 0 ? 1u : 0u);
-        tc_commit(&bars[B_SFULL + qk_s.slot]);
-        tc_commit(&bars[B_KEMPTY + qk_k.slot]);
+          umma_ss(s_tm, qdesc0 + ((((kk >> 2) * L::Q_CHUNK) + (kk & 3) * 32u) >> 4),
+                  kd + ((((kk >> 2) * L::KV_CHUNK) + (kk & 3) * 32u) >> 4), idesc, kk > 0 ? 1u : 0u);
+        tc_commit(&bars[B_SFULL + qk_s.slot]);   // S ready, and the K slot free
+        if (qk_t + 1 == qk_it.T) tc_commit(&bars[B_QEMPTY]);
         qk_k.next();
         qk_s.next();
         if (++qk_t == qk_it.T) {
@@ -319,7 +310,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         }
         return true;
       };
-      if (qk_item < n_items) ok = issue_qk();
+      for (int pre = 0; pre < 2 && ok && qk_item < n_items; ++pre) ok = issue_qk();
       while (ok && pv_item < n_items) {
         if (qk_item < n_items && !(ok = issue_qk())) break;
         if (!(ok = issue_pv())) break;
@@ -338,32 +329,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     int g = 0, qi = 0;
     bool ok = true;
 
-    // Q tile of the qi-th non-empty item: shared memory -> TMEM (bf16 pairs,
-    // row = lane), this half's d range.
-    auto copy_q = [&](int q_index) -> bool {
-      if (!mbar_wait(&bars[B_QFULL], q_index & 1, abort_flag)) return false;
-      constexpr int U = D / 16;               // 16-B units per half row
-      uint32_t w[U * 4];
-#pragma unroll
-      for (int j = 0; j < U; ++j) {
-        const int uu = half * U + j;          // unit index along d
-        const uint4 v = *reinterpret_cast<const uint4*>(
-            sQ + (uu >> 3) * L::Q_CHUNK + row * 128 + (((uu & 7) ^ (row & 7)) << 4));
-        w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
-      }
-      tmem_st_cols<U * 4>(tm + lane_addr + TM_Q + half * (U * 4), w);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bars[B_QEMPTY]);
-        mbar_arrive(&bars[B_QTMEM]);
-      }
-      return true;
-    };
-
     int item = next_nonempty(a, blockIdx.x, gridDim.x, n_items);
-    if (item < n_items) ok = copy_q(0);
     // items with no kept block before the first non-empty one
     for (int z = blockIdx.x; z < item; z += gridDim.x) {
       const Item it = load_item(a, z);
@@ -467,10 +433,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (lane == 0) mbar_arrive(&bars[B_PFULL + b]);
       }
       if (!ok) break;
-      // Every S of this item has landed, so no QK reads Q any more: bring in
-      // the next item's Q before finishing this one.
       const int next = next_nonempty(a, item + gridDim.x, gridDim.x, n_items);
-      if (next < n_items && !(ok = copy_q(qi + 1))) break;
       // ---------------------------------------------------------- epilogue
       if (!(ok = mbar_wait(&bars[B_OFULL], qi & 1, abort_flag))) break;
       tc_fence_after();
