@@ -29,7 +29,11 @@ constexpr int kLinTok = 128;       // tokens per tile (K extent of the state MMA
 constexpr int kLinThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 math
 constexpr int kLinStages = 3;
 
-__device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+// phi(x) = elu(x) + 1, written branch-free: exp(min(x, 0)) + max(x, 0)
+// (exactly x + 1 for x > 0, exp(x) otherwise).
+__device__ __forceinline__ float phi_f(float x) {
+  return fast_exp2(fminf(x, 0.f) * 1.4426950408889634f) + fmaxf(x, 0.f);
+}
 
 // Persistent geometry of the state kernel: the B*H*ceil(N/128) tiles, head
 // after head, are cut into one contiguous range per CTA. A range spans at most
@@ -67,8 +71,8 @@ struct StateLayout {
   static constexpr uint32_t V_BYTES = (D / 64) * CHUNK;
   static constexpr uint32_t STAGE = K_BYTES + V_BYTES;
   static constexpr uint32_t OFF_BAR = kLinStages * STAGE;
-  static constexpr uint32_t OFF_Z = OFF_BAR + 256;            // [phases][D] fp32 (2048 floats)
-  static constexpr uint32_t SMEM = OFF_Z + 2048 * 4 + 1024;
+  static constexpr uint32_t OFF_Z = OFF_BAR + 256;            // [phases][D] fp32 (4096 floats)
+  static constexpr uint32_t SMEM = OFF_Z + 4096 * 4 + 1024;
 };
 
 template <int D>
@@ -83,8 +87,8 @@ struct OutLayout {
   static constexpr uint32_t OFF_OS = OFF_Q + NSTG * T_BYTES;
   static constexpr uint32_t OFF_Z = OFF_OS + NSTG * T_BYTES;  // z of the current head, fp32
   static constexpr uint32_t OFF_ALPHA = OFF_Z + D * 4;         // alpha of the current head
-  static constexpr uint32_t OFF_RED = OFF_ALPHA + D * 4;       // [2 parity][2 halves][128 rows]
-  static constexpr uint32_t OFF_BAR = OFF_RED + 4 * 128 * 4;
+  static constexpr uint32_t OFF_RED = OFF_ALPHA + D * 4;       // [2 parity][4 groups][128 rows]
+  static constexpr uint32_t OFF_BAR = OFF_RED + 8 * 128 * 4;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
 };
 
@@ -108,7 +112,7 @@ size_t linear_out_ws_bytes(int, int) { return 0; }
 // accumulators per head segment; when a segment (the CTA's share of one head)
 // ends, the math warps copy its S and z into a partial slot while the next
 // segment accumulates into the other buffer.
-constexpr int kStateMathWarps = 8;
+constexpr int kStateMathWarps = 16;
 constexpr int kStateThreads = 64 + 32 * kStateMathWarps;
 
 template <int D>
@@ -223,7 +227,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const int gi = mt % NG, phase = mt / NG;
     const int chunk = gi / 8, lu = gi % 8;
     const int pu = lu ^ (phase % 8);     // physical 16-B unit (t % 8 == phase % 8 for every visited token)
-    const int quad = warp & 3, half = (warp - 2) >> 2;
+    constexpr int CG = kStateMathWarps / 4;            // column groups per lane quadrant
+    const int quad = warp & 3, cgrp = (warp - 2) >> 2;
     const int frow = quad * 32 + lane;   // TMEM lane = feature row of phi(K)^T
     float z[8];
 #pragma unroll
@@ -236,12 +241,13 @@ __global__ void __launch_bounds__(kStateThreads, 1)
       if (!mbar_wait(&full[s], (i / NS) & 1, abort_flag)) { ok = false; break; }
       uint8_t* kt = smem + s * L::STAGE + chunk * L::CHUNK + pu * 16;
       const int tok0 = (t % geo.tph) * lin::kLinTok;
-#pragma unroll 4
+      const bool full_tile = tok0 + lin::kLinTok <= N;
+#pragma unroll
       for (int tt = phase; tt < lin::kLinTok; tt += NP) {
         uint4* p = reinterpret_cast<uint4*>(kt + tt * 128);
         uint4 w = *p;
         uint32_t* u = reinterpret_cast<uint32_t*>(&w);
-        if (tok0 + tt < N) {
+        if (full_tile || tok0 + tt < N) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float a = lin::phi_f(__uint_as_float(u[e] << 16));
@@ -252,7 +258,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             z[2 * e + 1] += __uint_as_float(pk & 0xFFFF0000u);
           }
         } else {
-          w = make_uint4(0, 0, 0, 0);
+          w = make_uint4(0, 0, 0, 0);   // keys past N contribute nothing
         }
         *p = w;
       }
@@ -282,15 +288,22 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         const int ab = seg & 1;
         if (!mbar_wait(&acc_full[ab], (seg >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        constexpr int HC = D / 2;        // columns per half
-#pragma unroll
-        for (int c0 = 0; c0 < HC; c0 += 32) {
+        constexpr int HC = D / CG;       // columns per column group (32 or 16)
+        {
           uint32_t r[32];
-          tmem_ld32_wait(tm + ab * 128 + (static_cast<uint32_t>(quad * 32) << 16) + half * HC + c0, r);
-          if (frow < D) {
-            float4* dst = reinterpret_cast<float4*>(out + frow * D + half * HC + c0);
+          const uint32_t ta = tm + ab * 128 + (static_cast<uint32_t>(quad * 32) << 16) + cgrp * HC;
+          if (HC == 32) {
+            tmem_ld32_wait(ta, r);
+          } else {
+            uint32_t r16[16];
+            tmem_ld16_wait(ta, r16);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
+            for (int e = 0; e < 16; ++e) r[e] = r16[e];
+          }
+          if (frow < D) {
+            float4* dst = reinterpret_cast<float4*>(out + frow * D + cgrp * HC);
+#pragma unroll
+            for (int e = 0; e < HC / 4; ++e)
               dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
                                    __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
           }
@@ -336,8 +349,8 @@ __global__ void linear_reduce_kernel(const float* __restrict__ part, lin::StateG
 // D[t, :] = phi(Q)[t, :] S_hi + phi(Q)[t, :] S_lo (tcgen05, TMEM accumulator,
 // double buffered); the math warps then divide by phi(q_t) . z (CUDA cores,
 // from the phi(Q) tile still in shared memory), blend with O_s and store O.
-// Warp w and w+4 share TMEM lane quadrant w % 4 and split the d columns.
-constexpr int kOutMathWarps = 8;
+// The four warps that share TMEM lane quadrant w % 4 split the d columns.
+constexpr int kOutMathWarps = 16;
 constexpr int kOutThreads = 64 + 32 * kOutMathWarps;
 
 template <int D>
@@ -476,12 +489,12 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     }
   } else {
     const int mt = threadIdx.x - 64;
-    const int quad = warp & 3, half = (warp - 2) >> 2;
+    const int quad = warp & 3, half = (warp - 2) >> 2;   // half: column group 0..3
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    const int pair_bar = 1 + quad;
-    constexpr int HC = D / 2;                 // columns per half
-    constexpr int HU = HC / 8;                // 16-B units per half row
+    const int quad_bar = 1 + quad;            // named barrier of the four warps of this quadrant
+    constexpr int HC = D / 4;                 // columns per group
+    constexpr int HU = HC / 8;                // 16-B units per group of a row
     bool ok = true;
     int changes = 0;
     auto epilogue = [&](int j) -> bool {
@@ -491,12 +504,15 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       const int tok = (t % geo.tph) * lin::kLinTok + row;
       if (!mbar_wait(&acc_full[ab], (j >> 1) & 1, abort_flag)) return false;
       tc_fence_after();
-      uint32_t x0[32], x1[32];
-      tmem_ld32(tm + ab * 128 + lane_addr + half * HC, x0);
-      if (HC == 64) tmem_ld32(tm + ab * 128 + lane_addr + half * HC + 32, x1);
-      tmem_wait_ld();
-      reg_fence(x0);
-      if (HC == 64) reg_fence(x1);
+      uint32_t x0[32];
+      if (HC == 32) {
+        tmem_ld32_wait(tm + ab * 128 + lane_addr + half * HC, x0);
+      } else {
+        uint32_t r16[16];
+        tmem_ld16_wait(tm + ab * 128 + lane_addr + half * HC, r16);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x0[e] = r16[e];
+      }
       // phi(q) . z over this half's features, from the phi(Q) tile in shared memory
       const uint8_t* qrow = smem + L::OFF_Q + s * L::T_BYTES;
       float dz = 0.f;
@@ -511,10 +527,10 @@ __global__ void __launch_bounds__(kOutThreads, 1)
           dz = fmaf(__uint_as_float(wv[e] & 0xFFFF0000u), zsm[uu * 8 + 2 * e + 1], dz);
         }
       }
-      float* rj = red + (j & 1) * 2 * 128;
+      float* rj = red + (j & 1) * 4 * 128;
       rj[half * 128 + row] = dz;
-      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
-      const float inv = 1.f / (dz + rj[(half ^ 1) * 128 + row]);
+      asm volatile("bar.sync %0, 128;" ::"r"(quad_bar) : "memory");
+      const float inv = 1.f / ((rj[row] + rj[128 + row]) + (rj[256 + row] + rj[384 + row]));
       if (tok < N) {
         const uint8_t* osrow = smem + L::OFF_OS + s * L::T_BYTES;
         uint16_t* orow = o + (static_cast<long long>(bh) * N + tok) * D + half * HC;
@@ -524,10 +540,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
           const int c = j2 * 8;               // column within this half
           float l[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint32_t bits = (c + e) < 32 ? x0[c + e] : x1[c + e - 32];
-            l[e] = __uint_as_float(bits) * inv;
-          }
+          for (int e = 0; e < 8; ++e) l[e] = __uint_as_float(x0[c + e]) * inv;
           uint32_t pk[4];
           if (blend) {
             const uint4 w = *reinterpret_cast<const uint4*>(osrow + (uu >> 3) * L::T_CHUNK + row * 128 + (((uu & 7) ^ (row & 7)) << 4));
