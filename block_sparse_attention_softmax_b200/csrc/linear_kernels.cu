@@ -85,10 +85,8 @@ struct OutLayout {
   static constexpr uint32_t OFF_B = 0;
   static constexpr uint32_t OFF_Q = 2 * B_BYTES;
   static constexpr uint32_t OFF_OS = OFF_Q + NSTG * T_BYTES;
-  static constexpr uint32_t OFF_Z = OFF_OS + NSTG * T_BYTES;  // z of the current head, fp32
-  static constexpr uint32_t OFF_ALPHA = OFF_Z + D * 4;         // alpha of the current head
-  static constexpr uint32_t OFF_RED = OFF_ALPHA + D * 4;       // [2 parity][4 groups][128 rows]
-  static constexpr uint32_t OFF_BAR = OFF_RED + 8 * 128 * 4;
+  static constexpr uint32_t OFF_DEN = OFF_OS + NSTG * T_BYTES;  // [NSTG][4 parts][128 rows] fp32
+  static constexpr uint32_t OFF_BAR = OFF_DEN + NSTG * 4 * 128 * 4;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
 };
 
@@ -344,19 +342,19 @@ __global__ void linear_reduce_kernel(const float* __restrict__ part, lin::StateG
 
 // ---------------------------------------------------------------- output + blend
 // Persistent over the same head-major tile list as the state kernel. Per tile
-// of 128 tokens: TMA brings Q (and O_s when blending) into a 2-stage ring; the
-// math warps apply phi to Q in place; one thread issues
-// D[t, :] = phi(Q)[t, :] S_hi + phi(Q)[t, :] S_lo (tcgen05, TMEM accumulator,
-// double buffered); the math warps then divide by phi(q_t) . z (CUDA cores,
-// from the phi(Q) tile still in shared memory), blend with O_s and store O.
+// of 128 tokens: one warp loads Q and another O_s by TMA into 2-stage rings;
+// the math warps apply phi to Q in place and, four threads per token, form the
+// denominator phi(q_t) . z; one thread issues D[t, :] = phi(Q)[t, :] S_hi +
+// phi(Q)[t, :] S_lo (tcgen05, TMEM accumulator, double buffered), which also
+// frees the Q stage; the math warps then divide, blend with O_s and store O.
 // The four warps that share TMEM lane quadrant w % 4 split the d columns.
 constexpr int kOutMathWarps = 16;
-constexpr int kOutThreads = 64 + 32 * kOutMathWarps;
+constexpr int kOsWarp = 2 + kOutMathWarps;
+constexpr int kOutThreads = 32 * (kOsWarp + 1);
 
 template <int D>
 __device__ __forceinline__ void build_head_operand(uint8_t* smem, const float* __restrict__ kv_state,
-                                                   const float* __restrict__ ksum, const float* __restrict__ alpha,
-                                                   int bh, int h, int tid, int nthreads) {
+                                                   int bh, int tid, int nthreads) {
   using L = lin::OutLayout<D>;
   // S as bf16 hi + lo, MN-major with 128-B swizzle: element (row c, column e)
   // sits in chunk e/64, row c, 16-B unit ((e % 64) / 8) ^ (c % 8).
@@ -379,12 +377,6 @@ __device__ __forceinline__ void build_head_operand(uint8_t* smem, const float* _
     *reinterpret_cast<uint4*>(smem + L::OFF_B + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     *reinterpret_cast<uint4*>(smem + L::OFF_B + L::B_BYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
-  float* zsm = reinterpret_cast<float*>(smem + L::OFF_Z);
-  float* al = reinterpret_cast<float*>(smem + L::OFF_ALPHA);
-  for (int e = tid; e < D; e += nthreads) {
-    zsm[e] = ksum[static_cast<long long>(bh) * D + e];
-    al[e] = alpha ? alpha[static_cast<long long>(h) * D + e] : 0.f;
-  }
   fence_proxy_async_smem();
 }
 
@@ -399,17 +391,17 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = lin::align1k(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint64_t* st_full = bars;                 // [NS] Q (+ O_s) landed
-  uint64_t* phi_done = bars + NS;           // [NS] phi applied (math warps)
-  uint64_t* st_empty = bars + 2 * NS;       // [NS] tile finished (math warps)
-  uint64_t* acc_full = bars + 3 * NS;       // [2]
+  uint64_t* q_full = bars;                  // [NS] Q landed
+  uint64_t* q_empty = bars + NS;            // [NS] MMA on that Q completed
+  uint64_t* os_full = bars + 2 * NS;        // [NS] O_s landed
+  uint64_t* os_empty = bars + 3 * NS;       // [NS] epilogue done (math warps)
+  uint64_t* phi_done = bars + 4 * NS;       // [NS] phi and denominators ready (math warps)
+  uint64_t* acc_full = bars + 5 * NS;       // [2]
   uint64_t* acc_empty = acc_full + 2;       // [2] (math warps)
   uint64_t* b_ready = acc_empty + 2;        // operand of a new head built (math warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(b_ready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const float* zsm = reinterpret_cast<const float*>(smem + L::OFF_Z);
-  const float* al = reinterpret_cast<const float*>(smem + L::OFF_ALPHA);
-  float* red = reinterpret_cast<float*>(smem + L::OFF_RED);
+  float* den = reinterpret_cast<float*>(smem + L::OFF_DEN);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * geo.tpc;
@@ -419,9 +411,11 @@ __global__ void __launch_bounds__(kOutThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&st_full[s], 1);
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&os_full[s], 1);
+      mbar_init(&os_empty[s], kOutMathWarps);
       mbar_init(&phi_done[s], kOutMathWarps);
-      mbar_init(&st_empty[s], kOutMathWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -431,10 +425,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  {
-    const int bh0 = t0 / geo.tph;
-    build_head_operand<D>(smem, kv_state, ksum, alpha, bh0, bh0 % H, threadIdx.x, blockDim.x);
-  }
+  build_head_operand<D>(smem, kv_state, t0 / geo.tph, threadIdx.x, blockDim.x);
   if (warp == 1) {
     tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
@@ -444,25 +435,28 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   tc_fence_after();
   const uint32_t tm = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      if (blend) tma_prefetch_desc(&tmOs);
+  if (warp == 0 || warp == kOsWarp) {
+    // ------------------------------------------------------------ producers
+    const bool is_q = warp == 0;
+    if (lane == 0 && (is_q || blend)) {
+      const CUtensorMap* map = is_q ? &tmQ : &tmOs;
+      tma_prefetch_desc(map);
+      uint64_t* fullb = is_q ? q_full : os_full;
+      uint64_t* emptyb = is_q ? q_empty : os_empty;
+      const uint32_t base = is_q ? L::OFF_Q : L::OFF_OS;
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % NS;
-        if (!mbar_wait(&st_empty[s], ((i / NS) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&st_full[s], (blend ? 2u : 1u) * L::T_BYTES);
+        if (!mbar_wait(&emptyb[s], ((i / NS) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&fullb[s], L::T_BYTES);
         const int t = t0 + i;
         const int row = (t % geo.tph) * lin::kLinTok, bh = t / geo.tph;
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(smem + L::OFF_Q + s * L::T_BYTES + c * L::T_CHUNK, &tmQ, &st_full[s], c * 64, row, bh);
-          if (blend)
-            tma_load_3d(smem + L::OFF_OS + s * L::T_BYTES + c * L::T_CHUNK, &tmOs, &st_full[s], c * 64, row, bh);
-        }
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + base + s * L::T_BYTES + c * L::T_CHUNK, map, &fullb[s], c * 64, row, bh);
       }
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, D, false, true);
       const uint32_t bhi = smem_u32(smem + L::OFF_B), blo = bhi + L::B_BYTES;
@@ -485,16 +479,19 @@ __global__ void __launch_bounds__(kOutThreads, 1)
           umma_ss(tm + ab * 128, a, sw128_desc(blo + kk * 2048u, L::B_CHUNK, 1024), idesc, 1u);
         }
         tc_commit(&acc_full[ab]);
+        tc_commit(&q_empty[s]);
       }
     }
   } else {
-    const int mt = threadIdx.x - 64;
-    const int quad = warp & 3, half = (warp - 2) >> 2;   // half: column group 0..3
+    // ------------------------------------------------------------ math warps
+    const int mt = threadIdx.x - 64;          // 0 .. 511
+    const int quad = warp & 3, grp = (warp - 2) >> 2;   // column group 0..3 of this lane quadrant
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    const int quad_bar = 1 + quad;            // named barrier of the four warps of this quadrant
-    constexpr int HC = D / 4;                 // columns per group
+    constexpr int HC = D / 4;                 // output columns per group
     constexpr int HU = HC / 8;                // 16-B units per group of a row
+    // transform mapping: token trow, 16-B units [tpart * HU, +HU) of its d range
+    const int trow = mt >> 2, tpart = mt & 3;
     bool ok = true;
     int changes = 0;
     auto epilogue = [&](int j) -> bool {
@@ -503,53 +500,41 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       const int bh = t / geo.tph;
       const int tok = (t % geo.tph) * lin::kLinTok + row;
       if (!mbar_wait(&acc_full[ab], (j >> 1) & 1, abort_flag)) return false;
+      if (!mbar_wait(&phi_done[s], (j / NS) & 1, abort_flag)) return false;   // denominators visible
+      if (blend && !mbar_wait(&os_full[s], (j / NS) & 1, abort_flag)) return false;
       tc_fence_after();
       uint32_t x0[32];
       if (HC == 32) {
-        tmem_ld32_wait(tm + ab * 128 + lane_addr + half * HC, x0);
+        tmem_ld32_wait(tm + ab * 128 + lane_addr + grp * HC, x0);
       } else {
         uint32_t r16[16];
-        tmem_ld16_wait(tm + ab * 128 + lane_addr + half * HC, r16);
+        tmem_ld16_wait(tm + ab * 128 + lane_addr + grp * HC, r16);
 #pragma unroll
         for (int e = 0; e < 16; ++e) x0[e] = r16[e];
       }
-      // phi(q) . z over this half's features, from the phi(Q) tile in shared memory
-      const uint8_t* qrow = smem + L::OFF_Q + s * L::T_BYTES;
-      float dz = 0.f;
-#pragma unroll
-      for (int j2 = 0; j2 < HU; ++j2) {
-        const int uu = half * HU + j2;        // unit along d
-        const uint4 w = *reinterpret_cast<const uint4*>(qrow + (uu >> 3) * L::T_CHUNK + row * 128 + (((uu & 7) ^ (row & 7)) << 4));
-        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          dz = fmaf(__uint_as_float(wv[e] << 16), zsm[uu * 8 + 2 * e], dz);
-          dz = fmaf(__uint_as_float(wv[e] & 0xFFFF0000u), zsm[uu * 8 + 2 * e + 1], dz);
-        }
-      }
-      float* rj = red + (j & 1) * 4 * 128;
-      rj[half * 128 + row] = dz;
-      asm volatile("bar.sync %0, 128;" ::"r"(quad_bar) : "memory");
-      const float inv = 1.f / ((rj[row] + rj[128 + row]) + (rj[256 + row] + rj[384 + row]));
+      const float* dj = den + s * 4 * 128;
+      const float inv = 1.f / ((dj[row] + dj[128 + row]) + (dj[256 + row] + dj[384 + row]));
       if (tok < N) {
         const uint8_t* osrow = smem + L::OFF_OS + s * L::T_BYTES;
-        uint16_t* orow = o + (static_cast<long long>(bh) * N + tok) * D + half * HC;
+        const float* al = alpha + static_cast<long long>(bh % H) * D;
+        uint16_t* orow = o + (static_cast<long long>(bh) * N + tok) * D + grp * HC;
 #pragma unroll
         for (int j2 = 0; j2 < HU; ++j2) {
-          const int uu = half * HU + j2;
-          const int c = j2 * 8;               // column within this half
+          const int uu = grp * HU + j2;
           float l[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) l[e] = __uint_as_float(x0[c + e]) * inv;
+          for (int e = 0; e < 8; ++e) l[e] = __uint_as_float(x0[j2 * 8 + e]) * inv;
           uint32_t pk[4];
           if (blend) {
             const uint4 w = *reinterpret_cast<const uint4*>(osrow + (uu >> 3) * L::T_CHUNK + row * 128 + (((uu & 7) ^ (row & 7)) << 4));
+            const float4 a0 = __ldg(reinterpret_cast<const float4*>(al + uu * 8));
+            const float4 a1 = __ldg(reinterpret_cast<const float4*>(al + uu * 8 + 4));
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float a0 = al[uu * 8 + 2 * e], a1 = al[uu * 8 + 2 * e + 1];
               const float s0 = __uint_as_float(wv[e] << 16), s1 = __uint_as_float(wv[e] & 0xFFFF0000u);
-              pk[e] = pack_bf16x2(fmaf(a0, s0 - l[2 * e], l[2 * e]), fmaf(a1, s1 - l[2 * e + 1], l[2 * e + 1]));
+              pk[e] = pack_bf16x2(fmaf(av[2 * e], s0 - l[2 * e], l[2 * e]), fmaf(av[2 * e + 1], s1 - l[2 * e + 1], l[2 * e + 1]));
             }
           } else {
 #pragma unroll
@@ -562,24 +547,41 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&acc_empty[ab]);
-        mbar_arrive(&st_empty[s]);
+        mbar_arrive(&os_empty[s]);
       }
       return true;
     };
     for (int i = 0; ok && i < n_tiles; ++i) {
       const int s = i % NS;
       const int t = t0 + i;
-      if (!(ok = mbar_wait(&st_full[s], (i / NS) & 1, abort_flag))) break;
-      // phi in place: elementwise, so the swizzled layout does not matter
-      uint4* qt = reinterpret_cast<uint4*>(smem + L::OFF_Q + s * L::T_BYTES);
-#pragma unroll 4
-      for (int u = mt; u < static_cast<int>(L::T_BYTES / 16); u += 32 * kOutMathWarps) {
-        uint4 w = qt[u];
-        uint32_t* x = reinterpret_cast<uint32_t*>(&w);
+      if (!(ok = mbar_wait(&q_full[s], (i / NS) & 1, abort_flag))) break;
+      // the denominator slot of stage s is free once every warp has finished
+      // the epilogue of tile i - NS
+      if (i >= NS && !(ok = mbar_wait(&os_empty[s], ((i / NS) & 1) ^ 1, abort_flag))) break;
+      // phi(Q) in place and the partial denominator of token trow
+      {
+        const float* zg = ksum + static_cast<long long>(t / geo.tph) * D;
+        uint8_t* qt = smem + L::OFF_Q + s * L::T_BYTES;
+        float dz = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          x[e] = pack_bf16x2(lin::phi_f(__uint_as_float(x[e] << 16)), lin::phi_f(__uint_as_float(x[e] & 0xFFFF0000u)));
-        qt[u] = w;
+        for (int j2 = 0; j2 < HU; ++j2) {
+          const int uu = tpart * HU + j2;
+          uint4* p = reinterpret_cast<uint4*>(qt + (uu >> 3) * L::T_CHUNK + trow * 128 + (((uu & 7) ^ (trow & 7)) << 4));
+          uint4 w = *p;
+          uint32_t* x = reinterpret_cast<uint32_t*>(&w);
+          const float4 z0 = __ldg(reinterpret_cast<const float4*>(zg + uu * 8));
+          const float4 z1 = __ldg(reinterpret_cast<const float4*>(zg + uu * 8 + 4));
+          const float zv[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t pk = pack_bf16x2(lin::phi_f(__uint_as_float(x[e] << 16)), lin::phi_f(__uint_as_float(x[e] & 0xFFFF0000u)));
+            x[e] = pk;
+            dz = fmaf(__uint_as_float(pk << 16), zv[2 * e], dz);
+            dz = fmaf(__uint_as_float(pk & 0xFFFF0000u), zv[2 * e + 1], dz);
+          }
+          *p = w;
+        }
+        den[s * 4 * 128 + tpart * 128 + trow] = dz;
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -588,9 +590,8 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         if (!(ok = epilogue(i - 1))) break;
         if (t / geo.tph != (t - 1) / geo.tph) {
           // every MMA of the previous head has completed (its last accumulator
-          // was just read): rebuild the operand, z and alpha for this head
-          const int bh = t / geo.tph;
-          build_head_operand<D>(smem, kv_state, ksum, alpha, bh, bh % H, mt, 32 * kOutMathWarps);
+          // was just read): rebuild the operand for this head
+          build_head_operand<D>(smem, kv_state, t / geo.tph, mt, 32 * kOutMathWarps);
           __syncwarp();
           if (lane == 0) mbar_arrive(b_ready);
           if (!(ok = mbar_wait(b_ready, changes & 1, abort_flag))) break;
