@@ -35,6 +35,35 @@ DEFAULT_WORKLOAD = "wan14b_720p"
 METRIC = "sparse_attn_effective_tflops"
 
 
+# DRAM traffic of sparse_attn_kernel from one `ncu --set full` capture
+# (profiles/sparse_attn_kernel_wan13b_480p.md), taken on a smaller workload and
+# scaled to the benchmarked one by B*H*N*d (the kernel's DRAM traffic is Q, K, V
+# and O sized). `sources_sha` pins the kernel sources the counters belong to:
+# once they change, traffic is reported as null until a new capture is made.
+ATTN_TRAFFIC_CAPTURE = {
+    "workload": "wan13b_480p", "dram_bytes_read": 302483968, "dram_bytes_write": 82595072,
+    "sources_sha": "84ace7c820a9059b",
+    "sources": ("attn_kernel.cu", "sa_device.cuh", "sa_internal.h"),
+}
+
+
+def attn_traffic(wl):
+    import hashlib
+    cap = ATTN_TRAFFIC_CAPTURE
+    h = hashlib.sha256()
+    try:
+        for f in cap["sources"]:
+            with open(os.path.join(ROOT, "block_sparse_attention_softmax_b200", "csrc", f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    if h.hexdigest()[:16] != cap["sources_sha"]:
+        return None
+    ref = WORKLOADS[cap["workload"]]
+    scale = (wl.B * wl.H * wl.N * wl.d) / (ref.B * ref.H * ref.N * ref.d)
+    return round((cap["dram_bytes_read"] + cap["dram_bytes_write"]) * scale)
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -65,31 +94,104 @@ def executed_flops(wl, kv_idx, kv_cnt):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, board power and clock-event reasons sampled every 10 ms during
+    the timed region, through NVML read-only queries (nvidia-smi at 200 ms if
+    NVML is unavailable). Nothing is set on the GPU."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
-        self.index, self.proc, self.lines = index, None, []
+    def __init__(self, local, period_s=0.01):
+        self.local, self.period = local, period_s
+        self.samples = []          # (sm_mhz, power_w, set of reason names)
+        self.max_mhz = None
+        self.nvml = None
+        self.proc = None
+        self.stop = threading.Event()
+        self.source = None
+
+    def _nvml_handle(self, nv):
+        props = torch.cuda.get_device_properties(self.local)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            dom = getattr(props, "pci_domain_id", 0)
+            devn = getattr(props, "pci_device_id", 0)
+            try:
+                return nv.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{devn:02x}.0")
+            except Exception:
+                pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = int(vis.split(",")[self.local]) if vis and vis.split(",")[0].isdigit() else self.local
+        return nv.nvmlDeviceGetHandleByIndex(idx)
+
+    def _nvml_sample(self):
+        nv, h = self.nvml, self.handle
+        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+        try:
+            pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+        except Exception:
+            pw = None
+        bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        return sm, pw, {n for n, c in self.REASONS if bits & getattr(nv, c)}
+
+    def _poll(self):
+        while not self.stop.is_set():
+            try:
+                self.samples.append(self._nvml_sample())
+            except Exception:
+                return
+            self.stop.wait(self.period)
+
+    def _read_smi(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm, self.max_mhz = float(parts[0]), float(parts[1])
+                pw = float(parts[2])
+            except ValueError:
+                continue
+            names = [n for n, _ in self.REASONS]
+            self.samples.append((sm, pw, {n for n, v in zip(names, parts[4:8]) if v.lower() == "active"}))
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nvml = nv
+            self.handle = self._nvml_handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM))
+            self._nvml_sample()          # first query paid before the timed region
+            self.source = "nvml 10 ms"
+            self.t = threading.Thread(target=self._poll, daemon=True)
             self.t.start()
         except Exception:
-            self.proc = None
+            self.nvml = None
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.local}", f"--query-gpu={self.SMI_FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "200"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.t = threading.Thread(target=self._read_smi, daemon=True)
+                self.t.start()
+                self.source = "nvidia-smi 200 ms"
+            except Exception:
+                self.proc = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *exc):
+        self.stop.set()
+        if self.nvml is not None:
+            self.t.join(timeout=5)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc:
             self.proc.terminate()
             try:
@@ -98,24 +200,15 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": self.source}
+        sm = [x[0] for x in self.samples]
+        pw = [x[1] for x in self.samples if x[1] is not None]
+        reasons = sorted(set().union(*[x[2] for x in self.samples]))
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": self.max_mhz,
+                "power_w_median": round(statistics.median(pw), 1) if pw else None,
+                "reasons": reasons, "samples": len(sm), "source": self.source}
 
 
 def dist_setup(n_gpus):
@@ -251,7 +344,9 @@ def run_ours(args, wl, rank, world, local):
         "density": round(density, 5), "executed_tflop_per_call": round(ex_flops / 1e12, 4),
         "roofline": {"kernel": "sparse_attn_kernel<128>", "bound": "tensor", "achieved": round(achieved, 1),
                      "peak": bf16, "unit": "TFLOP/s", "frac": round(achieved / bf16, 4),
-                     "peak_source": f"{src} bf16 burst", "traffic": None},
+                     "peak_source": f"{src} bf16 burst", "traffic": attn_traffic(wl),
+                     "traffic_unit": "bytes per launch",
+                     "traffic_note": "ncu dram read+write of a smaller capture, scaled by B*H*N*d"},
         "e2e": e2e, "gpu_launches": args.steps * launches_per_step,
         "clocks": clk.summary(),
     }

@@ -47,6 +47,11 @@ constexpr int kSoftWarps = 8;
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
 constexpr int kSBufs = 3;
+// Column pairs c (of 32 per thread and tile) with bit (c % 8) set take the
+// FMA-pipe exponential instead of MUFU ex2. Measured on B200 the softmax is
+// bound by issue slots and latency rather than by the MUFU pipe, and the
+// 10-instruction polynomial costs more than it relieves, so none do.
+constexpr uint32_t kPolyPairs = 0x00u;
 constexpr int kVWarp = 2 + kSoftWarps;               // warp index of the V producer
 constexpr int kThreads = 32 * (kVWarp + 1);
 
@@ -373,13 +378,16 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           for (int c = 0; c < 64; ++c)
             if (c >= valid) x[c] = -INFINITY;
         }
+        // row max of this half: eight chains of 3-input max
         float mx8[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) mx8[j] = x[j];
-#pragma unroll
-        for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
-        float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int j = 0; j < 8; ++j) {
+          mx8[j] = fmax3(x[j], x[8 + j], x[16 + j]);
+          mx8[j] = fmax3(mx8[j], x[24 + j], x[32 + j]);
+          mx8[j] = fmax3(mx8[j], x[40 + j], x[48 + j]);
+          mx8[j] = fmaxf(mx8[j], x[56 + j]);
+        }
+        float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         float* rm = red_max + (g & 1) * 2 * kBM;
         rm[half * kBM + row] = mx;
         asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
@@ -391,26 +399,31 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           m = m_tile;
           l *= corr;
         }
-        // A quarter of the exponentials run on the FMA pipe so the MUFU unit
-        // is not the only path; partial sums in 4 chains.
-        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+        // P = 2^(S * scale * log2(e) - m), two columns per packed instruction.
+        const uint64_t sl2x2 = f2_make(sl2, sl2);
+        const uint64_t negm2 = f2_make(-m, -m);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // packed (+0, +0)
         uint32_t p[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float a0 = fmaf(x[2 * c], sl2, -m);
-          const float a1 = fmaf(x[2 * c + 1], sl2, -m);
+          const uint64_t a2 = ffma2(f2_make(x[2 * c], x[2 * c + 1]), sl2x2, negm2);
           float e0, e1;
-          if ((c & 3) == 3) {
-            e0 = exp2_poly(a0);
-            e1 = exp2_poly(a1);
+          if ((kPolyPairs >> (c & 7)) & 1) {
+            exp2_poly2(a2, e0, e1);
           } else {
+            float a0, a1;
+            f2_split(a2, a0, a1);
             e0 = fast_exp2(a0);
             e1 = fast_exp2(a1);
           }
-          sum4[c & 3] += e0 + e1;
+          acc[c & 3] = fadd2(acc[c & 3], f2_make(e0, e1));
           p[c] = pack_bf16x2(e0, e1);
         }
-        l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        {
+          float s0, s1;
+          f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), s0, s1);
+          l += s0 + s1;
+        }
         tmem_st32(tm + lane_addr + tm_s(b) + half * 32, p);
         if (t > 0 && __any_sync(0xFFFFFFFFu, corr != 1.f)) {
           // O is complete up to the previous tile once its P V has landed

@@ -268,17 +268,60 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// 2^x on the FMA pipe, for x <= 127: x = i + f with i = floor(x), f in [0, 1);
-// 2^f by a cubic fitted on [0, 1) for minimum maximum relative error (Lawson's
-// iteratively reweighted least squares; max relative error 7.7e-5), and 2^i
-// added to the exponent field. Inputs below -126 return a value below 2^-125
-// (or 0), which is negligible wherever it is used.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float xi = floorf(x);
-  const float f = x - xi;
-  const float p = fmaf(fmaf(fmaf(0.07809657f, f, 0.22596510f), f, 0.69586831f), f, 0.99992359f);
-  return __int_as_float(__float_as_int(p) + (static_cast<int>(xi) << 23));
+// ---------------------------------------------------------------- packed fp32 pairs
+// sm_100 executes fma/add on two fp32 lanes held in one 64-bit register pair
+// (one instruction for both), which halves the FMA-pipe issue of elementwise
+// softmax work.
+__device__ __forceinline__ uint64_t f2_make(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair, on the FMA and integer pipes only (no MUFU, no float/int
+// conversion instruction), for x <= 127. x is clamped below at -126; adding
+// 1.5 * 2^23 rounds it to the nearest integer n, which then sits in the low
+// mantissa bits of the sum; f = x - n lies in [-0.5, 0.5]. 2^f comes from a
+// cubic fitted on [-0.5, 0.5] for minimum maximum relative error (Lawson's
+// iteratively reweighted least squares; max relative error 7.5e-5 evaluated
+// in fp32), and n is added to its exponent field: shifting the sum's bit
+// pattern left by 23 leaves exactly n << 23, since the pattern of 1.5 * 2^23
+// has its low 9 bits clear. Inputs at or below -126 give a value of at most
+// 2^-125 (possibly subnormal), negligible wherever it is used.
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& e0, float& e1) {
+  float x0, x1;
+  f2_split(x2, x0, x1);
+  const uint64_t xc = f2_make(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t magic = f2_make(12582912.f, 12582912.f);
+  const uint64_t j = fadd2(xc, magic);                          // n in the low bits
+  const uint64_t n = fadd2(j, f2_make(-12582912.f, -12582912.f));
+  const uint64_t f = ffma2(n, f2_make(-1.f, -1.f), xc);          // x - n, exact
+  uint64_t p = ffma2(f2_make(0.05517168f, 0.05517168f), f, f2_make(0.24261117f, 0.24261117f));
+  p = ffma2(p, f, f2_make(0.69326097f, 0.69326097f));
+  p = ffma2(p, f, f2_make(0.99992806f, 0.99992806f));
+  float p0, p1, j0, j1;
+  f2_split(p, p0, p1);
+  f2_split(j, j0, j1);
+  e0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(j0) << 23));
+  e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(j1) << 23));
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
