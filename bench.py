@@ -41,8 +41,8 @@ METRIC = "sparse_attn_effective_tflops"
 # and O sized). `sources_sha` pins the kernel sources the counters belong to:
 # once they change, traffic is reported as null until a new capture is made.
 ATTN_TRAFFIC_CAPTURE = {
-    "workload": "wan13b_480p", "dram_bytes_read": 302483968, "dram_bytes_write": 82595072,
-    "sources_sha": "84ace7c820a9059b",
+    "workload": "wan13b_480p", "dram_bytes_read": 302419968, "dram_bytes_write": 82997760,
+    "sources_sha": "a67b05317a9dd7d0",
     "sources": ("attn_kernel.cu", "sa_device.cuh", "sa_internal.h"),
 }
 

@@ -54,10 +54,11 @@ constexpr int kKStages = 3;
 constexpr int kVStages = 2;
 constexpr int kSBufs = 3;
 // Column pairs c (of 32 per thread and tile) with bit (c % 8) set take the
-// FMA-pipe exponential instead of MUFU ex2. Measured on B200 the softmax is
-// bound by issue slots and latency rather than by the MUFU pipe, and the
-// 10-instruction polynomial costs more than it relieves, so none do.
-constexpr uint32_t kPolyPairs = 0x00u;
+// FMA-pipe exponential instead of MUFU ex2: one pair in four. Measured on B200
+// with two MMA issuers, where the softmax sets the pace: fastest of 0, 1, 2, 3
+// and 4 pairs in 8 (the polynomial costs 10 issue slots per pair, MUFU costs
+// pipe time), both in short runs and under the power cap.
+constexpr uint32_t kPolyPairs = 0x88u;
 constexpr int kVWarp = 2 + kSoftWarps;               // warp index of the V producer
 constexpr int kPVWarp = kVWarp + 1;                  // warp index of the P V issuer
 constexpr int kThreads = 32 * (kPVWarp + 1);
