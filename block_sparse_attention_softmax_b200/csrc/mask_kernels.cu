@@ -2,14 +2,16 @@
 // selection (pages: "SLA2" 提案手法 ① mean pooling of Q and K;
 // "SpargeAttention2" §2(1) hybrid Top-k + Top-p masking per attention row).
 //
-// Three kernels, all bound by memory or by a small amount of ALU work:
-//   pool_kernel    Q, K [BH, N, d] bf16  ->  block means [BH, nb, d] fp32
-//   score_kernel   means -> s[bh, qb, kb] = scale * <Qbar, Kbar> (fp32 partial
-//                  sums of 32 products, combined in fp64, rounded once)
-//   select_kernel  one query-block row per warp: radix select of the K_sel-th
-//                  largest score (Top-k), a probability-mass search for the
-//                  Top-p cut when Top-k alone does not reach p, and the
-//                  ascending compacted index list.
+//   pool_kernel      Q, K [BH, N, d] bf16 -> block means [BH, nb, d] fp32, and
+//                    the same means as four signed 7-bit slices per element
+//                    with a per-row power-of-two exponent
+//   score_i8_kernel  slices -> s[bh, qb, kb] = scale * <Qbar, Kbar> on the
+//                    int8 tensor cores (exact s32 slice products, combined in
+//                    int64, scaled in fp64, rounded once to fp32)
+//   select_kernel    one query-block row per warp: radix select of the K_sel-th
+//                    largest score (Top-k), a probability-mass search for the
+//                    Top-p cut when Top-k alone does not reach p, and the
+//                    ascending compacted index list.
 #include "sa_internal.h"
 
 namespace sa {
@@ -17,12 +19,21 @@ namespace sa {
 // ---------------------------------------------------------------- pooling
 // One warp per token block. Each lane loads 16 B (8 bf16) per row it visits;
 // d/8 lanes cover one row, so a warp reads 32*16 B per step.
+//
+// With `sl` set, each block mean row x (fp32) is also written as four signed
+// 7-bit slices for the integer tensor-core scores: with E the exponent for
+// which max|x| < 2^E, y = x * 2^-E lies in (-1, 1) and
+//   y = sum_{s=1..4} a_s 2^(-7 s) + r,  a_s = trunc of the running remainder
+//   times 128, |a_s| <= 127, 0 <= |r| < 2^-28,
+// computed exactly in fp32 (scaling by 128 and subtracting the integer part
+// are exact). Row layout: slice s at bytes [s * d, (s + 1) * d); E in `ex`.
+
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k, int BH,
                                                    int N, int bq, int bk, int nqb, int nkb,
                                                    float* __restrict__ q_pool,
-                                                   float* __restrict__ k_pool) {
+                                                   float* __restrict__ k_pool, SliceOut sl) {
   constexpr int LPR = D / 8;        // lanes per row
   constexpr int RPI = 32 / LPR;     // rows per warp step
   const int lane = threadIdx.x & 31;
@@ -74,92 +85,190 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], off);
   }
+  const float fc = static_cast<float>(cnt);
+  float mean[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mean[i] = __fdiv_rn(acc[i], fc);
   if (r0 == 0) {
-    const float fc = static_cast<float>(cnt);
-    float4 a = make_float4(__fdiv_rn(acc[0], fc), __fdiv_rn(acc[1], fc), __fdiv_rn(acc[2], fc),
-                           __fdiv_rn(acc[3], fc));
-    float4 c = make_float4(__fdiv_rn(acc[4], fc), __fdiv_rn(acc[5], fc), __fdiv_rn(acc[6], fc),
-                           __fdiv_rn(acc[7], fc));
-    reinterpret_cast<float4*>(dst + c8)[0] = a;
-    reinterpret_cast<float4*>(dst + c8)[1] = c;
+    reinterpret_cast<float4*>(dst + c8)[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
+    reinterpret_cast<float4*>(dst + c8)[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
+  }
+  if (sl.q_sl) {
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(mean[i]));
+#pragma unroll
+    for (int off = 1; off < LPR; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    int E = 0;
+    if (mx > 0.f) frexpf(mx, &E);      // mx = m * 2^E with m in [0.5, 1): max|x| < 2^E
+    if (r0 == 0) {
+      int8_t* srow = (is_q ? sl.q_sl : sl.k_sl) + w * (4 * D);
+      float y[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) y[i] = ldexpf(mean[i], -E);
+#pragma unroll
+      for (int sidx = 0; sidx < 4; ++sidx) {
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float t = y[i] * 128.f;
+          const float a = truncf(t);
+          y[i] = t - a;
+          const uint32_t byte = static_cast<uint32_t>(static_cast<int>(a)) & 0xFFu;
+          if (i < 4) lo |= byte << (8 * i);
+          else hi |= byte << (8 * (i - 4));
+        }
+        *reinterpret_cast<uint2*>(srow + sidx * D + c8) = make_uint2(lo, hi);
+      }
+      if (lane == 0) (is_q ? sl.q_ex : sl.k_ex)[w] = E;
+    }
   }
 }
 
-// ---------------------------------------------------------------- scores
-// 64 x 64 tile of one head per CTA; thread (ty, tx) owns a 4 x 4 sub-tile.
-// Products are summed in fp32 over 32 consecutive channels, the 32-channel
-// partial sums in fp64, so the rounding error stays near 1e-7 of the score
-// scale rather than the ~1e-6 of a 128-term fp32 sum.
-constexpr int kScoreTile = 64;
-constexpr int kScorePad = kScoreTile + 4;
+// ---------------------------------------------------------------- scores on the int8 tensor cores
+// The block means arrive as four 7-bit slices per element (see pool_kernel):
+// x = 2^E sum_s a_s 2^(-7 s) up to 2^(E-28). Then
+//   <xq, xk> = 2^(Eq + Ek) sum_{s,t} 2^(-7 (s + t)) <a_s, b_t>,
+// and every <a_s, b_t> (d products of |.| <= 127 values) is exact in the
+// tensor core's s32 accumulator. Pairs are grouped by level L = s + t into
+// four accumulators (L = 2..5; pairs with s + t > 5 weigh at most 2^-42 and
+// are dropped), combined exactly as the int64
+//   v = acc2 2^21 + acc3 2^14 + acc4 2^7 + acc5,
+// and the score is v * 2^(Eq + Ek - 35) * scale, rounded once in fp64 and
+// once to fp32. Its error stays near 1e-7 of the score scale, well inside the
+// 1e-6 band within which the mask comparison treats a cut as a tie.
+//
+// CTA tile: 128 query blocks (M, operand A) x 64 key blocks (N, operand B),
+// both K-major with 128-byte swizzled rows, one TMA box per 128-byte column
+// chunk. Thread 0 loads the tiles and issues the 4 d / 32 * 10 MMAs; the four
+// warps then read their TMEM lane quadrant and write the scores.
+constexpr int kI8TileM = 128;
+constexpr int kI8TileN = 64;
 
 template <int D>
-__global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ q_pool,
-                                                    const float* __restrict__ k_pool, int nqb,
-                                                    int nkb, double scale, float* __restrict__ s,
-                                                    long long s_ld) {
-  extern __shared__ float sm_score[];
-  float* qs = sm_score;                  // [D][kScorePad], transposed
-  float* ks = sm_score + D * kScorePad;  // [D][kScorePad]
+struct I8Layout {
+  static constexpr int ROW = 4 * D;                 // bytes per slice row
+  static constexpr int NCH = ROW / 128;             // 128-byte column chunks
+  static constexpr uint32_t A_CH = kI8TileM * 128;  // bytes of one A chunk
+  static constexpr uint32_t B_CH = kI8TileN * 128;
+  static constexpr uint32_t OFF_A = 0;
+  static constexpr uint32_t OFF_B = OFF_A + NCH * A_CH;
+  static constexpr uint32_t OFF_KEX = OFF_B + NCH * B_CH;
+  static constexpr uint32_t OFF_BAR = OFF_KEX + kI8TileN * 4;
+  static constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) score_i8_kernel(const __grid_constant__ CUtensorMap tmA,
+                                                       const __grid_constant__ CUtensorMap tmB,
+                                                       const int* __restrict__ q_ex,
+                                                       const int* __restrict__ k_ex, int nqb,
+                                                       int nkb, double scale,
+                                                       float* __restrict__ s, long long s_ld) {
+  using L = I8Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  int* kex = reinterpret_cast<int*>(smem + L::OFF_KEX);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);   // [0] tiles landed, [1] MMAs done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.z;
-  const int qb0 = blockIdx.y * kScoreTile;
-  const int kb0 = blockIdx.x * kScoreTile;
-  const float* qp = q_pool + static_cast<long long>(bh) * nqb * D;
-  const float* kp = k_pool + static_cast<long long>(bh) * nkb * D;
-  for (int i = threadIdx.x; i < kScoreTile * (D / 4); i += blockDim.x) {
-    const int r = i / (D / 4);
-    const int c4 = (i % (D / 4)) * 4;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-    if (qb0 + r < nqb) a = *reinterpret_cast<const float4*>(qp + static_cast<long long>(qb0 + r) * D + c4);
-    if (kb0 + r < nkb) b = *reinterpret_cast<const float4*>(kp + static_cast<long long>(kb0 + r) * D + c4);
-    qs[(c4 + 0) * kScorePad + r] = a.x;
-    qs[(c4 + 1) * kScorePad + r] = a.y;
-    qs[(c4 + 2) * kScorePad + r] = a.z;
-    qs[(c4 + 3) * kScorePad + r] = a.w;
-    ks[(c4 + 0) * kScorePad + r] = b.x;
-    ks[(c4 + 1) * kScorePad + r] = b.y;
-    ks[(c4 + 2) * kScorePad + r] = b.z;
-    ks[(c4 + 3) * kScorePad + r] = b.w;
+  const int qb0 = blockIdx.y * kI8TileM;
+  const int kb0 = blockIdx.x * kI8TileN;
+  constexpr uint32_t kCols = 4 * kI8TileN;            // four level accumulators
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
   }
+  if (threadIdx.x < kI8TileN)
+    kex[threadIdx.x] = kb0 + threadIdx.x < nkb ? __ldg(k_ex + static_cast<long long>(bh) * nkb + kb0 + threadIdx.x) : 0;
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
-  double acc64[4][4];
+  tc_fence_after();
+  const uint32_t tm = *tmem_slot;
+
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    mbar_arrive_expect_tx(&bars[0], L::NCH * (L::A_CH + L::B_CH));
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc64[i][j] = 0.0;
-  for (int c0 = 0; c0 < D; c0 += 32) {
-    float acc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll
-    for (int c = c0; c < c0 + 32; ++c) {
-      const float4 a = *reinterpret_cast<const float4*>(qs + c * kScorePad + ty * 4);
-      const float4 b = *reinterpret_cast<const float4*>(ks + c * kScorePad + tx * 4);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-      const float bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    for (int c = 0; c < L::NCH; ++c) {
+      tma_load_3d(smem + L::OFF_A + c * L::A_CH, &tmA, &bars[0], c * 128, qb0, bh);
+      tma_load_3d(smem + L::OFF_B + c * L::B_CH, &tmB, &bars[0], c * 128, kb0, bh);
     }
+    if (mbar_wait(&bars[0], 0, abort_flag)) {
+      tc_fence_after();
+      const uint64_t a0 = sw128_desc(smem_u32(smem + L::OFF_A), 16, 1024);
+      const uint64_t b0 = sw128_desc(smem_u32(smem + L::OFF_B), 16, 1024);
+      constexpr uint32_t idesc = idesc_s8_s32(kI8TileM, kI8TileN);
+      // byte offset of a K step inside the chunked, swizzled tile
+      auto off = [](int byte, uint32_t chunk_bytes) -> uint32_t {
+        return (static_cast<uint32_t>(byte >> 7) * chunk_bytes + static_cast<uint32_t>(byte & 127)) >> 4;
+      };
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int sa = 1; sa <= 4; ++sa)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc64[i][j] += static_cast<double>(acc[i][j]);
+        for (int tb = 1; sa + tb <= 5; ++tb)
+#pragma unroll
+          for (int j = 0; j < D / 32; ++j)
+            umma_i8_ss(tm + (sa + tb - 2) * kI8TileN, a0 + off(D * (sa - 1) + 32 * j, L::A_CH),
+                       b0 + off(D * (tb - 1) + 32 * j, L::B_CH), idesc, (sa == 1 && j == 0) ? 0u : 1u);
+      tc_commit(&bars[1]);
+    }
   }
+  __syncwarp();
+  if (mbar_wait(&bars[1], 0, abort_flag)) {
+    tc_fence_after();
+    const int row = qb0 + warp * 32 + lane;            // TMEM lane = query block
+    const bool rv = row < nqb;
+    const int eq = rv ? __ldg(q_ex + static_cast<long long>(bh) * nqb + row) : 0;
+    float* srow = s + (static_cast<long long>(bh) * nqb + (rv ? row : 0)) * s_ld;
+    const uint32_t la = tm + (static_cast<uint32_t>(warp * 32) << 16);
+#pragma unroll 1
+    for (int c0 = 0; c0 < kI8TileN; c0 += 16) {
+      uint32_t a2[16], a3[16], a4[16], a5[16];
+      tmem_ld16_wait(la + 0 * kI8TileN + c0, a2);
+      tmem_ld16_wait(la + 1 * kI8TileN + c0, a3);
+      tmem_ld16_wait(la + 2 * kI8TileN + c0, a4);
+      tmem_ld16_wait(la + 3 * kI8TileN + c0, a5);
+      float o[16];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int qb = qb0 + ty * 4 + i;
-    if (qb >= nqb) continue;
-    float* row = s + (static_cast<long long>(bh) * nqb + qb) * s_ld;
+      for (int i = 0; i < 16; ++i) {
+        const long long v = (static_cast<long long>(static_cast<int>(a2[i])) << 21) +
+                            (static_cast<long long>(static_cast<int>(a3[i])) << 14) +
+                            (static_cast<long long>(static_cast<int>(a4[i])) << 7) +
+                            static_cast<long long>(static_cast<int>(a5[i]));
+        const int e = eq + kex[c0 + i] - 35;
+        const double p2 = __longlong_as_double(static_cast<long long>(e + 1023) << 52);
+        o[i] = __double2float_rn(static_cast<double>(v) * p2 * scale);
+      }
+      if (rv) {
+        const int kb = kb0 + c0;
+        if (kb + 16 <= nkb) {
+          float4* dst = reinterpret_cast<float4*>(srow + kb);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int kb = kb0 + tx * 4 + j;
-      if (kb < nkb) row[kb] = __double2float_rn(acc64[i][j] * scale);
+          for (int i = 0; i < 4; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (kb + i < nkb) srow[kb + i] = o[i];
+        }
+      }
     }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tm, kCols);
   }
 }
 
@@ -383,6 +492,182 @@ __global__ void __launch_bounds__(kSelWarpsMax * 32) select_kernel(
   }
 }
 
+// ---------------------------------------------------------------- selection, keys in registers
+// The same decisions as select_kernel for rows of at most 32 * KPL key blocks,
+// with each lane holding the keys and weights of elements lane + 32 j in
+// registers (no shared-memory histograms, so nothing serialises on atomics).
+//
+//   Top-k   MSB-first bitwise search for the largest key v with
+//           count(key >= v) >= K_sel. Full passes over the registers run only
+//           until {key >= v} has at most kCandMax members; the remaining bits
+//           are searched on that set, compacted into shared memory.
+//   Top-p   the same search on fp64 mass instead of count.
+// Elements past the row end carry key 0, below every finite score's key, and
+// weight 0, so they are never counted.
+constexpr int kCandMax = 256;
+
+template <int KPL>
+__device__ __forceinline__ int count_ge(const uint32_t (&kr)[KPL], uint32_t c) {
+  int n = 0;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) n += kr[j] >= c ? 1 : 0;
+  return static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, static_cast<unsigned>(n)));
+}
+
+template <int KPL>
+__device__ Cut select_topk_reg(const uint32_t (&kr)[KPL], int k_sel, uint32_t* cand) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t v = 0;
+  int bit = 31;
+  bool small = false;
+  for (; bit >= 0; --bit) {
+    const uint32_t c = v | (1u << bit);
+    const int cnt = count_ge(kr, c);
+    if (cnt >= k_sel) {
+      v = c;
+      if (cnt <= kCandMax) {
+        small = true;
+        --bit;
+        break;
+      }
+    }
+  }
+  if (small) {
+    // every key that can still reach the threshold is >= v
+    int m = 0;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      const bool take = kr[j] >= v;
+      const uint32_t b = __ballot_sync(0xFFFFFFFFu, take);
+      if (take) cand[m + __popc(b & lt)] = kr[j];
+      m += __popc(b);
+    }
+    __syncwarp();
+    constexpr int CPL = kCandMax / 32;
+    uint32_t cr[CPL];
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) cr[i] = lane + 32 * i < m ? cand[lane + 32 * i] : 0u;
+    __syncwarp();
+    for (; bit >= 0; --bit) {
+      const uint32_t c = v | (1u << bit);
+      if (count_ge(cr, c) >= k_sel) v = c;
+    }
+  }
+  const int above = v == 0xFFFFFFFFu ? 0 : count_ge(kr, v + 1u);
+  return Cut{v, above, k_sel - above};
+}
+
+// Smallest m such that the m largest-key weights sum to >= target. Weights
+// are in shared memory, element i at er[i] (lane-strided, conflict-free).
+template <int KPL>
+__device__ Cut select_mass_reg(const uint32_t (&kr)[KPL], const float* er, double target) {
+  const int lane = threadIdx.x & 31;
+  uint32_t v = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t c = v | (1u << bit);
+    double w = 0.0;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j)
+      if (kr[j] >= c) w += static_cast<double>(er[lane + 32 * j]);
+    if (warp_sum_d(w) >= target) v = c;
+  }
+  int above = 0, nties = 0;
+  double w_above = 0.0;
+  float e_tie = 0.f;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) {
+    if (kr[j] > v) {
+      ++above;
+      w_above += static_cast<double>(er[lane + 32 * j]);
+    } else if (kr[j] == v) {
+      ++nties;
+      e_tie = er[lane + 32 * j];
+    }
+  }
+  above = warp_sum_i(above);
+  nties = warp_sum_i(nties);
+  w_above = warp_sum_d(w_above);
+  e_tie = warp_max(e_tie);            // every tie has the same weight
+  int t = 0;
+  double acc = w_above;
+  while (acc < target && t < nties) {
+    acc += static_cast<double>(e_tie);
+    ++t;
+  }
+  if (acc < target) t = nties;
+  if (above + t == 0) t = 1;
+  return Cut{v, above, t};
+}
+
+// One query-block row per warp: the row's keys in registers, its weights in
+// the warp's shared-memory slice er[32 * KPL]; decision and ascending
+// compaction as in select_kernel.
+template <int KPL>
+__device__ __forceinline__ void select_row_reg(const float* __restrict__ srow, int nkb, int k_sel,
+                                               double topp, int* __restrict__ out,
+                                               int* __restrict__ cnt_out, uint8_t* __restrict__ mrow,
+                                               uint32_t* cand, float* er) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t kr[KPL];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) {
+    const int i = lane + 32 * j;
+    const float v = i < nkb ? srow[i] : -INFINITY;
+    kr[j] = i < nkb ? score_key(v) : 0u;
+    er[i] = v;
+    mx = fmaxf(mx, v);
+  }
+  mx = warp_max(mx);
+  double z = 0.0;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) {
+    const int i = lane + 32 * j;
+    const float e = i < nkb ? expf(er[i] - mx) : 0.f;
+    er[i] = e;
+    z += static_cast<double>(e);
+  }
+  z = warp_sum_d(z);
+
+  Cut cut{0u, 0, nkb};                // keep everything (every finite score's key is > 0)
+  if (!(topp >= 1.0 || k_sel >= nkb)) {
+    cut = select_topk_reg(kr, k_sel, cand);
+    const double target = topp * z;
+    double wk = 0.0;
+    int tie_before = 0;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      const bool tie = kr[j] == cut.key;
+      const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
+      const bool keep = kr[j] > cut.key || (tie && tie_before + __popc(tb & lt) < cut.ties);
+      if (keep) wk += static_cast<double>(er[lane + 32 * j]);
+      tie_before += __popc(tb);
+    }
+    wk = warp_sum_d(wk);
+    if (wk < target) {
+      const Cut cp = select_mass_reg(kr, er, target);
+      if (cp.above + cp.ties > k_sel) cut = cp;
+    }
+  }
+  int written = 0, tie_before = 0;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) {
+    const int i = lane + 32 * j;
+    const bool valid = i < nkb;
+    const bool tie = valid && kr[j] == cut.key;
+    const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
+    const bool keep = valid && (kr[j] > cut.key || (tie && tie_before + __popc(tb & lt) < cut.ties));
+    const uint32_t kb = __ballot_sync(0xFFFFFFFFu, keep);
+    if (keep) out[written + __popc(kb & lt)] = i;
+    if (mrow && valid) mrow[i] = keep ? 1 : 0;
+    written += __popc(kb);
+    tie_before += __popc(tb);
+  }
+  if (lane == 0) *cnt_out = written;
+}
+
 // ---------------------------------------------------------------- uint8 mask -> lists
 __global__ void __launch_bounds__(kSelWarpsMax * 32) compact_mask_kernel(
     const uint8_t* __restrict__ mask, int n_rows, int nkb, int* __restrict__ kv_idx,
@@ -407,7 +692,8 @@ __global__ void __launch_bounds__(kSelWarpsMax * 32) compact_mask_kernel(
 
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, int bq, int bk,
-                        float* q_pool, float* k_pool, cudaStream_t st) {
+                        float* q_pool, float* k_pool, cudaStream_t st, const SliceOut* sl) {
+  const SliceOut so = sl ? *sl : SliceOut{nullptr, nullptr, nullptr, nullptr};
   const int nqb = ceil_div(N, bq), nkb = ceil_div(N, bk);
   const long long warps = static_cast<long long>(BH) * (nqb + nkb);
   const long long blocks = (warps * 32 + 255) / 256;
@@ -415,25 +701,31 @@ cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, int 
   const auto* qq = static_cast<const __nv_bfloat16*>(q);
   const auto* kk = static_cast<const __nv_bfloat16*>(k);
   if (d == 128)
-    pool_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(qq, kk, BH, N, bq, bk, nqb, nkb, q_pool, k_pool);
+    pool_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(qq, kk, BH, N, bq, bk, nqb, nkb, q_pool, k_pool, so);
   else
-    pool_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(qq, kk, BH, N, bq, bk, nqb, nkb, q_pool, k_pool);
+    pool_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(qq, kk, BH, N, bq, bk, nqb, nkb, q_pool, k_pool, so);
   return cudaGetLastError();
 }
 
-cudaError_t launch_scores(const float* q_pool, const float* k_pool, int BH, int nqb, int nkb,
-                          int d, double scale, float* s, long long s_ld, cudaStream_t st) {
-  dim3 grid(ceil_div(nkb, kScoreTile), ceil_div(nqb, kScoreTile), BH);
-  if (grid.y > 65535 || grid.z > 65535) return cudaErrorInvalidValue;
-  const size_t smem = static_cast<size_t>(2) * d * kScorePad * sizeof(float);
-  if (d == 128) {
-    cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    score_kernel<128><<<grid, 256, smem, st>>>(q_pool, k_pool, nqb, nkb, scale, s, s_ld);
-  } else {
-    cudaFuncSetAttribute(score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    score_kernel<64><<<grid, 256, smem, st>>>(q_pool, k_pool, nqb, nkb, scale, s, s_ld);
-  }
+template <int D>
+static cudaError_t launch_scores_i8_d(const SliceOut& sl, int BH, int nqb, int nkb, double scale,
+                                      float* s, long long s_ld, cudaStream_t st) {
+  using L = I8Layout<D>;
+  CUtensorMap ma, mb;
+  if (encode_tensor_map_3d_u8(&ma, sl.q_sl, L::ROW, nqb, BH, 128, kI8TileM) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (encode_tensor_map_3d_u8(&mb, sl.k_sl, L::ROW, nkb, BH, 128, kI8TileN) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(score_i8_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid(ceil_div(nkb, kI8TileN), ceil_div(nqb, kI8TileM), BH);
+  score_i8_kernel<D><<<grid, 128, L::SMEM, st>>>(ma, mb, sl.q_ex, sl.k_ex, nqb, nkb, scale, s, s_ld);
   return cudaGetLastError();
+}
+
+cudaError_t launch_scores_i8(const SliceOut& sl, int BH, int nqb, int nkb, int d, double scale,
+                             float* s, long long s_ld, cudaStream_t st) {
+  if (nqb > 65535 * kI8TileM || BH > 65535) return cudaErrorInvalidValue;
+  return d == 128 ? launch_scores_i8_d<128>(sl, BH, nqb, nkb, scale, s, s_ld, st)
+                  : launch_scores_i8_d<64>(sl, BH, nqb, nkb, scale, s, s_ld, st);
 }
 
 cudaError_t launch_select(const float* s, long long s_ld, int n_rows, int nkb, int k_sel,

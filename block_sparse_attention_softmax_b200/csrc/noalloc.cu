@@ -58,7 +58,7 @@ int sa_build_mask_noalloc(const uint16_t* q, const uint16_t* k, int B, int H, in
   if (!(topk_frac > 0.0 && topk_frac <= 1.0)) return fail(SA_ERR_INVALID_ARG, "topk_frac %g outside (0, 1]", topk_frac);
   if (!(topp >= 0.0 && topp <= 1.0)) return fail(SA_ERR_INVALID_ARG, "topp %g outside [0, 1]", topp);
   if (!isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "scale must be finite");
-  const int nkb = (N + bk - 1) / bk, nqb = (N + bq - 1) / bq;
+  const int nkb = (N + bk - 1) / bk;
   if (nkb > kMaxKeyBlocks) return fail(SA_ERR_UNSUPPORTED, "n_kb = %d exceeds %d", nkb, kMaxKeyBlocks);
   const void* ptrs[] = {q, k, kv_idx, kv_cnt, mask_opt};
   for (const void* p : ptrs)
@@ -78,13 +78,10 @@ int sa_build_mask_noalloc(const uint16_t* q, const uint16_t* k, int B, int H, in
   char* ws = static_cast<char*>(scratch);
   float* qp = reinterpret_cast<float*>(ws + w.q_pool);
   float* kp = reinterpret_cast<float*>(ws + w.k_pool);
-  float* s = reinterpret_cast<float*>(ws + w.s);
   const int BH = B * H;
   const int k_sel = static_cast<int>(fmin(static_cast<double>(nkb), fmax(1.0, ceil(topk_frac * nkb - 1e-9))));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_pool(q, k, BH, N, d, bq, bk, qp, kp, st);
-  if (e == cudaSuccess) e = launch_scores(qp, kp, BH, nqb, nkb, d, scale, s, w.s_ld, st);
-  if (e == cudaSuccess) e = launch_select(s, w.s_ld, BH * nqb, nkb, k_sel, topp, kv_idx, kv_cnt, mask_opt, st);
+  cudaError_t e = run_mask_builder(q, k, BH, N, d, bq, bk, k_sel, topp, scale, kv_idx, kv_cnt, mask_opt,
+                                   qp, kp, ws, w, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_build_mask_noalloc");
 }
 

@@ -51,10 +51,12 @@ int check_shape(int B, int H, int N, int d, int bq, int bk) {
 }
 
 struct MaskWs {
-  size_t q_pool, k_pool, s, total;
+  size_t q_pool, k_pool, q_sl, k_sl, q_ex, k_ex, s, total;
   long long s_ld;
 };
 
+// Workspace of the mask builder: pooled means (unless the caller takes them),
+// their int8 slices and exponents, and the fp32 block scores.
 MaskWs mask_ws(int B, int H, int N, int d, int bq, int bk, bool need_q, bool need_k) {
   const long long BH = static_cast<long long>(B) * H;
   const long long nqb = (N + bq - 1) / bq, nkb = (N + bk - 1) / bk;
@@ -65,10 +67,33 @@ MaskWs mask_ws(int B, int H, int N, int d, int bq, int bk, bool need_q, bool nee
   if (need_q) off += round_up(static_cast<size_t>(BH * nqb * d) * 4, 256);
   w.k_pool = off;
   if (need_k) off += round_up(static_cast<size_t>(BH * nkb * d) * 4, 256);
+  w.q_sl = off;
+  off += round_up(static_cast<size_t>(BH * nqb * 4 * d), 256);
+  w.k_sl = off;
+  off += round_up(static_cast<size_t>(BH * nkb * 4 * d), 256);
+  w.q_ex = off;
+  off += round_up(static_cast<size_t>(BH * nqb) * 4, 256);
+  w.k_ex = off;
+  off += round_up(static_cast<size_t>(BH * nkb) * 4, 256);
   w.s = off;
   off += round_up(static_cast<size_t>(BH * nqb) * w.s_ld * 4, 256);
   w.total = off;
   return w;
+}
+
+// The three launches of the mask builder, on carved workspace.
+cudaError_t run_mask_builder(const void* q, const void* k, int BH, int N, int d, int bq, int bk,
+                             int k_sel, double topp, double scale, int* kv_idx, int* kv_cnt,
+                             uint8_t* mask_opt, float* qp, float* kp, char* ws, const MaskWs& w,
+                             cudaStream_t st) {
+  const int nqb = (N + bq - 1) / bq, nkb = (N + bk - 1) / bk;
+  SliceOut sl{reinterpret_cast<int8_t*>(ws + w.q_sl), reinterpret_cast<int8_t*>(ws + w.k_sl),
+              reinterpret_cast<int*>(ws + w.q_ex), reinterpret_cast<int*>(ws + w.k_ex)};
+  float* s = reinterpret_cast<float*>(ws + w.s);
+  cudaError_t e = launch_pool(q, k, BH, N, d, bq, bk, qp, kp, st, &sl);
+  if (e == cudaSuccess) e = launch_scores_i8(sl, BH, nqb, nkb, d, scale, s, w.s_ld, st);
+  if (e == cudaSuccess) e = launch_select(s, w.s_ld, BH * nqb, nkb, k_sel, topp, kv_idx, kv_cnt, mask_opt, st);
+  return e;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -100,6 +125,20 @@ CUresult encode_tensor_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t 
   const cuuint32_t box[3] = {box_inner, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+CUresult encode_tensor_map_3d_u8(CUtensorMap* map, const void* base, uint64_t inner,
+                                 uint64_t rows, uint64_t planes, uint32_t box_inner,
+                                 uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return CUDA_ERROR_NOT_SUPPORTED;
+  const cuuint64_t dims[3] = {inner, rows, planes};
+  const cuuint64_t strides[2] = {inner, inner * rows};
+  const cuuint32_t box[3] = {box_inner, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
@@ -168,7 +207,7 @@ int sa_build_mask(const uint16_t* q, const uint16_t* k, int B, int H, int N, int
   if (!(topk_frac > 0.0 && topk_frac <= 1.0)) return fail(SA_ERR_INVALID_ARG, "topk_frac %g outside (0, 1]", topk_frac);
   if (!(topp >= 0.0 && topp <= 1.0)) return fail(SA_ERR_INVALID_ARG, "topp %g outside [0, 1]", topp);
   if (!isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "scale must be finite");
-  const int nkb = (N + bk - 1) / bk, nqb = (N + bq - 1) / bq;
+  const int nkb = (N + bk - 1) / bk;
   if (nkb > kMaxKeyBlocks) return fail(SA_ERR_UNSUPPORTED, "n_kb = %d exceeds %d", nkb, kMaxKeyBlocks);
   const void* ptrs[] = {q, k, kv_idx, kv_cnt, mask_opt, q_pool_opt, k_pool_opt, workspace};
   for (const void* p : ptrs)
@@ -180,13 +219,10 @@ int sa_build_mask(const uint16_t* q, const uint16_t* k, int B, int H, int N, int
   char* ws = static_cast<char*>(workspace);
   float* qp = q_pool_opt ? q_pool_opt : reinterpret_cast<float*>(ws + w.q_pool);
   float* kp = k_pool_opt ? k_pool_opt : reinterpret_cast<float*>(ws + w.k_pool);
-  float* s = reinterpret_cast<float*>(ws + w.s);
   const int BH = B * H;
   const int k_sel = static_cast<int>(fmin(static_cast<double>(nkb), fmax(1.0, ceil(topk_frac * nkb - 1e-9))));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_pool(q, k, BH, N, d, bq, bk, qp, kp, st);
-  if (e == cudaSuccess) e = launch_scores(qp, kp, BH, nqb, nkb, d, scale, s, w.s_ld, st);
-  if (e == cudaSuccess) e = launch_select(s, w.s_ld, BH * nqb, nkb, k_sel, topp, kv_idx, kv_cnt, mask_opt, st);
+  cudaError_t e = run_mask_builder(q, k, BH, N, d, bq, bk, k_sel, topp, scale, kv_idx, kv_cnt, mask_opt,
+                                   qp, kp, ws, w, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_build_mask");
 }
 

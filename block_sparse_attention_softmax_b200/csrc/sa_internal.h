@@ -14,10 +14,18 @@ __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; 
 __host__ __device__ inline int ceil_div_dev(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ inline long long ceil_div_ll(long long a, long long b) { return (a + b - 1) / b; }
 
+// Block means as four signed 7-bit slices per element plus a per-row power-of-two
+// exponent (written by the pooling kernel, read by the integer tensor-core scores).
+struct SliceOut {
+  int8_t* q_sl;   // [BH, nqb, 4 d]
+  int8_t* k_sl;   // [BH, nkb, 4 d]
+  int* q_ex;      // [BH, nqb]
+  int* k_ex;      // [BH, nkb]
+};
 cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, int bq, int bk,
-                        float* q_pool, float* k_pool, cudaStream_t st);
-cudaError_t launch_scores(const float* q_pool, const float* k_pool, int BH, int nqb, int nkb,
-                          int d, double scale, float* s, long long s_ld, cudaStream_t st);
+                        float* q_pool, float* k_pool, cudaStream_t st, const SliceOut* sl = nullptr);
+cudaError_t launch_scores_i8(const SliceOut& sl, int BH, int nqb, int nkb, int d, double scale,
+                             float* s, long long s_ld, cudaStream_t st);
 cudaError_t launch_select(const float* s, long long s_ld, int n_rows, int nkb, int k_sel,
                           double topp, int* kv_idx, int* kv_cnt, uint8_t* mask,
                           cudaStream_t st);
@@ -57,9 +65,13 @@ size_t linear_out_ws_bytes(int BH, int d);
 cudaError_t launch_linear_state(const LinearArgs& a, cudaStream_t st);
 cudaError_t launch_linear_out(const LinearArgs& a, cudaStream_t st);
 
-// Driver entry point for cuTensorMapEncodeTiled, resolved once.
+// Driver entry point for cuTensorMapEncodeTiled, resolved once. 3-D maps
+// (inner, rows, planes), 128-byte swizzle, zero fill out of bounds.
 CUresult encode_tensor_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t inner,
                                    uint64_t rows, uint64_t planes, uint32_t box_inner,
                                    uint32_t box_rows);
+CUresult encode_tensor_map_3d_u8(CUtensorMap* map, const void* base, uint64_t inner,
+                                 uint64_t rows, uint64_t planes, uint32_t box_inner,
+                                 uint32_t box_rows);
 
 }  // namespace sa
