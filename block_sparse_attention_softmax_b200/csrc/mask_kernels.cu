@@ -492,76 +492,91 @@ __global__ void __launch_bounds__(kSelWarpsMax * 32) select_kernel(
   }
 }
 
-// ---------------------------------------------------------------- selection, keys in registers
-// The same decisions as select_kernel for rows of at most 32 * KPL key blocks,
-// with each lane holding the keys and weights of elements lane + 32 j in
-// registers (no shared-memory histograms, so nothing serialises on atomics).
-//
-//   Top-k   MSB-first bitwise search for the largest key v with
-//           count(key >= v) >= K_sel. Full passes over the registers run only
-//           until {key >= v} has at most kCandMax members; the remaining bits
-//           are searched on that set, compacted into shared memory.
-//   Top-p   the same search on fp64 mass instead of count.
-// Elements past the row end carry key 0, below every finite score's key, and
-// weight 0, so they are never counted.
+// ---------------------------------------------------------------- selection, candidate path
+// The same decisions as select_kernel, for rows of at most 32 * KPL key
+// blocks, with the row's scores in registers (element lane + 32 j in x[j]).
+// K_sel is a small fraction of the row, so the exact search runs on a short
+// candidate list instead of the whole row:
+//   1. one pass gives the row max, mean and spread; a value t is then sought
+//      with K_sel <= count(s >= t) <= kCandMax, starting from the normal
+//      quantile of the row at about twice K_sel (tail quantile by Abramowitz
+//      and Stegun 26.2.23) and bracketing from there; usually 1-3 count
+//      passes;
+//   2. the elements >= t are compacted, in ascending block order, into shared
+//      memory, and the K_sel-th largest key is found by a bitwise search over
+//      the bits in which the candidates differ;
+//   3. the Top-k mass and the kept list come from the candidates alone.
+// Rows whose search does not settle (many equal scores), rows whose Top-p set
+// is longer than Top-k, and calls that want the u8 mask take full-row passes.
+// Weights are e^(s - max) by ex2.approx (relative error ~1e-7, an order of
+// magnitude inside the 1e-6 band within which a cumulative sum counts as a
+// tie with p); Z and all masses are summed in fp64.
 constexpr int kCandMax = 256;
+constexpr int kCandPL = kCandMax / 32;
 
-template <int KPL>
-__device__ __forceinline__ int count_ge(const uint32_t (&kr)[KPL], uint32_t c) {
+__device__ __forceinline__ float sel_weight(float x, float mx) {
+  return fast_exp2((x - mx) * 1.4426950408889634f);
+}
+
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// z with P(Z > z) = f for a standard normal Z, 0 < f <= 0.5 (Abramowitz and
+// Stegun 26.2.23, absolute error below 4.5e-4).
+__device__ __forceinline__ float normal_tail_quantile(float f) {
+  const float t = sqrtf(-2.f * logf(f));
+  return t - (2.515517f + t * (0.802853f + t * 0.010328f)) /
+                 (1.f + t * (1.432788f + t * (0.189269f + t * 0.001308f)));
+}
+
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+template <int N>
+__device__ __forceinline__ int count_ge_f(const float (&x)[N], float t) {
   int n = 0;
 #pragma unroll
-  for (int j = 0; j < KPL; ++j) n += kr[j] >= c ? 1 : 0;
+  for (int j = 0; j < N; ++j) n += x[j] >= t ? 1 : 0;
   return static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, static_cast<unsigned>(n)));
 }
 
+template <int N>
+__device__ __forceinline__ int count_ge_u(const uint32_t (&k)[N], uint32_t c) {
+  int n = 0;
+#pragma unroll
+  for (int j = 0; j < N; ++j) n += k[j] >= c ? 1 : 0;
+  return static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, static_cast<unsigned>(n)));
+}
+
+// Keys of x on the fly; elements past the row end never count.
 template <int KPL>
-__device__ Cut select_topk_reg(const uint32_t (&kr)[KPL], int k_sel, uint32_t* cand) {
+__device__ __forceinline__ int count_key_ge(const float (&x)[KPL], int nkb, uint32_t c) {
   const int lane = threadIdx.x & 31;
-  const uint32_t lt = (1u << lane) - 1u;
+  int n = 0;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) n += (lane + 32 * j < nkb && score_key(x[j]) >= c) ? 1 : 0;
+  return static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, static_cast<unsigned>(n)));
+}
+
+// Exact K_sel-th largest key of the whole row (fallback of the candidate path).
+template <int KPL>
+__device__ Cut topk_full(const float (&x)[KPL], int nkb, int k_sel) {
   uint32_t v = 0;
-  int bit = 31;
-  bool small = false;
-  for (; bit >= 0; --bit) {
+  for (int bit = 31; bit >= 0; --bit) {
     const uint32_t c = v | (1u << bit);
-    const int cnt = count_ge(kr, c);
-    if (cnt >= k_sel) {
-      v = c;
-      if (cnt <= kCandMax) {
-        small = true;
-        --bit;
-        break;
-      }
-    }
+    if (count_key_ge(x, nkb, c) >= k_sel) v = c;
   }
-  if (small) {
-    // every key that can still reach the threshold is >= v
-    int m = 0;
-#pragma unroll
-    for (int j = 0; j < KPL; ++j) {
-      const bool take = kr[j] >= v;
-      const uint32_t b = __ballot_sync(0xFFFFFFFFu, take);
-      if (take) cand[m + __popc(b & lt)] = kr[j];
-      m += __popc(b);
-    }
-    __syncwarp();
-    constexpr int CPL = kCandMax / 32;
-    uint32_t cr[CPL];
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) cr[i] = lane + 32 * i < m ? cand[lane + 32 * i] : 0u;
-    __syncwarp();
-    for (; bit >= 0; --bit) {
-      const uint32_t c = v | (1u << bit);
-      if (count_ge(cr, c) >= k_sel) v = c;
-    }
-  }
-  const int above = v == 0xFFFFFFFFu ? 0 : count_ge(kr, v + 1u);
+  const int above = v == 0xFFFFFFFFu ? 0 : count_key_ge(x, nkb, v + 1u);
   return Cut{v, above, k_sel - above};
 }
 
-// Smallest m such that the m largest-key weights sum to >= target. Weights
-// are in shared memory, element i at er[i] (lane-strided, conflict-free).
+// Smallest prefix (by key) whose weight reaches target; weights in er[i].
 template <int KPL>
-__device__ Cut select_mass_reg(const uint32_t (&kr)[KPL], const float* er, double target) {
+__device__ Cut mass_full(const float (&x)[KPL], int nkb, const float* er, double target) {
   const int lane = threadIdx.x & 31;
   uint32_t v = 0;
   for (int bit = 31; bit >= 0; --bit) {
@@ -569,7 +584,7 @@ __device__ Cut select_mass_reg(const uint32_t (&kr)[KPL], const float* er, doubl
     double w = 0.0;
 #pragma unroll
     for (int j = 0; j < KPL; ++j)
-      if (kr[j] >= c) w += static_cast<double>(er[lane + 32 * j]);
+      if (lane + 32 * j < nkb && score_key(x[j]) >= c) w += static_cast<double>(er[lane + 32 * j]);
     if (warp_sum_d(w) >= target) v = c;
   }
   int above = 0, nties = 0;
@@ -577,10 +592,12 @@ __device__ Cut select_mass_reg(const uint32_t (&kr)[KPL], const float* er, doubl
   float e_tie = 0.f;
 #pragma unroll
   for (int j = 0; j < KPL; ++j) {
-    if (kr[j] > v) {
+    if (lane + 32 * j >= nkb) continue;
+    const uint32_t key = score_key(x[j]);
+    if (key > v) {
       ++above;
       w_above += static_cast<double>(er[lane + 32 * j]);
-    } else if (kr[j] == v) {
+    } else if (key == v) {
       ++nties;
       e_tie = er[lane + 32 * j];
     }
@@ -595,70 +612,26 @@ __device__ Cut select_mass_reg(const uint32_t (&kr)[KPL], const float* er, doubl
     acc += static_cast<double>(e_tie);
     ++t;
   }
-  if (acc < target) t = nties;
+  if (acc < target) t = nties;        // rounding kept the total below the target
   if (above + t == 0) t = 1;
   return Cut{v, above, t};
 }
 
-// One query-block row per warp: the row's keys in registers, its weights in
-// the warp's shared-memory slice er[32 * KPL]; decision and ascending
-// compaction as in select_kernel.
+// Kept set of a cut over the whole row, in ascending block order.
 template <int KPL>
-__device__ __forceinline__ void select_row_reg(const float* __restrict__ srow, int nkb, int k_sel,
-                                               double topp, int* __restrict__ out,
-                                               int* __restrict__ cnt_out, uint8_t* __restrict__ mrow,
-                                               uint32_t* cand, float* er) {
+__device__ void output_full(const float (&x)[KPL], int nkb, const Cut& cut, int* __restrict__ out,
+                            int* __restrict__ cnt_out, uint8_t* __restrict__ mrow) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;
-  uint32_t kr[KPL];
-  float mx = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < KPL; ++j) {
-    const int i = lane + 32 * j;
-    const float v = i < nkb ? srow[i] : -INFINITY;
-    kr[j] = i < nkb ? score_key(v) : 0u;
-    er[i] = v;
-    mx = fmaxf(mx, v);
-  }
-  mx = warp_max(mx);
-  double z = 0.0;
-#pragma unroll
-  for (int j = 0; j < KPL; ++j) {
-    const int i = lane + 32 * j;
-    const float e = i < nkb ? expf(er[i] - mx) : 0.f;
-    er[i] = e;
-    z += static_cast<double>(e);
-  }
-  z = warp_sum_d(z);
-
-  Cut cut{0u, 0, nkb};                // keep everything (every finite score's key is > 0)
-  if (!(topp >= 1.0 || k_sel >= nkb)) {
-    cut = select_topk_reg(kr, k_sel, cand);
-    const double target = topp * z;
-    double wk = 0.0;
-    int tie_before = 0;
-#pragma unroll
-    for (int j = 0; j < KPL; ++j) {
-      const bool tie = kr[j] == cut.key;
-      const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
-      const bool keep = kr[j] > cut.key || (tie && tie_before + __popc(tb & lt) < cut.ties);
-      if (keep) wk += static_cast<double>(er[lane + 32 * j]);
-      tie_before += __popc(tb);
-    }
-    wk = warp_sum_d(wk);
-    if (wk < target) {
-      const Cut cp = select_mass_reg(kr, er, target);
-      if (cp.above + cp.ties > k_sel) cut = cp;
-    }
-  }
   int written = 0, tie_before = 0;
 #pragma unroll
   for (int j = 0; j < KPL; ++j) {
     const int i = lane + 32 * j;
     const bool valid = i < nkb;
-    const bool tie = valid && kr[j] == cut.key;
+    const uint32_t key = score_key(x[j]);
+    const bool tie = valid && key == cut.key;
     const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
-    const bool keep = valid && (kr[j] > cut.key || (tie && tie_before + __popc(tb & lt) < cut.ties));
+    const bool keep = valid && (key > cut.key || (tie && tie_before + __popc(tb & lt) < cut.ties));
     const uint32_t kb = __ballot_sync(0xFFFFFFFFu, keep);
     if (keep) out[written + __popc(kb & lt)] = i;
     if (mrow && valid) mrow[i] = keep ? 1 : 0;
@@ -666,6 +639,199 @@ __device__ __forceinline__ void select_row_reg(const float* __restrict__ srow, i
     tie_before += __popc(tb);
   }
   if (lane == 0) *cnt_out = written;
+}
+
+// One query-block row per warp. `ckey`/`cidx` hold kCandMax candidates and
+// `er` 32 * KPL weights, all in this warp's shared memory.
+template <int KPL>
+__device__ void select_row_fast(const float* __restrict__ srow, int nkb, int k_sel, double topp,
+                                int* __restrict__ out, int* __restrict__ cnt_out,
+                                uint8_t* __restrict__ mrow, uint32_t* ckey, int* cidx, float* er) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  float x[KPL];
+  float mx = -INFINITY, sum = 0.f, sq = 0.f;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) {
+    const int i = lane + 32 * j;
+    x[j] = i < nkb ? srow[i] : -INFINITY;
+    if (i < nkb) {
+      sum += x[j];
+      sq = fmaf(x[j], x[j], sq);
+    }
+    mx = fmaxf(mx, x[j]);
+  }
+  mx = warp_max(mx);
+  double z0 = 0.0, z1 = 0.0;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) {
+    const float e = sel_weight(x[j], mx);            // 0 past the row end (x = -inf)
+    er[lane + 32 * j] = e;
+    if (j & 1) z1 += static_cast<double>(e);
+    else z0 += static_cast<double>(e);
+  }
+  const double z = warp_sum_d(z0 + z1);
+
+  if (topp >= 1.0 || k_sel >= nkb) {
+    output_full(x, nkb, Cut{0u, 0, nkb}, out, cnt_out, mrow);   // every finite score's key is > 0
+    return;
+  }
+  const double target = topp * z;
+
+  // ---- 1. a threshold value with K_sel <= count <= kCandMax
+  bool found = false;
+  float t = mx;
+  if (k_sel <= kCandMax) {
+    sum = warp_sum_f(sum);
+    sq = warp_sum_f(sq);
+    const float mean = sum / nkb;
+    const float sd = sqrtf(fmaxf(sq / nkb - mean * mean, 0.f));
+    const int want = min(kCandMax - 32, max(2 * k_sel, k_sel + 32));
+    const float f = fminf(static_cast<float>(want) / nkb, 0.5f);
+    t = fminf(mean + normal_tail_quantile(f) * sd, mx);
+    const float step = fmaxf(sd, 1e-6f * fmaxf(fabsf(mx), 1.f));
+    float tlo = -INFINITY, thi = INFINITY;
+    for (int it = 0; it < 12; ++it) {
+      const int c = count_ge_f(x, t);
+      if (c >= k_sel && c <= kCandMax) {
+        found = true;
+        break;
+      }
+      if (c < k_sel) thi = t;
+      else tlo = t;
+      float nt;
+      if (tlo > -INFINITY && thi < INFINITY) nt = 0.5f * (tlo + thi);
+      else if (thi < INFINITY) nt = thi - step * static_cast<float>(1 << it);
+      else nt = fminf(tlo + step * static_cast<float>(1 << it), mx);
+      if (nt == t || nt == tlo || nt == thi) break;   // no float left between the bounds
+      t = nt;
+    }
+  }
+
+  Cut cut;
+  if (found) {
+    // ---- 2. candidates in ascending block order, exact search among them
+    int m = 0;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      const bool take = x[j] >= t;
+      const uint32_t b = __ballot_sync(0xFFFFFFFFu, take);
+      if (take) {
+        ckey[m + __popc(b & lt)] = score_key(x[j]);
+        cidx[m + __popc(b & lt)] = lane + 32 * j;
+      }
+      m += __popc(b);
+    }
+    __syncwarp();
+    uint32_t ck[kCandPL];
+    uint32_t kand = 0xFFFFFFFFu, kor = 0u;
+#pragma unroll
+    for (int q = 0; q < kCandPL; ++q) {
+      const bool valid = lane + 32 * q < m;
+      ck[q] = valid ? ckey[lane + 32 * q] : 0u;
+      if (valid) {
+        kand &= ck[q];
+        kor |= ck[q];
+      }
+    }
+    kand = __reduce_and_sync(0xFFFFFFFFu, kand);
+    kor = __reduce_or_sync(0xFFFFFFFFu, kor);
+    const uint32_t diff = kand ^ kor;
+    const int top = diff ? 31 - __clz(diff) : -1;
+    uint32_t v = top >= 0 ? (kand & ~(0xFFFFFFFFu >> (31 - top))) : kand;   // common high bits
+    for (int bit = top; bit >= 0; --bit) {
+      const uint32_t c = v | (1u << bit);
+      if (count_ge_u(ck, c) >= k_sel) v = c;
+    }
+    const int above = v == 0xFFFFFFFFu ? 0 : count_ge_u(ck, v + 1u);
+    cut = Cut{v, above, k_sel - above};
+    // ---- 3. Top-k mass over the kept candidates
+    double wk = 0.0;
+    int tie_before = 0;
+#pragma unroll
+    for (int q = 0; q < kCandPL; ++q) {
+      const bool valid = lane + 32 * q < m;
+      const bool tie = valid && ck[q] == v;
+      const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
+      const bool keep = valid && (ck[q] > v || (tie && tie_before + __popc(tb & lt) < cut.ties));
+      if (keep) wk += static_cast<double>(sel_weight(key_value(ck[q]), mx));
+      tie_before += __popc(tb);
+    }
+    wk = warp_sum_d(wk);
+    if (wk >= target && mrow == nullptr) {
+      int written = 0;
+      tie_before = 0;
+#pragma unroll
+      for (int q = 0; q < kCandPL; ++q) {
+        const bool valid = lane + 32 * q < m;
+        const bool tie = valid && ck[q] == v;
+        const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
+        const bool keep = valid && (ck[q] > v || (tie && tie_before + __popc(tb & lt) < cut.ties));
+        const uint32_t kb = __ballot_sync(0xFFFFFFFFu, keep);
+        if (keep) out[written + __popc(kb & lt)] = cidx[lane + 32 * q];
+        written += __popc(kb);
+        tie_before += __popc(tb);
+      }
+      if (lane == 0) *cnt_out = written;
+      __syncwarp();
+      return;
+    }
+    __syncwarp();
+    if (wk < target) {
+      const Cut cp = mass_full(x, nkb, er, target);
+      if (cp.above + cp.ties > k_sel) cut = cp;
+    }
+  } else {
+    cut = topk_full(x, nkb, k_sel);
+    // Top-k mass over the whole row
+    double wk = 0.0;
+    int tie_before = 0;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      const bool valid = lane + 32 * j < nkb;
+      const uint32_t key = score_key(x[j]);
+      const bool tie = valid && key == cut.key;
+      const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
+      const bool keep = valid && (key > cut.key || (tie && tie_before + __popc(tb & lt) < cut.ties));
+      if (keep) wk += static_cast<double>(er[lane + 32 * j]);
+      tie_before += __popc(tb);
+    }
+    wk = warp_sum_d(wk);
+    if (wk < target) {
+      const Cut cp = mass_full(x, nkb, er, target);
+      if (cp.above + cp.ties > k_sel) cut = cp;
+    }
+  }
+  output_full(x, nkb, cut, out, cnt_out, mrow);
+}
+
+constexpr int kSelFastWarps = 4;
+
+template <int KPL>
+__global__ void __launch_bounds__(kSelFastWarps * 32, 4) select_fast_kernel(
+    const float* __restrict__ s, long long s_ld, int n_rows, int nkb, int k_sel, double topp,
+    int* __restrict__ kv_idx, int* __restrict__ kv_cnt, uint8_t* __restrict__ mask) {
+  __shared__ uint32_t ckey_all[kSelFastWarps][kCandMax];
+  __shared__ int cidx_all[kSelFastWarps][kCandMax];
+  __shared__ float e_all[kSelFastWarps][32 * KPL];
+  const int warp = threadIdx.x >> 5;
+  for (int row = blockIdx.x * kSelFastWarps + warp; row < n_rows; row += gridDim.x * kSelFastWarps) {
+    select_row_fast<KPL>(s + static_cast<long long>(row) * s_ld, nkb, k_sel, topp,
+                         kv_idx + static_cast<long long>(row) * nkb, kv_cnt + row,
+                         mask ? mask + static_cast<long long>(row) * nkb : nullptr,
+                         ckey_all[warp], cidx_all[warp], e_all[warp]);
+    __syncwarp();
+  }
+}
+
+template <int KPL>
+static cudaError_t launch_select_fast(const float* s, long long s_ld, int n_rows, int nkb, int k_sel,
+                                      double topp, int* kv_idx, int* kv_cnt, uint8_t* mask,
+                                      cudaStream_t st) {
+  const int want = (n_rows + kSelFastWarps - 1) / kSelFastWarps;
+  const int grid = want < 65535 * 8 ? want : 65535 * 8;
+  select_fast_kernel<KPL><<<grid, kSelFastWarps * 32, 0, st>>>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask);
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- uint8 mask -> lists
@@ -731,6 +897,10 @@ cudaError_t launch_scores_i8(const SliceOut& sl, int BH, int nqb, int nkb, int d
 cudaError_t launch_select(const float* s, long long s_ld, int n_rows, int nkb, int k_sel,
                           double topp, int* kv_idx, int* kv_cnt, uint8_t* mask,
                           cudaStream_t st) {
+  // rows of up to 40 blocks per lane: candidate path with the row in registers
+  if (nkb <= 32 * 4) return launch_select_fast<4>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st);
+  if (nkb <= 32 * 16) return launch_select_fast<16>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st);
+  if (nkb <= 32 * 40) return launch_select_fast<40>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st);
   const size_t slice = static_cast<size_t>(nkb) * 8 + 256 * 4;
   int wpc = static_cast<int>((200u * 1024u) / slice);
   wpc = wpc < 1 ? 1 : (wpc > kSelWarpsMax ? kSelWarpsMax : wpc);
