@@ -86,7 +86,9 @@ struct OutLayout {
   static constexpr uint32_t OFF_Q = 2 * B_BYTES;
   static constexpr uint32_t OFF_OS = OFF_Q + NSTG * T_BYTES;
   static constexpr uint32_t OFF_DEN = OFF_OS + NSTG * T_BYTES;  // [NSTG][4 parts][128 rows] fp32
-  static constexpr uint32_t OFF_BAR = OFF_DEN + NSTG * 4 * 128 * 4;
+  static constexpr int ZA_HEADS = 8;                              // z and alpha of up to 8 heads per CTA
+  static constexpr uint32_t OFF_ZA = OFF_DEN + NSTG * 4 * 128 * 4;  // [ZA_HEADS][2][D] fp32
+  static constexpr uint32_t OFF_BAR = OFF_ZA + ZA_HEADS * 2 * D * 4;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
 };
 
@@ -346,8 +348,11 @@ __global__ void linear_reduce_kernel(const float* __restrict__ part, lin::StateG
 // the math warps apply phi to Q in place and, four threads per token, form the
 // denominator phi(q_t) . z; one thread issues D[t, :] = phi(Q)[t, :] S_hi +
 // phi(Q)[t, :] S_lo (tcgen05, TMEM accumulator, double buffered), which also
-// frees the Q stage; the math warps then divide, blend with O_s and store O.
-// The four warps that share TMEM lane quadrant w % 4 split the d columns.
+// frees the Q stage; the math warps then divide, blend with O_s and write O
+// over O_s in the stage, and the O_s warp stores the stage to O by TMA before
+// loading the next O_s into it. z and alpha of the CTA's heads sit in shared
+// memory. The four warps that share TMEM lane quadrant w % 4 split the d
+// columns.
 constexpr int kOutMathWarps = 16;
 constexpr int kOsWarp = 2 + kOutMathWarps;
 constexpr int kOutThreads = 32 * (kOsWarp + 1);
@@ -383,9 +388,10 @@ __device__ __forceinline__ void build_head_operand(uint8_t* smem, const float* _
 template <int D>
 __global__ void __launch_bounds__(kOutThreads, 1)
     linear_out_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmOs,
+                      const __grid_constant__ CUtensorMap tmO,
                       const float* __restrict__ kv_state, const float* __restrict__ ksum,
                       const float* __restrict__ alpha, int H, int N, lin::StateGeom geo,
-                      int blend, uint16_t* __restrict__ o) {
+                      int blend) {
   using L = lin::OutLayout<D>;
   constexpr int NS = L::NSTG;
   extern __shared__ uint8_t smem_raw[];
@@ -393,8 +399,8 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bars;                  // [NS] Q landed
   uint64_t* q_empty = bars + NS;            // [NS] MMA on that Q completed
-  uint64_t* os_full = bars + 2 * NS;        // [NS] O_s landed
-  uint64_t* os_empty = bars + 3 * NS;       // [NS] epilogue done (math warps)
+  uint64_t* os_full = bars + 2 * NS;        // [NS] O_s landed (or, without blend, the stage is free)
+  uint64_t* o_ready = bars + 3 * NS;        // [NS] O written into the stage (math warps)
   uint64_t* phi_done = bars + 4 * NS;       // [NS] phi and denominators ready (math warps)
   uint64_t* acc_full = bars + 5 * NS;       // [2]
   uint64_t* acc_empty = acc_full + 2;       // [2] (math warps)
@@ -402,6 +408,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(b_ready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* den = reinterpret_cast<float*>(smem + L::OFF_DEN);
+  float* za = reinterpret_cast<float*>(smem + L::OFF_ZA);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * geo.tpc;
@@ -414,7 +421,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
       mbar_init(&os_full[s], 1);
-      mbar_init(&os_empty[s], kOutMathWarps);
+      mbar_init(&o_ready[s], kOutMathWarps);
       mbar_init(&phi_done[s], kOutMathWarps);
     }
     for (int b = 0; b < 2; ++b) {
@@ -426,6 +433,18 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     fence_barrier_init();
   }
   build_head_operand<D>(smem, kv_state, t0 / geo.tph, threadIdx.x, blockDim.x);
+  // z and alpha of this CTA's heads (from global memory if there are more
+  // heads than slots)
+  const int h_first = t0 / geo.tph;
+  const int n_heads = (t1 - 1) / geo.tph - h_first + 1;
+  const bool za_smem = n_heads <= L::ZA_HEADS;
+  if (za_smem) {
+    for (int i = threadIdx.x; i < n_heads * D; i += blockDim.x) {
+      const int hh = i / D, c = i % D;
+      za[(hh * 2) * D + c] = ksum[static_cast<long long>(h_first + hh) * D + c];
+      za[(hh * 2 + 1) * D + c] = blend ? alpha[static_cast<long long>((h_first + hh) % H) * D + c] : 0.f;
+    }
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
@@ -435,25 +454,60 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   tc_fence_after();
   const uint32_t tm = *tmem_slot;
 
-  if (warp == 0 || warp == kOsWarp) {
-    // ------------------------------------------------------------ producers
-    const bool is_q = warp == 0;
-    if (lane == 0 && (is_q || blend)) {
-      const CUtensorMap* map = is_q ? &tmQ : &tmOs;
-      tma_prefetch_desc(map);
-      uint64_t* fullb = is_q ? q_full : os_full;
-      uint64_t* emptyb = is_q ? q_empty : os_empty;
-      const uint32_t base = is_q ? L::OFF_Q : L::OFF_OS;
+  if (warp == 0) {
+    // ------------------------------------------------------------ Q producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % NS;
-        if (!mbar_wait(&emptyb[s], ((i / NS) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&fullb[s], L::T_BYTES);
+        if (!mbar_wait(&q_empty[s], ((i / NS) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&q_full[s], L::T_BYTES);
         const int t = t0 + i;
         const int row = (t % geo.tph) * lin::kLinTok, bh = t / geo.tph;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + base + s * L::T_BYTES + c * L::T_CHUNK, map, &fullb[s], c * 64, row, bh);
+          tma_load_3d(smem + L::OFF_Q + s * L::T_BYTES + c * L::T_CHUNK, &tmQ, &q_full[s], c * 64, row, bh);
       }
+    }
+  } else if (warp == kOsWarp) {
+    // ------------------------------------------------------------ O_s loads, O stores
+    // Stage s of tile i: once the math warps have written O of tile i - NS
+    // into it, store that tile by TMA, wait until the store has read the
+    // stage, then load O_s of tile i (or, without blend, just release it).
+    if (lane == 0) {
+      if (blend) tma_prefetch_desc(&tmOs);
+      tma_prefetch_desc(&tmO);
+      auto store_tile = [&](int j) -> bool {
+        const int s = j % NS;
+        if (!mbar_wait(&o_ready[s], (j / NS) & 1, abort_flag)) return false;
+        const int t = t0 + j;
+        const int row = (t % geo.tph) * lin::kLinTok, bh = t / geo.tph;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_store_3d(&tmO, smem + L::OFF_OS + s * L::T_BYTES + c * L::T_CHUNK, c * 64, row, bh);
+        bulk_commit();
+        return true;
+      };
+      bool ok = true;
+      for (int i = 0; ok && i < n_tiles; ++i) {
+        const int s = i % NS;
+        if (i >= NS) {
+          if (!(ok = store_tile(i - NS))) break;
+          bulk_wait_read_all();
+        }
+        if (blend) {
+          mbar_arrive_expect_tx(&os_full[s], L::T_BYTES);
+          const int t = t0 + i;
+          const int row = (t % geo.tph) * lin::kLinTok, bh = t / geo.tph;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem + L::OFF_OS + s * L::T_BYTES + c * L::T_CHUNK, &tmOs, &os_full[s], c * 64, row, bh);
+        } else {
+          mbar_arrive(&os_full[s]);
+        }
+      }
+      for (int j = n_tiles > NS ? n_tiles - NS : 0; ok && j < n_tiles; ++j) ok = store_tile(j);
+      bulk_wait_all();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -501,7 +555,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       const int tok = (t % geo.tph) * lin::kLinTok + row;
       if (!mbar_wait(&acc_full[ab], (j >> 1) & 1, abort_flag)) return false;
       if (!mbar_wait(&phi_done[s], (j / NS) & 1, abort_flag)) return false;   // denominators visible
-      if (blend && !mbar_wait(&os_full[s], (j / NS) & 1, abort_flag)) return false;
+      if (!mbar_wait(&os_full[s], (j / NS) & 1, abort_flag)) return false;    // O_s in, stage free
       tc_fence_after();
       uint32_t x0[32];
       if (HC == 32) {
@@ -514,21 +568,22 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       }
       const float* dj = den + s * 4 * 128;
       const float inv = 1.f / ((dj[row] + dj[128 + row]) + (dj[256 + row] + dj[384 + row]));
-      if (tok < N) {
-        const uint8_t* osrow = smem + L::OFF_OS + s * L::T_BYTES;
-        const float* al = alpha + static_cast<long long>(bh % H) * D;
-        uint16_t* orow = o + (static_cast<long long>(bh) * N + tok) * D + grp * HC;
+      (void)tok;   // rows past N are clipped by the TMA store
+      {
+        uint8_t* osrow = smem + L::OFF_OS + s * L::T_BYTES;
+        const float* al = za_smem ? za + ((bh - h_first) * 2 + 1) * D : alpha + static_cast<long long>(bh % H) * D;
 #pragma unroll
         for (int j2 = 0; j2 < HU; ++j2) {
           const int uu = grp * HU + j2;
+          uint4* slot = reinterpret_cast<uint4*>(osrow + (uu >> 3) * L::T_CHUNK + row * 128 + (((uu & 7) ^ (row & 7)) << 4));
           float l[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) l[e] = __uint_as_float(x0[j2 * 8 + e]) * inv;
           uint32_t pk[4];
           if (blend) {
-            const uint4 w = *reinterpret_cast<const uint4*>(osrow + (uu >> 3) * L::T_CHUNK + row * 128 + (((uu & 7) ^ (row & 7)) << 4));
-            const float4 a0 = __ldg(reinterpret_cast<const float4*>(al + uu * 8));
-            const float4 a1 = __ldg(reinterpret_cast<const float4*>(al + uu * 8 + 4));
+            const uint4 w = *slot;
+            const float4 a0 = *reinterpret_cast<const float4*>(al + uu * 8);
+            const float4 a1 = *reinterpret_cast<const float4*>(al + uu * 8 + 4);
             const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -540,14 +595,15 @@ __global__ void __launch_bounds__(kOutThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) pk[e] = pack_bf16x2(l[2 * e], l[2 * e + 1]);
           }
-          reinterpret_cast<uint4*>(orow)[j2] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *slot = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       }
+      fence_proxy_async_smem();     // O visible to the TMA store
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&acc_empty[ab]);
-        mbar_arrive(&os_empty[s]);
+        mbar_arrive(&o_ready[s]);
       }
       return true;
     };
@@ -557,10 +613,10 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       if (!(ok = mbar_wait(&q_full[s], (i / NS) & 1, abort_flag))) break;
       // the denominator slot of stage s is free once every warp has finished
       // the epilogue of tile i - NS
-      if (i >= NS && !(ok = mbar_wait(&os_empty[s], ((i / NS) & 1) ^ 1, abort_flag))) break;
+      if (i >= NS && !(ok = mbar_wait(&o_ready[s], ((i / NS) & 1) ^ 1, abort_flag))) break;
       // phi(Q) in place and the partial denominator of token trow
       {
-        const float* zg = ksum + static_cast<long long>(t / geo.tph) * D;
+        const float* zg = za_smem ? za + ((t / geo.tph - h_first) * 2) * D : ksum + static_cast<long long>(t / geo.tph) * D;
         uint8_t* qt = smem + L::OFF_Q + s * L::T_BYTES;
         float dz = 0.f;
 #pragma unroll
@@ -569,8 +625,8 @@ __global__ void __launch_bounds__(kOutThreads, 1)
           uint4* p = reinterpret_cast<uint4*>(qt + (uu >> 3) * L::T_CHUNK + trow * 128 + (((uu & 7) ^ (trow & 7)) << 4));
           uint4 w = *p;
           uint32_t* x = reinterpret_cast<uint32_t*>(&w);
-          const float4 z0 = __ldg(reinterpret_cast<const float4*>(zg + uu * 8));
-          const float4 z1 = __ldg(reinterpret_cast<const float4*>(zg + uu * 8 + 4));
+          const float4 z0 = *reinterpret_cast<const float4*>(zg + uu * 8);
+          const float4 z1 = *reinterpret_cast<const float4*>(zg + uu * 8 + 4);
           const float zv[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -638,15 +694,16 @@ static cudaError_t out_d(const LinearArgs& a, cudaStream_t st) {
   using L = lin::OutLayout<D>;
   const int BH = a.B * a.H;
   const lin::StateGeom geo = lin::state_geom(BH, a.N, lin::sm_count());
-  CUtensorMap mq, mos;
+  CUtensorMap mq, mos, mo;
   if (encode_tensor_map_3d_bf16(&mq, a.q, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   const int blend = a.o_s != nullptr;
   if (encode_tensor_map_3d_bf16(&mos, blend ? a.o_s : a.q, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  if (encode_tensor_map_3d_bf16(&mo, a.o, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(linear_out_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   linear_out_kernel<D><<<geo.grid, kOutThreads, L::SMEM, st>>>(
-      mq, mos, a.kv_state, a.ksum, blend ? a.alpha : nullptr, a.H, a.N, geo, blend, static_cast<uint16_t*>(a.o));
+      mq, mos, mo, a.kv_state, a.ksum, blend ? a.alpha : nullptr, a.H, a.N, geo, blend);
   return cudaGetLastError();
 }
 
