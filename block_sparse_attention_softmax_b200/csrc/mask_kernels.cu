@@ -138,12 +138,19 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 // once to fp32. Its error stays near 1e-7 of the score scale, well inside the
 // 1e-6 band within which the mask comparison treats a cut as a tie.
 //
-// CTA tile: 128 query blocks (M, operand A) x 64 key blocks (N, operand B),
-// both K-major with 128-byte swizzled rows, one TMA box per 128-byte column
-// chunk. Thread 0 loads the tiles and issues the 4 d / 32 * 10 MMAs; the four
-// warps then read their TMEM lane quadrant and write the scores.
+// Persistent CTAs over work items (head, 128 query blocks, a range of 64-key
+// tiles): warp 0 loads the item's query slices (operand A, M = 128) and
+// streams the key-slice tiles (operand B, N = 64) through a 3-stage ring by
+// TMA (128-byte swizzled rows, one box per 128-byte column chunk); warp 1
+// issues the 10 * d / 32 MMAs of a key tile into one of two TMEM accumulator
+// sets; eight epilogue warps (two per TMEM lane quadrant, 32 key columns
+// each) combine the levels, transpose each 32 x 32 block through shared
+// memory and write score rows with coalesced 128-byte stores.
 constexpr int kI8TileM = 128;
 constexpr int kI8TileN = 64;
+constexpr int kI8BStages = 3;
+constexpr int kI8EpiWarps = 8;
+constexpr int kI8Threads = 32 * (2 + kI8EpiWarps);
 
 template <int D>
 struct I8Layout {
@@ -151,43 +158,57 @@ struct I8Layout {
   static constexpr int NCH = ROW / 128;             // 128-byte column chunks
   static constexpr uint32_t A_CH = kI8TileM * 128;  // bytes of one A chunk
   static constexpr uint32_t B_CH = kI8TileN * 128;
+  static constexpr uint32_t A_BYTES = NCH * A_CH;
+  static constexpr uint32_t B_BYTES = NCH * B_CH;
   static constexpr uint32_t OFF_A = 0;
-  static constexpr uint32_t OFF_B = OFF_A + NCH * A_CH;
-  static constexpr uint32_t OFF_KEX = OFF_B + NCH * B_CH;
-  static constexpr uint32_t OFF_BAR = OFF_KEX + kI8TileN * 4;
-  static constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
+  static constexpr uint32_t OFF_B = OFF_A + A_BYTES;
+  static constexpr uint32_t OFF_T = OFF_B + kI8BStages * B_BYTES;      // [epi warps][32][33] fp32
+  static constexpr uint32_t OFF_BAR = OFF_T + kI8EpiWarps * 32 * 33 * 4;
+  static constexpr uint32_t SMEM = OFF_BAR + 128 + 1024;
+};
+
+struct I8Work {
+  int nqb, nkb, n_qt, n_kt, kr_tiles, n_kr, n_items;
 };
 
 template <int D>
-__global__ void __launch_bounds__(128) score_i8_kernel(const __grid_constant__ CUtensorMap tmA,
-                                                       const __grid_constant__ CUtensorMap tmB,
-                                                       const int* __restrict__ q_ex,
-                                                       const int* __restrict__ k_ex, int nqb,
-                                                       int nkb, double scale,
-                                                       float* __restrict__ s, long long s_ld) {
+__global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_constant__ CUtensorMap tmA,
+                                                                 const __grid_constant__ CUtensorMap tmB,
+                                                                 const int* __restrict__ q_ex,
+                                                                 const int* __restrict__ k_ex, I8Work wk,
+                                                                 double scale, float* __restrict__ s,
+                                                                 long long s_ld) {
   using L = I8Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  int* kex = reinterpret_cast<int*>(smem + L::OFF_KEX);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);   // [0] tiles landed, [1] MMAs done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* a_full = bars;                        // item's query slices landed
+  uint64_t* a_empty = bars + 1;                   // item's last MMA completed
+  uint64_t* b_full = bars + 2;                    // [kI8BStages]
+  uint64_t* b_empty = b_full + kI8BStages;        // [kI8BStages]
+  uint64_t* acc_full = b_empty + kI8BStages;      // [2]
+  uint64_t* acc_empty = acc_full + 2;             // [2] (epilogue warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.z;
-  const int qb0 = blockIdx.y * kI8TileM;
-  const int kb0 = blockIdx.x * kI8TileN;
-  constexpr uint32_t kCols = 4 * kI8TileN;            // four level accumulators
+  constexpr uint32_t kSet = 4 * kI8TileN;         // columns of one accumulator set (four levels)
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    mbar_init(a_full, 1);
+    mbar_init(a_empty, 1);
+    for (int i = 0; i < kI8BStages; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], kI8EpiWarps);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (threadIdx.x < kI8TileN)
-    kex[threadIdx.x] = kb0 + threadIdx.x < nkb ? __ldg(k_ex + static_cast<long long>(bh) * nkb + kb0 + threadIdx.x) : 0;
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, kCols);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * kSet);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -195,80 +216,151 @@ __global__ void __launch_bounds__(128) score_i8_kernel(const __grid_constant__ C
   tc_fence_after();
   const uint32_t tm = *tmem_slot;
 
-  if (threadIdx.x == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-    mbar_arrive_expect_tx(&bars[0], L::NCH * (L::A_CH + L::B_CH));
+  // work item -> (head, query tile, first and end key tile)
+  auto decode = [&](int item, int& bh, int& qt, int& kt0, int& kt1) {
+    const int kr = item % wk.n_kr;
+    const int rest = item / wk.n_kr;
+    qt = rest % wk.n_qt;
+    bh = rest / wk.n_qt;
+    kt0 = kr * wk.kr_tiles;
+    kt1 = min(wk.n_kt, kt0 + wk.kr_tiles);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      int ic = 0, bt = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < wk.n_items; item += gridDim.x, ++ic) {
+        int bh, qt, kt0, kt1;
+        decode(item, bh, qt, kt0, kt1);
+        if (!(ok = mbar_wait(a_empty, (ic & 1) ^ 1, abort_flag))) break;
+        mbar_arrive_expect_tx(a_full, L::A_BYTES);
 #pragma unroll
-    for (int c = 0; c < L::NCH; ++c) {
-      tma_load_3d(smem + L::OFF_A + c * L::A_CH, &tmA, &bars[0], c * 128, qb0, bh);
-      tma_load_3d(smem + L::OFF_B + c * L::B_CH, &tmB, &bars[0], c * 128, kb0, bh);
+        for (int c = 0; c < L::NCH; ++c)
+          tma_load_3d(smem + L::OFF_A + c * L::A_CH, &tmA, a_full, c * 128, qt * kI8TileM, bh);
+        for (int kt = kt0; kt < kt1; ++kt, ++bt) {
+          const int st = bt % kI8BStages;
+          if (!(ok = mbar_wait(&b_empty[st], ((bt / kI8BStages) & 1) ^ 1, abort_flag))) break;
+          mbar_arrive_expect_tx(&b_full[st], L::B_BYTES);
+#pragma unroll
+          for (int c = 0; c < L::NCH; ++c)
+            tma_load_3d(smem + L::OFF_B + st * L::B_BYTES + c * L::B_CH, &tmB, &b_full[st], c * 128, kt * kI8TileN, bh);
+        }
+      }
     }
-    if (mbar_wait(&bars[0], 0, abort_flag)) {
-      tc_fence_after();
-      const uint64_t a0 = sw128_desc(smem_u32(smem + L::OFF_A), 16, 1024);
-      const uint64_t b0 = sw128_desc(smem_u32(smem + L::OFF_B), 16, 1024);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
       constexpr uint32_t idesc = idesc_s8_s32(kI8TileM, kI8TileN);
-      // byte offset of a K step inside the chunked, swizzled tile
+      const uint64_t a0 = sw128_desc(smem_u32(smem + L::OFF_A), 16, 1024);
+      const uint64_t b00 = sw128_desc(smem_u32(smem + L::OFF_B), 16, 1024);
+      // descriptor offset of a K step inside the chunked, swizzled tile
       auto off = [](int byte, uint32_t chunk_bytes) -> uint32_t {
         return (static_cast<uint32_t>(byte >> 7) * chunk_bytes + static_cast<uint32_t>(byte & 127)) >> 4;
       };
+      int ic = 0, bt = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < wk.n_items; item += gridDim.x, ++ic) {
+        int bh, qt, kt0, kt1;
+        decode(item, bh, qt, kt0, kt1);
+        if (!(ok = mbar_wait(a_full, ic & 1, abort_flag))) break;
+        for (int kt = kt0; kt < kt1; ++kt, ++bt) {
+          const int st = bt % kI8BStages, ab = bt & 1;
+          if (!(ok = mbar_wait(&b_full[st], (bt / kI8BStages) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(&acc_empty[ab], ((bt >> 1) & 1) ^ 1, abort_flag))) break;
+          tc_fence_after();
+          const uint64_t b0 = b00 + ((st * L::B_BYTES) >> 4);
+          const uint32_t acc = tm + ab * kSet;
 #pragma unroll
-      for (int sa = 1; sa <= 4; ++sa)
+          for (int sa = 1; sa <= 4; ++sa)
 #pragma unroll
-        for (int tb = 1; sa + tb <= 5; ++tb)
+            for (int tb = 1; sa + tb <= 5; ++tb)
 #pragma unroll
-          for (int j = 0; j < D / 32; ++j)
-            umma_i8_ss(tm + (sa + tb - 2) * kI8TileN, a0 + off(D * (sa - 1) + 32 * j, L::A_CH),
-                       b0 + off(D * (tb - 1) + 32 * j, L::B_CH), idesc, (sa == 1 && j == 0) ? 0u : 1u);
-      tc_commit(&bars[1]);
-    }
-  }
-  __syncwarp();
-  if (mbar_wait(&bars[1], 0, abort_flag)) {
-    tc_fence_after();
-    const int row = qb0 + warp * 32 + lane;            // TMEM lane = query block
-    const bool rv = row < nqb;
-    const int eq = rv ? __ldg(q_ex + static_cast<long long>(bh) * nqb + row) : 0;
-    float* srow = s + (static_cast<long long>(bh) * nqb + (rv ? row : 0)) * s_ld;
-    const uint32_t la = tm + (static_cast<uint32_t>(warp * 32) << 16);
-#pragma unroll 1
-    for (int c0 = 0; c0 < kI8TileN; c0 += 16) {
-      uint32_t a2[16], a3[16], a4[16], a5[16];
-      tmem_ld16_wait(la + 0 * kI8TileN + c0, a2);
-      tmem_ld16_wait(la + 1 * kI8TileN + c0, a3);
-      tmem_ld16_wait(la + 2 * kI8TileN + c0, a4);
-      tmem_ld16_wait(la + 3 * kI8TileN + c0, a5);
-      float o[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const long long v = (static_cast<long long>(static_cast<int>(a2[i])) << 21) +
-                            (static_cast<long long>(static_cast<int>(a3[i])) << 14) +
-                            (static_cast<long long>(static_cast<int>(a4[i])) << 7) +
-                            static_cast<long long>(static_cast<int>(a5[i]));
-        const int e = eq + kex[c0 + i] - 35;
-        const double p2 = __longlong_as_double(static_cast<long long>(e + 1023) << 52);
-        o[i] = __double2float_rn(static_cast<double>(v) * p2 * scale);
-      }
-      if (rv) {
-        const int kb = kb0 + c0;
-        if (kb + 16 <= nkb) {
-          float4* dst = reinterpret_cast<float4*>(srow + kb);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (kb + i < nkb) srow[kb + i] = o[i];
+              for (int j = 0; j < D / 32; ++j)
+                umma_i8_ss(acc + (sa + tb - 2) * kI8TileN, a0 + off(D * (sa - 1) + 32 * j, L::A_CH),
+                           b0 + off(D * (tb - 1) + 32 * j, L::B_CH), idesc, (sa == 1 && j == 0) ? 0u : 1u);
+          tc_commit(&b_empty[st]);
+          tc_commit(&acc_full[ab]);
         }
+        if (ok) tc_commit(a_empty);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;                       // 0..7
+    const int quad = warp & 3;                     // TMEM lane quadrant
+    const int hc = ew >> 2;                        // key columns [32 hc, 32 hc + 32) of the tile
+    const uint32_t la = tm + (static_cast<uint32_t>(quad * 32) << 16) + hc * 32;
+    float* tbuf = reinterpret_cast<float*>(smem + L::OFF_T) + ew * 32 * 33;
+    int bt = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < wk.n_items; item += gridDim.x) {
+      int bh, qt, kt0, kt1;
+      decode(item, bh, qt, kt0, kt1);
+      const int row0 = qt * kI8TileM + quad * 32;  // first query block of this warp's rows
+      const int row = row0 + lane;
+      const int eq = row < wk.nqb ? __ldg(q_ex + static_cast<long long>(bh) * wk.nqb + row) : 0;
+      for (int kt = kt0; kt < kt1; ++kt, ++bt) {
+        const int ab = bt & 1;
+        const int kcol = kt * kI8TileN + hc * 32 + lane;   // this lane's key in the store phase
+        const int ek_l = kcol < wk.nkb ? __ldg(k_ex + static_cast<long long>(bh) * wk.nkb + kcol) : 0;
+        if (!(ok = mbar_wait(&acc_full[ab], (bt >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        uint32_t a2[32], a3[32], a4[32], a5[32];
+        const uint32_t base = la + ab * kSet;
+        tmem_ld16(base + 0 * kI8TileN, a2);
+        tmem_ld16(base + 0 * kI8TileN + 16, a2 + 16);
+        tmem_ld16(base + 1 * kI8TileN, a3);
+        tmem_ld16(base + 1 * kI8TileN + 16, a3 + 16);
+        tmem_ld16(base + 2 * kI8TileN, a4);
+        tmem_ld16(base + 2 * kI8TileN + 16, a4 + 16);
+        tmem_ld16(base + 3 * kI8TileN, a5);
+        tmem_ld16(base + 3 * kI8TileN + 16, a5 + 16);
+        tmem_wait_ld();
+        reg_fence16(a2); reg_fence16(a2 + 16);
+        reg_fence16(a3); reg_fence16(a3 + 16);
+        reg_fence16(a4); reg_fence16(a4 + 16);
+        reg_fence16(a5); reg_fence16(a5 + 16);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);    // accumulators are in registers
+        // v = hi 2^14 + lo with hi = acc2 2^7 + acc3 and lo = acc4 2^7 + acc5,
+        // both exact in int32 (|acc2| <= d 127^2 < 2^22, |acc3| < 2^23, ...);
+        // v is then exact in one fp64 fma. The row's factor scale 2^(Eq - 35)
+        // rounds once, and 2^Ek is added to the result's exponent, which is
+        // exact for the score range.
+        const double crow = scale * __longlong_as_double(static_cast<long long>(eq - 35 + 1023) << 52);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int hi = (static_cast<int>(a2[i]) << 7) + static_cast<int>(a3[i]);
+          const int lo = (static_cast<int>(a4[i]) << 7) + static_cast<int>(a5[i]);
+          const double vd = fma(static_cast<double>(hi), 16384.0, static_cast<double>(lo));
+          const double r = vd * crow;
+          const int ek = __shfl_sync(0xFFFFFFFFu, ek_l, i);
+          const double sc = r == 0.0 ? 0.0
+                                     : __hiloint2double(__double2hiint(r) + (ek << 20), __double2loint(r));
+          tbuf[lane * 33 + i] = __double2float_rn(sc);
+        }
+        __syncwarp();
+        // row r of this warp's 32 x 32 block: 32 consecutive keys
+        if (kcol < wk.nkb) {
+#pragma unroll 4
+          for (int r = 0; r < 32; ++r)
+            if (row0 + r < wk.nqb)
+              s[(static_cast<long long>(bh) * wk.nqb + row0 + r) * s_ld + kcol] = tbuf[r * 33 + lane];
+        }
+        __syncwarp();
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tm, kCols);
+    tmem_dealloc(tm, 2 * kSet);
   }
 }
 
@@ -882,14 +974,30 @@ static cudaError_t launch_scores_i8_d(const SliceOut& sl, int BH, int nqb, int n
   if (encode_tensor_map_3d_u8(&mb, sl.k_sl, L::ROW, nkb, BH, 128, kI8TileN) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(score_i8_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid(ceil_div(nkb, kI8TileN), ceil_div(nqb, kI8TileM), BH);
-  score_i8_kernel<D><<<grid, 128, L::SMEM, st>>>(ma, mb, sl.q_ex, sl.k_ex, nqb, nkb, scale, s, s_ld);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  I8Work w;
+  w.nqb = nqb;
+  w.nkb = nkb;
+  w.n_qt = ceil_div(nqb, kI8TileM);
+  w.n_kt = ceil_div(nkb, kI8TileN);
+  // about four items per SM: key tiles per item from the total tile count
+  const long long tiles = static_cast<long long>(BH) * w.n_qt * w.n_kt;
+  long long per = (tiles + 4LL * sms - 1) / (4LL * sms);
+  per = per < 1 ? 1 : (per > w.n_kt ? w.n_kt : per);
+  w.kr_tiles = static_cast<int>(per);
+  w.n_kr = ceil_div(w.n_kt, w.kr_tiles);
+  const long long items = static_cast<long long>(BH) * w.n_qt * w.n_kr;
+  if (items > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  w.n_items = static_cast<int>(items);
+  const int grid = w.n_items < sms ? w.n_items : sms;
+  score_i8_kernel<D><<<grid, kI8Threads, L::SMEM, st>>>(ma, mb, sl.q_ex, sl.k_ex, w, scale, s, s_ld);
   return cudaGetLastError();
 }
 
 cudaError_t launch_scores_i8(const SliceOut& sl, int BH, int nqb, int nkb, int d, double scale,
                              float* s, long long s_ld, cudaStream_t st) {
-  if (nqb > 65535 * kI8TileM || BH > 65535) return cudaErrorInvalidValue;
   return d == 128 ? launch_scores_i8_d<128>(sl, BH, nqb, nkb, scale, s, s_ld, st)
                   : launch_scores_i8_d<64>(sl, BH, nqb, nkb, scale, s, s_ld, st);
 }
