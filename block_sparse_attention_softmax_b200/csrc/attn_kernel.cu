@@ -18,9 +18,10 @@
 // attention 1022 -> 1188 TFLOP/s). The QK that overwrites an S buffer waits for
 // the P V that read P from it.
 //
-//   warp 0       TMA producer of Q (one slot) and K (3-stage ring; a slot is
-//                free once the QK that read it has completed, which is the
-//                same event that fills the S buffer of that tile)
+//   warp 0       TMA producer of Q (two slots, so the next item's Q loads
+//                while the current item runs) and K (2-stage ring; a slot is
+//                free once the QK that read it has completed, the event that
+//                also fills that tile's S buffer)
 //   warp 10      TMA producer of V (2-stage ring; a slot is free once the P V
 //                that read it has completed); one TMA box per 64-key block,
 //                so the two blocks of a tile need not be adjacent
@@ -50,7 +51,9 @@ namespace attn {
 constexpr int kBM = 128;        // query rows per tile
 constexpr int kBN = 128;        // keys per tile (two 64-key blocks)
 constexpr int kSoftWarps = 8;
-constexpr int kKStages = 3;
+constexpr int kQSlots = 2;      // Q of the next item loads while the current one runs
+constexpr int kItemRing = 4;    // item facts the K producer posts ahead of the softmax warps
+constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 constexpr int kSBufs = 3;
 // Column pairs c (of 32 per thread and tile) with bit (c % 8) set take the
@@ -72,12 +75,13 @@ struct Layout {
   static constexpr uint32_t Q_CHUNK = kBM * 128;            // bytes per d-chunk of Q
   static constexpr uint32_t KV_CHUNK = kBN * 128;           // bytes per d-chunk of K/V
   static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
+  static constexpr uint32_t OFF_K = OFF_Q + kQSlots * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + kKStages * TILE_BYTES;
   static constexpr uint32_t OFF_RED = OFF_V + kVStages * TILE_BYTES;
   static constexpr uint32_t RED_BYTES = (2 * 2 + 2) * kBM * 4;   // row max [2][2][128], row sum [2][128]
   static constexpr uint32_t OFF_BAR = OFF_RED + RED_BYTES;
-  static constexpr uint32_t USED = OFF_BAR + 256;
+  static constexpr uint32_t OFF_RING = OFF_BAR + 256;    // item ring [kItemRing][4] int
+  static constexpr uint32_t USED = OFF_RING + 256;
   // at least 120 KB so that a second CTA never shares the SM (all 512 TMEM columns are held)
   static constexpr uint32_t SMEM = (USED + 1024 > 120 * 1024) ? USED + 1024 : 120 * 1024;
 };
@@ -86,12 +90,12 @@ __host__ __device__ constexpr uint32_t tm_s(int b) { return static_cast<uint32_t
 constexpr uint32_t TM_O = 384;
 constexpr uint32_t TM_COLS = 512;
 
-static_assert(kKStages == kSBufs, "a K slot is freed by the S_FULL commit of its tile");
+static_assert(kKStages <= kSBufs, "a K slot is freed by the S_FULL commit of the tile kKStages back");
 
 enum {
-  B_QFULL = 0,                       // Q tile landed in shared memory
-  B_QEMPTY = 1,                      // last QK of the item completed
-  B_KFULL = 2,                       // [kKStages]
+  B_QFULL = 0,                       // [kQSlots] Q tile landed in shared memory
+  B_QEMPTY = B_QFULL + kQSlots,      // [kQSlots] last QK of the item completed
+  B_KFULL = B_QEMPTY + kQSlots,      // [kKStages]
   B_VFULL = B_KFULL + kKStages,      // [kVStages]
   B_SFULL = B_VFULL + kVStages,      // [kSBufs]
   B_PFULL = B_SFULL + kSBufs,        // [kSBufs]
@@ -99,7 +103,9 @@ enum {
                                      // the S buffer and the tile's V slot are free again
   B_OFULL = B_PVDONE + kSBufs,       // last P V of the item completed
   B_OEMPTY = B_OFULL + 1,            // epilogue has copied O out of TMEM
-  B_COUNT = B_OEMPTY + 1
+  B_IFULL = B_OEMPTY + 1,            // [kItemRing] item facts posted by the K producer
+  B_IEMPTY = B_IFULL + kItemRing,    // [kItemRing] item facts read by the softmax warps
+  B_COUNT = B_IEMPTY + kItemRing
 };
 
 // Per-item facts every role derives the same way.
@@ -149,7 +155,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   float* red_max = reinterpret_cast<float*>(smem + L::OFF_RED);   // [2 tile parity][2 halves][128 rows]
   float* red_sum = red_max + 4 * kBM;                              // [2 halves][128 rows]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  static_assert(B_COUNT * 8 + 8 <= 256, "barrier region");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
+  volatile int* item_ring = reinterpret_cast<volatile int*>(smem + L::OFF_RING);   // [kItemRing][item, cnt, tail, -]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -157,8 +165,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   const int n_items = a.BH * a.nqb;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[B_QFULL], 1);
-    mbar_init(&bars[B_QEMPTY], 1);
+    for (int i = 0; i < kQSlots; ++i) {
+      mbar_init(&bars[B_QFULL + i], 1);
+      mbar_init(&bars[B_QEMPTY + i], 1);
+    }
+    for (int i = 0; i < kItemRing; ++i) {
+      mbar_init(&bars[B_IFULL + i], 1);
+      mbar_init(&bars[B_IEMPTY + i], kSoftWarps);
+    }
     mbar_init(&bars[B_OFULL], 1);
     mbar_init(&bars[B_OEMPTY], kSoftWarps);
     for (int i = 0; i < kKStages; ++i) mbar_init(&bars[B_KFULL + i], 1);
@@ -201,11 +215,20 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (it.T == 0) continue;
         const int* row = a.dense ? nullptr : a.kv_idx + (static_cast<long long>(it.bh) * a.nqb + it.qb) * a.nkb;
         if (is_k) {
-          if (!(ok = mbar_wait(&bars[B_QEMPTY], (qi & 1) ^ 1, abort_flag))) break;
-          mbar_arrive_expect_tx(&bars[B_QFULL], L::Q_BYTES);
+          // item facts for the softmax warps (they would otherwise read them
+          // from global memory on their critical path)
+          const int rs = qi % kItemRing;
+          if (!(ok = mbar_wait(&bars[B_IEMPTY + rs], ((qi / kItemRing) & 1) ^ 1, abort_flag))) break;
+          item_ring[rs * 4 + 0] = item;
+          item_ring[rs * 4 + 1] = it.cnt;
+          item_ring[rs * 4 + 2] = it.tail ? 1 : 0;
+          mbar_arrive(&bars[B_IFULL + rs]);
+          const int qs = qi % kQSlots;
+          if (!(ok = mbar_wait(&bars[B_QEMPTY + qs], ((qi / kQSlots) & 1) ^ 1, abort_flag))) break;
+          mbar_arrive_expect_tx(&bars[B_QFULL + qs], L::Q_BYTES);
 #pragma unroll
           for (int c = 0; c < L::NCH; ++c)
-            tma_load_3d(sQ + c * L::Q_CHUNK, &tmQ, &bars[B_QFULL], c * 64, it.qb * a.bq, it.bh);
+            tma_load_3d(sQ + qs * L::Q_BYTES + c * L::Q_CHUNK, &tmQ, &bars[B_QFULL + qs], c * 64, it.qb * a.bq, it.bh);
         }
         for (int t = 0; t < it.T; ++t, ++g) {
           const int s = g % stages;
@@ -213,10 +236,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           const int kb0 = a.dense ? 2 * t : __ldg(row + 2 * t);
           const int kb1 = nblk > 1 ? (a.dense ? 2 * t + 1 : __ldg(row + 2 * t + 1)) : 0;
           // slot reuse: a K slot is free once the QK that read it completed
-          // (S_FULL of that tile), a V slot once the P V that read it completed
-          // (PV_DONE of the tile kVStages back, an S-buffer-indexed barrier)
+          // (S_FULL of the tile kKStages back), a V slot once the P V that read
+          // it completed (PV_DONE of the tile kVStages back); both barriers
+          // are indexed by S buffer
           if (is_k) {
-            if (!(ok = mbar_wait(&bars[B_SFULL + s], ((g / stages) & 1) ^ 1, abort_flag))) break;
+            if (g >= kKStages) {
+              const int gp = g - kKStages;
+              if (!(ok = mbar_wait(&bars[B_SFULL + gp % kSBufs], (gp / kSBufs) & 1, abort_flag))) break;
+            }
           } else if (g >= kVStages) {
             const int gp = g - kVStages;
             if (!(ok = mbar_wait(&bars[B_PVDONE + gp % kSBufs], (gp / kSBufs) & 1, abort_flag))) break;
@@ -231,6 +258,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           }
         }
         ++qi;
+      }
+      if (is_k && ok) {
+        // end of this CTA's items
+        const int rs = qi % kItemRing;
+        if (mbar_wait(&bars[B_IEMPTY + rs], ((qi / kItemRing) & 1) ^ 1, abort_flag)) {
+          item_ring[rs * 4 + 0] = n_items;
+          mbar_arrive(&bars[B_IFULL + rs]);
+        }
       }
     }
   } else if (warp == 1 || warp == kPVWarp) {
@@ -259,8 +294,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       };
       Ring kv{0, is_qk ? kKStages : kVStages, 0};   // K ring (QK) or V ring (PV)
       Ring sb{0, kSBufs, 0};
-      uint32_t phase1 = 0;   // Q_FULL (QK) or O_EMPTY (PV) phase
-      int g = 0;
+      uint32_t phase1 = 0;   // O_EMPTY phase (PV)
+      int g = 0, qi = 0;
       bool ok = true;
       int item = next_nonempty(a, blockIdx.x, gridDim.x, n_items);
       Item it = item < n_items ? load_item(a, item) : Item{};
@@ -273,20 +308,19 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           if (is_qk) {
             if (g >= kSBufs && !(ok = mbar_wait(&bars[B_PVDONE + sb.slot], sb.phase ^ 1u, abort_flag))) break;
             if (!(ok = mbar_wait(&bars[B_KFULL + kv.slot], kv.phase, abort_flag))) break;
-            if (t == 0) {
-              if (!(ok = mbar_wait(&bars[B_QFULL], phase1, abort_flag))) break;
-              phase1 ^= 1u;
-            }
+            const int qs = qi % kQSlots;
+            if (t == 0 && !(ok = mbar_wait(&bars[B_QFULL + qs], (qi / kQSlots) & 1, abort_flag))) break;
             tc_fence_after();
             const uint32_t idesc = two ? idesc_qk2 : idesc_qk1;
+            const uint64_t qd = qdesc0 + ((qs * L::Q_BYTES) >> 4);
             const uint64_t kd = kdesc0 + ((kv.slot * L::TILE_BYTES) >> 4);
             const uint32_t s_tm = tm + tm_s(sb.slot);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              umma_ss(s_tm, qdesc0 + ((((kk >> 2) * L::Q_CHUNK) + (kk & 3) * 32u) >> 4),
+              umma_ss(s_tm, qd + ((((kk >> 2) * L::Q_CHUNK) + (kk & 3) * 32u) >> 4),
                       kd + ((((kk >> 2) * L::KV_CHUNK) + (kk & 3) * 32u) >> 4), idesc, kk > 0 ? 1u : 0u);
             tc_commit(&bars[B_SFULL + sb.slot]);   // S ready, and the K slot free
-            if (t + 1 == it.T) tc_commit(&bars[B_QEMPTY]);
+            if (t + 1 == it.T) tc_commit(&bars[B_QEMPTY + qs]);
           } else {
             if (!(ok = mbar_wait(&bars[B_PFULL + sb.slot], sb.phase, abort_flag))) break;
             if (!(ok = mbar_wait(&bars[B_VFULL + kv.slot], kv.phase, abort_flag))) break;
@@ -307,7 +341,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           kv.next();
           sb.next();
         }
+        if (!ok) break;
         item = nitem;
+        ++qi;
         if (item < n_items) {
           it.bh = item / a.nqb;
           it.qb = item % a.nqb;
@@ -329,19 +365,32 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     int g = 0, qi = 0;
     bool ok = true;
 
-    int item = next_nonempty(a, blockIdx.x, gridDim.x, n_items);
-    // items with no kept block before the first non-empty one
-    for (int z = blockIdx.x; z < item; z += gridDim.x) {
-      const Item it = load_item(a, z);
-      const int grow = it.qb * a.bq + row;
-      if (row < a.bq && grow < a.N) {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(it.bh) * a.N + grow) * D + half * (D / 2));
-        for (int c = 0; c < D / 16; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-        if (a.lse && half == 0) a.lse[static_cast<long long>(it.bh) * a.N + grow] = -INFINITY;
+    int prev = blockIdx.x - static_cast<int>(gridDim.x);   // last item handled
+    while (ok) {
+      // next non-empty item, as posted by the K producer; the items skipped
+      // on the way have no kept block
+      const int rs = qi % kItemRing;
+      if (!(ok = mbar_wait(&bars[B_IFULL + rs], (qi / kItemRing) & 1, abort_flag))) break;
+      const int item = item_ring[rs * 4 + 0];
+      Item it;
+      it.cnt = item_ring[rs * 4 + 1];
+      it.tail = item_ring[rs * 4 + 2] != 0;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_IEMPTY + rs]);
+      for (int z = prev + gridDim.x; z < item; z += gridDim.x) {
+        const Item iz = load_item(a, z);
+        const int gz = iz.qb * a.bq + row;
+        if (row < a.bq && gz < a.N) {
+          uint4* dz = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(iz.bh) * a.N + gz) * D + half * (D / 2));
+          for (int c = 0; c < D / 16; ++c) dz[c] = make_uint4(0, 0, 0, 0);
+          if (a.lse && half == 0) a.lse[static_cast<long long>(iz.bh) * a.N + gz] = -INFINITY;
+        }
       }
-    }
-    while (ok && item < n_items) {
-      const Item it = load_item(a, item);
+      if (item >= n_items) break;
+      prev = item;
+      it.bh = item / a.nqb;
+      it.qb = item % a.nqb;
+      it.T = (it.cnt + 1) >> 1;
       const int grow = it.qb * a.bq + row;
       const bool store = row < a.bq && grow < a.N;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(it.bh) * a.N + grow) * D + half * (D / 2);
@@ -441,7 +490,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (lane == 0) mbar_arrive(&bars[B_PFULL + b]);
       }
       if (!ok) break;
-      const int next = next_nonempty(a, item + gridDim.x, gridDim.x, n_items);
       // ---------------------------------------------------------- epilogue
       if (!(ok = mbar_wait(&bars[B_OFULL], qi & 1, abort_flag))) break;
       tc_fence_after();
@@ -476,17 +524,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       }
       if (store && a.lse && half == 0)
         a.lse[static_cast<long long>(it.bh) * a.N + grow] = (m + log2f(lt)) * 0.69314718055994531f;
-      // items with no kept block up to the next non-empty one
-      for (int z = item + gridDim.x; z < next; z += gridDim.x) {
-        const Item iz = load_item(a, z);
-        const int gz = iz.qb * a.bq + row;
-        if (row < a.bq && gz < a.N) {
-          uint4* dz = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(iz.bh) * a.N + gz) * D + half * (D / 2));
-          for (int c = 0; c < D / 16; ++c) dz[c] = make_uint4(0, 0, 0, 0);
-          if (a.lse && half == 0) a.lse[static_cast<long long>(iz.bh) * a.N + gz] = -INFINITY;
-        }
-      }
-      item = next;
       ++qi;
     }
   }
