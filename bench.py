@@ -41,8 +41,8 @@ METRIC = "sparse_attn_effective_tflops"
 # and O sized). `sources_sha` pins the kernel sources the counters belong to:
 # once they change, traffic is reported as null until a new capture is made.
 ATTN_TRAFFIC_CAPTURE = {
-    "workload": "wan13b_480p", "dram_bytes_read": 302419968, "dram_bytes_write": 82997760,
-    "sources_sha": "a67b05317a9dd7d0",
+    "workload": "wan13b_480p", "dram_bytes_read": 302478592, "dram_bytes_write": 82770176,
+    "sources_sha": "2023a76b34a8fbb8",
     "sources": ("attn_kernel.cu", "sa_device.cuh", "sa_internal.h"),
 }
 
