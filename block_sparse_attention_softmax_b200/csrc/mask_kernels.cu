@@ -8,10 +8,12 @@
 //   score_i8_kernel  slices -> s[bh, qb, kb] = scale * <Qbar, Kbar> on the
 //                    int8 tensor cores (exact s32 slice products, combined in
 //                    int64, scaled in fp64, rounded once to fp32)
-//   select_kernel    one query-block row per warp: radix select of the K_sel-th
-//                    largest score (Top-k), a probability-mass search for the
-//                    Top-p cut when Top-k alone does not reach p, and the
-//                    ascending compacted index list.
+//   select_*_kernel  one query-block row per warp: the K_sel-th largest score
+//                    (Top-k) by a short count search followed by an exact
+//                    search among at most 256 candidates, a probability-mass
+//                    search for the Top-p cut when Top-k alone does not reach
+//                    p, and the ascending compacted index list; the row sits
+//                    in registers (up to 1280 key blocks) or shared memory.
 #include "sa_internal.h"
 
 namespace sa {
@@ -366,17 +368,14 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
 
 // ---------------------------------------------------------------- selection
 // One warp per query-block row; rows of the grid are strided over the warps.
-// Each warp keeps its row's keys and exponentials in its own slice of shared
-// memory, so no block-wide barrier is ever needed.
 //
 //   keys    monotone uint32 image of the fp32 scores (larger score -> larger key)
-//   e       exp(s - max) in fp32; Z and every probability mass in fp64
-//   Top-k   4-pass radix select (8-bit digits, warp histogram with aggregated
-//           atomics) of the K_sel-th largest key; ties at the cut are kept in
-//           ascending block order (ballot prefix counts)
-//   Top-p   only when the Top-k set holds less than p of the mass: bitwise
-//           search for the largest key v with mass(key >= v) >= p * Z, then the
-//           ties at v in block order until the mass is reached
+//   Top-k   the K_sel-th largest key; ties at the cut are kept in ascending
+//           block order (ballot prefix counts)
+//   Top-p   only when the Top-k set holds less than p of the mass (Z and every
+//           mass in fp64): bitwise search for the largest key v with
+//           mass(key >= v) >= p * Z, then the ties at v in block order until
+//           the mass is reached
 //   output  the union is the longer of the two prefixes of the common order;
 //           kept indices are written in ascending order (ballot compaction)
 constexpr int kSelWarpsMax = 8;
@@ -408,185 +407,9 @@ struct Cut {
   int ties;        // elements equal to the threshold that are kept, lowest index first
 };
 
-// The `rank`-th largest key (1-based) of keys[0..n) and how many of its ties to keep.
-__device__ Cut warp_select_rank(const uint32_t* keys, int n, int rank, uint32_t* hist) {
-  const int lane = threadIdx.x & 31;
-  uint32_t prefix = 0, pmask = 0;
-  int need = rank, above = 0;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
-    __syncwarp();
-    for (int base = 0; base < n; base += 32) {
-      const int i = base + lane;
-      const uint32_t key = i < n ? keys[i] : 0u;
-      const bool in = i < n && (key & pmask) == prefix;
-      const uint32_t act = __ballot_sync(0xFFFFFFFFu, in);
-      if (in) {
-        const uint32_t dg = (key >> shift) & 255u;
-        const uint32_t same = __match_any_sync(act, dg);
-        if (lane == __ffs(same) - 1) atomicAdd(&hist[dg], static_cast<uint32_t>(__popc(same)));
-      }
-    }
-    __syncwarp();
-    // lane owns bins [8 lane, 8 lane + 8); suffix counts run from bin 255 down
-    uint32_t c[8];
-    uint32_t run = 0;
-#pragma unroll
-    for (int j = 7; j >= 0; --j) {
-      run += hist[lane * 8 + j];
-      c[j] = run;
-    }
-    uint32_t incl = run;  // inclusive suffix over lanes >= lane
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, incl, o);
-      if (lane + o < 32) incl += y;
-    }
-    const uint32_t higher = incl - run;   // elements in bins of higher lanes
-    int hit = -1;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (static_cast<int>(higher + c[j]) >= need) hit = j;
-    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, hit >= 0);
-    const int src = 31 - __clz(bal);
-    const int hit_s = __shfl_sync(0xFFFFFFFFu, hit, src);
-    uint32_t above_bin = 0;
-    if (lane == src) above_bin = higher + (hit < 7 ? c[hit + 1] : 0u);
-    above_bin = __shfl_sync(0xFFFFFFFFu, above_bin, src);
-    need -= static_cast<int>(above_bin);
-    above += static_cast<int>(above_bin);
-    prefix |= static_cast<uint32_t>(src * 8 + hit_s) << shift;
-    pmask |= 255u << shift;
-    __syncwarp();
-  }
-  return Cut{prefix, above, need};
-}
-
-// Mass (fp64) of the elements whose key is >= v.
-__device__ __forceinline__ double warp_mass_ge(const uint32_t* keys, const float* e, int n, uint32_t v) {
-  const int lane = threadIdx.x & 31;
-  double w = 0.0;
-  for (int i = lane; i < n; i += 32)
-    if (keys[i] >= v) w += static_cast<double>(e[i]);
-  return warp_sum_d(w);
-}
-
-// Smallest m such that the m largest-key weights sum to >= target.
-__device__ Cut warp_select_mass(const uint32_t* keys, const float* e, int n, double target) {
-  const int lane = threadIdx.x & 31;
-  uint32_t v = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = v | (1u << bit);
-    if (warp_mass_ge(keys, e, n, cand) >= target) v = cand;
-  }
-  // strictly above v, and the ties at v
-  int above = 0, nties = 0;
-  double w_above = 0.0;
-  float e_tie = 0.f;
-  for (int i = lane; i < n; i += 32) {
-    const uint32_t key = keys[i];
-    if (key > v) {
-      ++above;
-      w_above += static_cast<double>(e[i]);
-    } else if (key == v) {
-      ++nties;
-      e_tie = e[i];
-    }
-  }
-  above = warp_sum_i(above);
-  nties = warp_sum_i(nties);
-  w_above = warp_sum_d(w_above);
-  e_tie = warp_max(e_tie);            // every tie has the same weight
-  int t = 0;
-  double acc = w_above;
-  while (acc < target && t < nties) {
-    acc += static_cast<double>(e_tie);
-    ++t;
-  }
-  if (acc < target) t = nties;        // rounding kept the total below the target
-  if (above + t == 0) t = 1;
-  return Cut{v, above, t};
-}
-
-__global__ void __launch_bounds__(kSelWarpsMax * 32) select_kernel(
-    const float* __restrict__ s, long long s_ld, int n_rows, int nkb, int k_sel, double topp,
-    int* __restrict__ kv_idx, int* __restrict__ kv_cnt, uint8_t* __restrict__ mask) {
-  extern __shared__ __align__(16) uint8_t sm_sel[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wpc = blockDim.x >> 5;
-  const size_t slice = static_cast<size_t>(nkb) * 8 + 256 * 4;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(sm_sel + warp * slice);
-  float* e = reinterpret_cast<float*>(keys + nkb);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(e + nkb);
-  const uint32_t lt = (1u << lane) - 1u;
-
-  for (int row = blockIdx.x * wpc + warp; row < n_rows; row += gridDim.x * wpc) {
-    const float* srow = s + static_cast<long long>(row) * s_ld;
-    float mx = -INFINITY;
-    for (int i = lane; i < nkb; i += 32) {
-      const float v = __ldg(srow + i);
-      keys[i] = score_key(v);
-      e[i] = v;
-      mx = fmaxf(mx, v);
-    }
-    mx = warp_max(mx);
-    double z = 0.0;
-    for (int i = lane; i < nkb; i += 32) {
-      const float v = expf(e[i] - mx);
-      e[i] = v;
-      z += static_cast<double>(v);
-    }
-    z = warp_sum_d(z);
-    __syncwarp();
-
-    Cut cut{0u, 0, nkb};              // keep everything
-    if (!(topp >= 1.0 || k_sel >= nkb)) {
-      cut = warp_select_rank(keys, nkb, k_sel, hist);
-      const double target = topp * z;
-      // mass of the Top-k set (ties at the cut taken in block order)
-      double wk = 0.0;
-      int tie_before = 0;
-      for (int base = 0; base < nkb; base += 32) {
-        const int i = base + lane;
-        const uint32_t key = i < nkb ? keys[i] : 0u;
-        const bool tie = i < nkb && key == cut.key;
-        const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
-        const bool keep = i < nkb && (key > cut.key || (tie && tie_before + __popc(tb & lt) < cut.ties));
-        if (keep) wk += static_cast<double>(e[i]);
-        tie_before += __popc(tb);
-      }
-      wk = warp_sum_d(wk);
-      if (wk < target) {
-        const Cut cp = warp_select_mass(keys, e, nkb, target);
-        if (cp.above + cp.ties > k_sel) cut = cp;
-      }
-    }
-
-    // ascending compaction of the kept indices
-    int* out = kv_idx + static_cast<long long>(row) * nkb;
-    uint8_t* mrow = mask ? mask + static_cast<long long>(row) * nkb : nullptr;
-    int written = 0, tie_before = 0;
-    for (int base = 0; base < nkb; base += 32) {
-      const int i = base + lane;
-      const uint32_t key = i < nkb ? keys[i] : 0u;
-      const bool tie = i < nkb && key == cut.key;
-      const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
-      const bool keep = i < nkb && (key > cut.key || (tie && tie_before + __popc(tb & lt) < cut.ties));
-      const uint32_t kb = __ballot_sync(0xFFFFFFFFu, keep);
-      if (keep) out[written + __popc(kb & lt)] = i;
-      if (mrow && i < nkb) mrow[i] = keep ? 1 : 0;
-      written += __popc(kb);
-      tie_before += __popc(tb);
-    }
-    if (lane == 0) kv_cnt[row] = written;
-    __syncwarp();
-  }
-}
-
 // ---------------------------------------------------------------- selection, candidate path
-// The same decisions as select_kernel, for rows of at most 32 * KPL key
-// blocks, with the row's scores in registers (element lane + 32 j in x[j]).
+// Rows of at most 32 * KPL key blocks, with the row's scores in registers
+// (element lane + 32 j in x[j]).
 // K_sel is a small fraction of the row, so the exact search runs on a short
 // candidate list instead of the whole row:
 //   1. one pass gives the row max, mean and spread; a value t is then sought
@@ -926,6 +749,284 @@ static cudaError_t launch_select_fast(const float* s, long long s_ld, int n_rows
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- selection, long rows
+// Rows of more than 32 * 40 key blocks: the same candidate path with the row
+// staged once in the warp's shared memory (`xs`) instead of registers; every
+// count pass then reads shared memory. The full-row passes for the uncommon
+// cases read it too.
+__device__ __forceinline__ int smem_count_ge(const float* xs, int n, float t) {
+  const int lane = threadIdx.x & 31;
+  int c = 0;
+#pragma unroll 4
+  for (int i = lane; i < n; i += 32) c += xs[i] >= t ? 1 : 0;
+  return static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, static_cast<unsigned>(c)));
+}
+
+__device__ __forceinline__ int smem_count_key_ge(const float* xs, int n, uint32_t k) {
+  const int lane = threadIdx.x & 31;
+  int c = 0;
+#pragma unroll 4
+  for (int i = lane; i < n; i += 32) c += score_key(xs[i]) >= k ? 1 : 0;
+  return static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, static_cast<unsigned>(c)));
+}
+
+// Weight of the elements kept by `cut` (ties in ascending block order).
+__device__ double smem_cut_mass(const float* xs, int n, const Cut& cut, float mx) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  double w = 0.0;
+  int tie_before = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const float x = i < n ? xs[i] : -INFINITY;
+    const uint32_t key = score_key(x);
+    const bool tie = i < n && key == cut.key;
+    const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
+    const bool keep = i < n && (key > cut.key || (tie && tie_before + __popc(tb & lt) < cut.ties));
+    if (keep) w += static_cast<double>(sel_weight(x, mx));
+    tie_before += __popc(tb);
+  }
+  return warp_sum_d(w);
+}
+
+// Smallest prefix (by key) whose weight reaches target.
+__device__ Cut smem_mass(const float* xs, int n, float mx, double target) {
+  const int lane = threadIdx.x & 31;
+  uint32_t v = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t c = v | (1u << bit);
+    double w = 0.0;
+    for (int i = lane; i < n; i += 32) {
+      const float x = xs[i];
+      if (score_key(x) >= c) w += static_cast<double>(sel_weight(x, mx));
+    }
+    if (warp_sum_d(w) >= target) v = c;
+  }
+  int above = 0, nties = 0;
+  double w_above = 0.0;
+  float e_tie = 0.f;
+  for (int i = lane; i < n; i += 32) {
+    const float x = xs[i];
+    const uint32_t key = score_key(x);
+    if (key > v) {
+      ++above;
+      w_above += static_cast<double>(sel_weight(x, mx));
+    } else if (key == v) {
+      ++nties;
+      e_tie = sel_weight(x, mx);
+    }
+  }
+  above = warp_sum_i(above);
+  nties = warp_sum_i(nties);
+  w_above = warp_sum_d(w_above);
+  e_tie = warp_max(e_tie);            // every tie has the same weight
+  int t = 0;
+  double acc = w_above;
+  while (acc < target && t < nties) {
+    acc += static_cast<double>(e_tie);
+    ++t;
+  }
+  if (acc < target) t = nties;        // rounding kept the total below the target
+  if (above + t == 0) t = 1;
+  return Cut{v, above, t};
+}
+
+// Kept set of a cut over the whole row, in ascending block order.
+__device__ void smem_output(const float* xs, int n, const Cut& cut, int* __restrict__ out,
+                            int* __restrict__ cnt_out, uint8_t* __restrict__ mrow) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  int written = 0, tie_before = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const bool valid = i < n;
+    const uint32_t key = valid ? score_key(xs[i]) : 0u;
+    const bool tie = valid && key == cut.key;
+    const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
+    const bool keep = valid && (key > cut.key || (tie && tie_before + __popc(tb & lt) < cut.ties));
+    const uint32_t kb = __ballot_sync(0xFFFFFFFFu, keep);
+    if (keep) out[written + __popc(kb & lt)] = i;
+    if (mrow && valid) mrow[i] = keep ? 1 : 0;
+    written += __popc(kb);
+    tie_before += __popc(tb);
+  }
+  if (lane == 0) *cnt_out = written;
+}
+
+__device__ void select_row_long(const float* __restrict__ srow, int nkb, int k_sel, double topp,
+                                int* __restrict__ out, int* __restrict__ cnt_out,
+                                uint8_t* __restrict__ mrow, float* xs, uint32_t* ckey, int* cidx) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  float mx = -INFINITY, sum = 0.f, sq = 0.f, ns = 0.f;
+  for (int i = lane; i < nkb; i += 32) {
+    const float v = srow[i];
+    xs[i] = v;
+    mx = fmaxf(mx, v);
+    if (((i >> 5) & 7) == 0) {                 // every eighth column for the mean and spread
+      sum += v;
+      sq = fmaf(v, v, sq);
+      ns += 1.f;
+    }
+  }
+  mx = warp_max(mx);
+  __syncwarp();
+  double z = 0.0;
+  float part = 0.f;
+  int np = 0;
+  for (int i = lane; i < nkb; i += 32) {
+    part += sel_weight(xs[i], mx);             // four weights <= 1 each, exact to 2^-22
+    if (++np == 4) {
+      z += static_cast<double>(part);
+      part = 0.f;
+      np = 0;
+    }
+  }
+  z = warp_sum_d(z + static_cast<double>(part));
+
+  if (topp >= 1.0 || k_sel >= nkb) {
+    smem_output(xs, nkb, Cut{0u, 0, nkb}, out, cnt_out, mrow);   // every finite score's key is > 0
+    return;
+  }
+  const double target = topp * z;
+
+  // ---- 1. a threshold value with K_sel <= count <= kCandMax
+  bool found = false;
+  float t = mx;
+  if (k_sel <= kCandMax) {
+    sum = warp_sum_f(sum);
+    sq = warp_sum_f(sq);
+    ns = warp_sum_f(ns);
+    const float mean = sum / ns;
+    const float sd = sqrtf(fmaxf(sq / ns - mean * mean, 0.f));
+    const int want = min(kCandMax - 32, max(2 * k_sel, k_sel + 32));
+    const float f = fminf(static_cast<float>(want) / nkb, 0.5f);
+    t = fminf(mean + normal_tail_quantile(f) * sd, mx);
+    const float step = fmaxf(sd, 1e-6f * fmaxf(fabsf(mx), 1.f));
+    float tlo = -INFINITY, thi = INFINITY;
+    for (int it = 0; it < 12; ++it) {
+      const int c = smem_count_ge(xs, nkb, t);
+      if (c >= k_sel && c <= kCandMax) {
+        found = true;
+        break;
+      }
+      if (c < k_sel) thi = t;
+      else tlo = t;
+      float nt;
+      if (tlo > -INFINITY && thi < INFINITY) nt = 0.5f * (tlo + thi);
+      else if (thi < INFINITY) nt = thi - step * static_cast<float>(1 << it);
+      else nt = fminf(tlo + step * static_cast<float>(1 << it), mx);
+      if (nt == t || nt == tlo || nt == thi) break;   // no float left between the bounds
+      t = nt;
+    }
+  }
+  if (!found) {
+    uint32_t v = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t c = v | (1u << bit);
+      if (smem_count_key_ge(xs, nkb, c) >= k_sel) v = c;
+    }
+    const int above = v == 0xFFFFFFFFu ? 0 : smem_count_key_ge(xs, nkb, v + 1u);
+    Cut cut{v, above, k_sel - above};
+    if (smem_cut_mass(xs, nkb, cut, mx) < target) {
+      const Cut cp = smem_mass(xs, nkb, mx, target);
+      if (cp.above + cp.ties > k_sel) cut = cp;
+    }
+    smem_output(xs, nkb, cut, out, cnt_out, mrow);
+    return;
+  }
+
+  // ---- 2. candidates in ascending block order, exact search among them
+  int m = 0;
+  for (int base = 0; base < nkb; base += 32) {
+    const int i = base + lane;
+    const float x = i < nkb ? xs[i] : -INFINITY;
+    const bool take = i < nkb && x >= t;
+    const uint32_t b = __ballot_sync(0xFFFFFFFFu, take);
+    if (take) {
+      ckey[m + __popc(b & lt)] = score_key(x);
+      cidx[m + __popc(b & lt)] = i;
+    }
+    m += __popc(b);
+  }
+  __syncwarp();
+  uint32_t ck[kCandPL];
+  uint32_t kand = 0xFFFFFFFFu, kor = 0u;
+#pragma unroll
+  for (int q = 0; q < kCandPL; ++q) {
+    const bool valid = lane + 32 * q < m;
+    ck[q] = valid ? ckey[lane + 32 * q] : 0u;
+    if (valid) {
+      kand &= ck[q];
+      kor |= ck[q];
+    }
+  }
+  kand = __reduce_and_sync(0xFFFFFFFFu, kand);
+  kor = __reduce_or_sync(0xFFFFFFFFu, kor);
+  const uint32_t diff = kand ^ kor;
+  const int top = diff ? 31 - __clz(diff) : -1;
+  uint32_t v = top >= 0 ? (kand & ~(0xFFFFFFFFu >> (31 - top))) : kand;   // common high bits
+  for (int bit = top; bit >= 0; --bit) {
+    const uint32_t c = v | (1u << bit);
+    if (count_ge_u(ck, c) >= k_sel) v = c;
+  }
+  const int above = v == 0xFFFFFFFFu ? 0 : count_ge_u(ck, v + 1u);
+  Cut cut{v, above, k_sel - above};
+  // ---- 3. Top-k mass over the kept candidates
+  double wk = 0.0;
+  int tie_before = 0;
+#pragma unroll
+  for (int q = 0; q < kCandPL; ++q) {
+    const bool valid = lane + 32 * q < m;
+    const bool tie = valid && ck[q] == v;
+    const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
+    const bool keep = valid && (ck[q] > v || (tie && tie_before + __popc(tb & lt) < cut.ties));
+    if (keep) wk += static_cast<double>(sel_weight(key_value(ck[q]), mx));
+    tie_before += __popc(tb);
+  }
+  wk = warp_sum_d(wk);
+  if (wk >= target && mrow == nullptr) {
+    int written = 0;
+    tie_before = 0;
+#pragma unroll
+    for (int q = 0; q < kCandPL; ++q) {
+      const bool valid = lane + 32 * q < m;
+      const bool tie = valid && ck[q] == v;
+      const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
+      const bool keep = valid && (ck[q] > v || (tie && tie_before + __popc(tb & lt) < cut.ties));
+      const uint32_t kb = __ballot_sync(0xFFFFFFFFu, keep);
+      if (keep) out[written + __popc(kb & lt)] = cidx[lane + 32 * q];
+      written += __popc(kb);
+      tie_before += __popc(tb);
+    }
+    if (lane == 0) *cnt_out = written;
+    return;
+  }
+  if (wk < target) {
+    const Cut cp = smem_mass(xs, nkb, mx, target);
+    if (cp.above + cp.ties > k_sel) cut = cp;
+  }
+  smem_output(xs, nkb, cut, out, cnt_out, mrow);
+}
+
+// Per warp: the row (nkb floats), then kCandMax keys and indices.
+__global__ void __launch_bounds__(kSelWarpsMax * 32) select_long_kernel(
+    const float* __restrict__ s, long long s_ld, int n_rows, int nkb, int k_sel, double topp,
+    int* __restrict__ kv_idx, int* __restrict__ kv_cnt, uint8_t* __restrict__ mask, int slice) {
+  extern __shared__ __align__(16) uint8_t sm_long[];
+  const int warp = threadIdx.x >> 5;
+  const int wpc = blockDim.x >> 5;
+  float* xs = reinterpret_cast<float*>(sm_long + static_cast<size_t>(warp) * slice);
+  uint32_t* ckey = reinterpret_cast<uint32_t*>(xs + nkb);
+  int* cidx = reinterpret_cast<int*>(ckey + kCandMax);
+  for (int row = blockIdx.x * wpc + warp; row < n_rows; row += gridDim.x * wpc) {
+    select_row_long(s + static_cast<long long>(row) * s_ld, nkb, k_sel, topp,
+                    kv_idx + static_cast<long long>(row) * nkb, kv_cnt + row,
+                    mask ? mask + static_cast<long long>(row) * nkb : nullptr, xs, ckey, cidx);
+    __syncwarp();
+  }
+}
+
 // ---------------------------------------------------------------- uint8 mask -> lists
 __global__ void __launch_bounds__(kSelWarpsMax * 32) compact_mask_kernel(
     const uint8_t* __restrict__ mask, int n_rows, int nkb, int* __restrict__ kv_idx,
@@ -1009,20 +1110,16 @@ cudaError_t launch_select(const float* s, long long s_ld, int n_rows, int nkb, i
   if (nkb <= 32 * 4) return launch_select_fast<4>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st);
   if (nkb <= 32 * 16) return launch_select_fast<16>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st);
   if (nkb <= 32 * 40) return launch_select_fast<40>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st);
-  const size_t slice = static_cast<size_t>(nkb) * 8 + 256 * 4;
-  int wpc = static_cast<int>((200u * 1024u) / slice);
-  wpc = wpc < 1 ? 1 : (wpc > kSelWarpsMax ? kSelWarpsMax : wpc);
-  const size_t smem = slice * wpc;
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  // longer rows: candidate path with the row in shared memory
+  const int slice = (nkb * 4 + kCandMax * 8 + 15) / 16 * 16;
+  int wpc = (200 * 1024) / slice;
+  wpc = wpc < 1 ? 1 : (wpc > 4 ? 4 : wpc);
+  const size_t smem = static_cast<size_t>(slice) * wpc;
+  cudaError_t e = cudaFuncSetAttribute(select_long_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int want = (n_rows + wpc - 1) / wpc;
-  const int per_sm = static_cast<int>((228u * 1024u) / (smem + 1024));
-  const int cap = sms * (per_sm < 1 ? 1 : per_sm) * 2;
-  const int grid = want < cap ? want : cap;
-  select_kernel<<<grid, wpc * 32, smem, st>>>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask);
+  const int grid = want < 65535 * 16 ? want : 65535 * 16;
+  select_long_kernel<<<grid, wpc * 32, smem, st>>>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, slice);
   return cudaGetLastError();
 }
 

@@ -27,9 +27,19 @@ def _oracle_head_mask(q, k, b, h, bq, bk, topk, topp):
     return oracle.build_mask(_f64(q[b, h]), _f64(k[b, h]), bq, bk, topk, topp)
 
 
+def _assert_same_lists(a, b):
+    assert torch.equal(a["kv_cnt"], b["kv_cnt"])
+    n = a["kv_idx"].shape[-1]
+    valid = torch.arange(n, device=a["kv_idx"].device) < a["kv_cnt"].unsqueeze(-1)
+    assert torch.equal(torch.where(valid, a["kv_idx"], -1), torch.where(valid, b["kv_idx"], -1))
+
+
 def _check_masks(sa, q, k, bq, bk, topk, topp, heads):
     B, H, N, d = q.shape
     out = sa.sa_build_mask(q, k, bq, bk, topk, topp, want_mask=True, want_pools=True)
+    # without the u8 mask the selection emits the kept list from its candidate
+    # set instead of a full-row pass: the lists must be the same
+    _assert_same_lists(out, sa.sa_build_mask(q, k, bq, bk, topk, topp))
     torch.cuda.synchronize()
     idx = out["kv_idx"].cpu().numpy()
     cnt = out["kv_cnt"].cpu().numpy()
@@ -184,6 +194,7 @@ def test_full_size_workload(cuda_lib, name):
     heads = [(0, h) for h in hs]
     qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
     out = sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp, want_mask=True)
+    _assert_same_lists(out, sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp))
     torch.cuda.synchronize()
     idx, cnt = out["kv_idx"].cpu().numpy(), out["kv_cnt"].cpu().numpy()
     gmask = out["mask"].clone()
