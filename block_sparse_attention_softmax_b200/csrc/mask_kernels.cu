@@ -426,8 +426,10 @@ struct Cut {
 // Weights are e^(s - max) by ex2.approx (relative error ~1e-7, an order of
 // magnitude inside the 1e-6 band within which a cumulative sum counts as a
 // tie with p); Z and all masses are summed in fp64.
-constexpr int kCandMax = 256;
+constexpr int kCandMax = 256;                 // candidates of the shared-memory (long row) path
 constexpr int kCandPL = kCandMax / 32;
+constexpr int kRegCandMax = 128;              // candidates of the register path: the first
+constexpr int kRegCandPL = kRegCandMax / 32;  // guess aims near twice K_sel
 
 __device__ __forceinline__ float sel_weight(float x, float mx) {
   return fast_exp2((x - mx) * 1.4426950408889634f);
@@ -556,7 +558,7 @@ __device__ void output_full(const float (&x)[KPL], int nkb, const Cut& cut, int*
   if (lane == 0) *cnt_out = written;
 }
 
-// One query-block row per warp. `ckey`/`cidx` hold kCandMax candidates and
+// One query-block row per warp. `ckey`/`cidx` hold kRegCandMax candidates and
 // `er` 32 * KPL weights, all in this warp's shared memory.
 template <int KPL>
 __device__ void select_row_fast(const float* __restrict__ srow, int nkb, int k_sel, double topp,
@@ -593,22 +595,22 @@ __device__ void select_row_fast(const float* __restrict__ srow, int nkb, int k_s
   }
   const double target = topp * z;
 
-  // ---- 1. a threshold value with K_sel <= count <= kCandMax
+  // ---- 1. a threshold value with K_sel <= count <= kRegCandMax
   bool found = false;
   float t = mx;
-  if (k_sel <= kCandMax) {
+  if (k_sel <= kRegCandMax) {
     sum = warp_sum_f(sum);
     sq = warp_sum_f(sq);
     const float mean = sum / nkb;
     const float sd = sqrtf(fmaxf(sq / nkb - mean * mean, 0.f));
-    const int want = min(kCandMax - 32, max(2 * k_sel, k_sel + 32));
+    const int want = min(kRegCandMax - 32, max(2 * k_sel, k_sel + 32));
     const float f = fminf(static_cast<float>(want) / nkb, 0.5f);
     t = fminf(mean + normal_tail_quantile(f) * sd, mx);
     const float step = fmaxf(sd, 1e-6f * fmaxf(fabsf(mx), 1.f));
     float tlo = -INFINITY, thi = INFINITY;
     for (int it = 0; it < 12; ++it) {
       const int c = count_ge_f(x, t);
-      if (c >= k_sel && c <= kCandMax) {
+      if (c >= k_sel && c <= kRegCandMax) {
         found = true;
         break;
       }
@@ -638,10 +640,10 @@ __device__ void select_row_fast(const float* __restrict__ srow, int nkb, int k_s
       m += __popc(b);
     }
     __syncwarp();
-    uint32_t ck[kCandPL];
+    uint32_t ck[kRegCandPL];
     uint32_t kand = 0xFFFFFFFFu, kor = 0u;
 #pragma unroll
-    for (int q = 0; q < kCandPL; ++q) {
+    for (int q = 0; q < kRegCandPL; ++q) {
       const bool valid = lane + 32 * q < m;
       ck[q] = valid ? ckey[lane + 32 * q] : 0u;
       if (valid) {
@@ -664,7 +666,7 @@ __device__ void select_row_fast(const float* __restrict__ srow, int nkb, int k_s
     double wk = 0.0;
     int tie_before = 0;
 #pragma unroll
-    for (int q = 0; q < kCandPL; ++q) {
+    for (int q = 0; q < kRegCandPL; ++q) {
       const bool valid = lane + 32 * q < m;
       const bool tie = valid && ck[q] == v;
       const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
@@ -677,7 +679,7 @@ __device__ void select_row_fast(const float* __restrict__ srow, int nkb, int k_s
       int written = 0;
       tie_before = 0;
 #pragma unroll
-      for (int q = 0; q < kCandPL; ++q) {
+      for (int q = 0; q < kRegCandPL; ++q) {
         const bool valid = lane + 32 * q < m;
         const bool tie = valid && ck[q] == v;
         const uint32_t tb = __ballot_sync(0xFFFFFFFFu, tie);
@@ -726,8 +728,8 @@ template <int KPL>
 __global__ void __launch_bounds__(kSelFastWarps * 32, 4) select_fast_kernel(
     const float* __restrict__ s, long long s_ld, int n_rows, int nkb, int k_sel, double topp,
     int* __restrict__ kv_idx, int* __restrict__ kv_cnt, uint8_t* __restrict__ mask) {
-  __shared__ uint32_t ckey_all[kSelFastWarps][kCandMax];
-  __shared__ int cidx_all[kSelFastWarps][kCandMax];
+  __shared__ uint32_t ckey_all[kSelFastWarps][kRegCandMax];
+  __shared__ int cidx_all[kSelFastWarps][kRegCandMax];
   __shared__ float e_all[kSelFastWarps][32 * KPL];
   const int warp = threadIdx.x >> 5;
   for (int row = blockIdx.x * kSelFastWarps + warp; row < n_rows; row += gridDim.x * kSelFastWarps) {
