@@ -252,20 +252,33 @@ def run_ours(args, wl, rank, world, local):
     o = torch.empty_like(q)
     ev = []  # (start, end) events around the sparse attention launch
 
-    launches_per_step = 3 + 1 + (4 if wl.linear else 0)
+    # our kernels per step: pool, scores, selection; attention; linear state,
+    # its fixed-order reduction, and the fused output + blend
+    launches_per_step = 3 + 1 + (3 if wl.linear else 0)
+
+    ev_mask, ev_lin = [], []   # (start, end) events around the mask build and the linear branch
+
+    def mark():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        return e
 
     def step(record=False):
+        if record:
+            m0 = mark()
         m = sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp, workspace=ws_mask)
         if record:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
+            e0 = mark()
+            ev_mask.append((m0, e0))
         sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], out=o)
         if record:
-            e1.record()
+            e1 = mark()
             ev.append((e0, e1))
         if wl.linear:
             S, z = sa.sa_linear_branch(q, k, v, workspace=ws_lin)
             sa.sa_blend(o, q, S, z, alpha, out=o, workspace=ws_blend)
+            if record:
+                ev_lin.append((e1, mark()))
         return m
 
     for _ in range(args.warmup):
@@ -288,6 +301,8 @@ def run_ours(args, wl, rank, world, local):
     ms = t0.elapsed_time(t1) / args.steps
     ms_max = max_over_ranks(ms, world, dev)
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    mask_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_mask)
+    lin_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_lin) if ev_lin else None
     sa.sa_device_status(dev)
 
     # comparison points (not part of the step): dense attention through our kernel
@@ -304,6 +319,24 @@ def run_ours(args, wl, rank, world, local):
         e1.record()
         torch.cuda.synchronize()
         dense_ms = e0.elapsed_time(e1) / reps
+    # a library dense attention of the same shape, for context (PyTorch SDPA)
+    sdpa_ms = None
+    if not args.no_dense:
+        try:
+            import torch.nn.functional as F
+            for _ in range(2):
+                F.scaled_dot_product_attention(q, k, v)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            reps = 3
+            for _ in range(reps):
+                F.scaled_dot_product_attention(q, k, v)
+            e1.record()
+            torch.cuda.synchronize()
+            sdpa_ms = e0.elapsed_time(e1) / reps
+        except Exception:
+            sdpa_ms = None
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -329,6 +362,8 @@ def run_ours(args, wl, rank, world, local):
                "d2h_bytes_per_step": q.numel() * 2, "api": "block_sparse_attention (host tensors)"}
 
     hbm, bf16, bf16_s, src = peaks()
+    kept = float(m["kv_cnt"].sum().item())
+    mask_bytes = int(2 * B * H * N * d * 2 + 4 * kept + 4 * B * H * wl.n_qb)
     achieved = ex_flops / (attn_ms * 1e-3) / 1e12
     result = {
         "metric": METRIC, "value": round(world * dense_flops(wl) / (ms_max * 1e-3) / 1e12, 3),
@@ -339,7 +374,10 @@ def run_ours(args, wl, rank, world, local):
                    "block": f"{wl.bq}x{wl.bk}", "topk": wl.topk, "topp": wl.topp,
                    "linear_branch": wl.linear, "parallelism": f"replica x{world}",
                    "l2": "inputs larger than L2 (each tensor >= 774 MB); no flush"},
-        "sparse_attn_ms": round(attn_ms, 4), "dense_attn_ms": None if dense_ms is None else round(dense_ms, 3),
+        "sparse_attn_ms": round(attn_ms, 4), "mask_build_ms": round(mask_ms, 4),
+        "linear_blend_ms": None if lin_ms is None else round(lin_ms, 4),
+        "dense_attn_ms": None if dense_ms is None else round(dense_ms, 3),
+        "torch_sdpa_dense_ms": None if sdpa_ms is None else round(sdpa_ms, 3),
         "speedup_vs_dense": None if dense_ms is None else round(dense_ms / attn_ms, 2),
         "density": round(density, 5), "executed_tflop_per_call": round(ex_flops / 1e12, 4),
         "roofline": {"kernel": "sparse_attn_kernel<128>", "bound": "tensor", "achieved": round(achieved, 1),
@@ -347,6 +385,10 @@ def run_ours(args, wl, rank, world, local):
                      "peak_source": f"{src} bf16 burst", "traffic": attn_traffic(wl),
                      "traffic_unit": "bytes per launch",
                      "traffic_note": "ncu dram read+write of a smaller capture, scaled by B*H*N*d"},
+        "mask_builder_roofline": {"bound": "hbm", "achieved": round(mask_bytes / (mask_ms * 1e-3) / 1e9, 1),
+                                  "peak": hbm, "unit": "GB/s", "frac": round(mask_bytes / (mask_ms * 1e-3) / 1e9 / hbm, 4),
+                                  "bytes_per_call": mask_bytes,
+                                  "bytes_note": "Q and K read once plus the kept kv_idx entries and kv_cnt"},
         "e2e": e2e, "gpu_launches": args.steps * launches_per_step,
         "clocks": clk.summary(),
     }
