@@ -202,27 +202,65 @@ def sa_blend(o_s, q, kv_state, ksum, alpha, out=None, workspace=None):
     return o
 
 
-def block_sparse_attention(q, k, v, bq=128, bk=64, topk=0.05, topp=0.9, alpha=None, scale=0.0,
-                           device=None, out=None):
-    """Whole path: mask, sparse attention and (when alpha is given) the linear
-    branch blended in. Host tensors are copied to the device and the result is
-    copied back into `out` (a pinned host tensor is allocated when out is None);
-    device tensors stay on the device."""
-    host = not q.is_cuda
-    if host:
-        device = device or torch.device("cuda", torch.cuda.current_device())
-        q, k, v = (t.to(device, non_blocking=True) for t in (q, k, v))
-        if alpha is not None:
-            alpha = alpha.to(device, non_blocking=True)
+def _path_on_device(q, k, v, bq, bk, topk, topp, alpha, scale, out=None):
     m = sa_build_mask(q, k, bq, bk, topk, topp, scale)
-    o = sa_sparse_attn_fwd(q, k, v, bq, bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], scale=scale)
+    o = sa_sparse_attn_fwd(q, k, v, bq, bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], scale=scale, out=out)
     if alpha is not None:
         S, z = sa_linear_branch(q, k, v)
         o = sa_blend(o, q, S, z, alpha, out=o)
-    if host:
-        if out is None:
-            out = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        out.copy_(o, non_blocking=True)
-        torch.cuda.current_stream(device).synchronize()
-        return out
     return o
+
+
+def block_sparse_attention(q, k, v, bq=128, bk=64, topk=0.05, topp=0.9, alpha=None, scale=0.0,
+                           device=None, out=None, chunks=8):
+    """Whole path: mask, sparse attention and (when alpha is given) the linear
+    branch blended in. Device tensors stay on the device. Host tensors are
+    copied in, and the result is copied back into `out` (a pinned host tensor
+    is allocated when out is None). Every head is independent, so with host
+    tensors the heads are split into up to `chunks` groups that go through a
+    three-stream pipeline: the copy in of group c + 1, the path on group c and
+    the copy out of group c - 1 overlap. Pinned host tensors make the copies
+    asynchronous."""
+    if q.is_cuda:
+        return _path_on_device(q, k, v, bq, bk, topk, topp, alpha, scale, out)
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    B, H, N, d = q.shape
+    BH = B * H
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    qh, kh, vh, oh = (t.reshape(BH, N, d) for t in (q, k, v, out))
+    dq, dk, dv = (torch.empty((BH, N, d), dtype=t.dtype, device=device) for t in (q, k, v))
+    do = torch.empty((BH, N, d), dtype=q.dtype, device=device)
+    if alpha is not None:
+        # alpha row of each flattened (batch, head)
+        alpha_d = alpha.to(device)[torch.arange(BH, device=device) % H].contiguous()
+    n = max(1, min(int(chunks), BH))
+    per = (BH + n - 1) // n
+    caller = torch.cuda.current_stream(device)
+    s_in, s_run, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    for s in (s_in, s_run, s_out):
+        s.wait_stream(caller)
+    for c in range(n):
+        i0, i1 = c * per, min(BH, (c + 1) * per)
+        if i0 >= i1:
+            break
+        with torch.cuda.stream(s_in):
+            for dst, src in ((dq, qh), (dk, kh), (dv, vh)):
+                dst[i0:i1].copy_(src[i0:i1], non_blocking=True)
+        s_run.wait_stream(s_in)
+        with torch.cuda.stream(s_run):
+            view = lambda t: t[i0:i1].view(1, i1 - i0, N, d)
+            _path_on_device(view(dq), view(dk), view(dv), bq, bk, topk, topp,
+                            None if alpha is None else alpha_d[i0:i1], scale, out=view(do))
+        s_out.wait_stream(s_run)
+        with torch.cuda.stream(s_out):
+            oh[i0:i1].copy_(do[i0:i1], non_blocking=True)
+    # the device buffers were used on the side streams; keep the allocator from
+    # handing them out again before those streams are done with them
+    for t in (dq, dk, dv, do):
+        t.record_stream(s_in)
+        t.record_stream(s_run)
+        t.record_stream(s_out)
+    caller.wait_stream(s_out)
+    caller.synchronize()
+    return out
