@@ -252,9 +252,11 @@ def run_ours(args, wl, rank, world, local):
     o = torch.empty_like(q)
     ev = []  # (start, end) events around the sparse attention launch
 
-    # our kernels per step: pool, scores, selection; attention; linear state,
+    # our kernels per step: pool, row statistics, candidate scores, candidate
+    # selection, the two hand-back launches (return at once when no row was
+    # handed back); attention; linear state,
     # its fixed-order reduction, and the fused output + blend
-    launches_per_step = 3 + 1 + (3 if wl.linear else 0)
+    launches_per_step = 6 + 1 + (3 if wl.linear else 0)
 
     ev_mask, ev_lin = [], []   # (start, end) events around the mask build and the linear branch
 

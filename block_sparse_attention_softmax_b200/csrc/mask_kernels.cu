@@ -134,71 +134,214 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 // and every <a_s, b_t> (d products of |.| <= 127 values) is exact in the
 // tensor core's s32 accumulator. Pairs are grouped by level L = s + t into
 // four accumulators (L = 2..5; pairs with s + t > 5 weigh at most 2^-42 and
-// are dropped), combined exactly as the int64
-//   v = acc2 2^21 + acc3 2^14 + acc4 2^7 + acc5,
-// and the score is v * 2^(Eq + Ek - 35) * scale, rounded once in fp64 and
-// once to fp32. Its error stays near 1e-7 of the score scale, well inside the
-// 1e-6 band within which the mask comparison treats a cut as a tie.
+// are dropped), so that the score is
+//   (acc2 + acc3 2^-7 + acc4 2^-14 + acc5 2^-21) * scale 2^(Eq - 14) * 2^Ek.
+// Each accumulator is exact in fp32; the leading product is split exactly by
+// an fma and the smaller terms are added before one final rounding
+// (score_exact), so a score is within about half an ulp of the exact value:
+// at most 5e-7 for scores below 16, inside the 1e-6 band within which the
+// mask comparison treats a cut as a tie.
 //
 // Persistent CTAs over work items (head, 128 query blocks, a range of 64-key
 // tiles): warp 0 loads the item's query slices (operand A, M = 128) and
 // streams the key-slice tiles (operand B, N = 64) through a 3-stage ring by
 // TMA (128-byte swizzled rows, one box per 128-byte column chunk); warp 1
-// issues the 10 * d / 32 MMAs of a key tile into one of two TMEM accumulator
-// sets; eight epilogue warps (two per TMEM lane quadrant, 32 key columns
-// each) combine the levels, transpose each 32 x 32 block through shared
-// memory and write score rows with coalesced 128-byte stores.
+// issues the MMAs of a key tile into one of two TMEM accumulator sets; eight
+// epilogue warps (two per TMEM lane quadrant, 32 key columns each, so each
+// thread owns one query-block row) consume the accumulators. Three modes:
+//
+//   kScoreWrite  exact scores, transposed through shared memory and written
+//                as the fp32 score matrix with coalesced 128-byte stores;
+//                with a query-tile filter, only the flagged tiles (the rows
+//                the candidate selection handed back)
+//   kScoreStats  the first slice pair only (one level, d / 32 MMAs), an
+//                approximation of the score within about 2^-6 of
+//                sum |q||k|: per row and item, its max, sum and sum of
+//                squares, from which the candidate pass takes a reference
+//                maximum and a threshold t
+//   kScoreCands  exact scores as in kScoreWrite, never stored: per row and
+//                item, the exact max and the partial normaliser
+//                sum e^(s - m_ref) (fp32 pairwise over each 32-column
+//                chunk, fp64 across chunks), and every score >= t appended
+//                to the row's candidate list (one atomic per thread and tile
+//                reserves the slots)
 constexpr int kI8TileM = 128;
 constexpr int kI8TileN = 64;
 constexpr int kI8BStages = 3;
 constexpr int kI8EpiWarps = 8;
 constexpr int kI8Threads = 32 * (2 + kI8EpiWarps);
+constexpr int kMaxKr = 8;               // key ranges per row (bounds the partial arrays)
 
-template <int D>
+enum : int { kScoreWrite = 0, kScoreStats = 1, kScoreCands = 2 };
+
+template <int D, int MODE>
 struct I8Layout {
   static constexpr int ROW = 4 * D;                 // bytes per slice row
-  static constexpr int NCH = ROW / 128;             // 128-byte column chunks
+  static constexpr int NCH = MODE == kScoreStats ? 1 : ROW / 128;   // 128-byte chunks loaded
+  static constexpr int LEVELS = MODE == kScoreStats ? 1 : 4;
+  static constexpr int STAGES = MODE == kScoreStats ? 6 : kI8BStages;   // B ring depth
   static constexpr uint32_t A_CH = kI8TileM * 128;  // bytes of one A chunk
   static constexpr uint32_t B_CH = kI8TileN * 128;
   static constexpr uint32_t A_BYTES = NCH * A_CH;
   static constexpr uint32_t B_BYTES = NCH * B_CH;
   static constexpr uint32_t OFF_A = 0;
   static constexpr uint32_t OFF_B = OFF_A + A_BYTES;
-  static constexpr uint32_t OFF_T = OFF_B + kI8BStages * B_BYTES;      // [epi warps][32][33] fp32
-  static constexpr uint32_t OFF_BAR = OFF_T + kI8EpiWarps * 32 * 33 * 4;
-  static constexpr uint32_t SMEM = OFF_BAR + 128 + 1024;
+  static constexpr uint32_t OFF_T = OFF_B + STAGES * B_BYTES;
+  // kScoreWrite: [epi warps][32][33] fp32 transpose blocks
+  static constexpr uint32_t T_BYTES = MODE == kScoreWrite ? kI8EpiWarps * 32 * 33 * 4 : 0;
+  // [epi warps][32] fp32 column factors 2^Ek of the current tile
+  static constexpr uint32_t OFF_C = OFF_T + T_BYTES;
+  static constexpr uint32_t C_BYTES = kI8EpiWarps * 32 * 4;
+  // kScoreCands: two tiles' scores, [2][32 columns][epilogue threads] fp32,
+  // read back two tiles later for the candidates
+  static constexpr uint32_t OFF_X = OFF_C + C_BYTES;
+  static constexpr uint32_t X_BYTES = MODE == kScoreCands ? 2 * 32 * kI8EpiWarps * 32 * 4 : 0;
+  static constexpr uint32_t OFF_BAR = OFF_X + X_BYTES;
+  static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
 };
 
 struct I8Work {
   int nqb, nkb, n_qt, n_kt, kr_tiles, n_kr, n_items;
 };
 
-template <int D>
+// Partial results of one (row, key range, column half).
+struct __align__(16) ZPart {
+  double z;      // sum of e^(s - m_ref) over the part's columns
+  float mx;      // exact max of the part's scores
+  float pad;
+};
+
+// Buffers of the candidate selection (rows are bh * nqb + query block).
+struct CandBufs {
+  float4* st1;       // [rows][2 kMaxKr] approximate {max, sum, sum of squares, count}
+  ZPart* st2;        // [rows][2 kMaxKr]
+  float2* rowinfo;   // [rows] {m_ref, t}
+  int* cand_cnt;     // [rows][2] scores >= t, and t_lo <= score < t (may exceed the capacities)
+  uint2* cand;       // [rows][c_hi + c_lo] {key, key block}: the list >= t, then the list below
+  int c_hi, c_lo;
+  float zq;          // standard normal quantile with tail mass want / nkb (t)
+  float zq_lo;       // the same for the wider list (t_lo)
+  float p_lo;        // rows whose expected Top-k mass share is below this get the second list
+  int all_cand;      // every key block is a candidate of the first list
+  int* fb_cnt;       // rows handed back to the score-matrix path
+  int* fb_rows;      // [rows]
+  int* tile_flag;    // [BH * n_qt] query tiles holding such rows
+  int n_tile_flags;
+};
+
+// Monotone uint32 image of an fp32 score (larger score -> larger key).
+__device__ __forceinline__ uint32_t score_key(float s) {
+  const uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Row constants of the exact score: c = scale 2^(Eq - 14) as an unevaluated
+// fp32 pair ch + cl, and ch 2^-7, 2^-14, 2^-21 (exact scalings).
+struct RowC {
+  float ch, cl, ch7, ch14, ch21;
+};
+
+__device__ __forceinline__ RowC row_consts(double scale, int eq) {
+  const double c = scale * __longlong_as_double(static_cast<long long>(eq - 14 + 1023) << 52);
+  RowC r;
+  r.ch = static_cast<float>(c);
+  r.cl = static_cast<float>(c - static_cast<double>(r.ch));
+  r.ch7 = r.ch * 0.0078125f;
+  r.ch14 = r.ch * 6.103515625e-05f;
+  r.ch21 = r.ch * 4.76837158203125e-07f;
+  return r;
+}
+
+// 2^e as fp32 for a key-block exponent (clamped to the normal range; blocks
+// beyond it have scores far below the tie band).
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((min(max(e, -126), 127) + 127) << 23); }
+
+// Score without the column factor: (acc2 + acc3 2^-7 + acc4 2^-14 + acc5 2^-21) c.
+// Every accumulator is exact in fp32 (|acc_L| < 2^23); acc2 ch is split
+// exactly into p + e by one fma, the remaining terms (each at most 2^-6 of
+// the leading one) are summed in fp32 and the total rounds once, so the
+// result is within about half an ulp of the exact value.
+__device__ __forceinline__ float score_exact(uint32_t a2, uint32_t a3, uint32_t a4, uint32_t a5, const RowC& c) {
+  const float f2 = static_cast<float>(static_cast<int>(a2));
+  const float f3 = static_cast<float>(static_cast<int>(a3));
+  const float f4 = static_cast<float>(static_cast<int>(a4));
+  const float f5 = static_cast<float>(static_cast<int>(a5));
+  const float p = f2 * c.ch;
+  const float e = fmaf(f2, c.ch, -p);
+  float t = f5 * c.ch21;
+  t = fmaf(f4, c.ch14, t);
+  t = fmaf(f3, c.ch7, t);
+  t = fmaf(f2, c.cl, t);
+  return p + (e + t);
+}
+
+// Candidates of one staged tile whose list slots are reserved.
+struct CandPend {
+  uint32_t h = 0u, l = 0u;   // columns in the first / second list
+  int jh = 0, jl = 0;        // first reserved slot in each list
+  int kc0 = 0;               // key block of column 0
+  uint2* cl = nullptr;       // the row's lists
+  const float* xb = nullptr; // the staged scores
+};
+
+// Writes the candidates of one staged tile (bits of `pend`, slots from j on;
+// slots past cap are counted but not stored) and clears `pend`.
+__device__ __forceinline__ void flush_cands(uint32_t pend, int j, int kc0, const float* xst, uint2* cl, int cap) {
+  if (pend == 0u) return;
+  constexpr int XS = 32 * kI8EpiWarps;
+  uint32_t m = pend;
+  while (m != 0u) {
+    const int i = __ffs(m) - 1;
+    m &= m - 1u;
+    if (j < cap) cl[j] = make_uint2(score_key(xst[i * XS]), static_cast<uint32_t>(kc0 + i));
+    ++j;
+  }
+}
+
+// e^(x - m_ref) as computed for the normaliser and for every candidate mass.
+__device__ __forceinline__ float cand_weight(float x, float mlog) {
+  return fast_exp2(fmaf(x, 1.4426950408889634f, -mlog));
+}
+
+template <int D, int MODE>
 __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_constant__ CUtensorMap tmA,
                                                                  const __grid_constant__ CUtensorMap tmB,
                                                                  const int* __restrict__ q_ex,
                                                                  const int* __restrict__ k_ex, I8Work wk,
                                                                  double scale, float* __restrict__ s,
-                                                                 long long s_ld) {
-  using L = I8Layout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+                                                                 long long s_ld, CandBufs cb) {
+  using L = I8Layout<D, MODE>;
+  if constexpr (MODE == kScoreWrite) {
+    // filtered launch with nothing handed back: leave before any setup
+    if (cb.fb_cnt && *reinterpret_cast<volatile const int*>(cb.fb_cnt) == 0) return;
+  }
+  if constexpr (MODE == kScoreStats) {
+    // clear the hand-back state of this call (read only by later launches)
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < cb.n_tile_flags; i += gridDim.x * blockDim.x)
+      cb.tile_flag[i] = 0;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *cb.fb_cnt = 0;
+  }
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  // 1024-byte aligned (swizzle atoms), derived from the shared array so that
+  // accesses through it stay shared-memory instructions
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* a_full = bars;                        // item's query slices landed
   uint64_t* a_empty = bars + 1;                   // item's last MMA completed
-  uint64_t* b_full = bars + 2;                    // [kI8BStages]
-  uint64_t* b_empty = b_full + kI8BStages;        // [kI8BStages]
-  uint64_t* acc_full = b_empty + kI8BStages;      // [2]
+  uint64_t* b_full = bars + 2;                    // [STAGES]
+  uint64_t* b_empty = b_full + L::STAGES;        // [L::STAGES]
+  uint64_t* acc_full = b_empty + L::STAGES;      // [2]
   uint64_t* acc_empty = acc_full + 2;             // [2] (epilogue warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr uint32_t kSet = 4 * kI8TileN;         // columns of one accumulator set (four levels)
+  constexpr uint32_t kSet = L::LEVELS * kI8TileN;   // columns of one accumulator set
+  constexpr uint32_t kAlloc = 2 * kSet;             // 128 or 512 columns
 
   if (threadIdx.x == 0) {
     mbar_init(a_full, 1);
     mbar_init(a_empty, 1);
-    for (int i = 0; i < kI8BStages; ++i) {
+    for (int i = 0; i < L::STAGES; ++i) {
       mbar_init(&b_full[i], 1);
       mbar_init(&b_empty[i], 1);
     }
@@ -210,7 +353,7 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * kSet);
+    tmem_alloc(tmem_slot, kAlloc);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -218,34 +361,53 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tm = *tmem_slot;
 
-  // work item -> (head, query tile, first and end key tile)
-  auto decode = [&](int item, int& bh, int& qt, int& kt0, int& kt1) {
-    const int kr = item % wk.n_kr;
+  // work item -> (head, query tile, key range, first and end key tile)
+  auto decode = [&](int item, int& bh, int& qt, int& kr, int& kt0, int& kt1) {
+    kr = item % wk.n_kr;
     const int rest = item / wk.n_kr;
     qt = rest % wk.n_qt;
     bh = rest / wk.n_qt;
     kt0 = kr * wk.kr_tiles;
     kt1 = min(wk.n_kt, kt0 + wk.kr_tiles);
   };
+  // every role skips the same items (the flags do not change during the launch)
+  auto skip = [&](int bh, int qt) -> bool {
+    if constexpr (MODE == kScoreWrite) return cb.tile_flag != nullptr && cb.tile_flag[bh * wk.n_qt + qt] == 0;
+    else return false;
+  };
+  // Items of this CTA: a contiguous range (consecutive items mostly share the
+  // query tile, which then stays in shared memory), or for kScoreWrite a
+  // stride of the grid (the few flagged tiles spread over the CTAs).
+  constexpr bool kContig = MODE != kScoreWrite;
+  const int per = kContig ? (wk.n_items + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x) : 1;
+  const int it_begin = kContig ? static_cast<int>(blockIdx.x) * per : static_cast<int>(blockIdx.x);
+  const int it_end = kContig ? min(wk.n_items, it_begin + per) : wk.n_items;
+  const int it_step = kContig ? 1 : static_cast<int>(gridDim.x);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
-      int ic = 0, bt = 0;
+      int ic = 0, bt = 0, pbh = -1, pqt = -1;
       bool ok = true;
-      for (int item = blockIdx.x; ok && item < wk.n_items; item += gridDim.x, ++ic) {
-        int bh, qt, kt0, kt1;
-        decode(item, bh, qt, kt0, kt1);
-        if (!(ok = mbar_wait(a_empty, (ic & 1) ^ 1, abort_flag))) break;
-        mbar_arrive_expect_tx(a_full, L::A_BYTES);
+      for (int item = it_begin; ok && item < it_end; item += it_step) {
+        int bh, qt, kr, kt0, kt1;
+        decode(item, bh, qt, kr, kt0, kt1);
+        if (skip(bh, qt)) continue;
+        if (!kContig || bh != pbh || qt != pqt) {     // another query tile
+          if (!(ok = mbar_wait(a_empty, (ic & 1) ^ 1, abort_flag))) break;
+          mbar_arrive_expect_tx(a_full, L::A_BYTES);
 #pragma unroll
-        for (int c = 0; c < L::NCH; ++c)
-          tma_load_3d(smem + L::OFF_A + c * L::A_CH, &tmA, a_full, c * 128, qt * kI8TileM, bh);
+          for (int c = 0; c < L::NCH; ++c)
+            tma_load_3d(smem + L::OFF_A + c * L::A_CH, &tmA, a_full, c * 128, qt * kI8TileM, bh);
+          ++ic;
+          pbh = bh;
+          pqt = qt;
+        }
         for (int kt = kt0; kt < kt1; ++kt, ++bt) {
-          const int st = bt % kI8BStages;
-          if (!(ok = mbar_wait(&b_empty[st], ((bt / kI8BStages) & 1) ^ 1, abort_flag))) break;
+          const int st = bt % L::STAGES;
+          if (!(ok = mbar_wait(&b_empty[st], ((bt / L::STAGES) & 1) ^ 1, abort_flag))) break;
           mbar_arrive_expect_tx(&b_full[st], L::B_BYTES);
 #pragma unroll
           for (int c = 0; c < L::NCH; ++c)
@@ -263,31 +425,51 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
       auto off = [](int byte, uint32_t chunk_bytes) -> uint32_t {
         return (static_cast<uint32_t>(byte >> 7) * chunk_bytes + static_cast<uint32_t>(byte & 127)) >> 4;
       };
-      int ic = 0, bt = 0;
+      int ic = 0, bt = 0, pbh = -1, pqt = -1;
       bool ok = true;
-      for (int item = blockIdx.x; ok && item < wk.n_items; item += gridDim.x, ++ic) {
-        int bh, qt, kt0, kt1;
-        decode(item, bh, qt, kt0, kt1);
-        if (!(ok = mbar_wait(a_full, ic & 1, abort_flag))) break;
+      for (int item = it_begin; ok && item < it_end; item += it_step) {
+        int bh, qt, kr, kt0, kt1;
+        decode(item, bh, qt, kr, kt0, kt1);
+        if (skip(bh, qt)) continue;
+        if (!kContig || bh != pbh || qt != pqt) {
+          if (!(ok = mbar_wait(a_full, ic & 1, abort_flag))) break;
+          ++ic;
+          pbh = bh;
+          pqt = qt;
+        }
         for (int kt = kt0; kt < kt1; ++kt, ++bt) {
-          const int st = bt % kI8BStages, ab = bt & 1;
-          if (!(ok = mbar_wait(&b_full[st], (bt / kI8BStages) & 1, abort_flag))) break;
+          const int st = bt % L::STAGES, ab = bt & 1;
+          if (!(ok = mbar_wait(&b_full[st], (bt / L::STAGES) & 1, abort_flag))) break;
           if (!(ok = mbar_wait(&acc_empty[ab], ((bt >> 1) & 1) ^ 1, abort_flag))) break;
           tc_fence_after();
           const uint64_t b0 = b00 + ((st * L::B_BYTES) >> 4);
           const uint32_t acc = tm + ab * kSet;
+          if constexpr (MODE == kScoreStats) {
+            // slice 1 of both operands: level 2 only
 #pragma unroll
-          for (int sa = 1; sa <= 4; ++sa)
+            for (int j = 0; j < D / 32; ++j)
+              umma_i8_ss(acc, a0 + off(32 * j, L::A_CH), b0 + off(32 * j, L::B_CH), idesc, j == 0 ? 0u : 1u);
+          } else {
 #pragma unroll
-            for (int tb = 1; sa + tb <= 5; ++tb)
+            for (int sa = 1; sa <= 4; ++sa)
 #pragma unroll
-              for (int j = 0; j < D / 32; ++j)
-                umma_i8_ss(acc + (sa + tb - 2) * kI8TileN, a0 + off(D * (sa - 1) + 32 * j, L::A_CH),
-                           b0 + off(D * (tb - 1) + 32 * j, L::B_CH), idesc, (sa == 1 && j == 0) ? 0u : 1u);
+              for (int tb = 1; sa + tb <= 5; ++tb)
+#pragma unroll
+                for (int j = 0; j < D / 32; ++j)
+                  umma_i8_ss(acc + (sa + tb - 2) * kI8TileN, a0 + off(D * (sa - 1) + 32 * j, L::A_CH),
+                             b0 + off(D * (tb - 1) + 32 * j, L::B_CH), idesc, (sa == 1 && j == 0) ? 0u : 1u);
+          }
           tc_commit(&b_empty[st]);
           tc_commit(&acc_full[ab]);
         }
-        if (ok) tc_commit(a_empty);
+        // release the query tile unless the next item uses it too
+        bool release = true;
+        if (kContig && item + 1 < it_end) {
+          int nbh, nqt, nkr, nk0, nk1;
+          decode(item + 1, nbh, nqt, nkr, nk0, nk1);
+          release = nbh != bh || nqt != qt;
+        }
+        if (ok && release) tc_commit(a_empty);
       }
     }
   } else {
@@ -296,73 +478,272 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
     const int quad = warp & 3;                     // TMEM lane quadrant
     const int hc = ew >> 2;                        // key columns [32 hc, 32 hc + 32) of the tile
     const uint32_t la = tm + (static_cast<uint32_t>(quad * 32) << 16) + hc * 32;
-    float* tbuf = reinterpret_cast<float*>(smem + L::OFF_T) + ew * 32 * 33;
     int bt = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < wk.n_items; item += gridDim.x) {
-      int bh, qt, kt0, kt1;
-      decode(item, bh, qt, kt0, kt1);
+    // kScoreCands: candidates of the last two tiles (p2 two tiles ago, p1 the
+    // previous one), slots reserved, written two tiles later, when the
+    // reserving atomics have returned
+    CandPend p2, p1;
+    for (int item = it_begin; ok && item < it_end; item += it_step) {
+      int bh, qt, kr, kt0, kt1;
+      decode(item, bh, qt, kr, kt0, kt1);
+      if (skip(bh, qt)) continue;
       const int row0 = qt * kI8TileM + quad * 32;  // first query block of this warp's rows
       const int row = row0 + lane;
-      const int eq = row < wk.nqb ? __ldg(q_ex + static_cast<long long>(bh) * wk.nqb + row) : 0;
-      for (int kt = kt0; kt < kt1; ++kt, ++bt) {
-        const int ab = bt & 1;
-        const int kcol = kt * kI8TileN + hc * 32 + lane;   // this lane's key in the store phase
-        const int ek_l = kcol < wk.nkb ? __ldg(k_ex + static_cast<long long>(bh) * wk.nkb + kcol) : 0;
-        if (!(ok = mbar_wait(&acc_full[ab], (bt >> 1) & 1, abort_flag))) break;
-        tc_fence_after();
-        uint32_t a2[32], a3[32], a4[32], a5[32];
-        const uint32_t base = la + ab * kSet;
-        tmem_ld16(base + 0 * kI8TileN, a2);
-        tmem_ld16(base + 0 * kI8TileN + 16, a2 + 16);
-        tmem_ld16(base + 1 * kI8TileN, a3);
-        tmem_ld16(base + 1 * kI8TileN + 16, a3 + 16);
-        tmem_ld16(base + 2 * kI8TileN, a4);
-        tmem_ld16(base + 2 * kI8TileN + 16, a4 + 16);
-        tmem_ld16(base + 3 * kI8TileN, a5);
-        tmem_ld16(base + 3 * kI8TileN + 16, a5 + 16);
-        tmem_wait_ld();
-        reg_fence16(a2); reg_fence16(a2 + 16);
-        reg_fence16(a3); reg_fence16(a3 + 16);
-        reg_fence16(a4); reg_fence16(a4 + 16);
-        reg_fence16(a5); reg_fence16(a5 + 16);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[ab]);    // accumulators are in registers
-        // v = hi 2^14 + lo with hi = acc2 2^7 + acc3 and lo = acc4 2^7 + acc5,
-        // both exact in int32 (|acc2| <= d 127^2 < 2^22, |acc3| < 2^23, ...);
-        // v is then exact in one fp64 fma. The row's factor scale 2^(Eq - 35)
-        // rounds once, and 2^Ek is added to the result's exponent, which is
-        // exact for the score range.
-        const double crow = scale * __longlong_as_double(static_cast<long long>(eq - 35 + 1023) << 52);
+      const bool row_ok = row < wk.nqb;
+      const long long grow = static_cast<long long>(bh) * wk.nqb + row;
+      const int eq = row_ok ? __ldg(q_ex + grow) : 0;
+      // this lane's key-block exponent in tile kt (0 past the row end)
+      auto ld_ek = [&](int kt) -> int {
+        const int kcol = kt * kI8TileN + hc * 32 + lane;
+        return kcol < wk.nkb ? __ldg(k_ex + static_cast<long long>(bh) * wk.nkb + kcol) : 0;
+      };
+      if constexpr (MODE == kScoreWrite) {
+        float* tbuf = reinterpret_cast<float*>(smem + L::OFF_T) + ew * 32 * 33;
+        float* colf = reinterpret_cast<float*>(smem + L::OFF_C) + ew * 32;
+        const RowC rc = row_consts(scale, eq);
+        for (int kt = kt0; kt < kt1; ++kt, ++bt) {
+          const int ab = bt & 1;
+          const int kcol = kt * kI8TileN + hc * 32 + lane;   // this lane's key in the store phase
+          const int ek_l = kcol < wk.nkb ? __ldg(k_ex + static_cast<long long>(bh) * wk.nkb + kcol) : 0;
+          if (!(ok = mbar_wait(&acc_full[ab], (bt >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          uint32_t a2[32], a3[32], a4[32], a5[32];
+          const uint32_t base = la + ab * kSet;
+          tmem_ld16(base + 0 * kI8TileN, a2);
+          tmem_ld16(base + 0 * kI8TileN + 16, a2 + 16);
+          tmem_ld16(base + 1 * kI8TileN, a3);
+          tmem_ld16(base + 1 * kI8TileN + 16, a3 + 16);
+          tmem_ld16(base + 2 * kI8TileN, a4);
+          tmem_ld16(base + 2 * kI8TileN + 16, a4 + 16);
+          tmem_ld16(base + 3 * kI8TileN, a5);
+          tmem_ld16(base + 3 * kI8TileN + 16, a5 + 16);
+          tmem_wait_ld();
+          reg_fence16(a2); reg_fence16(a2 + 16);
+          reg_fence16(a3); reg_fence16(a3 + 16);
+          reg_fence16(a4); reg_fence16(a4 + 16);
+          reg_fence16(a5); reg_fence16(a5 + 16);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);    // accumulators are in registers
+          colf[lane] = pow2f(ek_l);
+          __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int hi = (static_cast<int>(a2[i]) << 7) + static_cast<int>(a3[i]);
-          const int lo = (static_cast<int>(a4[i]) << 7) + static_cast<int>(a5[i]);
-          const double vd = fma(static_cast<double>(hi), 16384.0, static_cast<double>(lo));
-          const double r = vd * crow;
-          const int ek = __shfl_sync(0xFFFFFFFFu, ek_l, i);
-          const double sc = r == 0.0 ? 0.0
-                                     : __hiloint2double(__double2hiint(r) + (ek << 20), __double2loint(r));
-          tbuf[lane * 33 + i] = __double2float_rn(sc);
-        }
-        __syncwarp();
-        // row r of this warp's 32 x 32 block: 32 consecutive keys
-        if (kcol < wk.nkb) {
+          for (int i = 0; i < 32; ++i) tbuf[lane * 33 + i] = score_exact(a2[i], a3[i], a4[i], a5[i], rc) * colf[i];
+          __syncwarp();
+          // row r of this warp's 32 x 32 block: 32 consecutive keys
+          if (kcol < wk.nkb) {
 #pragma unroll 4
-          for (int r = 0; r < 32; ++r)
-            if (row0 + r < wk.nqb)
-              s[(static_cast<long long>(bh) * wk.nqb + row0 + r) * s_ld + kcol] = tbuf[r * 33 + lane];
+            for (int r = 0; r < 32; ++r)
+              if (row0 + r < wk.nqb)
+                s[(static_cast<long long>(bh) * wk.nqb + row0 + r) * s_ld + kcol] = tbuf[r * 33 + lane];
+          }
+          __syncwarp();
         }
-        __syncwarp();
+      } else if constexpr (MODE == kScoreStats) {
+        float* colf = reinterpret_cast<float*>(smem + L::OFF_C) + ew * 32;
+        float vmax = -INFINITY, s0 = 0.f, s1 = 0.f, q0 = 0.f, q1 = 0.f;
+        int nv = 0;
+        int ek_next = kt0 < kt1 ? ld_ek(kt0) : 0;   // exponents one tile ahead
+        for (int kt = kt0; kt < kt1; ++kt, ++bt) {
+          const int ab = bt & 1;
+          const int kc0 = kt * kI8TileN + hc * 32;
+          const int ek = min(max(ek_next, -126), 127);
+          if (kt + 1 < kt1) ek_next = ld_ek(kt + 1);
+          if (!(ok = mbar_wait(&acc_full[ab], (bt >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          uint32_t a2[32];
+          tmem_ld16(la + ab * kSet, a2);
+          tmem_ld16(la + ab * kSet + 16, a2 + 16);
+          tmem_wait_ld();
+          reg_fence16(a2); reg_fence16(a2 + 16);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          colf[lane] = pow2f(ek);
+          __syncwarp();
+          const int nvalid = min(32, wk.nkb - kc0);
+          if (nvalid >= 32) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float2 c = *reinterpret_cast<const float2*>(colf + i);
+              const float v0 = static_cast<float>(static_cast<int>(a2[i])) * c.x;
+              const float v1 = static_cast<float>(static_cast<int>(a2[i + 1])) * c.y;
+              vmax = fmax3(vmax, v0, v1);
+              s0 += v0;
+              s1 += v1;
+              q0 = fmaf(v0, v0, q0);
+              q1 = fmaf(v1, v1, q1);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (i < nvalid) {
+                const float v = static_cast<float>(static_cast<int>(a2[i])) * colf[i];
+                vmax = fmaxf(vmax, v);
+                s0 += v;
+                q0 = fmaf(v, v, q0);
+              }
+            }
+          }
+          nv += max(nvalid, 0);
+          __syncwarp();
+        }
+        if (ok && row_ok) {
+          // approximate score = acc2 2^21 2^(Eq + Ek - 35) scale; 2^Ek applied above
+          const float rowf = static_cast<float>(scale * __longlong_as_double(static_cast<long long>(eq - 14 + 1023) << 52));
+          const float4 o = nv > 0 ? make_float4(vmax * rowf, (s0 + s1) * rowf, (q0 + q1) * rowf * rowf, static_cast<float>(nv))
+                                  : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+          cb.st1[grow * (2 * kMaxKr) + kr * 2 + hc] = o;
+          if (kr == 0 && hc == 0) *reinterpret_cast<int2*>(cb.cand_cnt + 2 * grow) = make_int2(0, 0);
+        }
+      } else {
+        // ---------------------------------------------------------- kScoreCands
+        float* colf = reinterpret_cast<float*>(smem + L::OFF_C) + ew * 32;
+        // reference max and threshold from the row's approximate statistics
+        // (the same arithmetic in every CTA that holds a part of the row)
+        float m_ref = -INFINITY, t = INFINITY, tl = INFINITY;
+        if (row_ok) {
+          const float4* p = cb.st1 + grow * (2 * kMaxKr);
+          float su = 0.f, sq = 0.f, n = 0.f;
+          for (int j = 0; j < 2 * wk.n_kr; ++j) {
+            const float4 a = p[j];
+            m_ref = fmaxf(m_ref, a.x);
+            su += a.y;
+            sq += a.z;
+            n += a.w;
+          }
+          const float mean = su / n;
+          const float var = fmaxf(sq / n - mean * mean, 0.f);
+          const float sd = sqrtf(var);
+          t = cb.all_cand ? -INFINITY : mean + cb.zq * sd;
+          if (!cb.all_cand) {
+            // share of the row's mass (weights e^s) above t if the scores were
+            // N(mean, sd^2): Q((t - mean - sd^2) / sd). Rows where Top-k alone
+            // is expected to hold well over p Z skip the second list.
+            const float share = 0.5f * erfcf((t - mean - sd * sd) / (sd * 1.41421356f));
+            if (!(share >= cb.p_lo)) tl = fminf(t, mean + cb.zq_lo * sd);
+          }
+        }
+        const float mlog = m_ref * 1.4426950408889634f;
+        const RowC rc = row_consts(scale, eq);
+        int* cntp = cb.cand_cnt + 2 * (row_ok ? grow : 0);
+        uint2* cl = cb.cand + (row_ok ? grow : 0) * (cb.c_hi + cb.c_lo);
+        constexpr int XS = 32 * kI8EpiWarps;                  // stride of a staged column
+        float* xst0 = reinterpret_cast<float*>(smem + L::OFF_X) + ew * 32 + lane;
+        double z = 0.0;
+        float mx = -INFINITY;
+        int ek_next = kt0 < kt1 ? ld_ek(kt0) : 0;
+        for (int kt = kt0; kt < kt1; ++kt, ++bt) {
+          const int ab = bt & 1;
+          const int kc0 = kt * kI8TileN + hc * 32;
+          const int ek = ek_next;
+          if (kt + 1 < kt1) ek_next = ld_ek(kt + 1);
+          if (!(ok = mbar_wait(&acc_full[ab], (bt >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t base = la + ab * kSet;
+          const int nvalid = min(32, wk.nkb - kc0);
+          colf[lane] = pow2f(ek);
+          float x[32];
+          uint32_t selm = 0u, sell = 0u;      // columns >= t and >= t_lo; size the reservations and the writes
+          float m = -INFINITY, zt = 0.f;
+          // two halves of 16 columns, so that only 64 accumulator registers are live
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t a2[16], a3[16], a4[16], a5[16];
+            tmem_ld16(base + 0 * kI8TileN + 16 * hh, a2);
+            tmem_ld16(base + 1 * kI8TileN + 16 * hh, a3);
+            tmem_ld16(base + 2 * kI8TileN + 16 * hh, a4);
+            tmem_ld16(base + 3 * kI8TileN + 16 * hh, a5);
+              if (hh == 0) {
+              // while the accumulators arrive: the candidates of two tiles ago
+              flush_cands(p2.h, p2.jh, p2.kc0, p2.xb, p2.cl, cb.c_hi);
+              flush_cands(p2.l, p2.jl, p2.kc0, p2.xb, p2.cl + cb.c_hi, cb.c_lo);
+            }
+            tmem_wait_ld();
+            reg_fence16(a2);
+            reg_fence16(a3);
+            reg_fence16(a4);
+            reg_fence16(a5);
+            if (hh == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&acc_empty[ab]);   // accumulators are in registers
+            } else {
+              __syncwarp();                                  // colf written
+            }
+            float w[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+              const float4 c = *reinterpret_cast<const float4*>(colf + 16 * hh + i);
+              x[16 * hh + i] = score_exact(a2[i], a3[i], a4[i], a5[i], rc) * c.x;
+              x[16 * hh + i + 1] = score_exact(a2[i + 1], a3[i + 1], a4[i + 1], a5[i + 1], rc) * c.y;
+              x[16 * hh + i + 2] = score_exact(a2[i + 2], a3[i + 2], a4[i + 2], a5[i + 2], rc) * c.z;
+              x[16 * hh + i + 3] = score_exact(a2[i + 3], a3[i + 3], a4[i + 3], a5[i + 3], rc) * c.w;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int ii = 16 * hh + i;
+              const bool v = nvalid >= 32 || ii < nvalid;
+              w[i] = v ? cand_weight(x[ii], mlog) : 0.f;
+              selm |= ((v && x[ii] >= t) ? 1u : 0u) << ii;
+              sell |= ((v && x[ii] >= tl) ? 1u : 0u) << ii;
+              m = v ? fmaxf(m, x[ii]) : m;
+            }
+            // pairwise sum of the half's weights (fp32, two lanes per add)
+            uint64_t p2[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) p2[i] = f2_make(w[2 * i], w[2 * i + 1]);
+#pragma unroll
+            for (int h = 4; h > 0; h >>= 1)
+#pragma unroll
+              for (int i = 0; i < h; ++i) p2[i] = fadd2(p2[i], p2[i + h]);
+            float z0, z1;
+            f2_split(p2[0], z0, z1);
+            zt += z0 + z1;
+          }
+          sell &= ~selm;
+          CandPend nw;                            // this tile's (buffer = tile parity, free since p2 is written)
+          if ((selm | sell) != 0u) {
+            if (selm != 0u) nw.jh = atomicAdd(cntp, __popc(selm));      // read two tiles later
+            if (sell != 0u) nw.jl = atomicAdd(cntp + 1, __popc(sell));
+            nw.h = selm;
+            nw.l = sell;
+            nw.kc0 = kc0;
+            nw.cl = cl;
+            float* xb = xst0 + ab * 32 * XS;
+            nw.xb = xb;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) xb[i * XS] = x[i];
+          }
+          p2 = p1;
+          p1 = nw;
+          z += static_cast<double>(zt);        // fp64 across chunks
+          mx = fmaxf(mx, m);
+          __syncwarp();
+        }
+        if (ok && row_ok) {
+          ZPart zp;
+          zp.z = z;
+          zp.mx = mx;
+          zp.pad = 0.f;
+          cb.st2[grow * (2 * kMaxKr) + kr * 2 + hc] = zp;
+          if (kr == 0 && hc == 0) cb.rowinfo[grow] = make_float2(m_ref, t);
+        }
       }
+    }
+    if constexpr (MODE == kScoreCands) {
+      flush_cands(p2.h, p2.jh, p2.kc0, p2.xb, p2.cl, cb.c_hi);
+      flush_cands(p2.l, p2.jl, p2.kc0, p2.xb, p2.cl + cb.c_hi, cb.c_lo);
+      flush_cands(p1.h, p1.jh, p1.kc0, p1.xb, p1.cl, cb.c_hi);
+      flush_cands(p1.l, p1.jl, p1.kc0, p1.xb, p1.cl + cb.c_hi, cb.c_lo);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tm, 2 * kSet);
+    tmem_dealloc(tm, kAlloc);
   }
 }
 
@@ -379,11 +760,6 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
 //   output  the union is the longer of the two prefixes of the common order;
 //           kept indices are written in ascending order (ballot compaction)
 constexpr int kSelWarpsMax = 8;
-
-__device__ __forceinline__ uint32_t score_key(float s) {
-  const uint32_t u = __float_as_uint(s);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -724,15 +1100,20 @@ __device__ void select_row_fast(const float* __restrict__ srow, int nkb, int k_s
 
 constexpr int kSelFastWarps = 4;
 
+// With `rows`, the rows are rows[0 .. *n_rows_dev) (rows handed back by the
+// candidate selection); otherwise 0 .. n_rows.
 template <int KPL>
 __global__ void __launch_bounds__(kSelFastWarps * 32, 4) select_fast_kernel(
     const float* __restrict__ s, long long s_ld, int n_rows, int nkb, int k_sel, double topp,
-    int* __restrict__ kv_idx, int* __restrict__ kv_cnt, uint8_t* __restrict__ mask) {
+    int* __restrict__ kv_idx, int* __restrict__ kv_cnt, uint8_t* __restrict__ mask,
+    const int* __restrict__ rows, const int* __restrict__ n_rows_dev) {
   __shared__ uint32_t ckey_all[kSelFastWarps][kRegCandMax];
   __shared__ int cidx_all[kSelFastWarps][kRegCandMax];
   __shared__ float e_all[kSelFastWarps][32 * KPL];
   const int warp = threadIdx.x >> 5;
-  for (int row = blockIdx.x * kSelFastWarps + warp; row < n_rows; row += gridDim.x * kSelFastWarps) {
+  const int nr = n_rows_dev ? *n_rows_dev : n_rows;
+  for (int ri = blockIdx.x * kSelFastWarps + warp; ri < nr; ri += gridDim.x * kSelFastWarps) {
+    const int row = rows ? rows[ri] : ri;
     select_row_fast<KPL>(s + static_cast<long long>(row) * s_ld, nkb, k_sel, topp,
                          kv_idx + static_cast<long long>(row) * nkb, kv_cnt + row,
                          mask ? mask + static_cast<long long>(row) * nkb : nullptr,
@@ -744,10 +1125,11 @@ __global__ void __launch_bounds__(kSelFastWarps * 32, 4) select_fast_kernel(
 template <int KPL>
 static cudaError_t launch_select_fast(const float* s, long long s_ld, int n_rows, int nkb, int k_sel,
                                       double topp, int* kv_idx, int* kv_cnt, uint8_t* mask,
-                                      cudaStream_t st) {
+                                      const int* rows, const int* n_rows_dev, int grid_cap, cudaStream_t st) {
   const int want = (n_rows + kSelFastWarps - 1) / kSelFastWarps;
-  const int grid = want < 65535 * 8 ? want : 65535 * 8;
-  select_fast_kernel<KPL><<<grid, kSelFastWarps * 32, 0, st>>>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask);
+  const int grid = want < grid_cap ? want : grid_cap;
+  select_fast_kernel<KPL><<<grid, kSelFastWarps * 32, 0, st>>>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt,
+                                                               mask, rows, n_rows_dev);
   return cudaGetLastError();
 }
 
@@ -1014,17 +1396,407 @@ __device__ void select_row_long(const float* __restrict__ srow, int nkb, int k_s
 // Per warp: the row (nkb floats), then kCandMax keys and indices.
 __global__ void __launch_bounds__(kSelWarpsMax * 32) select_long_kernel(
     const float* __restrict__ s, long long s_ld, int n_rows, int nkb, int k_sel, double topp,
-    int* __restrict__ kv_idx, int* __restrict__ kv_cnt, uint8_t* __restrict__ mask, int slice) {
+    int* __restrict__ kv_idx, int* __restrict__ kv_cnt, uint8_t* __restrict__ mask, int slice,
+    const int* __restrict__ rows, const int* __restrict__ n_rows_dev) {
   extern __shared__ __align__(16) uint8_t sm_long[];
   const int warp = threadIdx.x >> 5;
   const int wpc = blockDim.x >> 5;
   float* xs = reinterpret_cast<float*>(sm_long + static_cast<size_t>(warp) * slice);
   uint32_t* ckey = reinterpret_cast<uint32_t*>(xs + nkb);
   int* cidx = reinterpret_cast<int*>(ckey + kCandMax);
-  for (int row = blockIdx.x * wpc + warp; row < n_rows; row += gridDim.x * wpc) {
+  const int nr = n_rows_dev ? *n_rows_dev : n_rows;
+  for (int ri = blockIdx.x * wpc + warp; ri < nr; ri += gridDim.x * wpc) {
+    const int row = rows ? rows[ri] : ri;
     select_row_long(s + static_cast<long long>(row) * s_ld, nkb, k_sel, topp,
                     kv_idx + static_cast<long long>(row) * nkb, kv_cnt + row,
                     mask ? mask + static_cast<long long>(row) * nkb : nullptr, xs, ckey, cidx);
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------- selection from candidate lists
+// One warp per query-block row, after the kScoreStats and kScoreCands passes.
+// The row has two lists: every score >= t (first list), and every score in
+// [t_lo, t) (second list), each complete when its count is within its
+// capacity.
+//   Z       the sum of the row's partial normalisers (fp64, fixed order)
+//   Top-k   the K_sel-th largest key; when the first list holds at least
+//           K_sel scores it holds every score at or above that key
+//           (bitwise search over the bits in which the candidates differ)
+//   Top-p   only when the Top-k mass is below p Z: the largest key u whose
+//           candidate mass reaches p Z, then the ties at u in block order;
+//           the same key as over the whole row as long as the listed
+//           candidates' total mass reaches p Z, because every key above the
+//           list's threshold is listed
+//   output  the union is the longer prefix of the common order; the kept
+//           blocks are set as bits in the warp's shared memory (ties at the
+//           cut in ascending block order) and written as the ascending list
+// Fast path: the first list in registers (up to `cap` entries), when it
+// settles both cuts. Wide path: both lists staged in the warp's shared
+// memory. A row goes back to the score-matrix path (its query tile rescored
+// by kScoreWrite, then the full-row selection) when a list overflowed, when
+// even both lists hold less than p Z or fewer than K_sel scores, or when the
+// reference max is more than 30 from the exact one (weights relative to
+// m_ref could then overflow or lose the row's largest terms).
+struct CandSel {
+  const ZPart* st2;
+  const float2* rowinfo;
+  const int* cand_cnt;
+  const uint2* cand;
+  int c_hi, c_lo, cap, n_parts, nqb, n_qt;
+  int* fb_cnt;
+  int* fb_rows;
+  int* tile_flag;
+};
+constexpr int kCandSelWarps = 8;
+
+__device__ __forceinline__ void hand_back(const CandSel& cs, int row) {
+  if ((threadIdx.x & 31) == 0) {
+    const int p = atomicAdd(cs.fb_cnt, 1);
+    cs.fb_rows[p] = row;
+    cs.tile_flag[(row / cs.nqb) * cs.n_qt + (row % cs.nqb) / kI8TileM] = 1;
+  }
+}
+
+__device__ __forceinline__ double warp_max_d(double v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+// Exclusive prefix sum over the lanes.
+__device__ __forceinline__ int warp_excl_scan(int v) {
+  const int lane = threadIdx.x & 31;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  return x - v;
+}
+
+// Ties at the Top-p key u: how many (in block order) reach the target.
+__device__ __forceinline__ int topp_ties(double w_above, double e_tie, int above, int nties, double target) {
+  int tn = 0;
+  double acc = w_above;
+  while (acc < target && tn < nties) {
+    acc += e_tie;
+    ++tn;
+  }
+  if (acc < target) tn = nties;        // rounding kept the total below the target
+  if (above + tn == 0) tn = 1;
+  return tn;
+}
+
+__device__ __forceinline__ void clear_bits(uint32_t* keep, uint32_t* tieb, int W) {
+  const int lane = threadIdx.x & 31;
+  for (int i = lane; i < W; i += 32) {
+    keep[i] = 0u;
+    tieb[i] = 0u;
+  }
+  __syncwarp();
+}
+
+// Marks one candidate: kept above the cut (or at it when every tie is kept),
+// otherwise a tie at the cut goes to `tieb`.
+__device__ __forceinline__ void mark_bit(uint32_t key, int blk, const Cut& cut, bool all_ties, uint32_t* keep,
+                                         uint32_t* tieb) {
+  const uint32_t bit = 1u << (blk & 31);
+  if (key > cut.key || (key == cut.key && all_ties)) atomicOr(&keep[blk >> 5], bit);
+  else if (key == cut.key) atomicOr(&tieb[blk >> 5], bit);
+}
+
+// The kept set from the bits: the cut.ties lowest-index ties join unless all
+// do, then the ascending list, the optional u8 row and the count.
+__device__ void emit_bits(int nkb, const Cut& cut, bool all_ties, int* __restrict__ out, int* __restrict__ cnt_out,
+                          uint8_t* __restrict__ mrow, uint32_t* keep, const uint32_t* tieb) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();
+  const int W = (nkb + 31) >> 5;
+  const int wpl = (W + 31) >> 5;                // words per lane, in order
+  const int w0 = min(W, lane * wpl), w1 = min(W, w0 + wpl);
+  if (!all_ties) {
+    int c = 0;
+    for (int i = w0; i < w1; ++i) c += __popc(tieb[i]);
+    int before = warp_excl_scan(c);
+    for (int i = w0; i < w1 && before < cut.ties; ++i) {
+      uint32_t b = tieb[i];
+      while (b != 0u && before < cut.ties) {
+        const uint32_t low = b & (0u - b);
+        keep[i] |= low;
+        b ^= low;
+        ++before;
+      }
+    }
+    __syncwarp();
+  }
+  int c = 0;
+  for (int i = w0; i < w1; ++i) c += __popc(keep[i]);
+  int pos = warp_excl_scan(c);
+  const int total = __shfl_sync(0xFFFFFFFFu, pos + c, 31);
+  for (int i = w0; i < w1; ++i) {
+    uint32_t b = keep[i];
+    while (b != 0u) {
+      out[pos++] = i * 32 + (__ffs(b) - 1);
+      b &= b - 1u;
+    }
+  }
+  if (mrow)
+    for (int i = lane; i < nkb; i += 32) mrow[i] = static_cast<uint8_t>((keep[i >> 5] >> (i & 31)) & 1u);
+  if (lane == 0) *cnt_out = total;
+}
+
+// Fast path over the first list (cnt <= 32 CPL entries) in registers.
+// Returns false, having written nothing, when the Top-p prefix needs more
+// than the first list.
+template <int CPL>
+__device__ bool select_cand_fast(const uint2* cl, int cnt, int nkb, int k_sel, double target, float mlog,
+                                 int* __restrict__ out, int* __restrict__ cnt_out, uint8_t* __restrict__ mrow,
+                                 uint32_t* keep, uint32_t* tieb) {
+  const int lane = threadIdx.x & 31;
+  uint32_t ck[CPL];
+  int ci[CPL];
+  double wd[CPL];
+  uint32_t kand = 0xFFFFFFFFu, kor = 0u;
+#pragma unroll
+  for (int q = 0; q < CPL; ++q) {
+    const int sidx = lane + 32 * q;
+    ck[q] = 0u;                                 // no finite score has key 0
+    ci[q] = 0;
+    wd[q] = 0.0;
+    if (sidx < cnt) {
+      const uint2 e = cl[sidx];
+      ck[q] = e.x;
+      ci[q] = static_cast<int>(e.y);
+      wd[q] = static_cast<double>(cand_weight(key_value(e.x), mlog));
+      kand &= e.x;
+      kor |= e.x;
+    }
+  }
+  kand = __reduce_and_sync(0xFFFFFFFFu, kand);
+  kor = __reduce_or_sync(0xFFFFFFFFu, kor);
+  const uint32_t diff = kand ^ kor;
+  const int top = diff ? 31 - __clz(diff) : -1;
+  const uint32_t pre = top >= 0 ? (kand & ~(0xFFFFFFFFu >> (31 - top))) : kand;   // common high bits
+  // ---- Top-k
+  uint32_t v = pre;
+  for (int bit = top; bit >= 0; --bit) {
+    const uint32_t c = v | (1u << bit);
+    if (count_ge_u(ck, c) >= k_sel) v = c;
+  }
+  const int above = v == 0xFFFFFFFFu ? 0 : count_ge_u(ck, v + 1u);
+  Cut cut{v, above, k_sel - above};
+  double wa = 0.0, wt = 0.0, ev = 0.0;
+  int nv = 0;
+#pragma unroll
+  for (int q = 0; q < CPL; ++q) {
+    wt += wd[q];
+    if (ck[q] > v) {
+      wa += wd[q];
+    } else if (ck[q] == v) {
+      ev = wd[q];
+      ++nv;
+    }
+  }
+  wa = warp_sum_d(wa);
+  ev = warp_max_d(ev);                          // every tie has the same weight
+  nv = warp_sum_i(nv);
+  int n_cut = nv;                               // elements equal to the cut key
+  if (wa + static_cast<double>(cut.ties) * ev < target) {
+    wt = warp_sum_d(wt);
+    if (wt < target) return false;
+    // ---- Top-p: the largest key u with mass(key >= u) >= target
+    uint32_t u = pre;
+    for (int bit = top; bit >= 0; --bit) {
+      const uint32_t c = u | (1u << bit);
+      double m = 0.0;
+#pragma unroll
+      for (int q = 0; q < CPL; ++q)
+        if (ck[q] >= c) m += wd[q];
+      if (warp_sum_d(m) >= target) u = c;
+    }
+    int pa = 0, nu = 0;
+    double wpa = 0.0, eu = 0.0;
+#pragma unroll
+    for (int q = 0; q < CPL; ++q) {
+      if (ck[q] > u) {
+        ++pa;
+        wpa += wd[q];
+      } else if (ck[q] == u) {
+        ++nu;
+        eu = wd[q];
+      }
+    }
+    pa = warp_sum_i(pa);
+    nu = warp_sum_i(nu);
+    wpa = warp_sum_d(wpa);
+    eu = warp_max_d(eu);
+    const int tn = topp_ties(wpa, eu, pa, nu, target);
+    if (pa + tn > k_sel) {
+      cut = Cut{u, pa, tn};
+      n_cut = nu;
+    }
+  }
+  const bool all_ties = cut.ties >= n_cut;
+  clear_bits(keep, tieb, (nkb + 31) >> 5);
+#pragma unroll
+  for (int q = 0; q < CPL; ++q)
+    if (ck[q] != 0u) mark_bit(ck[q], ci[q], cut, all_ties, keep, tieb);
+  emit_bits(nkb, cut, all_ties, out, cnt_out, mrow, keep, tieb);
+  return true;
+}
+
+// Wide path: both lists (nh + nl entries) staged in `stg`. Returns false,
+// having written nothing, when they hold less than the target mass.
+__device__ bool select_cand_wide(const uint2* cl, int c_hi, int nh, int nl, int nkb, int k_sel, double target,
+                                 float mlog, int* __restrict__ out, int* __restrict__ cnt_out,
+                                 uint8_t* __restrict__ mrow, uint32_t* keep, uint32_t* tieb, uint2* stg) {
+  const int lane = threadIdx.x & 31;
+  const int n = nh + nl;
+  uint32_t kand = 0xFFFFFFFFu, kor = 0u;
+  double wt = 0.0;
+  for (int i = lane; i < n; i += 32) {
+    const uint2 e = i < nh ? cl[i] : cl[c_hi + (i - nh)];
+    stg[i] = e;
+    kand &= e.x;
+    kor |= e.x;
+    wt += static_cast<double>(cand_weight(key_value(e.x), mlog));
+  }
+  __syncwarp();
+  kand = __reduce_and_sync(0xFFFFFFFFu, kand);
+  kor = __reduce_or_sync(0xFFFFFFFFu, kor);
+  wt = warp_sum_d(wt);
+  const uint32_t diff = kand ^ kor;
+  const int top = diff ? 31 - __clz(diff) : -1;
+  const uint32_t pre = top >= 0 ? (kand & ~(0xFFFFFFFFu >> (31 - top))) : kand;
+  auto count_ge = [&](uint32_t c) -> int {
+    int k = 0;
+    for (int i = lane; i < n; i += 32) k += stg[i].x >= c ? 1 : 0;
+    return static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, static_cast<unsigned>(k)));
+  };
+  // ---- Top-k
+  uint32_t v = pre;
+  for (int bit = top; bit >= 0; --bit) {
+    const uint32_t c = v | (1u << bit);
+    if (count_ge(c) >= k_sel) v = c;
+  }
+  const int above = v == 0xFFFFFFFFu ? 0 : count_ge(v + 1u);
+  Cut cut{v, above, k_sel - above};
+  double wa = 0.0, ev = 0.0;
+  int nv = 0;
+  for (int i = lane; i < n; i += 32) {
+    const uint32_t key = stg[i].x;
+    if (key > v) {
+      wa += static_cast<double>(cand_weight(key_value(key), mlog));
+    } else if (key == v) {
+      ev = static_cast<double>(cand_weight(key_value(key), mlog));
+      ++nv;
+    }
+  }
+  wa = warp_sum_d(wa);
+  ev = warp_max_d(ev);
+  nv = warp_sum_i(nv);
+  int n_cut = nv;
+  if (wa + static_cast<double>(cut.ties) * ev < target) {
+    if (wt < target) return false;
+    // ---- Top-p
+    uint32_t u = pre;
+    for (int bit = top; bit >= 0; --bit) {
+      const uint32_t c = u | (1u << bit);
+      double m = 0.0;
+      for (int i = lane; i < n; i += 32) {
+        const uint32_t key = stg[i].x;
+        if (key >= c) m += static_cast<double>(cand_weight(key_value(key), mlog));
+      }
+      if (warp_sum_d(m) >= target) u = c;
+    }
+    int pa = 0, nu = 0;
+    double wpa = 0.0, eu = 0.0;
+    for (int i = lane; i < n; i += 32) {
+      const uint32_t key = stg[i].x;
+      if (key > u) {
+        ++pa;
+        wpa += static_cast<double>(cand_weight(key_value(key), mlog));
+      } else if (key == u) {
+        ++nu;
+        eu = static_cast<double>(cand_weight(key_value(key), mlog));
+      }
+    }
+    pa = warp_sum_i(pa);
+    nu = warp_sum_i(nu);
+    wpa = warp_sum_d(wpa);
+    eu = warp_max_d(eu);
+    const int tn = topp_ties(wpa, eu, pa, nu, target);
+    if (pa + tn > k_sel) {
+      cut = Cut{u, pa, tn};
+      n_cut = nu;
+    }
+  }
+  const bool all_ties = cut.ties >= n_cut;
+  clear_bits(keep, tieb, (nkb + 31) >> 5);
+  for (int i = lane; i < n; i += 32) mark_bit(stg[i].x, static_cast<int>(stg[i].y), cut, all_ties, keep, tieb);
+  emit_bits(nkb, cut, all_ties, out, cnt_out, mrow, keep, tieb);
+  return true;
+}
+
+template <int CPL>
+__device__ void select_cand_row(const CandSel& cs, int row, int nkb, int k_sel, double topp,
+                                int* __restrict__ out, int* __restrict__ cnt_out, uint8_t* __restrict__ mrow,
+                                uint32_t* keep, uint32_t* tieb, uint2* stg) {
+  const int lane = threadIdx.x & 31;
+  if (topp >= 1.0 || k_sel >= nkb) {          // every block (every finite score)
+    for (int i = lane; i < nkb; i += 32) {
+      out[i] = i;
+      if (mrow) mrow[i] = 1;
+    }
+    if (lane == 0) *cnt_out = nkb;
+    return;
+  }
+  double zp = 0.0;
+  float mxp = -INFINITY;
+  if (lane < cs.n_parts) {
+    const ZPart p = cs.st2[static_cast<long long>(row) * (2 * kMaxKr) + lane];
+    zp = p.z;
+    mxp = p.mx;
+  }
+  const double Z = warp_sum_d(zp);
+  const float mx = warp_max(mxp);
+  const float m_ref = cs.rowinfo[row].x;
+  const int2 cnt = *reinterpret_cast<const int2*>(cs.cand_cnt + 2 * static_cast<long long>(row));
+  if (!(fabsf(mx - m_ref) <= 30.f && Z > 0.0)) {   // NaN fails too
+    hand_back(cs, row);
+    return;
+  }
+  const float mlog = m_ref * 1.4426950408889634f;
+  const double target = topp * Z;
+  const uint2* cl = cs.cand + static_cast<long long>(row) * (cs.c_hi + cs.c_lo);
+  if (cnt.x >= k_sel && cnt.x <= cs.cap &&
+      select_cand_fast<CPL>(cl, cnt.x, nkb, k_sel, target, mlog, out, cnt_out, mrow, keep, tieb))
+    return;
+  if (cnt.x <= cs.c_hi && cnt.y <= cs.c_lo && cnt.x + cnt.y >= k_sel &&
+      select_cand_wide(cl, cs.c_hi, cnt.x, cnt.y, nkb, k_sel, target, mlog, out, cnt_out, mrow, keep, tieb, stg))
+    return;
+  hand_back(cs, row);
+}
+
+// Per warp: two bit rows of ceil(nkb / 32) words (kept, ties at the cut),
+// then c_hi + c_lo staged candidates.
+template <int CPL>
+__global__ void __launch_bounds__(kCandSelWarps * 32) select_cand_kernel(
+    CandSel cs, int n_rows, int nkb, int k_sel, double topp, int* __restrict__ kv_idx,
+    int* __restrict__ kv_cnt, uint8_t* __restrict__ mask) {
+  extern __shared__ __align__(16) uint32_t cand_smem[];
+  const int warp = threadIdx.x >> 5;
+  const int W = (nkb + 31) >> 5;
+  const int bw = (2 * W + 3) / 4 * 4;                          // bit words, 16-byte multiple
+  const int per_warp = bw + 2 * (cs.c_hi + cs.c_lo);
+  uint32_t* keep = cand_smem + static_cast<size_t>(warp) * per_warp;
+  uint32_t* tieb = keep + W;
+  uint2* stg = reinterpret_cast<uint2*>(keep + bw);
+  for (int row = blockIdx.x * kCandSelWarps + warp; row < n_rows; row += gridDim.x * kCandSelWarps) {
+    select_cand_row<CPL>(cs, row, nkb, k_sel, topp, kv_idx + static_cast<long long>(row) * nkb, kv_cnt + row,
+                         mask ? mask + static_cast<long long>(row) * nkb : nullptr, keep, tieb, stg);
     __syncwarp();
   }
 }
@@ -1068,15 +1840,14 @@ cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, int 
   return cudaGetLastError();
 }
 
-template <int D>
-static cudaError_t launch_scores_i8_d(const SliceOut& sl, int BH, int nqb, int nkb, double scale,
-                                      float* s, long long s_ld, cudaStream_t st) {
-  using L = I8Layout<D>;
-  CUtensorMap ma, mb;
-  if (encode_tensor_map_3d_u8(&ma, sl.q_sl, L::ROW, nqb, BH, 128, kI8TileM) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  if (encode_tensor_map_3d_u8(&mb, sl.k_sl, L::ROW, nkb, BH, 128, kI8TileN) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(score_i8_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
-  if (e != cudaSuccess) return e;
+// Work split of the score kernels: about four items per SM and at most
+// kMaxKr key ranges per row.
+struct I8Launch {
+  I8Work w;
+  int grid;
+};
+
+static cudaError_t i8_launch(int BH, int nqb, int nkb, I8Launch* out) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1085,33 +1856,63 @@ static cudaError_t launch_scores_i8_d(const SliceOut& sl, int BH, int nqb, int n
   w.nkb = nkb;
   w.n_qt = ceil_div(nqb, kI8TileM);
   w.n_kt = ceil_div(nkb, kI8TileN);
-  // about four items per SM: key tiles per item from the total tile count
   const long long tiles = static_cast<long long>(BH) * w.n_qt * w.n_kt;
   long long per = (tiles + 4LL * sms - 1) / (4LL * sms);
+  const long long per_min = (w.n_kt + kMaxKr - 1) / kMaxKr;
+  per = per < per_min ? per_min : per;
   per = per < 1 ? 1 : (per > w.n_kt ? w.n_kt : per);
   w.kr_tiles = static_cast<int>(per);
   w.n_kr = ceil_div(w.n_kt, w.kr_tiles);
   const long long items = static_cast<long long>(BH) * w.n_qt * w.n_kr;
   if (items > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   w.n_items = static_cast<int>(items);
-  const int grid = w.n_items < sms ? w.n_items : sms;
-  score_i8_kernel<D><<<grid, kI8Threads, L::SMEM, st>>>(ma, mb, sl.q_ex, sl.k_ex, w, scale, s, s_ld);
+  out->w = w;
+  out->grid = w.n_items < sms ? w.n_items : sms;
+  return cudaSuccess;
+}
+
+template <int D>
+static cudaError_t i8_maps(const SliceOut& sl, int BH, int nqb, int nkb, CUtensorMap* ma, CUtensorMap* mb) {
+  constexpr int ROW = 4 * D;
+  if (encode_tensor_map_3d_u8(ma, sl.q_sl, ROW, nqb, BH, 128, kI8TileM) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (encode_tensor_map_3d_u8(mb, sl.k_sl, ROW, nkb, BH, 128, kI8TileN) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  return cudaSuccess;
+}
+
+template <int D, int MODE>
+static cudaError_t launch_i8(const CUtensorMap& ma, const CUtensorMap& mb, const SliceOut& sl, const I8Launch& il,
+                             double scale, float* s, long long s_ld, const CandBufs& cb, cudaStream_t st) {
+  using L = I8Layout<D, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(score_i8_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+  if (e != cudaSuccess) return e;
+  score_i8_kernel<D, MODE><<<il.grid, kI8Threads, L::SMEM, st>>>(ma, mb, sl.q_ex, sl.k_ex, il.w, scale, s, s_ld, cb);
   return cudaGetLastError();
 }
 
 cudaError_t launch_scores_i8(const SliceOut& sl, int BH, int nqb, int nkb, int d, double scale,
                              float* s, long long s_ld, cudaStream_t st) {
-  return d == 128 ? launch_scores_i8_d<128>(sl, BH, nqb, nkb, scale, s, s_ld, st)
-                  : launch_scores_i8_d<64>(sl, BH, nqb, nkb, scale, s, s_ld, st);
+  I8Launch il;
+  cudaError_t e = i8_launch(BH, nqb, nkb, &il);
+  if (e != cudaSuccess) return e;
+  CUtensorMap ma, mb;
+  const CandBufs none{};
+  if (d == 128) {
+    if ((e = i8_maps<128>(sl, BH, nqb, nkb, &ma, &mb)) != cudaSuccess) return e;
+    return launch_i8<128, kScoreWrite>(ma, mb, sl, il, scale, s, s_ld, none, st);
+  }
+  if ((e = i8_maps<64>(sl, BH, nqb, nkb, &ma, &mb)) != cudaSuccess) return e;
+  return launch_i8<64, kScoreWrite>(ma, mb, sl, il, scale, s, s_ld, none, st);
 }
 
 cudaError_t launch_select(const float* s, long long s_ld, int n_rows, int nkb, int k_sel,
                           double topp, int* kv_idx, int* kv_cnt, uint8_t* mask,
-                          cudaStream_t st) {
+                          cudaStream_t st, const int* rows, const int* n_rows_dev) {
+  // with a device-side row count the grid is a fixed size, strided over the rows
+  const int cap8 = rows ? 148 * 8 : 65535 * 8;
   // rows of up to 40 blocks per lane: candidate path with the row in registers
-  if (nkb <= 32 * 4) return launch_select_fast<4>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st);
-  if (nkb <= 32 * 16) return launch_select_fast<16>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st);
-  if (nkb <= 32 * 40) return launch_select_fast<40>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st);
+  if (nkb <= 32 * 4) return launch_select_fast<4>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, rows, n_rows_dev, cap8, st);
+  if (nkb <= 32 * 16) return launch_select_fast<16>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, rows, n_rows_dev, cap8, st);
+  if (nkb <= 32 * 40) return launch_select_fast<40>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, rows, n_rows_dev, cap8, st);
   // longer rows: candidate path with the row in shared memory
   const int slice = (nkb * 4 + kCandMax * 8 + 15) / 16 * 16;
   int wpc = (200 * 1024) / slice;
@@ -1120,9 +1921,120 @@ cudaError_t launch_select(const float* s, long long s_ld, int n_rows, int nkb, i
   cudaError_t e = cudaFuncSetAttribute(select_long_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int want = (n_rows + wpc - 1) / wpc;
-  const int grid = want < 65535 * 16 ? want : 65535 * 16;
-  select_long_kernel<<<grid, wpc * 32, smem, st>>>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, slice);
+  const int cap16 = rows ? 148 * 16 : 65535 * 16;
+  const int grid = want < cap16 ? want : cap16;
+  select_long_kernel<<<grid, wpc * 32, smem, st>>>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, slice,
+                                                   rows, n_rows_dev);
   return cudaGetLastError();
+}
+
+// z with P(Z > z) = f for a standard normal Z (bisection on erfc, host fp64).
+static double normal_upper_quantile(double f) {
+  double lo = -40.0, hi = 40.0;
+  for (int i = 0; i < 200; ++i) {
+    const double mid = 0.5 * (lo + hi);
+    if (0.5 * erfc(mid / sqrt(2.0)) > f) lo = mid;
+    else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+CandPlan cand_plan(int k_sel, int nkb, long long s_ld) {
+  // the lists share the score rows' memory: cand_row_bytes per row
+  const long long per_row = cand_row_bytes(s_ld);
+  long long store = per_row / 8 / 32 * 32;
+  store = store > 2048 ? 2048 : store;
+  int lim = 128;
+  while (lim < 1024 && 2LL * lim <= store) lim *= 2;
+  CandPlan p;
+  p.want = k_sel + (k_sel / 2 > 32 ? k_sel / 2 : 32);
+  p.cap = 128;
+  while (p.cap < lim && p.cap < 1.6 * p.want) p.cap *= 2;
+  p.all_cand = nkb <= p.cap ? 1 : 0;
+  const long long half = store / 2 / 32 * 32;
+  p.c_hi = static_cast<int>(2LL * p.cap < half ? 2LL * p.cap : (half > p.cap ? half : p.cap));
+  p.c_lo = static_cast<int>(store - p.c_hi);
+  auto quantile = [&](double count) -> float {
+    double f = count / nkb;
+    f = f < 1e-12 ? 1e-12 : (f > 1.0 - 1e-12 ? 1.0 - 1e-12 : f);
+    return static_cast<float>(normal_upper_quantile(f));
+  };
+  p.zq = p.all_cand ? 0.f : quantile(p.want);
+  p.zq_lo = p.all_cand ? 0.f : quantile(p.want + 0.5 * p.c_lo);
+  return p;
+}
+
+template <int CPL>
+static cudaError_t launch_select_cand(const CandSel& cs, int n_rows, int nkb, int k_sel, double topp,
+                                      int* kv_idx, int* kv_cnt, uint8_t* mask, cudaStream_t st) {
+  const int W = (nkb + 31) >> 5;
+  const size_t per_warp = static_cast<size_t>((2 * W + 3) / 4 * 4 + 2 * (cs.c_hi + cs.c_lo));
+  const size_t smem = static_cast<size_t>(kCandSelWarps) * per_warp * 4;
+  cudaError_t e = cudaFuncSetAttribute(select_cand_kernel<CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int want = (n_rows + kCandSelWarps - 1) / kCandSelWarps;
+  const int grid = want < 148 * 64 ? want : 148 * 64;
+  select_cand_kernel<CPL><<<grid, kCandSelWarps * 32, smem, st>>>(cs, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask);
+  return cudaGetLastError();
+}
+
+// The candidate path of the mask builder: approximate row statistics,
+// exact scores reduced to normaliser partials and candidate lists, the
+// selection from the lists, and for the rows handed back the score-matrix
+// path on their query tiles (two launches that return at once when no row
+// was handed back).
+template <int D>
+static cudaError_t launch_mask_cand_d(const SliceOut& sl, int BH, int nqb, int nkb, double scale, int k_sel,
+                                      double topp, float* s, long long s_ld, const CandWs& cw, int* kv_idx,
+                                      int* kv_cnt, uint8_t* mask, cudaStream_t st) {
+  I8Launch il;
+  cudaError_t e = i8_launch(BH, nqb, nkb, &il);
+  if (e != cudaSuccess) return e;
+  CUtensorMap ma, mb;
+  if ((e = i8_maps<D>(sl, BH, nqb, nkb, &ma, &mb)) != cudaSuccess) return e;
+  const CandPlan plan = cand_plan(k_sel, nkb, s_ld);
+  CandBufs cb{};
+  cb.st1 = static_cast<float4*>(cw.st1);
+  cb.st2 = static_cast<ZPart*>(cw.st2);
+  cb.rowinfo = static_cast<float2*>(cw.rowinfo);
+  cb.cand_cnt = cw.cand_cnt;
+  cb.cand = reinterpret_cast<uint2*>(s);
+  cb.c_hi = plan.c_hi;
+  cb.c_lo = plan.c_lo;
+  cb.zq = plan.zq;
+  cb.zq_lo = plan.zq_lo;
+  cb.p_lo = static_cast<float>(topp + 0.5 * (1.0 - topp));
+  cb.all_cand = plan.all_cand;
+  cb.fb_cnt = cw.fb_cnt;
+  cb.fb_rows = cw.fb_rows;
+  cb.tile_flag = cw.tile_flag;
+  cb.n_tile_flags = BH * il.w.n_qt;
+  if ((e = launch_i8<D, kScoreStats>(ma, mb, sl, il, scale, nullptr, 0, cb, st)) != cudaSuccess) return e;
+  if ((e = launch_i8<D, kScoreCands>(ma, mb, sl, il, scale, nullptr, 0, cb, st)) != cudaSuccess) return e;
+  CandSel cs{cb.st2, cb.rowinfo, cb.cand_cnt, cb.cand, plan.c_hi, plan.c_lo, plan.cap, 2 * il.w.n_kr, nqb,
+             il.w.n_qt, cb.fb_cnt, cb.fb_rows, cb.tile_flag};
+  const int n_rows = BH * nqb;
+  switch (plan.cap) {
+    case 128: e = launch_select_cand<4>(cs, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st); break;
+    case 256: e = launch_select_cand<8>(cs, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st); break;
+    case 512: e = launch_select_cand<16>(cs, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st); break;
+    default: e = launch_select_cand<32>(cs, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st); break;
+  }
+  if (e != cudaSuccess) return e;
+  // rows handed back: their query tiles' score rows, then the full-row selection
+  CandBufs fb{};
+  fb.fb_cnt = cw.fb_cnt;
+  fb.tile_flag = cw.tile_flag;
+  if ((e = launch_i8<D, kScoreWrite>(ma, mb, sl, il, scale, s, s_ld, fb, st)) != cudaSuccess) return e;
+  return launch_select(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st, cw.fb_rows, cw.fb_cnt);
+}
+
+cudaError_t launch_mask_cand(const SliceOut& sl, int BH, int nqb, int nkb, int d, double scale, int k_sel,
+                             double topp, float* s, long long s_ld, const CandWs& cw, int* kv_idx, int* kv_cnt,
+                             uint8_t* mask, cudaStream_t st) {
+  return d == 128 ? launch_mask_cand_d<128>(sl, BH, nqb, nkb, scale, k_sel, topp, s, s_ld, cw, kv_idx, kv_cnt, mask, st)
+                  : launch_mask_cand_d<64>(sl, BH, nqb, nkb, scale, k_sel, topp, s, s_ld, cw, kv_idx, kv_cnt, mask, st);
 }
 
 cudaError_t launch_compact_mask(const uint8_t* mask, int n_rows, int nkb, int* kv_idx,

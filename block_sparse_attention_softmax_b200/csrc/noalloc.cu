@@ -16,8 +16,8 @@
 namespace sa {
 
 // Fixed scratch size. Enough for, e.g., B*H = 12 heads at N = 32760 tokens,
-// d = 128 (about 11 MB of pooled means and scores).
-constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+// d = 128 (about 17 MB of pooled means, slices, score rows and row buffers).
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 namespace {

@@ -51,15 +51,18 @@ int check_shape(int B, int H, int N, int d, int bq, int bk) {
 }
 
 struct MaskWs {
-  size_t q_pool, k_pool, q_sl, k_sl, q_ex, k_ex, s, total;
+  size_t q_pool, k_pool, q_sl, k_sl, q_ex, k_ex, s, st1, st2, rowinfo, cand_cnt, fb, fb_rows, tile_flag, total;
   long long s_ld;
 };
 
 // Workspace of the mask builder: pooled means (unless the caller takes them),
-// their int8 slices and exponents, and the fp32 block scores.
+// their int8 slices and exponents, the score rows (candidate lists first,
+// then the score rows of query tiles handed back to the full-row selection)
+// and the per-row buffers of the candidate path.
 MaskWs mask_ws(int B, int H, int N, int d, int bq, int bk, bool need_q, bool need_k) {
   const long long BH = static_cast<long long>(B) * H;
   const long long nqb = (N + bq - 1) / bq, nkb = (N + bk - 1) / bk;
+  const long long rows = BH * nqb;
   MaskWs w{};
   w.s_ld = (nkb + 3) / 4 * 4;
   size_t off = 0;
@@ -76,12 +79,27 @@ MaskWs mask_ws(int B, int H, int N, int d, int bq, int bk, bool need_q, bool nee
   w.k_ex = off;
   off += round_up(static_cast<size_t>(BH * nkb) * 4, 256);
   w.s = off;
-  off += round_up(static_cast<size_t>(BH * nqb) * w.s_ld * 4, 256);
+  off += round_up(static_cast<size_t>(rows * cand_row_bytes(w.s_ld)), 256);
+  w.st1 = off;
+  off += round_up(static_cast<size_t>(rows) * 2 * kMaxKr * 16, 256);
+  w.st2 = off;
+  off += round_up(static_cast<size_t>(rows) * 2 * kMaxKr * 16, 256);
+  w.rowinfo = off;
+  off += round_up(static_cast<size_t>(rows) * 8, 256);
+  w.cand_cnt = off;
+  off += round_up(static_cast<size_t>(rows) * 8, 256);
+  w.fb = off;
+  off += 256;
+  w.fb_rows = off;
+  off += round_up(static_cast<size_t>(rows) * 4, 256);
+  w.tile_flag = off;
+  off += round_up(static_cast<size_t>(BH * ((nqb + kI8TileM - 1) / kI8TileM)) * 4, 256);
   w.total = off;
   return w;
 }
 
-// The three launches of the mask builder, on carved workspace.
+// The launches of the mask builder, on carved workspace: pooling (with the
+// int8 slices), then the candidate path.
 cudaError_t run_mask_builder(const void* q, const void* k, int BH, int N, int d, int bq, int bk,
                              int k_sel, double topp, double scale, int* kv_idx, int* kv_cnt,
                              uint8_t* mask_opt, float* qp, float* kp, char* ws, const MaskWs& w,
@@ -90,9 +108,12 @@ cudaError_t run_mask_builder(const void* q, const void* k, int BH, int N, int d,
   SliceOut sl{reinterpret_cast<int8_t*>(ws + w.q_sl), reinterpret_cast<int8_t*>(ws + w.k_sl),
               reinterpret_cast<int*>(ws + w.q_ex), reinterpret_cast<int*>(ws + w.k_ex)};
   float* s = reinterpret_cast<float*>(ws + w.s);
+  CandWs cw{ws + w.st1, ws + w.st2, ws + w.rowinfo, reinterpret_cast<int*>(ws + w.cand_cnt),
+            reinterpret_cast<int*>(ws + w.fb), reinterpret_cast<int*>(ws + w.fb_rows),
+            reinterpret_cast<int*>(ws + w.tile_flag)};
   cudaError_t e = launch_pool(q, k, BH, N, d, bq, bk, qp, kp, st, &sl);
-  if (e == cudaSuccess) e = launch_scores_i8(sl, BH, nqb, nkb, d, scale, s, w.s_ld, st);
-  if (e == cudaSuccess) e = launch_select(s, w.s_ld, BH * nqb, nkb, k_sel, topp, kv_idx, kv_cnt, mask_opt, st);
+  if (e == cudaSuccess)
+    e = launch_mask_cand(sl, BH, nqb, nkb, d, scale, k_sel, topp, s, w.s_ld, cw, kv_idx, kv_cnt, mask_opt, st);
   return e;
 }
 

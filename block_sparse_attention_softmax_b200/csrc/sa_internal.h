@@ -26,9 +26,39 @@ cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, int 
                         float* q_pool, float* k_pool, cudaStream_t st, const SliceOut* sl = nullptr);
 cudaError_t launch_scores_i8(const SliceOut& sl, int BH, int nqb, int nkb, int d, double scale,
                              float* s, long long s_ld, cudaStream_t st);
+// Full-row selection over the fp32 score matrix; with `rows`, only the rows
+// rows[0 .. *n_rows_dev) (a device-side count).
 cudaError_t launch_select(const float* s, long long s_ld, int n_rows, int nkb, int k_sel,
                           double topp, int* kv_idx, int* kv_cnt, uint8_t* mask,
-                          cudaStream_t st);
+                          cudaStream_t st, const int* rows = nullptr, const int* n_rows_dev = nullptr);
+
+// Candidate path of the mask builder. Its per-row buffers (the candidate
+// lists share the score rows' memory, which the handed-back rows reuse after
+// the lists are read):
+struct CandWs {
+  void* st1;        // [rows][16] float4 approximate row statistics per key range and half
+  void* st2;        // [rows][16] 16-byte normaliser partials
+  void* rowinfo;    // [rows] float2
+  int* cand_cnt;    // [rows][2]
+  int* fb_cnt;      // 1
+  int* fb_rows;     // [rows]
+  int* tile_flag;   // [BH * ceil(nqb / 128)]
+};
+// Bytes of one score row (s_ld floats) or one candidate list, whichever is larger.
+inline long long cand_row_bytes(long long s_ld) { return s_ld * 4 > 1024 ? s_ld * 4 : 1024; }
+struct CandPlan {
+  int want;      // candidates aimed at per row in the first list
+  int cap;       // entries of the register selection (128 .. 1024)
+  int c_hi;      // capacity of the first list (scores >= t)
+  int c_lo;      // capacity of the second list (t_lo <= score < t)
+  int all_cand;  // nkb <= cap: every key block is in the first list
+  float zq;      // standard normal quantile with upper tail want / nkb (t)
+  float zq_lo;   // the same with upper tail (want + c_lo / 2) / nkb (t_lo)
+};
+CandPlan cand_plan(int k_sel, int nkb, long long s_ld);
+cudaError_t launch_mask_cand(const SliceOut& sl, int BH, int nqb, int nkb, int d, double scale, int k_sel,
+                             double topp, float* s, long long s_ld, const CandWs& cw, int* kv_idx, int* kv_cnt,
+                             uint8_t* mask, cudaStream_t st);
 cudaError_t launch_compact_mask(const uint8_t* mask, int n_rows, int nkb, int* kv_idx,
                                 int* kv_cnt, cudaStream_t st);
 

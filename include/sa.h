@@ -142,11 +142,11 @@ int sa_blend(const uint16_t* o_s, const uint16_t* q, const float* kv_state, cons
  * and cannot let a call grow it or synchronise the device to allocate. This
  * entry point computes exactly what sa_build_mask computes (same kernels, same
  * results) but keeps its scratch (pooled means and block scores) in a fixed
- * 16 MiB device array that is part of the library: every GPU that loads the
- * library holds those 16 MiB until the process exits. The caller still passes
+ * 32 MiB device array that is part of the library: every GPU that loads the
+ * library holds those 32 MiB until the process exits. The caller still passes
  * the inputs and the outputs.
  *   - Problems whose scratch, as counted by sa_build_mask_workspace_size(), is
- *     above 16 MiB (16777216 bytes) are rejected with SA_ERR_UNSUPPORTED before
+ *     above 32 MiB (33554432 bytes) are rejected with SA_ERR_UNSUPPORTED before
  *     anything is launched; about 12 heads of 32760 tokens at d = 128 fit.
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
