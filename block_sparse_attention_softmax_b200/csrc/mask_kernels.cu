@@ -170,7 +170,7 @@ constexpr int kI8TileN = 64;
 constexpr int kI8BStages = 3;
 constexpr int kI8EpiWarps = 8;
 constexpr int kI8Threads = 32 * (2 + kI8EpiWarps);
-constexpr int kMaxKr = 8;               // key ranges per row (bounds the partial arrays)
+constexpr int kMaxKr = 4;               // key ranges per row (bounds the partial arrays)
 
 enum : int { kScoreWrite = 0, kScoreStats = 1, kScoreCands = 2 };
 
@@ -180,6 +180,12 @@ struct I8Layout {
   static constexpr int NCH = MODE == kScoreStats ? 1 : ROW / 128;   // 128-byte chunks loaded
   static constexpr int LEVELS = MODE == kScoreStats ? 1 : 4;
   static constexpr int STAGES = MODE == kScoreStats ? 6 : kI8BStages;   // B ring depth
+  // epilogue warps and the key columns of a tile each one reads: kScoreCands
+  // splits a row's 64 columns over four warps (16 each) for more warps to
+  // hide its latency, the other modes over two (32 each)
+  static constexpr int EW = MODE == kScoreCands ? 16 : kI8EpiWarps;
+  static constexpr int CW = 4 * kI8TileN / EW;
+  static constexpr int THREADS = 32 * (2 + EW);
   static constexpr uint32_t A_CH = kI8TileM * 128;  // bytes of one A chunk
   static constexpr uint32_t B_CH = kI8TileN * 128;
   static constexpr uint32_t A_BYTES = NCH * A_CH;
@@ -188,14 +194,14 @@ struct I8Layout {
   static constexpr uint32_t OFF_B = OFF_A + A_BYTES;
   static constexpr uint32_t OFF_T = OFF_B + STAGES * B_BYTES;
   // kScoreWrite: [epi warps][32][33] fp32 transpose blocks
-  static constexpr uint32_t T_BYTES = MODE == kScoreWrite ? kI8EpiWarps * 32 * 33 * 4 : 0;
-  // [epi warps][32] fp32 column factors 2^Ek of the current tile
+  static constexpr uint32_t T_BYTES = MODE == kScoreWrite ? EW * 32 * 33 * 4 : 0;
+  // [epi warps][CW] fp32 column factors 2^Ek of the current tile
   static constexpr uint32_t OFF_C = OFF_T + T_BYTES;
-  static constexpr uint32_t C_BYTES = kI8EpiWarps * 32 * 4;
-  // kScoreCands: two tiles' scores, [2][32 columns][epilogue threads] fp32,
+  static constexpr uint32_t C_BYTES = EW * CW * 4;
+  // kScoreCands: two tiles' scores, [2][CW columns][epilogue threads] fp32,
   // read back two tiles later for the candidates
   static constexpr uint32_t OFF_X = OFF_C + C_BYTES;
-  static constexpr uint32_t X_BYTES = MODE == kScoreCands ? 2 * 32 * kI8EpiWarps * 32 * 4 : 0;
+  static constexpr uint32_t X_BYTES = MODE == kScoreCands ? 2 * CW * EW * 32 * 4 : 0;
   static constexpr uint32_t OFF_BAR = OFF_X + X_BYTES;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
 };
@@ -286,9 +292,9 @@ struct CandPend {
 
 // Writes the candidates of one staged tile (bits of `pend`, slots from j on;
 // slots past cap are counted but not stored) and clears `pend`.
-__device__ __forceinline__ void flush_cands(uint32_t pend, int j, int kc0, const float* xst, uint2* cl, int cap) {
+__device__ __forceinline__ void flush_cands(uint32_t pend, int j, int kc0, const float* xst, uint2* cl, int cap,
+                                            int XS) {
   if (pend == 0u) return;
-  constexpr int XS = 32 * kI8EpiWarps;
   uint32_t m = pend;
   while (m != 0u) {
     const int i = __ffs(m) - 1;
@@ -304,7 +310,7 @@ __device__ __forceinline__ float cand_weight(float x, float mlog) {
 }
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_constant__ CUtensorMap tmA,
+__global__ void __launch_bounds__(I8Layout<D, MODE>::THREADS, 1) score_i8_kernel(const __grid_constant__ CUtensorMap tmA,
                                                                  const __grid_constant__ CUtensorMap tmB,
                                                                  const int* __restrict__ q_ex,
                                                                  const int* __restrict__ k_ex, I8Work wk,
@@ -347,7 +353,7 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], kI8EpiWarps);
+      mbar_init(&acc_empty[i], L::EW);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -506,7 +512,8 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
           const int ab = bt & 1;
           const int kcol = kt * kI8TileN + hc * 32 + lane;   // this lane's key in the store phase
           const int ek_l = kcol < wk.nkb ? __ldg(k_ex + static_cast<long long>(bh) * wk.nkb + kcol) : 0;
-          if (!(ok = mbar_wait(&acc_full[ab], (bt >> 1) & 1, abort_flag))) break;
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[ab], (bt >> 1) & 1, abort_flag));   // warp-uniform
+          if (!ok) break;
           tc_fence_after();
           uint32_t a2[32], a3[32], a4[32], a5[32];
           const uint32_t base = la + ab * kSet;
@@ -550,7 +557,8 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
           const int kc0 = kt * kI8TileN + hc * 32;
           const int ek = min(max(ek_next, -126), 127);
           if (kt + 1 < kt1) ek_next = ld_ek(kt + 1);
-          if (!(ok = mbar_wait(&acc_full[ab], (bt >> 1) & 1, abort_flag))) break;
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[ab], (bt >> 1) & 1, abort_flag));   // warp-uniform
+          if (!ok) break;
           tc_fence_after();
           uint32_t a2[32];
           tmem_ld16(la + ab * kSet, a2);
@@ -594,17 +602,21 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
           const float rowf = static_cast<float>(scale * __longlong_as_double(static_cast<long long>(eq - 14 + 1023) << 52));
           const float4 o = nv > 0 ? make_float4(vmax * rowf, (s0 + s1) * rowf, (q0 + q1) * rowf * rowf, static_cast<float>(nv))
                                   : make_float4(-INFINITY, 0.f, 0.f, 0.f);
-          cb.st1[grow * (2 * kMaxKr) + kr * 2 + hc] = o;
+          cb.st1[grow * (4 * kMaxKr) + kr * 2 + hc] = o;
           if (kr == 0 && hc == 0) *reinterpret_cast<int2*>(cb.cand_cnt + 2 * grow) = make_int2(0, 0);
         }
       } else {
         // ---------------------------------------------------------- kScoreCands
-        float* colf = reinterpret_cast<float*>(smem + L::OFF_C) + ew * 32;
+        // this warp: key columns [16 cq, 16 cq + 16) of each tile
+        constexpr int CW = L::CW;
+        const int cq = ew >> 2;
+        const uint32_t lq = tm + (static_cast<uint32_t>(quad * 32) << 16) + cq * CW;
+        float* colf = reinterpret_cast<float*>(smem + L::OFF_C) + ew * CW;
         // reference max and threshold from the row's approximate statistics
         // (the same arithmetic in every CTA that holds a part of the row)
         float m_ref = -INFINITY, t = INFINITY, tl = INFINITY;
         if (row_ok) {
-          const float4* p = cb.st1 + grow * (2 * kMaxKr);
+          const float4* p = cb.st1 + grow * (4 * kMaxKr);
           float su = 0.f, sq = 0.f, n = 0.f;
           for (int j = 0; j < 2 * wk.n_kr; ++j) {
             const float4 a = p[j];
@@ -629,79 +641,74 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
         const RowC rc = row_consts(scale, eq);
         int* cntp = cb.cand_cnt + 2 * (row_ok ? grow : 0);
         uint2* cl = cb.cand + (row_ok ? grow : 0) * (cb.c_hi + cb.c_lo);
-        constexpr int XS = 32 * kI8EpiWarps;                  // stride of a staged column
+        constexpr int XS = 32 * L::EW;                       // stride of a staged column
         float* xst0 = reinterpret_cast<float*>(smem + L::OFF_X) + ew * 32 + lane;
+        auto ld_ekq = [&](int kt) -> int {
+          const int kcol = kt * kI8TileN + cq * CW + lane;
+          return (lane < CW && kcol < wk.nkb) ? __ldg(k_ex + static_cast<long long>(bh) * wk.nkb + kcol) : 0;
+        };
         double z = 0.0;
         float mx = -INFINITY;
-        int ek_next = kt0 < kt1 ? ld_ek(kt0) : 0;
+        int ek_next = kt0 < kt1 ? ld_ekq(kt0) : 0;
         for (int kt = kt0; kt < kt1; ++kt, ++bt) {
           const int ab = bt & 1;
-          const int kc0 = kt * kI8TileN + hc * 32;
+          const int kc0 = kt * kI8TileN + cq * CW;
           const int ek = ek_next;
-          if (kt + 1 < kt1) ek_next = ld_ek(kt + 1);
-          if (!(ok = mbar_wait(&acc_full[ab], (bt >> 1) & 1, abort_flag))) break;
+          if (kt + 1 < kt1) ek_next = ld_ekq(kt + 1);
+          // the candidates of two tiles ago, while this tile's MMAs run (their
+          // staging buffer is this tile's)
+          flush_cands(p2.h, p2.jh, p2.kc0, p2.xb, p2.cl, cb.c_hi, XS);
+          flush_cands(p2.l, p2.jl, p2.kc0, p2.xb, p2.cl + cb.c_hi, cb.c_lo, XS);
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[ab], (bt >> 1) & 1, abort_flag));   // warp-uniform
+          if (!ok) break;
           tc_fence_after();
-          const uint32_t base = la + ab * kSet;
-          const int nvalid = min(32, wk.nkb - kc0);
-          colf[lane] = pow2f(ek);
-          float x[32];
+          const uint32_t base = lq + ab * kSet;
+          uint32_t a2[CW], a3[CW], a4[CW], a5[CW];
+          tmem_ld16(base + 0 * kI8TileN, a2);
+          tmem_ld16(base + 1 * kI8TileN, a3);
+          tmem_ld16(base + 2 * kI8TileN, a4);
+          tmem_ld16(base + 3 * kI8TileN, a5);
+          if (lane < CW) colf[lane] = pow2f(ek);
+          tmem_wait_ld();
+          reg_fence16(a2);
+          reg_fence16(a3);
+          reg_fence16(a4);
+          reg_fence16(a5);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);   // accumulators are in registers: the MMA may go on
+          const int nvalid = min(CW, wk.nkb - kc0);
+          float* xb = xst0 + ab * CW * XS;
           uint32_t selm = 0u, sell = 0u;      // columns >= t and >= t_lo; size the reservations and the writes
-          float m = -INFINITY, zt = 0.f;
-          // two halves of 16 columns, so that only 64 accumulator registers are live
+          float m = -INFINITY;
+          float w[CW];
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t a2[16], a3[16], a4[16], a5[16];
-            tmem_ld16(base + 0 * kI8TileN + 16 * hh, a2);
-            tmem_ld16(base + 1 * kI8TileN + 16 * hh, a3);
-            tmem_ld16(base + 2 * kI8TileN + 16 * hh, a4);
-            tmem_ld16(base + 3 * kI8TileN + 16 * hh, a5);
-              if (hh == 0) {
-              // while the accumulators arrive: the candidates of two tiles ago
-              flush_cands(p2.h, p2.jh, p2.kc0, p2.xb, p2.cl, cb.c_hi);
-              flush_cands(p2.l, p2.jl, p2.kc0, p2.xb, p2.cl + cb.c_hi, cb.c_lo);
+          for (int i = 0; i < CW; i += 4) {
+            const float4 c = *reinterpret_cast<const float4*>(colf + i);
+            const float cc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int ii = i + u;
+              const float xv = score_exact(a2[ii], a3[ii], a4[ii], a5[ii], rc) * cc[u];
+              const bool v = nvalid >= CW || ii < nvalid;
+              w[ii] = v ? cand_weight(xv, mlog) : 0.f;
+              selm |= ((v && xv >= t) ? 1u : 0u) << ii;
+              sell |= ((v && xv >= tl) ? 1u : 0u) << ii;
+              m = v ? fmaxf(m, xv) : m;
+              xb[ii * XS] = xv;
             }
-            tmem_wait_ld();
-            reg_fence16(a2);
-            reg_fence16(a3);
-            reg_fence16(a4);
-            reg_fence16(a5);
-            if (hh == 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&acc_empty[ab]);   // accumulators are in registers
-            } else {
-              __syncwarp();                                  // colf written
-            }
-            float w[16];
-#pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-              const float4 c = *reinterpret_cast<const float4*>(colf + 16 * hh + i);
-              x[16 * hh + i] = score_exact(a2[i], a3[i], a4[i], a5[i], rc) * c.x;
-              x[16 * hh + i + 1] = score_exact(a2[i + 1], a3[i + 1], a4[i + 1], a5[i + 1], rc) * c.y;
-              x[16 * hh + i + 2] = score_exact(a2[i + 2], a3[i + 2], a4[i + 2], a5[i + 2], rc) * c.z;
-              x[16 * hh + i + 3] = score_exact(a2[i + 3], a3[i + 3], a4[i + 3], a5[i + 3], rc) * c.w;
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int ii = 16 * hh + i;
-              const bool v = nvalid >= 32 || ii < nvalid;
-              w[i] = v ? cand_weight(x[ii], mlog) : 0.f;
-              selm |= ((v && x[ii] >= t) ? 1u : 0u) << ii;
-              sell |= ((v && x[ii] >= tl) ? 1u : 0u) << ii;
-              m = v ? fmaxf(m, x[ii]) : m;
-            }
-            // pairwise sum of the half's weights (fp32, two lanes per add)
-            uint64_t p2[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) p2[i] = f2_make(w[2 * i], w[2 * i + 1]);
-#pragma unroll
-            for (int h = 4; h > 0; h >>= 1)
-#pragma unroll
-              for (int i = 0; i < h; ++i) p2[i] = fadd2(p2[i], p2[i + h]);
-            float z0, z1;
-            f2_split(p2[0], z0, z1);
-            zt += z0 + z1;
           }
+          // pairwise sum of the chunk's weights (fp32, two lanes per add)
+          uint64_t q2[CW / 2];
+#pragma unroll
+          for (int i = 0; i < CW / 2; ++i) q2[i] = f2_make(w[2 * i], w[2 * i + 1]);
+#pragma unroll
+          for (int h = CW / 4; h > 0; h >>= 1)
+#pragma unroll
+            for (int i = 0; i < h; ++i) q2[i] = fadd2(q2[i], q2[i + h]);
+          float z0, z1;
+          f2_split(q2[0], z0, z1);
+          const float zt = z0 + z1;
           sell &= ~selm;
           CandPend nw;                            // this tile's (buffer = tile parity, free since p2 is written)
           if ((selm | sell) != 0u) {
@@ -711,10 +718,7 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
             nw.l = sell;
             nw.kc0 = kc0;
             nw.cl = cl;
-            float* xb = xst0 + ab * 32 * XS;
             nw.xb = xb;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) xb[i * XS] = x[i];
           }
           p2 = p1;
           p1 = nw;
@@ -727,16 +731,17 @@ __global__ void __launch_bounds__(kI8Threads, 1) score_i8_kernel(const __grid_co
           zp.z = z;
           zp.mx = mx;
           zp.pad = 0.f;
-          cb.st2[grow * (2 * kMaxKr) + kr * 2 + hc] = zp;
-          if (kr == 0 && hc == 0) cb.rowinfo[grow] = make_float2(m_ref, t);
+          cb.st2[grow * (4 * kMaxKr) + kr * 4 + cq] = zp;
+          if (kr == 0 && cq == 0) cb.rowinfo[grow] = make_float2(m_ref, t);
         }
       }
     }
     if constexpr (MODE == kScoreCands) {
-      flush_cands(p2.h, p2.jh, p2.kc0, p2.xb, p2.cl, cb.c_hi);
-      flush_cands(p2.l, p2.jl, p2.kc0, p2.xb, p2.cl + cb.c_hi, cb.c_lo);
-      flush_cands(p1.h, p1.jh, p1.kc0, p1.xb, p1.cl, cb.c_hi);
-      flush_cands(p1.l, p1.jl, p1.kc0, p1.xb, p1.cl + cb.c_hi, cb.c_lo);
+      constexpr int XS = 32 * L::EW;
+      flush_cands(p2.h, p2.jh, p2.kc0, p2.xb, p2.cl, cb.c_hi, XS);
+      flush_cands(p2.l, p2.jl, p2.kc0, p2.xb, p2.cl + cb.c_hi, cb.c_lo, XS);
+      flush_cands(p1.h, p1.jh, p1.kc0, p1.xb, p1.cl, cb.c_hi, XS);
+      flush_cands(p1.l, p1.jl, p1.kc0, p1.xb, p1.cl + cb.c_hi, cb.c_lo, XS);
     }
   }
   tc_fence_before();
@@ -1647,23 +1652,22 @@ __device__ bool select_cand_fast(const uint2* cl, int cnt, int nkb, int k_sel, d
   return true;
 }
 
-// Wide path: both lists (nh + nl entries) staged in `stg`. Returns false,
-// having written nothing, when they hold less than the target mass.
-__device__ bool select_cand_wide(const uint2* cl, int c_hi, int nh, int nl, int nkb, int k_sel, double target,
-                                 float mlog, int* __restrict__ out, int* __restrict__ cnt_out,
-                                 uint8_t* __restrict__ mrow, uint32_t* keep, uint32_t* tieb, uint2* stg) {
+// Wide path: both lists (nh + nl entries), read in place (L1/L2). Returns
+// false, having written nothing, when they hold less than the target mass.
+__device__ bool select_cand_wide(const uint2* __restrict__ cl, int c_hi, int nh, int nl, int nkb, int k_sel,
+                                 double target, float mlog, int* __restrict__ out, int* __restrict__ cnt_out,
+                                 uint8_t* __restrict__ mrow, uint32_t* keep, uint32_t* tieb) {
   const int lane = threadIdx.x & 31;
   const int n = nh + nl;
+  auto entry = [&](int i) -> uint2 { return __ldg(i < nh ? cl + i : cl + c_hi + (i - nh)); };
   uint32_t kand = 0xFFFFFFFFu, kor = 0u;
   double wt = 0.0;
   for (int i = lane; i < n; i += 32) {
-    const uint2 e = i < nh ? cl[i] : cl[c_hi + (i - nh)];
-    stg[i] = e;
+    const uint2 e = entry(i);
     kand &= e.x;
     kor |= e.x;
     wt += static_cast<double>(cand_weight(key_value(e.x), mlog));
   }
-  __syncwarp();
   kand = __reduce_and_sync(0xFFFFFFFFu, kand);
   kor = __reduce_or_sync(0xFFFFFFFFu, kor);
   wt = warp_sum_d(wt);
@@ -1672,7 +1676,7 @@ __device__ bool select_cand_wide(const uint2* cl, int c_hi, int nh, int nl, int 
   const uint32_t pre = top >= 0 ? (kand & ~(0xFFFFFFFFu >> (31 - top))) : kand;
   auto count_ge = [&](uint32_t c) -> int {
     int k = 0;
-    for (int i = lane; i < n; i += 32) k += stg[i].x >= c ? 1 : 0;
+    for (int i = lane; i < n; i += 32) k += entry(i).x >= c ? 1 : 0;
     return static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, static_cast<unsigned>(k)));
   };
   // ---- Top-k
@@ -1686,7 +1690,7 @@ __device__ bool select_cand_wide(const uint2* cl, int c_hi, int nh, int nl, int 
   double wa = 0.0, ev = 0.0;
   int nv = 0;
   for (int i = lane; i < n; i += 32) {
-    const uint32_t key = stg[i].x;
+    const uint32_t key = entry(i).x;
     if (key > v) {
       wa += static_cast<double>(cand_weight(key_value(key), mlog));
     } else if (key == v) {
@@ -1706,7 +1710,7 @@ __device__ bool select_cand_wide(const uint2* cl, int c_hi, int nh, int nl, int 
       const uint32_t c = u | (1u << bit);
       double m = 0.0;
       for (int i = lane; i < n; i += 32) {
-        const uint32_t key = stg[i].x;
+        const uint32_t key = entry(i).x;
         if (key >= c) m += static_cast<double>(cand_weight(key_value(key), mlog));
       }
       if (warp_sum_d(m) >= target) u = c;
@@ -1714,7 +1718,7 @@ __device__ bool select_cand_wide(const uint2* cl, int c_hi, int nh, int nl, int 
     int pa = 0, nu = 0;
     double wpa = 0.0, eu = 0.0;
     for (int i = lane; i < n; i += 32) {
-      const uint32_t key = stg[i].x;
+      const uint32_t key = entry(i).x;
       if (key > u) {
         ++pa;
         wpa += static_cast<double>(cand_weight(key_value(key), mlog));
@@ -1735,7 +1739,10 @@ __device__ bool select_cand_wide(const uint2* cl, int c_hi, int nh, int nl, int 
   }
   const bool all_ties = cut.ties >= n_cut;
   clear_bits(keep, tieb, (nkb + 31) >> 5);
-  for (int i = lane; i < n; i += 32) mark_bit(stg[i].x, static_cast<int>(stg[i].y), cut, all_ties, keep, tieb);
+  for (int i = lane; i < n; i += 32) {
+    const uint2 e = entry(i);
+    mark_bit(e.x, static_cast<int>(e.y), cut, all_ties, keep, tieb);
+  }
   emit_bits(nkb, cut, all_ties, out, cnt_out, mrow, keep, tieb);
   return true;
 }
@@ -1743,7 +1750,7 @@ __device__ bool select_cand_wide(const uint2* cl, int c_hi, int nh, int nl, int 
 template <int CPL>
 __device__ void select_cand_row(const CandSel& cs, int row, int nkb, int k_sel, double topp,
                                 int* __restrict__ out, int* __restrict__ cnt_out, uint8_t* __restrict__ mrow,
-                                uint32_t* keep, uint32_t* tieb, uint2* stg) {
+                                uint32_t* keep, uint32_t* tieb) {
   const int lane = threadIdx.x & 31;
   if (topp >= 1.0 || k_sel >= nkb) {          // every block (every finite score)
     for (int i = lane; i < nkb; i += 32) {
@@ -1756,7 +1763,7 @@ __device__ void select_cand_row(const CandSel& cs, int row, int nkb, int k_sel, 
   double zp = 0.0;
   float mxp = -INFINITY;
   if (lane < cs.n_parts) {
-    const ZPart p = cs.st2[static_cast<long long>(row) * (2 * kMaxKr) + lane];
+    const ZPart p = cs.st2[static_cast<long long>(row) * (4 * kMaxKr) + lane];
     zp = p.z;
     mxp = p.mx;
   }
@@ -1775,13 +1782,12 @@ __device__ void select_cand_row(const CandSel& cs, int row, int nkb, int k_sel, 
       select_cand_fast<CPL>(cl, cnt.x, nkb, k_sel, target, mlog, out, cnt_out, mrow, keep, tieb))
     return;
   if (cnt.x <= cs.c_hi && cnt.y <= cs.c_lo && cnt.x + cnt.y >= k_sel &&
-      select_cand_wide(cl, cs.c_hi, cnt.x, cnt.y, nkb, k_sel, target, mlog, out, cnt_out, mrow, keep, tieb, stg))
+      select_cand_wide(cl, cs.c_hi, cnt.x, cnt.y, nkb, k_sel, target, mlog, out, cnt_out, mrow, keep, tieb))
     return;
   hand_back(cs, row);
 }
 
-// Per warp: two bit rows of ceil(nkb / 32) words (kept, ties at the cut),
-// then c_hi + c_lo staged candidates.
+// Per warp: two bit rows of ceil(nkb / 32) words (kept, ties at the cut).
 template <int CPL>
 __global__ void __launch_bounds__(kCandSelWarps * 32) select_cand_kernel(
     CandSel cs, int n_rows, int nkb, int k_sel, double topp, int* __restrict__ kv_idx,
@@ -1789,14 +1795,11 @@ __global__ void __launch_bounds__(kCandSelWarps * 32) select_cand_kernel(
   extern __shared__ __align__(16) uint32_t cand_smem[];
   const int warp = threadIdx.x >> 5;
   const int W = (nkb + 31) >> 5;
-  const int bw = (2 * W + 3) / 4 * 4;                          // bit words, 16-byte multiple
-  const int per_warp = bw + 2 * (cs.c_hi + cs.c_lo);
-  uint32_t* keep = cand_smem + static_cast<size_t>(warp) * per_warp;
+  uint32_t* keep = cand_smem + static_cast<size_t>(warp) * 2 * W;
   uint32_t* tieb = keep + W;
-  uint2* stg = reinterpret_cast<uint2*>(keep + bw);
   for (int row = blockIdx.x * kCandSelWarps + warp; row < n_rows; row += gridDim.x * kCandSelWarps) {
     select_cand_row<CPL>(cs, row, nkb, k_sel, topp, kv_idx + static_cast<long long>(row) * nkb, kv_cnt + row,
-                         mask ? mask + static_cast<long long>(row) * nkb : nullptr, keep, tieb, stg);
+                         mask ? mask + static_cast<long long>(row) * nkb : nullptr, keep, tieb);
     __syncwarp();
   }
 }
@@ -1885,7 +1888,7 @@ static cudaError_t launch_i8(const CUtensorMap& ma, const CUtensorMap& mb, const
   using L = I8Layout<D, MODE>;
   cudaError_t e = cudaFuncSetAttribute(score_i8_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  score_i8_kernel<D, MODE><<<il.grid, kI8Threads, L::SMEM, st>>>(ma, mb, sl.q_ex, sl.k_ex, il.w, scale, s, s_ld, cb);
+  score_i8_kernel<D, MODE><<<il.grid, L::THREADS, L::SMEM, st>>>(ma, mb, sl.q_ex, sl.k_ex, il.w, scale, s, s_ld, cb);
   return cudaGetLastError();
 }
 
@@ -1968,8 +1971,7 @@ template <int CPL>
 static cudaError_t launch_select_cand(const CandSel& cs, int n_rows, int nkb, int k_sel, double topp,
                                       int* kv_idx, int* kv_cnt, uint8_t* mask, cudaStream_t st) {
   const int W = (nkb + 31) >> 5;
-  const size_t per_warp = static_cast<size_t>((2 * W + 3) / 4 * 4 + 2 * (cs.c_hi + cs.c_lo));
-  const size_t smem = static_cast<size_t>(kCandSelWarps) * per_warp * 4;
+  const size_t smem = static_cast<size_t>(kCandSelWarps) * 2 * W * 4;
   cudaError_t e = cudaFuncSetAttribute(select_cand_kernel<CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -2012,7 +2014,7 @@ static cudaError_t launch_mask_cand_d(const SliceOut& sl, int BH, int nqb, int n
   cb.n_tile_flags = BH * il.w.n_qt;
   if ((e = launch_i8<D, kScoreStats>(ma, mb, sl, il, scale, nullptr, 0, cb, st)) != cudaSuccess) return e;
   if ((e = launch_i8<D, kScoreCands>(ma, mb, sl, il, scale, nullptr, 0, cb, st)) != cudaSuccess) return e;
-  CandSel cs{cb.st2, cb.rowinfo, cb.cand_cnt, cb.cand, plan.c_hi, plan.c_lo, plan.cap, 2 * il.w.n_kr, nqb,
+  CandSel cs{cb.st2, cb.rowinfo, cb.cand_cnt, cb.cand, plan.c_hi, plan.c_lo, plan.cap, 4 * il.w.n_kr, nqb,
              il.w.n_qt, cb.fb_cnt, cb.fb_rows, cb.tile_flag};
   const int n_rows = BH * nqb;
   switch (plan.cap) {

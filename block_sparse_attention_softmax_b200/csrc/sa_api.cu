@@ -81,9 +81,9 @@ MaskWs mask_ws(int B, int H, int N, int d, int bq, int bk, bool need_q, bool nee
   w.s = off;
   off += round_up(static_cast<size_t>(rows * cand_row_bytes(w.s_ld)), 256);
   w.st1 = off;
-  off += round_up(static_cast<size_t>(rows) * 2 * kMaxKr * 16, 256);
+  off += round_up(static_cast<size_t>(rows) * 4 * kMaxKr * 16, 256);
   w.st2 = off;
-  off += round_up(static_cast<size_t>(rows) * 2 * kMaxKr * 16, 256);
+  off += round_up(static_cast<size_t>(rows) * 4 * kMaxKr * 16, 256);
   w.rowinfo = off;
   off += round_up(static_cast<size_t>(rows) * 8, 256);
   w.cand_cnt = off;
