@@ -1850,7 +1850,7 @@ struct I8Launch {
   int grid;
 };
 
-static cudaError_t i8_launch(int BH, int nqb, int nkb, I8Launch* out) {
+static cudaError_t i8_launch(int BH, int nqb, int nkb, I8Launch* out, int max_tiles_per_item = 0) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1863,6 +1863,7 @@ static cudaError_t i8_launch(int BH, int nqb, int nkb, I8Launch* out) {
   long long per = (tiles + 4LL * sms - 1) / (4LL * sms);
   const long long per_min = (w.n_kt + kMaxKr - 1) / kMaxKr;
   per = per < per_min ? per_min : per;
+  if (max_tiles_per_item > 0 && per > max_tiles_per_item) per = max_tiles_per_item;
   per = per < 1 ? 1 : (per > w.n_kt ? w.n_kt : per);
   w.kr_tiles = static_cast<int>(per);
   w.n_kr = ceil_div(w.n_kt, w.kr_tiles);
@@ -2024,11 +2025,15 @@ static cudaError_t launch_mask_cand_d(const SliceOut& sl, int BH, int nqb, int n
     default: e = launch_select_cand<32>(cs, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st); break;
   }
   if (e != cudaSuccess) return e;
-  // rows handed back: their query tiles' score rows, then the full-row selection
+  // rows handed back: their query tiles' score rows (in short key ranges, so
+  // that a few flagged tiles spread over many CTAs), then the full-row
+  // selection
   CandBufs fb{};
   fb.fb_cnt = cw.fb_cnt;
   fb.tile_flag = cw.tile_flag;
-  if ((e = launch_i8<D, kScoreWrite>(ma, mb, sl, il, scale, s, s_ld, fb, st)) != cudaSuccess) return e;
+  I8Launch ilw;
+  if ((e = i8_launch(BH, nqb, nkb, &ilw, 4)) != cudaSuccess) return e;
+  if ((e = launch_i8<D, kScoreWrite>(ma, mb, sl, ilw, scale, s, s_ld, fb, st)) != cudaSuccess) return e;
   return launch_select(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st, cw.fb_rows, cw.fb_cnt);
 }
 
