@@ -41,8 +41,8 @@ METRIC = "sparse_attn_effective_tflops"
 # and O sized). `sources_sha` pins the kernel sources the counters belong to:
 # once they change, traffic is reported as null until a new capture is made.
 ATTN_TRAFFIC_CAPTURE = {
-    "workload": "wan13b_480p", "dram_bytes_read": 302478592, "dram_bytes_write": 82770176,
-    "sources_sha": "2023a76b34a8fbb8",
+    "workload": "wan13b_480p", "dram_bytes_read": 302395648, "dram_bytes_write": 82280192,
+    "sources_sha": "5ff27c5a7b12eed8",
     "sources": ("attn_kernel.cu", "sa_device.cuh", "sa_internal.h"),
 }
 
@@ -252,11 +252,12 @@ def run_ours(args, wl, rank, world, local):
     o = torch.empty_like(q)
     ev = []  # (start, end) events around the sparse attention launch
 
-    # our kernels per step: pool, row statistics, candidate scores, candidate
-    # selection, the two hand-back launches (return at once when no row was
-    # handed back); attention; linear state,
-    # its fixed-order reduction, and the fused output + blend
-    launches_per_step = 6 + 1 + (3 if wl.linear else 0)
+    # our kernels per step: the mask builder's (pooling, then scores and
+    # selection, or row statistics, candidate scores, candidate selection and
+    # two hand-back launches that return at once when no row was handed back,
+    # as the library reports for this shape); attention; linear state, its
+    # fixed-order reduction, and the fused output + blend
+    launches_per_step = lib.sa_build_mask_launches(B, H, N, d, wl.bq, wl.bk) + 1 + (3 if wl.linear else 0)
 
     ev_mask, ev_lin = [], []   # (start, end) events around the mask build and the linear branch
 

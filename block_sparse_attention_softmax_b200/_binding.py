@@ -22,6 +22,7 @@ _SIGNATURES = {
     "sa_pool_blocks": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                c_void_p, c_void_p, c_void_p]),
     "sa_build_mask_workspace_size": (c_size_t, [c_int] * 6),
+    "sa_build_mask_launches": (c_int, [c_int] * 6),
     "sa_build_mask": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                               c_double, c_double, c_double, c_void_p, c_void_p, c_void_p,
                               c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),

@@ -3,6 +3,7 @@
 // of every entry point are in include/sa.h.
 #include <math.h>
 #include <stdarg.h>
+#include <stdlib.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -98,8 +99,18 @@ MaskWs mask_ws(int B, int H, int N, int d, int bq, int bk, bool need_q, bool nee
   return w;
 }
 
+// Which builder a shape takes: the score-matrix path while the fp32 scores
+// fit in 32 MiB (cheap to write and re-read, three launches), else the
+// candidate path. SA_MASK_BUILDER=matrix / =candidates forces one.
+bool use_candidates(long long rows, long long s_ld) {
+  const char* env = getenv("SA_MASK_BUILDER");
+  if (env && strcmp(env, "matrix") == 0) return false;
+  if (env && strcmp(env, "candidates") == 0) return true;
+  return rows * s_ld * 4 > (32LL << 20);
+}
+
 // The launches of the mask builder, on carved workspace: pooling (with the
-// int8 slices), then the candidate path.
+// int8 slices), then the score-matrix or the candidate path.
 cudaError_t run_mask_builder(const void* q, const void* k, int BH, int N, int d, int bq, int bk,
                              int k_sel, double topp, double scale, int* kv_idx, int* kv_cnt,
                              uint8_t* mask_opt, float* qp, float* kp, char* ws, const MaskWs& w,
@@ -112,8 +123,11 @@ cudaError_t run_mask_builder(const void* q, const void* k, int BH, int N, int d,
             reinterpret_cast<int*>(ws + w.fb), reinterpret_cast<int*>(ws + w.fb_rows),
             reinterpret_cast<int*>(ws + w.tile_flag)};
   cudaError_t e = launch_pool(q, k, BH, N, d, bq, bk, qp, kp, st, &sl);
-  if (e == cudaSuccess)
-    e = launch_mask_cand(sl, BH, nqb, nkb, d, scale, k_sel, topp, s, w.s_ld, cw, kv_idx, kv_cnt, mask_opt, st);
+  if (e != cudaSuccess) return e;
+  if (use_candidates(static_cast<long long>(BH) * nqb, w.s_ld))
+    return launch_mask_cand(sl, BH, nqb, nkb, d, scale, k_sel, topp, s, w.s_ld, cw, kv_idx, kv_cnt, mask_opt, st);
+  e = launch_scores_i8(sl, BH, nqb, nkb, d, scale, s, w.s_ld, st);
+  if (e == cudaSuccess) e = launch_select(s, w.s_ld, BH * nqb, nkb, k_sel, topp, kv_idx, kv_cnt, mask_opt, st);
   return e;
 }
 
@@ -216,6 +230,15 @@ int sa_pool_blocks(const uint16_t* q, const uint16_t* k, int B, int H, int N, in
 size_t sa_build_mask_workspace_size(int B, int H, int N, int d, int bq, int bk) {
   if (check_shape(B, H, N, d, bq, bk)) return 0;
   return mask_ws(B, H, N, d, bq, bk, true, true).total;
+}
+
+int sa_build_mask_launches(int B, int H, int N, int d, int bq, int bk) {
+  if (check_shape(B, H, N, d, bq, bk)) return 0;
+  const MaskWs w = mask_ws(B, H, N, d, bq, bk, true, true);
+  const long long rows = static_cast<long long>(B) * H * ((N + bq - 1) / bq);
+  // pooling, then statistics, candidates, selection and the two hand-back
+  // launches, or scores and selection
+  return use_candidates(rows, w.s_ld) ? 6 : 3;
 }
 
 int sa_build_mask(const uint16_t* q, const uint16_t* k, int B, int H, int N, int d, int bq, int bk,

@@ -90,8 +90,16 @@ int sa_pool_blocks(const uint16_t* q, const uint16_t* k, int B, int H, int N, in
  * Order used by both rules: score descending, equal scores by lower block index.
  * The kept set of a row is therefore the first max(K_sel, m_p) blocks of that
  * order. Outputs kv_idx/kv_cnt (required) and, when non-NULL, the uint8 mask
- * and the pooled Q/K. Needs sa_build_mask_workspace_size() bytes of workspace. */
+ * and the pooled Q/K. Needs sa_build_mask_workspace_size() bytes of workspace.
+ * Two exact implementations, chosen by problem size: up to 32 MiB of fp32
+ * block scores, the scores are written and each row is selected from them;
+ * above, the scores are reduced on the fly to per-row normalisers and
+ * candidate lists (rows the lists cannot settle take the first way). The
+ * environment variable SA_MASK_BUILDER=matrix or =candidates forces one. */
 size_t sa_build_mask_workspace_size(int B, int H, int N, int d, int bq, int bk);
+/* Kernel launches one sa_build_mask call of this shape makes (for launch
+ * accounting); 0 for an invalid shape. */
+int sa_build_mask_launches(int B, int H, int N, int d, int bq, int bk);
 int sa_build_mask(const uint16_t* q, const uint16_t* k, int B, int H, int N, int d,
                   int bq, int bk, double topk_frac, double topp, double scale,
                   int32_t* kv_idx, int32_t* kv_cnt, uint8_t* mask_opt,

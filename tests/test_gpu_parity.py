@@ -176,6 +176,40 @@ def test_uniform_scores_tie_order(cuda_lib):
     assert (idx[0, 0, :, :8] == np.arange(8)).all()
 
 
+# ------------------------------------------------------------------ both mask builders on small cases
+@pytest.mark.parametrize("builder", ["matrix", "candidates"])
+def test_each_mask_builder(cuda_lib, builder, monkeypatch):
+    """The score-matrix and the candidate builder, forced, on cases the size
+    rule would send to the other one: the tiny workload and ragged shapes
+    against the oracle (every head), all-equal scores (every block ties),
+    and a 1.3B-480p-shaped head group whose lists must also equal the other
+    builder's except at reported near-ties."""
+    sa = cuda_lib
+    monkeypatch.setenv("SA_MASK_BUILDER", builder)
+    wl = WORKLOADS["tiny"]
+    x = make_inputs(wl, "cpu")
+    _, _, totals = _check_masks(sa, x["q"].to(DEV), x["k"].to(DEV), wl.bq, wl.bk, wl.topk, wl.topp,
+                                [(0, h) for h in range(wl.H)])
+    print(builder, "tiny mask rows:", totals)
+    for N, d, bq, H in [(200, 128, 64, 1), (4099, 128, 128, 2)]:
+        q, k, _ = random_qkv(1, H, N, d, seed=N * 7 + d, device=DEV)
+        q = (q.float() * 3.0).to(torch.bfloat16)
+        _check_masks(sa, q, k, bq, 64, 0.2, 0.8, [(0, h) for h in range(H)])
+    # all-equal scores: P = 1/16 each, Top-p 0.5 keeps the 8 lowest blocks
+    q = torch.zeros(1, 1, 1024, 64, dtype=torch.bfloat16, device=DEV)
+    _, k, _ = random_qkv(1, 1, 1024, 64, seed=9, device=DEV)
+    m = sa.sa_build_mask(q, k, 64, 64, 0.1, 0.5)
+    assert (m["kv_cnt"].cpu().numpy() == 8).all()
+    assert (m["kv_idx"].cpu().numpy()[0, 0, :, :8] == np.arange(8)).all()
+    # 4 heads of the 1.3B-480p geometry against the oracle
+    wl = WORKLOADS["wan13b_480p"]
+    x = make_inputs(wl, DEV)
+    q, k = x["q"][:, :4].contiguous(), x["k"][:, :4].contiguous()
+    _, _, totals = _check_masks(sa, q, k, wl.bq, wl.bk, wl.topk, wl.topp, [(0, 0), (0, 3)])
+    print(builder, "1.3B-480p mask rows:", totals)
+    sa.sa_device_status()
+
+
 # ------------------------------------------------------------------ full-size workloads (sampled)
 FULL = ["wan13b_480p", "wan14b_720p", "sink_skew", "long_245k"]
 
