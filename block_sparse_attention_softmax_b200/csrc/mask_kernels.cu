@@ -1964,7 +1964,7 @@ CandPlan cand_plan(int k_sel, int nkb, long long s_ld) {
     return static_cast<float>(normal_upper_quantile(f));
   };
   p.zq = p.all_cand ? 0.f : quantile(p.want);
-  p.zq_lo = p.all_cand ? 0.f : quantile(p.want + 0.5 * p.c_lo);
+  p.zq_lo = p.all_cand ? 0.f : quantile(p.want + 0.9 * p.c_lo);
   return p;
 }
 

@@ -53,7 +53,7 @@ struct CandPlan {
   int c_lo;      // capacity of the second list (t_lo <= score < t)
   int all_cand;  // nkb <= cap: every key block is in the first list
   float zq;      // standard normal quantile with upper tail want / nkb (t)
-  float zq_lo;   // the same with upper tail (want + c_lo / 2) / nkb (t_lo)
+  float zq_lo;   // the same with upper tail (want + 0.9 c_lo) / nkb (t_lo)
 };
 CandPlan cand_plan(int k_sel, int nkb, long long s_ld);
 cudaError_t launch_mask_cand(const SliceOut& sl, int BH, int nqb, int nkb, int d, double scale, int k_sel,
