@@ -1843,14 +1843,15 @@ cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, int 
   return cudaGetLastError();
 }
 
-// Work split of the score kernels: about four items per SM and at most
-// kMaxKr key ranges per row.
+// Work split of the score kernels: about four items per SM; at most kMaxKr
+// key ranges per row where per-row partials are kept (cap_ranges).
 struct I8Launch {
   I8Work w;
   int grid;
 };
 
-static cudaError_t i8_launch(int BH, int nqb, int nkb, I8Launch* out, int max_tiles_per_item = 0) {
+static cudaError_t i8_launch(int BH, int nqb, int nkb, I8Launch* out, bool cap_ranges,
+                             int max_tiles_per_item = 0) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1861,7 +1862,7 @@ static cudaError_t i8_launch(int BH, int nqb, int nkb, I8Launch* out, int max_ti
   w.n_kt = ceil_div(nkb, kI8TileN);
   const long long tiles = static_cast<long long>(BH) * w.n_qt * w.n_kt;
   long long per = (tiles + 4LL * sms - 1) / (4LL * sms);
-  const long long per_min = (w.n_kt + kMaxKr - 1) / kMaxKr;
+  const long long per_min = cap_ranges ? (w.n_kt + kMaxKr - 1) / kMaxKr : 1;
   per = per < per_min ? per_min : per;
   if (max_tiles_per_item > 0 && per > max_tiles_per_item) per = max_tiles_per_item;
   per = per < 1 ? 1 : (per > w.n_kt ? w.n_kt : per);
@@ -1896,7 +1897,7 @@ static cudaError_t launch_i8(const CUtensorMap& ma, const CUtensorMap& mb, const
 cudaError_t launch_scores_i8(const SliceOut& sl, int BH, int nqb, int nkb, int d, double scale,
                              float* s, long long s_ld, cudaStream_t st) {
   I8Launch il;
-  cudaError_t e = i8_launch(BH, nqb, nkb, &il);
+  cudaError_t e = i8_launch(BH, nqb, nkb, &il, false);
   if (e != cudaSuccess) return e;
   CUtensorMap ma, mb;
   const CandBufs none{};
@@ -1992,7 +1993,7 @@ static cudaError_t launch_mask_cand_d(const SliceOut& sl, int BH, int nqb, int n
                                       double topp, float* s, long long s_ld, const CandWs& cw, int* kv_idx,
                                       int* kv_cnt, uint8_t* mask, cudaStream_t st) {
   I8Launch il;
-  cudaError_t e = i8_launch(BH, nqb, nkb, &il);
+  cudaError_t e = i8_launch(BH, nqb, nkb, &il, true);
   if (e != cudaSuccess) return e;
   CUtensorMap ma, mb;
   if ((e = i8_maps<D>(sl, BH, nqb, nkb, &ma, &mb)) != cudaSuccess) return e;
@@ -2032,7 +2033,7 @@ static cudaError_t launch_mask_cand_d(const SliceOut& sl, int BH, int nqb, int n
   fb.fb_cnt = cw.fb_cnt;
   fb.tile_flag = cw.tile_flag;
   I8Launch ilw;
-  if ((e = i8_launch(BH, nqb, nkb, &ilw, 4)) != cudaSuccess) return e;
+  if ((e = i8_launch(BH, nqb, nkb, &ilw, false, 4)) != cudaSuccess) return e;
   if ((e = launch_i8<D, kScoreWrite>(ma, mb, sl, ilw, scale, s, s_ld, fb, st)) != cudaSuccess) return e;
   return launch_select(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, st, cw.fb_rows, cw.fb_cnt);
 }
