@@ -1538,14 +1538,22 @@ __device__ void emit_bits(int nkb, const Cut& cut, bool all_ties, int* __restric
   }
   int c = 0;
   for (int i = w0; i < w1; ++i) c += __popc(keep[i]);
-  int pos = warp_excl_scan(c);
-  const int total = __shfl_sync(0xFFFFFFFFu, pos + c, 31);
-  for (int i = w0; i < w1; ++i) {
-    uint32_t b = keep[i];
-    while (b != 0u) {
-      out[pos++] = i * 32 + (__ffs(b) - 1);
-      b &= b - 1u;
+  int pre = warp_excl_scan(c);                   // kept blocks before this lane's first word
+  const int total = __shfl_sync(0xFFFFFFFFu, pre + c, 31);
+  // round r: word r of every lane; its nonzero words one at a time, each
+  // lane writing its own bit of the word (coalesced, in block order)
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int r = 0; r < wpl; ++r) {
+    const uint32_t word = w0 + r < w1 ? keep[w0 + r] : 0u;
+    uint32_t nz = __ballot_sync(0xFFFFFFFFu, word != 0u);
+    while (nz != 0u) {
+      const int src = __ffs(nz) - 1;
+      nz &= nz - 1u;
+      const uint32_t wv = __shfl_sync(0xFFFFFFFFu, word, src);
+      const int base = __shfl_sync(0xFFFFFFFFu, pre, src);
+      if ((wv >> lane) & 1u) out[base + __popc(wv & lt)] = (src * wpl + r) * 32 + lane;
     }
+    pre += __popc(word);
   }
   if (mrow)
     for (int i = lane; i < nkb; i += 32) mrow[i] = static_cast<uint8_t>((keep[i >> 5] >> (i & 31)) & 1u);
