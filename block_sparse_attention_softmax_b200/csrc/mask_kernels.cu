@@ -2,18 +2,25 @@
 // selection (pages: "SLA2" 提案手法 ① mean pooling of Q and K;
 // "SpargeAttention2" §2(1) hybrid Top-k + Top-p masking per attention row).
 //
-//   pool_kernel      Q, K [BH, N, d] bf16 -> block means [BH, nb, d] fp32, and
-//                    the same means as four signed 7-bit slices per element
-//                    with a per-row power-of-two exponent
-//   score_i8_kernel  slices -> s[bh, qb, kb] = scale * <Qbar, Kbar> on the
-//                    int8 tensor cores (exact s32 slice products, combined in
-//                    int64, scaled in fp64, rounded once to fp32)
-//   select_*_kernel  one query-block row per warp: the K_sel-th largest score
-//                    (Top-k) by a short count search followed by an exact
-//                    search among at most 256 candidates, a probability-mass
-//                    search for the Top-p cut when Top-k alone does not reach
-//                    p, and the ascending compacted index list; the row sits
-//                    in registers (up to 1280 key blocks) or shared memory.
+//   pool_kernel        Q, K [BH, N, d] bf16 -> block means [BH, nb, d] fp32,
+//                      and the same means as four signed 7-bit slices per
+//                      element with a per-row power-of-two exponent
+//   score_i8_kernel    scale * <Qbar, Kbar> on the int8 tensor cores from the
+//                      slices (exact s32 slice products, combined in fp32 with
+//                      one final rounding), in three modes: the fp32 score
+//                      matrix; approximate per-row statistics; exact scores
+//                      reduced to per-row normaliser partials and candidate
+//                      lists
+//   select_cand_kernel one query-block row per warp from its candidate lists:
+//                      the K_sel-th largest score (Top-k), the Top-p cut when
+//                      Top-k alone does not reach p, the ascending kept list
+//   select_*_kernel    one row per warp from the score matrix: the same cuts by
+//                      a short count search and an exact search among at most
+//                      256 candidates, the row in registers (up to 1280 key
+//                      blocks) or shared memory
+// The score-matrix path (write mode, then select_fast / select_long) serves
+// problems of up to 32 MiB of scores and the rows the candidate lists cannot
+// settle; the candidate path (statistics, candidates, select_cand) the rest.
 #include "sa_internal.h"
 
 namespace sa {
