@@ -152,10 +152,11 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 // Persistent CTAs over work items (head, 128 query blocks, a range of 64-key
 // tiles): warp 0 loads the item's query slices (operand A, M = 128) and
 // streams the key-slice tiles (operand B, N = 64) through a 3-stage ring by
-// TMA (128-byte swizzled rows, one box per 128-byte column chunk); warp 1
-// issues the MMAs of a key tile into one of two TMEM accumulator sets; eight
-// epilogue warps (two per TMEM lane quadrant, 32 key columns each, so each
-// thread owns one query-block row) consume the accumulators. Three modes:
+// TMA (128-byte swizzled rows, one box per 128-byte column chunk; 6 stages
+// in kScoreStats); warp 1 issues the MMAs of a key tile into one of two TMEM
+// accumulator sets; the epilogue warps (per TMEM lane quadrant two warps of
+// 32 key columns, or in kScoreCands four of 16, so that each thread owns one
+// query-block row) consume the accumulators. Three modes:
 //
 //   kScoreWrite  exact scores, transposed through shared memory and written
 //                as the fp32 score matrix with coalesced 128-byte stores;
@@ -168,7 +169,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 //                maximum and a threshold t
 //   kScoreCands  exact scores as in kScoreWrite, never stored: per row and
 //                item, the exact max and the partial normaliser
-//                sum e^(s - m_ref) (fp32 pairwise over each 32-column
+//                sum e^(s - m_ref) (fp32 pairwise over each 16-column
 //                chunk, fp64 across chunks), and every score >= t appended
 //                to the row's candidate list (one atomic per thread and tile
 //                reserves the slots)
