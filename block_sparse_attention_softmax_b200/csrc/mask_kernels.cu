@@ -170,14 +170,14 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 //   kScoreCands  exact scores as in kScoreWrite, never stored: per row and
 //                item, the exact max and the partial normaliser
 //                sum e^(s - m_ref) (fp32 pairwise over each 16-column
-//                chunk, fp64 across chunks), and every score >= t appended
-//                to the row's candidate list (one atomic per thread and tile
-//                reserves the slots)
+//                chunk, fp64 across chunks), and every score >= t (and, for
+//                rows expected to need it, every score in [t_lo, t)) appended
+//                to the row's lists (one atomic per thread, list and tile
+//                reserves the slots; the entries are written two tiles later)
 constexpr int kI8TileM = 128;
 constexpr int kI8TileN = 64;
 constexpr int kI8BStages = 3;
 constexpr int kI8EpiWarps = 8;
-constexpr int kI8Threads = 32 * (2 + kI8EpiWarps);
 constexpr int kMaxKr = 4;               // key ranges per row (bounds the partial arrays)
 
 enum : int { kScoreWrite = 0, kScoreStats = 1, kScoreCands = 2 };
