@@ -82,3 +82,24 @@ def test_workspace_sizes_scale_with_shape(lib):
     assert big >= 40 * nqb * ((nkb + 3) // 4 * 4) * 4 + 40 * (nqb + nkb) * 128 * 4
     assert lib.sa_build_mask_workspace_size(1, 1, 128, 96, 64, 64) == 0   # unsupported -> 0
     assert lib.sa_linear_workspace_size(1, 40, 75600, 128) > 0
+
+
+def test_build_mask_launch_count(lib):
+    """The mask builder reports the launches it makes for a shape: three for
+    the score-matrix path (up to 32 MiB of fp32 scores), six for the candidate
+    path, zero for a rejected shape; SA_MASK_BUILDER overrides the choice."""
+    import os
+    saved = os.environ.pop("SA_MASK_BUILDER", None)
+    try:
+        assert lib.sa_build_mask_launches(1, 12, 32760, 128, 128, 64) == 3     # 6.3 MB of scores
+        assert lib.sa_build_mask_launches(1, 40, 75600, 128, 128, 64) == 6     # 112 MB of scores
+        assert lib.sa_build_mask_launches(1, 40, 245760, 128, 128, 64) == 6
+        assert lib.sa_build_mask_launches(1, 1, 128, 96, 64, 64) == 0          # unsupported d
+        os.environ["SA_MASK_BUILDER"] = "candidates"
+        assert lib.sa_build_mask_launches(1, 12, 32760, 128, 128, 64) == 6
+        os.environ["SA_MASK_BUILDER"] = "matrix"
+        assert lib.sa_build_mask_launches(1, 40, 75600, 128, 128, 64) == 3
+    finally:
+        os.environ.pop("SA_MASK_BUILDER", None)
+        if saved is not None:
+            os.environ["SA_MASK_BUILDER"] = saved
