@@ -210,6 +210,27 @@ def test_each_mask_builder(cuda_lib, builder, monkeypatch):
     sa.sa_device_status()
 
 
+def test_candidate_hand_back_all_rows(cuda_lib, monkeypatch):
+    """All-equal scores on 1,182-block rows under the candidate builder: every
+    threshold count is 0 or 1,182, above the lists' capacity, so every row is
+    handed back to the score-matrix selection. P = 1/1182 each, so Top-p 0.85
+    keeps the smallest m with m/1182 >= 0.85, the 1005 lowest blocks."""
+    sa = cuda_lib
+    monkeypatch.setenv("SA_MASK_BUILDER", "candidates")
+    N, d = 75600, 128
+    q = torch.zeros(1, 1, N, d, dtype=torch.bfloat16, device=DEV)
+    _, k, _ = random_qkv(1, 1, N, d, seed=11, device=DEV)
+    m = sa.sa_build_mask(q, k, 128, 64, 0.03, 0.85, want_mask=True)
+    cnt = m["kv_cnt"].cpu().numpy()
+    idx = m["kv_idx"].cpu().numpy()
+    want = math.ceil(0.85 * 1182 - 1e-9)
+    assert want == 1005
+    assert (cnt == want).all()
+    assert (idx[0, 0, :, :want] == np.arange(want)).all()
+    assert (m["mask"][0, 0, :, :want] == 1).all() and (m["mask"][0, 0, :, want:] == 0).all()
+    sa.sa_device_status()
+
+
 # ------------------------------------------------------------------ full-size workloads (sampled)
 FULL = ["wan13b_480p", "wan14b_720p", "sink_skew", "long_245k"]
 
