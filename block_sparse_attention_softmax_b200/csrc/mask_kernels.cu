@@ -236,6 +236,7 @@ struct CandBufs {
   float zq;          // standard normal quantile with tail mass want / nkb (t)
   float zq_lo;       // the same for the wider list (t_lo)
   float p_lo;        // rows whose expected Top-k mass share is below this get the second list
+  float zp;          // z with P(Z > z) = p (standard normal): the model's Top-p length is nkb Q(sd + zp)
   int all_cand;      // every key block is a candidate of the first list
   int* fb_cnt;       // rows handed back to the score-matrix path
   int* fb_rows;      // [rows]
@@ -642,7 +643,13 @@ __global__ void __launch_bounds__(I8Layout<D, MODE>::THREADS, 1) score_i8_kernel
             // N(mean, sd^2): Q((t - mean - sd^2) / sd). Rows where Top-k alone
             // is expected to hold well over p Z skip the second list.
             const float share = 0.5f * erfcf((t - mean - sd * sd) / (sd * 1.41421356f));
-            if (!(share >= cb.p_lo)) tl = fminf(t, mean + cb.zq_lo * sd);
+            if (!(share >= cb.p_lo)) {
+              // expected Top-p length: beyond both lists, the row goes straight
+              // back to the full-row selection (no candidates: its count stays 0)
+              const float need = static_cast<float>(wk.nkb) * 0.5f * erfcf((sd + cb.zp) * 0.70710678f);
+              if (need > static_cast<float>(cb.c_hi + cb.c_lo)) t = INFINITY;
+              else tl = fminf(t, mean + cb.zq_lo * sd);
+            }
           }
         }
         const float mlog = m_ref * 1.4426950408889634f;
@@ -2025,6 +2032,7 @@ static cudaError_t launch_mask_cand_d(const SliceOut& sl, int BH, int nqb, int n
   cb.zq = plan.zq;
   cb.zq_lo = plan.zq_lo;
   cb.p_lo = static_cast<float>(topp + 0.5 * (1.0 - topp));
+  cb.zp = static_cast<float>(normal_upper_quantile(topp <= 1e-12 ? 1e-12 : (topp >= 1.0 - 1e-12 ? 1.0 - 1e-12 : topp)));
   cb.all_cand = plan.all_cand;
   cb.fb_cnt = cw.fb_cnt;
   cb.fb_rows = cw.fb_rows;
