@@ -31,8 +31,10 @@
  *       ksum            [B, H, d] fp32, z = sum_j phi(k_j)
  *       alpha           [H, d] fp32
  *   - Supported shapes: d in {64, 128}; bq in {64, 128}; bk = 64; N >= 1;
- *     B*H >= 1; every element count below 2^31 per tensor. Other values give
- *     SA_ERR_UNSUPPORTED.
+ *     1 <= B*H <= 65535; B*H*N*d < 2^40 and B*H*n_qb*n_kb < 2^34 (offsets
+ *     are 64-bit); the mask builder also needs n_kb <= 16384 (N <= 1048576).
+ *     Other values give SA_ERR_UNSUPPORTED; B, H or N below 1 give
+ *     SA_ERR_INVALID_ARG.
  *   - Every device pointer must be 16-byte aligned (SA_ERR_ALIGN otherwise).
  *   - The caller owns every buffer. The library allocates no device memory; a
  *     call that needs scratch takes a caller-provided workspace whose size the

@@ -51,6 +51,13 @@ def test_argument_validation_without_launch(lib):
     assert lib.sa_pool_blocks(None, fake, 1, 1, 128, 64, 64, 64, fake, fake, None) == -1
     # misaligned pointer
     assert lib.sa_pool_blocks(P(0x1004), fake, 1, 1, 128, 64, 64, 64, fake, fake, None) == -3
+    # size limits of the header: B*H <= 65535, B*H*N*d < 2^40, n_kb <= 16384 for the mask
+    assert lib.sa_pool_blocks(fake, fake, 2, 32768, 128, 64, 64, 64, fake, fake, None) == -2
+    assert lib.sa_pool_blocks(fake, fake, 1, 65535, 200000, 128, 64, 64, fake, fake, None) == -2
+    assert lib.sa_build_mask_workspace_size(1, 1, 16384 * 64 + 1, 64, 64, 64) > 0
+    assert lib.sa_build_mask(fake, fake, 1, 1, 16384 * 64 + 1, 64, 64, 64, 0.1, 0.9, 0.0,
+                             fake, fake, None, None, None, fake, 1 << 40, None) == -2
+    assert b"16384" in lib.sa_last_error()
     # Top-k / Top-p ranges
     ws = lib.sa_build_mask_workspace_size(1, 1, 128, 64, 64, 64)
     assert ws > 0
