@@ -92,18 +92,50 @@ def _stream(device):
     return c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def _check_qkv(*ts):
-    for t in ts:
+def _expect(name, t, shape, dtypes):
+    """Checks what the C ABI cannot see behind a raw pointer: the tensor's
+    shape, element type and layout. Returns the tensor."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not isinstance(dtypes, tuple):
+        dtypes = (dtypes,)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {' or '.join(map(str, dtypes))}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: libsa takes contiguous tensors")
+    return t
+
+
+def _on_device(device, **tensors):
+    """Every given tensor is a CUDA tensor on `device`."""
+    for name, t in tensors.items():
         if t is None:
             continue
         if not t.is_cuda:
-            raise ValueError("libsa takes CUDA tensors")
-        if not t.is_contiguous():
-            raise ValueError("libsa takes contiguous tensors")
-    return ts[0].shape
+            raise ValueError(f"{name}: libsa takes CUDA tensors")
+        if t.device != device:
+            raise ValueError(f"{name} is on {t.device}, the other operands on {device}")
 
 
-def _workspace(nbytes, device):
+def _qkv(q, *others, names=("q", "k", "v")):
+    """[B, H, N, d] bf16 operands of one shape; returns (B, H, N, d)."""
+    if q is None or q.dim() != 4:
+        raise ValueError(f"{names[0]} must be a [B, H, N, d] tensor")
+    for name, t in zip(names, (q,) + others):
+        _expect(name, t, q.shape, torch.bfloat16)
+    return tuple(q.shape)
+
+
+def _workspace(nbytes, device, given=None):
+    """The caller's workspace when it is a large enough contiguous uint8
+    tensor on `device`, else a new one."""
+    if given is not None:
+        _expect("workspace", given, given.shape, torch.uint8)
+        _on_device(device, workspace=given)
+        if given.numel() >= nbytes:
+            return given
     return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
 
 
@@ -121,7 +153,8 @@ def sa_device_status(device=None):
 
 
 def sa_pool_blocks(q, k, bq, bk):
-    B, H, N, d = _check_qkv(q, k)
+    B, H, N, d = _qkv(q, k)
+    _on_device(q.device, q=q, k=k)
     nqb, nkb = -(-N // bq), -(-N // bk)
     qp = torch.empty(B, H, nqb, d, dtype=torch.float32, device=q.device)
     kp = torch.empty(B, H, nkb, d, dtype=torch.float32, device=q.device)
@@ -131,16 +164,16 @@ def sa_pool_blocks(q, k, bq, bk):
 
 def sa_build_mask(q, k, bq, bk, topk, topp, scale=0.0, want_mask=False, want_pools=False,
                   workspace=None):
-    B, H, N, d = _check_qkv(q, k)
-    nqb, nkb = -(-N // bq), -(-N // bk)
+    B, H, N, d = _qkv(q, k)
     dev = q.device
+    _on_device(dev, q=q, k=k)
+    nqb, nkb = -(-N // bq), -(-N // bk)
     kv_idx = torch.empty(B, H, nqb, nkb, dtype=torch.int32, device=dev)
     kv_cnt = torch.empty(B, H, nqb, dtype=torch.int32, device=dev)
     mask = torch.empty(B, H, nqb, nkb, dtype=torch.uint8, device=dev) if want_mask else None
     qp = torch.empty(B, H, nqb, d, dtype=torch.float32, device=dev) if want_pools else None
     kp = torch.empty(B, H, nkb, d, dtype=torch.float32, device=dev) if want_pools else None
-    need = load().sa_build_mask_workspace_size(B, H, N, d, bq, bk)
-    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
+    ws = _workspace(load().sa_build_mask_workspace_size(B, H, N, d, bq, bk), dev, workspace)
     _call("sa_build_mask", _ptr(q), _ptr(k), B, H, N, d, bq, bk, float(topk), float(topp),
           float(scale), _ptr(kv_idx), _ptr(kv_cnt), _ptr(mask), _ptr(qp), _ptr(kp), _ptr(ws),
           ws.numel(), _stream(dev))
@@ -154,14 +187,22 @@ def sa_build_mask(q, k, bq, bk, topk, topp, scale=0.0, want_mask=False, want_poo
 
 def sa_sparse_attn_fwd(q, k, v, bq, bk, kv_idx=None, kv_cnt=None, ext_mask=None, scale=0.0,
                        want_lse=False, out=None, workspace=None):
-    B, H, N, d = _check_qkv(q, k, v)
+    B, H, N, d = _qkv(q, k, v)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    if kv_idx is not None:
+        _expect("kv_idx", kv_idx, (B, H, nqb, nkb), torch.int32)
+    if kv_cnt is not None:
+        _expect("kv_cnt", kv_cnt, (B, H, nqb), torch.int32)
+    if ext_mask is not None:
+        _expect("ext_mask", ext_mask, (B, H, nqb, nkb), (torch.uint8, torch.bool))
+    if out is not None:
+        _expect("out", out, q.shape, torch.bfloat16)
     dev = q.device
+    _on_device(dev, q=q, k=k, v=v, kv_idx=kv_idx, kv_cnt=kv_cnt, ext_mask=ext_mask, out=out)
     o = out if out is not None else torch.empty_like(q)
     lse = torch.empty(B, H, N, dtype=torch.float32, device=dev) if want_lse else None
     need = load().sa_sparse_attn_workspace_size(B, H, N, d, bq, bk, int(ext_mask is not None))
-    ws = None
-    if need:
-        ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
+    ws = _workspace(need, dev, workspace) if need else None
     _call("sa_sparse_attn_fwd", _ptr(q), _ptr(k), _ptr(v), B, H, N, d, bq, bk, _ptr(kv_idx),
           _ptr(kv_cnt), _ptr(ext_mask), float(scale), _ptr(o), _ptr(lse), _ptr(ws),
           0 if ws is None else ws.numel(), _stream(dev))
@@ -169,7 +210,10 @@ def sa_sparse_attn_fwd(q, k, v, bq, bk, kv_idx=None, kv_cnt=None, ext_mask=None,
 
 
 def sa_dense_attn_fwd(q, k, v, bq=128, scale=0.0, want_lse=False, out=None):
-    B, H, N, d = _check_qkv(q, k, v)
+    B, H, N, d = _qkv(q, k, v)
+    if out is not None:
+        _expect("out", out, q.shape, torch.bfloat16)
+    _on_device(q.device, q=q, k=k, v=v, out=out)
     o = out if out is not None else torch.empty_like(q)
     lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device) if want_lse else None
     _call("sa_dense_attn_fwd", _ptr(q), _ptr(k), _ptr(v), B, H, N, d, bq, float(scale), _ptr(o),
@@ -178,26 +222,34 @@ def sa_dense_attn_fwd(q, k, v, bq=128, scale=0.0, want_lse=False, out=None):
 
 
 def sa_linear_branch(q, k, v, want_ol=False, workspace=None):
-    B, H, N, d = _check_qkv(k, v)
+    if want_ol:
+        B, H, N, d = _qkv(q, k, v)
+    else:
+        B, H, N, d = _qkv(k, v, names=("k", "v"))
+        q = None            # read only for O_l
     dev = k.device
+    _on_device(dev, q=q, k=k, v=v)
     S = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
     z = torch.empty(B, H, d, dtype=torch.float32, device=dev)
     o_l = torch.empty_like(k) if want_ol else None
-    need = load().sa_linear_workspace_size(B, H, N, d)
-    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
+    ws = _workspace(load().sa_linear_workspace_size(B, H, N, d), dev, workspace)
     _call("sa_linear_branch", _ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(S), _ptr(z), _ptr(o_l),
           _ptr(ws), ws.numel(), _stream(dev))
     return (S, z, o_l) if want_ol else (S, z)
 
 
 def sa_blend(o_s, q, kv_state, ksum, alpha, out=None, workspace=None):
-    B, H, N, d = _check_qkv(o_s, q, kv_state, ksum, alpha)
+    B, H, N, d = _qkv(o_s, q, names=("o_s", "q"))
+    _expect("kv_state", kv_state, (B, H, d, d), torch.float32)
+    _expect("ksum", ksum, (B, H, d), torch.float32)
+    _expect("alpha", alpha, (H, d), torch.float32)
+    if out is not None:
+        _expect("out", out, o_s.shape, torch.bfloat16)
     dev = q.device
+    _on_device(dev, o_s=o_s, q=q, kv_state=kv_state, ksum=ksum, alpha=alpha, out=out)
     o = out if out is not None else torch.empty_like(o_s)
     need = load().sa_blend_workspace_size(B, H, N, d)
-    ws = None
-    if need:
-        ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
+    ws = _workspace(need, dev, workspace) if need else None
     _call("sa_blend", _ptr(o_s), _ptr(q), _ptr(kv_state), _ptr(ksum), _ptr(alpha), B, H, N, d,
           _ptr(o), _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev))
     return o
@@ -224,8 +276,15 @@ def block_sparse_attention(q, k, v, bq=128, bk=64, topk=0.05, topp=0.9, alpha=No
     asynchronous."""
     if q.is_cuda:
         return _path_on_device(q, k, v, bq, bk, topk, topp, alpha, scale, out)
+    B, H, N, d = _qkv(q, k, v)
+    for name, t in (("k", k), ("v", v), ("out", out)):
+        if t is not None and t.is_cuda:
+            raise ValueError(f"{name} is a CUDA tensor while q is on the host")
+    if alpha is not None:
+        _expect("alpha", alpha, (H, d), torch.float32)
+    if out is not None:
+        _expect("out", out, q.shape, torch.bfloat16)
     device = device or torch.device("cuda", torch.cuda.current_device())
-    B, H, N, d = q.shape
     BH = B * H
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)

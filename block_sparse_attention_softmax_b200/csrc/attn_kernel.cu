@@ -114,6 +114,13 @@ struct Item {
   bool tail;     // the last kept block is the ragged last key block
 };
 
+// Kept-block count of list row r, clamped to [0, n_kb] so that a malformed
+// count cannot send any role past the end of its row of kv_idx (every role
+// reads the count through here, so all of them agree on it).
+__device__ __forceinline__ int kept_count(const AttnArgs& a, long long r) {
+  return min(max(__ldg(a.kv_cnt + r), 0), a.nkb);
+}
+
 __device__ __forceinline__ Item load_item(const AttnArgs& a, int item) {
   Item it;
   it.bh = item / a.nqb;
@@ -124,7 +131,7 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int item) {
     it.tail = ragged;
   } else {
     const long long r = static_cast<long long>(it.bh) * a.nqb + it.qb;
-    it.cnt = __ldg(a.kv_cnt + r);
+    it.cnt = kept_count(a, r);
     it.tail = ragged && it.cnt > 0 && __ldg(a.kv_idx + r * a.nkb + it.cnt - 1) == a.nkb - 1;
   }
   it.T = (it.cnt + 1) >> 1;
@@ -302,7 +309,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       while (ok && item < n_items) {
         // facts of the next item, fetched while this one is issued
         const int nitem = next_nonempty(a, item + gridDim.x, gridDim.x, n_items);
-        const int ncnt = nitem < n_items ? (a.dense ? a.nkb : __ldg(a.kv_cnt + nitem)) : 0;
+        const int ncnt = nitem < n_items ? (a.dense ? a.nkb : kept_count(a, nitem)) : 0;
         for (int t = 0; t < it.T; ++t, ++g) {
           const bool two = it.cnt - 2 * t >= 2;
           if (is_qk) {

@@ -115,7 +115,11 @@ int sa_build_mask(const uint16_t* q, const uint16_t* k, int B, int H, int N, int
  * uint8 mask is first compacted into the workspace
  * (sa_sparse_attn_workspace_size(); 0 bytes are needed for the list form).
  * A row with no kept block outputs zeros and lse = -inf. lse_opt may be NULL.
- * scale <= 0 selects 1/sqrt(d). */
+ * scale <= 0 selects 1/sqrt(d). The lists are device data and are not
+ * validated: a count outside [0, n_kb] is clamped into it, and an index
+ * outside [0, n_kb) makes the result meaningless but cannot make an access
+ * leave the caller's buffers (key and value tiles are fetched through tensor
+ * maps, which bound every load by the tensor's extent). */
 size_t sa_sparse_attn_workspace_size(int B, int H, int N, int d, int bq, int bk, int ext_mask);
 int sa_sparse_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                        int B, int H, int N, int d, int bq, int bk,
