@@ -41,8 +41,8 @@ METRIC = "sparse_attn_effective_tflops"
 # and O sized). `sources_sha` pins the kernel sources the counters belong to:
 # once they change, traffic is reported as null until a new capture is made.
 ATTN_TRAFFIC_CAPTURE = {
-    "workload": "wan13b_480p", "dram_bytes_read": 302395648, "dram_bytes_write": 82280192,
-    "sources_sha": "b8d78beec84e6d04",
+    "workload": "wan13b_480p", "dram_bytes_read": 302803968, "dram_bytes_write": 83264256,
+    "sources_sha": "d3dbd3485535a770",
     "sources": ("attn_kernel.cu", "sa_device.cuh", "sa_internal.h"),
 }
 

@@ -705,12 +705,24 @@ __global__ void __launch_bounds__(I8Layout<D, MODE>::THREADS, 1) score_i8_kernel
             for (int u = 0; u < 4; ++u) {
               const int ii = i + u;
               const float xv = score_exact(a2[ii], a3[ii], a4[ii], a5[ii], rc) * cc[u];
-              const bool v = nvalid >= CW || ii < nvalid;
-              w[ii] = v ? cand_weight(xv, mlog) : 0.f;
-              selm |= ((v && xv >= t) ? 1u : 0u) << ii;
-              sell |= ((v && xv >= tl) ? 1u : 0u) << ii;
-              m = v ? fmaxf(m, xv) : m;
+              w[ii] = cand_weight(xv, mlog);
+              selm |= (xv >= t ? 1u : 0u) << ii;
+              sell |= (xv >= tl ? 1u : 0u) << ii;
+              m = fmaxf(m, xv);
               xb[ii * XS] = xv;
+            }
+          }
+          if (nvalid < CW) {
+            // columns past the row end (warp-uniform, the row's last tile
+            // only): out of both lists, the normaliser and the max
+            const uint32_t vm = nvalid > 0 ? (1u << nvalid) - 1u : 0u;
+            selm &= vm;
+            sell &= vm;
+            m = -INFINITY;
+#pragma unroll
+            for (int ii = 0; ii < CW; ++ii) {
+              if (ii >= nvalid) w[ii] = 0.f;
+              else m = fmaxf(m, xb[ii * XS]);
             }
           }
           // pairwise sum of the chunk's weights (fp32, two lanes per add)
