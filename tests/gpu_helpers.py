@@ -11,31 +11,51 @@ MAX_ABS = 2e-2
 MEAN_ABS = 2e-3
 
 
-def compare_mask_rows(gpu_idx, gpu_cnt, s, k_frac, p):
+def _swap_within_tie(g, order, s, n, tol):
+    """True when the set g holds n blocks and differs from the first n blocks of
+    the oracle order only by exchanging blocks across a near-tie at that cut:
+    every block the oracle keeps and g drops scores at most tol above every
+    block g keeps and the oracle drops."""
+    pref = set(order[:n].tolist())
+    if len(g) != n:
+        return False
+    dropped, added = sorted(pref - g), sorted(g - pref)
+    if not dropped:
+        return True
+    return float(s[dropped].max() - s[added].min()) <= tol
+
+
+def compare_mask_rows(gpu_idx, gpu_cnt, s, k_frac, p, tol=oracle.NEAR_TIE_TOL):
     """Compare one head's GPU kv lists with the oracle decision on scores s.
 
-    Every differing row must be a tie the fp32 GPU evaluation may resolve the
-    other way: blocks within NEAR_TIE_TOL of the cut score, or a cumulative sum
-    within NEAR_TIE_TOL of p. Returns dict(exact, score_tie, cumsum_tie, bad).
-    """
+    A row that differs is accepted only as a decision the fp32 GPU evaluation
+    may take the other way:
+      score tie   the same number of blocks, exchanged across the cut between
+                  blocks whose scores differ by at most tol;
+      cumsum tie  another length, at least K_sel, where every cumulative sum
+                  between the two cuts lies within tol of p (so the fp32 sums
+                  may cross p at either), and the kept set is that length's
+                  prefix up to a score tie.
+    Returns dict(exact, score_tie, cumsum_tie, bad)."""
     stats = {"exact": 0, "score_tie": 0, "cumsum_tie": 0, "bad": []}
     n_qb = s.shape[0]
     for r in range(n_qb):
         g = set(gpu_idx[r, :gpu_cnt[r]].tolist())
-        info = oracle.row_threshold_info(s[r], k_frac, p)
-        L = info["L"]
-        ora = set(info["order"][:L].tolist())
+        info = oracle.row_threshold_info(s[r], k_frac, p, tol)
+        order, L = info["order"], info["L"]
+        ora = set(order[:L].tolist())
         if g == ora:
             stats["exact"] += 1
             continue
-        if (g ^ ora) <= info["near_blocks"]:
+        Lg = len(g)
+        if Lg == L and _swap_within_tie(g, order, s[r], L, tol):
             stats["score_tie"] += 1
             continue
-        Lg = len(g)
-        pref = set(info["order"][:Lg].tolist())
-        near = info["near_ranks"]
-        if Lg >= info["k_sel"] and (pref ^ g) <= info["near_blocks"] and \
-                ({Lg - 1, Lg - 2, L - 1, L - 2} & near):
+        # ranks whose cumulative sum decides between lengths L and Lg
+        between = range(min(L, Lg) - 1, max(L, Lg) - 1)
+        if Lg != L and Lg >= info["k_sel"] and min(L, Lg) >= 1 and \
+                all(i in info["near_ranks"] for i in between) and \
+                _swap_within_tie(g, order, s[r], Lg, tol):
             stats["cumsum_tie"] += 1
             continue
         stats["bad"].append((r, sorted(g - ora)[:8], sorted(ora - g)[:8], Lg, L))
