@@ -102,6 +102,40 @@ def test_topp_minimal_by_exhaustive_subsets_on_tiny_workload():
             assert P[order][:m_p].sum() >= p - 1e-12
 
 
+def test_topp_count_from_the_low_end_of_the_order():
+    """Top-p from the other end: the kept prefix of length m_p is the shortest
+    one whose complement (the n - m_p lowest blocks) holds at most 1 - p of
+    the mass, counted by accumulating from the last block of the order, on
+    peaked, spread, near-uniform and sink rows."""
+    rng = _rng(17)
+    for trial in range(60):
+        n = int(rng.choice([16, 100, 1182]))
+        kind = trial % 4
+        if kind == 0:
+            s = rng.standard_normal(n) * 3.0
+        elif kind == 1:
+            s = rng.standard_normal(n) * 0.5
+        elif kind == 2:
+            s = rng.standard_normal(n) * 0.005                 # near-uniform
+        else:
+            s = rng.standard_normal(n) * 0.5
+            s[rng.integers(n)] += 12.0                           # one sink block
+        order = oracle.descending_order(s)
+        P = oracle.block_softmax(s)[order]
+        for p in (0.5, 0.85, 0.9, 0.99):
+            m_p = oracle.topp_count(P, p)
+            j = 0                                                # blocks droppable from the end
+            while j < n - 1 and math.fsum(P[n - j - 1:]) <= 1.0 - p:
+                j += 1
+            t_keep = math.fsum(P[m_p:])
+            t_more = math.fsum(P[m_p - 1:])
+            near = abs(t_keep - (1.0 - p)) <= 1e-12 or abs(t_more - (1.0 - p)) <= 1e-12
+            if not near:
+                assert n - j == m_p, (trial, p, n - j, m_p)
+            assert t_keep <= 1.0 - p + 1e-12
+            assert m_p == 1 or t_more > 1.0 - p - 1e-12
+
+
 def test_hybrid_equals_union_of_rank_defined_sets():
     """Top-k and Top-p built from the rank definition, with deliberate ties."""
     rng = _rng(5)
