@@ -5,10 +5,12 @@ TEST INFRASTRUCTURE: imported only by tests, the smoke check and the bench's
 CPU-baseline leg. Written from the pages' definitions, in their order; numpy
 matmul, exp and a stable sort are the only library steps.
 
-Parity pins (tests/test_oracle_*.py) tie each function to something other than
-itself: brute force on tiny inputs, closed forms, exhaustive subset search for
-Top-p minimality, and torch's float64 scaled_dot_product_attention for dense
-and masked attention.
+Parity pins (tests/test_oracle_pins.py) tie each function to something other
+than itself: brute force on tiny inputs, closed forms, exhaustive subset search
+for Top-p minimality, the Top-p count from the low end of the order, and
+torch's float64 scaled_dot_product_attention for dense and masked attention.
+row_threshold_info, which the GPU comparison uses to recognise near-ties, is
+pinned with planted rows in tests/test_mask_comparator.py.
 """
 from __future__ import annotations
 
@@ -16,8 +18,9 @@ import math
 
 import numpy as np
 
-# A block whose score lies within this distance of the selection cut, or a row
-# whose cumulative probability lies within it of p, may legitimately differ
+# Near-tie band of the GPU comparison: blocks exchanged across the selection cut
+# whose scores lie within this distance of each other, or a row length decided
+# where the cumulative probability lies within it of p, may legitimately differ
 # between an fp32 GPU evaluation and this fp64 one; such cases are reported.
 NEAR_TIE_TOL = 1e-6
 
