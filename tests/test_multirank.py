@@ -1,27 +1,19 @@
 """Host logic of the multi-rank bench path, as two gloo ranks on CPU: every
 rank joins the barrier, and the reported time is the max over ranks."""
 import os
-import socket
 
 import pytest
 import torch
 import torch.multiprocessing as mp
 
 
-def _free_port():
-    s = socket.socket()
-    s.bind(("127.0.0.1", 0))
-    port = s.getsockname()[1]
-    s.close()
-    return port
-
-
-def _worker(rank, world, port, out):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
-                      WORLD_SIZE=str(world))
+def _worker(rank, world, store_path, out):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world))
     import datetime
-    torch.distributed.init_process_group("gloo", rank=rank, world_size=world,
-                                         timeout=datetime.timedelta(seconds=60))
+    # a file rendezvous: no TCP port that another process could take between
+    # choosing it and binding it
+    torch.distributed.init_process_group("gloo", init_method=f"file://{store_path}", rank=rank,
+                                         world_size=world, timeout=datetime.timedelta(seconds=60))
     import bench
     bench.barrier(world)
     ms = 10.0 + 5.0 * rank
@@ -29,12 +21,12 @@ def _worker(rank, world, port, out):
     torch.distributed.destroy_process_group()
 
 
-def test_max_over_ranks_gloo_world2():
+def test_max_over_ranks_gloo_world2(tmp_path):
     ctx = mp.get_context("spawn")
     mgr = ctx.Manager()
     out = mgr.dict()
-    port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    store = str(tmp_path / "rendezvous")
+    procs = [ctx.Process(target=_worker, args=(r, 2, store, out)) for r in range(2)]
     for p in procs:
         p.start()
     for p in procs:
