@@ -136,6 +136,41 @@ def test_topp_count_from_the_low_end_of_the_order():
             assert m_p == 1 or t_more > 1.0 - p - 1e-12
 
 
+def test_kept_set_from_the_low_end_with_ties():
+    """On heavily tied rows, dropping the lowest blocks while their mass stays
+    within 1 - p (ties at the last dropped score from the highest block index
+    down) leaves exactly the oracle's kept set whenever that set is at least
+    K_sel long: the order's tie rule (lower index first) seen from the other
+    end."""
+    rng = _rng(23)
+    checked = 0
+    for trial in range(200):
+        n = int(rng.choice([40, 300]))
+        s = np.round(rng.standard_normal(n) * 0.05, 2)          # many equal scores
+        p = float(rng.choice([0.5, 0.8, 0.9]))
+        k_frac = 0.05
+        mask, L, k_sel, m_p = oracle.hybrid_row(s, k_frac, p)
+        if m_p < k_sel:
+            continue
+        P = oracle.block_softmax(s)
+        csum = np.cumsum(P[oracle.descending_order(s)])
+        if np.any(np.abs(csum - p) <= 1e-12):
+            continue                                             # a cumulative-sum tie: either end may round
+        # ascending by score, equal scores by higher block index first
+        low = sorted(range(n), key=lambda i: (s[i], -i))
+        dropped, mass = [], 0.0
+        for i in low:
+            if mass + P[i] > 1.0 - p:
+                break
+            dropped.append(i)
+            mass += P[i]
+        kept = np.ones(n, dtype=bool)
+        kept[dropped] = False
+        assert (kept == mask).all(), (trial, n, p)
+        checked += 1
+    assert checked > 100
+
+
 def test_hybrid_equals_union_of_rank_defined_sets():
     """Top-k and Top-p built from the rank definition, with deliberate ties."""
     rng = _rng(5)
