@@ -210,7 +210,8 @@ int sa_device_status(void* stream) {
   if (e != cudaSuccess) return cuda_fail(e, "sa_device_status");
   if (v != 0) {
     const int zero = 0;
-    cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+    e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "sa_device_status (clearing the status word)");
     return fail(SA_ERR_DEVICE_TIMEOUT, "a bounded device-side wait ran out (code %d)", v);
   }
   return SA_OK;
