@@ -35,10 +35,9 @@ DEFAULT_WORKLOAD = "wan14b_720p"
 METRIC = "sparse_attn_effective_tflops"
 
 
-# DRAM traffic of sparse_attn_kernel from one `ncu --set full` capture
-# (profiles/sparse_attn_kernel_wan13b_480p.md), taken on a smaller workload and
-# scaled to the benchmarked one by B*H*N*d (the kernel's DRAM traffic is Q, K, V
-# and O sized). `sources_sha` pins the kernel sources the counters belong to:
+# DRAM traffic of sparse_attn_kernel from one `ncu --set full` capture of the
+# 1.3B-480p-shaped workload, scaled to the benchmarked one by B*H*N*d (the
+# kernel's DRAM traffic is Q, K, V and O sized). `sources_sha` pins the kernel sources the counters belong to:
 # once they change, traffic is reported as null until a new capture is made.
 ATTN_TRAFFIC_CAPTURE = {
     "workload": "wan13b_480p", "dram_bytes_read": 302803968, "dram_bytes_write": 83264256,
@@ -91,6 +90,22 @@ def executed_flops(wl, kv_idx, kv_cnt):
         has_tail = ((kv_idx == last) & (ar < cnt.unsqueeze(-1))).any(-1)
         keys = keys - has_tail.to(torch.int64) * tail_short
     return 4.0 * wl.d * float((keys * valid_q).sum().item())
+
+
+def run_config(wl, world):
+    """The `config` object of both arms' JSON lines (the same keys and values)."""
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d,
+            "block": f"{wl.bq}x{wl.bk}", "topk": wl.topk, "topp": wl.topp,
+            "linear_branch": wl.linear, "parallelism": f"replica x{world}",
+            "l2": "inputs larger than L2 (each tensor >= 774 MB); no flush"}
+
+
+def stats(ms):
+    """Median, min, p90 and mean of per-call times (ms)."""
+    xs = sorted(ms)
+    p90 = xs[min(len(xs) - 1, int(math.ceil(0.9 * len(xs))) - 1)]
+    return {"median": round(statistics.median(xs), 4), "min": round(xs[0], 4),
+            "p90": round(p90, 4), "mean": round(statistics.mean(xs), 4), "n": len(xs)}
 
 
 class ClockSampler:
@@ -237,20 +252,45 @@ def max_over_ranks(x, world, dev):
 
 
 # ------------------------------------------------------------------ our arm
+def _event():
+    e = torch.cuda.Event(enable_timing=True)
+    e.record()
+    return e
+
+
+def _dense_times(sa, q, k, v, bq, o, reps):
+    """Per-call ms of our dense attention and of torch SDPA on the same shape."""
+    out = {}
+    for name, fn in (("ours", lambda: sa.sa_dense_attn_fwd(q, k, v, bq, out=o)),
+                     ("sdpa", lambda: torch.nn.functional.scaled_dot_product_attention(q, k, v))):
+        try:
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize()
+            ev = []
+            for _ in range(reps):
+                e0 = _event()
+                fn()
+                ev.append((e0, _event()))
+            torch.cuda.synchronize()
+            out[name] = stats([x.elapsed_time(y) for x, y in ev])
+        except Exception:
+            out[name] = None
+    return out
+
+
 def run_ours(args, wl, rank, world, local):
     import block_sparse_attention_softmax_b200 as sa
-    sa.load()
+    lib = sa.load()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     x = make_inputs(wl, dev)
     q, k, v, alpha = x["q"], x["k"], x["v"], x["alpha"]
     B, H, N, d = q.shape
-    lib = sa.load()
     ws_mask = torch.empty(lib.sa_build_mask_workspace_size(B, H, N, d, wl.bq, wl.bk), dtype=torch.uint8, device=dev)
     ws_lin = torch.empty(max(1, lib.sa_linear_workspace_size(B, H, N, d)), dtype=torch.uint8, device=dev)
     ws_blend = torch.empty(max(1, lib.sa_blend_workspace_size(B, H, N, d)), dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
-    ev = []  # (start, end) events around the sparse attention launch
 
     # our kernels per step: the mask builder's (pooling, then scores and
     # selection, or row statistics, candidate scores, candidate selection and
@@ -259,29 +299,23 @@ def run_ours(args, wl, rank, world, local):
     # fixed-order reduction, and the fused output + blend
     launches_per_step = lib.sa_build_mask_launches(B, H, N, d, wl.bq, wl.bk) + 1 + (3 if wl.linear else 0)
 
-    ev_mask, ev_lin = [], []   # (start, end) events around the mask build and the linear branch
-
-    def mark():
-        e = torch.cuda.Event(enable_timing=True)
-        e.record()
-        return e
+    # (start, after mask, after attention, after linear + blend) events of each timed step
+    marks = []
 
     def step(record=False):
         if record:
-            m0 = mark()
+            m0 = _event()
         m = sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp, workspace=ws_mask)
         if record:
-            e0 = mark()
-            ev_mask.append((m0, e0))
+            m1 = _event()
         sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], out=o)
         if record:
-            e1 = mark()
-            ev.append((e0, e1))
+            m2 = _event()
         if wl.linear:
             S, z = sa.sa_linear_branch(q, k, v, workspace=ws_lin)
             sa.sa_blend(o, q, S, z, alpha, out=o, workspace=ws_blend)
-            if record:
-                ev_lin.append((e1, mark()))
+        if record:
+            marks.append((m0, m1, m2, _event() if wl.linear else None))
         return m
 
     for _ in range(args.warmup):
@@ -303,43 +337,16 @@ def run_ours(args, wl, rank, world, local):
     barrier(world)
     ms = t0.elapsed_time(t1) / args.steps
     ms_max = max_over_ranks(ms, world, dev)
-    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    mask_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_mask)
-    lin_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_lin) if ev_lin else None
+    mask_t = [a.elapsed_time(b) for a, b, _, _ in marks]
+    attn_t = [b.elapsed_time(c) for _, b, c, _ in marks]
+    lin_t = [c.elapsed_time(e) for _, _, c, e in marks if e is not None]
+    attn_ms, mask_ms = statistics.mean(attn_t), statistics.mean(mask_t)
+    lin_ms = statistics.mean(lin_t) if lin_t else None
     sa.sa_device_status(dev)
 
-    # comparison points (not part of the step): dense attention through our kernel
-    dense_ms = None
-    if not args.no_dense:
-        for _ in range(2):
-            sa.sa_dense_attn_fwd(q, k, v, wl.bq, out=o)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        reps = 3
-        for _ in range(reps):
-            sa.sa_dense_attn_fwd(q, k, v, wl.bq, out=o)
-        e1.record()
-        torch.cuda.synchronize()
-        dense_ms = e0.elapsed_time(e1) / reps
-    # a library dense attention of the same shape, for context (PyTorch SDPA)
-    sdpa_ms = None
-    if not args.no_dense:
-        try:
-            import torch.nn.functional as F
-            for _ in range(2):
-                F.scaled_dot_product_attention(q, k, v)
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            reps = 3
-            for _ in range(reps):
-                F.scaled_dot_product_attention(q, k, v)
-            e1.record()
-            torch.cuda.synchronize()
-            sdpa_ms = e0.elapsed_time(e1) / reps
-        except Exception:
-            sdpa_ms = None
+    # comparison points (not part of the step): dense attention through our
+    # kernel and a library dense attention of the same shape (PyTorch SDPA)
+    dense = _dense_times(sa, q, k, v, wl.bq, o, 3) if not args.no_dense else {"ours": None, "sdpa": None}
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -363,25 +370,26 @@ def run_ours(args, wl, rank, world, local):
         e2e = {"value": round(world * dense_flops(wl) / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": q.numel() * 2, "api": "block_sparse_attention (host tensors)"}
+        del qh, kh, vh, oh
 
     hbm, bf16, bf16_s, src = peaks()
     kept = float(m["kv_cnt"].sum().item())
     mask_bytes = int(2 * B * H * N * d * 2 + 4 * kept + 4 * B * H * wl.n_qb)
     achieved = ex_flops / (attn_ms * 1e-3) / 1e12
+    d_ours, d_sdpa = dense["ours"], dense["sdpa"]
     result = {
         "metric": METRIC, "value": round(world * dense_flops(wl) / (ms_max * 1e-3) / 1e12, 3),
         "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded video-DiT-shaped Q/K/V)",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d,
-                   "block": f"{wl.bq}x{wl.bk}", "topk": wl.topk, "topp": wl.topp,
-                   "linear_branch": wl.linear, "parallelism": f"replica x{world}",
-                   "l2": "inputs larger than L2 (each tensor >= 774 MB); no flush"},
+        "config": run_config(wl, world),
         "sparse_attn_ms": round(attn_ms, 4), "mask_build_ms": round(mask_ms, 4),
         "linear_blend_ms": None if lin_ms is None else round(lin_ms, 4),
-        "dense_attn_ms": None if dense_ms is None else round(dense_ms, 3),
-        "torch_sdpa_dense_ms": None if sdpa_ms is None else round(sdpa_ms, 3),
-        "speedup_vs_dense": None if dense_ms is None else round(dense_ms / attn_ms, 2),
+        "per_call_ms": {"sparse_attn": stats(attn_t), "mask_build": stats(mask_t),
+                        "linear_blend": stats(lin_t) if lin_t else None},
+        "dense_attn_ms": None if d_ours is None else d_ours["median"],
+        "torch_sdpa_dense_ms": None if d_sdpa is None else d_sdpa["median"],
+        "speedup_vs_dense": None if d_ours is None else round(d_ours["median"] / attn_ms, 2),
         "density": round(density, 5), "executed_tflop_per_call": round(ex_flops / 1e12, 4),
         "roofline": {"kernel": "sparse_attn_kernel<128>", "bound": "tensor", "achieved": round(achieved, 1),
                      "peak": bf16, "unit": "TFLOP/s", "frac": round(achieved / bf16, 4),
@@ -398,14 +406,103 @@ def run_ours(args, wl, rank, world, local):
     return result
 
 
+PER_WORKLOAD = ("tiny", "wan13b_480p", "sink_skew", "long_245k")
+
+
+def measure_workload(sa, wl, dev, calls, warmup, dense_reps, flush):
+    """One workload's step components, each call timed on its own with CUDA
+    events (an L2 flush between calls when the inputs fit in L2), with its own
+    clock record: mask build, sparse attention (executed-tile TFLOP/s and
+    fraction of the bf16 peak), linear + blend when the workload has them, and
+    dense attention, ours and torch SDPA."""
+    lib = sa.load()
+    x = make_inputs(wl, dev)
+    q, k, v, alpha = x["q"], x["k"], x["v"], x["alpha"]
+    B, H, N, d = q.shape
+    ws_mask = torch.empty(lib.sa_build_mask_workspace_size(B, H, N, d, wl.bq, wl.bk), dtype=torch.uint8, device=dev)
+    ws_lin = torch.empty(max(1, lib.sa_linear_workspace_size(B, H, N, d)), dtype=torch.uint8, device=dev)
+    ws_blend = torch.empty(max(1, lib.sa_blend_workspace_size(B, H, N, d)), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    scratch = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush else None
+    marks = []
+    for i in range(warmup + calls):
+        if scratch is not None:
+            scratch.fill_(i & 0xFF)
+        m0 = _event()
+        m = sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp, workspace=ws_mask)
+        m1 = _event()
+        if scratch is not None:
+            scratch.fill_((i + 1) & 0xFF)
+        m2 = _event()
+        sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], out=o)
+        m3 = _event()
+        m4 = m5 = None
+        if wl.linear:
+            m4 = _event()
+            S, z = sa.sa_linear_branch(q, k, v, workspace=ws_lin)
+            sa.sa_blend(o, q, S, z, alpha, out=o, workspace=ws_blend)
+            m5 = _event()
+        if i >= warmup:
+            marks.append((m0, m1, m2, m3, m4, m5))
+        if i == warmup - 1:
+            torch.cuda.synchronize()
+            clk = ClockSampler(dev.index).__enter__()
+    torch.cuda.synchronize()
+    clk.__exit__(None, None, None)
+    sa.sa_device_status(dev)
+    mask_t = [a.elapsed_time(b) for a, b, *_ in marks]
+    attn_t = [c.elapsed_time(e) for _, _, c, e, _, _ in marks]
+    lin_t = [a.elapsed_time(b) for *_, a, b in marks if a is not None]
+    ex = executed_flops(wl, m["kv_idx"], m["kv_cnt"])
+    kept = float(m["kv_cnt"].sum().item())
+    density = kept / (B * H * wl.n_qb * wl.n_kb)
+    hbm, bf16, _, src = peaks()
+    mask_bytes = 2 * B * H * N * d * 2 + 4 * kept + 4 * B * H * wl.n_qb
+    dense = _dense_times(sa, q, k, v, wl.bq, o, dense_reps) if dense_reps else {"ours": None, "sdpa": None}
+    sa.sa_device_status(dev)
+    sp, mk = stats(attn_t), stats(mask_t)
+    res = {
+        "config": {"B": B, "H": H, "N": N, "d": d, "block": f"{wl.bq}x{wl.bk}", "topk": wl.topk,
+                   "topp": wl.topp, "linear_branch": wl.linear,
+                   "l2": "256 MB flush before each timed call" if flush else "inputs larger than L2; no flush"},
+        "density": round(density, 5), "executed_tflop_per_call": round(ex / 1e12, 5),
+        "sparse_attn_ms": sp, "mask_build_ms": mk,
+        "sparse_exec_tflops": round(ex / (sp["median"] * 1e-3) / 1e12, 1),
+        "sparse_frac_of_bf16_peak": round(ex / (sp["median"] * 1e-3) / 1e12 / bf16, 4),
+        "mask_gbs": round(mask_bytes / (mk["median"] * 1e-3) / 1e9, 1),
+        "mask_frac_of_hbm": round(mask_bytes / (mk["median"] * 1e-3) / 1e9 / hbm, 4),
+        "linear_blend_ms": stats(lin_t) if lin_t else None,
+        "dense_attn_ms": dense["ours"], "torch_sdpa_dense_ms": dense["sdpa"],
+        "speedup_vs_our_dense": None if dense["ours"] is None else round(dense["ours"]["median"] / sp["median"], 2),
+        "peaks": f"{src}: bf16 {bf16} TFLOP/s burst, HBM {hbm} GB/s; fractions from medians",
+        "clocks": clk.summary(),
+    }
+    del x, q, k, v, o, ws_mask, ws_lin, ws_blend, scratch
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_per_workload(args, dev):
+    import block_sparse_attention_softmax_b200 as sa
+    out = {}
+    for name in PER_WORKLOAD:
+        wl = WORKLOADS[name]
+        fits_l2 = wl.B * wl.H * wl.N * wl.d * 2 < (256 << 20)
+        reps = 3 if wl.N > 100000 else 5
+        out[name] = measure_workload(sa, wl, dev, calls=20, warmup=3, dense_reps=0 if args.no_dense else reps,
+                                     flush=fits_l2)
+    return out
+
+
 # ------------------------------------------------------------------ oracle (CPU)
-def oracle_step_estimate(wl, x, budget_s=20.0):
+def oracle_step_estimate(wl, x, n_heads, n_blocks=32):
     """Time the fp64 oracle on a bounded sample of one step and scale it up.
 
-    Sample: the whole mask (pool, scores, selection) of one head, attention for
-    a few query blocks of that head (scaled by kept tiles), and, with the linear
-    branch, its state and output for that head. Returns (seconds per step,
-    description, threads).
+    Sample: for each of the first n_heads heads, the whole mask (pool, scores,
+    selection), attention on every row of n_blocks query blocks (scaled by
+    the head's kept tiles over the sample's), and, with the linear branch, its
+    state and output; the per-head mean is scaled by the number of heads.
+    Returns (seconds per step, description, threads).
     """
     import numpy as np
     import oracle
@@ -414,40 +511,42 @@ def oracle_step_estimate(wl, x, budget_s=20.0):
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
         cores = os.cpu_count() or 1
-    qh, kh, vh = (oracle.as_f64(x[n][0, 0]) for n in ("q", "k", "v"))
-    t0 = time.perf_counter()
-    ref = oracle.build_mask(qh, kh, wl.bq, wl.bk, wl.topk, wl.topp)
-    t_mask = time.perf_counter() - t0
     rng = np.random.default_rng(0)
-    n_blocks = min(wl.n_qb, 4)
-    blocks = rng.choice(wl.n_qb, size=n_blocks, replace=False)
-    rows = np.concatenate([np.arange(b * wl.bq, min(wl.N, (b + 1) * wl.bq)) for b in blocks])
-    t0 = time.perf_counter()
-    oracle.masked_attention(qh, kh, vh, ref["mask"], wl.bq, wl.bk, rows=rows)
-    t_attn_sample = time.perf_counter() - t0
-    tiles_sample = float(ref["mask"][blocks].sum())
-    tiles_head = float(ref["mask"].sum())
-    t_attn_head = t_attn_sample * tiles_head / max(tiles_sample, 1.0)
-    t_lin = 0.0
-    if wl.linear:
+    t_mask = t_attn = t_attn_sample = t_lin = 0.0
+    n_heads = min(n_heads, x["q"].shape[1])
+    nb = min(wl.n_qb, n_blocks)
+    for h in range(n_heads):
+        qh, kh, vh = (oracle.as_f64(x[n][0, h]) for n in ("q", "k", "v"))
         t0 = time.perf_counter()
-        S, z = oracle.linear_state(kh, vh)
-        oracle.linear_out(qh, S, z)
-        t_lin = time.perf_counter() - t0
-    per_head = t_mask + t_attn_head + t_lin
+        ref = oracle.build_mask(qh, kh, wl.bq, wl.bk, wl.topk, wl.topp)
+        t_mask += time.perf_counter() - t0
+        blocks = rng.choice(wl.n_qb, size=nb, replace=False)
+        rows = np.concatenate([np.arange(b * wl.bq, min(wl.N, (b + 1) * wl.bq)) for b in blocks])
+        t0 = time.perf_counter()
+        oracle.masked_attention(qh, kh, vh, ref["mask"], wl.bq, wl.bk, rows=rows)
+        dt = time.perf_counter() - t0
+        t_attn_sample += dt
+        t_attn += dt * float(ref["mask"].sum()) / max(float(ref["mask"][blocks].sum()), 1.0)
+        if wl.linear:
+            t0 = time.perf_counter()
+            S, z = oracle.linear_state(kh, vh)
+            oracle.linear_out(qh, S, z)
+            t_lin += time.perf_counter() - t0
+    per_head = (t_mask + t_attn + t_lin) / n_heads
     sec = per_head * wl.B * wl.H
-    desc = (f"1 of {wl.B * wl.H} heads: full mask ({t_mask:.2f}s), attention on {n_blocks} query blocks "
-            f"scaled by kept tiles ({t_attn_sample:.2f}s -> {t_attn_head:.1f}s/head)"
-            + (f", linear branch ({t_lin:.2f}s)" if wl.linear else "") + ", scaled x heads")
+    desc = (f"{n_heads} of {wl.B * wl.H} heads: full masks ({t_mask:.2f}s), attention on every row of {nb} "
+            f"query blocks per head ({t_attn_sample:.2f}s), scaled by kept tiles to whole heads"
+            + (f", linear branch ({t_lin:.2f}s)" if wl.linear else "")
+            + "; mean per head scaled by the head count (extrapolated)")
     return sec, desc, cores
 
 
 def run_reference(args, wl):
     """The oracle as the reference arm: each step is a bounded sample of the workload."""
-    x = make_inputs(wl, "cpu") if wl.N * wl.d * wl.H <= 2 ** 26 else _one_head_inputs(wl)
+    x = _head_inputs(wl, REF_HEADS)
     secs = []
     for i in range(args.warmup + args.steps):
-        s, desc, cores = oracle_step_estimate(wl, x)
+        s, desc, cores = oracle_step_estimate(wl, x, REF_HEADS)
         if i >= args.warmup:
             secs.append(s)
     ms = statistics.mean(secs) * 1e3
@@ -456,20 +555,23 @@ def run_reference(args, wl):
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded video-DiT-shaped Q/K/V)",
-            "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d,
-                       "block": f"{wl.bq}x{wl.bk}", "topk": wl.topk, "topp": wl.topp,
-                       "linear_branch": wl.linear},
+            "config": run_config(wl, int(os.environ.get("WORLD_SIZE", "1"))),
+            "extrapolated": True,
             "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": cores,
-                             "kind": "oracle", "sample": desc},
+                             "kind": "oracle", "sample": desc, "extrapolated": True},
             "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
-def _one_head_inputs(wl):
-    """Inputs of the first head only (the oracle sample never reads the others)."""
+REF_HEADS = 2          # heads per reference-arm step (a few seconds of CPU work each)
+BASELINE_HEADS = 8     # heads of the cpu_baseline sample (about 10 s of CPU work)
+
+
+def _head_inputs(wl, n):
+    """Inputs of the first n heads only (the oracle sample never reads the others;
+    the generator draws head by head, so these equal the full workload's)."""
     from dataclasses import replace
-    one = replace(wl, H=1)
-    return make_inputs(one, "cpu")
+    return make_inputs(replace(wl, H=min(n, wl.H)), "cpu")
 
 
 def main():
@@ -482,6 +584,8 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the per-workload measurements of the other four configurations")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -493,13 +597,23 @@ def main():
         return
     rank, world, local = dist_setup(args.gpus)
     res = run_ours(args, wl, rank, world, local)
+    if world == 1 and not args.no_per_workload:
+        res["per_workload"] = run_per_workload(args, torch.device("cuda", local))
     if rank == 0:
         if not args.no_cpu_baseline:
-            x = _one_head_inputs(wl)
-            sec, desc, cores = oracle_step_estimate(wl, x)
+            x = _head_inputs(wl, BASELINE_HEADS)
+            sec, desc, cores = oracle_step_estimate(wl, x, BASELINE_HEADS)
             res["cpu_baseline"] = {"value": round(dense_flops(wl) / sec / 1e12, 6), "unit": "TFLOP/s",
                                    "cores": cores, "kind": "oracle", "sample": desc,
-                                   "ms_per_step": round(sec * 1e3, 1)}
+                                   "ms_per_step": round(sec * 1e3, 1), "extrapolated": True}
+            try:
+                from threadpoolctl import threadpool_limits
+                with threadpool_limits(1):
+                    sec1, _, _ = oracle_step_estimate(wl, x, BASELINE_HEADS)
+                res["cpu_baseline"]["one_thread"] = {"value": round(dense_flops(wl) / sec1 / 1e12, 6),
+                                                     "ms_per_step": round(sec1 * 1e3, 1), "cores": 1}
+            except ImportError:
+                pass
         print(json.dumps(res), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

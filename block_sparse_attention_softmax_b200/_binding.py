@@ -41,6 +41,10 @@ _SIGNATURES = {
     "sa_blend_workspace_size": (c_size_t, [c_int] * 4),
     "sa_blend": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                          c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "sa_diag_set_device_status": (c_int, [c_int]),
+    "sa_diag_set_wait_limit": (c_int, [ctypes.c_longlong]),
+    "sa_diag_wait_timeout": (c_int, [c_void_p, c_void_p]),
+    "sa_diag_exp2": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_void_p]),
 }
 
 
@@ -150,6 +154,32 @@ def sa_status_string(status: int) -> str:
 def sa_device_status(device=None):
     device = device or torch.device("cuda", torch.cuda.current_device())
     _call("sa_device_status", _stream(device))
+
+
+def sa_diag_set_device_status(code: int):
+    _call("sa_diag_set_device_status", int(code))
+
+
+def sa_diag_set_wait_limit(cycles: int):
+    """Bound of every device-side wait, in SM cycles (<= 0 restores the default)."""
+    _call("sa_diag_set_wait_limit", int(cycles))
+
+
+def sa_diag_wait_timeout(device=None):
+    """Runs one bounded wait that nothing completes; returns (completed, abort flag)."""
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    out = torch.full((2,), -1, dtype=torch.int32, device=device)
+    _call("sa_diag_wait_timeout", _ptr(out), _stream(device))
+    return tuple(int(t) for t in out.cpu())
+
+
+def sa_diag_exp2(x):
+    """(FMA-pipe polynomial 2^x, ex2.approx 2^x) of a float32 CUDA tensor."""
+    _expect("x", x, x.shape, torch.float32)
+    _on_device(x.device, x=x)
+    yp, ym = torch.empty_like(x), torch.empty_like(x)
+    _call("sa_diag_exp2", _ptr(x), _ptr(yp), _ptr(ym), x.numel(), _stream(x.device))
+    return yp, ym
 
 
 def sa_pool_blocks(q, k, bq, bk):

@@ -6,3 +6,4 @@
 #include "linear_kernels.cu"
 #include "sa_api.cu"
 #include "noalloc.cu"
+#include "diag.cu"

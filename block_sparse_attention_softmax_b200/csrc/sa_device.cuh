@@ -23,6 +23,10 @@ static __device__ int g_device_status = 0;
 constexpr int kStatusTimeout = 5;
 // About one second at 1.9 GHz; waits normally end within microseconds.
 constexpr long long kWaitLimitCycles = 2000000000LL;
+// Limit of a bounded wait, in SM clock cycles. Read only once a wait has not
+// completed at its first try; a diagnostic entry point may lower it so that
+// a test can make a wait run out.
+static __device__ long long g_wait_limit = kWaitLimitCycles;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -58,14 +62,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait until the phase with the given parity has completed. Returns false (and
 // records a timeout in the device status word and in *abort) if it does not
-// complete within kWaitLimitCycles, or if another role already aborted.
+// complete within g_wait_limit cycles, or if another role already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
+  const long long limit = *static_cast<volatile long long*>(&g_wait_limit);
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       atomicExch(&g_device_status, kStatusTimeout);
       return false;

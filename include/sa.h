@@ -174,6 +174,31 @@ int sa_build_mask_noalloc(const uint16_t* q, const uint16_t* k, int B, int H, in
                           int bq, int bk, double topk_frac, double topp, double scale,
                           int32_t* kv_idx, int32_t* kv_cnt, uint8_t* mask_opt, void* stream);
 
+/* Diagnostics (no counterpart in the pages). They exist so that tests can
+ * reach the error-reporting path and the softmax's exponential helpers
+ * directly, without causing a fault.
+ *
+ * sa_diag_set_device_status: writes `code` into the device status word that
+ *   sa_device_status() reads and clears (synchronous; 0 clears it).
+ * sa_diag_set_wait_limit: sets the bound, in SM clock cycles, of every
+ *   device-side wait of the library's kernels (synchronous; <= 0 restores the
+ *   default of 2e9 cycles, about a second). A lowered limit makes waits run
+ *   out and the kernels stop early with SA_ERR_DEVICE_TIMEOUT: meant only for
+ *   tests, which must restore it.
+ * sa_diag_wait_timeout: launches one thread that waits on an mbarrier nothing
+ *   arrives at, through the same bounded wait as the kernels; out[0] = 1 if
+ *   the wait completed (never expected), out[1] = the CTA's abort flag after
+ *   the wait. `out` is a device int[2]. The status word then reports the
+ *   timeout.
+ * sa_diag_exp2: y_poly[i] = the FMA-pipe polynomial 2^x[i] used for one
+ *   column pair in four of the attention softmax (inputs clamped at -126, so
+ *   values at or below 2^-125 for x <= -126), y_mufu[i] = ex2.approx(x[i]).
+ *   Device float arrays of n elements, 16-byte aligned not required. */
+int sa_diag_set_device_status(int code);
+int sa_diag_set_wait_limit(long long cycles);
+int sa_diag_wait_timeout(int* out, void* stream);
+int sa_diag_exp2(const float* x, float* y_poly, float* y_mufu, int n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

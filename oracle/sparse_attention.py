@@ -203,7 +203,9 @@ def masked_attention(q, k, v, mask, bq, bk, scale=None, rows=None):
 
     rows: iterable of query indices to evaluate (default: all). Returns
     (O [len(rows), d], LSE [len(rows)]); a row with no kept key gives O = 0 and
-    LSE = -inf.
+    LSE = -inf. Rows of one query block share that block's kept keys, so they
+    are evaluated together: one logits matrix, then each row's own max,
+    exponentials and sum.
     """
     N, d = q.shape
     if scale is None:
@@ -211,17 +213,19 @@ def masked_attention(q, k, v, mask, bq, bk, scale=None, rows=None):
     rows = np.arange(N) if rows is None else np.asarray(list(rows), dtype=np.int64)
     out = np.zeros((rows.shape[0], d), dtype=np.float64)
     lse = np.full(rows.shape[0], -np.inf, dtype=np.float64)
-    for n, i in enumerate(rows):
-        kept = np.nonzero(mask[i // bq])[0]
+    qb_of_row = rows // bq
+    for qb in np.unique(qb_of_row):
+        at = np.nonzero(qb_of_row == qb)[0]
+        kept = np.nonzero(mask[qb])[0]
         if kept.shape[0] == 0:
             continue
         keys = np.concatenate([np.arange(kb * bk, min(N, (kb + 1) * bk)) for kb in kept])
-        logits = scale * (k[keys] @ q[i])
-        m = logits.max()
+        logits = scale * (q[rows[at]] @ k[keys].T)          # [rows of this block, kept keys]
+        m = logits.max(axis=1, keepdims=True)
         w = np.exp(logits - m)
-        z = w.sum()
-        out[n] = (w @ v[keys]) / z
-        lse[n] = m + math.log(z)
+        z = w.sum(axis=1, keepdims=True)
+        out[at] = (w @ v[keys]) / z
+        lse[at] = m[:, 0] + np.log(z[:, 0])
     return out, lse
 
 

@@ -110,3 +110,11 @@ def test_build_mask_launch_count(lib):
         os.environ.pop("SA_MASK_BUILDER", None)
         if saved is not None:
             os.environ["SA_MASK_BUILDER"] = saved
+
+
+def test_diagnostic_entry_points_validate_before_launch(lib):
+    fake = P(0x1000)
+    assert lib.sa_diag_exp2(fake, fake, fake, -1, None) == -1
+    assert lib.sa_diag_exp2(None, fake, fake, 8, None) == -1
+    assert lib.sa_diag_exp2(None, None, None, 0, None) == 0      # nothing to do, nothing launched
+    assert lib.sa_diag_wait_timeout(None, None) == -1

@@ -231,67 +231,120 @@ def test_candidate_hand_back_all_rows(cuda_lib, monkeypatch):
     sa.sa_device_status()
 
 
-# ------------------------------------------------------------------ full-size workloads (sampled)
+# ------------------------------------------------------------------ full-size workloads
 FULL = ["wan13b_480p", "wan14b_720p", "sink_skew", "long_245k"]
 
 
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_workload(cuda_lib, name):
+    """Full-size workloads: the mask of every head against the oracle, row by
+    row; attention on the oracle's mask of every head, on every row of at
+    least 8 sampled query blocks per head (first, ragged tail, densest,
+    sparsest, random), O and LSE; with the linear branch, S and z of every
+    head and the blended output on the same rows."""
     sa = cuda_lib
     wl = WORKLOADS[name]
     x = make_inputs(wl, DEV)
     q, k, v = x["q"], x["k"], x["v"]
     rng = np.random.default_rng(wl.seed)
-    n_heads = 2 if wl.N > 100000 else 3
-    hs = sorted({0, wl.H - 1} | set(rng.choice(wl.H, size=n_heads, replace=False).tolist()))[:n_heads + 1]
-    if wl.kind == "sink" and x["flat_heads"]:
-        hs = sorted(set(hs) | {x["flat_heads"][0]})
-    heads = [(0, h) for h in hs]
     qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
     out = sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp, want_mask=True)
     _assert_same_lists(out, sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp))
     torch.cuda.synchronize()
     idx, cnt = out["kv_idx"].cpu().numpy(), out["kv_cnt"].cpu().numpy()
-    gmask = out["mask"].clone()
+    gmask = out["mask"].cpu().numpy().astype(bool)
+    ext = torch.empty(wl.B, wl.H, wl.n_qb, wl.n_kb, dtype=torch.uint8)
     totals = {"exact": 0, "score_tie": 0, "cumsum_tie": 0}
     ora = {}
-    for (b, h) in heads:
-        ref = _oracle_head_mask(qc, kc, b, h, wl.bq, wl.bk, wl.topk, wl.topp)
-        st = compare_mask_rows(idx[b, h], cnt[b, h], ref["s"], wl.topk, wl.topp)
-        assert not st["bad"], f"{name} head {h}: {st['bad'][:3]}"
-        for kk in totals:
-            totals[kk] += st[kk]
-        ora[(b, h)] = ref
-        gmask[b, h] = torch.from_numpy(ref["mask"].astype(np.uint8)).to(DEV)
-    density = float(cnt.sum()) / (wl.H * wl.n_qb * wl.n_kb)
+    for b in range(wl.B):
+        for h in range(wl.H):
+            ref = _oracle_head_mask(qc, kc, b, h, wl.bq, wl.bk, wl.topk, wl.topp)
+            st = compare_mask_rows(idx[b, h], cnt[b, h], ref["s"], wl.topk, wl.topp, ora_mask=ref["mask"])
+            assert not st["bad"], f"{name} head {h}: {st['bad'][:3]}"
+            for kk in totals:
+                totals[kk] += st[kk]
+            ora[(b, h)] = (ref["mask"], (gmask[b, h] == ref["mask"]).all(1))
+            ext[b, h] = torch.from_numpy(ref["mask"].astype(np.uint8))
+    assert sum(totals.values()) == wl.B * wl.H * wl.n_qb
+    density = float(cnt.sum()) / (wl.B * wl.H * wl.n_qb * wl.n_kb)
     print(f"{name}: mask rows {totals}, realised density {density:.4f}")
-    # attention on the oracle's mask for the sampled heads (GPU mask elsewhere)
-    o = sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, ext_mask=gmask)
+    # attention on the oracle's mask (every head), and on the GPU's own lists
+    o, lse = sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, ext_mask=ext.to(DEV), want_lse=True)
     o_list = sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=out["kv_idx"], kv_cnt=out["kv_cnt"])
     torch.cuda.synchronize()
-    for (b, h), ref in ora.items():
-        rows = sample_rows(wl.n_qb, wl.bq, wl.N, ref["mask"].sum(1), rng)
-        ro, _ = _oracle_attention_rows(qc, kc, vc, ref["mask"], b, h, wl.bq, wl.bk, rows)
-        got = o[b, h][torch.from_numpy(rows).to(DEV)].float().cpu().numpy()
-        assert_close(got, ro, f"{name} O head {h}")
-        same = np.nonzero((out["mask"][b, h].cpu().numpy().astype(bool) == ref["mask"]).all(1))[0]
-        sel = torch.from_numpy(np.concatenate([np.arange(r * wl.bq, min(wl.N, (r + 1) * wl.bq)) for r in same[:8]])).to(DEV)
-        assert torch.equal(o_list[b, h][sel], o[b, h][sel])
+    rows_of = {}
+    for (b, h), (mask, same) in ora.items():
+        rows = sample_rows(wl.n_qb, wl.bq, wl.N, mask.sum(1), rng)
+        rows_of[(b, h)] = rows
+        ro, rl = _oracle_attention_rows(qc, kc, vc, mask, b, h, wl.bq, wl.bk, rows)
+        sel = torch.from_numpy(rows).to(DEV)
+        assert_close(o[b, h][sel].float().cpu().numpy(), ro, f"{name} O head {h}")
+        assert_close(lse[b, h][sel].cpu().numpy(), rl, f"{name} LSE head {h}", 1e-2, 1e-3)
+        # rows whose GPU mask equals the oracle's: the list path gives the same bits
+        eq = rows[same[rows // wl.bq]]
+        if eq.size:
+            eq = torch.from_numpy(eq).to(DEV)
+            assert torch.equal(o_list[b, h][eq], o[b, h][eq])
     if wl.linear:
         alpha = x["alpha"]
         S, z = sa.sa_linear_branch(q, k, v)
         ob = sa.sa_blend(o, q, S, z, alpha)
         torch.cuda.synchronize()
-        for (b, h) in heads[:2]:
+        for (b, h), (mask, _) in ora.items():
             kS, kz = oracle.linear_state(_f64(kc[b, h]), _f64(vc[b, h]))
             # phi(k) is rounded to bf16 on the GPU: relative error ~4e-3 per term
             assert np.abs(S[b, h].cpu().numpy() - kS).max() <= 5e-3 * np.abs(kS).max()
             assert np.abs(z[b, h].cpu().numpy() - kz).max() <= 5e-3 * np.abs(kz).max()
-            rows = sample_rows(wl.n_qb, wl.bq, wl.N, ora[(b, h)]["mask"].sum(1), rng)
-            ro, _ = _oracle_attention_rows(qc, kc, vc, ora[(b, h)]["mask"], b, h, wl.bq, wl.bk, rows)
+            rows = rows_of[(b, h)]
+            ro, _ = _oracle_attention_rows(qc, kc, vc, mask, b, h, wl.bq, wl.bk, rows)
             ol = oracle.linear_out(_f64(qc[b, h])[rows], kS, kz)
             ref = oracle.blend(ro, ol, alpha[h].double().cpu().numpy())
             assert_close(ob[b, h][torch.from_numpy(rows).to(DEV)].float().cpu().numpy(), ref, f"{name} blend head {h}")
+    sa.sa_device_status()
+
+
+# ------------------------------------------------------------------ several items per CTA, all rows
+@pytest.mark.parametrize("ragged", [False, True])
+def test_many_items_per_cta_all_rows(cuda_lib, ragged):
+    """8 heads of 16384 (or 16344: ragged last query and key blocks) tokens in
+    128-row query blocks: 1,024 work items, about 7 per persistent CTA, so the
+    second Q slot, the wrap of the item ring and the hand-over of O between
+    items all run. Every output row and LSE is compared with the oracle, on
+    the GPU-built lists (odd kept counts among them) and on an external mask
+    that empties runs of consecutive items (the zero-fill of skipped items)."""
+    sa = cuda_lib
+    B, H, d, bq, bk = 1, 8, 128, 128, 64
+    N = 16344 if ragged else 16384
+    q, k, v = random_qkv(B, H, N, d, seed=4242 + N, device=DEV)
+    q = (q.float() * 2.0).to(torch.bfloat16)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    m = sa.sa_build_mask(q, k, bq, bk, 0.04, 0.6, want_mask=True)
+    o1, l1 = sa.sa_sparse_attn_fwd(q, k, v, bq, bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], want_lse=True)
+    gm = m["mask"].clone()
+    cnt = m["kv_cnt"].cpu().numpy()
+    assert (cnt % 2 == 1).any() and (cnt % 2 == 0).any()
+    if ragged:
+        assert gm[..., nkb - 1].any()              # the short last key block is kept somewhere
+    ext = gm.clone()
+    rng = np.random.default_rng(N)
+    for h in range(H):
+        for start in rng.choice(nqb - 4, size=3, replace=False):
+            ext[0, h, start:start + 1 + (h % 4)] = 0     # 1-4 consecutive empty items
+    ext[0, H - 1, nqb - 1] = 0                           # the very last item empty
+    o2, l2 = sa.sa_sparse_attn_fwd(q, k, v, bq, bk, ext_mask=ext, want_lse=True)
+    torch.cuda.synchronize()
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    for h in range(H):
+        for mask_t, o, lse in ((gm, o1, l1), (ext, o2, l2)):
+            mk = mask_t[0, h].cpu().numpy().astype(bool)
+            ro, rl = _oracle_attention_rows(qc, kc, vc, mk, 0, h, bq, bk, None)
+            assert_close(o[0, h].float().cpu().numpy(), ro, f"O head {h}")
+            empty = ~mk.any(1)
+            rows_empty = np.repeat(empty, bq)[:N]
+            got_l = lse[0, h].cpu().numpy()
+            assert np.isneginf(got_l[rows_empty]).all()
+            assert (o[0, h].float().cpu().numpy()[rows_empty] == 0).all()
+            assert_close(got_l[~rows_empty], rl[~rows_empty], f"LSE head {h}", 1e-2, 1e-3)
     sa.sa_device_status()
 
 

@@ -94,3 +94,29 @@ def test_cumsum_tie_never_goes_below_top_k():
     _, L, k_sel, _ = oracle.hybrid_row(s, k_frac, p)
     assert (L, k_sel) == (5, 5)
     assert _verdict(s, _oracle_prefix(s, 4), k_frac, p) == "bad"        # below K_sel
+
+
+def test_fast_path_with_the_oracle_mask_gives_the_same_verdicts():
+    """Given the oracle's mask, rows equal to it are counted exact without the
+    tie analysis; every other row still gets it, so the verdicts match."""
+    rng = np.random.default_rng(21)
+    n_qb, n_kb, k_frac, p = 12, 40, 0.1, 0.8
+    s = rng.standard_normal((n_qb, n_kb)) * 2.0
+    s[3, 5] = s[3, int(oracle.descending_order(s[3])[0])]          # a tie with the top block
+    ora = np.zeros((n_qb, n_kb), dtype=bool)
+    for r in range(n_qb):
+        ora[r] = oracle.hybrid_row(s[r], k_frac, p)[0]
+    gpu = ora.copy()
+    order = oracle.descending_order(s[7])
+    L = int(ora[7].sum())
+    gpu[7, order[L - 1]] = False                                   # one short: bad
+    gpu[9, oracle.descending_order(s[9])[int(ora[9].sum())]] = True  # one extra: bad
+    idx = np.full((n_qb, n_kb), -1, dtype=np.int64)
+    cnt = gpu.sum(1)
+    for r in range(n_qb):
+        kept = np.nonzero(gpu[r])[0]
+        idx[r, :kept.shape[0]] = kept
+    slow = compare_mask_rows(idx, cnt, s, k_frac, p)
+    fast = compare_mask_rows(idx, cnt, s, k_frac, p, ora_mask=ora)
+    assert slow["exact"] == fast["exact"] == n_qb - 2
+    assert [b[0] for b in slow["bad"]] == [b[0] for b in fast["bad"]] == [7, 9]

@@ -314,6 +314,74 @@ def test_blend_endpoints_and_midpoint():
     assert np.allclose(oracle.blend(a, b, np.full(4, 0.5)), (a + b) / 2)
 
 
+# ---------------------------------------------------------------- build_mask wiring
+def _brute_force_mask(q, k, bq, bk, k_frac, p, scale):
+    """The whole mask of one head from the definitions, by scalar loops only:
+    block means over valid tokens (query blocks of bq tokens, key blocks of bk),
+    s = scale * sum_c Qbar_c Kbar_c, P by exp and sum, ranks by counting
+    (higher score first, equal scores lower index first), keep rank < max(K_sel, m_p)."""
+    N, d = q.shape
+    nq, nk = -(-N // bq), -(-N // bk)
+
+    def means(x, b, n):
+        out = []
+        for blk in range(n):
+            acc, cnt = [0.0] * d, 0
+            for t in range(blk * b, min(N, (blk + 1) * b)):
+                for c in range(d):
+                    acc[c] += float(x[t, c])
+                cnt += 1
+            out.append([a / cnt for a in acc])
+        return out
+
+    qm, km = means(q, bq, nq), means(k, bk, nk)
+    k_sel = min(nk, max(1, math.ceil(k_frac * nk - 1e-9)))
+    mask = np.zeros((nq, nk), dtype=bool)
+    for r in range(nq):
+        s = [scale * sum(qm[r][c] * km[j][c] for c in range(d)) for j in range(nk)]
+        top = max(s)
+        e = [math.exp(x - top) for x in s]
+        z = sum(e)
+        P = [x / z for x in e]
+        rank = [sum(1 for j in range(nk) if s[j] > s[i] or (s[j] == s[i] and j < i)) for i in range(nk)]
+        by_rank = [P[i] for i in sorted(range(nk), key=lambda i: rank[i])]
+        m_p, acc = nk, 0.0
+        for m in range(1, nk + 1):
+            acc += by_rank[m - 1]
+            if acc >= p:
+                m_p = m
+                break
+        L = max(k_sel, m_p)
+        for i in range(nk):
+            mask[r, i] = rank[i] < L
+    return mask
+
+
+@pytest.mark.parametrize("N,d,bq,bk,k_frac,p,seed", [
+    (200, 8, 32, 16, 0.2, 0.7, 31),     # 7 query blocks (last 8 tokens), 13 key blocks (last 8)
+    (700, 16, 128, 64, 0.2, 0.6, 32),   # the video geometry's 2:1 block ratio, both tails 60 tokens
+    (130, 8, 16, 64, 0.34, 0.7, 33),    # key blocks wider than query blocks
+])
+def test_build_mask_wiring_by_brute_force(N, d, bq, bk, k_frac, p, seed):
+    """build_mask's pooling sizes (Q by bq, K by bk), its default scale 1/sqrt(d)
+    and its per-row selection, against scalar loops on ragged bq != bk shapes;
+    the rows' cumulative sums are checked to stay clear of p so rounding order
+    cannot decide them."""
+    rng = _rng(seed)
+    q = rng.standard_normal((N, d)) * 2.0 + rng.standard_normal(d)
+    k = rng.standard_normal((N, d)) + rng.standard_normal(d)
+    out = oracle.build_mask(q, k, bq, bk, k_frac, p)
+    want = _brute_force_mask(q, k, bq, bk, k_frac, p, 1.0 / math.sqrt(d))
+    assert out["mask"].shape == want.shape == (-(-N // bq), -(-N // bk))
+    s = out["s"]
+    for r in range(s.shape[0]):
+        csum = np.cumsum(oracle.block_softmax(s[r])[oracle.descending_order(s[r])])
+        assert np.abs(csum - p).min() > 1e-9
+    assert (out["mask"] == want).all()
+    # the mask depends on the scale: 1/d in place of 1/sqrt(d) changes some row here
+    assert (_brute_force_mask(q, k, bq, bk, k_frac, p, 1.0 / d) != want).any()
+
+
 # ---------------------------------------------------------------- golden regression
 def test_tiny_workload_masks_match_golden():
     import os
