@@ -289,17 +289,18 @@ def run_ours(args, wl, rank, world, local):
     B, H, N, d = q.shape
     ws_mask = torch.empty(lib.sa_build_mask_workspace_size(B, H, N, d, wl.bq, wl.bk), dtype=torch.uint8, device=dev)
     ws_lin = torch.empty(max(1, lib.sa_linear_workspace_size(B, H, N, d)), dtype=torch.uint8, device=dev)
-    ws_blend = torch.empty(max(1, lib.sa_blend_workspace_size(B, H, N, d)), dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
+    o_l = torch.empty_like(q) if wl.linear else None
 
     # our kernels per step: the mask builder's (pooling, then scores and
     # selection, or row statistics, candidate scores, candidate selection and
     # two hand-back launches that return at once when no row was handed back,
-    # as the library reports for this shape); attention; linear state, its
-    # fixed-order reduction, and the fused output + blend
+    # as the library reports for this shape); with the linear branch, its
+    # state, the state's fixed-order reduction and O_l; then the sparse
+    # attention, which blends O_l into its output
     launches_per_step = lib.sa_build_mask_launches(B, H, N, d, wl.bq, wl.bk) + 1 + (3 if wl.linear else 0)
 
-    # (start, after mask, after attention, after linear + blend) events of each timed step
+    # (start, after mask, after linear branch, after attention) events of each timed step
     marks = []
 
     def step(record=False):
@@ -308,14 +309,14 @@ def run_ours(args, wl, rank, world, local):
         m = sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp, workspace=ws_mask)
         if record:
             m1 = _event()
-        sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], out=o)
+        if wl.linear:
+            sa.sa_linear_branch(q, k, v, want_ol=True, workspace=ws_lin, out_ol=o_l)
         if record:
             m2 = _event()
-        if wl.linear:
-            S, z = sa.sa_linear_branch(q, k, v, workspace=ws_lin)
-            sa.sa_blend(o, q, S, z, alpha, out=o, workspace=ws_blend)
+        sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], out=o,
+                              o_l=o_l, alpha=alpha if wl.linear else None)
         if record:
-            marks.append((m0, m1, m2, _event() if wl.linear else None))
+            marks.append((m0, m1, m2, _event()))
         return m
 
     for _ in range(args.warmup):
@@ -338,8 +339,8 @@ def run_ours(args, wl, rank, world, local):
     ms = t0.elapsed_time(t1) / args.steps
     ms_max = max_over_ranks(ms, world, dev)
     mask_t = [a.elapsed_time(b) for a, b, _, _ in marks]
-    attn_t = [b.elapsed_time(c) for _, b, c, _ in marks]
-    lin_t = [c.elapsed_time(e) for _, _, c, e in marks if e is not None]
+    lin_t = [b.elapsed_time(c) for _, b, c, _ in marks] if wl.linear else []
+    attn_t = [c.elapsed_time(e) for _, _, c, e in marks]
     attn_ms, mask_ms = statistics.mean(attn_t), statistics.mean(mask_t)
     lin_ms = statistics.mean(lin_t) if lin_t else None
     sa.sa_device_status(dev)
@@ -384,9 +385,10 @@ def run_ours(args, wl, rank, world, local):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded video-DiT-shaped Q/K/V)",
         "config": run_config(wl, world),
         "sparse_attn_ms": round(attn_ms, 4), "mask_build_ms": round(mask_ms, 4),
-        "linear_blend_ms": None if lin_ms is None else round(lin_ms, 4),
+        "linear_branch_ms": None if lin_ms is None else round(lin_ms, 4),
+        "blend": "in the sparse attention epilogue" if wl.linear else None,
         "per_call_ms": {"sparse_attn": stats(attn_t), "mask_build": stats(mask_t),
-                        "linear_blend": stats(lin_t) if lin_t else None},
+                        "linear_branch": stats(lin_t) if lin_t else None},
         "dense_attn_ms": None if d_ours is None else d_ours["median"],
         "torch_sdpa_dense_ms": None if d_sdpa is None else d_sdpa["median"],
         "speedup_vs_dense": None if d_ours is None else round(d_ours["median"] / attn_ms, 2),
@@ -421,8 +423,8 @@ def measure_workload(sa, wl, dev, calls, warmup, dense_reps, flush):
     B, H, N, d = q.shape
     ws_mask = torch.empty(lib.sa_build_mask_workspace_size(B, H, N, d, wl.bq, wl.bk), dtype=torch.uint8, device=dev)
     ws_lin = torch.empty(max(1, lib.sa_linear_workspace_size(B, H, N, d)), dtype=torch.uint8, device=dev)
-    ws_blend = torch.empty(max(1, lib.sa_blend_workspace_size(B, H, N, d)), dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
+    o_l = torch.empty_like(q) if wl.linear else None
     scratch = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush else None
     marks = []
     for i in range(warmup + calls):
@@ -433,15 +435,15 @@ def measure_workload(sa, wl, dev, calls, warmup, dense_reps, flush):
         m1 = _event()
         if scratch is not None:
             scratch.fill_((i + 1) & 0xFF)
-        m2 = _event()
-        sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], out=o)
-        m3 = _event()
         m4 = m5 = None
         if wl.linear:
             m4 = _event()
-            S, z = sa.sa_linear_branch(q, k, v, workspace=ws_lin)
-            sa.sa_blend(o, q, S, z, alpha, out=o, workspace=ws_blend)
+            sa.sa_linear_branch(q, k, v, want_ol=True, workspace=ws_lin, out_ol=o_l)
             m5 = _event()
+        m2 = _event()
+        sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], out=o,
+                              o_l=o_l, alpha=alpha if wl.linear else None)
+        m3 = _event()
         if i >= warmup:
             marks.append((m0, m1, m2, m3, m4, m5))
         if i == warmup - 1:
@@ -471,13 +473,13 @@ def measure_workload(sa, wl, dev, calls, warmup, dense_reps, flush):
         "sparse_frac_of_bf16_peak": round(ex / (sp["median"] * 1e-3) / 1e12 / bf16, 4),
         "mask_gbs": round(mask_bytes / (mk["median"] * 1e-3) / 1e9, 1),
         "mask_frac_of_hbm": round(mask_bytes / (mk["median"] * 1e-3) / 1e9 / hbm, 4),
-        "linear_blend_ms": stats(lin_t) if lin_t else None,
+        "linear_branch_ms": stats(lin_t) if lin_t else None,
         "dense_attn_ms": dense["ours"], "torch_sdpa_dense_ms": dense["sdpa"],
         "speedup_vs_our_dense": None if dense["ours"] is None else round(dense["ours"]["median"] / sp["median"], 2),
         "peaks": f"{src}: bf16 {bf16} TFLOP/s burst, HBM {hbm} GB/s; fractions from medians",
         "clocks": clk.summary(),
     }
-    del x, q, k, v, o, ws_mask, ws_lin, ws_blend, scratch
+    del x, q, k, v, o, o_l, ws_mask, ws_lin, scratch
     torch.cuda.empty_cache()
     return res
 

@@ -33,6 +33,10 @@ _SIGNATURES = {
     "sa_sparse_attn_fwd": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
                                    c_int, c_int, c_void_p, c_void_p, c_void_p, c_double,
                                    c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "sa_sparse_attn_blend_fwd": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
+                                         c_int, c_int, c_void_p, c_void_p, c_void_p, c_double,
+                                         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                         c_void_p]),
     "sa_dense_attn_fwd": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
                                   c_int, c_double, c_void_p, c_void_p, c_void_p]),
     "sa_linear_workspace_size": (c_size_t, [c_int] * 4),
@@ -216,8 +220,17 @@ def sa_build_mask(q, k, bq, bk, topk, topp, scale=0.0, want_mask=False, want_poo
 
 
 def sa_sparse_attn_fwd(q, k, v, bq, bk, kv_idx=None, kv_cnt=None, ext_mask=None, scale=0.0,
-                       want_lse=False, out=None, workspace=None):
+                       want_lse=False, out=None, workspace=None, o_l=None, alpha=None):
+    """Sparse attention; with o_l and alpha (sa_sparse_attn_blend_fwd) the
+    epilogue also blends O = alpha * O_s + (1 - alpha) * O_l."""
     B, H, N, d = _qkv(q, k, v)
+    if (o_l is None) != (alpha is None):
+        raise ValueError("o_l and alpha go together")
+    if o_l is not None:
+        _expect("o_l", o_l, q.shape, torch.bfloat16)
+        _expect("alpha", alpha, (H, d), torch.float32)
+        if out is not None and out.data_ptr() == o_l.data_ptr():
+            raise ValueError("out must not alias o_l")
     nqb, nkb = -(-N // bq), -(-N // bk)
     if kv_idx is not None:
         _expect("kv_idx", kv_idx, (B, H, nqb, nkb), torch.int32)
@@ -228,14 +241,19 @@ def sa_sparse_attn_fwd(q, k, v, bq, bk, kv_idx=None, kv_cnt=None, ext_mask=None,
     if out is not None:
         _expect("out", out, q.shape, torch.bfloat16)
     dev = q.device
-    _on_device(dev, q=q, k=k, v=v, kv_idx=kv_idx, kv_cnt=kv_cnt, ext_mask=ext_mask, out=out)
+    _on_device(dev, q=q, k=k, v=v, kv_idx=kv_idx, kv_cnt=kv_cnt, ext_mask=ext_mask, out=out,
+               o_l=o_l, alpha=alpha)
     o = out if out is not None else torch.empty_like(q)
     lse = torch.empty(B, H, N, dtype=torch.float32, device=dev) if want_lse else None
     need = load().sa_sparse_attn_workspace_size(B, H, N, d, bq, bk, int(ext_mask is not None))
     ws = _workspace(need, dev, workspace) if need else None
-    _call("sa_sparse_attn_fwd", _ptr(q), _ptr(k), _ptr(v), B, H, N, d, bq, bk, _ptr(kv_idx),
-          _ptr(kv_cnt), _ptr(ext_mask), float(scale), _ptr(o), _ptr(lse), _ptr(ws),
-          0 if ws is None else ws.numel(), _stream(dev))
+    common = (_ptr(q), _ptr(k), _ptr(v), B, H, N, d, bq, bk, _ptr(kv_idx), _ptr(kv_cnt),
+              _ptr(ext_mask), float(scale))
+    tail = (_ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev))
+    if o_l is None:
+        _call("sa_sparse_attn_fwd", *common, _ptr(o), *tail)
+    else:
+        _call("sa_sparse_attn_blend_fwd", *common, _ptr(o_l), _ptr(alpha), _ptr(o), *tail)
     return (o, lse) if want_lse else o
 
 
@@ -251,7 +269,7 @@ def sa_dense_attn_fwd(q, k, v, bq=128, scale=0.0, want_lse=False, out=None):
     return (o, lse) if want_lse else o
 
 
-def sa_linear_branch(q, k, v, want_ol=False, workspace=None):
+def sa_linear_branch(q, k, v, want_ol=False, workspace=None, out_ol=None):
     if want_ol:
         B, H, N, d = _qkv(q, k, v)
     else:
@@ -261,7 +279,10 @@ def sa_linear_branch(q, k, v, want_ol=False, workspace=None):
     _on_device(dev, q=q, k=k, v=v)
     S = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
     z = torch.empty(B, H, d, dtype=torch.float32, device=dev)
-    o_l = torch.empty_like(k) if want_ol else None
+    if out_ol is not None:
+        _expect("out_ol", out_ol, k.shape, torch.bfloat16)
+        _on_device(dev, out_ol=out_ol)
+    o_l = (out_ol if out_ol is not None else torch.empty_like(k)) if want_ol else None
     ws = _workspace(load().sa_linear_workspace_size(B, H, N, d), dev, workspace)
     _call("sa_linear_branch", _ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(S), _ptr(z), _ptr(o_l),
           _ptr(ws), ws.numel(), _stream(dev))
@@ -287,11 +308,12 @@ def sa_blend(o_s, q, kv_state, ksum, alpha, out=None, workspace=None):
 
 def _path_on_device(q, k, v, bq, bk, topk, topp, alpha, scale, out=None):
     m = sa_build_mask(q, k, bq, bk, topk, topp, scale)
-    o = sa_sparse_attn_fwd(q, k, v, bq, bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], scale=scale, out=out)
-    if alpha is not None:
-        S, z = sa_linear_branch(q, k, v)
-        o = sa_blend(o, q, S, z, alpha, out=o)
-    return o
+    if alpha is None:
+        return sa_sparse_attn_fwd(q, k, v, bq, bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], scale=scale, out=out)
+    # linear branch first, then the sparse attention blends it in its epilogue
+    _, _, o_l = sa_linear_branch(q, k, v, want_ol=True)
+    return sa_sparse_attn_fwd(q, k, v, bq, bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], scale=scale,
+                              out=out, o_l=o_l, alpha=alpha)
 
 
 def block_sparse_attention(q, k, v, bq=128, bk=64, topk=0.05, topp=0.9, alpha=None, scale=0.0,

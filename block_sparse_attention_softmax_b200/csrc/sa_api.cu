@@ -278,20 +278,26 @@ size_t sa_sparse_attn_workspace_size(int B, int H, int N, int d, int bq, int bk,
   return round_up(static_cast<size_t>(BH * nqb * nkb) * 4, 256) + round_up(static_cast<size_t>(BH * nqb) * 4, 256);
 }
 
-int sa_sparse_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H,
-                       int N, int d, int bq, int bk, const int32_t* kv_idx,
-                       const int32_t* kv_cnt, const uint8_t* ext_mask, double scale, uint16_t* o,
-                       float* lse_opt, void* workspace, size_t ws_bytes, void* stream) {
+namespace {
+
+// Shared body of sa_sparse_attn_fwd and sa_sparse_attn_blend_fwd (o_l and
+// alpha both null, or both given).
+int sparse_attn(const char* fn, const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H,
+                int N, int d, int bq, int bk, const int32_t* kv_idx, const int32_t* kv_cnt,
+                const uint8_t* ext_mask, double scale, const uint16_t* o_l, const float* alpha,
+                uint16_t* o, float* lse_opt, void* workspace, size_t ws_bytes, void* stream) {
   int rc = check_shape(B, H, N, d, bq, bk);
   if (rc) return rc;
-  if (!q || !k || !v || !o) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: null tensor pointer");
+  if (!q || !k || !v || !o) return fail(SA_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
   const bool lists = kv_idx && kv_cnt;
   if (lists == (ext_mask != nullptr) || (!lists && (kv_idx || kv_cnt)))
-    return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: give exactly one of (kv_idx, kv_cnt) or ext_mask");
+    return fail(SA_ERR_INVALID_ARG, "%s: give exactly one of (kv_idx, kv_cnt) or ext_mask", fn);
+  if ((o_l == nullptr) != (alpha == nullptr)) return fail(SA_ERR_INVALID_ARG, "%s: o_l and alpha go together", fn);
+  if (o_l && o_l == o) return fail(SA_ERR_INVALID_ARG, "%s: o must not alias o_l", fn);
   if (!isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "scale must be finite");
-  const void* ptrs[] = {q, k, v, o, kv_idx, kv_cnt, lse_opt, workspace};
+  const void* ptrs[] = {q, k, v, o, kv_idx, kv_cnt, lse_opt, workspace, o_l, alpha};
   for (const void* p : ptrs)
-    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "sa_sparse_attn_fwd: pointers must be 16-byte aligned");
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "%s: pointers must be 16-byte aligned", fn);
   if (scale <= 0.0) scale = 1.0 / sqrt(static_cast<double>(d));
   const int BH = B * H;
   const int nqb = (N + bq - 1) / bq, nkb = (N + bk - 1) / bk;
@@ -301,18 +307,38 @@ int sa_sparse_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
   if (!lists) {
     const size_t need = sa_sparse_attn_workspace_size(B, H, N, d, bq, bk, 1);
     if (!workspace || ws_bytes < need)
-      return fail(SA_ERR_WORKSPACE, "sa_sparse_attn_fwd: workspace of %zu bytes needed for ext_mask", need);
+      return fail(SA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed for ext_mask", fn, need);
     int* widx = static_cast<int*>(workspace);
     int* wcnt = reinterpret_cast<int*>(static_cast<char*>(workspace) + round_up(static_cast<size_t>(BH) * nqb * nkb * 4, 256));
     cudaError_t e = launch_compact_mask(ext_mask, BH * nqb, nkb, widx, wcnt, st);
-    if (e != cudaSuccess) return cuda_fail(e, "sa_sparse_attn_fwd (mask compaction)");
+    if (e != cudaSuccess) return cuda_fail(e, "mask compaction");
     idx = widx;
     cnt = wcnt;
   }
   AttnArgs a{q, k, v, o, lse_opt, idx, cnt, BH, N, d, bq, bk, nqb, nkb,
-             static_cast<float>(scale * 1.4426950408889634), 0};
+             static_cast<float>(scale * 1.4426950408889634), 0, o_l, alpha, H};
   cudaError_t e = launch_sparse_attn(a, st);
-  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_sparse_attn_fwd");
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, fn);
+}
+
+}  // namespace
+
+int sa_sparse_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H,
+                       int N, int d, int bq, int bk, const int32_t* kv_idx,
+                       const int32_t* kv_cnt, const uint8_t* ext_mask, double scale, uint16_t* o,
+                       float* lse_opt, void* workspace, size_t ws_bytes, void* stream) {
+  return sparse_attn("sa_sparse_attn_fwd", q, k, v, B, H, N, d, bq, bk, kv_idx, kv_cnt, ext_mask, scale,
+                     nullptr, nullptr, o, lse_opt, workspace, ws_bytes, stream);
+}
+
+int sa_sparse_attn_blend_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H,
+                             int N, int d, int bq, int bk, const int32_t* kv_idx,
+                             const int32_t* kv_cnt, const uint8_t* ext_mask, double scale,
+                             const uint16_t* o_l, const float* alpha, uint16_t* o, float* lse_opt,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  if (!o_l || !alpha) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_blend_fwd: o_l and alpha are required");
+  return sparse_attn("sa_sparse_attn_blend_fwd", q, k, v, B, H, N, d, bq, bk, kv_idx, kv_cnt, ext_mask,
+                     scale, o_l, alpha, o, lse_opt, workspace, ws_bytes, stream);
 }
 
 int sa_dense_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H, int N,

@@ -78,6 +78,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Wait, bounded by the default limit and whatever the abort flag says, for a
+// phase that work already issued will complete on its own (a TMA load in
+// flight, a tcgen05.commit after issued MMAs). Used on the way out of a kernel
+// that stopped early, so that no asynchronous write lands in shared or tensor
+// memory after the CTA has given it up.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicExch(&g_device_status, kStatusTimeout);
+      return;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -75,6 +75,11 @@ struct AttnArgs {
   int BH, N, d, bq, bk, nqb, nkb;
   float scale_log2;
   int dense;
+  // optional blend in the epilogue: O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l with
+  // O_s still in fp32; alpha [H, d] fp32, o_l [BH, N, d] bf16
+  const void* o_l = nullptr;
+  const float* alpha = nullptr;
+  int H = 1;
 };
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t st);
 

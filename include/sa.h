@@ -127,6 +127,21 @@ int sa_sparse_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                        double scale, uint16_t* o, float* lse_opt,
                        void* workspace, size_t ws_bytes, void* stream);
 
+/* Steps 4 and 5b in one kernel (SpargeAttention2 §2(3); SLA2 提案手法 ②):
+ * the sparse attention above, with its epilogue blending
+ *   O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l
+ * while O_s is still fp32, so O is rounded to bf16 once. o_l [B, H, N, d]
+ * bf16 is the linear branch's output (sa_linear_branch with o_l_opt), alpha
+ * [H, d] fp32. Both are required; o must not alias o_l. lse_opt is the log-sum-exp
+ * of the sparse attention alone. Arguments, workspace and errors otherwise as
+ * sa_sparse_attn_fwd. */
+int sa_sparse_attn_blend_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             int B, int H, int N, int d, int bq, int bk,
+                             const int32_t* kv_idx, const int32_t* kv_cnt, const uint8_t* ext_mask,
+                             double scale, const uint16_t* o_l, const float* alpha,
+                             uint16_t* o, float* lse_opt,
+                             void* workspace, size_t ws_bytes, void* stream);
+
 /* Dense attention through the same kernel, every tile kept (the comparison
  * point for the sparse speed-up). */
 int sa_dense_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,

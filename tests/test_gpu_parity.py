@@ -286,9 +286,11 @@ def test_full_size_workload(cuda_lib, name):
             eq = torch.from_numpy(eq).to(DEV)
             assert torch.equal(o_list[b, h][eq], o[b, h][eq])
     if wl.linear:
+        # the linear branch, then the sparse attention on the oracle's mask with
+        # the blend in its epilogue (one rounding of O)
         alpha = x["alpha"]
-        S, z = sa.sa_linear_branch(q, k, v)
-        ob = sa.sa_blend(o, q, S, z, alpha)
+        S, z, o_l = sa.sa_linear_branch(q, k, v, want_ol=True)
+        ob = sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, ext_mask=ext.to(DEV), o_l=o_l, alpha=alpha)
         torch.cuda.synchronize()
         for (b, h), (mask, _) in ora.items():
             kS, kz = oracle.linear_state(_f64(kc[b, h]), _f64(vc[b, h]))
@@ -349,20 +351,31 @@ def test_many_items_per_cta_all_rows(cuda_lib, ragged):
 
 
 def test_linear_branch_small(cuda_lib):
+    """O_l, the standalone blend (sa_blend, on a given bf16 O_s) and the blend
+    in the sparse attention's epilogue (on the oracle's mask), with batch 2 so
+    that alpha's row is the head's, not the flattened (batch, head)'s."""
     sa = cuda_lib
-    for (N, d) in [(1000, 128), (257, 64)]:
-        q, k, v = random_qkv(1, 2, N, d, seed=N, device=DEV)
+    for (N, d, B) in [(1000, 128, 2), (257, 64, 1)]:
+        H = 2
+        q, k, v = random_qkv(B, H, N, d, seed=N, device=DEV)
         S, z, ol = sa.sa_linear_branch(q, k, v, want_ol=True)
-        alpha = torch.rand(2, d, device=DEV)
+        alpha = torch.rand(H, d, device=DEV)
         os_ = torch.randn_like(q.float()).to(torch.bfloat16)
         ob = sa.sa_blend(os_, q, S, z, alpha)
+        m = sa.sa_build_mask(q, k, 128, 64, 0.2, 0.8, want_mask=True)
+        of = sa.sa_sparse_attn_fwd(q, k, v, 128, 64, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], o_l=ol, alpha=alpha)
         torch.cuda.synchronize()
-        for h in range(2):
-            kS, kz = oracle.linear_state(_f64(k[0, h]), _f64(v[0, h]))
-            ref_l = oracle.linear_out(_f64(q[0, h]), kS, kz)
-            assert_close(ol[0, h].float().cpu().numpy(), ref_l, f"O_l N={N}")
-            ref_b = oracle.blend(_f64(os_[0, h]), ref_l, alpha[h].double().cpu().numpy())
-            assert_close(ob[0, h].float().cpu().numpy(), ref_b, f"blend N={N}")
+        for b in range(B):
+            for h in range(H):
+                kS, kz = oracle.linear_state(_f64(k[b, h]), _f64(v[b, h]))
+                ref_l = oracle.linear_out(_f64(q[b, h]), kS, kz)
+                assert_close(ol[b, h].float().cpu().numpy(), ref_l, f"O_l N={N}")
+                al = alpha[h].double().cpu().numpy()
+                ref_b = oracle.blend(_f64(os_[b, h]), ref_l, al)
+                assert_close(ob[b, h].float().cpu().numpy(), ref_b, f"blend N={N}")
+                mk = m["mask"][b, h].cpu().numpy().astype(bool)
+                ro, _ = oracle.masked_attention(_f64(q[b, h]), _f64(k[b, h]), _f64(v[b, h]), mk, 128, 64)
+                assert_close(of[b, h].float().cpu().numpy(), oracle.blend(ro, ref_l, al), f"fused blend N={N}")
     sa.sa_device_status()
 
 
