@@ -45,6 +45,12 @@ _SIGNATURES = {
     "sa_blend_workspace_size": (c_size_t, [c_int] * 4),
     "sa_blend": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                          c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "sa_trip_pool": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
+                             c_void_p, c_void_p, c_void_p]),
+    "sa_tile_heatmap": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                c_double, c_void_p, c_int, c_void_p, c_void_p, c_void_p]),
+    "sa_select_mask": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_double, c_double,
+                               c_void_p, c_void_p, c_void_p, c_void_p]),
     "sa_diag_set_device_status": (c_int, [c_int]),
     "sa_diag_set_wait_limit": (c_int, [ctypes.c_longlong]),
     "sa_diag_wait_timeout": (c_int, [c_void_p, c_void_p]),
@@ -304,6 +310,55 @@ def sa_blend(o_s, q, kv_state, ksum, alpha, out=None, workspace=None):
     _call("sa_blend", _ptr(o_s), _ptr(q), _ptr(kv_state), _ptr(ksum), _ptr(alpha), B, H, N, d,
           _ptr(o), _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev))
     return o
+
+
+def sa_trip_pool(q, k, bq, bk):
+    """TripPool descriptors [mean | max | min] of the query and key blocks."""
+    B, H, N, d = _qkv(q, k, names=("q", "k"))
+    _on_device(q.device, q=q, k=k)
+    qd = torch.empty(B, H, -(-N // bq), 3 * d, dtype=torch.float32, device=q.device)
+    kd = torch.empty(B, H, -(-N // bk), 3 * d, dtype=torch.float32, device=q.device)
+    _call("sa_trip_pool", _ptr(q), _ptr(k), B, H, N, d, bq, bk, _ptr(qd), _ptr(kd), _stream(q.device))
+    return qd, kd
+
+
+def sa_tile_heatmap(q, k, bq, bk=64, scale=0.0, rows=None, want_lse=False, out=None):
+    """Max-pooled full-attention heatmap (natural log) of every (query block,
+    key block) tile; with `rows` (int32 query-block rows) only those rows are
+    evaluated and the others of `out` are left as they were."""
+    B, H, N, d = _qkv(q, k, names=("q", "k"))
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    if rows is not None:
+        if rows.dtype != torch.int32 or rows.dim() != 1 or not rows.is_contiguous():
+            raise ValueError("rows: contiguous 1-D int32 tensor of query-block rows")
+    if out is not None:
+        _expect("out", out, (B, H, nqb, nkb), torch.float32)
+    dev = q.device
+    _on_device(dev, q=q, k=k, rows=rows, out=out)
+    heat = out if out is not None else torch.full((B, H, nqb, nkb), float("nan"), dtype=torch.float32, device=dev)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=dev) if want_lse else None
+    _call("sa_tile_heatmap", _ptr(q), _ptr(k), B, H, N, d, bq, bk, float(scale), _ptr(rows),
+          0 if rows is None else rows.numel(), _ptr(heat), _ptr(lse), _stream(dev))
+    return (heat, lse) if want_lse else heat
+
+
+def sa_select_mask(scores, topk, topp, want_mask=False):
+    """Hybrid Top-k ∪ Top-p selection from given block scores [B, H, n_qb, n_kb]."""
+    if scores.dim() != 4:
+        raise ValueError("scores must be [B, H, n_qb, n_kb]")
+    B, H, nqb, nkb = scores.shape
+    _expect("scores", scores, scores.shape, torch.float32)
+    dev = scores.device
+    _on_device(dev, scores=scores)
+    kv_idx = torch.empty(B, H, nqb, nkb, dtype=torch.int32, device=dev)
+    kv_cnt = torch.empty(B, H, nqb, dtype=torch.int32, device=dev)
+    mask = torch.empty(B, H, nqb, nkb, dtype=torch.uint8, device=dev) if want_mask else None
+    _call("sa_select_mask", _ptr(scores), B, H, nqb, nkb, float(topk), float(topp), _ptr(kv_idx),
+          _ptr(kv_cnt), _ptr(mask), _stream(dev))
+    out = {"kv_idx": kv_idx, "kv_cnt": kv_cnt}
+    if want_mask:
+        out["mask"] = mask
+    return out
 
 
 def _path_on_device(q, k, v, bq, bk, topk, topp, alpha, scale, out=None):

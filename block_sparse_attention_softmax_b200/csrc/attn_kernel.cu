@@ -8,52 +8,59 @@
 // the K/V blocks of one head in L2. Inside an item, two 64-key blocks from the
 // item's kept list form one 128-key tile.
 //
-// Each CTA keeps two items in flight, in two "lanes". A lane has its own S and
-// O accumulators in tensor memory and its own softmax warpgroup, one thread
-// per query row over all 128 columns of a tile (no exchange of row maxima
-// between warps). One thread issues the MMAs of both lanes in the order
-//     ... PV_0(j-1), QK_0(j), PV_1(j-1), QK_1(j), PV_0(j), QK_0(j+1) ...
-// so that while one lane's softmax works on its S the tensor core runs the
-// other lane's P V and Q K^T: each softmax has about two MMA groups of time.
-// P is written as bf16 over the first 64 columns of its lane's S buffer and
-// read from there by the P V; the Q K^T that next overwrites that buffer is
-// issued by the same thread after that P V, and the tcgen05.mma operations of
-// one thread execute in the order issued. A commit after a lane's Q K^T also
-// covers the P V issued before it, so when the softmax sees S(j) the lane's O
-// already holds tile j-1: the lazy rescale of O needs no extra wait.
+// The per-tile chain QK(g) -> softmax(g) -> PV(g) is what limits this kernel,
+// so the tensor core is kept fed from three S buffers (QK can run up to three
+// tiles ahead of PV) and by two MMA-issuing threads: a thread that issues
+// tcgen05.mma stalls while the tensor pipe's short queue is full, and its
+// mbarrier waits and commits queue behind its own MMAs, so with one thread
+// the pipe idles between MMA groups. With one thread for QK and one for PV the
+// waits of one overlap the MMAs of the other (measured on B200: dense 1.3B-480p
+// attention 1022 -> 1188 TFLOP/s). The QK that overwrites an S buffer waits for
+// the P V that read P from it.
 //
-//   warp 0       scheduler and K producer: hands the CTA's items, in order, to
-//                whichever lane finished its previous item (lanes alternate
-//                tile by tile), posts each item's facts to that lane's ring,
-//                and loads K tiles (one TMA box per 64-key block, so the two
-//                blocks of a tile need not be adjacent) into a 2-slot ring in
-//                the same alternating order. It also owns the three Q slots:
-//                each lane holds the slot of its current item, and the third
-//                receives the next non-empty item; when a lane takes that
-//                item, the slot of the item it finished is requested for the
-//                one after (a slot tied to an item's position in the list
-//                could be the slot the other lane still holds).
-//   warp 1       TMEM allocation and the MMA-issuing thread
-//   warp 2       V producer (2-slot ring, same order as K)
-//   warp 3       Q producer: loads each requested Q tile into its slot once
-//                the last Q K^T of the slot's previous item has completed, so
-//                the next item's Q is resident before a lane takes it
-//   warps 4..7   softmax of lane 0, warps 8..11 softmax of lane 1: warp w
-//                reads TMEM lane quadrant w % 4 (query rows 32 (w % 4) .. +31
-//                of its tile). The running max m is kept in the log2 domain
-//                and raised only when a tile's max exceeds it by more than 8
-//                (P <= 256 otherwise); then O is rescaled in TMEM. P =
-//                exp2(S*scale*log2e - m). At the end of an item the warps copy
-//                O to registers, release it, and write O / l as bf16 and the
-//                row log-sum-exp; an item with no kept block gets zeros and
-//                -inf. With the linear branch, the epilogue blends while O_s
-//                is still fp32: O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l (SLA2
-//                提案手法 ②), one bf16 rounding of O in all.
+//   warp 0       TMA producer of Q (two slots, so the next item's Q loads
+//                while the current item runs) and K (2-stage ring; a slot is
+//                free once the QK that read it has completed, the event that
+//                also fills that tile's S buffer)
+//   warp 10      TMA producer of V (2-stage ring; a slot is free once the P V
+//                that read it has completed); one TMA box per 64-key block,
+//                so the two blocks of a tile need not be adjacent
+//   warp 1       TMEM allocation and the thread issuing
+//                  S_g = Q K_g^T  (A = Q, B = K, both from shared memory)
+//   warp 11      the thread issuing
+//                  O  += P_g V_g  (A = P_g from TMEM, B = V from shared memory)
+//   warps 2..9   softmax: TMEM lane quadrant q = warp % 4 holds query rows
+//                32q..32q+31; warp w and w+4 split the 128 columns of those
+//                rows (64 each) and exchange the row max (and, at the end of
+//                an item, the row sum) through shared memory at a named
+//                barrier of the pair. Every bounded wait of these warps is
+//                followed by such a barrier at which each warp also posts
+//                whether its wait succeeded: in place of the row max or row
+//                sum it posts a NaN with a payload of its own (kStopBits;
+//                arithmetic yields the canonical NaN, never this one), or a
+//                flag word in the rare rescale path. Each warp stops if either
+//                post says so, the same decision in both, so the two warps of
+//                a pair stop together. A warp whose wait for the next item
+//                fails (no barrier follows that wait) posts the stop word in
+//                both places its partner reads next and arrives once at the
+//                pair barrier before it leaves, so the partner completes its
+//                next exchange, reads the stop word and stops too: neither
+//                waits at a barrier the other has left.
+//                (All lanes of a warp take the same decision in a wait: they
+//                read the same barrier state, clock and abort flag.)
+//                The running max m is kept in the log2 domain and only
+//                raised when a tile's max exceeds it by more than 8 (P <= 256
+//                otherwise); then O is rescaled in TMEM. P = exp2(S*scale*log2e
+//                - m) is written back over S as packed bf16. At the end of an
+//                item the warps copy O to registers, release it, and write
+//                O / l as bf16 and the row log-sum-exp. With the linear branch
+//                the epilogue blends while O_s is still fp32, O = alpha ⊙ O_s
+//                + (1 - alpha) ⊙ O_l (SLA2 提案手法 ②): one bf16 rounding of O.
 //
-// TMEM columns: S_0 [0,128), S_1 [128,256) (fp32, 128 wide; P aliases the
-// first 64 columns), O_0 at 256, O_1 at 384 (D wide). Every mbarrier wait is
-// bounded (sa_device.cuh). A CTA that stops early waits (bounded) for its
-// TMA loads and MMAs in flight before it releases shared and tensor memory.
+// TMEM columns: S buffers at 0, 128 and 256 (fp32, 128 wide; P aliases their
+// first 64 columns), O at 384 (d wide). Every mbarrier wait is bounded (see
+// sa_device.cuh), and a CTA that stops early waits (bounded) for the TMA loads
+// and MMAs it has issued before it gives up shared and tensor memory.
 #include "sa_internal.h"
 
 namespace sa {
@@ -62,21 +69,21 @@ namespace attn {
 
 constexpr int kBM = 128;        // query rows per tile
 constexpr int kBN = 128;        // keys per tile (two 64-key blocks)
-constexpr int kLanes = 2;       // items in flight per CTA
-constexpr int kQSlots = 3;      // Q slots: both lanes' items plus the next one
-constexpr int kQReqRing = 4;    // Q load requests posted ahead of the Q producer
+constexpr int kSoftWarps = 8;
+constexpr int kQSlots = 2;      // Q of the next item loads while the current one runs
+constexpr int kItemRing = 4;    // item facts the K producer posts ahead of the softmax warps
 constexpr int kKStages = 2;
 constexpr int kVStages = 2;
-constexpr int kItemRing = 4;    // item facts per lane posted ahead of its consumers
-// Column pairs c (of 64 per thread and tile) with bit (c % 8) set take the
-// FMA-pipe exponential instead of MUFU ex2: one pair in four.
+constexpr int kSBufs = 3;
+// Column pairs c (of 32 per thread and tile) with bit (c % 8) set take the
+// FMA-pipe exponential instead of MUFU ex2: one pair in four. Measured on B200
+// with two MMA issuers, where the softmax sets the pace: fastest of 0, 1, 2, 3
+// and 4 pairs in 8 (the polynomial costs 10 issue slots per pair, MUFU costs
+// pipe time), both in short runs and under the power cap.
 constexpr uint32_t kPolyPairs = 0x88u;
-constexpr float kRescaleLog2 = 8.f;
-constexpr int kKWarp = 0, kMmaWarp = 1, kVWarp = 2, kQWarp = 3, kSoftWarp0 = 4;
-constexpr int kLaneWarps = 4;
-constexpr int kThreads = 32 * (kSoftWarp0 + kLanes * kLaneWarps);
-// consumers of a lane's item ring: V producer, MMA issuer, the lane's softmax warps
-constexpr int kRingConsumers = 2 + kLaneWarps;
+constexpr int kVWarp = 2 + kSoftWarps;               // warp index of the V producer
+constexpr int kPVWarp = kVWarp + 1;                  // warp index of the P V issuer
+constexpr int kThreads = 32 * (kPVWarp + 1);
 
 template <int D>
 struct Layout {
@@ -89,37 +96,55 @@ struct Layout {
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + kQSlots * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + kKStages * TILE_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_V + kVStages * TILE_BYTES;
-  static constexpr uint32_t OFF_RING = OFF_BAR + 512;      // [kLanes][kItemRing] int4
-  static constexpr uint32_t OFF_QREQ = OFF_RING + kLanes * kItemRing * 16;   // [kQReqRing] int2
-  static constexpr uint32_t USED = OFF_QREQ + kQReqRing * 8;
+  static constexpr uint32_t OFF_RED = OFF_V + kVStages * TILE_BYTES;
+  static constexpr uint32_t RED_BYTES = (2 * 2 + 2) * kBM * 4 + 4 * 16 * 4;   // row max [2][2][128], row sum [2][128], pair flags [4][16]
+  static constexpr uint32_t OFF_BAR = OFF_RED + RED_BYTES;
+  static constexpr uint32_t OFF_RING = OFF_BAR + 512;    // item ring [kItemRing][4] int
+  static constexpr uint32_t USED = OFF_RING + 256;
   // at least 120 KB so that a second CTA never shares the SM (all 512 TMEM columns are held)
   static constexpr uint32_t SMEM = (USED + 1024 > 120 * 1024) ? USED + 1024 : 120 * 1024;
 };
-static_assert(Layout<128>::SMEM <= 232448, "shared memory of the d = 128 kernel");
 
-__host__ __device__ constexpr uint32_t tm_s(int l) { return static_cast<uint32_t>(l) * 128u; }
-__host__ __device__ constexpr uint32_t tm_o(int l) { return 256u + static_cast<uint32_t>(l) * 128u; }
+__host__ __device__ constexpr uint32_t tm_s(int b) { return static_cast<uint32_t>(b) * 128u; }
+constexpr uint32_t TM_O = 384;
 constexpr uint32_t TM_COLS = 512;
 
+static_assert(kKStages <= kSBufs, "a K slot is freed by the S_FULL commit of the tile kKStages back");
+
 enum {
-  B_QFULL = 0,                          // [kQSlots] Q tile landed
-  B_QEMPTY = B_QFULL + kQSlots,         // [kQSlots] last Q K^T of the item completed
-  B_KFULL = B_QEMPTY + kQSlots,         // [kKStages]
-  B_KEMPTY = B_KFULL + kKStages,        // [kKStages] the Q K^T that read the slot completed
-  B_VFULL = B_KEMPTY + kKStages,        // [kVStages]
-  B_VEMPTY = B_VFULL + kVStages,        // [kVStages] the P V that read the slot completed
-  B_SFULL = B_VEMPTY + kVStages,        // [kLanes] S of the lane's tile ready (and O through the tile before)
-  B_PFULL = B_SFULL + kLanes,           // [kLanes] P written by the lane's softmax warps
-  B_OFULL = B_PFULL + kLanes,           // [kLanes] last P V of the lane's item completed
-  B_OEMPTY = B_OFULL + kLanes,          // [kLanes] the lane's epilogue copied O out of TMEM
-  B_IFULL = B_OEMPTY + kLanes,          // [kLanes][kItemRing] item facts posted
-  B_IEMPTY = B_IFULL + kLanes * kItemRing,  // [kLanes][kItemRing] item facts read by every consumer
-  B_RFULL = B_IEMPTY + kLanes * kItemRing,  // [kQReqRing] Q load request posted
-  B_REMPTY = B_RFULL + kQReqRing,           // [kQReqRing] Q load request read
-  B_DRAIN = B_REMPTY + kQReqRing,           // the MMA thread's last commit (early exit)
-  B_COUNT = B_DRAIN + 1
+  B_QFULL = 0,                       // [kQSlots] Q tile landed in shared memory
+  B_QEMPTY = B_QFULL + kQSlots,      // [kQSlots] last QK of the item completed
+  B_KFULL = B_QEMPTY + kQSlots,      // [kKStages]
+  B_VFULL = B_KFULL + kKStages,      // [kVStages]
+  B_SFULL = B_VFULL + kVStages,      // [kSBufs]
+  B_PFULL = B_SFULL + kSBufs,        // [kSBufs]
+  B_PVDONE = B_PFULL + kSBufs,       // [kSBufs] P V of the tile held in that S buffer completed:
+                                     // the S buffer and the tile's V slot are free again
+  B_OFULL = B_PVDONE + kSBufs,       // last P V of the item completed
+  B_OEMPTY = B_OFULL + 1,            // epilogue has copied O out of TMEM
+  B_IFULL = B_OEMPTY + 1,            // [kItemRing] item facts posted by the K producer
+  B_IEMPTY = B_IFULL + kItemRing,    // [kItemRing] item facts read by the softmax warps
+  B_DRAIN = B_IEMPTY + kItemRing,    // [2] each MMA thread's last commit (early exit)
+  B_COUNT = B_DRAIN + 2
 };
+
+// Word a softmax warp posts in place of its row max or row sum when its wait
+// failed: a NaN whose payload no arithmetic produces.
+constexpr uint32_t kStopBits = 0x7FC0DEADu;
+
+// Named barrier of the two softmax warps of one TMEM lane quadrant; shared
+// memory written before it by either warp is visible to both after it.
+__device__ __forceinline__ void pair_sync(int bar_id) {
+  asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+}
+
+// Both warps of a pair post whether their wait succeeded and meet; true only
+// if both did. slot[half] is this warp's word, slot[half ^ 1] the partner's.
+__device__ __forceinline__ bool pair_agree(int bar_id, volatile int* slot, int half, bool ok) {
+  slot[half] = ok ? 1 : 0;
+  pair_sync(bar_id);
+  return ok && slot[half ^ 1] != 0;
+}
 
 // Per-item facts every role derives the same way.
 struct Item {
@@ -151,63 +176,11 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int item) {
   return it;
 }
 
-// Where one lane stands in the schedule. The scheduler and every role that
-// follows the alternating tile order keep one per lane and update it the same
-// way: a lane that has issued its item's last tile takes a new item at its
-// next turn; a lane that met the end marker is out, and the other lane then
-// takes every turn.
-struct LaneState {
-  int item, cnt, T, t, qslot;   // current item, kept blocks, tiles, next tile, Q slot
-  int n;                         // ring entries posted (scheduler) or read (consumer)
-  bool tail, need, active;
-};
-
-__device__ __forceinline__ void lane_init(LaneState& s) {
-  s.item = s.cnt = s.T = s.t = s.n = 0;
-  s.qslot = -1;
-  s.tail = false;
-  s.need = s.active = true;
-}
-
-// Reads lane l's ring until a non-empty item or the end marker (single-thread
-// consumer). Returns false if a wait ran out or another role aborted.
-__device__ __forceinline__ bool take_item(uint64_t* bars, const volatile int* ring, int l, LaneState& s,
-                                          int n_items, volatile int* abort) {
-  while (true) {
-    const int slot = s.n % kItemRing;
-    if (!mbar_wait(&bars[B_IFULL + l * kItemRing + slot], (s.n / kItemRing) & 1, abort)) return false;
-    const volatile int* e = ring + (l * kItemRing + slot) * 4;
-    const int item = e[0], cnt = e[1], tail = e[2], qslot = e[3];
-    mbar_arrive(&bars[B_IEMPTY + l * kItemRing + slot]);
-    ++s.n;
-    if (item >= n_items) {
-      s.active = false;
-      return true;
-    }
-    if (cnt == 0) continue;     // nothing to load or compute; the lane's softmax writes its zeros
-    s.item = item;
-    s.cnt = cnt;
-    s.T = (cnt + 1) >> 1;
-    s.t = 0;
-    s.tail = tail != 0;
-    s.qslot = qslot;
-    s.need = false;
-    return true;
-  }
-}
-
-// Key blocks of tile t of an item: the first, the second (if any) and their count.
-__device__ __forceinline__ int tile_blocks(const AttnArgs& a, int item, int cnt, int t, int& kb0, int& kb1) {
-  const int nblk = min(2, cnt - 2 * t);
-  if (a.dense) {
-    kb0 = 2 * t;
-    kb1 = 2 * t + 1;
-  } else {
-    const int* row = a.kv_idx + static_cast<long long>(item) * a.nkb;   // item = bh * nqb + qb
-    kb0 = __ldg(row + 2 * t);
-    kb1 = nblk > 1 ? __ldg(row + 2 * t + 1) : 0;
-  }
-  return nblk;
+// First item at or after `item` (stepping by `stride`) with at least one tile.
+__device__ __forceinline__ int next_nonempty(const AttnArgs& a, int item, int stride, int n_items) {
+  for (; item < n_items; item += stride)
+    if (load_item(a, item).T > 0) break;
+  return item;
 }
 
 }  // namespace attn
@@ -224,12 +197,15 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   uint8_t* sQ = smem + L::OFF_Q;
   uint8_t* sK = smem + L::OFF_K;
   uint8_t* sV = smem + L::OFF_V;
+  float* red_max = reinterpret_cast<float*>(smem + L::OFF_RED);   // [2 tile parity][2 halves][128 rows]
+  float* red_sum = red_max + 4 * kBM;                              // [2 halves][128 rows]
+  // per quadrant: [6,8) rescale (half 0, half 1)
+  volatile int* pair_flags = reinterpret_cast<volatile int*>(red_sum + 2 * kBM);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   static_assert(B_COUNT * 8 + 8 <= 512, "barrier region");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
+  volatile int* item_ring = reinterpret_cast<volatile int*>(smem + L::OFF_RING);   // [kItemRing][item, cnt, tail, -]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* ring = reinterpret_cast<volatile int*>(smem + L::OFF_RING);   // [lane][slot][item, cnt, tail, Q slot]
-  volatile int* qreq = reinterpret_cast<volatile int*>(smem + L::OFF_QREQ);   // [slot][item, Q slot]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -240,33 +216,25 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       mbar_init(&bars[B_QFULL + i], 1);
       mbar_init(&bars[B_QEMPTY + i], 1);
     }
-    for (int i = 0; i < kKStages; ++i) {
-      mbar_init(&bars[B_KFULL + i], 1);
-      mbar_init(&bars[B_KEMPTY + i], 1);
+    for (int i = 0; i < kItemRing; ++i) {
+      mbar_init(&bars[B_IFULL + i], 1);
+      mbar_init(&bars[B_IEMPTY + i], kSoftWarps);
     }
-    for (int i = 0; i < kVStages; ++i) {
-      mbar_init(&bars[B_VFULL + i], 1);
-      mbar_init(&bars[B_VEMPTY + i], 1);
+    mbar_init(&bars[B_OFULL], 1);
+    mbar_init(&bars[B_OEMPTY], kSoftWarps);
+    mbar_init(&bars[B_DRAIN + 0], 1);
+    mbar_init(&bars[B_DRAIN + 1], 1);
+    for (int i = 0; i < kKStages; ++i) mbar_init(&bars[B_KFULL + i], 1);
+    for (int i = 0; i < kVStages; ++i) mbar_init(&bars[B_VFULL + i], 1);
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(&bars[B_SFULL + i], 1);
+      mbar_init(&bars[B_PFULL + i], kSoftWarps);
+      mbar_init(&bars[B_PVDONE + i], 1);
     }
-    for (int l = 0; l < kLanes; ++l) {
-      mbar_init(&bars[B_SFULL + l], 1);
-      mbar_init(&bars[B_PFULL + l], kLaneWarps);
-      mbar_init(&bars[B_OFULL + l], 1);
-      mbar_init(&bars[B_OEMPTY + l], kLaneWarps);
-      for (int i = 0; i < kItemRing; ++i) {
-        mbar_init(&bars[B_IFULL + l * kItemRing + i], 1);
-        mbar_init(&bars[B_IEMPTY + l * kItemRing + i], kRingConsumers);
-      }
-    }
-    for (int i = 0; i < kQReqRing; ++i) {
-      mbar_init(&bars[B_RFULL + i], 1);
-      mbar_init(&bars[B_REMPTY + i], 1);
-    }
-    mbar_init(&bars[B_DRAIN], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, TM_COLS);
     tmem_relinquish();
   }
@@ -275,459 +243,411 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   tc_fence_after();
   const uint32_t tm = *tmem_slot;
 
-  if (warp == kKWarp) {
-    // ------------------------------------------------------------ scheduler + K producer
+  if (warp == 0 || warp == kVWarp) {
+    // ------------------------------------------------------------ producers
     if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      LaneState s0, s1;
-      lane_init(s0);
-      lane_init(s1);
-      int g = 0, nreq = 0;
-      uint32_t free_slots = (1u << kQSlots) - 1;
+      const bool is_k = warp == 0;
+      if (is_k) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+      } else {
+        tma_prefetch_desc(&tmV);
+      }
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      uint8_t* ring = is_k ? sK : sV;
+      const int stages = is_k ? kKStages : kVStages;
+      const int b_full = is_k ? B_KFULL : B_VFULL;
+      int g = 0, qi = 0, q_armed = 0;
       bool ok = true;
-      // first non-empty item at or after `from` in this CTA's list (n_items if none)
-      auto find_nonempty = [&](int from) {
-        for (int i = from; i < n_items; i += gridDim.x)
-          if (load_item(a, i).T > 0) return i;
-        return n_items;
-      };
-      // asks the Q producer to load item's Q into `slot`
-      auto request_q = [&](int item, int slot) -> bool {
-        const int r = nreq % kQReqRing;
-        if (!mbar_wait(&bars[B_REMPTY + r], ((nreq / kQReqRing) & 1) ^ 1, abort_flag)) return false;
-        qreq[r * 2 + 0] = item;
-        qreq[r * 2 + 1] = slot;
-        mbar_arrive(&bars[B_RFULL + r]);
-        ++nreq;
-        return true;
-      };
-      // posts one item's facts to lane l's ring
-      auto post = [&](int ln, LaneState& c, int item, int cnt, bool tail, int qslot) -> bool {
-        const int slot = c.n % kItemRing;
-        if (!mbar_wait(&bars[B_IEMPTY + ln * kItemRing + slot], ((c.n / kItemRing) & 1) ^ 1, abort_flag)) return false;
-        volatile int* e = ring + (ln * kItemRing + slot) * 4;
-        e[0] = item;
-        e[1] = cnt;
-        e[2] = tail ? 1 : 0;
-        e[3] = qslot;
-        mbar_arrive(&bars[B_IFULL + ln * kItemRing + slot]);
-        ++c.n;
-        return true;
-      };
-      int next = blockIdx.x;               // first item not yet handed to a lane
-      int pf = find_nonempty(next);        // the next non-empty item, its Q requested into pf_slot
-      int pf_slot = 0;
-      if (pf < n_items) free_slots &= ~1u;
-      ok = request_q(pf, pf_slot);         // item n_items: no more requests (the Q producer stops)
-      // one turn of lane l: a new item if it needs one, then its next K tile
-      auto turn = [&](LaneState& c, const int l) -> bool {
-        bool ok = true;
-        if (c.active && c.need) {
-          // the empty items before the next non-empty one go to this lane for their zeros
-          for (; ok && next < pf; next += gridDim.x) ok = post(l, c, next, 0, false, -1);
-          if (!ok) return false;
-          if (pf >= n_items) {
-            if (!post(l, c, n_items, 0, false, -1)) return false;
-            c.active = false;
-          } else {
-            const Item it = load_item(a, pf);
-            if (!post(l, c, pf, it.cnt, it.tail, pf_slot)) return false;
-            if (c.qslot >= 0) free_slots |= 1u << c.qslot;   // reloaded after its last Q K^T
-            c.item = pf;
-            c.cnt = it.cnt;
-            c.T = it.T;
-            c.t = 0;
-            c.qslot = pf_slot;
-            c.need = false;
-            next = pf + gridDim.x;
-            pf = find_nonempty(next);
-            if (pf < n_items) {
-              pf_slot = __ffs(free_slots) - 1;
-              free_slots &= ~(1u << pf_slot);
-            }
-            if (!(ok = request_q(pf, pf_slot))) return false;
-          }
-        }
-        if (c.active) {
-          const int ks = g % kKStages;
-          int kb0, kb1;
-          const int nblk = tile_blocks(a, c.item, c.cnt, c.t, kb0, kb1);
-          const int bh = c.item / a.nqb;
-          if (!mbar_wait(&bars[B_KEMPTY + ks], ((g / kKStages) & 1) ^ 1, abort_flag)) return false;
-          mbar_arrive_expect_tx(&bars[B_KFULL + ks], nblk * L::BLK_BYTES);
-          uint8_t* dst = sK + ks * L::TILE_BYTES;
+      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+        const Item it = load_item(a, item);
+        if (it.T == 0) continue;
+        const int* row = a.dense ? nullptr : a.kv_idx + (static_cast<long long>(it.bh) * a.nqb + it.qb) * a.nkb;
+        if (is_k) {
+          // item facts for the softmax warps (they would otherwise read them
+          // from global memory on their critical path)
+          const int rs = qi % kItemRing;
+          if (!(ok = mbar_wait(&bars[B_IEMPTY + rs], ((qi / kItemRing) & 1) ^ 1, abort_flag))) break;
+          item_ring[rs * 4 + 0] = item;
+          item_ring[rs * 4 + 1] = it.cnt;
+          item_ring[rs * 4 + 2] = it.tail ? 1 : 0;
+          mbar_arrive(&bars[B_IFULL + rs]);
+          const int qs = qi % kQSlots;
+          if (!(ok = mbar_wait(&bars[B_QEMPTY + qs], ((qi / kQSlots) & 1) ^ 1, abort_flag))) break;
+          mbar_arrive_expect_tx(&bars[B_QFULL + qs], L::Q_BYTES);
 #pragma unroll
-          for (int ch = 0; ch < L::NCH; ++ch) {
-            tma_load_3d(dst + ch * L::KV_CHUNK, &tmK, &bars[B_KFULL + ks], ch * 64, kb0 * 64, bh);
-            if (nblk > 1)
-              tma_load_3d(dst + ch * L::KV_CHUNK + 64 * 128, &tmK, &bars[B_KFULL + ks], ch * 64, kb1 * 64, bh);
-          }
-          ++g;
-          if (++c.t == c.T) c.need = true;
+          for (int c = 0; c < L::NCH; ++c)
+            tma_load_3d(sQ + qs * L::Q_BYTES + c * L::Q_CHUNK, &tmQ, &bars[B_QFULL + qs], c * 64, it.qb * a.bq, it.bh);
+          q_armed = qi + 1;
         }
-        return true;
-      };
-      while (ok && (s0.active || s1.active)) {
-        ok = turn(s0, 0);
-        if (ok) ok = turn(s1, 1);
+        for (int t = 0; t < it.T; ++t, ++g) {
+          const int s = g % stages;
+          const int nblk = min(2, it.cnt - 2 * t);
+          const int kb0 = a.dense ? 2 * t : __ldg(row + 2 * t);
+          const int kb1 = nblk > 1 ? (a.dense ? 2 * t + 1 : __ldg(row + 2 * t + 1)) : 0;
+          // slot reuse: a K slot is free once the QK that read it completed
+          // (S_FULL of the tile kKStages back), a V slot once the P V that read
+          // it completed (PV_DONE of the tile kVStages back); both barriers
+          // are indexed by S buffer
+          if (is_k) {
+            if (g >= kKStages) {
+              const int gp = g - kKStages;
+              if (!(ok = mbar_wait(&bars[B_SFULL + gp % kSBufs], (gp / kSBufs) & 1, abort_flag))) break;
+            }
+          } else if (g >= kVStages) {
+            const int gp = g - kVStages;
+            if (!(ok = mbar_wait(&bars[B_PVDONE + gp % kSBufs], (gp / kSBufs) & 1, abort_flag))) break;
+          }
+          mbar_arrive_expect_tx(&bars[b_full + s], nblk * L::BLK_BYTES);
+          uint8_t* dst = ring + s * L::TILE_BYTES;
+#pragma unroll
+          for (int c = 0; c < L::NCH; ++c) {
+            tma_load_3d(dst + c * L::KV_CHUNK, map, &bars[b_full + s], c * 64, kb0 * 64, it.bh);
+            if (nblk > 1)
+              tma_load_3d(dst + c * L::KV_CHUNK + 64 * 128, map, &bars[b_full + s], c * 64, kb1 * 64, it.bh);
+          }
+        }
+        ++qi;
+      }
+      if (is_k && ok) {
+        // end of this CTA's items
+        const int rs = qi % kItemRing;
+        if (mbar_wait(&bars[B_IEMPTY + rs], ((qi / kItemRing) & 1) ^ 1, abort_flag)) {
+          item_ring[rs * 4 + 0] = n_items;
+          mbar_arrive(&bars[B_IFULL + rs]);
+        }
       }
       // loads still in flight land before the CTA gives up its shared memory
-      for (int i = 1; i <= kKStages && i <= g; ++i)
-        mbar_drain(&bars[B_KFULL + (g - i) % kKStages], ((g - i) / kKStages) & 1);
+      // (g tiles and qi Q tiles were issued; a break can leave the last Q
+      // unissued, so only the tiles whose barriers were armed are waited for)
+      for (int i = 1; i <= stages && i <= g; ++i)
+        mbar_drain(&bars[b_full + (g - i) % stages], ((g - i) / stages) & 1);
+      if (is_k)
+        for (int i = 1; i <= kQSlots && i <= q_armed; ++i)
+          mbar_drain(&bars[B_QFULL + (q_armed - i) % kQSlots], ((q_armed - i) / kQSlots) & 1);
     }
-  } else if (warp == kVWarp) {
-    // ------------------------------------------------------------ V producer
+  } else if (warp == 1 || warp == kPVWarp) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two threads feed the tensor pipe: warp 1 issues S = Q K^T, warp kPVWarp
+    // issues O += P V. Each thread stalls while the tensor pipe's queue is
+    // full, and its mbarrier waits and commits queue behind its own MMAs; with
+    // two issuers the waits of one overlap the MMAs of the other. Since the
+    // two streams are not ordered with each other, the QK that overwrites an
+    // S buffer first waits for the P V that read P from it (PV_DONE).
     if (lane == 0) {
-      tma_prefetch_desc(&tmV);
-      LaneState s0, s1;
-      lane_init(s0);
-      lane_init(s1);
-      int g = 0;
-      bool ok = true;
-      auto turn = [&](LaneState& c, const int l) -> bool {
-        if (c.active && c.need && !take_item(bars, ring, l, c, n_items, abort_flag)) return false;
-        if (c.active) {
-          const int vs = g % kVStages;
-          int kb0, kb1;
-          const int nblk = tile_blocks(a, c.item, c.cnt, c.t, kb0, kb1);
-          const int bh = c.item / a.nqb;
-          if (!mbar_wait(&bars[B_VEMPTY + vs], ((g / kVStages) & 1) ^ 1, abort_flag)) return false;
-          mbar_arrive_expect_tx(&bars[B_VFULL + vs], nblk * L::BLK_BYTES);
-          uint8_t* dst = sV + vs * L::TILE_BYTES;
-#pragma unroll
-          for (int ch = 0; ch < L::NCH; ++ch) {
-            tma_load_3d(dst + ch * L::KV_CHUNK, &tmV, &bars[B_VFULL + vs], ch * 64, kb0 * 64, bh);
-            if (nblk > 1)
-              tma_load_3d(dst + ch * L::KV_CHUNK + 64 * 128, &tmV, &bars[B_VFULL + vs], ch * 64, kb1 * 64, bh);
-          }
-          ++g;
-          if (++c.t == c.T) c.need = true;
-        }
-        return true;
-      };
-      while (ok && (s0.active || s1.active)) {
-        ok = turn(s0, 0);
-        if (ok) ok = turn(s1, 1);
-      }
-      for (int i = 1; i <= kVStages && i <= g; ++i)
-        mbar_drain(&bars[B_VFULL + (g - i) % kVStages], ((g - i) / kVStages) & 1);
-    }
-  } else if (warp == kQWarp) {
-    // ------------------------------------------------------------ Q producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      int loads[kQSlots] = {0, 0, 0};
-      bool ok = true;
-      for (int r = 0; ok; ++r) {
-        // one request per non-empty item of this CTA, in order, then one with item n_items
-        const int rs = r % kQReqRing;
-        if (!(ok = mbar_wait(&bars[B_RFULL + rs], (r / kQReqRing) & 1, abort_flag))) break;
-        const int item = qreq[rs * 2 + 0];
-        const int qs = qreq[rs * 2 + 1];
-        mbar_arrive(&bars[B_REMPTY + rs]);
-        if (item >= n_items) break;
-        if (!(ok = mbar_wait(&bars[B_QEMPTY + qs], (loads[qs] & 1) ^ 1, abort_flag))) break;
-        const Item it = load_item(a, item);
-        mbar_arrive_expect_tx(&bars[B_QFULL + qs], L::Q_BYTES);
-#pragma unroll
-        for (int ch = 0; ch < L::NCH; ++ch)
-          tma_load_3d(sQ + qs * L::Q_BYTES + ch * L::Q_CHUNK, &tmQ, &bars[B_QFULL + qs], ch * 64, it.qb * a.bq, it.bh);
-        ++loads[qs];
-      }
-      for (int qs = 0; qs < kQSlots; ++qs)
-        if (loads[qs] > 0) mbar_drain(&bars[B_QFULL + qs], (loads[qs] - 1) & 1);
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+      const bool is_qk = warp == 1;
       const uint64_t qdesc0 = sw128_desc(smem_u32(sQ), 16, 1024);
       const uint64_t kdesc0 = sw128_desc(smem_u32(sK), 16, 1024);
       const uint64_t vdesc0 = sw128_desc(smem_u32(sV), L::KV_CHUNK, 1024);
       const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
       const uint32_t idesc_qk2 = idesc_bf16_f32(kBM, 128, false, false);
       const uint32_t idesc_qk1 = idesc_bf16_f32(kBM, 64, false, false);
-      // the P V each lane still owes for the last tile whose Q K^T it issued
-      struct Pend {
-        int g, nblk, lt, oi;
-        bool first, last, valid;
+      const uint32_t o_tm = tm + TM_O;
+      struct Ring {
+        int slot, n;
+        uint32_t phase;
+        __device__ void next() {
+          if (++slot == n) { slot = 0; phase ^= 1u; }
+        }
       };
-      // per lane: the pending P V, tiles issued (S / P phases), items issued (O phases)
-      struct LaneMma {
-        Pend pend;
-        int lt, oi;
-      };
-      LaneMma m0{}, m1{};
-      int quse0 = 0, quse1 = 0, quse2 = 0;   // items that have read each Q slot (Q phases)
-      LaneState s0, s1;
-      lane_init(s0);
-      lane_init(s1);
-      int g = 0;
+      Ring kv{0, is_qk ? kKStages : kVStages, 0};   // K ring (QK) or V ring (PV)
+      Ring sb{0, kSBufs, 0};
+      uint32_t phase1 = 0;   // O_EMPTY phase (PV)
+      int g = 0, qi = 0;
       bool ok = true;
-      auto issue_pv = [&](LaneMma& mm, const int ln) -> bool {
-        Pend& p = mm.pend;
-        if (!mbar_wait(&bars[B_PFULL + ln], p.lt & 1, abort_flag)) return false;
-        if (!mbar_wait(&bars[B_VFULL + p.g % kVStages], (p.g / kVStages) & 1, abort_flag)) return false;
-        if (p.first && !mbar_wait(&bars[B_OEMPTY + ln], (p.oi & 1) ^ 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint64_t vd = vdesc0 + (((p.g % kVStages) * L::TILE_BYTES) >> 4);
-        const uint32_t p_tm = tm + tm_s(ln);
-        const uint32_t o_tm = tm + tm_o(ln);
-        const int nk = p.nblk * 4;
+      int item = next_nonempty(a, blockIdx.x, gridDim.x, n_items);
+      Item it = item < n_items ? load_item(a, item) : Item{};
+      while (ok && item < n_items) {
+        // facts of the next item, fetched while this one is issued
+        const int nitem = next_nonempty(a, item + gridDim.x, gridDim.x, n_items);
+        const int ncnt = nitem < n_items ? (a.dense ? a.nkb : kept_count(a, nitem)) : 0;
+        for (int t = 0; t < it.T; ++t, ++g) {
+          const bool two = it.cnt - 2 * t >= 2;
+          if (is_qk) {
+            if (g >= kSBufs && !(ok = mbar_wait(&bars[B_PVDONE + sb.slot], sb.phase ^ 1u, abort_flag))) break;
+            if (!(ok = mbar_wait(&bars[B_KFULL + kv.slot], kv.phase, abort_flag))) break;
+            const int qs = qi % kQSlots;
+            if (t == 0 && !(ok = mbar_wait(&bars[B_QFULL + qs], (qi / kQSlots) & 1, abort_flag))) break;
+            tc_fence_after();
+            const uint32_t idesc = two ? idesc_qk2 : idesc_qk1;
+            const uint64_t qd = qdesc0 + ((qs * L::Q_BYTES) >> 4);
+            const uint64_t kd = kdesc0 + ((kv.slot * L::TILE_BYTES) >> 4);
+            const uint32_t s_tm = tm + tm_s(sb.slot);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          if (kk < nk) umma_ts(o_tm, p_tm + kk * 8, vd + ((kk * 2048u) >> 4), idesc_pv, (p.first && kk == 0) ? 0u : 1u);
-        tc_commit(&bars[B_VEMPTY + p.g % kVStages]);   // V slot free once this P V has read it
-        if (p.last) tc_commit(&bars[B_OFULL + ln]);
-        p.valid = false;
-        return true;
-      };
-      auto turn = [&](LaneState& c, LaneMma& mm, const int l) -> bool {
-        if (c.active && c.need) {
-          if (!take_item(bars, ring, l, c, n_items, abort_flag)) return false;
-          if (!c.active && mm.pend.valid && !issue_pv(mm, l)) return false;
-        }
-        if (c.active) {
-          if (mm.pend.valid && !issue_pv(mm, l)) return false;
-          const int ks = g % kKStages;
-          const int qs = c.qslot;
-          int& quse = qs == 0 ? quse0 : (qs == 1 ? quse1 : quse2);
-          if (!mbar_wait(&bars[B_KFULL + ks], (g / kKStages) & 1, abort_flag)) return false;
-          if (c.t == 0 && !mbar_wait(&bars[B_QFULL + qs], quse & 1, abort_flag)) return false;
-          tc_fence_after();
-          const int nblk = min(2, c.cnt - 2 * c.t);
-          const uint32_t idesc = nblk == 2 ? idesc_qk2 : idesc_qk1;
-          const uint64_t qd = qdesc0 + ((qs * L::Q_BYTES) >> 4);
-          const uint64_t kd = kdesc0 + ((ks * L::TILE_BYTES) >> 4);
-          const uint32_t s_tm = tm + tm_s(l);
+            for (int kk = 0; kk < D / 16; ++kk)
+              umma_ss(s_tm, qd + ((((kk >> 2) * L::Q_CHUNK) + (kk & 3) * 32u) >> 4),
+                      kd + ((((kk >> 2) * L::KV_CHUNK) + (kk & 3) * 32u) >> 4), idesc, kk > 0 ? 1u : 0u);
+            tc_commit(&bars[B_SFULL + sb.slot]);   // S ready, and the K slot free
+            if (t + 1 == it.T) tc_commit(&bars[B_QEMPTY + qs]);
+          } else {
+            if (!(ok = mbar_wait(&bars[B_PFULL + sb.slot], sb.phase, abort_flag))) break;
+            if (!(ok = mbar_wait(&bars[B_VFULL + kv.slot], kv.phase, abort_flag))) break;
+            if (t == 0) {
+              if (!(ok = mbar_wait(&bars[B_OEMPTY], phase1 ^ 1u, abort_flag))) break;
+              phase1 ^= 1u;
+            }
+            tc_fence_after();
+            const int nk = two ? 8 : 4;
+            const uint64_t vd = vdesc0 + ((kv.slot * L::TILE_BYTES) >> 4);
+            const uint32_t p_tm = tm + tm_s(sb.slot);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_ss(s_tm, qd + ((((kk >> 2) * L::Q_CHUNK) + (kk & 3) * 32u) >> 4),
-                    kd + ((((kk >> 2) * L::KV_CHUNK) + (kk & 3) * 32u) >> 4), idesc, kk > 0 ? 1u : 0u);
-          tc_commit(&bars[B_SFULL + l]);      // S ready (and O through the lane's previous tile)
-          tc_commit(&bars[B_KEMPTY + ks]);
-          mm.pend = Pend{g, nblk, mm.lt, mm.oi, c.t == 0, c.t + 1 == c.T, true};
-          if (c.t + 1 == c.T) {
-            tc_commit(&bars[B_QEMPTY + qs]);   // the slot may take another item's Q
-            ++quse;
-            ++mm.oi;
+            for (int kk = 0; kk < 8; ++kk)
+              if (kk < nk) umma_ts(o_tm, p_tm + kk * 8, vd + ((kk * 2048u) >> 4), idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&bars[B_PVDONE + sb.slot]);   // O updated; S buffer and V slot free
+            if (t + 1 == it.T) tc_commit(&bars[B_OFULL]);
           }
-          ++mm.lt;
-          ++g;
-          if (++c.t == c.T) c.need = true;
+          kv.next();
+          sb.next();
         }
-        return true;
-      };
-      while (ok && (s0.active || s1.active)) {
-        ok = turn(s0, m0, 0);
-        if (ok) ok = turn(s1, m1, 1);
+        if (!ok) break;
+        item = nitem;
+        ++qi;
+        if (item < n_items) {
+          it.bh = item / a.nqb;
+          it.qb = item % a.nqb;
+          it.cnt = ncnt;
+          it.T = (ncnt + 1) >> 1;
+        }
       }
-      // every MMA issued has completed before tensor memory is released
-      tc_commit(&bars[B_DRAIN]);
-      mbar_drain(&bars[B_DRAIN], 0);
+      // every MMA this thread issued has completed before tensor memory is released
+      tc_commit(&bars[B_DRAIN + (is_qk ? 0 : 1)]);
+      mbar_drain(&bars[B_DRAIN + (is_qk ? 0 : 1)], 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax + epilogue of one lane
-    const int ln = (warp - kSoftWarp0) / kLaneWarps;
+    // ------------------------------------------------------------ softmax + epilogue
+    const int sw = warp - 2;                  // 0..7
     const int quad = warp & 3;                // TMEM lane quadrant
+    const int half = sw >> 2;                 // which 64 columns of the tile
     const int row = quad * 32 + lane;         // query row within the tile
+    const int pair_bar = 1 + quad;            // named barrier of the two warps of this quadrant
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t s_tm = tm + lane_addr + tm_s(ln);
-    const uint32_t o_tm = tm + lane_addr + tm_o(ln);
     const float sl2 = a.scale_log2;
     const int tail_valid = a.N - (a.nkb - 1) * 64;
-    int n = 0, lt = 0, oi = 0;
+    int g = 0, qi = 0;
     bool ok = true;
+
+    int prev = blockIdx.x - static_cast<int>(gridDim.x);   // last item handled
     while (ok) {
-      const int slot = n % kItemRing;
-      // waits in these warps end the same way on every lane (a timeout on one
-      // lane stops the whole warp), so the warp stays converged
-      if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars[B_IFULL + ln * kItemRing + slot], (n / kItemRing) & 1, abort_flag)))) break;
-      const volatile int* e = ring + (ln * kItemRing + slot) * 4;
-      const int item = e[0], cnt = e[1];
-      const bool tail = e[2] != 0;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_IEMPTY + ln * kItemRing + slot]);
-      ++n;
-      if (item >= n_items) break;
-      const int bh = item / a.nqb, qb = item % a.nqb;
-      const int grow = qb * a.bq + row;
-      const bool store = row < a.bq && grow < a.N;
-      const long long orow_off = (static_cast<long long>(bh) * a.N + grow) * D;
-      if (cnt == 0) {
-        if (store) {
-          uint4* dz = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow_off);
-#pragma unroll
-          for (int c = 0; c < D / 8; ++c) dz[c] = make_uint4(0, 0, 0, 0);
-          if (a.lse) a.lse[static_cast<long long>(bh) * a.N + grow] = -INFINITY;
-        }
-        continue;
+      // next non-empty item, as posted by the K producer; the items skipped
+      // on the way have no kept block
+      const int rs = qi % kItemRing;
+      if (!mbar_wait(&bars[B_IFULL + rs], (qi / kItemRing) & 1, abort_flag)) {
+        // leaving without the partner: post the stop word where it reads next
+        // and give it the one arrival its next exchange needs
+        red_max[(g & 1) * 2 * kBM + half * kBM + row] = __uint_as_float(kStopBits);
+        red_sum[half * kBM + row] = __uint_as_float(kStopBits);
+        asm volatile("bar.arrive %0, 64;" ::"r"(pair_bar) : "memory");
+        ok = false;
+        break;
       }
-      const int T = (cnt + 1) >> 1;
+      const int item = item_ring[rs * 4 + 0];
+      Item it;
+      it.cnt = item_ring[rs * 4 + 1];
+      it.tail = item_ring[rs * 4 + 2] != 0;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_IEMPTY + rs]);
+      for (int z = prev + gridDim.x; z < item; z += gridDim.x) {
+        const Item iz = load_item(a, z);
+        const int gz = iz.qb * a.bq + row;
+        if (row < a.bq && gz < a.N) {
+          uint4* dz = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(iz.bh) * a.N + gz) * D + half * (D / 2));
+          for (int c = 0; c < D / 16; ++c) dz[c] = make_uint4(0, 0, 0, 0);
+          if (a.lse && half == 0) a.lse[static_cast<long long>(iz.bh) * a.N + gz] = -INFINITY;
+        }
+      }
+      if (item >= n_items) break;
+      prev = item;
+      it.bh = item / a.nqb;
+      it.qb = item % a.nqb;
+      it.T = (it.cnt + 1) >> 1;
+      const int grow = it.qb * a.bq + row;
+      const bool store = row < a.bq && grow < a.N;
+      const long long orow_off = (static_cast<long long>(it.bh) * a.N + grow) * D + half * (D / 2);
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + orow_off;
       if (a.alpha && store) {
-        // the epilogue reads this row of O_l: bring it into L2 while the item runs
+        // the epilogue reads this half row of O_l: bring it into L2 while the item runs
         const char* olr = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.o_l) + orow_off);
 #pragma unroll
-        for (int b = 0; b < D * 2; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(olr + b));
+        for (int b = 0; b < D; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(olr + b));
       }
-      float m = -INFINITY;     // running max, log2 domain
-      float lsum = 0.f;        // running row sum
-      for (int t = 0; t < T; ++t, ++lt) {
-        if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars[B_SFULL + ln], lt & 1, abort_flag)))) break;
-        tc_fence_after();
-        uint32_t r[128];
+      float m = -INFINITY;     // running max (log2 domain), identical in both halves
+      float l = 0.f;           // this half's share of the row sum
+      for (int t = 0; t < it.T; ++t, ++g) {
+        const int b = g % kSBufs;
+        // (after a failed wait the loads below read stale tensor memory; the
+        // values are dropped when the pair stops at the barrier that follows)
+        const bool s_ok = mbar_wait(&bars[B_SFULL + b], (g / kSBufs) & 1, abort_flag);
+        float x[64];
+        float mx;
+        {
+          tc_fence_after();
+          uint32_t r0[32], r1[32];
+          const uint32_t sa = tm + lane_addr + tm_s(b) + half * 64;
+          tmem_ld32(sa, r0);
+          tmem_ld32(sa + 32, r1);
+          tmem_wait_ld();
+          reg_fence(r0);
+          reg_fence(r1);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(s_tm + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * q4));
-        tmem_wait_ld();
+          for (int c = 0; c < 32; ++c) {
+            x[c] = __uint_as_float(r0[c]);
+            x[32 + c] = __uint_as_float(r1[c]);
+          }
+          if (t == it.T - 1) {
+            // last tile: possibly a single block, possibly the ragged last key block
+            const int nblk = it.cnt - 2 * t;
+            int valid = (half < nblk) ? 64 : 0;
+            if (it.tail && half == nblk - 1) valid = tail_valid;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(r + 32 * q4));
-        float x[128];
+            for (int c = 0; c < 64; ++c)
+              if (c >= valid) x[c] = -INFINITY;
+          }
+          // row max of this half: eight chains of 3-input max
+          float mx8[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(r[c]);
-        if (t == T - 1) {
-          // last tile: possibly a single block, possibly the ragged last key block
-          const int nblk = cnt - 2 * t;
-          const int valid = (nblk - 1) * 64 + (tail ? tail_valid : 64);
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c >= valid) x[c] = -INFINITY;
+          for (int j = 0; j < 8; ++j) {
+            mx8[j] = fmax3(x[j], x[8 + j], x[16 + j]);
+            mx8[j] = fmax3(mx8[j], x[24 + j], x[32 + j]);
+            mx8[j] = fmax3(mx8[j], x[40 + j], x[48 + j]);
+            mx8[j] = fmaxf(mx8[j], x[56 + j]);
+          }
+          mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         }
-        // row max: eight chains of 3-input max
-        float mx8[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          mx8[j] = x[j];
-#pragma unroll
-          for (int c = 8; c < 128; c += 16) mx8[j] = fmax3(mx8[j], x[c + j], x[c + 8 + j]);
-        }
-        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+        float* rm = red_max + (g & 1) * 2 * kBM;
+        const float posted = s_ok ? mx : __uint_as_float(kStopBits);
+        rm[half * kBM + row] = posted;
+        pair_sync(pair_bar);
+        const float pmx = rm[(half ^ 1) * kBM + row];
+        // Both warps combine the two posted words the same way (fmaxf skips the
+        // NaN stop word), so everything up to the end of the tile, branches
+        // included, is the same in both; the stop, if any, is taken there.
+        const bool stop = !s_ok || __float_as_uint(pmx) == kStopBits;
+        mx = fmaxf(posted, pmx);
         const float m_tile = mx * sl2;
         float corr = 1.f;
-        if (m_tile > m + kRescaleLog2) {
+        if (m_tile > m + 8.f) {
           corr = fast_exp2(m - m_tile);   // 0 on the first tile (m = -inf)
           m = m_tile;
-          lsum *= corr;
+          l *= corr;
         }
-        if (t > 0 && __any_sync(0xFFFFFFFFu, corr != 1.f)) {
-          // O holds the lane's tiles up to t-1 (their P V completed before this S)
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32_wait(o_tm + c0, o);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
-            tmem_st32(o_tm + c0, o);
-          }
-        }
-        // P = 2^(S * scale * log2(e) - m), two columns per packed instruction,
-        // written as bf16 over the first 64 columns of S.
+        // P = 2^(S * scale * log2(e) - m), two columns per packed instruction.
         const uint64_t sl2x2 = f2_make(sl2, sl2);
         const uint64_t negm2 = f2_make(-m, -m);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // packed (+0, +0)
-        auto exp_quarter = [&](const float* xq, int h) {
-          uint32_t p[16];
+        uint32_t p[32];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const uint64_t a2 = ffma2(f2_make(xq[2 * c], xq[2 * c + 1]), sl2x2, negm2);
-            float e0, e1;
-            if ((kPolyPairs >> (c & 7)) & 1) {
-              exp2_poly2(a2, e0, e1);
-            } else {
-              float a0, a1;
-              f2_split(a2, a0, a1);
-              e0 = fast_exp2(a0);
-              e1 = fast_exp2(a1);
-            }
-            acc[c & 3] = fadd2(acc[c & 3], f2_make(e0, e1));
-            p[c] = pack_bf16x2(e0, e1);
+        for (int c = 0; c < 32; ++c) {
+          const uint64_t a2 = ffma2(f2_make(x[2 * c], x[2 * c + 1]), sl2x2, negm2);
+          float e0, e1;
+          if ((kPolyPairs >> (c & 7)) & 1) {
+            exp2_poly2(a2, e0, e1);
+          } else {
+            float a0, a1;
+            f2_split(a2, a0, a1);
+            e0 = fast_exp2(a0);
+            e1 = fast_exp2(a1);
           }
-          tmem_st16(s_tm + h * 16, p);
-        };
-        exp_quarter(x, 0);
-        exp_quarter(x + 32, 1);
-        // columns 64..127 again from S (P only covers columns 0..63), so the
-        // upper half of the row need not stay in registers through the first half
-        {
-          uint32_t r2[64];
-          tmem_ld32(s_tm + 64, *reinterpret_cast<uint32_t(*)[32]>(r2));
-          tmem_ld32(s_tm + 96, *reinterpret_cast<uint32_t(*)[32]>(r2 + 32));
-          tmem_wait_ld();
-          reg_fence(*reinterpret_cast<uint32_t(*)[32]>(r2));
-          reg_fence(*reinterpret_cast<uint32_t(*)[32]>(r2 + 32));
-          float y[64];
-#pragma unroll
-          for (int c = 0; c < 64; ++c) y[c] = __uint_as_float(r2[c]);
-          if (t == T - 1) {
-            const int nblk = cnt - 2 * t;
-            const int valid = (nblk - 1) * 64 + (tail ? tail_valid : 64) - 64;
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (c >= valid) y[c] = -INFINITY;
-          }
-          exp_quarter(y, 2);
-          exp_quarter(y + 32, 3);
+          acc[c & 3] = fadd2(acc[c & 3], f2_make(e0, e1));
+          p[c] = pack_bf16x2(e0, e1);
         }
         {
           float s0, s1;
           f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), s0, s1);
-          lsum += s0 + s1;
+          l += s0 + s1;
+        }
+        tmem_st32(tm + lane_addr + tm_s(b) + half * 32, p);
+        if (!stop && t > 0 && __any_sync(0xFFFFFFFFu, corr != 1.f)) {
+          // O is complete up to the previous tile once its P V has landed
+          const int pb = (g - 1) % kSBufs;
+          if (!(ok = pair_agree(pair_bar, pair_flags + quad * 16 + 6, half, mbar_wait(&bars[B_PVDONE + pb], ((g - 1) / kSBufs) & 1, abort_flag)))) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c0 = 0; c0 < D / 2; c0 += 32) {
+            uint32_t o[32];
+            const uint32_t oa = tm + lane_addr + TM_O + half * (D / 2) + c0;
+            tmem_ld32_wait(oa, o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
+            tmem_st32(oa, o);
+          }
         }
         tmem_wait_st();
+        if (stop) {   // either warp's wait failed: both stop here
+          ok = false;
+          break;
+        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_PFULL + ln]);
+        if (lane == 0) mbar_arrive(&bars[B_PFULL + b]);
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
-      if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars[B_OFULL + ln], oi & 1, abort_flag)))) break;
-      ++oi;
-      tc_fence_after();
-      uint32_t o[D];
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) tmem_ld32(o_tm + c0, *reinterpret_cast<uint32_t(*)[32]>(o + c0));
-      tmem_wait_ld();
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(o + c0));
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_OEMPTY + ln]);   // the lane's next item may overwrite O now
+      const bool o_ok = mbar_wait(&bars[B_OFULL], qi & 1, abort_flag);
+      uint32_t o0[32], o1[32];
+      {
+        tc_fence_after();
+        tmem_ld32(tm + lane_addr + TM_O + half * (D / 2), o0);
+        if (D == 128) tmem_ld32(tm + lane_addr + TM_O + half * (D / 2) + 32, o1);
+        tmem_wait_ld();
+        reg_fence(o0);
+        if (D == 128) reg_fence(o1);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_OEMPTY]);   // the next item may overwrite O now
+      }
+      red_sum[half * kBM + row] = o_ok ? l : __uint_as_float(kStopBits);
+      pair_sync(pair_bar);
+      const float pl = red_sum[(half ^ 1) * kBM + row];
+      if (!(ok = o_ok && __float_as_uint(pl) != kStopBits)) break;
+      const float lt = l + pl;
+      const float inv_l = 1.f / lt;
       if (store) {
-        const float inv_l = 1.f / lsum;
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow_off);
+        uint4* dst = reinterpret_cast<uint4*>(orow);
         if (a.alpha) {
-          // O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l, O_s = o / l not yet rounded
-          const uint4* ol = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.o_l) + orow_off);
-          const float4* al = reinterpret_cast<const float4*>(a.alpha + static_cast<long long>(bh % a.H) * D);
+          // O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l with O_s = o / l not yet rounded
+          const uint4* olv = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.o_l) + orow_off);
+          const float4* alv = reinterpret_cast<const float4*>(a.alpha + static_cast<long long>(it.bh % a.H) * D + half * (D / 2));
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c) {
-            const uint4 lv = __ldg(ol + c);
-            const float4 a0 = __ldg(al + 2 * c), a1 = __ldg(al + 2 * c + 1);
+          for (int c = 0; c < D / 16; ++c) {
+            const uint32_t* oc = (c < 4) ? o0 + 8 * c : o1 + 8 * (c - 4);
+            const uint4 lv = __ldg(olv + c);
+            const float4 a0 = __ldg(alv + 2 * c), a1 = __ldg(alv + 2 * c + 1);
             const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
             const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             float r8[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const float olj = __uint_as_float((j & 1) ? (lw[j >> 1] & 0xFFFF0000u) : (lw[j >> 1] << 16));
-              r8[j] = fmaf(av[j], __uint_as_float(o[8 * c + j]) * inv_l - olj, olj);
+              r8[j] = fmaf(av[j], __uint_as_float(oc[j]) * inv_l - olj, olj);
             }
             dst[c] = make_uint4(pack_bf16x2(r8[0], r8[1]), pack_bf16x2(r8[2], r8[3]),
                                 pack_bf16x2(r8[4], r8[5]), pack_bf16x2(r8[6], r8[7]));
           }
         } else {
+          uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c)
-            dst[c] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv_l, __uint_as_float(o[8 * c + 1]) * inv_l),
-                                pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv_l, __uint_as_float(o[8 * c + 3]) * inv_l),
-                                pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv_l, __uint_as_float(o[8 * c + 5]) * inv_l),
-                                pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv_l, __uint_as_float(o[8 * c + 7]) * inv_l));
+          for (int c = 0; c < 16; ++c)
+            pk[c] = pack_bf16x2(__uint_as_float(o0[2 * c]) * inv_l, __uint_as_float(o0[2 * c + 1]) * inv_l);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          if (D == 128) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              pk[c] = pack_bf16x2(__uint_as_float(o1[2 * c]) * inv_l, __uint_as_float(o1[2 * c + 1]) * inv_l);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) dst[4 + c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
         }
-        if (a.lse) a.lse[static_cast<long long>(bh) * a.N + grow] = (m + log2f(lsum)) * 0.69314718055994531f;
       }
+      if (store && a.lse && half == 0)
+        a.lse[static_cast<long long>(it.bh) * a.N + grow] = (m + log2f(lt)) * 0.69314718055994531f;
+      ++qi;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tm, TM_COLS);
   }

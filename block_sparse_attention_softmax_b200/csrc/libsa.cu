@@ -4,6 +4,7 @@
 #include "mask_kernels.cu"
 #include "attn_kernel.cu"
 #include "linear_kernels.cu"
+#include "tile_kernels.cu"
 #include "sa_api.cu"
 #include "noalloc.cu"
 #include "diag.cu"

@@ -6,8 +6,11 @@
 // The array is created when the library's device code is loaded on a GPU and
 // stays allocated on every GPU that loads the library until the process exits.
 // Host code cannot use the array's name as a device address, so the first call
-// on each device looks the address up with cudaGetSymbolAddress (with that
-// device current) and caches it; later calls on that device reuse it.
+// in each CUDA context looks the address up with cudaGetSymbolAddress (with
+// that context's device current) and caches it under the context; later calls
+// in that context reuse it. A new context (after cudaDeviceReset, or a caller
+// that switches contexts) loads the module again, has its own copy of the
+// array, and gets its own lookup.
 //
 // Included from libsa.cu after sa_api.cu (same translation unit), so it reuses
 // that file's argument checks and error reporting.
@@ -22,24 +25,55 @@ static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBy
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 
-// Device address of g_static_scratch on the current device (looked up once).
-int static_scratch(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "sa_build_mask_noalloc (cudaGetDevice)");
-  if (dev < 0 || dev >= kMaxDevices) return fail(SA_ERR_UNSUPPORTED, "device ordinal %d exceeds %d", dev, kMaxDevices);
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "sa_build_mask_noalloc (cudaGetSymbolAddress)");
-    g_scratch_ptr[dev] = p;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
   }
-  *out = g_scratch_ptr[dev];
+  return fn;
+}
+
+constexpr int kMaxContexts = 64;
+std::mutex g_scratch_mutex;
+CUcontext g_scratch_ctx[kMaxContexts] = {};
+void* g_scratch_ptr[kMaxContexts] = {};
+int g_scratch_n = 0;
+
+// Device address of g_static_scratch in the current context (looked up once
+// per context). The lookup may load the module, which must not happen inside
+// a stream capture: a first call while `stream` captures is refused.
+int static_scratch(cudaStream_t stream, void** out) {
+  // also makes the device's primary context current if no context is
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(stream, &cap);
+  if (e != cudaSuccess) return cuda_fail(e, "sa_build_mask_noalloc (cudaStreamIsCapturing)");
+  CtxGetCurrentFn get = ctx_get_current();
+  CUcontext ctx = nullptr;
+  if (!get || get(&ctx) != CUDA_SUCCESS || !ctx)
+    return fail(SA_ERR_CUDA, "sa_build_mask_noalloc: no current CUDA context");
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  for (int i = 0; i < g_scratch_n; ++i)
+    if (g_scratch_ctx[i] == ctx) {
+      *out = g_scratch_ptr[i];
+      return SA_OK;
+    }
+  if (cap != cudaStreamCaptureStatusNone)
+    return fail(SA_ERR_INVALID_ARG,
+                "sa_build_mask_noalloc: the first call in a CUDA context must come before any stream "
+                "capture (it looks up the fixed scratch's address)");
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "sa_build_mask_noalloc (cudaGetSymbolAddress)");
+  const int slot = g_scratch_n < kMaxContexts ? g_scratch_n++ : kMaxContexts - 1;
+  g_scratch_ctx[slot] = ctx;
+  g_scratch_ptr[slot] = p;
+  *out = p;
   return SA_OK;
 }
 
@@ -70,7 +104,7 @@ int sa_build_mask_noalloc(const uint16_t* q, const uint16_t* k, int B, int H, in
                 "sa_build_mask_noalloc: this problem needs %zu bytes of scratch; the fixed scratch holds %zu "
                 "(use sa_build_mask with a caller workspace)", w.total, kStaticScratchBytes);
   void* scratch = nullptr;
-  rc = static_scratch(&scratch);
+  rc = static_scratch(static_cast<cudaStream_t>(stream), &scratch);
   if (rc) return rc;
   if (scale <= 0.0) scale = 1.0 / sqrt(static_cast<double>(d));
   // Nothing here must start at zero: every scratch byte that is read was

@@ -405,4 +405,57 @@ int sa_blend(const uint16_t* o_s, const uint16_t* q, const float* kv_state, cons
   return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_blend");
 }
 
+int sa_trip_pool(const uint16_t* q, const uint16_t* k, int B, int H, int N, int d, int bq, int bk,
+                 float* q_desc, float* k_desc, void* stream) {
+  int rc = check_shape(B, H, N, d, bq, bk);
+  if (rc) return rc;
+  if (!q || !k || !q_desc || !k_desc) return fail(SA_ERR_INVALID_ARG, "sa_trip_pool: null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_desc) || !aligned16(k_desc))
+    return fail(SA_ERR_ALIGN, "sa_trip_pool: pointers must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_trip_pool(q, B * H, N, d, bq, q_desc, st);
+  if (e == cudaSuccess) e = launch_trip_pool(k, B * H, N, d, bk, k_desc, st);
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_trip_pool");
+}
+
+int sa_tile_heatmap(const uint16_t* q, const uint16_t* k, int B, int H, int N, int d, int bq, int bk,
+                    double scale, const int32_t* rows_opt, int n_rows, float* heat, float* lse_opt,
+                    void* stream) {
+  int rc = check_shape(B, H, N, d, bq, bk);
+  if (rc) return rc;
+  if (!q || !k || !heat) return fail(SA_ERR_INVALID_ARG, "sa_tile_heatmap: null pointer");
+  if (!isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "scale must be finite");
+  const void* ptrs[] = {q, k, heat, lse_opt, rows_opt};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "sa_tile_heatmap: pointers must be 16-byte aligned");
+  const long long all_rows = static_cast<long long>(B) * H * ((N + bq - 1) / bq);
+  if (rows_opt && (n_rows < 0 || n_rows > all_rows))
+    return fail(SA_ERR_INVALID_ARG, "sa_tile_heatmap: n_rows = %d outside [0, %lld]", n_rows, all_rows);
+  if (all_rows > 0x7FFFFFFFLL) return fail(SA_ERR_UNSUPPORTED, "sa_tile_heatmap: too many query-block rows");
+  if (scale <= 0.0) scale = 1.0 / sqrt(static_cast<double>(d));
+  const int n_items = rows_opt ? n_rows : static_cast<int>(all_rows);
+  cudaError_t e = launch_heat(q, k, B * H, N, d, bq, rows_opt, n_items, scale, heat, lse_opt,
+                              static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_tile_heatmap");
+}
+
+int sa_select_mask(const float* scores, int B, int H, int n_qb, int n_kb, double topk_frac, double topp,
+                   int32_t* kv_idx, int32_t* kv_cnt, uint8_t* mask_opt, void* stream) {
+  if (B <= 0 || H <= 0 || n_qb <= 0 || n_kb <= 0)
+    return fail(SA_ERR_INVALID_ARG, "sa_select_mask: B, H, n_qb and n_kb must be positive");
+  if (n_kb > kMaxKeyBlocks) return fail(SA_ERR_UNSUPPORTED, "n_kb = %d exceeds %d", n_kb, kMaxKeyBlocks);
+  const long long rows = static_cast<long long>(B) * H * n_qb;
+  if (rows > 0x7FFFFFFFLL || rows * n_kb >= (1LL << 34)) return fail(SA_ERR_UNSUPPORTED, "sa_select_mask: too large");
+  if (!scores || !kv_idx || !kv_cnt) return fail(SA_ERR_INVALID_ARG, "sa_select_mask: null pointer");
+  if (!(topk_frac > 0.0 && topk_frac <= 1.0)) return fail(SA_ERR_INVALID_ARG, "topk_frac %g outside (0, 1]", topk_frac);
+  if (!(topp >= 0.0 && topp <= 1.0)) return fail(SA_ERR_INVALID_ARG, "topp %g outside [0, 1]", topp);
+  const void* ptrs[] = {scores, kv_idx, kv_cnt, mask_opt};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "sa_select_mask: pointers must be 16-byte aligned");
+  const int k_sel = static_cast<int>(fmin(static_cast<double>(n_kb), fmax(1.0, ceil(topk_frac * n_kb - 1e-9))));
+  cudaError_t e = launch_select(scores, n_kb, static_cast<int>(rows), n_kb, k_sel, topp, kv_idx, kv_cnt, mask_opt,
+                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_select_mask");
+}
+
 }  // extern "C"

@@ -100,6 +100,11 @@ size_t linear_out_ws_bytes(int BH, int d);
 cudaError_t launch_linear_state(const LinearArgs& a, cudaStream_t st);
 cudaError_t launch_linear_out(const LinearArgs& a, cudaStream_t st);
 
+// Tile scoring: TripPool descriptors and the two-pass max-pooled heatmap.
+cudaError_t launch_trip_pool(const void* x, int BH, int N, int d, int b, float* out, cudaStream_t st);
+cudaError_t launch_heat(const void* q, const void* k, int BH, int N, int d, int bq, const int* rows, int n_items,
+                        double scale, float* heat, float* lse, cudaStream_t st);
+
 // Driver entry point for cuTensorMapEncodeTiled, resolved once. 3-D maps
 // (inner, rows, planes), 128-byte swizzle, zero fill out of bounds.
 CUresult encode_tensor_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t inner,

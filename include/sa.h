@@ -164,6 +164,42 @@ int sa_blend(const uint16_t* o_s, const uint16_t* q, const float* kv_state, cons
              const float* alpha, int B, int H, int N, int d, uint16_t* o,
              void* workspace, size_t ws_bytes, void* stream);
 
+/* Tile scoring from the full attention map ("Veda" §2.1 and §2.3).
+ *
+ * sa_trip_pool: TripPool descriptors of every query block (bq tokens) and key
+ *   block (bk tokens): per channel the mean, the maximum and the minimum over
+ *   the block's valid tokens, concatenated as [mean | max | min]:
+ *     q_desc [B, H, n_qb, 3d] fp32,  k_desc [B, H, n_kb, 3d] fp32.
+ *   The learned estimator that maps them to tile scores is not part of this
+ *   library (it needs trained weights); its scores can be passed to
+ *   sa_select_mask.
+ *
+ * sa_tile_heatmap: the reference tile scores, in two passes over every key
+ *   tile of each evaluated query block: (1) the log-sum-exp of each query row
+ *   over all N keys, (2) per (query block, key block) tile
+ *     heat[qb, kb] = max over rows i of qb and keys j of kb of (scale q_i.k_j - LSE_i),
+ *   the natural log of the largest full-attention probability in the tile
+ *   (max pooling of the attention map over the tile; always <= 0).
+ *   heat [B, H, n_qb, n_kb] fp32. rows_opt: device int32 list of n_rows
+ *   query-block rows (b * H * n_qb + h * n_qb + qb) to evaluate, the sparse
+ *   teacher of a random subset of query tiles; NULL evaluates every row (n_rows
+ *   ignored). Rows not evaluated are left untouched. lse_opt [B, H, N] fp32
+ *   (natural log) receives the first pass for the evaluated rows' tokens, or
+ *   NULL. scale <= 0 selects 1/sqrt(d). Shape rules as sa_sparse_attn_fwd.
+ *
+ * sa_select_mask: the hybrid Top-k ∪ Top-p rule of sa_build_mask applied to
+ *   given block scores (softmax over each row, the same order and ties):
+ *   scores [B, H, n_qb, n_kb] fp32, finite; with scores = heat the row
+ *   distribution is the max-pooled probabilities normalised over the row.
+ *   Outputs as sa_build_mask (kv_idx, kv_cnt, optional uint8 mask). n_kb <= 16384. */
+int sa_trip_pool(const uint16_t* q, const uint16_t* k, int B, int H, int N, int d, int bq, int bk,
+                 float* q_desc, float* k_desc, void* stream);
+int sa_tile_heatmap(const uint16_t* q, const uint16_t* k, int B, int H, int N, int d, int bq, int bk,
+                    double scale, const int32_t* rows_opt, int n_rows, float* heat, float* lse_opt,
+                    void* stream);
+int sa_select_mask(const float* scores, int B, int H, int n_qb, int n_kb, double topk_frac, double topp,
+                   int32_t* kv_idx, int32_t* kv_cnt, uint8_t* mask_opt, void* stream);
+
 /* Mask builder that allocates nothing (no counterpart in the pages: it exists
  * for callers, not for the method). Some callers may not allocate device memory
  * when they call in: an inference engine's per-request callback that must not
@@ -177,9 +213,11 @@ int sa_blend(const uint16_t* o_s, const uint16_t* q, const float* kv_state, cons
  *   - Problems whose scratch, as counted by sa_build_mask_workspace_size(), is
  *     above 32 MiB (33554432 bytes) are rejected with SA_ERR_UNSUPPORTED before
  *     anything is launched; about 12 heads of 32760 tokens at d = 128 fit.
- *   - The first call on each device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *   - The first call in each CUDA context looks up the array's device address
+ *     (with that context current) and caches it under the context, so a new
+ *     context (after cudaDeviceReset, or another context on the same device)
+ *     gets its own lookup. Make that first call before any stream capture: a
+ *     first call while `stream` is capturing returns SA_ERR_INVALID_ARG.
  *   - All calls share the one array and it keeps the last call's contents.
  *     Calls whose work overlaps on the GPU (for example on two streams without
  *     ordering between them) race on it; order them on one stream or with

@@ -11,6 +11,8 @@ Pages followed (titles and sections):
   * "SLA2" (ai-papers.net), 提案手法 ① mean pooling of queries and keys before
     scoring, ② O = alpha * O_s + (1 - alpha) * O_l.
   * "SALAD", §2.1 a linear-attention branch in parallel with sparse attention.
+  * "Veda", §2.1 TripPool descriptors and the reference mask from max-pooling
+    the full attention map over tiles, §2.3 the two-pass heatmap.
 
 Every function works on one (batch, head) slice in float64 numpy arrays.
 """
@@ -18,5 +20,6 @@ from .sparse_attention import (  # noqa: F401
     as_f64, pool_blocks, block_scores, block_softmax, topk_count, descending_order,
     topp_count, topk_set, topp_set, hybrid_row, build_mask, kv_lists, mask_from_lists,
     masked_attention, dense_attention, phi, linear_state, linear_out, blend,
-    row_threshold_info, NEAR_TIE_TOL,
+    row_threshold_info, NEAR_TIE_TOL, trip_pool, full_attention_lse, tile_max_heatmap,
+    mask_from_scores,
 )

@@ -262,3 +262,69 @@ def linear_out(q: np.ndarray, S: np.ndarray, z: np.ndarray) -> np.ndarray:
 
 def blend(o_s: np.ndarray, o_l: np.ndarray, alpha_h: np.ndarray) -> np.ndarray:
     return alpha_h[None, :] * o_s + (1.0 - alpha_h[None, :]) * o_l
+
+
+# --------------------------------------------------------------------------
+# Tile scoring from the full attention map (Veda §2.1 and §2.3): TripPool
+# descriptors (mean, max and min of each block, per channel), and the
+# reference heatmap that max-pools the full attention probabilities over each
+# (query block, key block) tile, computed in two passes. Either kind of block
+# score can feed the same hybrid Top-k ∪ Top-p selection.
+# --------------------------------------------------------------------------
+
+def trip_pool(x: np.ndarray, b: int) -> np.ndarray:
+    """TripPool descriptor of each block of b tokens of x [N, d]: the mean, the
+    maximum and the minimum over the block's valid tokens, per channel,
+    concatenated as [mean | max | min] -> [ceil(N/b), 3d]."""
+    N, d = x.shape
+    n = -(-N // b)
+    out = np.empty((n, 3 * d), dtype=np.float64)
+    for i in range(n):
+        rows = x[i * b:min(N, (i + 1) * b)]
+        out[i, :d] = rows.sum(axis=0) / rows.shape[0]
+        out[i, d:2 * d] = rows.max(axis=0)
+        out[i, 2 * d:] = rows.min(axis=0)
+    return out
+
+
+def full_attention_lse(q: np.ndarray, k: np.ndarray, scale=None, rows=None) -> np.ndarray:
+    """First pass: the natural-log log-sum-exp of each query row's logits
+    scale * q_i . k_j over all N keys (the full softmax's normaliser)."""
+    N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rows = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
+    logits = scale * (q[rows] @ k.T)
+    m = logits.max(axis=1, keepdims=True)
+    return (m + np.log(np.exp(logits - m).sum(axis=1, keepdims=True)))[:, 0]
+
+
+def tile_max_heatmap(q: np.ndarray, k: np.ndarray, bq: int, bk: int, scale=None, q_blocks=None):
+    """Second pass: for each (query block, key block) tile, the log of the
+    largest full-attention probability inside it,
+        logH[qb, kb] = max over i in qb, j in kb of (scale * q_i . k_j - LSE_i),
+    with LSE from the first pass (valid tokens only). q_blocks: the query
+    blocks to evaluate (default all); the other rows are -inf."""
+    N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    n_qb, n_kb = -(-N // bq), -(-N // bk)
+    q_blocks = range(n_qb) if q_blocks is None else q_blocks
+    out = np.full((n_qb, n_kb), -np.inf, dtype=np.float64)
+    for qb in q_blocks:
+        rows = np.arange(qb * bq, min(N, (qb + 1) * bq))
+        lse = full_attention_lse(q, k, scale, rows)
+        logp = scale * (q[rows] @ k.T) - lse[:, None]            # [rows, N] log probabilities
+        for kb in range(n_kb):
+            out[qb, kb] = logp[:, kb * bk:min(N, (kb + 1) * bk)].max()
+    return out
+
+
+def mask_from_scores(s: np.ndarray, k_frac: float, p: float) -> np.ndarray:
+    """The hybrid Top-k ∪ Top-p rule applied to each row of given block scores
+    (softmax over the row, SpargeAttention2 §2(1)); with s = logH the row
+    distribution is the max-pooled probabilities normalised over the row."""
+    mask = np.zeros(s.shape, dtype=bool)
+    for r in range(s.shape[0]):
+        mask[r] = hybrid_row(s[r], k_frac, p)[0]
+    return mask

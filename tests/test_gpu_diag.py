@@ -73,3 +73,37 @@ def test_fma_pipe_exp2_accuracy(cuda_lib):
     lo = xs < -125.0
     assert (yp[lo] >= 0).all() and (yp[lo] <= 2.0 ** -124).all()
     assert np.isfinite(yp).all()
+
+
+def test_attention_wait_runs_out_on_the_tiny_workload(cuda_lib):
+    """With the wait bound lowered to 100 cycles the attention kernel's waits
+    for data run out: every role stops, the producers wait for the TMA loads
+    they issued and the MMA threads for their MMAs, the two softmax warps of
+    each pair stop at the same barrier, and the kernel returns. The status
+    reports the timeout once; with the default bound restored the same call
+    matches the oracle."""
+    import oracle
+    from gpu_helpers import assert_close
+    sa = cuda_lib
+    wl = WORKLOADS["tiny"]
+    x = make_inputs(wl, "cpu")
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    m = sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp, want_mask=True)
+    torch.cuda.synchronize()
+    assert _status_code(sa) == "SA_OK"
+    try:
+        sa.sa_diag_set_wait_limit(100)
+        sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"])
+        torch.cuda.synchronize()
+    finally:
+        sa.sa_diag_set_wait_limit(0)
+    assert _status_code(sa) == "SA_ERR_DEVICE_TIMEOUT"
+    assert _status_code(sa) == "SA_OK"
+    o = sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"])
+    torch.cuda.synchronize()
+    assert _status_code(sa) == "SA_OK"
+    f64 = oracle.as_f64
+    for h in range(wl.H):
+        ro, _ = oracle.masked_attention(f64(x["q"][0, h]), f64(x["k"][0, h]), f64(x["v"][0, h]),
+                                        m["mask"][0, h].cpu().numpy().astype(bool), wl.bq, wl.bk)
+        assert_close(o[0, h].float().cpu().numpy(), ro, f"O head {h} after the timeout")

@@ -401,3 +401,62 @@ def test_tiny_workload_masks_match_golden():
         idx, cnt = oracle.kv_lists(out["mask"])
         for r in range(idx.shape[0]):
             assert want[(h, r)] == (int(cnt[r]), idx[r, :cnt[r]].tolist())
+
+
+# ---------------------------------------------------------------- tile scoring (Veda §2.1, §2.3)
+def test_trip_pool_by_brute_force_loops():
+    x = _rng(41).standard_normal((37, 5))
+    desc = oracle.trip_pool(x, 8)
+    assert desc.shape == (5, 15)
+    for blk in range(5):
+        rows = [t for t in range(37) if t // 8 == blk]
+        for c in range(5):
+            vals = [x[t, c] for t in rows]
+            assert abs(desc[blk, c] - sum(vals) / len(vals)) < 1e-14
+            assert desc[blk, 5 + c] == max(vals)
+            assert desc[blk, 10 + c] == min(vals)
+    means, _ = oracle.pool_blocks(x, 8)
+    assert np.array_equal(desc[:, :5], means)
+
+
+def test_tile_max_heatmap_by_brute_force_probabilities():
+    """logH against the full attention matrix built entry by entry (exp and
+    row sums by scalar loops), max-pooled over ragged tiles."""
+    rng = _rng(42)
+    N, d, bq, bk = 45, 6, 16, 8
+    q, k = rng.standard_normal((N, d)) * 1.5, rng.standard_normal((N, d))
+    scale = 1.0 / math.sqrt(d)
+    P = np.zeros((N, N))
+    for i in range(N):
+        w = [math.exp(scale * sum(q[i, c] * k[j, c] for c in range(d))) for j in range(N)]
+        z = sum(w)
+        for j in range(N):
+            P[i, j] = w[j] / z
+    want = np.zeros((-(-N // bq), -(-N // bk)))
+    for qb in range(want.shape[0]):
+        for kb in range(want.shape[1]):
+            want[qb, kb] = math.log(P[qb * bq:(qb + 1) * bq, kb * bk:(kb + 1) * bk].max())
+    got = oracle.tile_max_heatmap(q, k, bq, bk)
+    assert np.abs(got - want).max() < 1e-12
+    assert (got <= 1e-15).all()
+    # every row of each query block holds a probability >= 1/N somewhere
+    assert (got.max(axis=1) >= math.log(1.0 / N) - 1e-12).all()
+    # the first pass alone: LSE against torch.logsumexp
+    lse = oracle.full_attention_lse(q, k)
+    ref = torch.logsumexp(torch.from_numpy(scale * q @ k.T), dim=1).numpy()
+    assert np.abs(lse - ref).max() < 1e-12
+    # a subset of query blocks (the sparse teacher): the same rows, -inf elsewhere
+    part = oracle.tile_max_heatmap(q, k, bq, bk, q_blocks=[1])
+    assert np.array_equal(part[1], got[1]) and np.isneginf(part[[0, 2]]).all()
+
+
+def test_mask_from_scores_is_the_hybrid_rule_per_row():
+    rng = _rng(43)
+    s = rng.standard_normal((6, 20)) * 2.0
+    m = oracle.mask_from_scores(s, 0.1, 0.7)
+    for r in range(6):
+        assert (m[r] == oracle.hybrid_row(s[r], 0.1, 0.7)[0]).all()
+    # on a head's own block scores it reproduces build_mask
+    q, k = rng.standard_normal((300, 8)) * 2, rng.standard_normal((300, 8))
+    out = oracle.build_mask(q, k, 32, 16, 0.2, 0.8)
+    assert (oracle.mask_from_scores(out["s"], 0.2, 0.8) == out["mask"]).all()

@@ -67,3 +67,50 @@ def test_noalloc_rejects_problems_above_the_fixed_scratch(cuda_lib):
                                    wl.topp, 0.0, fake, fake, None, None)
     assert rc == -2
     assert b"fixed scratch" in lib.sa_last_error()
+
+
+def test_noalloc_call_allocates_no_device_memory(cuda_lib):
+    """After a first call (which looks up the fixed scratch), a further call
+    with its outputs already allocated leaves the device's free memory as it
+    was: the entry point draws on no allocator."""
+    sa = cuda_lib
+    lib = sa.load()
+    dev = torch.device("cuda", 0)
+    wl = WORKLOADS["wan13b_480p"]
+    x = make_inputs(wl, dev)
+    q, k = x["q"], x["k"]
+    B, H, N, d = q.shape
+    nqb, nkb = -(-N // wl.bq), -(-N // wl.bk)
+    idx = torch.empty((B, H, nqb, nkb), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B, H, nqb), dtype=torch.int32, device=dev)
+    stream = P(torch.cuda.current_stream().cuda_stream)
+    args = (P(q.data_ptr()), P(k.data_ptr()), B, H, N, d, wl.bq, wl.bk, float(wl.topk), float(wl.topp),
+            0.0, P(idx.data_ptr()), P(cnt.data_ptr()), None, stream)
+    assert lib.sa_build_mask_noalloc(*args) == 0
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info(dev)
+    assert lib.sa_build_mask_noalloc(*args) == 0, lib.sa_last_error().decode()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info(dev)
+    assert free0 == free1
+    sa.sa_device_status(dev)
+
+
+def test_noalloc_candidate_builder_on_the_shared_array(cuda_lib, monkeypatch):
+    """The candidate builder (forced on shapes the size rule would send to the
+    score-matrix builder) keeps its per-row statistics, candidate counts and
+    hand-back state in the same fixed array; two calls in a row against
+    sa_build_mask under the same setting."""
+    sa = cuda_lib
+    lib = sa.load()
+    dev = torch.device("cuda", 0)
+    monkeypatch.setenv("SA_MASK_BUILDER", "candidates")
+    wl = WORKLOADS["tiny"]
+    x = make_inputs(wl, dev)
+    for q, k in ((x["q"], x["k"]), ((x["q"].float() * 3).to(torch.bfloat16), x["k"])):
+        idx, cnt, mask = _noalloc(lib, q, k, wl.bq, wl.bk, wl.topk, wl.topp, True)
+        ref = sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp, want_mask=True)
+        torch.cuda.synchronize()
+        _same_lists(ref, idx, cnt)
+        assert torch.equal(ref["mask"], mask)
+    sa.sa_device_status(dev)
