@@ -51,6 +51,17 @@ _SIGNATURES = {
                                 c_double, c_void_p, c_int, c_void_p, c_void_p, c_void_p]),
     "sa_select_mask": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_double, c_double,
                                c_void_p, c_void_p, c_void_p, c_void_p]),
+    "sa_tile_permutation": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "sa_permute_tokens": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p]),
+    "sa_sparse_attn_bwd_workspace_size": (c_size_t, [c_int] * 6),
+    "sa_sparse_attn_bwd": (c_int, [c_void_p] * 6 + [c_int] * 6 + [c_void_p, c_void_p, c_double, c_void_p, c_void_p,
+                                                                c_void_p, c_void_p, c_size_t, c_void_p]),
+    "sa_linear_bwd_workspace_size": (c_size_t, [c_int] * 4),
+    "sa_linear_bwd": (c_int, [c_void_p] * 6 + [c_int] * 5 + [c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                                              c_void_p]),
+    "sa_blend_bwd_workspace_size": (c_size_t, [c_int] * 4),
+    "sa_blend_bwd": (c_int, [c_void_p] * 4 + [c_int] * 4 + [c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                                            c_void_p]),
     "sa_diag_set_device_status": (c_int, [c_int]),
     "sa_diag_set_wait_limit": (c_int, [ctypes.c_longlong]),
     "sa_diag_wait_timeout": (c_int, [c_void_p, c_void_p]),
@@ -361,6 +372,83 @@ def sa_select_mask(scores, topk, topp, want_mask=False):
     return out
 
 
+def sa_tile_permutation(grid, tiles, device=None):
+    """[H, N] int32 tile-major token orders of a (T, Hh, W) grid, one tiling
+    (p_t, p_h, p_w) per head."""
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    T, Hh, W = (int(g) for g in grid)
+    flat = [int(v) for tile in tiles for v in tile]
+    H = len(flat) // 3
+    if H * 3 != len(flat) or H == 0:
+        raise ValueError("tiles: one (p_t, p_h, p_w) triple per head")
+    perm = torch.empty(H, T * Hh * W, dtype=torch.int32, device=device)
+    arr = (ctypes.c_int32 * len(flat))(*flat)
+    _call("sa_tile_permutation", H, T, Hh, W, ctypes.cast(arr, c_void_p), _ptr(perm), _stream(device))
+    return perm
+
+
+def sa_permute_tokens(x, perm, inverse=False, out=None):
+    """Rows of x [B, H, N, d] in each head's order (or back, with inverse)."""
+    B, H, N, d = _qkv(x, names=("x",))
+    _expect("perm", perm, (H, N), torch.int32)
+    if out is not None:
+        _expect("out", out, x.shape, torch.bfloat16)
+    _on_device(x.device, x=x, perm=perm, out=out)
+    y = out if out is not None else torch.empty_like(x)
+    _call("sa_permute_tokens", _ptr(x), _ptr(perm), B, H, N, d, int(bool(inverse)), _ptr(y), _stream(x.device))
+    return y
+
+
+def sa_sparse_attn_bwd(q, k, v, o, lse, dout, bq, bk, kv_idx, kv_cnt, scale=0.0):
+    """(dq, dk, dv) fp32 of the sparse attention for the upstream gradient dout."""
+    B, H, N, d = _qkv(q, k, v, o, dout, names=("q", "k", "v", "o", "dout"))
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    _expect("lse", lse, (B, H, N), torch.float32)
+    _expect("kv_idx", kv_idx, (B, H, nqb, nkb), torch.int32)
+    _expect("kv_cnt", kv_cnt, (B, H, nqb), torch.int32)
+    dev = q.device
+    _on_device(dev, q=q, k=k, v=v, o=o, lse=lse, dout=dout, kv_idx=kv_idx, kv_cnt=kv_cnt)
+    dq, dk, dv = (torch.empty(B, H, N, d, dtype=torch.float32, device=dev) for _ in range(3))
+    ws = _workspace(load().sa_sparse_attn_bwd_workspace_size(B, H, N, d, bq, bk), dev)
+    _call("sa_sparse_attn_bwd", _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), B, H, N, d, bq, bk,
+          _ptr(kv_idx), _ptr(kv_cnt), float(scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(dev))
+    return dq, dk, dv
+
+
+def sa_linear_bwd(q, k, v, kv_state, ksum, dout_l, grads=None):
+    """(dq, dk, dv) fp32 of the linear branch; with grads=(dq, dk, dv) it adds into them."""
+    B, H, N, d = _qkv(q, k, v, dout_l, names=("q", "k", "v", "dout_l"))
+    _expect("kv_state", kv_state, (B, H, d, d), torch.float32)
+    _expect("ksum", ksum, (B, H, d), torch.float32)
+    dev = q.device
+    _on_device(dev, q=q, k=k, v=v, kv_state=kv_state, ksum=ksum, dout_l=dout_l)
+    if grads is None:
+        grads = tuple(torch.empty(B, H, N, d, dtype=torch.float32, device=dev) for _ in range(3))
+        acc = 0
+    else:
+        for name, t in zip(("dq", "dk", "dv"), grads):
+            _expect(name, t, (B, H, N, d), torch.float32)
+        acc = 1
+    ws = _workspace(load().sa_linear_bwd_workspace_size(B, H, N, d), dev)
+    _call("sa_linear_bwd", _ptr(q), _ptr(k), _ptr(v), _ptr(kv_state), _ptr(ksum), _ptr(dout_l), B, H, N, d, acc,
+          *(_ptr(t) for t in grads), _ptr(ws), ws.numel(), _stream(dev))
+    return grads
+
+
+def sa_blend_bwd(o_s, o_l, alpha, dout):
+    """(do_s, do_l, dalpha) of O = alpha * o_s + (1 - alpha) * o_l."""
+    B, H, N, d = _qkv(o_s, o_l, dout, names=("o_s", "o_l", "dout"))
+    _expect("alpha", alpha, (H, d), torch.float32)
+    dev = o_s.device
+    _on_device(dev, o_s=o_s, o_l=o_l, alpha=alpha, dout=dout)
+    do_s, do_l = torch.empty_like(o_s), torch.empty_like(o_s)
+    da = torch.empty(H, d, dtype=torch.float32, device=dev)
+    ws = _workspace(load().sa_blend_bwd_workspace_size(B, H, N, d), dev)
+    _call("sa_blend_bwd", _ptr(o_s), _ptr(o_l), _ptr(alpha), _ptr(dout), B, H, N, d, _ptr(do_s), _ptr(do_l),
+          _ptr(da), _ptr(ws), ws.numel(), _stream(dev))
+    return do_s, do_l, da
+
+
 def _path_on_device(q, k, v, bq, bk, topk, topp, alpha, scale, out=None):
     m = sa_build_mask(q, k, bq, bk, topk, topp, scale)
     if alpha is None:
@@ -372,7 +460,7 @@ def _path_on_device(q, k, v, bq, bk, topk, topp, alpha, scale, out=None):
 
 
 def block_sparse_attention(q, k, v, bq=128, bk=64, topk=0.05, topp=0.9, alpha=None, scale=0.0,
-                           device=None, out=None, chunks=8):
+                           device=None, out=None, chunks=8, perm=None):
     """Whole path: mask, sparse attention and (when alpha is given) the linear
     branch blended in. Device tensors stay on the device. Host tensors are
     copied in, and the result is copied back into `out` (a pinned host tensor
@@ -380,7 +468,16 @@ def block_sparse_attention(q, k, v, bq=128, bk=64, topk=0.05, topp=0.9, alpha=No
     tensors the heads are split into up to `chunks` groups that go through a
     three-stream pipeline: the copy in of group c + 1, the path on group c and
     the copy out of group c - 1 overlap. Pinned host tensors make the copies
-    asynchronous."""
+    asynchronous. With `perm` ([H, N] int32 device orders, e.g. from
+    sa_tile_permutation; device tensors only) the tokens are gathered into
+    each head's order, the path runs on the permuted sequence and the output
+    is scattered back."""
+    if perm is not None:
+        if not q.is_cuda:
+            raise ValueError("perm: the permuted path takes device tensors")
+        qp, kp, vp = (sa_permute_tokens(t, perm) for t in (q, k, v))
+        op = _path_on_device(qp, kp, vp, bq, bk, topk, topp, alpha, scale)
+        return sa_permute_tokens(op, perm, inverse=True, out=out)
     if q.is_cuda:
         return _path_on_device(q, k, v, bq, bk, topk, topp, alpha, scale, out)
     B, H, N, d = _qkv(q, k, v)

@@ -582,6 +582,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
+      // with the blend, this half row of O_l is loaded before the wait for
+      // the last P V, so the wait hides the load
+      uint4 olv[D / 16];
+      if (a.alpha && store) {
+        const uint4* olp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.o_l) + orow_off);
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) olv[c] = __ldg(olp + c);
+      }
       const bool o_ok = mbar_wait(&bars[B_OFULL], qi & 1, abort_flag);
       uint32_t o0[32], o1[32];
       {
@@ -605,12 +613,11 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         uint4* dst = reinterpret_cast<uint4*>(orow);
         if (a.alpha) {
           // O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l with O_s = o / l not yet rounded
-          const uint4* olv = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.o_l) + orow_off);
           const float4* alv = reinterpret_cast<const float4*>(a.alpha + static_cast<long long>(it.bh % a.H) * D + half * (D / 2));
 #pragma unroll
           for (int c = 0; c < D / 16; ++c) {
             const uint32_t* oc = (c < 4) ? o0 + 8 * c : o1 + 8 * (c - 4);
-            const uint4 lv = __ldg(olv + c);
+            const uint4 lv = olv[c];
             const float4 a0 = __ldg(alv + 2 * c), a1 = __ldg(alv + 2 * c + 1);
             const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
             const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};

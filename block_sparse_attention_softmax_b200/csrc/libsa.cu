@@ -5,6 +5,9 @@
 #include "attn_kernel.cu"
 #include "linear_kernels.cu"
 #include "tile_kernels.cu"
+#include "permute_kernels.cu"
+#include "bwd_kernels.cu"
+#include "lin_bwd_kernels.cu"
 #include "sa_api.cu"
 #include "noalloc.cu"
 #include "diag.cu"

@@ -458,4 +458,102 @@ int sa_select_mask(const float* scores, int B, int H, int n_qb, int n_kb, double
   return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_select_mask");
 }
 
+int sa_tile_permutation(int H, int T, int Hh, int W, const int32_t* tiles, int32_t* perm, void* stream) {
+  if (H < 1 || H > kMaxPermHeads) return fail(SA_ERR_INVALID_ARG, "sa_tile_permutation: H = %d outside [1, %d]", H, kMaxPermHeads);
+  if (T < 1 || Hh < 1 || W < 1) return fail(SA_ERR_INVALID_ARG, "sa_tile_permutation: grid dimensions must be positive");
+  if (static_cast<long long>(T) * Hh * W * H >= (1LL << 31)) return fail(SA_ERR_UNSUPPORTED, "sa_tile_permutation: grid too large");
+  if (!tiles || !perm) return fail(SA_ERR_INVALID_ARG, "sa_tile_permutation: null pointer");
+  if (!aligned16(perm)) return fail(SA_ERR_ALIGN, "sa_tile_permutation: perm must be 16-byte aligned");
+  for (int h = 0; h < H; ++h)
+    if (tiles[3 * h] < 1 || tiles[3 * h + 1] < 1 || tiles[3 * h + 2] < 1)
+      return fail(SA_ERR_INVALID_ARG, "sa_tile_permutation: tile of head %d has a dimension below 1", h);
+  cudaError_t e = launch_tile_perm(H, T, Hh, W, tiles, perm, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_tile_permutation");
+}
+
+int sa_permute_tokens(const uint16_t* x, const int32_t* perm, int B, int H, int N, int d, int inverse,
+                      uint16_t* y, void* stream) {
+  int rc = check_shape(B, H, N, d, 64, 64);
+  if (rc) return rc;
+  if (!x || !perm || !y) return fail(SA_ERR_INVALID_ARG, "sa_permute_tokens: null pointer");
+  if (x == y) return fail(SA_ERR_INVALID_ARG, "sa_permute_tokens: y must not alias x");
+  if (!aligned16(x) || !aligned16(y) || !aligned16(perm))
+    return fail(SA_ERR_ALIGN, "sa_permute_tokens: pointers must be 16-byte aligned");
+  cudaError_t e = launch_permute_rows(x, perm, B * H, H, N, d, inverse ? 1 : 0, y, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_permute_tokens");
+}
+
+size_t sa_sparse_attn_bwd_workspace_size(int B, int H, int N, int d, int bq, int bk) {
+  if (check_shape(B, H, N, d, bq, bk)) return 0;
+  return bwd_ws_bytes(B * H, N, (N + bq - 1) / bq, (N + bk - 1) / bk);
+}
+
+int sa_sparse_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* o,
+                       const float* lse, const uint16_t* dout, int B, int H, int N, int d, int bq, int bk,
+                       const int32_t* kv_idx, const int32_t* kv_cnt, double scale, float* dq, float* dk,
+                       float* dv, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_shape(B, H, N, d, bq, bk);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !lse || !dout || !kv_idx || !kv_cnt || !dq || !dk || !dv)
+    return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_bwd: null pointer");
+  if (!isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "scale must be finite");
+  const void* ptrs[] = {q, k, v, o, lse, dout, kv_idx, kv_cnt, dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "sa_sparse_attn_bwd: pointers must be 16-byte aligned");
+  const int nqb = (N + bq - 1) / bq, nkb = (N + bk - 1) / bk;
+  const size_t need = bwd_ws_bytes(B * H, N, nqb, nkb);
+  if (!workspace || ws_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "sa_sparse_attn_bwd: workspace of %zu bytes needed", need);
+  if (scale <= 0.0) scale = 1.0 / sqrt(static_cast<double>(d));
+  BwdArgs a{q, k, v, dout, lse, nullptr, kv_idx, kv_cnt, nullptr, nullptr, dq, dk, dv,
+            B * H, N, bq, nqb, nkb, (nkb + 1) / 2, static_cast<float>(scale),
+            static_cast<float>(scale * 1.4426950408889634)};
+  cudaError_t e = launch_sparse_attn_bwd(a, d, o, workspace, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_sparse_attn_bwd");
+}
+
+size_t sa_linear_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d, 64, 64)) return 0;
+  return lin_bwd_ws_bytes(B * H, N, d);
+}
+
+int sa_linear_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* kv_state, const float* ksum,
+                  const uint16_t* dout_l, int B, int H, int N, int d, int accumulate, float* dq, float* dk, float* dv,
+                  void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_shape(B, H, N, d, 64, 64);
+  if (rc) return rc;
+  if (!q || !k || !v || !kv_state || !ksum || !dout_l || !dq || !dk || !dv)
+    return fail(SA_ERR_INVALID_ARG, "sa_linear_bwd: null pointer");
+  const void* ptrs[] = {q, k, v, kv_state, ksum, dout_l, dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "sa_linear_bwd: pointers must be 16-byte aligned");
+  const size_t need = lin_bwd_ws_bytes(B * H, N, d);
+  if (!workspace || ws_bytes < need) return fail(SA_ERR_WORKSPACE, "sa_linear_bwd: workspace of %zu bytes needed", need);
+  cudaError_t e = launch_linear_bwd(q, k, v, kv_state, ksum, dout_l, B * H, N, d, dq, dk, dv, accumulate ? 1 : 0,
+                                    workspace, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_linear_bwd");
+}
+
+size_t sa_blend_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d, 64, 64)) return 0;
+  return blend_bwd_ws_bytes(B * H, N, d);
+}
+
+int sa_blend_bwd(const uint16_t* o_s, const uint16_t* o_l, const float* alpha, const uint16_t* dout, int B, int H,
+                 int N, int d, uint16_t* do_s, uint16_t* do_l, float* dalpha, void* workspace, size_t ws_bytes,
+                 void* stream) {
+  int rc = check_shape(B, H, N, d, 64, 64);
+  if (rc) return rc;
+  if (!o_s || !o_l || !alpha || !dout || !do_s || !do_l || !dalpha)
+    return fail(SA_ERR_INVALID_ARG, "sa_blend_bwd: null pointer");
+  const void* ptrs[] = {o_s, o_l, alpha, dout, do_s, do_l, dalpha, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGN, "sa_blend_bwd: pointers must be 16-byte aligned");
+  const size_t need = blend_bwd_ws_bytes(B * H, N, d);
+  if (!workspace || ws_bytes < need) return fail(SA_ERR_WORKSPACE, "sa_blend_bwd: workspace of %zu bytes needed", need);
+  cudaError_t e = launch_blend_bwd(o_s, o_l, alpha, dout, B, H, N, d, do_s, do_l, dalpha, workspace,
+                                   static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_blend_bwd");
+}
+
 }  // extern "C"

@@ -105,6 +105,26 @@ cudaError_t launch_trip_pool(const void* x, int BH, int N, int d, int b, float* 
 cudaError_t launch_heat(const void* q, const void* k, int BH, int N, int d, int bq, const int* rows, int n_items,
                         double scale, float* heat, float* lse, cudaStream_t st);
 
+// Permuted token layouts: per-head tile-major permutations of a (T, Hh, W)
+// grid and the row gather / scatter.
+constexpr int kMaxPermHeads = 256;
+cudaError_t launch_tile_perm(int H, int T, int Hh, int W, const int* tiles, int* perm, cudaStream_t st);
+cudaError_t launch_permute_rows(const void* x, const int* perm, int BH, int H, int N, int d, int inverse, void* y,
+                                cudaStream_t st);
+
+// Backward pass of the sparse attention (declared with its argument block in
+// bwd_kernels.cu) and the linear branch and blend (linear_kernels.cu).
+struct BwdArgs;
+size_t bwd_ws_bytes(int BH, int N, int nqb, int nkb);
+cudaError_t launch_sparse_attn_bwd(const BwdArgs& a, int d, const void* o, void* ws, cudaStream_t st);
+size_t lin_bwd_ws_bytes(int BH, int N, int d);
+size_t blend_bwd_ws_bytes(int BH, int N, int d);
+cudaError_t launch_linear_bwd(const void* q, const void* k, const void* v, const float* S, const float* z,
+                              const void* dol, int BH, int N, int d, float* dq, float* dk, float* dv, int accumulate,
+                              void* ws, cudaStream_t st);
+cudaError_t launch_blend_bwd(const void* o_s, const void* o_l, const float* alpha, const void* dout, int B, int H,
+                             int N, int d, void* do_s, void* do_l, float* dalpha, void* ws, cudaStream_t st);
+
 // Driver entry point for cuTensorMapEncodeTiled, resolved once. 3-D maps
 // (inner, rows, planes), 128-byte swizzle, zero fill out of bounds.
 CUresult encode_tensor_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t inner,

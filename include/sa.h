@@ -164,6 +164,43 @@ int sa_blend(const uint16_t* o_s, const uint16_t* q, const float* kv_state, cons
              const float* alpha, int B, int H, int N, int d, uint16_t* o,
              void* workspace, size_t ws_bytes, void* stream);
 
+/* Backward pass ("SpargeAttention2" §2(2): the sparse attention is trainable and
+ * fine-tuned by distillation, which needs gradients through the sparse path;
+ * "SLA2" 提案手法 ③: the backward pass runs in full precision). Gradients are
+ * fp32 [B, H, N, d]; upstream gradients are bf16 like the forward's outputs.
+ *
+ * sa_sparse_attn_bwd: gradients of O_s = sa_sparse_attn_fwd(q, k, v, lists)
+ *   for dout = dL/dO_s, given the forward's o (O_s) and lse (its lse_opt):
+ *     D = rowsum(dout * o),  dS = P * (dout v^T - D) over the kept tiles,
+ *     dq = scale dS k,  dk = scale dS^T q,  dv = P^T dout,
+ *   with P recomputed from lse. dq, dk and dv are written (every element: rows
+ *   and keys that no kept tile reaches get zeros). The lists are the forward's
+ *   (kv_idx, kv_cnt); the key-block to query-block lists that dk and dv need
+ *   are built in the workspace (sa_sparse_attn_bwd_workspace_size()).
+ *   Deterministic: every sum is owned by one CTA, in a fixed order.
+ *
+ * sa_linear_bwd: gradients of O_l = phi(q) S / phi(q) . z (the linear branch,
+ *   kv_state = S and ksum = z from sa_linear_branch) for dout_l = dL/dO_l.
+ *   accumulate != 0 adds into dq, dk, dv (for example onto the sparse
+ *   attention's), else writes them. Deterministic (fixed-order partial sums).
+ *
+ * sa_blend_bwd: for O = alpha ⊙ o_s + (1 - alpha) ⊙ o_l and dout = dL/dO:
+ *   do_s = alpha ⊙ dout and do_l = (1 - alpha) ⊙ dout (bf16 [B, H, N, d]),
+ *   dalpha [H, d] fp32 = sum over batches and tokens of dout ⊙ (o_s - o_l). */
+size_t sa_sparse_attn_bwd_workspace_size(int B, int H, int N, int d, int bq, int bk);
+int sa_sparse_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* o,
+                       const float* lse, const uint16_t* dout, int B, int H, int N, int d, int bq, int bk,
+                       const int32_t* kv_idx, const int32_t* kv_cnt, double scale, float* dq, float* dk,
+                       float* dv, void* workspace, size_t ws_bytes, void* stream);
+size_t sa_linear_bwd_workspace_size(int B, int H, int N, int d);
+int sa_linear_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* kv_state,
+                  const float* ksum, const uint16_t* dout_l, int B, int H, int N, int d, int accumulate,
+                  float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes, void* stream);
+size_t sa_blend_bwd_workspace_size(int B, int H, int N, int d);
+int sa_blend_bwd(const uint16_t* o_s, const uint16_t* o_l, const float* alpha, const uint16_t* dout,
+                 int B, int H, int N, int d, uint16_t* do_s, uint16_t* do_l, float* dalpha,
+                 void* workspace, size_t ws_bytes, void* stream);
+
 /* Tile scoring from the full attention map ("Veda" §2.1 and §2.3).
  *
  * sa_trip_pool: TripPool descriptors of every query block (bq tokens) and key
@@ -199,6 +236,28 @@ int sa_tile_heatmap(const uint16_t* q, const uint16_t* k, int B, int H, int N, i
                     void* stream);
 int sa_select_mask(const float* scores, int B, int H, int n_qb, int n_kb, double topk_frac, double topp,
                    int32_t* kv_idx, int32_t* kv_cnt, uint8_t* mask_opt, void* stream);
+
+/* Permuted token layouts ("Veda" §2.2: a tiling (p_t, p_h, p_w) of the latent
+ * grid chosen per head; "SparsePR" §2C: tokens reordered into a contiguous
+ * group-major layout before the block-sparse call). The sparse path runs
+ * unchanged on the permuted sequence, whose blocks are runs of consecutive
+ * permuted tokens; the output is scattered back. Where a grid dimension is not
+ * a multiple of the tile's, the edge tiles are partial and a block may span
+ * two tiles.
+ *
+ * sa_tile_permutation: perm [H, N] int32 (device), N = T * Hh * W, for tokens
+ *   flattened in raster order t-major over the (T, Hh, W) grid: perm[h, i] is
+ *   the raster index of the token at position i of head h's order, which
+ *   visits the tiles of tiles[3 h .. 3 h + 2] = (p_t, p_h, p_w) (a host array
+ *   of H triples, each >= 1) in raster order of the tile grid and the tokens of
+ *   a tile in raster order. 1 <= H <= 256.
+ * sa_permute_tokens: rows of x [B, H, N, d] bf16 gathered into y in head h's
+ *   order, y[b, h, i] = x[b, h, perm[h, i]] (inverse = 0), or scattered back,
+ *   y[b, h, perm[h, i]] = x[b, h, i] (inverse = 1). perm must be a permutation
+ *   of 0..N-1 for each head (it is not checked); y must not alias x. */
+int sa_tile_permutation(int H, int T, int Hh, int W, const int32_t* tiles, int32_t* perm, void* stream);
+int sa_permute_tokens(const uint16_t* x, const int32_t* perm, int B, int H, int N, int d, int inverse,
+                      uint16_t* y, void* stream);
 
 /* Mask builder that allocates nothing (no counterpart in the pages: it exists
  * for callers, not for the method). Some callers may not allocate device memory

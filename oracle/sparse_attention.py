@@ -328,3 +328,108 @@ def mask_from_scores(s: np.ndarray, k_frac: float, p: float) -> np.ndarray:
     for r in range(s.shape[0]):
         mask[r] = hybrid_row(s[r], k_frac, p)[0]
     return mask
+
+
+# --------------------------------------------------------------------------
+# Permuted token layouts (Veda §2.2: per-head tilings (p_t, p_h, p_w) of the
+# latent grid; SparsePR §2C: tokens reordered into a contiguous group-major
+# layout before the block-sparse call). Blocks of the sparse path are then
+# runs of consecutive tokens of the permuted sequence.
+# --------------------------------------------------------------------------
+
+def tile_permutation(grid, tile) -> np.ndarray:
+    """Token order that visits the (T, Hh, W) raster grid tile by tile: tiles
+    of (p_t, p_h, p_w) tokens in raster order of the tile grid (edge tiles
+    may be partial), tokens inside a tile in raster order. perm[i] is the
+    raster index of the token placed at position i."""
+    T, Hh, W = grid
+    pt, ph, pw = tile
+    perm = []
+    for t0 in range(0, T, pt):
+        for y0 in range(0, Hh, ph):
+            for x0 in range(0, W, pw):
+                for t in range(t0, min(T, t0 + pt)):
+                    for y in range(y0, min(Hh, y0 + ph)):
+                        for x in range(x0, min(W, x0 + pw)):
+                            perm.append((t * Hh + y) * W + x)
+    return np.asarray(perm, dtype=np.int64)
+
+
+def permute_rows(x: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """Rows of x in the permuted order: y[i] = x[perm[i]]."""
+    return x[perm]
+
+
+def unpermute_rows(y: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """Inverse of permute_rows: x[perm[i]] = y[i]."""
+    x = np.empty_like(y)
+    x[perm] = y
+    return x
+
+
+# --------------------------------------------------------------------------
+# Backward pass (SpargeAttention2 §2(2): the sparse attention is made
+# trainable and fine-tuned by distillation, which needs gradients through the
+# sparse path; SLA2 提案手法 ③: the backward pass runs in full precision).
+# Gradients of the forward definitions above by the chain rule.
+# --------------------------------------------------------------------------
+
+def masked_attention_bwd(q, k, v, mask, bq, bk, dout, scale=None):
+    """(dq, dk, dv) of O = masked_attention(q, k, v, mask) for the upstream
+    gradient dout [N, d]. Per query block, with P the softmax of
+    scale * q_i . k_j over the kept keys and O = P v:
+        dv += P^T dout,  dP = dout v^T,  dS = P * (dP - rowsum(dout * O)),
+        dq += scale * dS k,  dk += scale * dS^T q.
+    Rows with no kept key have O = 0 and pass no gradient."""
+    N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for qb in range(mask.shape[0]):
+        rows = np.arange(qb * bq, min(N, (qb + 1) * bq))
+        kept = np.nonzero(mask[qb])[0]
+        if kept.shape[0] == 0:
+            continue
+        keys = np.concatenate([np.arange(kb * bk, min(N, (kb + 1) * bk)) for kb in kept])
+        logits = scale * (q[rows] @ k[keys].T)
+        w = np.exp(logits - logits.max(axis=1, keepdims=True))
+        P = w / w.sum(axis=1, keepdims=True)
+        O = P @ v[keys]
+        dP = dout[rows] @ v[keys].T
+        dS = P * (dP - (dout[rows] * O).sum(axis=1, keepdims=True))
+        dq[rows] += scale * (dS @ k[keys])
+        dk[keys] += scale * (dS.T @ q[rows])          # keys of one row are distinct
+        dv[keys] += P.T @ dout[rows]
+    return dq, dk, dv
+
+
+def phi_grad(x: np.ndarray) -> np.ndarray:
+    """d phi / dx for phi = elu + 1: 1 above zero, e^x at or below."""
+    return np.where(x > 0, 1.0, np.exp(np.minimum(x, 0.0)))
+
+
+def linear_bwd(q, k, v, dout_l):
+    """(dq, dk, dv) of O_l = phi(q) S / phi(q) . z with S = sum_j phi(k_j) v_j^T
+    and z = sum_j phi(k_j), for the upstream gradient dout_l [N, d]:
+        dnum = dout_l / den,  dden = -rowsum(dout_l * O_l) / den,
+        dphi(q) = dnum S^T + dden z^T,  dS = phi(q)^T dnum,  dz = phi(q)^T dden,
+        dphi(k) = v dS^T + dz,  dv = phi(k) dS,
+    then dq = dphi(q) * phi'(q) and dk = dphi(k) * phi'(k)."""
+    fq, fk = phi(q), phi(k)
+    S, z = fk.T @ v, fk.sum(axis=0)
+    den = fq @ z
+    O = (fq @ S) / den[:, None]
+    dnum = dout_l / den[:, None]
+    dden = -(dout_l * O).sum(axis=1) / den
+    dfq = dnum @ S.T + dden[:, None] * z[None, :]
+    dS = fq.T @ dnum
+    dz = fq.T @ dden
+    dfk = v @ dS.T + dz[None, :]
+    dv = fk @ dS
+    return dfq * phi_grad(q), dfk * phi_grad(k), dv
+
+
+def blend_bwd(o_s, o_l, alpha_h, dout):
+    """(do_s, do_l, dalpha) of O = alpha * O_s + (1 - alpha) * O_l: alpha * dout,
+    (1 - alpha) * dout, and the sum over tokens of dout * (O_s - O_l)."""
+    return alpha_h[None, :] * dout, (1.0 - alpha_h[None, :]) * dout, (dout * (o_s - o_l)).sum(axis=0)

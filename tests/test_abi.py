@@ -118,3 +118,15 @@ def test_diagnostic_entry_points_validate_before_launch(lib):
     assert lib.sa_diag_exp2(None, fake, fake, 8, None) == -1
     assert lib.sa_diag_exp2(None, None, None, 0, None) == 0      # nothing to do, nothing launched
     assert lib.sa_diag_wait_timeout(None, None) == -1
+
+
+def test_permutation_entry_points_validate_before_launch(lib):
+    fake = P(0x1000)
+    tiles = (ctypes.c_int32 * 3)(1, 2, 0)
+    assert lib.sa_tile_permutation(1, 4, 4, 4, ctypes.cast(tiles, P), fake, None) == -1   # tile dimension 0
+    assert lib.sa_tile_permutation(0, 4, 4, 4, ctypes.cast(tiles, P), fake, None) == -1   # no heads
+    assert lib.sa_tile_permutation(300, 4, 4, 4, ctypes.cast(tiles, P), fake, None) == -1
+    assert lib.sa_permute_tokens(fake, fake, 1, 1, 64, 64, 0, fake, None) == -1           # y aliases x
+    assert lib.sa_permute_tokens(fake, fake, 1, 1, 64, 96, 0, P(0x2000), None) == -2
+    assert lib.sa_select_mask(fake, 1, 1, 4, 20000, 0.1, 0.9, fake, fake, None, None) == -2
+    assert lib.sa_tile_heatmap(fake, fake, 1, 1, 128, 64, 64, 64, 0.0, fake, -1, fake, None, None) == -1

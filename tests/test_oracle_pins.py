@@ -460,3 +460,112 @@ def test_mask_from_scores_is_the_hybrid_rule_per_row():
     q, k = rng.standard_normal((300, 8)) * 2, rng.standard_normal((300, 8))
     out = oracle.build_mask(q, k, 32, 16, 0.2, 0.8)
     assert (oracle.mask_from_scores(out["s"], 0.2, 0.8) == out["mask"]).all()
+
+
+# ---------------------------------------------------------------- permuted layouts (Veda §2.2, SparsePR §2C)
+@pytest.mark.parametrize("grid,tile", [((3, 4, 6), (1, 2, 3)), ((5, 7, 9), (2, 4, 4)), ((2, 8, 8), (1, 8, 8))])
+def test_tile_permutation_by_coordinates(grid, tile):
+    """A bijection of the raster tokens in which each tile's tokens are
+    consecutive, tiles follow the tile grid's raster order, and tokens inside a
+    tile follow the raster order; checked from each token's coordinates."""
+    T, Hh, W = grid
+    perm = oracle.tile_permutation(grid, tile)
+    N = T * Hh * W
+    assert sorted(perm.tolist()) == list(range(N))
+    coords = [(r // (Hh * W), (r // W) % Hh, r % W) for r in perm.tolist()]
+    tiles = [(t // tile[0], y // tile[1], x // tile[2]) for t, y, x in coords]
+    nt = (-(-T // tile[0]), -(-Hh // tile[1]), -(-W // tile[2]))
+    tile_rank = [(a * nt[1] + b) * nt[2] + c for a, b, c in tiles]
+    assert tile_rank == sorted(tile_rank)                      # tiles contiguous, in raster order
+    for i in range(1, N):
+        if tile_rank[i] == tile_rank[i - 1]:
+            assert perm[i] > perm[i - 1]                       # raster order inside a tile
+    if all(g % p == 0 for g, p in zip(grid, tile)):            # full tiles: fixed-size runs
+        size = tile[0] * tile[1] * tile[2]
+        assert all(tile_rank[i] == i // size for i in range(N))
+
+
+def test_permuted_dense_attention_is_equivariant():
+    """Dense attention commutes with a permutation of the tokens (softmax over
+    all keys), so un-permuting the permuted call's output gives the plain one."""
+    rng = _rng(44)
+    grid = (2, 3, 5)
+    N, d = 30, 6
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    perm = oracle.tile_permutation(grid, (1, 2, 2))
+    op, _ = oracle.dense_attention(oracle.permute_rows(q, perm), oracle.permute_rows(k, perm),
+                                   oracle.permute_rows(v, perm))
+    o, _ = oracle.dense_attention(q, k, v)
+    assert np.abs(oracle.unpermute_rows(op, perm) - o).max() < 1e-12
+    assert np.array_equal(oracle.unpermute_rows(oracle.permute_rows(q, perm), perm), q)
+
+
+# ---------------------------------------------------------------- backward pass
+def test_masked_attention_bwd_against_torch_autograd_of_sdpa():
+    """The oracle's hand-derived gradients against float64 torch.autograd through
+    scaled_dot_product_attention with the expanded token mask (ragged blocks,
+    bq != bk; every query row keeps at least one block)."""
+    rng = _rng(51)
+    N, d, bq, bk = 70, 8, 16, 8
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    q *= 2.0
+    mask = rng.random((-(-N // bq), -(-N // bk))) < 0.4
+    mask[np.arange(mask.shape[0]), rng.integers(0, mask.shape[1], mask.shape[0])] = True
+    dout = rng.standard_normal((N, d))
+    tok = np.zeros((N, N), dtype=bool)
+    for i in range(N):
+        for j in range(N):
+            tok[i, j] = mask[i // bq, j // bk]
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(tq[None, None], tk[None, None], tv[None, None],
+                                                         attn_mask=torch.from_numpy(tok)[None, None])[0, 0]
+    o.backward(torch.from_numpy(dout))
+    dq, dk, dv = oracle.masked_attention_bwd(q, k, v, mask, bq, bk, dout)
+    for got, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.abs(got - ref.numpy()).max() < 1e-10
+
+
+def test_masked_attention_bwd_empty_rows_pass_no_gradient():
+    rng = _rng(52)
+    N, d = 40, 4
+    q, k, v, dout = (rng.standard_normal((N, d)) for _ in range(4))
+    mask = np.ones((3, 5), dtype=bool)
+    mask[1] = False
+    dq, dk, dv = oracle.masked_attention_bwd(q, k, v, mask, 16, 8, dout)
+    assert (dq[16:32] == 0).all()
+    dout2 = dout.copy()
+    dout2[16:32] = 123.0                     # the empty rows' upstream gradient changes nothing
+    _, dk2, dv2 = oracle.masked_attention_bwd(q, k, v, mask, 16, 8, dout2)
+    assert np.array_equal(dk, dk2) and np.array_equal(dv, dv2)
+
+
+def _central_diff(f, x, h=1e-6):
+    g = np.zeros_like(x)
+    for idx in np.ndindex(x.shape):
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += h
+        xm[idx] -= h
+        g[idx] = (f(xp) - f(xm)) / (2 * h)
+    return g
+
+
+def test_linear_and_blend_bwd_by_finite_differences():
+    """Linear-branch and blend gradients against central differences of the
+    oracle's forward (a scalar loss <dout, O>), on inputs that straddle zero."""
+    rng = _rng(53)
+    N, d = 9, 4
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    dout = rng.standard_normal((N, d))
+    dq, dk, dv = oracle.linear_bwd(q, k, v, dout)
+    loss = lambda q_, k_, v_: float((dout * oracle.linear_out(q_, *oracle.linear_state(k_, v_))).sum())
+    assert np.abs(dq - _central_diff(lambda x: loss(x, k, v), q)).max() < 1e-6
+    assert np.abs(dk - _central_diff(lambda x: loss(q, x, v), k)).max() < 1e-6
+    assert np.abs(dv - _central_diff(lambda x: loss(q, k, x), v)).max() < 1e-6
+    o_s, o_l, al = rng.standard_normal((N, d)), rng.standard_normal((N, d)), rng.random(d)
+    ds, dl, da = oracle.blend_bwd(o_s, o_l, al, dout)
+    bl = lambda a_, s_, l_: float((dout * oracle.blend(s_, l_, a_)).sum())
+    assert np.abs(da - _central_diff(lambda x: bl(x, o_s, o_l), al)).max() < 1e-6
+    assert np.abs(ds - _central_diff(lambda x: bl(al, x, o_l), o_s)).max() < 1e-6
+    assert np.abs(dl - _central_diff(lambda x: bl(al, o_s, x), o_l)).max() < 1e-6
+    x = np.linspace(-3, 3, 61)
+    assert np.abs(oracle.phi_grad(x) - _central_diff(lambda t: oracle.phi(t).sum(), x)).max() < 1e-6
