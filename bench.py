@@ -40,9 +40,9 @@ METRIC = "sparse_attn_effective_tflops"
 # kernel's DRAM traffic is Q, K, V and O sized). `sources_sha` pins the kernel sources the counters belong to:
 # once they change, traffic is reported as null until a new capture is made.
 ATTN_TRAFFIC_CAPTURE = {
-    "workload": "wan13b_480p", "dram_bytes_read": 302803968, "dram_bytes_write": 83264256,
-    "sources_sha": "d3dbd3485535a770",
-    "sources": ("attn_kernel.cu", "sa_device.cuh", "sa_internal.h"),
+    "workload": "wan13b_480p", "dram_bytes_read": 302507008, "dram_bytes_write": 82581760,
+    "sources_sha": "02bd3a6c1943bcd8",
+    "sources": ("attn_kernel.cu", "sa_device.cuh"),
 }
 
 
@@ -411,6 +411,79 @@ def run_ours(args, wl, rank, world, local):
 PER_WORKLOAD = ("tiny", "wan13b_480p", "sink_skew", "long_245k")
 
 
+def _times(fn, calls=5, warmup=2):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = []
+    for _ in range(calls):
+        e0 = _event()
+        fn()
+        ev.append((e0, _event()))
+    torch.cuda.synchronize()
+    return stats([x.elapsed_time(y) for x, y in ev])
+
+
+def measure_backward(sa, wl, dev):
+    """The backward of one step on the workload: the sparse attention's dq, dk,
+    dv over the step's lists, and with the linear branch its gradients and the
+    blend's. Algorithmic flops of the sparse backward: 7 products per kept tile
+    (S and dP recomputed for dq and for dk/dv, then dq, dk, dv), 3.5 x the
+    forward's 2."""
+    x = make_inputs(wl, dev)
+    q, k, v, alpha = x["q"], x["k"], x["v"], x["alpha"]
+    m = sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp)
+    o, lse = sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"], want_lse=True)
+    dout = torch.randn(q.shape, generator=torch.Generator(device=dev).manual_seed(5), device=dev).to(torch.bfloat16)
+    ex = executed_flops(wl, m["kv_idx"], m["kv_cnt"])
+    res = {"sparse_attn_bwd_ms": _times(lambda: sa.sa_sparse_attn_bwd(q, k, v, o, lse, dout, wl.bq, wl.bk,
+                                                                       m["kv_idx"], m["kv_cnt"]))}
+    hbm, bf16, _, src = peaks()
+    tf = 3.5 * ex / (res["sparse_attn_bwd_ms"]["median"] * 1e-3) / 1e12
+    res.update({"sparse_attn_bwd_exec_tflops": round(tf, 1), "sparse_attn_bwd_frac_of_bf16_peak": round(tf / bf16, 4),
+                "flops_note": "3.5 x the forward's executed flops (7 tile products: S, dP twice, dq, dk, dv)"})
+    if wl.linear:
+        S, z, o_l = sa.sa_linear_branch(q, k, v, want_ol=True)
+        res["linear_bwd_ms"] = _times(lambda: sa.sa_linear_bwd(q, k, v, S, z, dout))
+        res["blend_bwd_ms"] = _times(lambda: sa.sa_blend_bwd(o, o_l, alpha, dout))
+    sa.sa_device_status(dev)
+    del x, q, k, v, o, lse, dout, m
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_tile_scoring_and_layouts(sa, dev):
+    """Veda's max-pooled heatmap (two tensor-core sweeps of Q K^T over every
+    tile: 4 N^2 d flops per head) on the 1.3B-480p shape, all query blocks and
+    a 1/8 sample; and the sparse path on per-head 3-D tilings of its latent
+    grid (gather, mask, attention, scatter) against the raster order."""
+    wl = WORKLOADS["wan13b_480p"]
+    x = make_inputs(wl, dev)
+    q, k, v = x["q"], x["k"], x["v"]
+    hbm, bf16, _, src = peaks()
+    heat = torch.empty(wl.B, wl.H, wl.n_qb, wl.n_kb, dtype=torch.float32, device=dev)
+    full = _times(lambda: sa.sa_tile_heatmap(q, k, wl.bq, out=heat), calls=3)
+    fl = 4.0 * wl.B * wl.H * wl.N * wl.N * wl.d
+    rows = torch.arange(0, wl.B * wl.H * wl.n_qb, 8, dtype=torch.int32, device=dev)
+    part = _times(lambda: sa.sa_tile_heatmap(q, k, wl.bq, rows=rows, out=heat), calls=3)
+    tiles = [(1, 2, 32), (3, 5, 4), (1, 1, 64), (3, 2, 8)] * (wl.H // 4)
+    perm = sa.sa_tile_permutation(wl.grid, tiles)
+    raster = _times(lambda: sa.block_sparse_attention(q, k, v, wl.bq, wl.bk, wl.topk, wl.topp), calls=5)
+    permuted = _times(lambda: sa.block_sparse_attention(q, k, v, wl.bq, wl.bk, wl.topk, wl.topp, perm=perm), calls=5)
+    qp, kp = sa.sa_permute_tokens(q, perm), sa.sa_permute_tokens(k, perm)
+    dens = float(sa.sa_build_mask(qp, kp, wl.bq, wl.bk, wl.topk, wl.topp)["kv_cnt"].sum()) / (wl.H * wl.n_qb * wl.n_kb)
+    sa.sa_device_status(dev)
+    del x, q, k, v, heat, qp, kp
+    torch.cuda.empty_cache()
+    return {"workload": wl.name,
+            "tile_heatmap_ms": full, "tile_heatmap_tflops": round(fl / (full["median"] * 1e-3) / 1e12, 1),
+            "tile_heatmap_frac_of_bf16_peak": round(fl / (full["median"] * 1e-3) / 1e12 / bf16, 4),
+            "tile_heatmap_sampled_1_in_8_ms": part,
+            "path_raster_ms": raster, "path_per_head_tilings_ms": permuted,
+            "tilings": "per head, cycling (1,2,32), (3,5,4), (1,1,64), (3,2,8) over the 21x30x52 grid",
+            "density_per_head_tilings": round(dens, 5)}
+
+
 def measure_workload(sa, wl, dev, calls, warmup, dense_reps, flush):
     """One workload's step components, each call timed on its own with CUDA
     events (an L2 flush between calls when the inputs fit in L2), with its own
@@ -600,7 +673,11 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     res = run_ours(args, wl, rank, world, local)
     if world == 1 and not args.no_per_workload:
-        res["per_workload"] = run_per_workload(args, torch.device("cuda", local))
+        import block_sparse_attention_softmax_b200 as sa
+        dev = torch.device("cuda", local)
+        res["backward"] = measure_backward(sa, wl, dev)
+        res["tile_scoring_and_layouts"] = measure_tile_scoring_and_layouts(sa, dev)
+        res["per_workload"] = run_per_workload(args, dev)
     if rank == 0:
         if not args.no_cpu_baseline:
             x = _head_inputs(wl, BASELINE_HEADS)

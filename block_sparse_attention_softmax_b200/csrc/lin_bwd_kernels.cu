@@ -37,11 +37,12 @@ __global__ void __launch_bounds__(linb::kWarps * 32) lin_q_kernel(
     float* __restrict__ dnum, float* __restrict__ dden) {
   constexpr int J = D / 32;
   extern __shared__ float sm[];
-  float* sS = sm;                        // [D][D]
-  float* sz = sS + D * D;                // [D]
+  constexpr int LD = D + 1;              // padded row stride: row and column walks are both conflict-free
+  float* sS = sm;                        // [D][LD]
+  float* sz = sS + D * LD;               // [D]
   float* sv = sz + D;                    // [kWarps][2][D] per-warp vectors
   const int bh = blockIdx.y;
-  for (int i = threadIdx.x; i < D * D; i += blockDim.x) sS[i] = S[static_cast<long long>(bh) * D * D + i];
+  for (int i = threadIdx.x; i < D * D; i += blockDim.x) sS[(i / D) * LD + i % D] = S[static_cast<long long>(bh) * D * D + i];
   for (int i = threadIdx.x; i < D; i += blockDim.x) sz[i] = z[static_cast<long long>(bh) * D + i];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -70,7 +71,7 @@ __global__ void __launch_bounds__(linb::kWarps * 32) lin_q_kernel(
     for (int aa = 0; aa < D; ++aa) {
       const float f = fqv[aa];
 #pragma unroll
-      for (int j = 0; j < J; ++j) num[j] = fmaf(f, sS[aa * D + lane + 32 * j], num[j]);
+      for (int j = 0; j < J; ++j) num[j] = fmaf(f, sS[aa * LD + lane + 32 * j], num[j]);
     }
     const float inv = 1.f / den;
     float dot = 0.f;
@@ -93,7 +94,7 @@ __global__ void __launch_bounds__(linb::kWarps * 32) lin_q_kernel(
     for (int j = 0; j < J; ++j) {
       const int aa = lane + 32 * j;
       float acc = dd * sz[aa];
-      for (int c = 0; c < D; ++c) acc = fmaf(sS[aa * D + c], dnv[c], acc);
+      for (int c = 0; c < D; ++c) acc = fmaf(sS[aa * LD + c], dnv[c], acc);
       const float g = acc * phi_grad_f(qx[j]);
       dq[r * D + aa] = accumulate ? dq[r * D + aa] + g : g;
     }
@@ -160,12 +161,14 @@ __global__ void __launch_bounds__(linb::kWarps * 32) lin_k_kernel(
     int N, int tok_per_cta, float* __restrict__ dk, float* __restrict__ dv, int accumulate) {
   constexpr int J = D / 32;
   extern __shared__ float sm[];
-  float* sS = sm;                         // dS [D][D]
-  float* sz = sS + D * D;                 // dz [D]
+  constexpr int LD = D + 1;               // padded row stride, as in lin_q_kernel
+  float* sS = sm;                         // dS [D][LD]
+  float* sz = sS + D * LD;                // dz [D]
   float* sv = sz + D;                     // [kWarps][2][D]
   const int bh = blockIdx.y;
   const float* src = dsz + static_cast<long long>(bh) * (D * D + D);
-  for (int i = threadIdx.x; i < D * D + D; i += blockDim.x) sm[i] = src[i];
+  for (int i = threadIdx.x; i < D * D; i += blockDim.x) sS[(i / D) * LD + i % D] = src[i];
+  for (int i = threadIdx.x; i < D; i += blockDim.x) sz[i] = src[D * D + i];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* vv = sv + warp * 2 * D;
@@ -187,8 +190,8 @@ __global__ void __launch_bounds__(linb::kWarps * 32) lin_k_kernel(
       const int aa = lane + 32 * j;
       float gk = sz[aa], gv = 0.f;
       for (int c = 0; c < D; ++c) {
-        gk = fmaf(sS[aa * D + c], vv[c], gk);       // (dS v)[a]
-        gv = fmaf(fk[c], sS[c * D + aa], gv);       // (phi(k)^T dS)[a]
+        gk = fmaf(sS[aa * LD + c], vv[c], gk);      // (dS v)[a]
+        gv = fmaf(fk[c], sS[c * LD + aa], gv);      // (phi(k)^T dS)[a]
       }
       gk *= phi_grad_f(kx[j]);
       dk[r * D + aa] = accumulate ? dk[r * D + aa] + gk : gk;
@@ -254,7 +257,7 @@ static cudaError_t launch_lin_bwd_d(const void* q, const void* k, const void* v,
   float* dden = reinterpret_cast<float*>(ws + up(static_cast<long long>(BH) * N * D * 4));
   float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(dden) + up(static_cast<long long>(BH) * N * 4));
   float* dsz = reinterpret_cast<float*>(reinterpret_cast<char*>(part) + up(static_cast<long long>(BH) * nch * (D * D + D) * 4));
-  const size_t smem = (D * D + D + linb::kWarps * 2 * D) * 4;
+  const size_t smem = (D * (D + 1) + D + linb::kWarps * 2 * D) * 4;
   cudaError_t e = cudaFuncSetAttribute(lin_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(lin_k_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))) != cudaSuccess) return e;
