@@ -10,7 +10,8 @@ Pages followed (titles and sections):
     §2(2) trainable sparse attention (hence the backward pass), §2(3)
     block-sparse FlashAttention that skips masked tiles.
   * "SLA2" (ai-papers.net), 提案手法 ① mean pooling of queries and keys before
-    scoring, ② O = alpha * O_s + (1 - alpha) * O_l.
+    scoring, ② O = alpha * O_s + (1 - alpha) * O_l, ③ a low-bit forward
+    (queries, keys and values quantised) with a full-precision backward.
   * "SALAD", §2.1 a linear-attention branch in parallel with sparse attention.
   * "Veda", §2.1 TripPool descriptors and the reference mask from max-pooling
     the full attention map over tiles, §2.2 per-head tilings of the latent
@@ -26,5 +27,5 @@ from .sparse_attention import (  # noqa: F401
     masked_attention, dense_attention, phi, linear_state, linear_out, blend,
     row_threshold_info, NEAR_TIE_TOL, trip_pool, full_attention_lse, tile_max_heatmap,
     mask_from_scores, tile_permutation, permute_rows, unpermute_rows, masked_attention_bwd,
-    phi_grad, linear_bwd, blend_bwd,
+    phi_grad, linear_bwd, blend_bwd, E4M3_MAX, e4m3_round, quantize_fp8_head, fp8_masked_attention,
 )

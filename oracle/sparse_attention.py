@@ -10,7 +10,10 @@ than itself: brute force on tiny inputs, closed forms, exhaustive subset search
 for Top-p minimality, the Top-p count from the low end of the order, and
 torch's float64 scaled_dot_product_attention for dense and masked attention.
 row_threshold_info, which the GPU comparison uses to recognise near-ties, is
-pinned with planted rows in tests/test_mask_comparator.py.
+pinned with planted rows in tests/test_mask_comparator.py. The E4M3 rounding
+of the low-bit forward is pinned by the format's own table of values (fixed
+points, ties to even, saturation) and by torch's float8_e4m3fn cast; the
+low-bit attention by inputs that quantise exactly.
 """
 from __future__ import annotations
 
@@ -433,3 +436,60 @@ def blend_bwd(o_s, o_l, alpha_h, dout):
     """(do_s, do_l, dalpha) of O = alpha * O_s + (1 - alpha) * O_l: alpha * dout,
     (1 - alpha) * dout, and the sum over tokens of dout * (O_s - O_l)."""
     return alpha_h[None, :] * dout, (1.0 - alpha_h[None, :]) * dout, (dout * (o_s - o_l)).sum(axis=0)
+
+
+# --------------------------------------------------------------------------
+# Low-bit forward (SLA2 提案手法 ③: the forward pass quantises queries, keys
+# and values to a low-bit format and computes with them; the backward stays in
+# full precision). The pages name neither the format nor the scale granularity.
+# Reading: 8-bit floats in the E4M3 layout (1 sign bit, 4 exponent bits with
+# bias 7, 3 mantissa bits, no infinities, largest finite value 448), one fp32
+# scale per (batch, head) and tensor, s = amax / 448, codes = E4M3(x / s) with
+# the division in fp32 and round-to-nearest-even with saturation at +-448. The
+# low-bit attention is then the masked attention above on the dequantised
+# tensors codes * s.
+# --------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Nearest E4M3 value (ties to even mantissa), saturated to +-448.
+
+    Normal numbers 2^e * 1.mmm for e in [-6, 8] are spaced 2^(e-3) apart;
+    below 2^-6 the subnormals m/8 * 2^-6 are spaced 2^-9 apart, and zero keeps
+    its sign. NaN stays NaN.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, ex = np.frexp(a)                      # a = f * 2^ex with f in [0.5, 1)
+    e = np.maximum(ex - 1, -6)               # binade exponent, clamped to the subnormal range
+    quantum = np.ldexp(1.0, e - 3)
+    r = np.round(a / quantum) * quantum      # np.round: ties to even
+    r = np.minimum(r, E4M3_MAX)
+    return np.where(np.isnan(x), np.nan, np.copysign(r, x))
+
+
+def quantize_fp8_head(x) -> tuple[np.ndarray, float]:
+    """One (batch, head) slice [N, d] -> (E4M3 code values as float64, fp32 scale).
+
+    s = amax / 448 in fp32 (1 when the slice is all zeros); each code is the
+    E4M3 rounding of the fp32 quotient x / s.
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.float32(np.max(np.abs(x32))) if x32.size else np.float32(0)
+    s = np.float32(amax) / np.float32(E4M3_MAX) if amax > 0 else np.float32(1.0)
+    codes = e4m3_round((x32 / s).astype(np.float64))
+    return codes, float(s)
+
+
+def fp8_masked_attention(q, k, v, mask, bq, bk, scale=None, rows=None):
+    """Masked attention on the per-head E4M3 quantisations of q, k and v.
+
+    Returns (O, LSE) as masked_attention does, computed in fp64 from the
+    dequantised tensors codes * s.
+    """
+    qc, sq = quantize_fp8_head(q)
+    kc, sk = quantize_fp8_head(k)
+    vc, sv = quantize_fp8_head(v)
+    return masked_attention(qc * sq, kc * sk, vc * sv, mask, bq, bk, scale=scale, rows=rows)

@@ -569,3 +569,89 @@ def test_linear_and_blend_bwd_by_finite_differences():
     assert np.abs(dl - _central_diff(lambda x: bl(al, o_s, x), o_l)).max() < 1e-6
     x = np.linspace(-3, 3, 61)
     assert np.abs(oracle.phi_grad(x) - _central_diff(lambda t: oracle.phi(t).sum(), x)).max() < 1e-6
+
+
+# ---------------------------------------------------------------- low-bit forward
+def _e4m3_table():
+    """Every finite non-negative E4M3 value, from the format's fields: exponent
+    field E (bias 7, E = 0 subnormal), mantissa field M; E = 15, M = 7 is NaN."""
+    vals = {}
+    for E in range(16):
+        for M in range(8):
+            if E == 15 and M == 7:
+                continue
+            v = (M / 8) * 2.0 ** -6 if E == 0 else (1 + M / 8) * 2.0 ** (E - 7)
+            vals[v] = M
+    return sorted(vals.items())
+
+
+def test_e4m3_fixed_points_and_ties_to_even():
+    table = _e4m3_table()
+    assert len(table) == 127 and table[-1][0] == 448.0 and table[1][0] == 2.0 ** -9
+    vals = np.array([v for v, _ in table])
+    assert np.array_equal(oracle.e4m3_round(vals), vals)
+    assert np.array_equal(oracle.e4m3_round(-vals[1:]), -vals[1:])
+    for (a, ma), (b, mb) in zip(table[:-1], table[1:]):
+        mid = (a + b) / 2
+        want = a if ma % 2 == 0 else b              # exactly one neighbour has an even mantissa
+        assert oracle.e4m3_round(mid) == want, (a, b)
+        assert oracle.e4m3_round(np.nextafter(mid, 0)) == a
+        assert oracle.e4m3_round(np.nextafter(mid, np.inf)) == b
+    assert oracle.e4m3_round(449.0) == 448.0 and oracle.e4m3_round(1e9) == 448.0
+    assert oracle.e4m3_round(-1e9) == -448.0 and np.isnan(oracle.e4m3_round(np.nan))
+
+
+def test_e4m3_matches_torch_float8_conversion():
+    """torch's float32 -> float8_e4m3fn cast (a library routine) below its
+    overflow threshold, over random magnitudes from the subnormals up."""
+    rng = _rng(60)
+    mag = np.exp2(rng.uniform(-12, 8.85, 200000))
+    x = (mag * rng.choice([-1.0, 1.0], mag.shape)).astype(np.float32)
+    x = x[np.abs(x) < 464]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.e4m3_round(x.astype(np.float64)), ref)
+
+
+def test_quantize_fp8_head_scale_and_codes():
+    rng = _rng(61)
+    x = rng.standard_normal((300, 16)).astype(np.float32)
+    x[17, 3] = -5.25                                   # the largest magnitude
+    codes, s = oracle.quantize_fp8_head(x)
+    assert s == float(np.float32(5.25) / np.float32(448))
+    assert codes[17, 3] == -448.0 and np.abs(codes).max() == 448.0
+    deq = codes * s
+    big = np.abs(x) >= 2.0 ** -6 * s
+    assert (np.abs(deq - x)[big] <= 2.0 ** -4 * np.abs(x)[big] * (1 + 1e-6)).all()
+    assert (np.abs(deq - x)[~big] <= 2.0 ** -10 * s * (1 + 1e-6)).all()
+    z, s0 = oracle.quantize_fp8_head(np.zeros((5, 4)))
+    assert s0 == 1.0 and (z == 0).all()
+
+
+def test_fp8_attention_exact_on_representable_inputs():
+    """Integers in [-7, 7] with 7 present quantise exactly (s = 7/448 = 2^-6 and
+    every 64 n, |n| <= 7, is an E4M3 value), so the low-bit attention equals the
+    masked attention of the inputs themselves."""
+    rng = _rng(62)
+    N, d, bq, bk = 90, 8, 16, 8
+    q, k, v = (rng.integers(-7, 8, (N, d)).astype(np.float64) for _ in range(3))
+    for t in (q, k, v):
+        t[0, 0] = 7.0
+    mask = rng.random((-(-N // bq), -(-N // bk))) < 0.5
+    mask[2] = False
+    o8, l8 = oracle.fp8_masked_attention(q, k, v, mask, bq, bk, scale=0.05)
+    o, l = oracle.masked_attention(q, k, v, mask, bq, bk, scale=0.05)
+    assert np.array_equal(o8, o) and np.array_equal(l8, l)
+    assert (o8[32:48] == 0).all() and np.isneginf(l8[32:48]).all()
+
+
+def test_fp8_attention_within_quantisation_error():
+    """On unit-variance inputs the low-bit attention stays near the
+    full-precision one (each operand within 2^-4 relative)."""
+    rng = _rng(63)
+    N, d = 256, 32
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    mask = np.ones((4, 4), dtype=bool)
+    o8, _ = oracle.fp8_masked_attention(q, k, v, mask, 64, 64)
+    o, _ = oracle.dense_attention(q, k, v)
+    err = np.abs(o8 - o)
+    assert 0 < err.max() < 0.05 and err.mean() < 0.01
