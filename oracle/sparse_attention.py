@@ -444,10 +444,10 @@ def blend_bwd(o_s, o_l, alpha_h, dout):
 # full precision). The pages name neither the format nor the scale granularity.
 # Reading: 8-bit floats in the E4M3 layout (1 sign bit, 4 exponent bits with
 # bias 7, 3 mantissa bits, no infinities, largest finite value 448), one fp32
-# scale per (batch, head) and tensor, s = amax / 448, codes = E4M3(x / s) with
-# the division in fp32 and round-to-nearest-even with saturation at +-448. The
-# low-bit attention is then the masked attention above on the dequantised
-# tensors codes * s.
+# scale per (batch, head) and tensor, s = amax / 448, codes = E4M3(x * r) with
+# r = 448 / amax, both in fp32, the product rounded to fp32 and then to E4M3 by
+# round-to-nearest-even with saturation at +-448. The low-bit attention is then
+# the masked attention above on the dequantised tensors codes * s.
 # --------------------------------------------------------------------------
 
 E4M3_MAX = 448.0
@@ -473,13 +473,17 @@ def e4m3_round(x) -> np.ndarray:
 def quantize_fp8_head(x) -> tuple[np.ndarray, float]:
     """One (batch, head) slice [N, d] -> (E4M3 code values as float64, fp32 scale).
 
-    s = amax / 448 in fp32 (1 when the slice is all zeros); each code is the
-    E4M3 rounding of the fp32 quotient x / s.
+    s = amax / 448 and r = 448 / amax in fp32 (both 1 when the slice is all
+    zeros); each code is the E4M3 rounding of the fp32 product x * r.
     """
     x32 = np.asarray(x, dtype=np.float32)
     amax = np.float32(np.max(np.abs(x32))) if x32.size else np.float32(0)
-    s = np.float32(amax) / np.float32(E4M3_MAX) if amax > 0 else np.float32(1.0)
-    codes = e4m3_round((x32 / s).astype(np.float64))
+    if amax > 0:
+        s = np.float32(amax) / np.float32(E4M3_MAX)
+        r = np.float32(E4M3_MAX) / np.float32(amax)
+    else:
+        s = r = np.float32(1.0)
+    codes = e4m3_round((x32 * r).astype(np.float64))
     return codes, float(s)
 
 
