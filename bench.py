@@ -452,6 +452,49 @@ def measure_backward(sa, wl, dev):
     return res
 
 
+def measure_low_bit_forward(sa, wl, dev):
+    """The low-bit forward on the workload: per-head E4M3 quantisation of Q, K
+    and V, and the sparse attention on E4M3 operands (with the blend when the
+    workload has the linear branch) over the step's lists. Its roofline peak is
+    the measured bf16 peak times the nominal fp8 / bf16 ratio of 2."""
+    x = make_inputs(wl, dev)
+    q, k, v, alpha = x["q"], x["k"], x["v"], x["alpha"]
+    m = sa.sa_build_mask(q, k, wl.bq, wl.bk, wl.topk, wl.topp)
+    ex = executed_flops(wl, m["kv_idx"], m["kv_cnt"])
+    q8, qs = sa.sa_quantize_fp8(q)
+    k8, ks = sa.sa_quantize_fp8(k)
+    v8, vs = sa.sa_quantize_fp8(v)
+    quant = _times(lambda: (sa.sa_quantize_fp8(q, out=q8, scale_out=qs), sa.sa_quantize_fp8(k, out=k8, scale_out=ks),
+                            sa.sa_quantize_fp8(v, out=v8, scale_out=vs)))
+    o_l = alpha_t = None
+    if wl.linear:
+        _, _, o_l = sa.sa_linear_branch(q, k, v, want_ol=True)
+        alpha_t = alpha
+    o8 = torch.empty_like(q)
+    attn8 = _times(lambda: sa.sa_sparse_attn_fp8_fwd(q8, k8, v8, qs, ks, vs, wl.bq, wl.bk, kv_idx=m["kv_idx"],
+                                                     kv_cnt=m["kv_cnt"], out=o8, o_l=o_l, alpha=alpha_t), calls=10)
+    o16 = torch.empty_like(q)
+    attn16 = _times(lambda: sa.sa_sparse_attn_fwd(q, k, v, wl.bq, wl.bk, kv_idx=m["kv_idx"], kv_cnt=m["kv_cnt"],
+                                                  out=o16, o_l=o_l, alpha=alpha_t), calls=10)
+    diff = (o8.float() - o16.float()).abs()
+    hbm, bf16, _, src = peaks()
+    tf = ex / (attn8["median"] * 1e-3) / 1e12
+    qbytes = 3 * q.numel() * (2 + 1)             # algorithmic: x read once, codes written (the amax pass reads x again)
+    res = {"quantize_qkv_ms": quant, "quantize_gbs": round(qbytes / (quant["median"] * 1e-3) / 1e9, 1),
+           "quantize_frac_of_hbm": round(qbytes / (quant["median"] * 1e-3) / 1e9 / hbm, 4),
+           "sparse_attn_fp8_ms": attn8, "sparse_attn_bf16_same_calls_ms": attn16,
+           "sparse_attn_fp8_exec_tflops": round(tf, 1),
+           "sparse_attn_fp8_frac_of_fp8_peak": round(tf / (2 * bf16), 4),
+           "peak_note": f"fp8 peak = 2 x the {src} bf16 burst peak ({2 * bf16:.0f} TFLOP/s)",
+           "blend": bool(wl.linear),
+           "max_abs_diff_vs_bf16_path": round(float(diff.max()), 5),
+           "mean_abs_diff_vs_bf16_path": round(float(diff.mean()), 6)}
+    sa.sa_device_status(dev)
+    del x, q, k, v, q8, k8, v8, o8, o16, m, o_l, diff
+    torch.cuda.empty_cache()
+    return res
+
+
 def measure_tile_scoring_and_layouts(sa, dev):
     """Veda's max-pooled heatmap (two tensor-core sweeps of Q K^T over every
     tile: 4 N^2 d flops per head) on the 1.3B-480p shape, all query blocks and
@@ -676,6 +719,7 @@ def main():
         import block_sparse_attention_softmax_b200 as sa
         dev = torch.device("cuda", local)
         res["backward"] = measure_backward(sa, wl, dev)
+        res["low_bit_forward"] = measure_low_bit_forward(sa, wl, dev)
         res["tile_scoring_and_layouts"] = measure_tile_scoring_and_layouts(sa, dev)
         res["per_workload"] = run_per_workload(args, dev)
     if rank == 0:

@@ -37,6 +37,10 @@ _SIGNATURES = {
                                          c_int, c_int, c_void_p, c_void_p, c_void_p, c_double,
                                          c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                          c_void_p]),
+    "sa_quantize_fp8": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "sa_sparse_attn_fp8_fwd": (c_int, [c_void_p] * 6 + [c_int] * 6 + [c_void_p, c_void_p, c_void_p, c_double,
+                                                                    c_void_p, c_void_p, c_void_p, c_void_p,
+                                                                    c_void_p, c_size_t, c_void_p]),
     "sa_dense_attn_fwd": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
                                   c_int, c_double, c_void_p, c_void_p, c_void_p]),
     "sa_linear_workspace_size": (c_size_t, [c_int] * 4),
@@ -271,6 +275,66 @@ def sa_sparse_attn_fwd(q, k, v, bq, bk, kv_idx=None, kv_cnt=None, ext_mask=None,
         _call("sa_sparse_attn_fwd", *common, _ptr(o), *tail)
     else:
         _call("sa_sparse_attn_blend_fwd", *common, _ptr(o_l), _ptr(alpha), _ptr(o), *tail)
+    return (o, lse) if want_lse else o
+
+
+_FP8 = (torch.float8_e4m3fn, torch.uint8)
+
+
+def sa_quantize_fp8(x, out=None, scale_out=None):
+    """Per-(batch, head) E4M3 quantisation of a [B, H, N, d] bf16 tensor:
+    returns (codes [B, H, N, d] float8_e4m3fn, scale [B, H] fp32) with
+    x ~ codes * scale."""
+    B, H, N, d = _qkv(x, names=("x",))
+    dev = x.device
+    x8 = out if out is not None else torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=dev)
+    _expect("out", x8, x.shape, _FP8)
+    sc = scale_out if scale_out is not None else torch.empty(B, H, dtype=torch.float32, device=dev)
+    _expect("scale_out", sc, (B, H), torch.float32)
+    _on_device(dev, x=x, out=x8, scale_out=sc)
+    _call("sa_quantize_fp8", _ptr(x), B, H, N, d, _ptr(x8), _ptr(sc), _stream(dev))
+    return x8, sc
+
+
+def sa_sparse_attn_fp8_fwd(q8, k8, v8, q_scale, k_scale, v_scale, bq, bk, kv_idx=None, kv_cnt=None,
+                           ext_mask=None, scale=0.0, want_lse=False, out=None, workspace=None, o_l=None,
+                           alpha=None):
+    """Sparse attention on E4M3 inputs (codes as float8_e4m3fn or uint8, one
+    fp32 scale per (batch, head) each, as sa_quantize_fp8 returns them); with
+    o_l and alpha the epilogue also blends the linear branch. d = 128."""
+    if q8 is None or q8.dim() != 4:
+        raise ValueError("q8 must be a [B, H, N, d] tensor")
+    B, H, N, d = q8.shape
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _expect(name, t, q8.shape, _FP8)
+    for name, t in (("q_scale", q_scale), ("k_scale", k_scale), ("v_scale", v_scale)):
+        _expect(name, t, (B, H), torch.float32)
+    if (o_l is None) != (alpha is None):
+        raise ValueError("o_l and alpha go together")
+    if o_l is not None:
+        _expect("o_l", o_l, q8.shape, torch.bfloat16)
+        _expect("alpha", alpha, (H, d), torch.float32)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    if kv_idx is not None:
+        _expect("kv_idx", kv_idx, (B, H, nqb, nkb), torch.int32)
+    if kv_cnt is not None:
+        _expect("kv_cnt", kv_cnt, (B, H, nqb), torch.int32)
+    if ext_mask is not None:
+        _expect("ext_mask", ext_mask, (B, H, nqb, nkb), (torch.uint8, torch.bool))
+    if out is not None:
+        _expect("out", out, q8.shape, torch.bfloat16)
+        if o_l is not None and out.data_ptr() == o_l.data_ptr():
+            raise ValueError("out must not alias o_l")
+    dev = q8.device
+    _on_device(dev, q8=q8, k8=k8, v8=v8, q_scale=q_scale, k_scale=k_scale, v_scale=v_scale, kv_idx=kv_idx,
+               kv_cnt=kv_cnt, ext_mask=ext_mask, out=out, o_l=o_l, alpha=alpha)
+    o = out if out is not None else torch.empty(q8.shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=dev) if want_lse else None
+    need = load().sa_sparse_attn_workspace_size(B, H, N, d, bq, bk, int(ext_mask is not None))
+    ws = _workspace(need, dev, workspace) if need else None
+    _call("sa_sparse_attn_fp8_fwd", _ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
+          B, H, N, d, bq, bk, _ptr(kv_idx), _ptr(kv_cnt), _ptr(ext_mask), float(scale), _ptr(o_l), _ptr(alpha),
+          _ptr(o), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev))
     return (o, lse) if want_lse else o
 
 

@@ -57,8 +57,16 @@
 //                the epilogue blends while O_s is still fp32, O = alpha ⊙ O_s
 //                + (1 - alpha) ⊙ O_l (SLA2 提案手法 ②): one bf16 rounding of O.
 //
+// Low-bit form (F8 = true; SLA2 提案手法 ③, a forward on low-bit queries, keys
+// and values): Q, K and V arrive as E4M3 bytes with one fp32 scale per (batch,
+// head) each. Both products run as tcgen05.mma kind::f8f6f4 (32 bytes of K per
+// instruction, half the instructions of bf16); the softmax folds scale * s_q *
+// s_k into its per-item exponent factor, P is written over S as E4M3 (P <= 256
+// < 448, so it needs no scale of its own), and the epilogue multiplies by s_v.
+// Item facts carry the two factors, posted by the K producer with the rest.
+//
 // TMEM columns: S buffers at 0, 128 and 256 (fp32, 128 wide; P aliases their
-// first 64 columns), O at 384 (d wide). Every mbarrier wait is bounded (see
+// first 64 columns, 32 in the low-bit form), O at 384 (d wide). Every mbarrier wait is bounded (see
 // sa_device.cuh), and a CTA that stops early waits (bounded) for the TMA loads
 // and MMAs it has issued before it gives up shared and tensor memory.
 #include "sa_internal.h"
@@ -85,12 +93,17 @@ constexpr int kVWarp = 2 + kSoftWarps;               // warp index of the V prod
 constexpr int kPVWarp = kVWarp + 1;                  // warp index of the P V issuer
 constexpr int kThreads = 32 * (kPVWarp + 1);
 
-template <int D>
+constexpr int kRingWords = 8;   // item facts: item, count, tail, then the low-bit factors
+
+template <int D, bool F8 = false>
 struct Layout {
-  static constexpr int NCH = D / 64;                       // 128-byte chunks along d
-  static constexpr uint32_t Q_BYTES = kBM * D * 2;
-  static constexpr uint32_t TILE_BYTES = kBN * D * 2;       // one K or V tile
-  static constexpr uint32_t BLK_BYTES = 64 * D * 2;         // one 64-key block
+  static constexpr int ES = F8 ? 1 : 2;                    // bytes per element of Q, K and V
+  static constexpr int NCH = D * ES / 128;                 // 128-byte chunks along d
+  static constexpr int CH_ELEMS = 128 / ES;                // elements per chunk
+  static constexpr int KSTEP = 32 / ES;                    // K elements per MMA instruction (32 bytes)
+  static constexpr uint32_t Q_BYTES = kBM * D * ES;
+  static constexpr uint32_t TILE_BYTES = kBN * D * ES;      // one K or V tile
+  static constexpr uint32_t BLK_BYTES = 64 * D * ES;        // one 64-key block
   static constexpr uint32_t Q_CHUNK = kBM * 128;            // bytes per d-chunk of Q
   static constexpr uint32_t KV_CHUNK = kBN * 128;           // bytes per d-chunk of K/V
   static constexpr uint32_t OFF_Q = 0;
@@ -99,7 +112,9 @@ struct Layout {
   static constexpr uint32_t OFF_RED = OFF_V + kVStages * TILE_BYTES;
   static constexpr uint32_t RED_BYTES = (2 * 2 + 2) * kBM * 4 + 4 * 16 * 4;   // row max [2][2][128], row sum [2][128], pair flags [4][16]
   static constexpr uint32_t OFF_BAR = OFF_RED + RED_BYTES;
-  static constexpr uint32_t OFF_RING = OFF_BAR + 512;    // item ring [kItemRing][4] int
+  static constexpr uint32_t OFF_RING = OFF_BAR + 512;    // item ring [kItemRing][kRingWords] int
+  static_assert(kItemRing * kRingWords * 4 <= 256, "item ring region");
+  static_assert(NCH >= 1, "the low-bit form needs d = 128");
   static constexpr uint32_t USED = OFF_RING + 256;
   // at least 120 KB so that a second CTA never shares the SM (all 512 TMEM columns are held)
   static constexpr uint32_t SMEM = (USED + 1024 > 120 * 1024) ? USED + 1024 : 120 * 1024;
@@ -185,13 +200,13 @@ __device__ __forceinline__ int next_nonempty(const AttnArgs& a, int item, int st
 
 }  // namespace attn
 
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(attn::kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, AttnArgs a) {
   using namespace attn;
-  using L = Layout<D>;
+  using L = Layout<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + L::OFF_Q;
@@ -204,7 +219,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   static_assert(B_COUNT * 8 + 8 <= 512, "barrier region");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
-  volatile int* item_ring = reinterpret_cast<volatile int*>(smem + L::OFF_RING);   // [kItemRing][item, cnt, tail, -]
+  // [kItemRing][item, cnt, tail, exponent factor, value factor, -, -, -]
+  volatile int* item_ring = reinterpret_cast<volatile int*>(smem + L::OFF_RING);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -268,16 +284,21 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           // from global memory on their critical path)
           const int rs = qi % kItemRing;
           if (!(ok = mbar_wait(&bars[B_IEMPTY + rs], ((qi / kItemRing) & 1) ^ 1, abort_flag))) break;
-          item_ring[rs * 4 + 0] = item;
-          item_ring[rs * 4 + 1] = it.cnt;
-          item_ring[rs * 4 + 2] = it.tail ? 1 : 0;
+          item_ring[rs * kRingWords + 0] = item;
+          item_ring[rs * kRingWords + 1] = it.cnt;
+          item_ring[rs * kRingWords + 2] = it.tail ? 1 : 0;
+          if constexpr (F8) {
+            // exponent factor scale * log2(e) * s_q * s_k, and s_v
+            item_ring[rs * kRingWords + 3] = __float_as_int(a.scale_log2 * __ldg(a.q_scale + it.bh) * __ldg(a.k_scale + it.bh));
+            item_ring[rs * kRingWords + 4] = __float_as_int(__ldg(a.v_scale + it.bh));
+          }
           mbar_arrive(&bars[B_IFULL + rs]);
           const int qs = qi % kQSlots;
           if (!(ok = mbar_wait(&bars[B_QEMPTY + qs], ((qi / kQSlots) & 1) ^ 1, abort_flag))) break;
           mbar_arrive_expect_tx(&bars[B_QFULL + qs], L::Q_BYTES);
 #pragma unroll
           for (int c = 0; c < L::NCH; ++c)
-            tma_load_3d(sQ + qs * L::Q_BYTES + c * L::Q_CHUNK, &tmQ, &bars[B_QFULL + qs], c * 64, it.qb * a.bq, it.bh);
+            tma_load_3d(sQ + qs * L::Q_BYTES + c * L::Q_CHUNK, &tmQ, &bars[B_QFULL + qs], c * L::CH_ELEMS, it.qb * a.bq, it.bh);
           q_armed = qi + 1;
         }
         for (int t = 0; t < it.T; ++t, ++g) {
@@ -302,9 +323,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           uint8_t* dst = ring + s * L::TILE_BYTES;
 #pragma unroll
           for (int c = 0; c < L::NCH; ++c) {
-            tma_load_3d(dst + c * L::KV_CHUNK, map, &bars[b_full + s], c * 64, kb0 * 64, it.bh);
+            tma_load_3d(dst + c * L::KV_CHUNK, map, &bars[b_full + s], c * L::CH_ELEMS, kb0 * 64, it.bh);
             if (nblk > 1)
-              tma_load_3d(dst + c * L::KV_CHUNK + 64 * 128, map, &bars[b_full + s], c * 64, kb1 * 64, it.bh);
+              tma_load_3d(dst + c * L::KV_CHUNK + 64 * 128, map, &bars[b_full + s], c * L::CH_ELEMS, kb1 * 64, it.bh);
           }
         }
         ++qi;
@@ -313,7 +334,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         // end of this CTA's items
         const int rs = qi % kItemRing;
         if (mbar_wait(&bars[B_IEMPTY + rs], ((qi / kItemRing) & 1) ^ 1, abort_flag)) {
-          item_ring[rs * 4 + 0] = n_items;
+          item_ring[rs * kRingWords + 0] = n_items;
           mbar_arrive(&bars[B_IFULL + rs]);
         }
       }
@@ -339,9 +360,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       const uint64_t qdesc0 = sw128_desc(smem_u32(sQ), 16, 1024);
       const uint64_t kdesc0 = sw128_desc(smem_u32(sK), 16, 1024);
       const uint64_t vdesc0 = sw128_desc(smem_u32(sV), L::KV_CHUNK, 1024);
-      const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
-      const uint32_t idesc_qk2 = idesc_bf16_f32(kBM, 128, false, false);
-      const uint32_t idesc_qk1 = idesc_bf16_f32(kBM, 64, false, false);
+      const uint32_t idesc_pv = F8 ? idesc_e4m3_f32(kBM, D, false, true) : idesc_bf16_f32(kBM, D, false, true);
+      const uint32_t idesc_qk2 = F8 ? idesc_e4m3_f32(kBM, 128, false, false) : idesc_bf16_f32(kBM, 128, false, false);
+      const uint32_t idesc_qk1 = F8 ? idesc_e4m3_f32(kBM, 64, false, false) : idesc_bf16_f32(kBM, 64, false, false);
       const uint32_t o_tm = tm + TM_O;
       struct Ring {
         int slot, n;
@@ -374,9 +395,12 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             const uint64_t kd = kdesc0 + ((kv.slot * L::TILE_BYTES) >> 4);
             const uint32_t s_tm = tm + tm_s(sb.slot);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              umma_ss(s_tm, qd + ((((kk >> 2) * L::Q_CHUNK) + (kk & 3) * 32u) >> 4),
-                      kd + ((((kk >> 2) * L::KV_CHUNK) + (kk & 3) * 32u) >> 4), idesc, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / L::KSTEP; ++kk) {
+              const uint64_t ad = qd + ((((kk >> 2) * L::Q_CHUNK) + (kk & 3) * 32u) >> 4);
+              const uint64_t bd = kd + ((((kk >> 2) * L::KV_CHUNK) + (kk & 3) * 32u) >> 4);
+              if constexpr (F8) umma_f8_ss(s_tm, ad, bd, idesc, kk > 0 ? 1u : 0u);
+              else umma_ss(s_tm, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            }
             tc_commit(&bars[B_SFULL + sb.slot]);   // S ready, and the K slot free
             if (t + 1 == it.T) tc_commit(&bars[B_QEMPTY + qs]);
           } else {
@@ -387,12 +411,17 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
               phase1 ^= 1u;
             }
             tc_fence_after();
-            const int nk = two ? 8 : 4;
+            const int nk = (two ? 128 : 64) / L::KSTEP;
             const uint64_t vd = vdesc0 + ((kv.slot * L::TILE_BYTES) >> 4);
             const uint32_t p_tm = tm + tm_s(sb.slot);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              if (kk < nk) umma_ts(o_tm, p_tm + kk * 8, vd + ((kk * 2048u) >> 4), idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 128 / L::KSTEP; ++kk) {
+              // K step kk: keys [kk * KSTEP, +KSTEP), 8 TMEM columns of P, KSTEP rows of V
+              if (kk >= nk) break;
+              const uint64_t bd = vd + ((kk * L::KSTEP * 128u) >> 4);
+              if constexpr (F8) umma_f8_ts(o_tm, p_tm + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+              else umma_ts(o_tm, p_tm + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+            }
             tc_commit(&bars[B_PVDONE + sb.slot]);   // O updated; S buffer and V slot free
             if (t + 1 == it.T) tc_commit(&bars[B_OFULL]);
           }
@@ -440,10 +469,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         ok = false;
         break;
       }
-      const int item = item_ring[rs * 4 + 0];
+      const int item = item_ring[rs * kRingWords + 0];
       Item it;
-      it.cnt = item_ring[rs * 4 + 1];
-      it.tail = item_ring[rs * 4 + 2] != 0;
+      it.cnt = item_ring[rs * kRingWords + 1];
+      it.tail = item_ring[rs * kRingWords + 2] != 0;
+      // exponent factor of the scores and factor of the output (the low-bit
+      // form's scales folded in)
+      const float fexp = F8 ? __int_as_float(item_ring[rs * kRingWords + 3]) : sl2;
+      const float fout = F8 ? __int_as_float(item_ring[rs * kRingWords + 4]) : 1.f;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_IEMPTY + rs]);
       for (int z = prev + gridDim.x; z < item; z += gridDim.x) {
@@ -514,7 +547,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         }
         float* rm = red_max + (g & 1) * 2 * kBM;
-        const float posted = s_ok ? mx : __uint_as_float(kStopBits);
+        // the low-bit form posts its max in the log2 domain (the factor is the
+        // same for both halves; bf16 scales after the exchange)
+        const float posted = s_ok ? (F8 ? mx * fexp : mx) : __uint_as_float(kStopBits);
         rm[half * kBM + row] = posted;
         pair_sync(pair_bar);
         const float pmx = rm[(half ^ 1) * kBM + row];
@@ -523,7 +558,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         // included, is the same in both; the stop, if any, is taken there.
         const bool stop = !s_ok || __float_as_uint(pmx) == kStopBits;
         mx = fmaxf(posted, pmx);
-        const float m_tile = mx * sl2;
+        const float m_tile = F8 ? mx : mx * sl2;
         float corr = 1.f;
         if (m_tile > m + 8.f) {
           corr = fast_exp2(m - m_tile);   // 0 on the first tile (m = -inf)
@@ -531,10 +566,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           l *= corr;
         }
         // P = 2^(S * scale * log2(e) - m), two columns per packed instruction.
-        const uint64_t sl2x2 = f2_make(sl2, sl2);
+        const uint64_t sl2x2 = f2_make(fexp, fexp);
         const uint64_t negm2 = f2_make(-m, -m);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // packed (+0, +0)
-        uint32_t p[32];
+        uint32_t p[F8 ? 16 : 32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const uint64_t a2 = ffma2(f2_make(x[2 * c], x[2 * c + 1]), sl2x2, negm2);
@@ -548,14 +583,21 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             e1 = fast_exp2(a1);
           }
           acc[c & 3] = fadd2(acc[c & 3], f2_make(e0, e1));
-          p[c] = pack_bf16x2(e0, e1);
+          if constexpr (F8) {
+            // four E4M3 values per column, the lowest key in the lowest byte
+            const uint32_t h = pack_e4m3x2(e0, e1);
+            p[c >> 1] = (c & 1) ? (p[c >> 1] | (h << 16)) : h;
+          } else {
+            p[c] = pack_bf16x2(e0, e1);
+          }
         }
         {
           float s0, s1;
           f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), s0, s1);
           l += s0 + s1;
         }
-        tmem_st32(tm + lane_addr + tm_s(b) + half * 32, p);
+        if constexpr (F8) tmem_st16(tm + lane_addr + tm_s(b) + half * 16, p);
+        else tmem_st32(tm + lane_addr + tm_s(b) + half * 32, p);
         if (!stop && t > 0 && __any_sync(0xFFFFFFFFu, corr != 1.f)) {
           // O is complete up to the previous tile once its P V has landed
           const int pb = (g - 1) % kSBufs;
@@ -608,7 +650,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       const float pl = red_sum[(half ^ 1) * kBM + row];
       if (!(ok = o_ok && __float_as_uint(pl) != kStopBits)) break;
       const float lt = l + pl;
-      const float inv_l = 1.f / lt;
+      const float inv_l = F8 ? fout / lt : 1.f / lt;
       if (store) {
         uint4* dst = reinterpret_cast<uint4*>(orow);
         if (a.alpha) {
@@ -660,27 +702,32 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool F8>
 static cudaError_t launch_d(const AttnArgs& a, cudaStream_t st) {
-  using L = attn::Layout<D>;
+  using L = attn::Layout<D, F8>;
   CUtensorMap mq, mk, mv;
-  if (encode_tensor_map_3d_bf16(&mq, a.q, D, a.N, a.BH, 64, attn::kBM) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  if (encode_tensor_map_3d_bf16(&mk, a.k, D, a.N, a.BH, 64, 64) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  if (encode_tensor_map_3d_bf16(&mv, a.v, D, a.N, a.BH, 64, 64) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+  auto enc = [&](CUtensorMap* m, const void* base, uint32_t rows) {
+    return F8 ? encode_tensor_map_3d_u8(m, base, D, a.N, a.BH, L::CH_ELEMS, rows)
+              : encode_tensor_map_3d_bf16(m, base, D, a.N, a.BH, L::CH_ELEMS, rows);
+  };
+  if (enc(&mq, a.q, attn::kBM) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (enc(&mk, a.k, 64) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (enc(&mv, a.v, 64) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long items = static_cast<long long>(a.BH) * a.nqb;
   const int grid = static_cast<int>(items < sms ? items : sms);
-  sparse_attn_kernel<D><<<grid, attn::kThreads, L::SMEM, st>>>(mq, mk, mv, a);
+  sparse_attn_kernel<D, F8><<<grid, attn::kThreads, L::SMEM, st>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t st) {
   if (static_cast<long long>(a.BH) * a.nqb > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  return a.d == 128 ? launch_d<128>(a, st) : launch_d<64>(a, st);
+  if (a.fp8) return a.d == 128 ? launch_d<128, true>(a, st) : cudaErrorInvalidValue;
+  return a.d == 128 ? launch_d<128, false>(a, st) : launch_d<64, false>(a, st);
 }
 
 }  // namespace sa

@@ -8,6 +8,7 @@
 #include "permute_kernels.cu"
 #include "bwd_kernels.cu"
 #include "lin_bwd_kernels.cu"
+#include "fp8_kernels.cu"
 #include "sa_api.cu"
 #include "noalloc.cu"
 #include "diag.cu"

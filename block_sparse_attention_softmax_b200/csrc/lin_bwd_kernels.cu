@@ -8,11 +8,21 @@
 //   dq   = (S dnum + dden z) * phi'(q)
 //   dS   = sum_i phi(q_i) dnum_i^T,  dz = sum_i dden_i phi(q_i)
 //   dk   = (dS v + dz) * phi'(k),  dv = phi(k)^T dS
-// These are O(N d^2) per head, small next to the sparse attention, and run on
-// fp32 CUDA cores: lin_q_kernel (one warp per query token, S and z of the head
-// in shared memory), lin_dsz_kernel (partial dS, dz over token chunks),
-// lin_reduce_kernel (fixed-order sum of the partials: deterministic),
-// lin_k_kernel (one warp per key token, dS and dz in shared memory).
+// Every product is a 128-token tile times a d x d matrix of the head, so each
+// runs on the tensor core (bf16 operands, the d x d matrix split into bf16
+// hi + lo parts as in the forward, fp32 accumulators in TMEM):
+//   lin_bwd_q_kernel   per (128-token tile, head): num = phi(Q) S; then, from
+//                      num, dO_l and den = phi(q) . z, the rows' dnum and dden;
+//                      dq = (dnum S^T + dden z) * phi'(q) with phi'(q) =
+//                      min(phi(q), 1); dnum (bf16) to global memory for the
+//                      next step, and the tile's partial dz
+//   dS = phi(Q)^T dnum the linear branch's state kernel run on (Q, dnum)
+//   lin_reduce_kernel  dz = fixed-order sum of the tiles' partials
+//   lin_bwd_k_kernel   per (128-token tile, head): dk = (V dS^T + dz) *
+//                      phi'(k) and dv = phi(K) dS
+// The d x d operand in shared memory serves as B both ways: its rows of 64
+// bf16 are MN-major for X S and K-major for X S^T. Deterministic: every sum
+// has one owner and a fixed order.
 // blend_bwd_kernel: dO_s = alpha dO, dO_l = (1 - alpha) dO and partial sums of
 // dO (O_s - O_l) per head and chunk, reduced in a fixed order into dalpha.
 #include "sa_internal.h"
@@ -20,128 +30,375 @@
 namespace sa {
 
 namespace linb {
-constexpr int kChunk = 512;           // tokens per partial of dS, dz and dalpha
-constexpr int kWarps = 8;
+constexpr int kChunk = 512;           // tokens per partial of dalpha
+constexpr int kThreads = 256;         // 8 warps: two per TMEM lane quadrant
+
+template <int D>
+struct BwdLayout {
+  using O = lin::OutLayout<D>;                 // the d x d operand (hi, lo) at offset 0
+  static constexpr uint32_t OFF_X = 2 * O::B_BYTES;                   // first token tile
+  static constexpr uint32_t OFF_Y = OFF_X + O::T_BYTES;               // second token tile
+  static constexpr uint32_t OFF_RED = OFF_Y + O::T_BYTES;             // [2 halves][128 rows] float2
+  static constexpr uint32_t OFF_ROW = OFF_RED + 2 * 128 * 8;          // [128] per-row value
+  static constexpr uint32_t OFF_VEC = OFF_ROW + 128 * 4;              // [D] z or dz
+  static constexpr uint32_t OFF_PART = OFF_VEC + D * 4;               // [256] partial sums
+  static constexpr uint32_t OFF_BAR = OFF_PART + 256 * 4;             // 4 mbarriers + TMEM slot
+  // at least 80 KB, so that at most two CTAs (2 x 256 TMEM columns) share an SM
+  static constexpr uint32_t SMEM = (OFF_BAR + 64 + 1024 > 80 * 1024) ? OFF_BAR + 64 + 1024 : 80 * 1024;
+};
+
+// 16-byte unit u (8 features) of token row r in a [128 tokens x D] tile with
+// 128-byte swizzle, 64 features per chunk
+template <int D>
+__device__ __forceinline__ uint32_t tile_unit(int r, int u) {
+  return (u >> 3) * lin::OutLayout<D>::T_CHUNK + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+}
 }
 
-__device__ __forceinline__ float bf16_at(const __nv_bfloat16* p, long long i) { return __bfloat162float(p[i]); }
-__device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : __expf(x); }
-__device__ __forceinline__ float phi_grad_f(float x) { return x > 0.f ? 1.f : __expf(x); }
 
-// One warp per query token; lane l owns columns c = l + 32 j. Writes dq (or adds
-// into it), dnum [BH, N, d] and dden [BH, N].
+// phi applied in place to a [128 x D] bf16 tile (all 256 threads)
 template <int D>
-__global__ void __launch_bounds__(linb::kWarps * 32) lin_q_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dol, const float* __restrict__ S,
-    const float* __restrict__ z, int N, int tok_per_cta, float* __restrict__ dq, int accumulate,
-    float* __restrict__ dnum, float* __restrict__ dden) {
-  constexpr int J = D / 32;
-  extern __shared__ float sm[];
-  constexpr int LD = D + 1;              // padded row stride: row and column walks are both conflict-free
-  float* sS = sm;                        // [D][LD]
-  float* sz = sS + D * LD;               // [D]
-  float* sv = sz + D;                    // [kWarps][2][D] per-warp vectors
-  const int bh = blockIdx.y;
-  for (int i = threadIdx.x; i < D * D; i += blockDim.x) sS[(i / D) * LD + i % D] = S[static_cast<long long>(bh) * D * D + i];
-  for (int i = threadIdx.x; i < D; i += blockDim.x) sz[i] = z[static_cast<long long>(bh) * D + i];
+__device__ __forceinline__ void phi_tile_inplace(uint8_t* tile, int tid) {
+  constexpr int UPT = D / 16;                   // 16-byte units per thread: half a row
+  const int r = tid >> 1, u0 = (tid & 1) * UPT;
+#pragma unroll
+  for (int j = 0; j < UPT; ++j) {
+    uint4* p = reinterpret_cast<uint4*>(tile + linb::tile_unit<D>(r, u0 + j));
+    uint4 w = *p;
+    uint32_t* x = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      x[e] = pack_bf16x2(lin::phi_f(__uint_as_float(x[e] << 16)), lin::phi_f(__uint_as_float(x[e] & 0xFFFF0000u)));
+    *p = w;
+  }
+}
+
+// D/2 fp32 accumulator columns [col0, col0 + D/2) of this thread's TMEM lane
+template <int D>
+__device__ __forceinline__ void tmem_ld_half(uint32_t taddr, float (&v)[D / 2]) {
+  uint32_t r[32];
+#pragma unroll
+  for (int c = 0; c < D / 2; c += 32) {
+    tmem_ld32_wait(taddr + c, r);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[c + e] = __uint_as_float(r[e]);
+  }
+}
+
+// the 8 bf16 of 16-byte unit u of row r as floats
+template <int D>
+__device__ __forceinline__ void unit_f32(const uint8_t* tile, int r, int u, float (&f)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4*>(tile + linb::tile_unit<D>(r, u));
+  const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = __uint_as_float(x[e] << 16);
+    f[2 * e + 1] = __uint_as_float(x[e] & 0xFFFF0000u);
+  }
+}
+
+// K-major view of the d x d operand: the product X M^T (its rows of 64 bf16 are
+// the K extent; chunks of 64 columns are B_CHUNK apart)
+template <int D>
+__device__ __forceinline__ uint64_t head_desc_k(uint32_t base, int kk) {
+  return sw128_desc(base + (kk >> 2) * lin::OutLayout<D>::B_CHUNK + (kk & 3) * 32u, 16, 1024);
+}
+// MN-major view: the product X M
+template <int D>
+__device__ __forceinline__ uint64_t head_desc_mn(uint32_t base, int kk) {
+  return sw128_desc(base + kk * 2048u, lin::OutLayout<D>::B_CHUNK, 1024);
+}
+template <int D>
+__device__ __forceinline__ uint64_t tile_desc(uint32_t base, int kk) {
+  return sw128_desc(base + (kk >> 2) * lin::OutLayout<D>::T_CHUNK + (kk & 3) * 32u, 16, 1024);
+}
+
+// acc (+)= X M (mn = true) or X M^T, with M as hi + lo
+template <int D>
+__device__ __forceinline__ void issue_tile_by_head(uint32_t acc, uint32_t x, uint32_t m, bool mn) {
+  const uint32_t idesc = idesc_bf16_f32(128, D, false, mn);
+  const uint32_t mlo = m + lin::OutLayout<D>::B_BYTES;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t a = tile_desc<D>(x, kk);
+    umma_ss(acc, a, mn ? head_desc_mn<D>(m, kk) : head_desc_k<D>(m, kk), idesc, kk > 0 ? 1u : 0u);
+    umma_ss(acc, a, mn ? head_desc_mn<D>(mlo, kk) : head_desc_k<D>(mlo, kk), idesc, 1u);
+  }
+}
+
+// dq (and dnum, the tile's dz partial) for one (tile, head)
+template <int D>
+__global__ void __launch_bounds__(linb::kThreads, 1)
+    lin_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                     const __grid_constant__ CUtensorMap tmDN, const float* __restrict__ S,
+                     const float* __restrict__ z, int N, float* __restrict__ dq, int accumulate,
+                     float* __restrict__ dz_part) {
+  using L = linb::BwdLayout<D>;
+  constexpr int HC = D / 2, HU = HC / 8;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = lin::align1k(smem_raw);
+  uint8_t* sX = smem + L::OFF_X;              // Q, then phi(Q)
+  uint8_t* sY = smem + L::OFF_Y;              // dO_l, then dnum
+  float2* red = reinterpret_cast<float2*>(smem + L::OFF_RED);
+  float* srow = reinterpret_cast<float*>(smem + L::OFF_ROW);      // dden per row
+  float* sz = reinterpret_cast<float*>(smem + L::OFF_VEC);
+  float* spart = reinterpret_cast<float*>(smem + L::OFF_PART);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);   // [0] loads, [1] num, [2] dq
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y, tile = blockIdx.x, tok0 = tile * 128;
+  if (tid == 0) {
+    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* fqv = sv + warp * 2 * D;
-  float* dnv = fqv + D;
-  const int t0 = blockIdx.x * tok_per_cta, t1 = min(N, t0 + tok_per_cta);
-  for (int t = t0 + warp; t < t1; t += linb::kWarps) {
-    const long long r = static_cast<long long>(bh) * N + t;
-    float fq[J], qx[J], go[J];
-    float den = 0.f;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[0], 2 * lin::OutLayout<D>::T_BYTES);
 #pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int c = lane + 32 * j;
-      qx[j] = bf16_at(q, r * D + c);
-      fq[j] = phi_f(qx[j]);
-      go[j] = bf16_at(dol, r * D + c);
-      fqv[c] = fq[j];
-      den = fmaf(fq[j], sz[c], den);
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(sX + c * lin::OutLayout<D>::T_CHUNK, &tmQ, &bars[0], c * 64, tok0, bh);
+      tma_load_3d(sY + c * lin::OutLayout<D>::T_CHUNK, &tmDO, &bars[0], c * 64, tok0, bh);
     }
+  }
+  build_head_operand<D>(smem, S, bh, tid, linb::kThreads);
+  for (int i = tid; i < D; i += linb::kThreads) sz[i] = z[static_cast<long long>(bh) * D + i];
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tmem_slot;
+  bool ok = mbar_wait(&bars[0], 0, abort_flag);
+  phi_tile_inplace<D>(sX, tid);
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (tid == 0) {
+    tc_fence_after();
+    if (ok) issue_tile_by_head<D>(tm, smem_u32(sX), smem_u32(smem), true);   // num = phi(Q) S
+    tc_commit(&bars[1]);
+  }
+  // epilogue 1: this thread's row, half the columns
+  const int quad = warp & 3, half = warp >> 2;
+  const int r = quad * 32 + lane;
+  const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+  ok = mbar_wait(&bars[1], 0, abort_flag) && ok;
+  tc_fence_after();
+  float acc[HC];
+  tmem_ld_half<D>(tm + lane_addr + half * HC, acc);
+  float pden = 0.f, pdot = 0.f;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xFFFFFFFFu, den, off);
-    __syncwarp();
-    float num[J];
+  for (int j = 0; j < HU; ++j) {
+    float fq[8], go[8];
+    unit_f32<D>(sX, r, half * HU + j, fq);
+    unit_f32<D>(sY, r, half * HU + j, go);
 #pragma unroll
-    for (int j = 0; j < J; ++j) num[j] = 0.f;
-    for (int aa = 0; aa < D; ++aa) {
-      const float f = fqv[aa];
-#pragma unroll
-      for (int j = 0; j < J; ++j) num[j] = fmaf(f, sS[aa * LD + lane + 32 * j], num[j]);
+    for (int e = 0; e < 8; ++e) {
+      pden = fmaf(fq[e], sz[(half * HU + j) * 8 + e], pden);
+      pdot = fmaf(go[e], acc[j * 8 + e], pdot);
     }
-    const float inv = 1.f / den;
-    float dot = 0.f;
+  }
+  red[half * 128 + r] = make_float2(pden, pdot);
+  __syncthreads();
+  const float2 r0 = red[r], r1 = red[128 + r];
+  const float den = r0.x + r1.x;
+  const float inv = 1.f / den;
+  const float dden = -((r0.y + r1.y) * inv) * inv;   // -(dO . num / den) / den
 #pragma unroll
-    for (int j = 0; j < J; ++j) dot = fmaf(go[j], num[j] * inv, dot);
+  for (int j = 0; j < HU; ++j) {
+    float go[8];
+    unit_f32<D>(sY, r, half * HU + j, go);
+    uint4 w;
+    w.x = pack_bf16x2(go[0] * inv, go[1] * inv);
+    w.y = pack_bf16x2(go[2] * inv, go[3] * inv);
+    w.z = pack_bf16x2(go[4] * inv, go[5] * inv);
+    w.w = pack_bf16x2(go[6] * inv, go[7] * inv);
+    *reinterpret_cast<uint4*>(sY + linb::tile_unit<D>(r, half * HU + j)) = w;
+  }
+  if (half == 0) srow[r] = dden;          // rows past N have dO = 0, so dden = 0
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0) {
+    tc_fence_after();
+    if (ok) issue_tile_by_head<D>(tm + 128, smem_u32(sY), smem_u32(smem), false);   // dnum S^T
+    tc_commit(&bars[2]);
+  } else if (tid == 32) {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, off);
-    const float dd = -dot * inv;
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int c = lane + 32 * j;
-      const float dn = go[j] * inv;
-      dnv[c] = dn;
-      dnum[r * D + c] = dn;
+    for (int c = 0; c < D / 64; ++c)
+      tma_store_3d(&tmDN, sY + c * lin::OutLayout<D>::T_CHUNK, c * 64, tok0, bh);   // rows past N are clipped
+    bulk_commit();
+  }
+  {
+    // partial dz[a] = sum over the tile's rows of dden * phi(q)[a]: feature a,
+    // a share of the rows per thread, shares added in a fixed order
+    constexpr int TPF = linb::kThreads / D, RPT = 128 / TPF;
+    const int a = tid % D, part = tid / D;
+    float sacc = 0.f;
+    for (int rr = part * RPT; rr < (part + 1) * RPT; ++rr) {
+      const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(sX + linb::tile_unit<D>(rr, a >> 3)) + (a & 7);
+      sacc = fmaf(srow[rr], __bfloat162float(*e), sacc);
     }
-    if (lane == 0) dden[r] = dd;
-    __syncwarp();
-    // dfq[a] = sum_c S[a, c] dnum[c] + dden z[a]; lane owns rows a = lane + 32 j
+    spart[tid] = sacc;
+  }
+  ok = mbar_wait(&bars[2], 0, abort_flag) && ok;
+  tc_fence_after();
+  tmem_ld_half<D>(tm + 128 + lane_addr + half * HC, acc);
+  const int tok = tok0 + r;
+  if (tok < N) {
+    float* dst = dq + (static_cast<long long>(bh) * N + tok) * D + half * HC;
 #pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int aa = lane + 32 * j;
-      float acc = dd * sz[aa];
-      for (int c = 0; c < D; ++c) acc = fmaf(sS[aa * LD + c], dnv[c], acc);
-      const float g = acc * phi_grad_f(qx[j]);
-      dq[r * D + aa] = accumulate ? dq[r * D + aa] + g : g;
+    for (int j = 0; j < HU; ++j) {
+      float fq[8];
+      unit_f32<D>(sX, r, half * HU + j, fq);
+      float g[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int c = (half * HU + j) * 8 + e;
+        g[e] = (acc[j * 8 + e] + dden * sz[c]) * fminf(fq[e], 1.f);     // phi'(q) = min(phi(q), 1)
+      }
+      float4* d4 = reinterpret_cast<float4*>(dst + j * 8);
+      if (accumulate) {
+        const float4 o0 = d4[0], o1 = d4[1];
+        g[0] += o0.x; g[1] += o0.y; g[2] += o0.z; g[3] += o0.w;
+        g[4] += o1.x; g[5] += o1.y; g[6] += o1.z; g[7] += o1.w;
+      }
+      d4[0] = make_float4(g[0], g[1], g[2], g[3]);
+      d4[1] = make_float4(g[4], g[5], g[6], g[7]);
     }
-    __syncwarp();
+  }
+  __syncthreads();
+  if (tid < D) {
+    float sacc = 0.f;
+    for (int p2 = 0; p2 < linb::kThreads / D; ++p2) sacc += spart[p2 * D + tid];
+    dz_part[(static_cast<long long>(bh) * gridDim.x + tile) * D + tid] = sacc;
+  }
+  if (tid == 32) bulk_wait_all();
+  if (tid == 0) {
+    // anything still in flight after a failed wait lands before the memory is released
+    mbar_drain(&bars[0], 0);
+    mbar_drain(&bars[1], 0);
+    mbar_drain(&bars[2], 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tm, 256);
   }
 }
 
-// Partial dS (d x d) and dz over one chunk of tokens: thread i owns entries
-// e = i, i + blockDim, ... of dS; phi(q) and dnum of each token are staged in
-// shared memory.
+// dk and dv for one (tile, head)
 template <int D>
-__global__ void __launch_bounds__(256) lin_dsz_kernel(const __nv_bfloat16* __restrict__ q,
-                                                      const float* __restrict__ dnum, const float* __restrict__ dden,
-                                                      int N, int n_chunks, float* __restrict__ part) {
-  __shared__ float fq[32][D];
-  __shared__ float dn[32][D];
-  __shared__ float ddv[32];
-  const int bh = blockIdx.y, ch = blockIdx.x;
-  const int t0 = ch * linb::kChunk, t1 = min(N, t0 + linb::kChunk);
-  constexpr int E = D * D / 256;          // dS entries per thread
-  float acc[E], accz = 0.f;
-#pragma unroll
-  for (int e = 0; e < E; ++e) acc[e] = 0.f;
-  for (int tb = t0; tb < t1; tb += 32) {
-    const int nt = min(32, t1 - tb);
-    for (int i = threadIdx.x; i < 32 * D; i += 256) {
-      const int tt = i / D, c = i % D;
-      const long long r = static_cast<long long>(bh) * N + tb + tt;
-      fq[tt][c] = tt < nt ? phi_f(bf16_at(q, r * D + c)) : 0.f;
-      dn[tt][c] = tt < nt ? dnum[r * D + c] : 0.f;
-    }
-    if (threadIdx.x < 32) ddv[threadIdx.x] = threadIdx.x < nt ? dden[static_cast<long long>(bh) * N + tb + threadIdx.x] : 0.f;
-    __syncthreads();
-    for (int tt = 0; tt < nt; ++tt) {
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const int idx = threadIdx.x + 256 * e;
-        acc[e] = fmaf(fq[tt][idx / D], dn[tt][idx % D], acc[e]);
-      }
-      if (threadIdx.x < D) accz = fmaf(ddv[tt], fq[tt][threadIdx.x], accz);
-    }
-    __syncthreads();
+__global__ void __launch_bounds__(linb::kThreads, 1)
+    lin_bwd_k_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const float* __restrict__ dS, const float* __restrict__ dz, int N, float* __restrict__ dk,
+                     float* __restrict__ dv, int accumulate) {
+  using L = linb::BwdLayout<D>;
+  constexpr int HC = D / 2, HU = HC / 8;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = lin::align1k(smem_raw);
+  uint8_t* sX = smem + L::OFF_X;              // K, then phi(K)
+  uint8_t* sY = smem + L::OFF_Y;              // V
+  float* sz = reinterpret_cast<float*>(smem + L::OFF_VEC);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);   // [0] loads, [1] products
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y, tok0 = blockIdx.x * 128;
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) mbar_init(&bars[i], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
   }
-  float* p = part + (static_cast<long long>(bh) * n_chunks + ch) * (D * D + D);
+  __syncthreads();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[0], 2 * lin::OutLayout<D>::T_BYTES);
 #pragma unroll
-  for (int e = 0; e < E; ++e) p[threadIdx.x + 256 * e] = acc[e];
-  if (threadIdx.x < D) p[D * D + threadIdx.x] = accz;
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(sX + c * lin::OutLayout<D>::T_CHUNK, &tmK, &bars[0], c * 64, tok0, bh);
+      tma_load_3d(sY + c * lin::OutLayout<D>::T_CHUNK, &tmV, &bars[0], c * 64, tok0, bh);
+    }
+  }
+  build_head_operand<D>(smem, dS, bh, tid, linb::kThreads);
+  for (int i = tid; i < D; i += linb::kThreads) sz[i] = dz[static_cast<long long>(bh) * D + i];
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tmem_slot;
+  bool ok = mbar_wait(&bars[0], 0, abort_flag);
+  phi_tile_inplace<D>(sX, tid);
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (tid == 0) {
+    tc_fence_after();
+    if (ok) {
+      issue_tile_by_head<D>(tm, smem_u32(sY), smem_u32(smem), false);        // V dS^T
+      issue_tile_by_head<D>(tm + 128, smem_u32(sX), smem_u32(smem), true);   // phi(K) dS
+    }
+    tc_commit(&bars[1]);
+  }
+  const int quad = warp & 3, half = warp >> 2;
+  const int r = quad * 32 + lane;
+  const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+  ok = mbar_wait(&bars[1], 0, abort_flag) && ok;
+  tc_fence_after();
+  const int tok = tok0 + r;
+  float acc[HC];
+  tmem_ld_half<D>(tm + lane_addr + half * HC, acc);
+  if (tok < N) {
+    float* dst = dk + (static_cast<long long>(bh) * N + tok) * D + half * HC;
+#pragma unroll
+    for (int j = 0; j < HU; ++j) {
+      float fk[8], g[8];
+      unit_f32<D>(sX, r, half * HU + j, fk);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) g[e] = (acc[j * 8 + e] + sz[(half * HU + j) * 8 + e]) * fminf(fk[e], 1.f);
+      float4* d4 = reinterpret_cast<float4*>(dst + j * 8);
+      if (accumulate) {
+        const float4 o0 = d4[0], o1 = d4[1];
+        g[0] += o0.x; g[1] += o0.y; g[2] += o0.z; g[3] += o0.w;
+        g[4] += o1.x; g[5] += o1.y; g[6] += o1.z; g[7] += o1.w;
+      }
+      d4[0] = make_float4(g[0], g[1], g[2], g[3]);
+      d4[1] = make_float4(g[4], g[5], g[6], g[7]);
+    }
+  }
+  tmem_ld_half<D>(tm + 128 + lane_addr + half * HC, acc);
+  if (tok < N) {
+    float* dst = dv + (static_cast<long long>(bh) * N + tok) * D + half * HC;
+#pragma unroll
+    for (int j = 0; j < HU; ++j) {
+      float g[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) g[e] = acc[j * 8 + e];
+      float4* d4 = reinterpret_cast<float4*>(dst + j * 8);
+      if (accumulate) {
+        const float4 o0 = d4[0], o1 = d4[1];
+        g[0] += o0.x; g[1] += o0.y; g[2] += o0.z; g[3] += o0.w;
+        g[4] += o1.x; g[5] += o1.y; g[6] += o1.z; g[7] += o1.w;
+      }
+      d4[0] = make_float4(g[0], g[1], g[2], g[3]);
+      d4[1] = make_float4(g[4], g[5], g[6], g[7]);
+    }
+  }
+  if (tid == 0) {
+    mbar_drain(&bars[0], 0);
+    mbar_drain(&bars[1], 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tm, 256);
+  }
 }
 
 // Fixed-order sum of the chunk partials: out[bh][e] for e < len.
@@ -152,53 +409,6 @@ __global__ void lin_reduce_kernel(const float* __restrict__ part, int n_chunks, 
   float acc = 0.f;
   for (int c = 0; c < n_chunks; ++c) acc += part[(static_cast<long long>(bh) * n_chunks + c) * len + e];
   out[static_cast<long long>(bh) * len + e] = acc;
-}
-
-// One warp per key token: dk = (dS v + dz) * phi'(k), dv = phi(k)^T dS.
-template <int D>
-__global__ void __launch_bounds__(linb::kWarps * 32) lin_k_kernel(
-    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, const float* __restrict__ dsz,
-    int N, int tok_per_cta, float* __restrict__ dk, float* __restrict__ dv, int accumulate) {
-  constexpr int J = D / 32;
-  extern __shared__ float sm[];
-  constexpr int LD = D + 1;               // padded row stride, as in lin_q_kernel
-  float* sS = sm;                         // dS [D][LD]
-  float* sz = sS + D * LD;                // dz [D]
-  float* sv = sz + D;                     // [kWarps][2][D]
-  const int bh = blockIdx.y;
-  const float* src = dsz + static_cast<long long>(bh) * (D * D + D);
-  for (int i = threadIdx.x; i < D * D; i += blockDim.x) sS[(i / D) * LD + i % D] = src[i];
-  for (int i = threadIdx.x; i < D; i += blockDim.x) sz[i] = src[D * D + i];
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* vv = sv + warp * 2 * D;
-  float* fk = vv + D;
-  const int t0 = blockIdx.x * tok_per_cta, t1 = min(N, t0 + tok_per_cta);
-  for (int t = t0 + warp; t < t1; t += linb::kWarps) {
-    const long long r = static_cast<long long>(bh) * N + t;
-    float kx[J];
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int c = lane + 32 * j;
-      kx[j] = bf16_at(k, r * D + c);
-      fk[c] = phi_f(kx[j]);
-      vv[c] = bf16_at(v, r * D + c);
-    }
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int aa = lane + 32 * j;
-      float gk = sz[aa], gv = 0.f;
-      for (int c = 0; c < D; ++c) {
-        gk = fmaf(sS[aa * LD + c], vv[c], gk);      // (dS v)[a]
-        gv = fmaf(fk[c], sS[c * LD + aa], gv);      // (phi(k)^T dS)[a]
-      }
-      gk *= phi_grad_f(kx[j]);
-      dk[r * D + aa] = accumulate ? dk[r * D + aa] + gk : gk;
-      dv[r * D + aa] = accumulate ? dv[r * D + aa] + gv : gv;
-    }
-    __syncwarp();
-  }
 }
 
 // dO_s = alpha dO, dO_l = (1 - alpha) dO, and per (head, chunk) partials of
@@ -236,10 +446,11 @@ __global__ void blend_alpha_kernel(const float* __restrict__ part, int B, int H,
 }
 
 size_t lin_bwd_ws_bytes(int BH, int N, int d) {
-  const long long nch = (N + linb::kChunk - 1) / linb::kChunk;
+  const long long nt = (N + 127) / 128;
   auto up = [](long long x) { return static_cast<size_t>((x + 255) / 256 * 256); };
-  return up(static_cast<long long>(BH) * N * d * 4) + up(static_cast<long long>(BH) * N * 4) +
-         up(static_cast<long long>(BH) * nch * (d * d + d) * 4) + up(static_cast<long long>(BH) * (d * d + d) * 4);
+  return up(static_cast<long long>(BH) * N * d * 2) + up(static_cast<long long>(BH) * nt * d * 4) +
+         up(static_cast<long long>(BH) * d * d * 4) + 2 * up(static_cast<long long>(BH) * d * 4) +
+         up(static_cast<long long>(linear_state_ws_bytes(BH, N, d)));
 }
 
 size_t blend_bwd_ws_bytes(int BH, int N, int d) {
@@ -251,24 +462,50 @@ template <int D>
 static cudaError_t launch_lin_bwd_d(const void* q, const void* k, const void* v, const float* S, const float* z,
                                     const void* dol, int BH, int N, float* dq, float* dk, float* dv, int accumulate,
                                     char* ws, cudaStream_t st) {
+  using L = linb::BwdLayout<D>;
   auto up = [](long long x) { return static_cast<size_t>((x + 255) / 256 * 256); };
-  const int nch = (N + linb::kChunk - 1) / linb::kChunk;
-  float* dnum = reinterpret_cast<float*>(ws);
-  float* dden = reinterpret_cast<float*>(ws + up(static_cast<long long>(BH) * N * D * 4));
-  float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(dden) + up(static_cast<long long>(BH) * N * 4));
-  float* dsz = reinterpret_cast<float*>(reinterpret_cast<char*>(part) + up(static_cast<long long>(BH) * nch * (D * D + D) * 4));
-  const size_t smem = (D * (D + 1) + D + linb::kWarps * 2 * D) * 4;
-  cudaError_t e = cudaFuncSetAttribute(lin_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  const int nt = (N + 127) / 128;
+  char* w = ws;
+  void* dnum = w;                                       // [BH, N, d] bf16
+  w += up(static_cast<long long>(BH) * N * D * 2);
+  float* dz_part = reinterpret_cast<float*>(w);         // [BH, nt, d]
+  w += up(static_cast<long long>(BH) * nt * D * 4);
+  float* dS = reinterpret_cast<float*>(w);              // [BH, d, d]
+  w += up(static_cast<long long>(BH) * D * D * 4);
+  float* dz = reinterpret_cast<float*>(w);              // [BH, d]
+  w += up(static_cast<long long>(BH) * D * 4);
+  float* zq = reinterpret_cast<float*>(w);              // [BH, d] (sum of phi(q); unused)
+  w += up(static_cast<long long>(BH) * D * 4);
+  void* state_ws = w;
+  CUtensorMap mq, mdo, mdn, mk, mv;
+  if (encode_tensor_map_3d_bf16(&mq, q, D, N, BH, 64, 128) != CUDA_SUCCESS ||
+      encode_tensor_map_3d_bf16(&mdo, dol, D, N, BH, 64, 128) != CUDA_SUCCESS ||
+      encode_tensor_map_3d_bf16(&mdn, dnum, D, N, BH, 64, 128) != CUDA_SUCCESS ||
+      encode_tensor_map_3d_bf16(&mk, k, D, N, BH, 64, 128) != CUDA_SUCCESS ||
+      encode_tensor_map_3d_bf16(&mv, v, D, N, BH, 64, 128) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(lin_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(lin_k_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))) != cudaSuccess) return e;
-  const int tpc = 256;
-  const dim3 gt((N + tpc - 1) / tpc, BH);
-  lin_q_kernel<D><<<gt, linb::kWarps * 32, smem, st>>>(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dol),
-                                                       S, z, N, tpc, dq, accumulate, dnum, dden);
-  lin_dsz_kernel<D><<<dim3(nch, BH), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), dnum, dden, N, nch, part);
-  lin_reduce_kernel<<<dim3((D * D + D + 255) / 256, BH), 256, 0, st>>>(part, nch, D * D + D, dsz);
-  lin_k_kernel<D><<<gt, linb::kWarps * 32, smem, st>>>(static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-                                                       dsz, N, tpc, dk, dv, accumulate);
+  if ((e = cudaFuncSetAttribute(lin_bwd_k_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM)) != cudaSuccess)
+    return e;
+  const dim3 grid(nt, BH);
+  lin_bwd_q_kernel<D><<<grid, linb::kThreads, L::SMEM, st>>>(mq, mdo, mdn, S, z, N, dq, accumulate, dz_part);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // dS = phi(Q)^T dnum: the state kernel with (Q, dnum) in the places of (K, V)
+  LinearArgs la{};
+  la.k = q;
+  la.v = dnum;
+  la.kv_state = dS;
+  la.ksum = zq;
+  la.B = BH;
+  la.H = 1;
+  la.N = N;
+  la.d = D;
+  la.ws = state_ws;
+  if ((e = launch_linear_state(la, st)) != cudaSuccess) return e;
+  lin_reduce_kernel<<<dim3((D + 255) / 256, BH), 256, 0, st>>>(dz_part, nt, D, dz);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  lin_bwd_k_kernel<D><<<grid, linb::kThreads, L::SMEM, st>>>(mk, mv, dS, dz, N, dk, dv, accumulate);
   return cudaGetLastError();
 }
 

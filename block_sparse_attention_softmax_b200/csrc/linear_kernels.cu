@@ -81,13 +81,14 @@ struct OutLayout {
   static constexpr uint32_t B_BYTES = (D / 64) * B_CHUNK;    // one of hi / lo
   static constexpr uint32_t T_CHUNK = kLinTok * 128;         // 128 tokens x 64 features
   static constexpr uint32_t T_BYTES = (D / 64) * T_CHUNK;    // one Q or O_s tile
-  static constexpr int NSTG = 2;
+  static constexpr int NSTG = 2;          // Q and O_s stages with the blend
+  static constexpr int NSTG_OL = 4;       // Q stages without it (O_l is staged in the consumed Q stage)
   static constexpr uint32_t OFF_B = 0;
   static constexpr uint32_t OFF_Q = 2 * B_BYTES;
-  static constexpr uint32_t OFF_OS = OFF_Q + NSTG * T_BYTES;
-  static constexpr uint32_t OFF_DEN = OFF_OS + NSTG * T_BYTES;  // [NSTG][4 parts][128 rows] fp32
+  static constexpr uint32_t OFF_OS = OFF_Q + NSTG * T_BYTES;    // = Q stages 2, 3 without the blend
+  static constexpr uint32_t OFF_DEN = OFF_OS + NSTG * T_BYTES;  // [NSTG_OL][4 parts][128 rows] fp32
   static constexpr int ZA_HEADS = 8;                              // z and alpha of up to 8 heads per CTA
-  static constexpr uint32_t OFF_ZA = OFF_DEN + NSTG * 4 * 128 * 4;  // [ZA_HEADS][2][D] fp32
+  static constexpr uint32_t OFF_ZA = OFF_DEN + NSTG_OL * 4 * 128 * 4;  // [ZA_HEADS][2][D] fp32
   static constexpr uint32_t OFF_BAR = OFF_ZA + ZA_HEADS * 2 * D * 4;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
 };
@@ -344,15 +345,21 @@ __global__ void linear_reduce_kernel(const float* __restrict__ part, lin::StateG
 
 // ---------------------------------------------------------------- output + blend
 // Persistent over the same head-major tile list as the state kernel. Per tile
-// of 128 tokens: one warp loads Q and another O_s by TMA into 2-stage rings;
-// the math warps apply phi to Q in place and, four threads per token, form the
-// denominator phi(q_t) . z; one thread issues D[t, :] = phi(Q)[t, :] S_hi +
-// phi(Q)[t, :] S_lo (tcgen05, TMEM accumulator, double buffered), which also
-// frees the Q stage; the math warps then divide, blend with O_s and write O
-// over O_s in the stage, and the O_s warp stores the stage to O by TMA before
-// loading the next O_s into it. z and alpha of the CTA's heads sit in shared
-// memory. The four warps that share TMEM lane quadrant w % 4 split the d
-// columns.
+// of 128 tokens: one warp loads Q by TMA; the math warps apply phi to Q in
+// place and, four threads per token, form the denominator phi(q_t) . z; one
+// thread issues D[t, :] = phi(Q)[t, :] S_hi + phi(Q)[t, :] S_lo (tcgen05, TMEM
+// accumulator, double buffered); the math warps then divide and stage the
+// output in shared memory, from where the store warp writes it by TMA.
+//   BLEND    2 Q stages (freed by the MMA) and 2 O_s stages: the store warp
+//            loads O_s into a stage, the math warps blend alpha O_s + (1 -
+//            alpha) O_l over it, and the store warp writes it to O before
+//            loading the next O_s into it.
+//   !BLEND   O_l only, 4 Q stages: the math warps write O_l over the consumed
+//            Q stage (the MMA that read it has completed), and the store warp
+//            frees the stage for the next Q once its store has read it. The
+//            deeper ring keeps two Q tiles in flight per SM.
+// z and alpha of the CTA's heads sit in shared memory. The four warps that
+// share TMEM lane quadrant w % 4 split the d columns.
 constexpr int kOutMathWarps = 16;
 constexpr int kOsWarp = 2 + kOutMathWarps;
 constexpr int kOutThreads = 32 * (kOsWarp + 1);
@@ -385,21 +392,21 @@ __device__ __forceinline__ void build_head_operand(uint8_t* smem, const float* _
   fence_proxy_async_smem();
 }
 
-template <int D>
+template <int D, bool BLEND>
 __global__ void __launch_bounds__(kOutThreads, 1)
     linear_out_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmOs,
                       const __grid_constant__ CUtensorMap tmO,
                       const float* __restrict__ kv_state, const float* __restrict__ ksum,
-                      const float* __restrict__ alpha, int H, int N, lin::StateGeom geo,
-                      int blend) {
+                      const float* __restrict__ alpha, int H, int N, lin::StateGeom geo) {
   using L = lin::OutLayout<D>;
-  constexpr int NS = L::NSTG;
+  constexpr int NS = BLEND ? L::NSTG : L::NSTG_OL;   // Q stages (and, with the blend, O_s stages)
+  constexpr bool blend = BLEND;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = lin::align1k(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bars;                  // [NS] Q landed
-  uint64_t* q_empty = bars + NS;            // [NS] MMA on that Q completed
-  uint64_t* os_full = bars + 2 * NS;        // [NS] O_s landed (or, without blend, the stage is free)
+  uint64_t* q_empty = bars + NS;            // [NS] Q stage free: MMA completed (blend) or O_l store read it
+  uint64_t* os_full = bars + 2 * NS;        // [NS] O_s landed (blend only)
   uint64_t* o_ready = bars + 3 * NS;        // [NS] O written into the stage (math warps)
   uint64_t* phi_done = bars + 4 * NS;       // [NS] phi and denominators ready (math warps)
   uint64_t* acc_full = bars + 5 * NS;       // [2]
@@ -458,6 +465,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     // ------------------------------------------------------------ Q producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
+      int issued = 0;
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % NS;
         if (!mbar_wait(&q_empty[s], ((i / NS) & 1) ^ 1, abort_flag)) break;
@@ -467,13 +475,35 @@ __global__ void __launch_bounds__(kOutThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(smem + L::OFF_Q + s * L::T_BYTES + c * L::T_CHUNK, &tmQ, &q_full[s], c * 64, row, bh);
+        issued = i + 1;
       }
+      // loads still in flight after an early stop land before the CTA gives up its shared memory
+      for (int k = 1; k <= NS && k <= issued; ++k) mbar_drain(&q_full[(issued - k) % NS], ((issued - k) / NS) & 1);
+    }
+  } else if (warp == kOsWarp && !BLEND) {
+    // ------------------------------------------------------------ O_l stores from the Q stages
+    if (lane == 0) {
+      tma_prefetch_desc(&tmO);
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % NS;
+        if (!mbar_wait(&o_ready[s], (j / NS) & 1, abort_flag)) break;
+        const int t = t0 + j;
+        const int row = (t % geo.tph) * lin::kLinTok, bh = t / geo.tph;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_store_3d(&tmO, smem + L::OFF_Q + s * L::T_BYTES + c * L::T_CHUNK, c * 64, row, bh);
+        bulk_commit();
+        // every store but this one has read its stage: hand the previous stage back
+        bulk_wait_read<1>();
+        if (j > 0) mbar_arrive(&q_empty[(j - 1) % NS]);
+      }
+      bulk_wait_all();
     }
   } else if (warp == kOsWarp) {
     // ------------------------------------------------------------ O_s loads, O stores
     // Stage s of tile i: once the math warps have written O of tile i - NS
     // into it, store that tile by TMA, wait until the store has read the
-    // stage, then load O_s of tile i (or, without blend, just release it).
+    // stage, then load O_s of tile i.
     if (lane == 0) {
       if (blend) tma_prefetch_desc(&tmOs);
       tma_prefetch_desc(&tmO);
@@ -533,7 +563,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
           umma_ss(tm + ab * 128, a, sw128_desc(blo + kk * 2048u, L::B_CHUNK, 1024), idesc, 1u);
         }
         tc_commit(&acc_full[ab]);
-        tc_commit(&q_empty[s]);
+        if (BLEND) tc_commit(&q_empty[s]);
       }
     }
   } else {
@@ -555,7 +585,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       const int tok = (t % geo.tph) * lin::kLinTok + row;
       if (!mbar_wait(&acc_full[ab], (j >> 1) & 1, abort_flag)) return false;
       if (!mbar_wait(&phi_done[s], (j / NS) & 1, abort_flag)) return false;   // denominators visible
-      if (!mbar_wait(&os_full[s], (j / NS) & 1, abort_flag)) return false;    // O_s in, stage free
+      if (BLEND && !mbar_wait(&os_full[s], (j / NS) & 1, abort_flag)) return false;   // O_s in, stage free
       tc_fence_after();
       uint32_t x0[32];
       if (HC == 32) {
@@ -570,7 +600,8 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       const float inv = 1.f / ((dj[row] + dj[128 + row]) + (dj[256 + row] + dj[384 + row]));
       (void)tok;   // rows past N are clipped by the TMA store
       {
-        uint8_t* osrow = smem + L::OFF_OS + s * L::T_BYTES;
+        // the output stage: O_s's (blend) or the consumed Q stage (O_l only)
+        uint8_t* osrow = smem + (BLEND ? L::OFF_OS : L::OFF_Q) + s * L::T_BYTES;
         const float* al = za_smem ? za + ((bh - h_first) * 2 + 1) * D : alpha + static_cast<long long>(bh % H) * D;
 #pragma unroll
         for (int j2 = 0; j2 < HU; ++j2) {
@@ -696,14 +727,15 @@ static cudaError_t out_d(const LinearArgs& a, cudaStream_t st) {
   const lin::StateGeom geo = lin::state_geom(BH, a.N, lin::sm_count());
   CUtensorMap mq, mos, mo;
   if (encode_tensor_map_3d_bf16(&mq, a.q, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  const int blend = a.o_s != nullptr;
+  const bool blend = a.o_s != nullptr;
   if (encode_tensor_map_3d_bf16(&mos, blend ? a.o_s : a.q, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   if (encode_tensor_map_3d_bf16(&mo, a.o, D, a.N, BH, 64, lin::kLinTok) != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(linear_out_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+  auto kern = blend ? linear_out_kernel<D, true> : linear_out_kernel<D, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  linear_out_kernel<D><<<geo.grid, kOutThreads, L::SMEM, st>>>(
-      mq, mos, mo, a.kv_state, a.ksum, blend ? a.alpha : nullptr, a.H, a.N, geo, blend);
+  kern<<<geo.grid, kOutThreads, L::SMEM, st>>>(mq, mos, mo, a.kv_state, a.ksum, blend ? a.alpha : nullptr, a.H,
+                                               a.N, geo);
   return cudaGetLastError();
 }
 

@@ -282,13 +282,27 @@ namespace {
 
 // Shared body of sa_sparse_attn_fwd and sa_sparse_attn_blend_fwd (o_l and
 // alpha both null, or both given).
-int sparse_attn(const char* fn, const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H,
+struct Fp8Scales {
+  const float* q = nullptr;
+  const float* k = nullptr;
+  const float* v = nullptr;
+};
+
+int sparse_attn(const char* fn, const void* q, const void* k, const void* v, int B, int H,
                 int N, int d, int bq, int bk, const int32_t* kv_idx, const int32_t* kv_cnt,
                 const uint8_t* ext_mask, double scale, const uint16_t* o_l, const float* alpha,
-                uint16_t* o, float* lse_opt, void* workspace, size_t ws_bytes, void* stream) {
+                uint16_t* o, float* lse_opt, void* workspace, size_t ws_bytes, void* stream,
+                const Fp8Scales* f8 = nullptr) {
   int rc = check_shape(B, H, N, d, bq, bk);
   if (rc) return rc;
   if (!q || !k || !v || !o) return fail(SA_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
+  if (f8) {
+    if (d != 128) return fail(SA_ERR_UNSUPPORTED, "%s: the low-bit forward needs d = 128 (got %d)", fn, d);
+    if (!f8->q || !f8->k || !f8->v) return fail(SA_ERR_INVALID_ARG, "%s: null scale pointer", fn);
+    const void* sp[] = {f8->q, f8->k, f8->v};
+    for (const void* p : sp)
+      if (!aligned16(p)) return fail(SA_ERR_ALIGN, "%s: pointers must be 16-byte aligned", fn);
+  }
   const bool lists = kv_idx && kv_cnt;
   if (lists == (ext_mask != nullptr) || (!lists && (kv_idx || kv_cnt)))
     return fail(SA_ERR_INVALID_ARG, "%s: give exactly one of (kv_idx, kv_cnt) or ext_mask", fn);
@@ -317,6 +331,12 @@ int sparse_attn(const char* fn, const uint16_t* q, const uint16_t* k, const uint
   }
   AttnArgs a{q, k, v, o, lse_opt, idx, cnt, BH, N, d, bq, bk, nqb, nkb,
              static_cast<float>(scale * 1.4426950408889634), 0, o_l, alpha, H};
+  if (f8) {
+    a.fp8 = 1;
+    a.q_scale = f8->q;
+    a.k_scale = f8->k;
+    a.v_scale = f8->v;
+  }
   cudaError_t e = launch_sparse_attn(a, st);
   return e == cudaSuccess ? SA_OK : cuda_fail(e, fn);
 }
@@ -339,6 +359,29 @@ int sa_sparse_attn_blend_fwd(const uint16_t* q, const uint16_t* k, const uint16_
   if (!o_l || !alpha) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_blend_fwd: o_l and alpha are required");
   return sparse_attn("sa_sparse_attn_blend_fwd", q, k, v, B, H, N, d, bq, bk, kv_idx, kv_cnt, ext_mask,
                      scale, o_l, alpha, o, lse_opt, workspace, ws_bytes, stream);
+}
+
+int sa_quantize_fp8(const uint16_t* x, int B, int H, int N, int d, uint8_t* x8, float* scale, void* stream) {
+  if (B <= 0 || H <= 0 || N <= 0) return fail(SA_ERR_INVALID_ARG, "B, H and N must be positive (got %d, %d, %d)", B, H, N);
+  if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "head dim %d unsupported (64 or 128)", d);
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH > 65535) return fail(SA_ERR_UNSUPPORTED, "B*H = %lld exceeds 65535", BH);
+  if (BH * N * d >= (1LL << 40)) return fail(SA_ERR_UNSUPPORTED, "tensor too large");
+  if (!x || !x8 || !scale) return fail(SA_ERR_INVALID_ARG, "sa_quantize_fp8: null pointer");
+  if (!aligned16(x) || !aligned16(x8) || !aligned16(scale))
+    return fail(SA_ERR_ALIGN, "sa_quantize_fp8: pointers must be 16-byte aligned");
+  cudaError_t e = launch_quantize_fp8(x, BH, static_cast<long long>(N) * d, x8, scale, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "sa_quantize_fp8");
+}
+
+int sa_sparse_attn_fp8_fwd(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* q_scale,
+                           const float* k_scale, const float* v_scale, int B, int H, int N, int d, int bq,
+                           int bk, const int32_t* kv_idx, const int32_t* kv_cnt, const uint8_t* ext_mask,
+                           double scale, const uint16_t* o_l_opt, const float* alpha_opt, uint16_t* o,
+                           float* lse_opt, void* workspace, size_t ws_bytes, void* stream) {
+  const Fp8Scales f8{q_scale, k_scale, v_scale};
+  return sparse_attn("sa_sparse_attn_fp8_fwd", q8, k8, v8, B, H, N, d, bq, bk, kv_idx, kv_cnt, ext_mask, scale,
+                     o_l_opt, alpha_opt, o, lse_opt, workspace, ws_bytes, stream, &f8);
 }
 
 int sa_dense_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H, int N,

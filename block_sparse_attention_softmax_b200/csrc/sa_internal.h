@@ -80,8 +80,18 @@ struct AttnArgs {
   const void* o_l = nullptr;
   const float* alpha = nullptr;
   int H = 1;
+  // low-bit form: q, k, v are E4M3 bytes with one fp32 scale per (batch, head)
+  // each (d = 128 only)
+  int fp8 = 0;
+  const float* q_scale = nullptr;
+  const float* k_scale = nullptr;
+  const float* v_scale = nullptr;
 };
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t st);
+// Per-slice E4M3 quantisation of BH slices of per_slice bf16 values (a multiple
+// of 8): x8 codes, scale[BH] = amax / 448 (1 for an all-zero slice).
+cudaError_t launch_quantize_fp8(const void* x, long long BH, long long per_slice, uint8_t* x8, float* scale,
+                                cudaStream_t st);
 
 struct LinearArgs {
   const void* q;

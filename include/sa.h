@@ -142,6 +142,38 @@ int sa_sparse_attn_blend_fwd(const uint16_t* q, const uint16_t* k, const uint16_
                              uint16_t* o, float* lse_opt,
                              void* workspace, size_t ws_bytes, void* stream);
 
+/* Low-bit forward (SLA2 提案手法 ③: the forward pass computes with queries,
+ * keys and values quantised to a low-bit format; the pages name neither the
+ * format nor the scale granularity).
+ *
+ * sa_quantize_fp8: for each (batch, head) slice of x [B, H, N, d] bf16,
+ *   amax = max |x|, scale = amax / 448 and r = 448 / amax in fp32 (both 1 for
+ *   an all-zero slice), x8 = E4M3(x * r) with the product rounded to fp32 and
+ *   then to E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; round
+ *   to nearest even, saturating at +-448). Outputs: x8 [B, H, N, d] bytes,
+ *   scale [B * H] fp32. d = 64 or 128; pointers 16-byte aligned. Launches a
+ *   memset and three kernels on `stream`.
+ *
+ * sa_sparse_attn_fp8_fwd: the sparse attention of sa_sparse_attn_fwd on
+ *   E4M3 inputs, O_s = softmax(scale * (s_q q8) . (s_k k8)) (s_v v8) over the
+ *   kept tiles, with one fp32 scale per (batch, head) for each of q8, k8 and
+ *   v8 (as sa_quantize_fp8 writes them; positive and finite). Both products
+ *   run on E4M3 tensor-core operands with fp32 accumulation; the softmax is
+ *   fp32 and P is rounded to E4M3 for the second product. d must be 128
+ *   (SA_ERR_UNSUPPORTED otherwise). o_l_opt and alpha_opt (both or neither)
+ *   blend the linear branch into the epilogue as sa_sparse_attn_blend_fwd
+ *   does. Lists, mask, workspace, outputs and errors otherwise as
+ *   sa_sparse_attn_fwd. */
+int sa_quantize_fp8(const uint16_t* x, int B, int H, int N, int d, uint8_t* x8, float* scale,
+                    void* stream);
+int sa_sparse_attn_fp8_fwd(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
+                           const float* q_scale, const float* k_scale, const float* v_scale,
+                           int B, int H, int N, int d, int bq, int bk,
+                           const int32_t* kv_idx, const int32_t* kv_cnt, const uint8_t* ext_mask,
+                           double scale, const uint16_t* o_l_opt, const float* alpha_opt,
+                           uint16_t* o, float* lse_opt, void* workspace, size_t ws_bytes,
+                           void* stream);
+
 /* Dense attention through the same kernel, every tile kept (the comparison
  * point for the sparse speed-up). */
 int sa_dense_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,

@@ -104,3 +104,49 @@ def sample_rows(n_qb, bq, N, kv_cnt, rng, n_random=4):
     lane quadrants and both column halves of each sampled tile are compared."""
     blocks = sample_blocks(n_qb, kv_cnt, rng, n_random)
     return np.concatenate([np.arange(b * bq, min(N, (b + 1) * bq)) for b in blocks]).astype(np.int64)
+
+
+def fp8_p_rounding_bound(q, k, v, mask, bq, bk, scale=None, rows=None):
+    """Per-element bound on how far the low-bit attention may move from the
+    oracle's (masked attention on the dequantised E4M3 inputs) through its own
+    roundings: P rounded to E4M3 (within 2^-4 of P in the normal range, 2^-10
+    absolute below it; P is normalised by the unrounded row sum), O rounded to
+    bf16 (2^-9 relative), plus 1e-4 for fp32 accumulation.
+
+    Inputs are one head's bf16 values as float64 [N, d]; returns [len(rows), d].
+    """
+    N, d = q.shape
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    qd, kd, vd = (c * s for c, s in (oracle.quantize_fp8_head(t) for t in (q, k, v)))
+    rows = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
+    bound = np.zeros((rows.shape[0], d))
+    for qb in np.unique(rows // bq):
+        at = np.nonzero(rows // bq == qb)[0]
+        kept = np.nonzero(mask[qb])[0]
+        if kept.shape[0] == 0:
+            continue
+        keys = np.concatenate([np.arange(kb * bk, min(N, (kb + 1) * bk)) for kb in kept])
+        logits = scale * (qd[rows[at]] @ kd[keys].T)
+        p = np.exp(logits - logits.max(axis=1, keepdims=True))
+        l = p.sum(axis=1, keepdims=True)
+        av = np.abs(vd[keys])
+        o = np.abs(p @ vd[keys]) / l
+        bound[at] = (2.0 ** -4 * (p @ av) + 2.0 ** -10 * av.sum(axis=0)[None, :]) / l + 2.0 ** -9 * o + 1e-4
+    return bound
+
+
+def assert_within_bound(gpu, ref, bound, what, mean_abs=MEAN_ABS, mean_frac=0.15):
+    """Every element within its bound, and the mean error within mean_frac of
+    the mean bound or mean_abs, whichever is larger: the bound assumes every
+    rounding error points the same way, while rounding errors of independent
+    weights largely cancel (a CPU simulation of the E4M3 rounding of P on
+    unit-variance rows gives a mean error of 0.05 of the mean bound), so a
+    systematic fault shows in the mean long before it reaches the bound."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    err = np.abs(gpu - np.asarray(ref, dtype=np.float64))
+    assert np.isfinite(gpu).all(), f"{what}: non-finite values"
+    worst = np.unravel_index(np.argmax(err - bound), err.shape)
+    assert (err <= bound).all(), f"{what}: err {err[worst]:.3e} > bound {bound[worst]:.3e} at {worst}"
+    lim = max(mean_abs, mean_frac * float(bound.mean()))
+    assert err.mean() <= lim, f"{what}: mean abs err {err.mean():.3e} > {lim:.3e}"
+    return float(err.max()), float(err.mean())

@@ -130,3 +130,22 @@ def test_permutation_entry_points_validate_before_launch(lib):
     assert lib.sa_permute_tokens(fake, fake, 1, 1, 64, 96, 0, P(0x2000), None) == -2
     assert lib.sa_select_mask(fake, 1, 1, 4, 20000, 0.1, 0.9, fake, fake, None, None) == -2
     assert lib.sa_tile_heatmap(fake, fake, 1, 1, 128, 64, 64, 64, 0.0, fake, -1, fake, None, None) == -1
+
+
+def test_low_bit_entry_points_validate_before_launch(lib):
+    fake, other = P(0x1000), P(0x2000)
+    # quantiser: shape, null and alignment checks
+    assert lib.sa_quantize_fp8(fake, 1, 1, 64, 96, other, fake, None) == -2       # d unsupported
+    assert lib.sa_quantize_fp8(fake, 0, 1, 64, 128, other, fake, None) == -1      # B < 1
+    assert lib.sa_quantize_fp8(None, 1, 1, 64, 128, other, fake, None) == -1      # null input
+    assert lib.sa_quantize_fp8(P(0x1001), 1, 1, 64, 128, other, fake, None) == -3  # misaligned
+    # low-bit attention: d = 128 only, scales required, lists xor mask
+    args = (fake, fake, fake, fake, fake, fake)
+    assert lib.sa_sparse_attn_fp8_fwd(*args, 1, 1, 256, 64, 128, 64, fake, fake, None, 0.0, None, None,
+                                      other, None, None, 0, None) == -2
+    assert lib.sa_sparse_attn_fp8_fwd(fake, fake, fake, None, fake, fake, 1, 1, 256, 128, 128, 64, fake, fake,
+                                      None, 0.0, None, None, other, None, None, 0, None) == -1
+    assert lib.sa_sparse_attn_fp8_fwd(*args, 1, 1, 256, 128, 128, 64, None, None, None, 0.0, None, None,
+                                      other, None, None, 0, None) == -1
+    assert lib.sa_sparse_attn_fp8_fwd(*args, 1, 1, 256, 128, 128, 64, fake, fake, None, 0.0, fake, None,
+                                      other, None, None, 0, None) == -1            # o_l without alpha
