@@ -35,13 +35,15 @@ DEFAULT_WORKLOAD = "wan14b_720p"
 METRIC = "sparse_attn_effective_tflops"
 
 
-# DRAM traffic of sparse_attn_kernel from one `ncu --set full` capture of the
-# 1.3B-480p-shaped workload, scaled to the benchmarked one by B*H*N*d (the
-# kernel's DRAM traffic is Q, K, V and O sized). `sources_sha` pins the kernel sources the counters belong to:
-# once they change, traffic is reported as null until a new capture is made.
+# DRAM traffic of one sparse_attn_kernel launch (bf16, blend in the epilogue)
+# on the 14B-720p-shaped workload, from an ncu capture of dram__bytes_read.sum
+# and dram__bytes_write.sum (one pass) of the bench's own launch; for another
+# workload it is scaled by B*H*N*d. `sources_sha` pins the kernel sources the
+# counters belong to: once they change, traffic is reported as null until a
+# new capture is made.
 ATTN_TRAFFIC_CAPTURE = {
-    "workload": "wan13b_480p", "dram_bytes_read": 302507008, "dram_bytes_write": 82581760,
-    "sources_sha": "02bd3a6c1943bcd8",
+    "workload": "wan14b_720p", "dram_bytes_read": 3482988800, "dram_bytes_write": 764509440,
+    "sources_sha": "f4d0cca2e28e24f7",
     "sources": ("attn_kernel.cu", "sa_device.cuh"),
 }
 
@@ -397,7 +399,7 @@ def run_ours(args, wl, rank, world, local):
                      "peak": bf16, "unit": "TFLOP/s", "frac": round(achieved / bf16, 4),
                      "peak_source": f"{src} bf16 burst", "traffic": attn_traffic(wl),
                      "traffic_unit": "bytes per launch",
-                     "traffic_note": "ncu dram read+write of a smaller capture, scaled by B*H*N*d"},
+                     "traffic_note": "ncu dram read+write of this launch on the 14B-720p workload (scaled by B*H*N*d for others)"},
         "mask_builder_roofline": {"bound": "hbm", "achieved": round(mask_bytes / (mask_ms * 1e-3) / 1e9, 1),
                                   "peak": hbm, "unit": "GB/s", "frac": round(mask_bytes / (mask_ms * 1e-3) / 1e9 / hbm, 4),
                                   "bytes_per_call": mask_bytes,
