@@ -99,7 +99,8 @@ def run_config(wl, world):
     return {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d,
             "block": f"{wl.bq}x{wl.bk}", "topk": wl.topk, "topp": wl.topp,
             "linear_branch": wl.linear, "parallelism": f"replica x{world}",
-            "l2": "inputs larger than L2 (each tensor >= 774 MB); no flush"}
+            "l2": (f"inputs larger than L2 (each tensor {wl.B * wl.H * wl.N * wl.d * 2 / 1e6:.0f} MB); no flush"
+                   if wl.B * wl.H * wl.N * wl.d * 2 > 126e6 else "inputs smaller than L2; no flush")}
 
 
 def stats(ms):
@@ -684,7 +685,7 @@ def run_reference(args, wl):
 
 
 REF_HEADS = 2          # heads per reference-arm step (a few seconds of CPU work each)
-BASELINE_HEADS = 8     # heads of the cpu_baseline sample (about 10 s of CPU work)
+CPU_SAMPLE_HEADS = 8     # heads of the cpu_baseline sample (about 10 s of CPU work)
 
 
 def _head_inputs(wl, n):
@@ -706,10 +707,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the per-workload measurements of the other four configurations")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only the first H heads of the workload (small cases for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     wl = WORKLOADS[args.workload]
+    if args.heads > 0:
+        from dataclasses import replace
+        wl = replace(wl, H=min(args.heads, wl.H))
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
             return
@@ -726,15 +732,15 @@ def main():
         res["per_workload"] = run_per_workload(args, dev)
     if rank == 0:
         if not args.no_cpu_baseline:
-            x = _head_inputs(wl, BASELINE_HEADS)
-            sec, desc, cores = oracle_step_estimate(wl, x, BASELINE_HEADS)
+            x = _head_inputs(wl, CPU_SAMPLE_HEADS)
+            sec, desc, cores = oracle_step_estimate(wl, x, CPU_SAMPLE_HEADS)
             res["cpu_baseline"] = {"value": round(dense_flops(wl) / sec / 1e12, 6), "unit": "TFLOP/s",
                                    "cores": cores, "kind": "oracle", "sample": desc,
                                    "ms_per_step": round(sec * 1e3, 1), "extrapolated": True}
             try:
                 from threadpoolctl import threadpool_limits
                 with threadpool_limits(1):
-                    sec1, _, _ = oracle_step_estimate(wl, x, BASELINE_HEADS)
+                    sec1, _, _ = oracle_step_estimate(wl, x, CPU_SAMPLE_HEADS)
                 res["cpu_baseline"]["one_thread"] = {"value": round(dense_flops(wl) / sec1 / 1e12, 6),
                                                      "ms_per_step": round(sec1 * 1e3, 1), "cores": 1}
             except ImportError:

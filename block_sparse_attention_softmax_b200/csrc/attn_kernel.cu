@@ -258,6 +258,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tmem_slot;
+  // the set-up above may overlap the previous kernel in the stream; every
+  // input (lists, Q, K, V, O_l) is read after this
+  grid_dep_wait();
+  grid_dep_trigger();
 
   if (warp == 0 || warp == kVWarp) {
     // ------------------------------------------------------------ producers
@@ -720,8 +724,7 @@ static cudaError_t launch_d(const AttnArgs& a, cudaStream_t st) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long items = static_cast<long long>(a.BH) * a.nqb;
   const int grid = static_cast<int>(items < sms ? items : sms);
-  sparse_attn_kernel<D, F8><<<grid, attn::kThreads, L::SMEM, st>>>(mq, mk, mv, a);
-  return cudaGetLastError();
+  return launch_pdl(sparse_attn_kernel<D, F8>, dim3(grid), dim3(attn::kThreads), L::SMEM, st, mq, mk, mv, a);
 }
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t st) {

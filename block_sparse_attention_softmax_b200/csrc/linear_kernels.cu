@@ -439,6 +439,9 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
+  // the state (and O_s) come from earlier kernels in the stream
+  grid_dep_wait();
+  grid_dep_trigger();
   build_head_operand<D>(smem, kv_state, t0 / geo.tph, threadIdx.x, blockDim.x);
   // z and alpha of this CTA's heads (from global memory if there are more
   // heads than slots)
@@ -734,9 +737,8 @@ static cudaError_t out_d(const LinearArgs& a, cudaStream_t st) {
   auto kern = blend ? linear_out_kernel<D, true> : linear_out_kernel<D, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<geo.grid, kOutThreads, L::SMEM, st>>>(mq, mos, mo, a.kv_state, a.ksum, blend ? a.alpha : nullptr, a.H,
-                                               a.N, geo);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(geo.grid), dim3(kOutThreads), L::SMEM, st, mq, mos, mo, a.kv_state, a.ksum,
+                    blend ? a.alpha : nullptr, a.H, a.N, geo);
 }
 
 cudaError_t launch_linear_out(const LinearArgs& a, cudaStream_t st) {

@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
                                                    float* __restrict__ k_pool, SliceOut sl) {
   constexpr int LPR = D / 8;        // lanes per row
   constexpr int RPI = 32 / LPR;     // rows per warp step
+  grid_dep_trigger();               // the scoring kernel may begin its set-up
   const int lane = threadIdx.x & 31;
   const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nq = static_cast<long long>(BH) * nqb;
@@ -328,13 +329,8 @@ __global__ void __launch_bounds__(I8Layout<D, MODE>::THREADS, 1) score_i8_kernel
   using L = I8Layout<D, MODE>;
   if constexpr (MODE == kScoreWrite) {
     // filtered launch with nothing handed back: leave before any setup
+    grid_dep_wait();
     if (cb.fb_cnt && *reinterpret_cast<volatile const int*>(cb.fb_cnt) == 0) return;
-  }
-  if constexpr (MODE == kScoreStats) {
-    // clear the hand-back state of this call (read only by later launches)
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < cb.n_tile_flags; i += gridDim.x * blockDim.x)
-      cb.tile_flag[i] = 0;
-    if (blockIdx.x == 0 && threadIdx.x == 0) *cb.fb_cnt = 0;
   }
   extern __shared__ __align__(16) uint8_t smem_raw[];
   // 1024-byte aligned (swizzle atoms), derived from the shared array so that
@@ -375,6 +371,15 @@ __global__ void __launch_bounds__(I8Layout<D, MODE>::THREADS, 1) score_i8_kernel
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tmem_slot;
+  // set-up above overlaps the previous kernel's tail; inputs are read below
+  if constexpr (MODE != kScoreWrite) grid_dep_wait();
+  grid_dep_trigger();
+  if constexpr (MODE == kScoreStats) {
+    // clear the hand-back state of this call (read only by later launches)
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < cb.n_tile_flags; i += gridDim.x * blockDim.x)
+      cb.tile_flag[i] = 0;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *cb.fb_cnt = 0;
+  }
 
   // work item -> (head, query tile, key range, first and end key tile)
   auto decode = [&](int item, int& bh, int& qt, int& kr, int& kt0, int& kt1) {
@@ -1142,6 +1147,7 @@ __global__ void __launch_bounds__(kSelFastWarps * 32, 4) select_fast_kernel(
   __shared__ uint32_t ckey_all[kSelFastWarps][kRegCandMax];
   __shared__ int cidx_all[kSelFastWarps][kRegCandMax];
   __shared__ float e_all[kSelFastWarps][32 * KPL];
+  grid_dep_wait();
   const int warp = threadIdx.x >> 5;
   const int nr = n_rows_dev ? *n_rows_dev : n_rows;
   for (int ri = blockIdx.x * kSelFastWarps + warp; ri < nr; ri += gridDim.x * kSelFastWarps) {
@@ -1160,9 +1166,8 @@ static cudaError_t launch_select_fast(const float* s, long long s_ld, int n_rows
                                       const int* rows, const int* n_rows_dev, int grid_cap, cudaStream_t st) {
   const int want = (n_rows + kSelFastWarps - 1) / kSelFastWarps;
   const int grid = want < grid_cap ? want : grid_cap;
-  select_fast_kernel<KPL><<<grid, kSelFastWarps * 32, 0, st>>>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt,
-                                                               mask, rows, n_rows_dev);
-  return cudaGetLastError();
+  return launch_pdl(select_fast_kernel<KPL>, dim3(grid), dim3(kSelFastWarps * 32), 0, st, s, s_ld, n_rows, nkb, k_sel,
+                    topp, kv_idx, kv_cnt, mask, rows, n_rows_dev);
 }
 
 // ---------------------------------------------------------------- selection, long rows
@@ -1431,6 +1436,7 @@ __global__ void __launch_bounds__(kSelWarpsMax * 32) select_long_kernel(
     int* __restrict__ kv_idx, int* __restrict__ kv_cnt, uint8_t* __restrict__ mask, int slice,
     const int* __restrict__ rows, const int* __restrict__ n_rows_dev) {
   extern __shared__ __align__(16) uint8_t sm_long[];
+  grid_dep_wait();
   const int warp = threadIdx.x >> 5;
   const int wpc = blockDim.x >> 5;
   float* xs = reinterpret_cast<float*>(sm_long + static_cast<size_t>(warp) * slice);
@@ -1828,6 +1834,8 @@ __global__ void __launch_bounds__(kCandSelWarps * 32) select_cand_kernel(
     CandSel cs, int n_rows, int nkb, int k_sel, double topp, int* __restrict__ kv_idx,
     int* __restrict__ kv_cnt, uint8_t* __restrict__ mask) {
   extern __shared__ __align__(16) uint32_t cand_smem[];
+  grid_dep_wait();
+  grid_dep_trigger();
   const int warp = threadIdx.x >> 5;
   const int W = (nkb + 31) >> 5;
   uint32_t* keep = cand_smem + static_cast<size_t>(warp) * 2 * W;
@@ -1925,8 +1933,8 @@ static cudaError_t launch_i8(const CUtensorMap& ma, const CUtensorMap& mb, const
   using L = I8Layout<D, MODE>;
   cudaError_t e = cudaFuncSetAttribute(score_i8_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  score_i8_kernel<D, MODE><<<il.grid, L::THREADS, L::SMEM, st>>>(ma, mb, sl.q_ex, sl.k_ex, il.w, scale, s, s_ld, cb);
-  return cudaGetLastError();
+  return launch_pdl(score_i8_kernel<D, MODE>, dim3(il.grid), dim3(L::THREADS), L::SMEM, st, ma, mb, sl.q_ex, sl.k_ex,
+                    il.w, scale, s, s_ld, cb);
 }
 
 cudaError_t launch_scores_i8(const SliceOut& sl, int BH, int nqb, int nkb, int d, double scale,
@@ -1963,9 +1971,8 @@ cudaError_t launch_select(const float* s, long long s_ld, int n_rows, int nkb, i
   const int want = (n_rows + wpc - 1) / wpc;
   const int cap16 = rows ? 148 * 16 : 65535 * 16;
   const int grid = want < cap16 ? want : cap16;
-  select_long_kernel<<<grid, wpc * 32, smem, st>>>(s, s_ld, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask, slice,
-                                                   rows, n_rows_dev);
-  return cudaGetLastError();
+  return launch_pdl(select_long_kernel, dim3(grid), dim3(wpc * 32), smem, st, s, s_ld, n_rows, nkb, k_sel, topp, kv_idx,
+                    kv_cnt, mask, slice, rows, n_rows_dev);
 }
 
 // z with P(Z > z) = f for a standard normal Z (bisection on erfc, host fp64).
@@ -2014,8 +2021,8 @@ static cudaError_t launch_select_cand(const CandSel& cs, int n_rows, int nkb, in
   if (e != cudaSuccess) return e;
   const int want = (n_rows + kCandSelWarps - 1) / kCandSelWarps;
   const int grid = want < 148 * 64 ? want : 148 * 64;
-  select_cand_kernel<CPL><<<grid, kCandSelWarps * 32, smem, st>>>(cs, n_rows, nkb, k_sel, topp, kv_idx, kv_cnt, mask);
-  return cudaGetLastError();
+  return launch_pdl(select_cand_kernel<CPL>, dim3(grid), dim3(kCandSelWarps * 32), smem, st, cs, n_rows, nkb, k_sel,
+                    topp, kv_idx, kv_cnt, mask);
 }
 
 // The candidate path of the mask builder: approximate row statistics,

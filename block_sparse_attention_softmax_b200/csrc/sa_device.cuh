@@ -124,6 +124,15 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // Wait until every committed bulk store has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Until at most N of this thread's committed bulk groups still read shared memory.
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization (launch_pdl) may start while the kernel before it in the
+// stream is still running: grid_dep_wait() blocks until that kernel has
+// completed and its writes are visible (it returns at once after an ordinary
+// launch), and grid_dep_trigger() lets the next such kernel begin launching
+// once every CTA of this one has issued it (or exited).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 template <int N>
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
 // Wait until every committed bulk store has completed.

@@ -88,6 +88,26 @@ struct AttnArgs {
   const float* v_scale = nullptr;
 };
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t st);
+
+// Launch with programmatic stream serialization: the kernel's CTAs may start
+// (and run their set-up) while the previous kernel in the stream finishes;
+// the kernel itself calls grid_dep_wait() before it touches memory that
+// earlier work writes or reads.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 // Per-slice E4M3 quantisation of BH slices of per_slice bf16 values (a multiple
 // of 8): x8 codes, scale[BH] = amax / 448 (1 for an all-zero slice).
 cudaError_t launch_quantize_fp8(const void* x, long long BH, long long per_slice, uint8_t* x8, float* scale,
