@@ -56,14 +56,18 @@ __device__ __forceinline__ uint32_t tile_unit(int r, int u) {
 }
 
 
-// phi applied in place to a [128 x D] bf16 tile (all 256 threads)
+// phi applied in place to a [128 x D] bf16 tile (all 256 threads). Two threads
+// per row; thread h takes units 4h..4h+3 of the first 64-feature chunk and the
+// other four of the second, so that a quarter-warp's eight 16-byte accesses
+// fall in eight different bank groups of the swizzled rows.
 template <int D>
 __device__ __forceinline__ void phi_tile_inplace(uint8_t* tile, int tid) {
   constexpr int UPT = D / 16;                   // 16-byte units per thread: half a row
-  const int r = tid >> 1, u0 = (tid & 1) * UPT;
+  const int r = tid >> 1, h = tid & 1;
 #pragma unroll
   for (int j = 0; j < UPT; ++j) {
-    uint4* p = reinterpret_cast<uint4*>(tile + linb::tile_unit<D>(r, u0 + j));
+    const int c = j >> 2;
+    uint4* p = reinterpret_cast<uint4*>(tile + linb::tile_unit<D>(r, c * 8 + (j & 3) + 4 * (h ^ c)));
     uint4 w = *p;
     uint32_t* x = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll

@@ -577,7 +577,11 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
     constexpr int HC = D / 4;                 // output columns per group
     constexpr int HU = HC / 8;                // 16-B units per group of a row
-    // transform mapping: token trow, 16-B units [tpart * HU, +HU) of its d range
+    // transform mapping: token trow, four threads per token; thread tpart
+    // takes units tpart and tpart + 4 of each 64-feature chunk, the even rows
+    // of a quarter-warp in one order and the odd rows in the other, so that
+    // the quarter-warp's eight 16-byte accesses fall in eight different bank
+    // groups of the swizzled rows
     const int trow = mt >> 2, tpart = mt & 3;
     bool ok = true;
     int changes = 0;
@@ -655,7 +659,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         float dz = 0.f;
 #pragma unroll
         for (int j2 = 0; j2 < HU; ++j2) {
-          const int uu = tpart * HU + j2;
+          const int uu = (j2 >> 1) * 8 + tpart + 4 * ((j2 & 1) ^ (trow & 1));
           uint4* p = reinterpret_cast<uint4*>(qt + (uu >> 3) * L::T_CHUNK + trow * 128 + (((uu & 7) ^ (trow & 7)) << 4));
           uint4 w = *p;
           uint32_t* x = reinterpret_cast<uint32_t*>(&w);
