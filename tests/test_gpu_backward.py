@@ -92,8 +92,11 @@ def test_sparse_attention_bwd_empty_rows(cuda_lib):
 
 
 def test_linear_and_blend_bwd(cuda_lib):
+    """Tiles of 128 tokens, one CTA per (tile, head): 8 and 3 tiles (ragged),
+    and 128 tiles per head, where dz sums 128 partials and dS comes from the
+    state kernel's split over many CTAs."""
     sa = cuda_lib
-    for (N, d, B) in [(1000, 128, 2), (257, 64, 1)]:
+    for (N, d, B) in [(1000, 128, 2), (257, 64, 1), (16344, 128, 1)]:
         H = 2
         q, k, v = random_qkv(B, H, N, d, seed=N + 1, device=DEV)
         S, z, ol = sa.sa_linear_branch(q, k, v, want_ol=True)
