@@ -585,26 +585,27 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           l_b += s0 + s1;
         }
         if constexpr (F8) {
-          // four E4M3 keys per TMEM column, the lowest key in the lowest byte:
-          // column 2 k + (j4 >> 1) holds keys 8 k + 4 (j4 >> 1) .. + 3, the
-          // 16-bit halves of threads j4 and j4 ^ 1; the 16x128b store writes
-          // column 4 k' + j4 (k = 2 k' + (j4 >> 1)) from the pair whose
-          // j4 >> 1 equals this thread's j4 & 1
-          uint32_t w[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, p[i], 1);
-            w[i] = (j4 & 1) ? (other | (p[i] << 16)) : (p[i] | (other << 16));
-          }
-          const int src = (lane & ~3) | ((j4 & 1) << 1);
+          // Four E4M3 keys per TMEM column, the lowest key in the lowest byte.
+          // Column 2 k + (j4 >> 1) holds keys 8 k + 4 (j4 >> 1) .. + 3: the
+          // 16-bit halves (two keys each) of threads j4 and j4 ^ 1 at index k.
+          // Step 1: the two threads of a pair swap their halves of indices
+          // 2 m and 2 m + 1 in one word; thread j4 keeps index 2 m + (j4 & 1),
+          // i.e. column 4 m + sg with sg = 2 (j4 & 1) + (j4 >> 1).
+          // Step 2: the 16x128b store writes column 4 m + j4 from thread j4,
+          // which thread sg(j4) holds (sg swaps 1 and 2).
+          const int e1 = j4 & 1;
+          const int sg = 2 * e1 + (j4 >> 1);
           uint32_t q8[16];
 #pragma unroll
-          for (int kp = 0; kp < 8; ++kp) {
+          for (int rr = 0; rr < 2; ++rr) {
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-              const uint32_t v0 = __shfl_sync(0xFFFFFFFFu, w[2 * (2 * kp) + rr], src);
-              const uint32_t v1 = __shfl_sync(0xFFFFFFFFu, w[2 * (2 * kp + 1) + rr], src);
-              q8[2 * kp + rr] = (j4 >> 1) ? v1 : v0;
+            for (int m = 0; m < 8; ++m) {
+              const uint32_t lo = p[2 * (2 * m) + rr], hi = p[2 * (2 * m + 1) + rr];
+              const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, lo | (hi << 16), 1);
+              const uint32_t own = e1 ? hi : lo;
+              const uint32_t oth = e1 ? (got >> 16) : (got & 0xFFFFu);
+              const uint32_t word = (j4 & 1) ? (oth | (own << 16)) : (own | (oth << 16));
+              q8[2 * m + rr] = __shfl_sync(0xFFFFFFFFu, word, (lane & ~3) | sg);
             }
           }
           tmem_st_16x128b_x8(tm + lane_addr + tm_s(b), q8);

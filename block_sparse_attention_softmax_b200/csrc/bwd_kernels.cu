@@ -13,7 +13,8 @@
 // bwd_dq_kernel    per query block (the forward's items and lists): for each
 //                  kept tile of two key blocks, S = Q K^T and dP = dO V^T on the
 //                  tensor core into TMEM; 8 warps form dS (bf16, written over S);
-//                  dQ += dS K accumulates in TMEM.
+//                  dQ += dS K accumulates in TMEM. S has two buffers, so S and
+//                  dP of the next tile are computed while the warps form dS.
 // bwd_dkdv_kernel  per tile of two key blocks: the query blocks that keep
 //                  either block (a transposed list with a flag per block, from
 //                  col_lists_kernel), for each S^T = K Q^T and dP^T = V dO^T;
@@ -140,8 +141,11 @@ struct DQLayout : Sizes<D> {
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
 };
 enum {
-  DQ_QFULL = 0, DQ_QEMPTY, DQ_KVFULL, DQ_KVEMPTY = DQ_KVFULL + kStages, DQ_SFULL = DQ_KVEMPTY + kStages,
-  DQ_PFULL, DQ_OFULL, DQ_OEMPTY, DQ_DRAIN, DQ_COUNT
+  DQ_QFULL = 0, DQ_QEMPTY, DQ_KVFULL, DQ_KVEMPTY = DQ_KVFULL + kStages,
+  DQ_SFULL = DQ_KVEMPTY + kStages,   // [2] S and dP of the tile in that S buffer landed
+  DQ_PFULL = DQ_SFULL + 2,           // [2] dS written over that S buffer
+  DQ_DPEMPTY = DQ_PFULL + 2,         // dP read by every compute warp (the next dP may land)
+  DQ_OFULL, DQ_OEMPTY, DQ_DRAIN, DQ_COUNT
 };
 constexpr int kDQThreads = 32 * (2 + kCWarps);
 }  // namespace bwd
@@ -160,7 +164,8 @@ __global__ void __launch_bounds__(bwd::kDQThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = a.BH * a.nqb;
-  constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256;
+  // two S buffers (dS is written over S), one dP buffer, the dQ accumulator
+  constexpr uint32_t TM_S = 0, TM_DP = 256, TM_DQ = 384;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[DQ_QFULL], 1);
@@ -169,8 +174,11 @@ __global__ void __launch_bounds__(bwd::kDQThreads, 1)
       mbar_init(&bars[DQ_KVFULL + i], 1);
       mbar_init(&bars[DQ_KVEMPTY + i], 1);
     }
-    mbar_init(&bars[DQ_SFULL], 1);
-    mbar_init(&bars[DQ_PFULL], kCWarps);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[DQ_SFULL + i], 1);
+      mbar_init(&bars[DQ_PFULL + i], kCWarps);
+    }
+    mbar_init(&bars[DQ_DPEMPTY], kCWarps);
     mbar_init(&bars[DQ_OFULL], 1);
     mbar_init(&bars[DQ_OEMPTY], kCWarps);
     mbar_init(&bars[DQ_DRAIN], 1);
@@ -242,6 +250,33 @@ __global__ void __launch_bounds__(bwd::kDQThreads, 1)
       const uint32_t id2 = idesc_bf16_f32(kBM, 128, false, false);
       const uint32_t id1 = idesc_bf16_f32(kBM, 64, false, false);
       const uint32_t idq = idesc_bf16_f32(kBM, D, false, true);
+      // S and dP of tile t + 1 are issued before the dQ product of tile t, so
+      // they run while the compute warps form dS(t); S alternates between two
+      // buffers, and dP(t + 1) waits until every compute warp has read dP(t).
+      // (tcgen05.mma executes in issue order, so S(t + 2) follows the dQ
+      // product that read dS(t) from the same buffer.)
+      auto issue_s_dp = [&](int g, int cnt, int t) -> bool {
+        const int s = g % kStages, b = g & 1;
+        const int nblk = min(2, cnt - 2 * t);
+        if (!mbar_wait(&bars[DQ_KVFULL + s], (g / kStages) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t id = nblk == 2 ? id2 : id1;
+        const uint64_t kd = kdesc0 + ((s * L::ROWS_BYTES) >> 4), vd = vdesc0 + ((s * L::ROWS_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (((kk >> 2) * L::CHUNK) + (kk & 3) * 32u) >> 4;
+          umma_ss(tm + TM_S + b * 128, qdesc + off, kd + off, id, kk > 0 ? 1u : 0u);
+        }
+        if (g > 0 && !mbar_wait(&bars[DQ_DPEMPTY], (g - 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (((kk >> 2) * L::CHUNK) + (kk & 3) * 32u) >> 4;
+          umma_ss(tm + TM_DP, dodesc + off, vd + off, id, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bars[DQ_SFULL + b]);
+        return true;
+      };
       int g = 0, ii = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
@@ -249,31 +284,20 @@ __global__ void __launch_bounds__(bwd::kDQThreads, 1)
         if (cnt == 0) continue;
         if (!(ok = mbar_wait(&bars[DQ_QFULL], ii & 1, abort_flag))) break;
         const int T = (cnt + 1) / 2;
+        if (!(ok = issue_s_dp(g, cnt, 0))) break;
         for (int t = 0; ok && t < T; ++t, ++g) {
-          const int s = g % kStages;
+          const int s = g % kStages, b = g & 1;
           const int nblk = min(2, cnt - 2 * t);
-          if (!(ok = mbar_wait(&bars[DQ_KVFULL + s], (g / kStages) & 1, abort_flag))) break;
-          tc_fence_after();
-          const uint32_t id = nblk == 2 ? id2 : id1;
-          const uint64_t kd = kdesc0 + ((s * L::ROWS_BYTES) >> 4), vd = vdesc0 + ((s * L::ROWS_BYTES) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (((kk >> 2) * L::CHUNK) + (kk & 3) * 32u) >> 4;
-            umma_ss(tm + TM_S, qdesc + off, kd + off, id, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (((kk >> 2) * L::CHUNK) + (kk & 3) * 32u) >> 4;
-            umma_ss(tm + TM_DP, dodesc + off, vd + off, id, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&bars[DQ_SFULL]);
-          if (!(ok = mbar_wait(&bars[DQ_PFULL], g & 1, abort_flag))) break;
+          if (t + 1 < T && !(ok = issue_s_dp(g + 1, cnt, t + 1))) break;
+          if (!(ok = mbar_wait(&bars[DQ_PFULL + b], (g >> 1) & 1, abort_flag))) break;
           if (t == 0 && !(ok = mbar_wait(&bars[DQ_OEMPTY], (ii & 1) ^ 1, abort_flag))) break;
           tc_fence_after();
           const uint64_t km = kmn0 + ((s * L::ROWS_BYTES) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            if (kk < nblk * 4) umma_ts(tm + TM_DQ, tm + TM_S + kk * 8, km + ((kk * 2048u) >> 4), idq, (t > 0 || kk > 0) ? 1u : 0u);
+            if (kk < nblk * 4)
+              umma_ts(tm + TM_DQ, tm + TM_S + b * 128 + (kk >> 2) * 64 + (kk & 3) * 8, km + ((kk * 2048u) >> 4), idq,
+                      (t > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&bars[DQ_KVEMPTY + s]);
           if (t + 1 == T) {
             tc_commit(&bars[DQ_QEMPTY]);
@@ -310,11 +334,12 @@ __global__ void __launch_bounds__(bwd::kDQThreads, 1)
       if (a.N % 64) tail = __ldg(a.kv_idx + static_cast<long long>(item) * a.nkb + cnt - 1) == a.nkb - 1;
       const int T = (cnt + 1) / 2;
       for (int t = 0; ok && t < T; ++t, ++g) {
-        if (!(ok = mbar_wait(&bars[DQ_SFULL], g & 1, abort_flag))) break;
+        const int b = g & 1;
+        if (!(ok = mbar_wait(&bars[DQ_SFULL + b], (g >> 1) & 1, abort_flag))) break;
         tc_fence_after();
         uint32_t s0[32], s1[32], p0[32], p1[32];
-        tmem_ld32(tm + la + TM_S + half * 64, s0);
-        tmem_ld32(tm + la + TM_S + half * 64 + 32, s1);
+        tmem_ld32(tm + la + TM_S + b * 128 + half * 64, s0);
+        tmem_ld32(tm + la + TM_S + b * 128 + half * 64 + 32, s1);
         tmem_ld32(tm + la + TM_DP + half * 64, p0);
         tmem_ld32(tm + la + TM_DP + half * 64 + 32, p1);
         tmem_wait_ld();
@@ -322,6 +347,9 @@ __global__ void __launch_bounds__(bwd::kDQThreads, 1)
         reg_fence(s1);
         reg_fence(p0);
         reg_fence(p1);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[DQ_DPEMPTY]);   // dP(t) read: the next dP may land
         int valid = 64;
         if (t == T - 1) {
           const int nblk = cnt - 2 * t;
@@ -342,11 +370,13 @@ __global__ void __launch_bounds__(bwd::kDQThreads, 1)
           }
           ds[c] = pack_bf16x2(e[0], e[1]);
         }
-        tmem_st32(tm + la + TM_S + half * 32, ds);
+        // dS over the first 32 of this half's own 64 S columns (the other
+        // half may not have read its S yet)
+        tmem_st32(tm + la + TM_S + b * 128 + half * 64, ds);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[DQ_PFULL]);
+        if (lane == 0) mbar_arrive(&bars[DQ_PFULL + b]);
       }
       if (!ok) break;
       if (!(ok = mbar_wait(&bars[DQ_OFULL], ii & 1, abort_flag))) break;
@@ -525,10 +555,12 @@ __global__ void __launch_bounds__(bwd::kKVThreads, 1)
           const uint64_t dmn = domn0 + ((s * L::ROWS_BYTES) >> 4), qmn = qmn0 + ((s * L::ROWS_BYTES) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tm + TM_DV, tm + TM_ST + kk * 8, dmn + ((kk * 2048u) >> 4), id_acc, (j > 0 || kk > 0) ? 1u : 0u);
+            umma_ts(tm + TM_DV, tm + TM_ST + (kk >> 2) * 64 + (kk & 3) * 8, dmn + ((kk * 2048u) >> 4), id_acc,
+                    (j > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tm + TM_DK, tm + TM_DPT + kk * 8, qmn + ((kk * 2048u) >> 4), id_acc, (j > 0 || kk > 0) ? 1u : 0u);
+            umma_ts(tm + TM_DK, tm + TM_DPT + (kk >> 2) * 64 + (kk & 3) * 8, qmn + ((kk * 2048u) >> 4), id_acc,
+                    (j > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&bars[KV_QEMPTY + s]);
           if (j + 1 == cnt) {
             tc_commit(&bars[KV_KEMPTY]);
@@ -620,8 +652,10 @@ __global__ void __launch_bounds__(bwd::kKVThreads, 1)
           pt[c] = pack_bf16x2(pp[0], pp[1]);
           dst[c] = pack_bf16x2(dd[0], dd[1]);
         }
-        tmem_st32(tm + la + TM_ST + half * 32, pt);
-        tmem_st32(tm + la + TM_DPT + half * 32, dst);
+        // P^T and dS^T over the first 32 of this half's own 64 columns (the
+        // other half may not have read its columns yet)
+        tmem_st32(tm + la + TM_ST + half * 64, pt);
+        tmem_st32(tm + la + TM_DPT + half * 64, dst);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
