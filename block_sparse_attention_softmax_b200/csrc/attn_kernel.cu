@@ -53,8 +53,10 @@
 // head) each. Both products run as tcgen05.mma kind::f8f6f4 (32 bytes of K per
 // instruction, half the instructions of bf16); the softmax folds scale * s_q *
 // s_k into its per-item exponent factor, P is written over S as E4M3 (P <= 256
-// < 448, so it needs no scale of its own; the four keys of a TMEM column are
-// gathered from two threads by shuffles), and the epilogue multiplies by s_v.
+// < 448, so it needs no scale of its own), and the epilogue multiplies by s_v.
+// Its softmax keeps the earlier split of each row between two warps with a
+// per-tile max exchange (see that branch): four E4M3 keys share a TMEM column,
+// and in the 16-lane layout they would lie in two threads.
 // Item facts carry the two factors, posted by the K producer with the rest.
 //
 // TMEM columns: S buffers at 0, 128 and 256 (fp32, 128 wide; P aliases their
@@ -101,7 +103,10 @@ struct Layout {
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + kQSlots * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + kKStages * TILE_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_V + kVStages * TILE_BYTES;
+  static constexpr uint32_t OFF_RED = OFF_V + kVStages * TILE_BYTES;
+  // row max [2][2][128], row sum [2][128], pair flags [4][16] of the E4M3 form's exchange
+  static constexpr uint32_t RED_BYTES = F8 ? (2 * 2 + 2) * kBM * 4 + 4 * 16 * 4 : 0;
+  static constexpr uint32_t OFF_BAR = OFF_RED + RED_BYTES;
   static constexpr uint32_t OFF_RING = OFF_BAR + 512;    // item ring [kItemRing][kRingWords] int
   static_assert(kItemRing * kRingWords * 4 <= 256, "item ring region");
   static_assert(NCH >= 1, "the low-bit form needs d = 128");
@@ -132,6 +137,24 @@ enum {
   B_DRAIN = B_IEMPTY + kItemRing,    // [2] each MMA thread's last commit (early exit)
   B_COUNT = B_DRAIN + 2
 };
+
+// Word a softmax warp of the E4M3 form posts in place of its row max or row
+// sum when its wait failed: a NaN whose payload no arithmetic produces.
+constexpr uint32_t kStopBits = 0x7FC0DEADu;
+
+// Named barrier of the two softmax warps of one TMEM lane quadrant (E4M3 form);
+// shared memory written before it by either warp is visible to both after it.
+__device__ __forceinline__ void pair_sync(int bar_id) {
+  asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+}
+
+// Both warps of a pair post whether their wait succeeded and meet; true only
+// if both did. slot[half] is this warp's word, slot[half ^ 1] the partner's.
+__device__ __forceinline__ bool pair_agree(int bar_id, volatile int* slot, int half, bool ok) {
+  slot[half] = ok ? 1 : 0;
+  pair_sync(bar_id);
+  return ok && slot[half ^ 1] != 0;
+}
 
 // Per-item facts every role derives the same way.
 struct Item {
@@ -415,309 +438,551 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       mbar_drain(&bars[B_DRAIN + (is_qk ? 0 : 1)], 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax + epilogue
-    // Each warp owns 16 of its quadrant's TMEM lanes (query rows), all 128
-    // columns of every tile: thread t holds rows ra and ra + 8 and, of each,
-    // the columns 8 k + 2 j4 and 8 k + 2 j4 + 1 (j4 = t % 4, k = 0..15). The
-    // four threads of a row combine its max and sum with two shuffles.
-    const int sw = warp - 2;                  // 0..7
-    const int quad = warp & 3;                // TMEM lane quadrant
-    const int half = sw >> 2;                 // which 16 lanes of the quadrant
-    const int j4 = lane & 3;
-    const int ra = quad * 32 + half * 16 + (lane >> 2);   // rows ra and ra + 8 of the tile
-    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32 + half * 16) << 16;
-    const int zrow = quad * 32 + lane;        // row and half columns this thread zero-fills
-    const float sl2 = a.scale_log2;
-    const int tail_valid = a.N - (a.nkb - 1) * 64;
-    int g = 0, qi = 0;
-    bool ok = true;
+    if constexpr (F8) {
+      // ------------------------------------------------------------ softmax + epilogue (E4M3)
+      // The low-bit form keeps the split of each row's 128 columns between the
+      // two warps of a lane quadrant (32x32b accesses, 64 columns each), with a
+      // per-tile exchange of the row max: its P packs four keys into each TMEM
+      // column, which a thread of the 16-lane layout (two keys per column pair)
+      // could only do with cross-thread shuffles, and those cost more than the
+      // exchange. Every bounded wait of these warps is followed by a barrier of
+      // the pair at which each warp also posts whether its wait succeeded: in
+      // place of the row max or row sum it posts a NaN with a payload of its own
+      // (kStopBits; arithmetic yields the canonical NaN, never this one), or a
+      // flag word in the rare rescale path. Each warp stops if either post says
+      // so, the same decision in both. A warp whose wait for the next item fails
+      // (no barrier follows that wait) posts the stop word in both places its
+      // partner reads next and arrives once at the pair barrier before it leaves,
+      // so neither waits at a barrier the other has left.
+      float* red_max = reinterpret_cast<float*>(smem + L::OFF_RED);   // [2 tile parity][2 halves][128 rows]
+      float* red_sum = red_max + 4 * kBM;                              // [2 halves][128 rows]
+      // per quadrant: [6,8) rescale (half 0, half 1)
+      volatile int* pair_flags = reinterpret_cast<volatile int*>(red_sum + 2 * kBM);
+      const int sw = warp - 2;                  // 0..7
+      const int quad = warp & 3;                // TMEM lane quadrant
+      const int half = sw >> 2;                 // which 64 columns of the tile
+      const int row = quad * 32 + lane;         // query row within the tile
+      const int pair_bar = 1 + quad;            // named barrier of the two warps of this quadrant
+      const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+      const float sl2 = a.scale_log2;
+      const int tail_valid = a.N - (a.nkb - 1) * 64;
+      int g = 0, qi = 0;
+      bool ok = true;
 
-    int prev = blockIdx.x - static_cast<int>(gridDim.x);   // last item handled
-    while (ok) {
-      // next non-empty item, as posted by the K producer; the items skipped
-      // on the way have no kept block
-      const int rs = qi % kItemRing;
-      if (!mbar_wait(&bars[B_IFULL + rs], (qi / kItemRing) & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      const int item = item_ring[rs * kRingWords + 0];
-      Item it;
-      it.cnt = item_ring[rs * kRingWords + 1];
-      it.tail = item_ring[rs * kRingWords + 2] != 0;
-      // exponent factor of the scores and factor of the output (the low-bit
-      // form's scales folded in)
-      const float fexp = F8 ? __int_as_float(item_ring[rs * kRingWords + 3]) : sl2;
-      const float fout = F8 ? __int_as_float(item_ring[rs * kRingWords + 4]) : 1.f;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_IEMPTY + rs]);
-      for (int z = prev + gridDim.x; z < item; z += gridDim.x) {
-        const Item iz = load_item(a, z);
-        const int gz = iz.qb * a.bq + zrow;
-        if (zrow < a.bq && gz < a.N) {
-          uint4* dz = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(iz.bh) * a.N + gz) * D + half * (D / 2));
-          for (int c = 0; c < D / 16; ++c) dz[c] = make_uint4(0, 0, 0, 0);
-          if (a.lse && half == 0) a.lse[static_cast<long long>(iz.bh) * a.N + gz] = -INFINITY;
-        }
-      }
-      if (item >= n_items) break;
-      prev = item;
-      it.bh = item / a.nqb;
-      it.qb = item % a.nqb;
-      it.T = (it.cnt + 1) >> 1;
-      const int grow_a = it.qb * a.bq + ra;
-      const bool store_a = ra < a.bq && grow_a < a.N;
-      const bool store_b = ra + 8 < a.bq && grow_a + 8 < a.N;
-      const long long off_a = (static_cast<long long>(it.bh) * a.N + grow_a) * D;
-      const long long off_b = off_a + 8LL * D;
-      if (a.alpha && j4 == 0) {
-        // the epilogue reads these rows of O_l: bring them into L2 while the item runs
-        const char* ola = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.o_l) + off_a);
-        const char* olb = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.o_l) + off_b);
-#pragma unroll
-        for (int b = 0; b < 2 * D; b += 128) {
-          if (store_a) asm volatile("prefetch.global.L2 [%0];" ::"l"(ola + b));
-          if (store_b) asm volatile("prefetch.global.L2 [%0];" ::"l"(olb + b));
-        }
-      }
-      float m_a = -INFINITY, m_b = -INFINITY;   // running maxima of the two rows (log2 domain)
-      float l_a = 0.f, l_b = 0.f;               // this thread's shares of the row sums
-      for (int t = 0; t < it.T; ++t, ++g) {
-        const int b = g % kSBufs;
-        if (!mbar_wait(&bars[B_SFULL + b], (g / kSBufs) & 1, abort_flag)) {
+      int prev = blockIdx.x - static_cast<int>(gridDim.x);   // last item handled
+      while (ok) {
+        // next non-empty item, as posted by the K producer; the items skipped
+        // on the way have no kept block
+        const int rs = qi % kItemRing;
+        if (!mbar_wait(&bars[B_IFULL + rs], (qi / kItemRing) & 1, abort_flag)) {
+          // leaving without the partner: post the stop word where it reads next
+          // and give it the one arrival its next exchange needs
+          red_max[(g & 1) * 2 * kBM + half * kBM + row] = __uint_as_float(kStopBits);
+          red_sum[half * kBM + row] = __uint_as_float(kStopBits);
+          asm volatile("bar.arrive %0, 64;" ::"r"(pair_bar) : "memory");
           ok = false;
           break;
         }
-        float xa[32], xb[32];   // [2 k + e]: column 8 k + 2 j4 + e of rows ra, ra + 8
-        {
-          tc_fence_after();
-          uint32_t r0[32], r1[32];
-          tmem_ld_16x256b_x8(tm + lane_addr + tm_s(b), r0);
-          tmem_ld_16x256b_x8(tm + lane_addr + tm_s(b) + 64, r1);
-          tmem_wait_ld();
-          reg_fence(r0);
-          reg_fence(r1);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            xa[2 * k] = __uint_as_float(r0[4 * k]);
-            xa[2 * k + 1] = __uint_as_float(r0[4 * k + 1]);
-            xb[2 * k] = __uint_as_float(r0[4 * k + 2]);
-            xb[2 * k + 1] = __uint_as_float(r0[4 * k + 3]);
-            xa[16 + 2 * k] = __uint_as_float(r1[4 * k]);
-            xa[16 + 2 * k + 1] = __uint_as_float(r1[4 * k + 1]);
-            xb[16 + 2 * k] = __uint_as_float(r1[4 * k + 2]);
-            xb[16 + 2 * k + 1] = __uint_as_float(r1[4 * k + 3]);
+        const int item = item_ring[rs * kRingWords + 0];
+        Item it;
+        it.cnt = item_ring[rs * kRingWords + 1];
+        it.tail = item_ring[rs * kRingWords + 2] != 0;
+        // exponent factor of the scores and factor of the output (the low-bit
+        // form's scales folded in)
+        const float fexp = F8 ? __int_as_float(item_ring[rs * kRingWords + 3]) : sl2;
+        const float fout = F8 ? __int_as_float(item_ring[rs * kRingWords + 4]) : 1.f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_IEMPTY + rs]);
+        for (int z = prev + gridDim.x; z < item; z += gridDim.x) {
+          const Item iz = load_item(a, z);
+          const int gz = iz.qb * a.bq + row;
+          if (row < a.bq && gz < a.N) {
+            uint4* dz = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(iz.bh) * a.N + gz) * D + half * (D / 2));
+            for (int c = 0; c < D / 16; ++c) dz[c] = make_uint4(0, 0, 0, 0);
+            if (a.lse && half == 0) a.lse[static_cast<long long>(iz.bh) * a.N + gz] = -INFINITY;
           }
         }
-        if (t == it.T - 1) {
-          // last tile: possibly a single block, possibly the ragged last key block
-          const int nblk = it.cnt - 2 * t;
-          const int limit = (nblk == 2 ? 64 : 0) + (it.tail ? tail_valid : 64);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (8 * (i >> 1) + 2 * j4 + (i & 1) >= limit) {
-              xa[i] = -INFINITY;
-              xb[i] = -INFINITY;
+        if (item >= n_items) break;
+        prev = item;
+        it.bh = item / a.nqb;
+        it.qb = item % a.nqb;
+        it.T = (it.cnt + 1) >> 1;
+        const int grow = it.qb * a.bq + row;
+        const bool store = row < a.bq && grow < a.N;
+        const long long orow_off = (static_cast<long long>(it.bh) * a.N + grow) * D + half * (D / 2);
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + orow_off;
+        if (a.alpha && store) {
+          // the epilogue reads this half row of O_l: bring it into L2 while the item runs
+          const char* olr = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.o_l) + orow_off);
+  #pragma unroll
+          for (int b = 0; b < D; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(olr + b));
+        }
+        float m = -INFINITY;     // running max (log2 domain), identical in both halves
+        float l = 0.f;           // this half's share of the row sum
+        for (int t = 0; t < it.T; ++t, ++g) {
+          const int b = g % kSBufs;
+          // (after a failed wait the loads below read stale tensor memory; the
+          // values are dropped when the pair stops at the barrier that follows)
+          const bool s_ok = mbar_wait(&bars[B_SFULL + b], (g / kSBufs) & 1, abort_flag);
+          float x[64];
+          float mx;
+          {
+            tc_fence_after();
+            uint32_t r0[32], r1[32];
+            const uint32_t sa = tm + lane_addr + tm_s(b) + half * 64;
+            tmem_ld32(sa, r0);
+            tmem_ld32(sa + 32, r1);
+            tmem_wait_ld();
+            reg_fence(r0);
+            reg_fence(r1);
+  #pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              x[c] = __uint_as_float(r0[c]);
+              x[32 + c] = __uint_as_float(r1[c]);
+            }
+            if (t == it.T - 1) {
+              // last tile: possibly a single block, possibly the ragged last key block
+              const int nblk = it.cnt - 2 * t;
+              int valid = (half < nblk) ? 64 : 0;
+              if (it.tail && half == nblk - 1) valid = tail_valid;
+  #pragma unroll
+              for (int c = 0; c < 64; ++c)
+                if (c >= valid) x[c] = -INFINITY;
+            }
+            // row max of this half: eight chains of 3-input max
+            float mx8[8];
+  #pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              mx8[j] = fmax3(x[j], x[8 + j], x[16 + j]);
+              mx8[j] = fmax3(mx8[j], x[24 + j], x[32 + j]);
+              mx8[j] = fmax3(mx8[j], x[40 + j], x[48 + j]);
+              mx8[j] = fmaxf(mx8[j], x[56 + j]);
+            }
+            mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+          }
+          float* rm = red_max + (g & 1) * 2 * kBM;
+          // the low-bit form posts its max in the log2 domain (the factor is the
+          // same for both halves; bf16 scales after the exchange)
+          const float posted = s_ok ? (F8 ? mx * fexp : mx) : __uint_as_float(kStopBits);
+          rm[half * kBM + row] = posted;
+          pair_sync(pair_bar);
+          const float pmx = rm[(half ^ 1) * kBM + row];
+          // Both warps combine the two posted words the same way (fmaxf skips the
+          // NaN stop word), so everything up to the end of the tile, branches
+          // included, is the same in both; the stop, if any, is taken there.
+          const bool stop = !s_ok || __float_as_uint(pmx) == kStopBits;
+          mx = fmaxf(posted, pmx);
+          const float m_tile = F8 ? mx : mx * sl2;
+          float corr = 1.f;
+          if (m_tile > m + 8.f) {
+            corr = fast_exp2(m - m_tile);   // 0 on the first tile (m = -inf)
+            m = m_tile;
+            l *= corr;
+          }
+          // P = 2^(S * scale * log2(e) - m), two columns per packed instruction.
+          const uint64_t sl2x2 = f2_make(fexp, fexp);
+          const uint64_t negm2 = f2_make(-m, -m);
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // packed (+0, +0)
+          uint32_t p[F8 ? 16 : 32];
+  #pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const uint64_t a2 = ffma2(f2_make(x[2 * c], x[2 * c + 1]), sl2x2, negm2);
+            float e0, e1;
+            if ((kPolyPairs >> (c & 7)) & 1) {
+              exp2_poly2(a2, e0, e1);
+            } else {
+              float a0, a1;
+              f2_split(a2, a0, a1);
+              e0 = fast_exp2(a0);
+              e1 = fast_exp2(a1);
+            }
+            acc[c & 3] = fadd2(acc[c & 3], f2_make(e0, e1));
+            if constexpr (F8) {
+              // four E4M3 values per column, the lowest key in the lowest byte
+              const uint32_t h = pack_e4m3x2(e0, e1);
+              p[c >> 1] = (c & 1) ? (p[c >> 1] | (h << 16)) : h;
+            } else {
+              p[c] = pack_bf16x2(e0, e1);
             }
           }
-        }
-        float mx_a, mx_b;
-        {
-          float ma4[4], mb4[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            ma4[j] = fmax3(fmax3(xa[j], xa[4 + j], xa[8 + j]), fmax3(xa[12 + j], xa[16 + j], xa[20 + j]), fmaxf(xa[24 + j], xa[28 + j]));
-            mb4[j] = fmax3(fmax3(xb[j], xb[4 + j], xb[8 + j]), fmax3(xb[12 + j], xb[16 + j], xb[20 + j]), fmaxf(xb[24 + j], xb[28 + j]));
+          {
+            float s0, s1;
+            f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), s0, s1);
+            l += s0 + s1;
           }
-          mx_a = fmaxf(fmaxf(ma4[0], ma4[1]), fmaxf(ma4[2], ma4[3]));
-          mx_b = fmaxf(fmaxf(mb4[0], mb4[1]), fmaxf(mb4[2], mb4[3]));
-          mx_a = fmaxf(mx_a, __shfl_xor_sync(0xFFFFFFFFu, mx_a, 1));
-          mx_b = fmaxf(mx_b, __shfl_xor_sync(0xFFFFFFFFu, mx_b, 1));
-          mx_a = fmaxf(mx_a, __shfl_xor_sync(0xFFFFFFFFu, mx_a, 2));
-          mx_b = fmaxf(mx_b, __shfl_xor_sync(0xFFFFFFFFu, mx_b, 2));
-        }
-        float corr_a = 1.f, corr_b = 1.f;
-        {
-          const float mt_a = mx_a * fexp, mt_b = mx_b * fexp;
-          if (mt_a > m_a + 8.f) {
-            corr_a = fast_exp2(m_a - mt_a);   // 0 on the first tile (m = -inf)
-            m_a = mt_a;
-            l_a *= corr_a;
-          }
-          if (mt_b > m_b + 8.f) {
-            corr_b = fast_exp2(m_b - mt_b);
-            m_b = mt_b;
-            l_b *= corr_b;
-          }
-        }
-        // P = 2^(S * factor - m), two columns per packed instruction: pairs
-        // c < 16 are row ra (columns 8 c + 2 j4, + 1), c >= 16 row ra + 8.
-        const uint64_t fx2 = f2_make(fexp, fexp);
-        const uint64_t negm_a = f2_make(-m_a, -m_a), negm_b = f2_make(-m_b, -m_b);
-        uint64_t acc_a[2] = {0ull, 0ull}, acc_b[2] = {0ull, 0ull};   // packed (+0, +0)
-        uint32_t p[32];   // bf16: [2 k] row ra, [2 k + 1] row ra + 8, column 4 k + j4
-                          // E4M3: 16-bit halves, [2 k] / [2 k + 1] as for bf16
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const bool rb = c >= 16;
-          const int k = c & 15;
-          const float* xr = rb ? xb : xa;
-          const uint64_t a2 = ffma2(f2_make(xr[2 * k], xr[2 * k + 1]), fx2, rb ? negm_b : negm_a);
-          float e0, e1;
-          if ((kPolyPairs >> (c & 7)) & 1) {
-            exp2_poly2(a2, e0, e1);
-          } else {
-            float a0, a1;
-            f2_split(a2, a0, a1);
-            e0 = fast_exp2(a0);
-            e1 = fast_exp2(a1);
-          }
-          if (rb) acc_b[c & 1] = fadd2(acc_b[c & 1], f2_make(e0, e1));
-          else acc_a[c & 1] = fadd2(acc_a[c & 1], f2_make(e0, e1));
-          if constexpr (F8) p[2 * k + (rb ? 1 : 0)] = pack_e4m3x2(e0, e1);
-          else p[2 * k + (rb ? 1 : 0)] = pack_bf16x2(e0, e1);
-        }
-        {
-          float s0, s1;
-          f2_split(fadd2(acc_a[0], acc_a[1]), s0, s1);
-          l_a += s0 + s1;
-          f2_split(fadd2(acc_b[0], acc_b[1]), s0, s1);
-          l_b += s0 + s1;
-        }
-        if constexpr (F8) {
-          // Four E4M3 keys per TMEM column, the lowest key in the lowest byte.
-          // Column 2 k + (j4 >> 1) holds keys 8 k + 4 (j4 >> 1) .. + 3: the
-          // 16-bit halves (two keys each) of threads j4 and j4 ^ 1 at index k.
-          // Step 1: the two threads of a pair swap their halves of indices
-          // 2 m and 2 m + 1 in one word; thread j4 keeps index 2 m + (j4 & 1),
-          // i.e. column 4 m + sg with sg = 2 (j4 & 1) + (j4 >> 1).
-          // Step 2: the 16x128b store writes column 4 m + j4 from thread j4,
-          // which thread sg(j4) holds (sg swaps 1 and 2).
-          const int e1 = j4 & 1;
-          const int sg = 2 * e1 + (j4 >> 1);
-          uint32_t q8[16];
-#pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-              const uint32_t lo = p[2 * (2 * m) + rr], hi = p[2 * (2 * m + 1) + rr];
-              const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, lo | (hi << 16), 1);
-              const uint32_t own = e1 ? hi : lo;
-              const uint32_t oth = e1 ? (got >> 16) : (got & 0xFFFFu);
-              const uint32_t word = (j4 & 1) ? (oth | (own << 16)) : (own | (oth << 16));
-              q8[2 * m + rr] = __shfl_sync(0xFFFFFFFFu, word, (lane & ~3) | sg);
+          if constexpr (F8) tmem_st16(tm + lane_addr + tm_s(b) + half * 16, p);
+          else tmem_st32(tm + lane_addr + tm_s(b) + half * 32, p);
+          if (!stop && t > 0 && __any_sync(0xFFFFFFFFu, corr != 1.f)) {
+            // O is complete up to the previous tile once its P V has landed
+            const int pb = (g - 1) % kSBufs;
+            if (!(ok = pair_agree(pair_bar, pair_flags + quad * 16 + 6, half, mbar_wait(&bars[B_PVDONE + pb], ((g - 1) / kSBufs) & 1, abort_flag)))) break;
+            tc_fence_after();
+  #pragma unroll 1
+            for (int c0 = 0; c0 < D / 2; c0 += 32) {
+              uint32_t o[32];
+              const uint32_t oa = tm + lane_addr + TM_O + half * (D / 2) + c0;
+              tmem_ld32_wait(oa, o);
+  #pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
+              tmem_st32(oa, o);
             }
           }
-          tmem_st_16x128b_x8(tm + lane_addr + tm_s(b), q8);
-        } else {
-          tmem_st_16x128b_x16(tm + lane_addr + tm_s(b), p);
-        }
-        if (t > 0 && __any_sync(0xFFFFFFFFu, corr_a != 1.f || corr_b != 1.f)) {
-          // O is complete up to the previous tile once its P V has landed
-          const int pb = (g - 1) % kSBufs;
-          if (!mbar_wait(&bars[B_PVDONE + pb], ((g - 1) / kSBufs) & 1, abort_flag)) {
+          tmem_wait_st();
+          if (stop) {   // either warp's wait failed: both stop here
             ok = false;
             break;
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[B_PFULL + b]);
+        }
+        if (!ok) break;
+        // ---------------------------------------------------------- epilogue
+        // with the blend, this half row of O_l is loaded before the wait for
+        // the last P V, so the wait hides the load
+        uint4 olv[D / 16];
+        if (a.alpha && store) {
+          const uint4* olp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.o_l) + orow_off);
+  #pragma unroll
+          for (int c = 0; c < D / 16; ++c) olv[c] = __ldg(olp + c);
+        }
+        const bool o_ok = mbar_wait(&bars[B_OFULL], qi & 1, abort_flag);
+        uint32_t o0[32], o1[32];
+        {
           tc_fence_after();
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 64) {
-            uint32_t o[32];
-            const uint32_t oa = tm + lane_addr + TM_O + c0;
-            tmem_ld_16x256b_x8(oa, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              o[4 * k] = __float_as_uint(__uint_as_float(o[4 * k]) * corr_a);
-              o[4 * k + 1] = __float_as_uint(__uint_as_float(o[4 * k + 1]) * corr_a);
-              o[4 * k + 2] = __float_as_uint(__uint_as_float(o[4 * k + 2]) * corr_b);
-              o[4 * k + 3] = __float_as_uint(__uint_as_float(o[4 * k + 3]) * corr_b);
-            }
-            tmem_st_16x256b_x8(oa, o);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_PFULL + b]);
-      }
-      if (!ok) break;
-      // ---------------------------------------------------------- epilogue
-      // row sums over the four threads of each row
-      l_a += __shfl_xor_sync(0xFFFFFFFFu, l_a, 1);
-      l_b += __shfl_xor_sync(0xFFFFFFFFu, l_b, 1);
-      l_a += __shfl_xor_sync(0xFFFFFFFFu, l_a, 2);
-      l_b += __shfl_xor_sync(0xFFFFFFFFu, l_b, 2);
-      const float inv_a = fout / l_a, inv_b = fout / l_b;
-      // with the blend, this thread's elements of O_l are loaded before the
-      // wait for the last P V, so the wait hides the loads
-      uint32_t ol_a[D / 8], ol_b[D / 8];
-      if (a.alpha) {
-        const __nv_bfloat16* olp = static_cast<const __nv_bfloat16*>(a.o_l);
-#pragma unroll
-        for (int k = 0; k < D / 8; ++k) {
-          ol_a[k] = store_a ? __ldg(reinterpret_cast<const unsigned int*>(olp + off_a + 8 * k + 2 * j4)) : 0u;
-          ol_b[k] = store_b ? __ldg(reinterpret_cast<const unsigned int*>(olp + off_b + 8 * k + 2 * j4)) : 0u;
-        }
-      }
-      if (!mbar_wait(&bars[B_OFULL], qi & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      uint32_t o[D / 2];   // [32 h + 4 k + 0..3]: columns 64 h + 8 k + 2 j4 (+1) of rows ra, ra + 8
-      {
-        tc_fence_after();
-        uint32_t r0[32];
-        tmem_ld_16x256b_x8(tm + lane_addr + TM_O, r0);
-        if constexpr (D == 128) {
-          uint32_t r1[32];
-          tmem_ld_16x256b_x8(tm + lane_addr + TM_O + 64, r1);
+          tmem_ld32(tm + lane_addr + TM_O + half * (D / 2), o0);
+          if (D == 128) tmem_ld32(tm + lane_addr + TM_O + half * (D / 2) + 32, o1);
           tmem_wait_ld();
-          reg_fence(r0);
-          reg_fence(r1);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            o[i] = r0[i];
-            o[32 + i] = r1[i];
-          }
-        } else {
-          tmem_wait_ld();
-          reg_fence(r0);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = r0[i];
+          reg_fence(o0);
+          if (D == 128) reg_fence(o1);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[B_OEMPTY]);   // the next item may overwrite O now
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_OEMPTY]);   // the next item may overwrite O now
-      }
-      {
-        __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.o);
-        const float* alr = a.alpha ? a.alpha + static_cast<long long>(it.bh % a.H) * D : nullptr;
-#pragma unroll
-        for (int k = 0; k < D / 8; ++k) {
-          const int col = 8 * k + 2 * j4;
-          const int i0 = 32 * (k >> 3) + 4 * (k & 7);
-          float va0 = __uint_as_float(o[i0]) * inv_a, va1 = __uint_as_float(o[i0 + 1]) * inv_a;
-          float vb0 = __uint_as_float(o[i0 + 2]) * inv_b, vb1 = __uint_as_float(o[i0 + 3]) * inv_b;
+        red_sum[half * kBM + row] = o_ok ? l : __uint_as_float(kStopBits);
+        pair_sync(pair_bar);
+        const float pl = red_sum[(half ^ 1) * kBM + row];
+        if (!(ok = o_ok && __float_as_uint(pl) != kStopBits)) break;
+        const float lt = l + pl;
+        const float inv_l = F8 ? fout / lt : 1.f / lt;
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow);
           if (a.alpha) {
-            // O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l with O_s not yet rounded
-            const float2 al = __ldg(reinterpret_cast<const float2*>(alr + col));
-            const float la0 = __uint_as_float(ol_a[k] << 16), la1 = __uint_as_float(ol_a[k] & 0xFFFF0000u);
-            const float lb0 = __uint_as_float(ol_b[k] << 16), lb1 = __uint_as_float(ol_b[k] & 0xFFFF0000u);
-            va0 = fmaf(al.x, va0 - la0, la0);
-            va1 = fmaf(al.y, va1 - la1, la1);
-            vb0 = fmaf(al.x, vb0 - lb0, lb0);
-            vb1 = fmaf(al.y, vb1 - lb1, lb1);
+            // O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l with O_s = o / l not yet rounded
+            const float4* alv = reinterpret_cast<const float4*>(a.alpha + static_cast<long long>(it.bh % a.H) * D + half * (D / 2));
+  #pragma unroll
+            for (int c = 0; c < D / 16; ++c) {
+              const uint32_t* oc = (c < 4) ? o0 + 8 * c : o1 + 8 * (c - 4);
+              const uint4 lv = olv[c];
+              const float4 a0 = __ldg(alv + 2 * c), a1 = __ldg(alv + 2 * c + 1);
+              const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
+              const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+              float r8[8];
+  #pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float olj = __uint_as_float((j & 1) ? (lw[j >> 1] & 0xFFFF0000u) : (lw[j >> 1] << 16));
+                r8[j] = fmaf(av[j], __uint_as_float(oc[j]) * inv_l - olj, olj);
+              }
+              dst[c] = make_uint4(pack_bf16x2(r8[0], r8[1]), pack_bf16x2(r8[2], r8[3]),
+                                  pack_bf16x2(r8[4], r8[5]), pack_bf16x2(r8[6], r8[7]));
+            }
+          } else {
+            uint32_t pk[16];
+  #pragma unroll
+            for (int c = 0; c < 16; ++c)
+              pk[c] = pack_bf16x2(__uint_as_float(o0[2 * c]) * inv_l, __uint_as_float(o0[2 * c + 1]) * inv_l);
+  #pragma unroll
+            for (int c = 0; c < 4; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            if (D == 128) {
+  #pragma unroll
+              for (int c = 0; c < 16; ++c)
+                pk[c] = pack_bf16x2(__uint_as_float(o1[2 * c]) * inv_l, __uint_as_float(o1[2 * c + 1]) * inv_l);
+  #pragma unroll
+              for (int c = 0; c < 4; ++c) dst[4 + c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            }
           }
-          if (store_a) *reinterpret_cast<uint32_t*>(ob + off_a + col) = pack_bf16x2(va0, va1);
-          if (store_b) *reinterpret_cast<uint32_t*>(ob + off_b + col) = pack_bf16x2(vb0, vb1);
         }
+        if (store && a.lse && half == 0)
+          a.lse[static_cast<long long>(it.bh) * a.N + grow] = (m + log2f(lt)) * 0.69314718055994531f;
+        ++qi;
       }
-      if (a.lse && j4 == 0) {
-        if (store_a) a.lse[static_cast<long long>(it.bh) * a.N + grow_a] = (m_a + log2f(l_a)) * 0.69314718055994531f;
-        if (store_b) a.lse[static_cast<long long>(it.bh) * a.N + grow_a + 8] = (m_b + log2f(l_b)) * 0.69314718055994531f;
+    } else {
+      // ------------------------------------------------------------ softmax + epilogue
+      // Each warp owns 16 of its quadrant's TMEM lanes (query rows), all 128
+      // columns of every tile: thread t holds rows ra and ra + 8 and, of each,
+      // the columns 8 k + 2 j4 and 8 k + 2 j4 + 1 (j4 = t % 4, k = 0..15). The
+      // four threads of a row combine its max and sum with two shuffles.
+      const int sw = warp - 2;                  // 0..7
+      const int quad = warp & 3;                // TMEM lane quadrant
+      const int half = sw >> 2;                 // which 16 lanes of the quadrant
+      const int j4 = lane & 3;
+      const int ra = quad * 32 + half * 16 + (lane >> 2);   // rows ra and ra + 8 of the tile
+      const uint32_t lane_addr = static_cast<uint32_t>(quad * 32 + half * 16) << 16;
+      const int zrow = quad * 32 + lane;        // row and half columns this thread zero-fills
+      const float sl2 = a.scale_log2;
+      const int tail_valid = a.N - (a.nkb - 1) * 64;
+      int g = 0, qi = 0;
+      bool ok = true;
+
+      int prev = blockIdx.x - static_cast<int>(gridDim.x);   // last item handled
+      while (ok) {
+        // next non-empty item, as posted by the K producer; the items skipped
+        // on the way have no kept block
+        const int rs = qi % kItemRing;
+        if (!mbar_wait(&bars[B_IFULL + rs], (qi / kItemRing) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int item = item_ring[rs * kRingWords + 0];
+        Item it;
+        it.cnt = item_ring[rs * kRingWords + 1];
+        it.tail = item_ring[rs * kRingWords + 2] != 0;
+        // exponent factor of the scores and factor of the output (the low-bit
+        // form's scales folded in)
+        const float fexp = F8 ? __int_as_float(item_ring[rs * kRingWords + 3]) : sl2;
+        const float fout = F8 ? __int_as_float(item_ring[rs * kRingWords + 4]) : 1.f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_IEMPTY + rs]);
+        for (int z = prev + gridDim.x; z < item; z += gridDim.x) {
+          const Item iz = load_item(a, z);
+          const int gz = iz.qb * a.bq + zrow;
+          if (zrow < a.bq && gz < a.N) {
+            uint4* dz = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + (static_cast<long long>(iz.bh) * a.N + gz) * D + half * (D / 2));
+            for (int c = 0; c < D / 16; ++c) dz[c] = make_uint4(0, 0, 0, 0);
+            if (a.lse && half == 0) a.lse[static_cast<long long>(iz.bh) * a.N + gz] = -INFINITY;
+          }
+        }
+        if (item >= n_items) break;
+        prev = item;
+        it.bh = item / a.nqb;
+        it.qb = item % a.nqb;
+        it.T = (it.cnt + 1) >> 1;
+        const int grow_a = it.qb * a.bq + ra;
+        const bool store_a = ra < a.bq && grow_a < a.N;
+        const bool store_b = ra + 8 < a.bq && grow_a + 8 < a.N;
+        const long long off_a = (static_cast<long long>(it.bh) * a.N + grow_a) * D;
+        const long long off_b = off_a + 8LL * D;
+        if (a.alpha && j4 == 0) {
+          // the epilogue reads these rows of O_l: bring them into L2 while the item runs
+          const char* ola = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.o_l) + off_a);
+          const char* olb = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.o_l) + off_b);
+  #pragma unroll
+          for (int b = 0; b < 2 * D; b += 128) {
+            if (store_a) asm volatile("prefetch.global.L2 [%0];" ::"l"(ola + b));
+            if (store_b) asm volatile("prefetch.global.L2 [%0];" ::"l"(olb + b));
+          }
+        }
+        float m_a = -INFINITY, m_b = -INFINITY;   // running maxima of the two rows (log2 domain)
+        float l_a = 0.f, l_b = 0.f;               // this thread's shares of the row sums
+        for (int t = 0; t < it.T; ++t, ++g) {
+          const int b = g % kSBufs;
+          if (!mbar_wait(&bars[B_SFULL + b], (g / kSBufs) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          float xa[32], xb[32];   // [2 k + e]: column 8 k + 2 j4 + e of rows ra, ra + 8
+          {
+            tc_fence_after();
+            uint32_t r0[32], r1[32];
+            tmem_ld_16x256b_x8(tm + lane_addr + tm_s(b), r0);
+            tmem_ld_16x256b_x8(tm + lane_addr + tm_s(b) + 64, r1);
+            tmem_wait_ld();
+            reg_fence(r0);
+            reg_fence(r1);
+  #pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              xa[2 * k] = __uint_as_float(r0[4 * k]);
+              xa[2 * k + 1] = __uint_as_float(r0[4 * k + 1]);
+              xb[2 * k] = __uint_as_float(r0[4 * k + 2]);
+              xb[2 * k + 1] = __uint_as_float(r0[4 * k + 3]);
+              xa[16 + 2 * k] = __uint_as_float(r1[4 * k]);
+              xa[16 + 2 * k + 1] = __uint_as_float(r1[4 * k + 1]);
+              xb[16 + 2 * k] = __uint_as_float(r1[4 * k + 2]);
+              xb[16 + 2 * k + 1] = __uint_as_float(r1[4 * k + 3]);
+            }
+          }
+          if (t == it.T - 1) {
+            // last tile: possibly a single block, possibly the ragged last key block
+            const int nblk = it.cnt - 2 * t;
+            const int limit = (nblk == 2 ? 64 : 0) + (it.tail ? tail_valid : 64);
+  #pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (8 * (i >> 1) + 2 * j4 + (i & 1) >= limit) {
+                xa[i] = -INFINITY;
+                xb[i] = -INFINITY;
+              }
+            }
+          }
+          float mx_a, mx_b;
+          {
+            float ma4[4], mb4[4];
+  #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              ma4[j] = fmax3(fmax3(xa[j], xa[4 + j], xa[8 + j]), fmax3(xa[12 + j], xa[16 + j], xa[20 + j]), fmaxf(xa[24 + j], xa[28 + j]));
+              mb4[j] = fmax3(fmax3(xb[j], xb[4 + j], xb[8 + j]), fmax3(xb[12 + j], xb[16 + j], xb[20 + j]), fmaxf(xb[24 + j], xb[28 + j]));
+            }
+            mx_a = fmaxf(fmaxf(ma4[0], ma4[1]), fmaxf(ma4[2], ma4[3]));
+            mx_b = fmaxf(fmaxf(mb4[0], mb4[1]), fmaxf(mb4[2], mb4[3]));
+            mx_a = fmaxf(mx_a, __shfl_xor_sync(0xFFFFFFFFu, mx_a, 1));
+            mx_b = fmaxf(mx_b, __shfl_xor_sync(0xFFFFFFFFu, mx_b, 1));
+            mx_a = fmaxf(mx_a, __shfl_xor_sync(0xFFFFFFFFu, mx_a, 2));
+            mx_b = fmaxf(mx_b, __shfl_xor_sync(0xFFFFFFFFu, mx_b, 2));
+          }
+          float corr_a = 1.f, corr_b = 1.f;
+          {
+            const float mt_a = mx_a * fexp, mt_b = mx_b * fexp;
+            if (mt_a > m_a + 8.f) {
+              corr_a = fast_exp2(m_a - mt_a);   // 0 on the first tile (m = -inf)
+              m_a = mt_a;
+              l_a *= corr_a;
+            }
+            if (mt_b > m_b + 8.f) {
+              corr_b = fast_exp2(m_b - mt_b);
+              m_b = mt_b;
+              l_b *= corr_b;
+            }
+          }
+          // P = 2^(S * factor - m), two columns per packed instruction: pairs
+          // c < 16 are row ra (columns 8 c + 2 j4, + 1), c >= 16 row ra + 8.
+          const uint64_t fx2 = f2_make(fexp, fexp);
+          const uint64_t negm_a = f2_make(-m_a, -m_a), negm_b = f2_make(-m_b, -m_b);
+          uint64_t acc_a[2] = {0ull, 0ull}, acc_b[2] = {0ull, 0ull};   // packed (+0, +0)
+          uint32_t p[32];   // bf16 pairs: [2 k] row ra, [2 k + 1] row ra + 8, column 4 k + j4
+  #pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const bool rb = c >= 16;
+            const int k = c & 15;
+            const float* xr = rb ? xb : xa;
+            const uint64_t a2 = ffma2(f2_make(xr[2 * k], xr[2 * k + 1]), fx2, rb ? negm_b : negm_a);
+            float e0, e1;
+            if ((kPolyPairs >> (c & 7)) & 1) {
+              exp2_poly2(a2, e0, e1);
+            } else {
+              float a0, a1;
+              f2_split(a2, a0, a1);
+              e0 = fast_exp2(a0);
+              e1 = fast_exp2(a1);
+            }
+            if (rb) acc_b[c & 1] = fadd2(acc_b[c & 1], f2_make(e0, e1));
+            else acc_a[c & 1] = fadd2(acc_a[c & 1], f2_make(e0, e1));
+            p[2 * k + (rb ? 1 : 0)] = pack_bf16x2(e0, e1);
+          }
+          {
+            float s0, s1;
+            f2_split(fadd2(acc_a[0], acc_a[1]), s0, s1);
+            l_a += s0 + s1;
+            f2_split(fadd2(acc_b[0], acc_b[1]), s0, s1);
+            l_b += s0 + s1;
+          }
+          tmem_st_16x128b_x16(tm + lane_addr + tm_s(b), p);
+          if (t > 0 && __any_sync(0xFFFFFFFFu, corr_a != 1.f || corr_b != 1.f)) {
+            // O is complete up to the previous tile once its P V has landed
+            const int pb = (g - 1) % kSBufs;
+            if (!mbar_wait(&bars[B_PVDONE + pb], ((g - 1) / kSBufs) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+  #pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 64) {
+              uint32_t o[32];
+              const uint32_t oa = tm + lane_addr + TM_O + c0;
+              tmem_ld_16x256b_x8(oa, o);
+              tmem_wait_ld();
+  #pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                o[4 * k] = __float_as_uint(__uint_as_float(o[4 * k]) * corr_a);
+                o[4 * k + 1] = __float_as_uint(__uint_as_float(o[4 * k + 1]) * corr_a);
+                o[4 * k + 2] = __float_as_uint(__uint_as_float(o[4 * k + 2]) * corr_b);
+                o[4 * k + 3] = __float_as_uint(__uint_as_float(o[4 * k + 3]) * corr_b);
+              }
+              tmem_st_16x256b_x8(oa, o);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[B_PFULL + b]);
+        }
+        if (!ok) break;
+        // ---------------------------------------------------------- epilogue
+        // row sums over the four threads of each row
+        l_a += __shfl_xor_sync(0xFFFFFFFFu, l_a, 1);
+        l_b += __shfl_xor_sync(0xFFFFFFFFu, l_b, 1);
+        l_a += __shfl_xor_sync(0xFFFFFFFFu, l_a, 2);
+        l_b += __shfl_xor_sync(0xFFFFFFFFu, l_b, 2);
+        const float inv_a = fout / l_a, inv_b = fout / l_b;
+        // with the blend, this thread's elements of O_l are loaded before the
+        // wait for the last P V, so the wait hides the loads
+        uint32_t ol_a[D / 8], ol_b[D / 8];
+        if (a.alpha) {
+          const __nv_bfloat16* olp = static_cast<const __nv_bfloat16*>(a.o_l);
+  #pragma unroll
+          for (int k = 0; k < D / 8; ++k) {
+            ol_a[k] = store_a ? __ldg(reinterpret_cast<const unsigned int*>(olp + off_a + 8 * k + 2 * j4)) : 0u;
+            ol_b[k] = store_b ? __ldg(reinterpret_cast<const unsigned int*>(olp + off_b + 8 * k + 2 * j4)) : 0u;
+          }
+        }
+        if (!mbar_wait(&bars[B_OFULL], qi & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint32_t o[D / 2];   // [32 h + 4 k + 0..3]: columns 64 h + 8 k + 2 j4 (+1) of rows ra, ra + 8
+        {
+          tc_fence_after();
+          uint32_t r0[32];
+          tmem_ld_16x256b_x8(tm + lane_addr + TM_O, r0);
+          if constexpr (D == 128) {
+            uint32_t r1[32];
+            tmem_ld_16x256b_x8(tm + lane_addr + TM_O + 64, r1);
+            tmem_wait_ld();
+            reg_fence(r0);
+            reg_fence(r1);
+  #pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              o[i] = r0[i];
+              o[32 + i] = r1[i];
+            }
+          } else {
+            tmem_wait_ld();
+            reg_fence(r0);
+  #pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = r0[i];
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[B_OEMPTY]);   // the next item may overwrite O now
+        }
+        {
+          __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.o);
+          const float* alr = a.alpha ? a.alpha + static_cast<long long>(it.bh % a.H) * D : nullptr;
+  #pragma unroll
+          for (int k = 0; k < D / 8; ++k) {
+            const int col = 8 * k + 2 * j4;
+            const int i0 = 32 * (k >> 3) + 4 * (k & 7);
+            float va0 = __uint_as_float(o[i0]) * inv_a, va1 = __uint_as_float(o[i0 + 1]) * inv_a;
+            float vb0 = __uint_as_float(o[i0 + 2]) * inv_b, vb1 = __uint_as_float(o[i0 + 3]) * inv_b;
+            if (a.alpha) {
+              // O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l with O_s not yet rounded
+              const float2 al = __ldg(reinterpret_cast<const float2*>(alr + col));
+              const float la0 = __uint_as_float(ol_a[k] << 16), la1 = __uint_as_float(ol_a[k] & 0xFFFF0000u);
+              const float lb0 = __uint_as_float(ol_b[k] << 16), lb1 = __uint_as_float(ol_b[k] & 0xFFFF0000u);
+              va0 = fmaf(al.x, va0 - la0, la0);
+              va1 = fmaf(al.y, va1 - la1, la1);
+              vb0 = fmaf(al.x, vb0 - lb0, lb0);
+              vb1 = fmaf(al.y, vb1 - lb1, lb1);
+            }
+            if (store_a) *reinterpret_cast<uint32_t*>(ob + off_a + col) = pack_bf16x2(va0, va1);
+            if (store_b) *reinterpret_cast<uint32_t*>(ob + off_b + col) = pack_bf16x2(vb0, vb1);
+          }
+        }
+        if (a.lse && j4 == 0) {
+          if (store_a) a.lse[static_cast<long long>(it.bh) * a.N + grow_a] = (m_a + log2f(l_a)) * 0.69314718055994531f;
+          if (store_b) a.lse[static_cast<long long>(it.bh) * a.N + grow_a + 8] = (m_b + log2f(l_b)) * 0.69314718055994531f;
+        }
+        ++qi;
       }
-      ++qi;
+
     }
   }
 
