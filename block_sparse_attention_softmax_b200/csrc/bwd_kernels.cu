@@ -19,8 +19,9 @@
 //                  either block (a transposed list with a flag per block, from
 //                  col_lists_kernel), for each S^T = K Q^T and dP^T = V dO^T;
 //                  8 warps form P^T and dS^T (rows of the block that does not
-//                  keep this query block are zero); dV += P^T dO and
-//                  dK += dS^T Q accumulate in TMEM.
+//                  keep this query block are zero) into the dP^T columns, so
+//                  the next block's S^T lands while they work; dV += P^T dO
+//                  and dK += dS^T Q accumulate in TMEM.
 // Roles in both: warp 0 TMA producer, warp 1 TMEM allocation and the MMA
 // thread, then (dK/dV only) a warp staging the query blocks' LSE and D in
 // shared memory, and 8 warps, two per TMEM lane quadrant, 64 columns each.
@@ -428,7 +429,9 @@ struct KVLayout : Sizes<D> {
 };
 enum {
   KV_KFULL = 0, KV_KEMPTY, KV_QFULL, KV_QEMPTY = KV_QFULL + kStages, KV_STFULL = KV_QEMPTY + kStages,
-  KV_STEMPTY = KV_STFULL + kStages, KV_SFULL = KV_STEMPTY + kStages, KV_PFULL, KV_OFULL, KV_OEMPTY, KV_DRAIN, KV_COUNT
+  KV_STEMPTY = KV_STFULL + kStages, KV_SFULL = KV_STEMPTY + kStages,
+  KV_SEMPTY,     // S^T and dP^T read by every compute warp (the next S^T may land)
+  KV_PFULL, KV_OFULL, KV_OEMPTY, KV_DRAIN, KV_COUNT
 };
 constexpr int kKVThreads = 32 * (3 + kCWarps);
 }  // namespace bwd
@@ -460,6 +463,7 @@ __global__ void __launch_bounds__(bwd::kKVThreads, 1)
       mbar_init(&bars[KV_STEMPTY + i], kCWarps);
     }
     mbar_init(&bars[KV_SFULL], 1);
+    mbar_init(&bars[KV_SEMPTY], kCWarps);
     mbar_init(&bars[KV_PFULL], kCWarps);
     mbar_init(&bars[KV_OFULL], 1);
     mbar_init(&bars[KV_OEMPTY], kCWarps);
@@ -527,42 +531,70 @@ __global__ void __launch_bounds__(bwd::kKVThreads, 1)
       const uint64_t domn0 = sw128_desc(smem_u32(smem + L::OFF_DO), L::CHUNK, 1024);    // MN-major (dV += P^T dO)
       const uint32_t id_s = idesc_bf16_f32(kBM, 128, false, false);
       const uint32_t id_acc = idesc_bf16_f32(kBM, D, false, true);
+      // P^T and dS^T are written into the dP^T columns, so the S^T buffer is
+      // free once the compute warps have read it: S^T of the next query block
+      // is computed while they form P^T and dS^T of this one. dP^T of the next
+      // block follows the dV and dK products that read this one's P^T and
+      // dS^T (tcgen05.mma executes in issue order).
+      auto issue_st = [&](int s) {
+        const uint64_t qd = qdesc0 + ((s * L::ROWS_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (((kk >> 2) * L::CHUNK) + (kk & 3) * 32u) >> 4;
+          umma_ss(tm + TM_ST, kdesc + off, qd + off, id_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_dpt = [&](int s) {
+        const uint64_t dd = dodesc0 + ((s * L::ROWS_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (((kk >> 2) * L::CHUNK) + (kk & 3) * 32u) >> 4;
+          umma_ss(tm + TM_DPT, vdesc + off, dd + off, id_s, kk > 0 ? 1u : 0u);
+        }
+      };
       int g = 0, ii = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
         const int cnt = list_cnt(item);
         if (cnt == 0) continue;
         if (!(ok = mbar_wait(&bars[KV_KFULL], ii & 1, abort_flag))) break;
-        for (int j = 0; ok && j < cnt; ++j, ++g) {
+        {
+          // the item's first query block
           const int s = g % kStages;
           if (!(ok = mbar_wait(&bars[KV_QFULL + s], (g / kStages) & 1, abort_flag))) break;
+          if (g > 0 && !(ok = mbar_wait(&bars[KV_SEMPTY], (g - 1) & 1, abort_flag))) break;
           tc_fence_after();
-          const uint64_t qd = qdesc0 + ((s * L::ROWS_BYTES) >> 4), dd = dodesc0 + ((s * L::ROWS_BYTES) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (((kk >> 2) * L::CHUNK) + (kk & 3) * 32u) >> 4;
-            umma_ss(tm + TM_ST, kdesc + off, qd + off, id_s, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (((kk >> 2) * L::CHUNK) + (kk & 3) * 32u) >> 4;
-            umma_ss(tm + TM_DPT, vdesc + off, dd + off, id_s, kk > 0 ? 1u : 0u);
-          }
+          issue_st(s);
+          issue_dpt(s);
           tc_commit(&bars[KV_SFULL]);
+        }
+        for (int j = 0; ok && j < cnt; ++j, ++g) {
+          const int s = g % kStages;
+          if (j + 1 < cnt) {
+            const int s1 = (g + 1) % kStages;
+            if (!(ok = mbar_wait(&bars[KV_QFULL + s1], ((g + 1) / kStages) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait(&bars[KV_SEMPTY], g & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_st(s1);
+          }
           if (!(ok = mbar_wait(&bars[KV_PFULL], g & 1, abort_flag))) break;
           if (j == 0 && !(ok = mbar_wait(&bars[KV_OEMPTY], (ii & 1) ^ 1, abort_flag))) break;
           tc_fence_after();
           const uint64_t dmn = domn0 + ((s * L::ROWS_BYTES) >> 4), qmn = qmn0 + ((s * L::ROWS_BYTES) >> 4);
+          // P^T in the second 32, dS^T in the first 32 of each half's 64 dP^T columns
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tm + TM_DV, tm + TM_ST + (kk >> 2) * 64 + (kk & 3) * 8, dmn + ((kk * 2048u) >> 4), id_acc,
+            umma_ts(tm + TM_DV, tm + TM_DPT + (kk >> 2) * 64 + 32 + (kk & 3) * 8, dmn + ((kk * 2048u) >> 4), id_acc,
                     (j > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             umma_ts(tm + TM_DK, tm + TM_DPT + (kk >> 2) * 64 + (kk & 3) * 8, qmn + ((kk * 2048u) >> 4), id_acc,
                     (j > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&bars[KV_QEMPTY + s]);
-          if (j + 1 == cnt) {
+          if (j + 1 < cnt) {
+            issue_dpt((g + 1) % kStages);
+            tc_commit(&bars[KV_SFULL]);
+          } else {
             tc_commit(&bars[KV_KEMPTY]);
             tc_commit(&bars[KV_OFULL]);
           }
@@ -633,6 +665,9 @@ __global__ void __launch_bounds__(bwd::kKVThreads, 1)
         reg_fence(s1);
         reg_fence(p0);
         reg_fence(p1);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[KV_SEMPTY]);   // S^T and dP^T read: the next S^T may land
         const float* st = stats + s * 256 + half * 64;
         uint32_t pt[32], dst[32];
 #pragma unroll
@@ -652,10 +687,11 @@ __global__ void __launch_bounds__(bwd::kKVThreads, 1)
           pt[c] = pack_bf16x2(pp[0], pp[1]);
           dst[c] = pack_bf16x2(dd[0], dd[1]);
         }
-        // P^T and dS^T over the first 32 of this half's own 64 columns (the
-        // other half may not have read its columns yet)
-        tmem_st32(tm + la + TM_ST + half * 64, pt);
+        // dS^T and P^T over the first and second 32 of this half's own 64 dP^T
+        // columns (the other half may not have read its columns yet; the S^T
+        // buffer already holds the next block's S^T)
         tmem_st32(tm + la + TM_DPT + half * 64, dst);
+        tmem_st32(tm + la + TM_DPT + half * 64 + 32, pt);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
