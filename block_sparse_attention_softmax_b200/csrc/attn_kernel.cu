@@ -24,7 +24,11 @@
 //                also fills that tile's S buffer)
 //   warp 10      TMA producer of V (2-stage ring; a slot is free once the P V
 //                that read it has completed); one TMA box per 64-key block,
-//                so the two blocks of a tile need not be adjacent
+//                so the two blocks of a tile need not be adjacent. It also
+//                runs the O buffer: once per item, after the item's first two
+//                V tiles, it stores the previous item's O (staged by the
+//                softmax warps) by TMA, waits until the store has read the
+//                buffer, and loads this item's O_l into it (with the blend)
 //   warp 1       TMEM allocation and the thread issuing
 //                  S_g = Q K_g^T  (A = Q, B = K, both from shared memory)
 //   warp 11      the thread issuing
@@ -42,9 +46,14 @@
 //                64 columns of S as packed bf16. At the end of an item the
 //                warps sum the row's four shares of l with two shuffles,
 //                copy O to registers, release it, and write O / l as bf16 and
-//                the row log-sum-exp. With the linear branch the epilogue
-//                blends while O_s is still fp32, O = alpha ⊙ O_s + (1 - alpha)
-//                ⊙ O_l (SLA2 提案手法 ②): one bf16 rounding of O. A warp whose
+//                the row log-sum-exp. O / l is written as bf16 into the O
+//                buffer in shared memory (the TMA store's 128-byte swizzled
+//                layout, conflict-free for the 16-lane layout), and warp 10
+//                stores it while the next item runs: the softmax warps issue
+//                no global loads or stores for O. With the linear branch the
+//                epilogue blends while O_s is still fp32, O = alpha ⊙ O_s +
+//                (1 - alpha) ⊙ O_l (SLA2 提案手法 ②), reading O_l from the same
+//                bytes it overwrites: one bf16 rounding of O. A warp whose
 //                bounded wait runs out stops; the others learn of it through
 //                their own bounded waits (no named barrier is shared).
 //
@@ -60,7 +69,8 @@
 // Item facts carry the two factors, posted by the K producer with the rest.
 //
 // TMEM columns: S buffers at 0, 128 and 256 (fp32, 128 wide; P aliases their
-// first 64 columns, 32 in the low-bit form), O at 384 (d wide). Every mbarrier wait is bounded (see
+// first 64 columns, 32 in the low-bit form), O at 384 (d wide). Shared memory:
+// two Q slots, two K and two V stages, and the O buffer (128 rows x d bf16). Every mbarrier wait is bounded (see
 // sa_device.cuh), and a CTA that stops early waits (bounded) for the TMA loads
 // and MMAs it has issued before it gives up shared and tensor memory.
 #include "sa_internal.h"
@@ -103,7 +113,10 @@ struct Layout {
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + kQSlots * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + kKStages * TILE_BYTES;
-  static constexpr uint32_t OFF_RED = OFF_V + kVStages * TILE_BYTES;
+  static constexpr uint32_t OB_CHUNK = kBM * 128;            // bytes per 64-column chunk of the O buffer
+  static constexpr int NCH_O = D * 2 / 128;                  // 64-column chunks of a bf16 O row
+  static constexpr uint32_t OFF_OB = OFF_V + kVStages * TILE_BYTES;
+  static constexpr uint32_t OFF_RED = OFF_OB + NCH_O * OB_CHUNK;
   // row max [2][2][128], row sum [2][128], pair flags [4][16] of the E4M3 form's exchange
   static constexpr uint32_t RED_BYTES = F8 ? (2 * 2 + 2) * kBM * 4 + 4 * 16 * 4 : 0;
   static constexpr uint32_t OFF_BAR = OFF_RED + RED_BYTES;
@@ -113,6 +126,7 @@ struct Layout {
   static constexpr uint32_t USED = OFF_RING + 256;
   // at least 120 KB so that a second CTA never shares the SM (all 512 TMEM columns are held)
   static constexpr uint32_t SMEM = (USED + 1024 > 120 * 1024) ? USED + 1024 : 120 * 1024;
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
 __host__ __device__ constexpr uint32_t tm_s(int b) { return static_cast<uint32_t>(b) * 128u; }
@@ -132,7 +146,10 @@ enum {
                                      // the S buffer and the tile's V slot are free again
   B_OFULL = B_PVDONE + kSBufs,       // last P V of the item completed
   B_OEMPTY = B_OFULL + 1,            // epilogue has copied O out of TMEM
-  B_IFULL = B_OEMPTY + 1,            // [kItemRing] item facts posted by the K producer
+  B_OREADY = B_OEMPTY + 1,           // O buffer free of the previous item's O (its store has read
+                                     // it) and, with the blend, holding this item's O_l
+  B_OSTAGED = B_OREADY + 1,          // softmax warps have written this item's O into the buffer
+  B_IFULL = B_OSTAGED + 1,           // [kItemRing] item facts posted by the K producer
   B_IEMPTY = B_IFULL + kItemRing,    // [kItemRing] item facts read by the softmax warps
   B_DRAIN = B_IEMPTY + kItemRing,    // [2] each MMA thread's last commit (early exit)
   B_COUNT = B_DRAIN + 2
@@ -199,7 +216,9 @@ template <int D, bool F8>
 __global__ void __launch_bounds__(attn::kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, AttnArgs a) {
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmO,
+                       const __grid_constant__ CUtensorMap tmOL, AttnArgs a) {
   using namespace attn;
   using L = Layout<D, F8>;
   extern __shared__ uint8_t smem_raw[];
@@ -207,6 +226,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   uint8_t* sQ = smem + L::OFF_Q;
   uint8_t* sK = smem + L::OFF_K;
   uint8_t* sV = smem + L::OFF_V;
+  uint8_t* sOB = smem + L::OFF_OB;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   static_assert(B_COUNT * 8 + 8 <= 512, "barrier region");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
@@ -229,6 +249,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     }
     mbar_init(&bars[B_OFULL], 1);
     mbar_init(&bars[B_OEMPTY], kSoftWarps);
+    mbar_init(&bars[B_OREADY], 1);
+    mbar_init(&bars[B_OSTAGED], kSoftWarps);
     mbar_init(&bars[B_DRAIN + 0], 1);
     mbar_init(&bars[B_DRAIN + 1], 1);
     for (int i = 0; i < kKStages; ++i) mbar_init(&bars[B_KFULL + i], 1);
@@ -263,6 +285,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         tma_prefetch_desc(&tmK);
       } else {
         tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmO);
+        if (a.alpha) tma_prefetch_desc(&tmOL);
       }
       const CUtensorMap* map = is_k ? &tmK : &tmV;
       uint8_t* ring = is_k ? sK : sV;
@@ -270,6 +294,32 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       const int b_full = is_k ? B_KFULL : B_VFULL;
       int g = 0, qi = 0, q_armed = 0;
       bool ok = true;
+      // O buffer turns (V producer): one per item, after the item's first two
+      // V tiles (those never wait for the item's own P V). The previous item's
+      // O goes out once the softmax warps have staged it; this item's O_l (or,
+      // without the blend, the free buffer) is then handed to them.
+      int ob_bh = 0, ob_qb = 0, ol_armed = 0;
+      auto o_turn = [&](const Item& it) -> bool {
+        if (qi > 0) {
+          if (!mbar_wait(&bars[B_OSTAGED], (qi - 1) & 1, abort_flag)) return false;
+#pragma unroll
+          for (int c = 0; c < L::NCH_O; ++c) tma_store_3d(&tmO, sOB + c * L::OB_CHUNK, c * 64, ob_qb * a.bq, ob_bh);
+          bulk_commit();
+          bulk_wait_read<0>();
+        }
+        if (a.alpha) {
+          mbar_arrive_expect_tx(&bars[B_OREADY], L::NCH_O * a.bq * 128);
+#pragma unroll
+          for (int c = 0; c < L::NCH_O; ++c)
+            tma_load_3d(sOB + c * L::OB_CHUNK, &tmOL, &bars[B_OREADY], c * 64, it.qb * a.bq, it.bh);
+          ol_armed = qi + 1;
+        } else {
+          mbar_arrive(&bars[B_OREADY]);
+        }
+        ob_bh = it.bh;
+        ob_qb = it.qb;
+        return true;
+      };
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
         const Item it = load_item(a, item);
         if (it.T == 0) continue;
@@ -297,6 +347,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           q_armed = qi + 1;
         }
         for (int t = 0; t < it.T; ++t, ++g) {
+          if (!is_k && t == 2 && !(ok = o_turn(it))) break;
           const int s = g % stages;
           const int nblk = min(2, it.cnt - 2 * t);
           const int kb0 = a.dense ? 2 * t : __ldg(row + 2 * t);
@@ -323,6 +374,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
               tma_load_3d(dst + c * L::KV_CHUNK + 64 * 128, map, &bars[b_full + s], c * L::CH_ELEMS, kb1 * 64, it.bh);
           }
         }
+        if (ok && !is_k && it.T <= 2) ok = o_turn(it);
         ++qi;
       }
       if (is_k && ok) {
@@ -341,6 +393,16 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       if (is_k)
         for (int i = 1; i <= kQSlots && i <= q_armed; ++i)
           mbar_drain(&bars[B_QFULL + (q_armed - i) % kQSlots], ((q_armed - i) / kQSlots) & 1);
+      if (!is_k) {
+        // the last item's O, then every store complete and the last O_l load landed
+        if (ok && qi > 0 && mbar_wait(&bars[B_OSTAGED], (qi - 1) & 1, abort_flag)) {
+#pragma unroll
+          for (int c = 0; c < L::NCH_O; ++c) tma_store_3d(&tmO, sOB + c * L::OB_CHUNK, c * 64, ob_qb * a.bq, ob_bh);
+          bulk_commit();
+        }
+        bulk_wait_all();
+        if (ol_armed > 0) mbar_drain(&bars[B_OREADY], (ol_armed - 1) & 1);
+      }
     }
   } else if (warp == 1 || warp == kPVWarp) {
     // ------------------------------------------------------------ MMA issuers
@@ -509,14 +571,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         it.T = (it.cnt + 1) >> 1;
         const int grow = it.qb * a.bq + row;
         const bool store = row < a.bq && grow < a.N;
-        const long long orow_off = (static_cast<long long>(it.bh) * a.N + grow) * D + half * (D / 2);
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + orow_off;
-        if (a.alpha && store) {
-          // the epilogue reads this half row of O_l: bring it into L2 while the item runs
-          const char* olr = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.o_l) + orow_off);
-  #pragma unroll
-          for (int b = 0; b < D; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(olr + b));
-        }
         float m = -INFINITY;     // running max (log2 domain), identical in both halves
         float l = 0.f;           // this half's share of the row sum
         for (int t = 0; t < it.T; ++t, ++g) {
@@ -638,15 +692,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         }
         if (!ok) break;
         // ---------------------------------------------------------- epilogue
-        // with the blend, this half row of O_l is loaded before the wait for
-        // the last P V, so the wait hides the load
-        uint4 olv[D / 16];
-        if (a.alpha && store) {
-          const uint4* olp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.o_l) + orow_off);
-  #pragma unroll
-          for (int c = 0; c < D / 16; ++c) olv[c] = __ldg(olp + c);
-        }
-        const bool o_ok = mbar_wait(&bars[B_OFULL], qi & 1, abort_flag);
+        bool o_ok = mbar_wait(&bars[B_OFULL], qi & 1, abort_flag);
         uint32_t o0[32], o1[32];
         {
           tc_fence_after();
@@ -659,49 +705,47 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars[B_OEMPTY]);   // the next item may overwrite O now
         }
+        // the O buffer is free of the previous item's O and, with the blend,
+        // holds this item's O_l
+        o_ok = o_ok && mbar_wait(&bars[B_OREADY], qi & 1, abort_flag);
         red_sum[half * kBM + row] = o_ok ? l : __uint_as_float(kStopBits);
         pair_sync(pair_bar);
         const float pl = red_sum[(half ^ 1) * kBM + row];
         if (!(ok = o_ok && __float_as_uint(pl) != kStopBits)) break;
         const float lt = l + pl;
         const float inv_l = F8 ? fout / lt : 1.f / lt;
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow);
-          if (a.alpha) {
-            // O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l with O_s = o / l not yet rounded
-            const float4* alv = reinterpret_cast<const float4*>(a.alpha + static_cast<long long>(it.bh % a.H) * D + half * (D / 2));
+        {
+          // this thread's half row is 64-column chunk `half` of row `row` (d =
+          // 128): its 16-byte unit c lies at position c ^ (row % 8)
+          uint4* ub = reinterpret_cast<uint4*>(sOB + half * L::OB_CHUNK + row * 128);
+          const float4* alv = a.alpha ? reinterpret_cast<const float4*>(a.alpha + static_cast<long long>(it.bh % a.H) * D + half * (D / 2)) : nullptr;
   #pragma unroll
-            for (int c = 0; c < D / 16; ++c) {
-              const uint32_t* oc = (c < 4) ? o0 + 8 * c : o1 + 8 * (c - 4);
-              const uint4 lv = olv[c];
+          for (int c = 0; c < D / 16; ++c) {
+            const uint32_t* oc = (c < 4) ? o0 + 8 * c : o1 + 8 * (c - 4);
+            uint4* u = ub + (c ^ (row & 7));
+            float r8[8];
+  #pragma unroll
+            for (int j = 0; j < 8; ++j) r8[j] = __uint_as_float(oc[j]) * inv_l;
+            if (a.alpha) {
+              // O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l with O_s = o / l not yet rounded
+              const uint4 lv = *u;
               const float4 a0 = __ldg(alv + 2 * c), a1 = __ldg(alv + 2 * c + 1);
               const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
               const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-              float r8[8];
   #pragma unroll
               for (int j = 0; j < 8; ++j) {
                 const float olj = __uint_as_float((j & 1) ? (lw[j >> 1] & 0xFFFF0000u) : (lw[j >> 1] << 16));
-                r8[j] = fmaf(av[j], __uint_as_float(oc[j]) * inv_l - olj, olj);
+                r8[j] = fmaf(av[j], r8[j] - olj, olj);
               }
-              dst[c] = make_uint4(pack_bf16x2(r8[0], r8[1]), pack_bf16x2(r8[2], r8[3]),
-                                  pack_bf16x2(r8[4], r8[5]), pack_bf16x2(r8[6], r8[7]));
             }
-          } else {
-            uint32_t pk[16];
-  #pragma unroll
-            for (int c = 0; c < 16; ++c)
-              pk[c] = pack_bf16x2(__uint_as_float(o0[2 * c]) * inv_l, __uint_as_float(o0[2 * c + 1]) * inv_l);
-  #pragma unroll
-            for (int c = 0; c < 4; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            if (D == 128) {
-  #pragma unroll
-              for (int c = 0; c < 16; ++c)
-                pk[c] = pack_bf16x2(__uint_as_float(o1[2 * c]) * inv_l, __uint_as_float(o1[2 * c + 1]) * inv_l);
-  #pragma unroll
-              for (int c = 0; c < 4; ++c) dst[4 + c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            }
+            *u = make_uint4(pack_bf16x2(r8[0], r8[1]), pack_bf16x2(r8[2], r8[3]),
+                            pack_bf16x2(r8[4], r8[5]), pack_bf16x2(r8[6], r8[7]));
           }
         }
+        // the TMA store that reads the buffer is issued by the V producer
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_OSTAGED]);
         if (store && a.lse && half == 0)
           a.lse[static_cast<long long>(it.bh) * a.N + grow] = (m + log2f(lt)) * 0.69314718055994531f;
         ++qi;
@@ -760,18 +804,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         const int grow_a = it.qb * a.bq + ra;
         const bool store_a = ra < a.bq && grow_a < a.N;
         const bool store_b = ra + 8 < a.bq && grow_a + 8 < a.N;
-        const long long off_a = (static_cast<long long>(it.bh) * a.N + grow_a) * D;
-        const long long off_b = off_a + 8LL * D;
-        if (a.alpha && j4 == 0) {
-          // the epilogue reads these rows of O_l: bring them into L2 while the item runs
-          const char* ola = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.o_l) + off_a);
-          const char* olb = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.o_l) + off_b);
-  #pragma unroll
-          for (int b = 0; b < 2 * D; b += 128) {
-            if (store_a) asm volatile("prefetch.global.L2 [%0];" ::"l"(ola + b));
-            if (store_b) asm volatile("prefetch.global.L2 [%0];" ::"l"(olb + b));
-          }
-        }
         float m_a = -INFINITY, m_b = -INFINITY;   // running maxima of the two rows (log2 domain)
         float l_a = 0.f, l_b = 0.f;               // this thread's shares of the row sums
         for (int t = 0; t < it.T; ++t, ++g) {
@@ -912,17 +944,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         l_a += __shfl_xor_sync(0xFFFFFFFFu, l_a, 2);
         l_b += __shfl_xor_sync(0xFFFFFFFFu, l_b, 2);
         const float inv_a = fout / l_a, inv_b = fout / l_b;
-        // with the blend, this thread's elements of O_l are loaded before the
-        // wait for the last P V, so the wait hides the loads
-        uint32_t ol_a[D / 8], ol_b[D / 8];
-        if (a.alpha) {
-          const __nv_bfloat16* olp = static_cast<const __nv_bfloat16*>(a.o_l);
-  #pragma unroll
-          for (int k = 0; k < D / 8; ++k) {
-            ol_a[k] = store_a ? __ldg(reinterpret_cast<const unsigned int*>(olp + off_a + 8 * k + 2 * j4)) : 0u;
-            ol_b[k] = store_b ? __ldg(reinterpret_cast<const unsigned int*>(olp + off_b + 8 * k + 2 * j4)) : 0u;
-          }
-        }
         if (!mbar_wait(&bars[B_OFULL], qi & 1, abort_flag)) {
           ok = false;
           break;
@@ -953,29 +974,45 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars[B_OEMPTY]);   // the next item may overwrite O now
         }
+        // the O buffer is free of the previous item's O and, with the blend,
+        // holds this item's O_l
+        if (!mbar_wait(&bars[B_OREADY], qi & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
         {
-          __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.o);
+          // column 8 k + 2 j4 of row r lies in 64-column chunk k / 8, 16-byte
+          // unit (k % 8) ^ (r % 8) of the row's 128 bytes; rows ra and ra + 8
+          // share r % 8, and the 32 lanes of one k hit 32 distinct banks
           const float* alr = a.alpha ? a.alpha + static_cast<long long>(it.bh % a.H) * D : nullptr;
+          uint8_t* rowa = sOB + ra * 128 + 4 * j4;
   #pragma unroll
           for (int k = 0; k < D / 8; ++k) {
             const int col = 8 * k + 2 * j4;
             const int i0 = 32 * (k >> 3) + 4 * (k & 7);
+            uint32_t* pa = reinterpret_cast<uint32_t*>(rowa + (k >> 3) * L::OB_CHUNK + (((k & 7) ^ (ra & 7)) << 4));
+            uint32_t* pb = pa + 8 * 128 / 4;
             float va0 = __uint_as_float(o[i0]) * inv_a, va1 = __uint_as_float(o[i0 + 1]) * inv_a;
             float vb0 = __uint_as_float(o[i0 + 2]) * inv_b, vb1 = __uint_as_float(o[i0 + 3]) * inv_b;
             if (a.alpha) {
               // O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l with O_s not yet rounded
               const float2 al = __ldg(reinterpret_cast<const float2*>(alr + col));
-              const float la0 = __uint_as_float(ol_a[k] << 16), la1 = __uint_as_float(ol_a[k] & 0xFFFF0000u);
-              const float lb0 = __uint_as_float(ol_b[k] << 16), lb1 = __uint_as_float(ol_b[k] & 0xFFFF0000u);
+              const uint32_t wa = *pa, wb = *pb;
+              const float la0 = __uint_as_float(wa << 16), la1 = __uint_as_float(wa & 0xFFFF0000u);
+              const float lb0 = __uint_as_float(wb << 16), lb1 = __uint_as_float(wb & 0xFFFF0000u);
               va0 = fmaf(al.x, va0 - la0, la0);
               va1 = fmaf(al.y, va1 - la1, la1);
               vb0 = fmaf(al.x, vb0 - lb0, lb0);
               vb1 = fmaf(al.y, vb1 - lb1, lb1);
             }
-            if (store_a) *reinterpret_cast<uint32_t*>(ob + off_a + col) = pack_bf16x2(va0, va1);
-            if (store_b) *reinterpret_cast<uint32_t*>(ob + off_b + col) = pack_bf16x2(vb0, vb1);
+            *pa = pack_bf16x2(va0, va1);
+            *pb = pack_bf16x2(vb0, vb1);
           }
         }
+        // the TMA store that reads the buffer is issued by the V producer
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_OSTAGED]);
         if (a.lse && j4 == 0) {
           if (store_a) a.lse[static_cast<long long>(it.bh) * a.N + grow_a] = (m_a + log2f(l_a)) * 0.69314718055994531f;
           if (store_b) a.lse[static_cast<long long>(it.bh) * a.N + grow_a + 8] = (m_b + log2f(l_b)) * 0.69314718055994531f;
@@ -997,7 +1034,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 template <int D, bool F8>
 static cudaError_t launch_d(const AttnArgs& a, cudaStream_t st) {
   using L = attn::Layout<D, F8>;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo, mol;
   auto enc = [&](CUtensorMap* m, const void* base, uint32_t rows) {
     return F8 ? encode_tensor_map_3d_u8(m, base, D, a.N, a.BH, L::CH_ELEMS, rows)
               : encode_tensor_map_3d_bf16(m, base, D, a.N, a.BH, L::CH_ELEMS, rows);
@@ -1005,6 +1042,13 @@ static cudaError_t launch_d(const AttnArgs& a, cudaStream_t st) {
   if (enc(&mq, a.q, attn::kBM) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   if (enc(&mk, a.k, 64) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   if (enc(&mv, a.v, 64) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  // O (stored) and O_l (loaded) in bf16, one box per 64 columns and query block
+  if (encode_tensor_map_3d_bf16(&mo, a.o, D, a.N, a.BH, 64, a.bq) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (a.alpha) {
+    if (encode_tensor_map_3d_bf16(&mol, a.o_l, D, a.N, a.BH, 64, a.bq) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  } else {
+    mol = mo;   // not read without the blend
+  }
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
@@ -1012,7 +1056,7 @@ static cudaError_t launch_d(const AttnArgs& a, cudaStream_t st) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long items = static_cast<long long>(a.BH) * a.nqb;
   const int grid = static_cast<int>(items < sms ? items : sms);
-  return launch_pdl(sparse_attn_kernel<D, F8>, dim3(grid), dim3(attn::kThreads), L::SMEM, st, mq, mk, mv, a);
+  return launch_pdl(sparse_attn_kernel<D, F8>, dim3(grid), dim3(attn::kThreads), L::SMEM, st, mq, mk, mv, mo, mol, a);
 }
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t st) {
