@@ -307,7 +307,12 @@ int sparse_attn(const char* fn, const void* q, const void* k, const void* v, int
   if (lists == (ext_mask != nullptr) || (!lists && (kv_idx || kv_cnt)))
     return fail(SA_ERR_INVALID_ARG, "%s: give exactly one of (kv_idx, kv_cnt) or ext_mask", fn);
   if ((o_l == nullptr) != (alpha == nullptr)) return fail(SA_ERR_INVALID_ARG, "%s: o_l and alpha go together", fn);
-  if (o_l && o_l == o) return fail(SA_ERR_INVALID_ARG, "%s: o must not alias o_l", fn);
+  if (o_l) {
+    // O is stored tile by tile while later tiles of O_l are still to be read
+    const uintptr_t bytes = static_cast<uintptr_t>(B) * H * N * d * 2;
+    const uintptr_t po = reinterpret_cast<uintptr_t>(o), pl = reinterpret_cast<uintptr_t>(o_l);
+    if (po < pl + bytes && pl < po + bytes) return fail(SA_ERR_INVALID_ARG, "%s: o must not overlap o_l", fn);
+  }
   if (!isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "scale must be finite");
   const void* ptrs[] = {q, k, v, o, kv_idx, kv_cnt, lse_opt, workspace, o_l, alpha};
   for (const void* p : ptrs)

@@ -132,9 +132,9 @@ int sa_sparse_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
  *   O = alpha ⊙ O_s + (1 - alpha) ⊙ O_l
  * while O_s is still fp32, so O is rounded to bf16 once. o_l [B, H, N, d]
  * bf16 is the linear branch's output (sa_linear_branch with o_l_opt), alpha
- * [H, d] fp32. Both are required; o must not alias o_l. lse_opt is the log-sum-exp
- * of the sparse attention alone. Arguments, workspace and errors otherwise as
- * sa_sparse_attn_fwd. */
+ * [H, d] fp32. Both are required; o must not overlap o_l (SA_ERR_INVALID_ARG).
+ * lse_opt is the log-sum-exp of the sparse attention alone. Arguments,
+ * workspace and errors otherwise as sa_sparse_attn_fwd. */
 int sa_sparse_attn_blend_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                              int B, int H, int N, int d, int bq, int bk,
                              const int32_t* kv_idx, const int32_t* kv_cnt, const uint8_t* ext_mask,

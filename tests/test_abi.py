@@ -75,6 +75,12 @@ def test_argument_validation_without_launch(lib):
     need = lib.sa_sparse_attn_workspace_size(1, 1, 128, 64, 64, 64, 1)
     assert need > 0 and lib.sa_sparse_attn_workspace_size(1, 1, 128, 64, 64, 64, 0) == 0
     assert lib.sa_sparse_attn_fwd(*a, None, None, fake, 0.0, fake, None, fake, need - 1, None) == -6
+    # the blended form: o must not overlap o_l (size checks come first)
+    blend = lambda o_l, o: lib.sa_sparse_attn_blend_fwd(*a, None, None, fake, 0.0, o_l, fake, o, None, fake, need,
+                                                        None)
+    assert blend(fake, fake) == -1
+    assert blend(P(0x1000 + 128 * 64 * 2 - 16), fake) == -1
+    assert b"overlap" in lib.sa_last_error()
     # linear branch and blend
     assert lib.sa_linear_branch(None, fake, fake, 1, 1, 128, 64, fake, fake, fake, fake, 1 << 20, None) == -1
     assert lib.sa_blend(fake, fake, fake, fake, None, 1, 1, 128, 64, fake, None, 0, None) == -1
