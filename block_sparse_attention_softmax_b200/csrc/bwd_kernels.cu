@@ -19,9 +19,9 @@
 //                  either block (a transposed list with a flag per block, from
 //                  col_lists_kernel), for each S^T = K Q^T and dP^T = V dO^T;
 //                  8 warps form P^T and dS^T (rows of the block that does not
-//                  keep this query block are zero) into the dP^T columns, so
-//                  the next block's S^T lands while they work; dV += P^T dO
-//                  and dK += dS^T Q accumulate in TMEM.
+//                  keep this query block are zero) over the dP^T columns they
+//                  came from, so the next block's S^T lands while they work;
+//                  dV += P^T dO and dK += dS^T Q accumulate in TMEM.
 // Roles in both: warp 0 TMA producer, warp 1 TMEM allocation and the MMA
 // thread, then (dK/dV only) a warp staging the query blocks' LSE and D in
 // shared memory, and 8 warps, two per TMEM lane quadrant, 64 columns each.
@@ -581,15 +581,17 @@ __global__ void __launch_bounds__(bwd::kKVThreads, 1)
           if (j == 0 && !(ok = mbar_wait(&bars[KV_OEMPTY], (ii & 1) ^ 1, abort_flag))) break;
           tc_fence_after();
           const uint64_t dmn = domn0 + ((s * L::ROWS_BYTES) >> 4), qmn = qmn0 + ((s * L::ROWS_BYTES) >> 4);
-          // P^T in the second 32, dS^T in the first 32 of each half's 64 dP^T columns
+          // K step kk (16 query columns) reads 8 TMEM columns: in each half's
+          // 64 dP^T columns, each 32 hold dS^T of 32 query columns in their
+          // first 16 and P^T of the same query columns in their second 16
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tm + TM_DV, tm + TM_DPT + (kk >> 2) * 64 + 32 + (kk & 3) * 8, dmn + ((kk * 2048u) >> 4), id_acc,
-                    (j > 0 || kk > 0) ? 1u : 0u);
+            umma_ts(tm + TM_DV, tm + TM_DPT + (kk >> 2) * 64 + ((kk & 3) >> 1) * 32 + 16 + (kk & 1) * 8,
+                    dmn + ((kk * 2048u) >> 4), id_acc, (j > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tm + TM_DK, tm + TM_DPT + (kk >> 2) * 64 + (kk & 3) * 8, qmn + ((kk * 2048u) >> 4), id_acc,
-                    (j > 0 || kk > 0) ? 1u : 0u);
+            umma_ts(tm + TM_DK, tm + TM_DPT + (kk >> 2) * 64 + ((kk & 3) >> 1) * 32 + (kk & 1) * 8,
+                    qmn + ((kk * 2048u) >> 4), id_acc, (j > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&bars[KV_QEMPTY + s]);
           if (j + 1 < cnt) {
             issue_dpt((g + 1) % kStages);
@@ -655,43 +657,52 @@ __global__ void __launch_bounds__(bwd::kKVThreads, 1)
         if (!(ok = mbar_wait(&bars[KV_SFULL], g & 1, abort_flag))) break;
         if (!(ok = mbar_wait(&bars[KV_STFULL + s], (g / kStages) & 1, abort_flag))) break;
         tc_fence_after();
-        uint32_t s0[32], s1[32], p0[32], p1[32];
+        uint32_t s0[32], s1[32], p0[32];
         tmem_ld32(tm + la + TM_ST + half * 64, s0);
         tmem_ld32(tm + la + TM_ST + half * 64 + 32, s1);
         tmem_ld32(tm + la + TM_DPT + half * 64, p0);
-        tmem_ld32(tm + la + TM_DPT + half * 64 + 32, p1);
         tmem_wait_ld();
         reg_fence(s0);
         reg_fence(s1);
         reg_fence(p0);
-        reg_fence(p1);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[KV_SEMPTY]);   // S^T and dP^T read: the next S^T may land
+        if (lane == 0) mbar_arrive(&bars[KV_SEMPTY]);   // S^T read: the next S^T may land
         const float* st = stats + s * 256 + half * 64;
-        uint32_t pt[32], dst[32];
+        // dS^T and P^T of query columns [32 h2, 32 h2 + 32) of this half go
+        // over the 32 dP^T columns those query columns came from (dS^T in the
+        // first 16, P^T in the second), so the second 32 dP^T columns are
+        // loaded only after the first 32 are done with: fewer live registers.
+        // Each half writes only its own 64 columns (the other half may not have
+        // read its columns yet; the S^T buffer already holds the next block's S^T).
+        auto form = [&](int h2, const uint32_t (&sr)[32], const uint32_t (&pr)[32]) {
+          uint32_t pt[16], dst[16];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          float pp[2], dd[2];
+          for (int c = 0; c < 16; ++c) {
+            float pp[2], dd[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = 2 * c + u;
-            const float sv = __uint_as_float(col < 32 ? s0[col] : s1[col - 32]);
-            const float pv = __uint_as_float(col < 32 ? p0[col] : p1[col - 32]);
-            // rows of a key block that does not keep this query block (or past
-            // the last key block, with stale values) contribute exact zeros
-            const float p = keep ? fast_exp2(fmaf(sv, a.scale_log2, -st[col])) : 0.f;
-            pp[u] = p;
-            dd[u] = keep ? p * (pv - st[128 + col]) : 0.f;
+            for (int u = 0; u < 2; ++u) {
+              const int col = 32 * h2 + 2 * c + u;
+              // rows of a key block that does not keep this query block (or past
+              // the last key block, with stale values) contribute exact zeros
+              const float p = keep ? fast_exp2(fmaf(__uint_as_float(sr[2 * c + u]), a.scale_log2, -st[col])) : 0.f;
+              pp[u] = p;
+              dd[u] = keep ? p * (__uint_as_float(pr[2 * c + u]) - st[128 + col]) : 0.f;
+            }
+            pt[c] = pack_bf16x2(pp[0], pp[1]);
+            dst[c] = pack_bf16x2(dd[0], dd[1]);
           }
-          pt[c] = pack_bf16x2(pp[0], pp[1]);
-          dst[c] = pack_bf16x2(dd[0], dd[1]);
+          tmem_st16(tm + la + TM_DPT + half * 64 + 32 * h2, dst);
+          tmem_st16(tm + la + TM_DPT + half * 64 + 32 * h2 + 16, pt);
+        };
+        form(0, s0, p0);
+        {
+          uint32_t p1[32];
+          tmem_ld32(tm + la + TM_DPT + half * 64 + 32, p1);
+          tmem_wait_ld();
+          reg_fence(p1);
+          form(1, s1, p1);
         }
-        // dS^T and P^T over the first and second 32 of this half's own 64 dP^T
-        // columns (the other half may not have read its columns yet; the S^T
-        // buffer already holds the next block's S^T)
-        tmem_st32(tm + la + TM_DPT + half * 64, dst);
-        tmem_st32(tm + la + TM_DPT + half * 64 + 32, pt);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
